@@ -1,0 +1,197 @@
+"""Seeded synthetic calibration inputs for the AWQ per-layer scale search.
+
+This module draws random numbers and shapes them like the workloads the AWQ
+pages describe; it performs none of the method's arithmetic (no statistic, no
+scale, no quantisation).  Both the CPU oracle and the CUDA path consume what it
+returns, so it is the only code the two sides share.
+
+Recipe (the pages calibrate on ~128 samples of an unnamed text set, "05 — AWQ"
+study notes §4; no dataset or trained weight is available, so these stand in):
+
+* heavy-tailed activations  X[t, j] = RN16(z[t, j] * c[j]) with z ~ N(0, 1) and
+  c[j] = exp(0.5 * n[j]), n ~ N(0, 1) (log-normal(0, 0.5) channel scales); a set
+  of round(p * d) outlier channels, drawn without replacement, has c[j]
+  multiplied by m[j] (a constant or U[lo, hi]);  salient channels are the ~0.1–1 %
+  with large activations ("AWQ and Activation-Aware Scaling", The observation).
+* weights  W = RN16(0.02 * N(0, 1)), laid out [out, in] like nn.Linear.
+
+All draws are fp32 from ``torch.Generator('cpu')`` and are rounded once to fp16.
+Each tensor gets its own generator, derived from the config seed, so that a
+tensor does not change when another one's shape does.
+"""
+
+from __future__ import annotations
+
+import dataclasses
+from typing import Optional, Tuple
+
+import torch
+
+__all__ = [
+    "OutlierSpec",
+    "heavy_tailed_activations",
+    "gaussian_weight",
+    "swiglu_activations",
+    "Workload",
+    "WORKLOADS",
+    "workload_inputs",
+]
+
+
+@dataclasses.dataclass(frozen=True)
+class OutlierSpec:
+    """Outlier channels: ``round(frac * d)`` channels multiplied by ``lo`` (if
+    ``hi`` is None) or by U[lo, hi]."""
+
+    frac: float
+    lo: float
+    hi: Optional[float] = None
+
+
+def _gen(seed: int) -> torch.Generator:
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    return g
+
+
+def channel_profile(d: int, outliers: OutlierSpec, seed: int) -> torch.Tensor:
+    """Per-channel magnitudes c[j] (fp32 [d]) of the heavy-tailed recipe."""
+    g = _gen(seed)
+    c = torch.exp(0.5 * torch.randn(d, generator=g, dtype=torch.float32))
+    n_out = int(round(outliers.frac * d))
+    if n_out > 0:
+        idx = torch.randperm(d, generator=g)[:n_out]
+        if outliers.hi is None:
+            m = torch.full((n_out,), float(outliers.lo), dtype=torch.float32)
+        else:
+            m = outliers.lo + (outliers.hi - outliers.lo) * torch.rand(
+                n_out, generator=g, dtype=torch.float32)
+        c[idx] = c[idx] * m
+    return c
+
+
+def heavy_tailed_activations(T: int, d: int, outliers: OutlierSpec, seed: int,
+                             chunk: int = 8192) -> torch.Tensor:
+    """Calibration activations X [T, d] fp16 (CPU), token-major.
+
+    Rows are drawn in chunks of ``chunk`` tokens, each chunk from its own
+    generator, so the first T' rows do not depend on T."""
+    c = channel_profile(d, outliers, seed)
+    X = torch.empty((T, d), dtype=torch.float16)
+    for i, t0 in enumerate(range(0, T, chunk)):
+        t1 = min(T, t0 + chunk)
+        g = _gen(seed * 1_000_003 + 17 + i)
+        z = torch.randn((t1 - t0, d), generator=g, dtype=torch.float32)
+        X[t0:t1] = (z * c).to(torch.float16)
+    return X
+
+
+def gaussian_weight(out: int, inn: int, seed: int, std: float = 0.02) -> torch.Tensor:
+    """Weight W [out, in] fp16 (CPU), entries RN16(std * N(0, 1))."""
+    g = _gen(seed * 1_000_003 + 5)
+    return (std * torch.randn((out, inn), generator=g, dtype=torch.float32)).to(torch.float16)
+
+
+def swiglu_activations(X: torch.Tensor, W_gate: torch.Tensor, W_up: torch.Tensor,
+                       outliers: OutlierSpec, seed: int, device: str = "cpu",
+                       chunk: int = 4096) -> torch.Tensor:
+    """Input of a down projection: SiLU(X W_gate^T) * (X W_up^T) in fp32,
+    divided by its global RMS (keeps the product inside fp16's range once the
+    outlier profile is applied), multiplied by its own heavy-tailed channel
+    profile, rounded once to fp16.  Returns a CPU tensor [T, d_ff].
+
+    This is the model's forward pass (synthetic input), not part of AWQ."""
+    T = X.shape[0]
+    d_ff = W_gate.shape[0]
+    c = channel_profile(d_ff, outliers, seed).to(device)
+    wg = W_gate.to(device=device, dtype=torch.float32)
+    wu = W_up.to(device=device, dtype=torch.float32)
+    sq = torch.zeros((), dtype=torch.float64, device=device)
+    parts = []
+    for t0 in range(0, T, chunk):
+        x = X[t0:t0 + chunk].to(device=device, dtype=torch.float32)
+        h = torch.nn.functional.silu(x @ wg.T) * (x @ wu.T)
+        sq += (h.double() ** 2).sum()
+        parts.append(h)
+    rms = float(torch.sqrt(sq / (T * d_ff)))
+    out = torch.empty((T, d_ff), dtype=torch.float16)
+    t0 = 0
+    for h in parts:
+        out[t0:t0 + h.shape[0]] = ((h / rms) * c).to(torch.float16).cpu()
+        t0 += h.shape[0]
+    return out
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    """One of the five benchmark workloads (shapes and value recipes)."""
+
+    name: str
+    T: int
+    w_bit: int
+    group_size: int
+    n_alpha: int
+    n_clip: int
+    seed: int
+    description: str
+
+
+WORKLOADS: Tuple[Workload, ...] = (
+    Workload("tiny_linear_512", 256, 4, 128, 20, 0, 0,
+             "X [256 x 512], W [512 x 512], 5 outlier channels x20, INT4 g128, 20 alphas, no clip"),
+    Workload("llama7b_q_proj_4096", 65536, 4, 128, 20, 20, 1,
+             "X [65536 x 4096], W [4096 x 4096], 41 outlier channels x U[20,50], INT4 g128, "
+             "20 alphas + 20 clip ratios, packed"),
+    Workload("llama7b_mlp_4096_11008", 65536, 4, 128, 20, 0, 2,
+             "X [65536 x 4096]; gate|up [22016 x 4096] jointly; down [4096 x 11008] on the "
+             "SwiGLU output; INT4 g128, 20 alphas"),
+    Workload("llama13b_attn_5120_int3", 65536, 3, 128, 20, 20, 3,
+             "X [65536 x 5120] (5 outlier channels x50); qkv [15360 x 5120]; o_proj [5120 x 5120] "
+             "on its own X; INT3 g128, 20 alphas + 20 clip ratios"),
+)
+
+
+def workload_inputs(index: int, T: Optional[int] = None, device: str = "cpu") -> dict:
+    """Inputs of workload ``index`` (0-based into WORKLOADS) as CPU fp16 tensors.
+
+    Returns {"groups": [(name, X, W), ...], "workload": Workload}.  Joint
+    scaling groups are returned with their weights already concatenated along
+    ``out`` (they share one scale vector).  ``T`` overrides the token count
+    (smaller parity cases of the same structure); ``device`` is only used for
+    the SwiGLU forward of workload 2."""
+    wl = WORKLOADS[index]
+    T = wl.T if T is None else int(T)
+    s = wl.seed
+    if index == 0:
+        X = heavy_tailed_activations(T, 512, OutlierSpec(0.01, 20.0), s)
+        W = gaussian_weight(512, 512, s)
+        return {"groups": [("linear", X, W)], "workload": wl}
+    if index == 1:
+        X = heavy_tailed_activations(T, 4096, OutlierSpec(0.01, 20.0, 50.0), s)
+        W = gaussian_weight(4096, 4096, s)
+        return {"groups": [("q_proj", X, W)], "workload": wl}
+    if index == 2:
+        X = heavy_tailed_activations(T, 4096, OutlierSpec(0.01, 20.0, 50.0), s)
+        Wg = gaussian_weight(11008, 4096, s * 10 + 1)
+        Wu = gaussian_weight(11008, 4096, s * 10 + 2)
+        Wd = gaussian_weight(4096, 11008, s * 10 + 3)
+        Xd = swiglu_activations(X, Wg, Wu, OutlierSpec(0.01, 20.0, 50.0), s * 10 + 4, device=device)
+        return {"groups": [("gate_up", X, torch.cat([Wg, Wu], 0)), ("down_proj", Xd, Wd)],
+                "workload": wl}
+    if index == 3:
+        X = heavy_tailed_activations(T, 5120, OutlierSpec(0.001, 50.0), s)
+        Wqkv = gaussian_weight(15360, 5120, s * 10 + 1)
+        Xo = heavy_tailed_activations(T, 5120, OutlierSpec(0.001, 50.0), s + 100)
+        Wo = gaussian_weight(5120, 5120, s * 10 + 2)
+        return {"groups": [("qkv", X, Wqkv), ("o_proj", Xo, Wo)], "workload": wl}
+    raise ValueError(f"no workload {index}")
+
+
+def random_layer(T: int, d_in: int, d_out: int, seed: int,
+                 outliers: OutlierSpec = OutlierSpec(0.01, 20.0, 50.0),
+                 w_std: float = 0.02) -> Tuple[torch.Tensor, torch.Tensor]:
+    """A small (X, W) pair of arbitrary shape with the same recipe, for
+    parity and edge-case tests."""
+    X = heavy_tailed_activations(T, d_in, outliers, seed)
+    W = gaussian_weight(d_out, d_in, seed, std=w_std)
+    return X, W

@@ -1,0 +1,375 @@
+"""Pins for the CPU oracle: each test checks the oracle against something
+other than itself — hand-worked examples, exact rational arithmetic, brute
+force, closed forms and the special cases the AWQ pages state.  CPU only."""
+
+import math
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+from oracle import awq_oracle as O
+from synthetic import OutlierSpec, heavy_tailed_activations, gaussian_weight, random_layer
+
+
+def _group_row(entries, group, fill=0.0):
+    w = np.full((1, group), fill, dtype=np.float16)
+    for j, v in entries.items():
+        w[0, j] = np.float16(v)
+    return w
+
+
+# --------------------------------------------------------------------------
+# D1  activation statistic
+# --------------------------------------------------------------------------
+def test_act_stats_matches_exact_rational_mean():
+    rng = np.random.default_rng(1)
+    T, d = 37, 24
+    mags = 2.0 ** rng.integers(-24, 15, size=(T, d))
+    X = (np.clip(rng.standard_normal((T, d)), -1.9, 1.9) * mags).astype(np.float16)
+    X[0, 0] = np.float16(65504.0)
+    X[1:, 0] = np.float16(2.0 ** -24)          # subnormal tail next to the max
+    X[:, 1] = np.float16(-1.0)
+    abar = O.act_stats(X)
+    for j in range(d):
+        S = sum(Fraction(float(abs(x))) for x in X[:, j].astype(np.float64))
+        want = float(S) / T                      # RN64(S), then RN64(. / T)
+        assert abar[j] == want, (j, abar[j], want)
+    assert abar[1] == 1.0
+
+
+def test_act_stats_single_nonzero_and_fp32_loss():
+    T = 4096
+    X = np.zeros((T, 8), dtype=np.float16)
+    X[5, 3] = np.float16(-3.0)
+    X[:, 4] = np.float16(2.0 ** -24)
+    X[0, 4] = np.float16(2048.0)
+    abar = O.act_stats(X)
+    assert abar[3] == 3.0 / T
+    assert np.all(abar[[0, 1, 2, 5, 6, 7]] == 0.0)
+    exact = (2048.0 + (T - 1) * 2.0 ** -24) / T
+    assert abar[4] == exact
+    # a naive fp32 running sum loses the small terms entirely
+    acc = np.float32(0)
+    for x in X[:, 4].astype(np.float32):
+        acc = np.float32(acc + abs(x))
+    assert float(acc) / T != exact
+
+
+# --------------------------------------------------------------------------
+# D2, D3  alpha grid and s = abar^alpha
+# --------------------------------------------------------------------------
+def test_alpha_grid_endpoints_and_spacing():
+    a = O.alpha_grid(20)
+    assert a[0] == 0.0 and a[-1] == 1.0 and len(a) == 20
+    assert np.allclose(np.diff(a), 1.0 / 19, rtol=0, atol=1e-15)
+    assert list(O.alpha_grid(1)) == [0.0]
+
+
+def test_scale_grid_closed_forms():
+    rng = np.random.default_rng(2)
+    abar = np.exp(rng.normal(0, 2, size=2000))
+    abar[:5] = [0.0, 1e-9, 1e-4, 1.0, 300.0]
+    S = O.scale_grid(abar, O.alpha_grid(3))   # alpha = 0, 0.5, 1
+    floor = np.maximum(abar, 1e-4)
+    assert np.all(S[0] == np.float32(1.0))                       # alpha = 0: plain RTN scale
+    assert np.array_equal(S[2], floor.astype(np.float32))       # alpha = 1: s = abar
+    assert np.array_equal(S[1], np.sqrt(floor).astype(np.float32))  # alpha = 1/2: sqrt
+    assert S[0, 0] == 1.0 and S[2, 0] == np.float32(1e-4)
+
+
+# --------------------------------------------------------------------------
+# D4  quantiser
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("name", ["quant_group_int4.txt", "quant_group_int3.txt", "quant_group_clip.txt"])
+def test_quantiser_hand_worked(golden, name):
+    hdr, rows = golden(name)
+    g, b = int(hdr["group"]), int(hdr["w_bit"])
+    W = _group_row({int(r[0]): float(r[1]) for r in rows}, g)
+    ratio = None
+    if "clip_index" in hdr:
+        r = O.clip_ratios(int(hdr["n_clip"]), 0.5)[int(hdr["clip_index"])]
+        ratio = np.full((1, 1), np.float32(r), dtype=np.float32)
+    qd = O.quantize_groups(W, None, g, b, ratio)
+    assert qd["delta"][0, 0] == np.float32(float(hdr["delta"]))
+    assert int(qd["z"][0, 0]) == int(hdr["zero"])
+    for r in rows:
+        j = int(r[0])
+        assert int(qd["q"][0, j]) == int(r[2]), (name, j)
+        assert float(qd["deq"][0, j]) == float(r[3]), (name, j)
+    zero_code = int(hdr["zero"])
+    listed = {int(r[0]) for r in rows}
+    for j in range(g):
+        if j not in listed:
+            assert int(qd["q"][0, j]) == zero_code and qd["deq"][0, j] == 0.0
+
+
+def _nearest_code_bruteforce(wt, delta, z, qmax):
+    """Exact nearest point of the grid {(q - z) delta : 0 <= q <= qmax};
+    a tie goes to even (q - z).  Returns (code, margin), margin being the
+    exact distance of wt/delta from the nearest half-integer."""
+    wt, delta = Fraction(float(wt)), Fraction(float(delta))
+    best, bestd = None, None
+    for q in range(qmax + 1):
+        dist = abs((q - z) * delta - wt)
+        if bestd is None or dist < bestd or (dist == bestd and (q - z) % 2 == 0):
+            best, bestd = q, dist
+    u = wt / delta
+    margin = abs(u - (math.floor(u) + Fraction(1, 2)))
+    return best, margin
+
+
+@pytest.mark.parametrize("w_bit", [3, 4])
+def test_alpha0_is_plain_rtn_nearest_grid_point(w_bit):
+    """alpha = 0 reduces to plain round-to-nearest ("AWQ and Activation-Aware
+    Scaling", Scaling instead of protecting): codes are the nearest in-range
+    grid point, checked by exhaustive search in exact arithmetic."""
+    X, W = random_layer(16, 256, 12, seed=11)
+    abar = O.act_stats(X.numpy())
+    S = O.scale_grid(abar, O.alpha_grid(20))
+    Wn = W.numpy()
+    q0 = O.quantize_groups(Wn, S[0], 128, w_bit)
+    qr = O.quantize_groups(Wn, None, 128, w_bit)
+    assert np.array_equal(q0["q"], qr["q"]) and np.array_equal(q0["delta"], qr["delta"])
+    qmax = 2 ** w_bit - 1
+    checked = 0
+    for o in range(Wn.shape[0]):
+        for j in range(Wn.shape[1]):
+            k = j // 128
+            code, margin = _nearest_code_bruteforce(qr["wt"][o, j], qr["delta"][o, k], int(qr["z"][o, k]), qmax)
+            if margin < Fraction(1, 2 ** 18):
+                continue  # the fp32 quotient may round across a half-integer
+            assert int(qr["q"][o, j]) == code, (o, j)
+            checked += 1
+    assert checked > 0.99 * Wn.size
+
+
+@pytest.mark.parametrize("w_bit", [3, 4])
+def test_half_step_bound(w_bit):
+    """|deq - s w| <= delta / 2 (+ fp32 rounding) for groups whose range spans 0
+    ("05 — AWQ" §3: rounding error at most half a step)."""
+    X, W = random_layer(64, 512, 64, seed=3)
+    abar = O.act_stats(X.numpy())
+    S = O.scale_grid(abar, O.alpha_grid(20))
+    for i in (0, 7, 19):
+        qd = O.quantize_groups(W.numpy(), S[i], 128, w_bit)
+        wt3 = qd["wt"].reshape(64, 4, 128)
+        spans0 = (wt3.min(2) <= 0) & (wt3.max(2) >= 0)
+        assert spans0.all()
+        err = np.abs(qd["deq"].astype(np.float64) - qd["wt"]).reshape(64, 4, 128)
+        bound = qd["delta"].astype(np.float64)[:, :, None] * (0.5 + 2.0 ** -18)
+        assert np.all(err <= bound)
+
+
+def test_one_signed_group_clamps():
+    """A group with min > 0: the zero point clamps to 0 and codes clamp to
+    2^b - 1 (the range is not widened to include 0)."""
+    W = _group_row({j: 1.0 + j / 128.0 for j in range(128)}, 128)
+    qd = O.quantize_groups(W, None, 128, 4)
+    assert int(qd["z"][0, 0]) == 0
+    delta = float(qd["delta"][0, 0])
+    assert delta == float(np.float32(np.float32(1.0 + 127 / 128 - 1.0) / np.float32(15)))
+    want = np.clip(np.rint(qd["wt"][0] / np.float32(delta)), 0, 15)
+    assert np.array_equal(qd["q"][0], want.astype(np.uint8))
+    assert qd["q"][0].max() == 15
+
+
+def test_constant_group_guard():
+    W = _group_row({}, 128, fill=0.25)
+    qd = O.quantize_groups(W, None, 128, 4)
+    assert qd["delta"][0, 0] == np.float32(np.float32(1e-5) / np.float32(15))
+    assert int(qd["z"][0, 0]) == 0 and np.all(qd["q"] == 15)
+
+
+@pytest.mark.parametrize("k", [-3, 4])
+def test_power_of_two_scale_invariance(k):
+    """s -> 2^k s leaves codes and zeros unchanged and scales delta by 2^k
+    exactly (every fp32 step commutes with an exact power-of-two scaling)."""
+    X, W = random_layer(32, 256, 16, seed=5)
+    abar = O.act_stats(X.numpy())
+    s = O.scale_grid(abar, O.alpha_grid(20))[12]
+    a = O.quantize_groups(W.numpy(), s, 128, 4)
+    b = O.quantize_groups(W.numpy(), (s * np.float32(2.0 ** k)).astype(np.float32), 128, 4)
+    assert np.array_equal(a["q"], b["q"]) and np.array_equal(a["z"], b["z"])
+    assert np.array_equal(a["delta"] * np.float32(2.0 ** k), b["delta"])
+
+
+# --------------------------------------------------------------------------
+# D5, D6  scoring and the alpha search
+# --------------------------------------------------------------------------
+def _literal_mse(X, W, s, deq):
+    """The pages' score written literally: ((X diag(s)^-1) Qdeq^T - X W^T)^2
+    averaged over tokens and outputs, fp64."""
+    X64 = X.astype(np.float64)
+    Yhat = (X64 / s.astype(np.float64)[None, :]) @ deq.astype(np.float64).T
+    Y = X64 @ W.astype(np.float64).T
+    return float(np.mean((Yhat - Y) ** 2))
+
+
+def _pure_python_mse(X, W, s, deq):
+    T, inn = X.shape
+    out = W.shape[0]
+    tot = 0.0
+    for t in range(T):
+        for o in range(out):
+            yh = sum(float(X[t, j]) / float(s[j]) * float(deq[o, j]) for j in range(inn))
+            y = sum(float(X[t, j]) * float(W[o, j]) for j in range(inn))
+            tot += (yh - y) ** 2
+    return tot / (T * out)
+
+
+def test_scaling_invariance_identity():
+    """X W^T = (X diag(s)^-1)(diag(s) W)^T in fp64 ("05 — AWQ" §3)."""
+    X, W = random_layer(64, 256, 16, seed=6)
+    abar = O.act_stats(X.numpy())
+    s = O.scale_grid(abar, O.alpha_grid(20))[19].astype(np.float64)
+    X64, W64 = X.numpy().astype(np.float64), W.numpy().astype(np.float64)
+    a = X64 @ W64.T
+    b = (X64 / s[None, :]) @ (W64 * s[None, :]).T
+    assert np.max(np.abs(a - b)) <= 1e-12 * np.max(np.abs(a))
+
+
+def test_mse_forms_match_pure_python_definition():
+    X, W = random_layer(6, 128, 8, seed=7)
+    Xn, Wn = X.numpy(), W.numpy()
+    abar = O.act_stats(Xn)
+    S = O.scale_grid(abar, O.alpha_grid(20))
+    for i in (0, 10, 19):
+        qd = O.quantize_groups(Wn, S[i], 128, 4)
+        want = _pure_python_mse(Xn, Wn, S[i], qd["deq"])
+        delta = O.effective_error(Wn, S[i], qd["deq"])
+        assert O.mse_direct(Xn, delta) == pytest.approx(want, rel=1e-10)
+        assert O.mse_gram(O.gram(Xn), delta, Xn.shape[0]) == pytest.approx(want, rel=1e-10)
+
+
+@pytest.mark.parametrize("T,inn,out,w_bit", [(64, 128, 16, 4), (48, 256, 8, 3), (33, 256, 16, 4)])
+def test_search_bruteforce_tiny(T, inn, out, w_bit):
+    X, W = random_layer(T, inn, out, seed=T + inn + out + w_bit)
+    Xn, Wn = X.numpy(), W.numpy()
+    abar = O.act_stats(Xn)
+    mse, best, s_best, S = O.search_scale(Xn, Wn, abar, w_bit, 128, 20, form="direct")
+    mse_g, best_g, _, _ = O.search_scale(Xn, Wn, abar, w_bit, 128, 20, form="gram")
+    lit = np.array([_literal_mse(Xn, Wn, S[i], O.quantize_groups(Wn, S[i], 128, w_bit)["deq"])
+                    for i in range(20)])
+    assert np.allclose(mse, lit, rtol=1e-10, atol=0)
+    assert np.allclose(mse_g, lit, rtol=1e-10, atol=0)
+    assert best == int(np.argmin(lit)) == best_g
+    assert np.array_equal(s_best, S[best])
+
+
+def test_ties_resolve_to_lowest_alpha():
+    """abar = 1 everywhere makes s = 1 for every alpha: all scores are equal
+    bit for bit and the search keeps alpha = 0."""
+    T, inn = 32, 256
+    X = np.where(np.arange(T * inn).reshape(T, inn) % 2 == 0, 1.0, -1.0).astype(np.float16)
+    _, W = random_layer(4, inn, 8, seed=9)
+    abar = O.act_stats(X)
+    assert np.all(abar == 1.0)
+    mse, best, s_best, _ = O.search_scale(X, W.numpy(), abar, 4, 128, 20)
+    assert np.all(mse == mse[0]) and best == 0 and np.all(s_best == 1.0)
+
+
+def test_search_beats_rtn_on_heavy_tailed_tiny_workload():
+    """Qualitative expectations on heavy-tailed activations ("AWQ and
+    Activation-Aware Scaling"): scaling improves on plain RTN (alpha = 0) and
+    alpha = 1 over-corrects relative to the optimum."""
+    X = heavy_tailed_activations(256, 512, OutlierSpec(0.01, 20.0), 0)
+    W = gaussian_weight(512, 512, 0)
+    Xn, Wn = X.numpy(), W.numpy()
+    mse, best, _, _ = O.search_scale(Xn, Wn, O.act_stats(Xn), 4, 128, 20)
+    assert mse[best] < mse[0] and mse[best] < mse[-1] and 0 < best < 19
+
+
+# --------------------------------------------------------------------------
+# D7  clip search
+# --------------------------------------------------------------------------
+def test_clip_ratio_grid():
+    r = O.clip_ratios(20, 0.5)
+    assert r[0] == 1.0 and r[-1] == 0.5 and np.all(np.diff(r) < 0)
+    assert list(O.clip_ratios(1, 0.5)) == [1.0]
+
+
+def test_clip_ratio_one_is_unclipped():
+    X, W = random_layer(16, 256, 8, seed=12)
+    abar = O.act_stats(X.numpy())
+    s = O.scale_grid(abar, O.alpha_grid(20))[9]
+    a = O.quantize_groups(W.numpy(), s, 128, 4)
+    b = O.quantize_groups(W.numpy(), s, 128, 4, np.ones((8, 2), np.float32))
+    for key in ("q", "z", "delta", "deq"):
+        assert np.array_equal(a[key], b[key])
+
+
+def test_clip_search_bruteforce_tokens():
+    T, inn, out, nc = 40, 256, 8, 6
+    X, W = random_layer(T, inn, out, seed=13)
+    Xn, Wn = X.numpy(), W.numpy()
+    s = O.scale_grid(O.act_stats(Xn), O.alpha_grid(20))[8]
+    idx, E = O.search_clip(Xn, Wn, s, 4, 128, nc, 0.5)
+    r = O.clip_ratios(nc, 0.5).astype(np.float32)
+    X64 = Xn.astype(np.float64)
+    for c in range(nc):
+        qd = O.quantize_groups(Wn, s, 128, 4, np.full((out, 2), r[c], np.float32))
+        for o in range(out):
+            for k in range(2):
+                sl = slice(128 * k, 128 * (k + 1))
+                d = qd["deq"][o, sl].astype(np.float64) / s[sl].astype(np.float64) - Wn[o, sl].astype(np.float64)
+                e = float(np.sum((X64[:, sl] @ d) ** 2))
+                assert E[o, k, c] == pytest.approx(e, rel=1e-10)
+    assert np.array_equal(idx, np.argmin(E, axis=2))
+
+
+# --------------------------------------------------------------------------
+# D8  packing
+# --------------------------------------------------------------------------
+def test_pack_hand_worked(golden):
+    hdr, rows = golden("pack_int4.txt")
+    out, inn = int(hdr["out"]), int(hdr["in"])
+    W = np.zeros((out, inn), dtype=np.float16)
+    for o in range(out):
+        for j in range(8):
+            W[o, j] = ((o + j) % 16) - 8
+        W[o, 126], W[o, 127] = -8.0, 7.0
+    qweight, qzeros, scales = O.quant_pack(W, None, None, 4, 128)
+    assert qweight.shape == (inn, out // 8) and qzeros.shape == (1, 1) and scales.shape == (1, out)
+    for r in rows:
+        assert int(qweight.view(np.uint32)[int(r[0]), 0]) == int(r[1], 16), r
+    assert int(qzeros.view(np.uint32)[0, 0]) == int(hdr["qzeros_hex"], 16)
+    assert np.all(scales == np.float16(float(hdr["scale"])))
+
+
+def test_pack_roundtrip_and_storage_bits(golden):
+    hdr, _ = golden("storage_bits.txt")
+    X, W = random_layer(16, 512, 64, seed=15)
+    Wn = W.numpy()
+    s = O.scale_grid(O.act_stats(X.numpy()), O.alpha_grid(20))[11]
+    idx = np.random.default_rng(0).integers(0, 20, size=(64, 4)).astype(np.uint8)
+    qweight, qzeros, scales = O.quant_pack(Wn, s, idx, 3, 128, 20, 0.5)
+    r = O.clip_ratios(20, 0.5).astype(np.float32)[idx.astype(np.int64)]
+    qd = O.quantize_groups(Wn, s, 128, 3, r)
+    assert np.array_equal(O.unpack_nibbles(qweight), qd["q"])
+    assert np.array_equal(O.unpack_nibbles(qzeros), qd["z"])
+    assert np.array_equal(scales, qd["delta"].T.astype(np.float16))
+    assert O.unpack_nibbles(qweight).max() <= 7
+    g = int(hdr["group"])
+    Xg, Wg = random_layer(4, 1024, 256, seed=16)
+    qw, qz, sc = O.quant_pack(Wg.numpy(), None, None, 4, g)
+    bits = 8.0 * (qw.nbytes + qz.nbytes + sc.nbytes) / Wg.numel()
+    assert bits == float(hdr["bits_per_weight"])
+    assert round(bits, 3) == float(hdr["printed"])
+
+
+def test_fold_keeps_the_product():
+    """Folding 1/s into the preceding op keeps the layer's function
+    ("AWQ and Activation-Aware Scaling"): (gamma / s) * (s w) = gamma * w up to
+    the fp16 rounding of the folded vector."""
+    rng = np.random.default_rng(3)
+    gamma = rng.uniform(0.5, 1.5, 256).astype(np.float16)
+    s = np.exp(rng.normal(0, 1, 256)).astype(np.float32)
+    g2 = O.fold_inv_scale(gamma, s)
+    assert np.allclose(g2.astype(np.float64) * s, gamma.astype(np.float64), rtol=2 ** -10)
+    rows = rng.normal(0, 0.02, (256, 64)).astype(np.float16)
+    r2 = O.fold_inv_scale(rows, s)
+    # half an fp16 ulp of the folded value (relative 2^-11, or 2^-25 absolute in
+    # the subnormal range), carried back through the multiplication by s
+    err = np.abs(r2.astype(np.float64) * s[:, None] - rows.astype(np.float64))
+    assert np.all(err <= 2.0 ** -11 * np.abs(rows.astype(np.float64)) * 1.001 + 2.0 ** -25 * s[:, None])
