@@ -1,0 +1,175 @@
+/*
+ * awq.h — C ABI of the B200 (sm_100a) AWQ per-layer scale search.
+ *
+ * AWQ ("AWQ and Activation-Aware Scaling", "Scaling instead of protecting";
+ * "05 — AWQ: Activation-Aware Weight Scaling" §3–§5) protects the weight
+ * channels that meet large activations by a per-input-channel scale
+ * s = abar^alpha applied before quantisation, with 1/s folded into the
+ * activations.  This library runs the search that picks s for one linear
+ * layer (or one group of linears that share an input), then the optional
+ * per-group clip search, then packs the result.  Call order per layer:
+ *
+ *   awq_act_stats -> awq_search_scale -> [awq_search_clip] -> awq_quant_pack
+ *
+ * Conventions shared by every call
+ *   - Pointers named as "device" are CUDA device pointers owned by the caller;
+ *     the library allocates no device memory.  Scratch memory comes from the
+ *     caller's workspace `ws` of at least awq_workspace_size() bytes,
+ *     256-byte aligned.  X and W must be 16-byte aligned.
+ *   - Every call is asynchronous and ordered on `stream` (a cudaStream_t; NULL
+ *     is the legacy default stream).  Outputs are valid once the stream has
+ *     been synchronised.  Calls that share a workspace must not overlap.
+ *   - Arguments are checked on the host before anything is launched; a failed
+ *     check returns AWQ_ERR_INVALID_ARG or AWQ_ERR_UNSUPPORTED and has no side
+ *     effect.  awq_last_error() returns a message for the calling thread.
+ *   - Device-side failures (a bounded wait in a kernel that ran out) are
+ *     recorded in a status word inside the workspace; awq_device_status()
+ *     synchronises the stream and reports and clears it.  Every call that
+ *     takes a workspace clears that word first, so it describes the latest
+ *     such call.
+ *   - X is [T, in] fp16, token-major, row stride ldx >= in elements (ldx a
+ *     multiple of 8).  W is [out, in] fp16, row-major and contiguous, laid out
+ *     like nn.Linear.  Linears that share one input and one scale (q|k|v,
+ *     gate|up) are passed concatenated along out.
+ *   - Quantisation (all calls): groups of g consecutive input channels of one
+ *     output row, asymmetric min/max with a zero point, b-bit codes, every
+ *     float step in fp32 with round-half-to-even:
+ *        wt = s*w;  mx, mn = max, min of wt (times r when clipping);
+ *        d = max(mx - mn, 1e-5);  delta = d / (2^b - 1);
+ *        z = clamp(rne(-mn/delta), 0, 2^b - 1);
+ *        q = clamp(rne(wt/delta) + z, 0, 2^b - 1);  deq = (q - z)*delta.
+ */
+#ifndef AWQ_H_
+#define AWQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void *awq_stream_t; /* a cudaStream_t */
+
+typedef enum {
+  AWQ_OK = 0,
+  AWQ_ERR_INVALID_ARG = 1, /* a size, stride, pointer or alignment is wrong   */
+  AWQ_ERR_UNSUPPORTED = 2, /* a valid setting this build does not implement   */
+  AWQ_ERR_WORKSPACE = 3,   /* workspace missing, misaligned or too small      */
+  AWQ_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed               */
+  AWQ_ERR_TIMEOUT = 5,     /* a bounded device-side wait ran out              */
+  AWQ_ERR_NONFINITE = 6    /* a score came out NaN or infinite                */
+} awq_status;
+
+/* Quantisation and search settings; the first three fields are the pages'
+ * quant_config ("05 — AWQ" §9: w_bit, q_group_size, zero_point). */
+typedef struct {
+  int32_t w_bit;      /* 3 or 4                                                  */
+  int32_t group_size; /* 128 (the pages' g); must divide in                      */
+  int32_t zero_point; /* 1 = asymmetric min/max with zero point (only mode)      */
+  int32_t n_alpha;    /* alpha grid size, 1..64; alpha_i = i/(n_alpha-1) ("05 — AWQ" §4: ~20) */
+  int32_t n_clip;     /* clip grid size, 0 = no clip search, else 1..64          */
+  float clip_min;     /* smallest clip ratio, in (0, 1]; ("05 — AWQ" §4: 0.5)    */
+} awq_config;
+
+/* Bytes of workspace needed by awq_search_scale and awq_search_clip for a
+ * layer with T tokens, `in` input and `out` output channels.  Returns 0 when
+ * the arguments are invalid (see awq_last_error()). */
+size_t awq_workspace_size(int64_t T, int64_t in, int64_t out, const awq_config *cfg);
+
+/* Per-input-channel mean activation magnitude ("AWQ and Activation-Aware
+ * Scaling", Scaling instead of protecting: abar; "05 — AWQ" §4, step 1).
+ *   X    device fp16 [T, in], row stride ldx (elements)
+ *   abar device fp64 [in] (output): abar_j = (sum_t |X_tj|) / T.  The sum is
+ *        exact (each fp16 is an integer multiple of 2^-24, summed as int64),
+ *        then converted to fp64 and divided by T with one rounding each.
+ *        abar's storage doubles as the int64 accumulator while the call runs.
+ * Requires T >= 1, in % 8 == 0, T * 65504 * 2^24 < 2^63 (T <= 2^22). */
+awq_status awq_act_stats(const void *X, int64_t T, int64_t in, int64_t ldx,
+                         double *abar, awq_stream_t stream);
+
+/* The candidate scale grid s_ij = RN32(pow(max(abar_j, 1e-4), alpha_i)),
+ * alpha_i = i/(n_alpha-1) ("AWQ and Activation-Aware Scaling": s = abar^alpha;
+ * "05 — AWQ" §4: ~20 values in [0, 1]).
+ *   abar device fp64 [in];  s device fp32 [n_alpha, in] (output). */
+awq_status awq_scale_grid(const double *abar, int64_t in, int32_t n_alpha, float *s,
+                          awq_stream_t stream);
+
+/* alpha-grid search ("05 — AWQ" §4 step 2–3; "AWQ and Activation-Aware
+ * Scaling": alpha found by a small per-layer grid search minimising
+ * reconstruction error).  For each alpha_i it fake-quantises diag(s_i) W and
+ * scores MSE_i = mean over tokens and outputs of
+ *   ((X diag(s_i)^-1) Qdeq(diag(s_i) W)^T - X W^T)^2,
+ * evaluated as ||X dW_i^T||^2 / (T out) with dW_i = Qdeq/s_i - W (the
+ * scaling invariance of "05 — AWQ" §3), on the tensor cores.
+ *   abar     device fp64 [in] from awq_act_stats
+ *   s_best   device fp32 [in]      (output) s of the selected alpha
+ *   mse      device fp64 [n_alpha] (output) MSE_i
+ *   best_idx device int32 [1]      (output) first index of the smallest MSE
+ * Requires in % 64 == 0, out % 8 == 0, ldx % 8 == 0. */
+awq_status awq_search_scale(const void *X, int64_t T, int64_t in, int64_t ldx,
+                            const void *W, int64_t out, const double *abar,
+                            const awq_config *cfg, void *ws, size_t ws_bytes,
+                            float *s_best, double *mse, int32_t *best_idx,
+                            awq_stream_t stream);
+
+/* Clip-ratio search ("05 — AWQ" §4, optional clipping: a ratio of 0.5–1.0 of
+ * the range, grid-searched after alpha).  For every output row o and group k
+ * it tries r_c = 1 - c (1 - clip_min)/(n_clip - 1), c = 0..n_clip-1, shrinking
+ * both ends of the group range, and keeps the first c minimising that
+ * group's own output error over all tokens,
+ *   E_okc = sum_t (sum_{j in k} X_tj (deq_c,oj / s_j - W_oj))^2
+ *         = d^T (X_k^T X_k) d,
+ * evaluated with an fp32 block Gram X_k^T X_k and fp32 quadratic forms.
+ *   s        device fp32 [in] (normally s_best); NULL means s = 1
+ *   clip_idx device uint8 [out, in/g] (output)
+ *   err      device fp32 [out, in/g, n_clip] (output, optional, may be NULL)
+ * Requires cfg->n_clip >= 1. */
+awq_status awq_search_clip(const void *X, int64_t T, int64_t in, int64_t ldx,
+                           const void *W, int64_t out, const float *s,
+                           const awq_config *cfg, void *ws, size_t ws_bytes,
+                           uint8_t *clip_idx, float *err, awq_stream_t stream);
+
+/* Final quantisation and packing ("05 — AWQ" §5 bit-level output format).
+ *   s        device fp32 [in] or NULL (s = 1)
+ *   clip_idx device uint8 [out, in/g] or NULL (ratio 1)
+ *   qweight  device int32 [in, out/8]:   code of (o, j) in bits 4(o%8)..+3 of [j][o/8]
+ *   qzeros   device int32 [in/g, out/8]: zero of (o, k) in bits 4(o%8)..+3 of [k][o/8]
+ *   scales   device fp16 [in/g, out]:    RN16(delta of (o, k))
+ * INT3 codes use the same 4-bit container. */
+awq_status awq_quant_pack(const void *W, int64_t out, int64_t in, const float *s,
+                          const uint8_t *clip_idx, const awq_config *cfg,
+                          int32_t *qweight, int32_t *qzeros, void *scales,
+                          awq_stream_t stream);
+
+/* Folds 1/s into the operation that feeds the scaled linear ("AWQ and
+ * Activation-Aware Scaling": the activation-side division is absorbed by the
+ * preceding normalisation's scale or linear layer).  v is device fp16
+ * [rows, cols]; row j is replaced by RN16(RN32(v_j) / s_j) (rows = in; cols = 1
+ * for a norm's gamma, or the preceding linear's input width). */
+awq_status awq_fold_inv_scale(void *v, int64_t rows, int64_t cols, const float *s,
+                              awq_stream_t stream);
+
+/* Synchronises `stream`, then returns and clears the device status recorded in
+ * workspace `ws` (AWQ_OK, AWQ_ERR_TIMEOUT or AWQ_ERR_NONFINITE). */
+awq_status awq_device_status(void *ws, awq_stream_t stream);
+
+/* Message describing the last failure on the calling thread ("" if none). */
+const char *awq_last_error(void);
+
+/* Per-kernel timing with CUDA events recorded on the launch stream.
+ * awq_profile_enable(1) starts recording every kernel this library launches;
+ * awq_profile_read() synchronises the recorded events and returns, for the
+ * kernel named `name`, the summed device time in ms and the launch count;
+ * awq_profile_reset() forgets all records.  Off by default. */
+awq_status awq_profile_enable(int32_t on);
+awq_status awq_profile_read(const char *name, double *total_ms, int64_t *launches);
+awq_status awq_profile_reset(void);
+
+/* Library version string. */
+const char *awq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* AWQ_H_ */

@@ -270,7 +270,7 @@ def quant_pack(W: np.ndarray, s: Optional[np.ndarray], clip_idx: Optional[np.nda
     for e in range(8):
         qweight |= q[e::8, :].T << np.uint32(4 * e)
         qzeros |= z[e::8, :].T << np.uint32(4 * e)
-    scales = qd["delta"].T.astype(np.float16)
+    scales = np.ascontiguousarray(qd["delta"].T.astype(np.float16))
     return qweight.view(np.int32), qzeros.view(np.int32), scales
 
 

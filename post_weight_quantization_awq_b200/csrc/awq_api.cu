@@ -1,0 +1,433 @@
+// Host implementation of the C ABI declared in include/awq.h: argument
+// checks, workspace carving, kernel launches, per-thread error messages and
+// optional per-kernel event timing.
+#include <cuda_runtime.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "awq.h"
+#include "awq_launch.h"
+
+using namespace awq;
+
+namespace {
+
+thread_local std::string g_err;
+
+awq_status fail(awq_status st, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_err = buf;
+  return st;
+}
+
+awq_status cuda_fail(cudaError_t e, const char *what) {
+  return fail(AWQ_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int64_t round_up(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
+
+int num_sms_current() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!cached[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+// --------------------------------------------------------------- profiling
+struct ProfRec {
+  const char *name;
+  cudaEvent_t a, b;
+};
+std::mutex g_prof_mu;
+bool g_prof_on = false;
+std::vector<ProfRec> g_prof;
+std::vector<cudaEvent_t> g_ev_pool;
+
+cudaEvent_t take_event() {
+  if (!g_ev_pool.empty()) {
+    cudaEvent_t e = g_ev_pool.back();
+    g_ev_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+struct ProfScope {
+  const char *name;
+  cudaStream_t s;
+  cudaEvent_t a = nullptr;
+  ProfScope(const char *n, cudaStream_t st) : name(n), s(st) {
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    if (g_prof_on) {
+      a = take_event();
+      cudaEventRecord(a, s);
+    }
+  }
+  ~ProfScope() {
+    if (!a) return;
+    std::lock_guard<std::mutex> lk(g_prof_mu);
+    cudaEvent_t b = take_event();
+    cudaEventRecord(b, s);
+    g_prof.push_back({name, a, b});
+  }
+};
+
+// ------------------------------------------------------------ validation
+awq_status check_cfg(const awq_config *cfg) {
+  if (!cfg) return fail(AWQ_ERR_INVALID_ARG, "cfg is NULL");
+  if (cfg->w_bit < 1 || cfg->w_bit > 8) return fail(AWQ_ERR_INVALID_ARG, "w_bit=%d", cfg->w_bit);
+  if (cfg->w_bit != 3 && cfg->w_bit != 4)
+    return fail(AWQ_ERR_UNSUPPORTED, "w_bit=%d (3 or 4 supported)", cfg->w_bit);
+  if (cfg->group_size <= 0) return fail(AWQ_ERR_INVALID_ARG, "group_size=%d", cfg->group_size);
+  if (cfg->group_size != 128)
+    return fail(AWQ_ERR_UNSUPPORTED, "group_size=%d (128 supported)", cfg->group_size);
+  if (cfg->zero_point != 1)
+    return fail(AWQ_ERR_UNSUPPORTED, "zero_point=%d (asymmetric, 1, supported)", cfg->zero_point);
+  if (cfg->n_alpha < 1 || cfg->n_alpha > 64)
+    return fail(AWQ_ERR_INVALID_ARG, "n_alpha=%d (1..64)", cfg->n_alpha);
+  if (cfg->n_clip < 0 || cfg->n_clip > 64)
+    return fail(AWQ_ERR_INVALID_ARG, "n_clip=%d (0..64)", cfg->n_clip);
+  if (!(cfg->clip_min > 0.0f && cfg->clip_min <= 1.0f))
+    return fail(AWQ_ERR_INVALID_ARG, "clip_min=%g (must be in (0, 1])", (double)cfg->clip_min);
+  return AWQ_OK;
+}
+
+awq_status check_shape(int64_t T, int64_t in, int64_t out, const awq_config *cfg) {
+  if (T < 1 || T > (int64_t(1) << 22)) return fail(AWQ_ERR_INVALID_ARG, "T=%lld (1..2^22)", (long long)T);
+  if (in < cfg->group_size || in % cfg->group_size != 0)
+    return fail(AWQ_ERR_INVALID_ARG, "in=%lld must be a positive multiple of group_size=%d",
+                (long long)in, cfg->group_size);
+  if (in > (int64_t(1) << 20)) return fail(AWQ_ERR_INVALID_ARG, "in=%lld too large", (long long)in);
+  if (out < 8 || out % 8 != 0 || out > (int64_t(1) << 22))
+    return fail(AWQ_ERR_INVALID_ARG, "out=%lld must be a positive multiple of 8", (long long)out);
+  return AWQ_OK;
+}
+
+awq_status check_x(const void *X, int64_t in, int64_t ldx) {
+  if (!X) return fail(AWQ_ERR_INVALID_ARG, "X is NULL");
+  if (!aligned(X, 16)) return fail(AWQ_ERR_INVALID_ARG, "X must be 16-byte aligned");
+  if (ldx < in || ldx % 8 != 0)
+    return fail(AWQ_ERR_INVALID_ARG, "ldx=%lld must be >= in and a multiple of 8", (long long)ldx);
+  return AWQ_OK;
+}
+
+// ------------------------------------------------------------ workspace
+constexpr size_t kHeader = 256;
+
+struct ScaleWs {
+  size_t s_grid, inv_s, dW, partials, end;
+  int64_t out_pad;
+  int num_m, nb_per_alpha;
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+ScaleWs scale_layout(int64_t T, int64_t in, int64_t out, const awq_config *cfg) {
+  ScaleWs w;
+  w.out_pad = round_up(out, kGemmBN);
+  w.num_m = (int)((T + kGemmBM - 1) / kGemmBM);
+  w.nb_per_alpha = (int)(w.out_pad / kGemmBN);
+  size_t off = kHeader;
+  w.s_grid = off;
+  off = align256(off + sizeof(float) * (size_t)cfg->n_alpha * in);
+  w.inv_s = off;
+  off = align256(off + sizeof(float) * (size_t)cfg->n_alpha * in);
+  w.dW = off;
+  off = align256(off + sizeof(__half) * (size_t)cfg->n_alpha * w.out_pad * in);
+  w.partials = off;
+  off = align256(off + sizeof(double) * (size_t)cfg->n_alpha * w.nb_per_alpha * w.num_m * 4);
+  w.end = off;
+  return w;
+}
+
+struct ClipWs {
+  size_t gpart, G, end;
+  int n_chunks;
+};
+
+ClipWs clip_layout(int64_t T, int64_t in) {
+  ClipWs w;
+  int64_t c = (T + 1023) / 1024;
+  w.n_chunks = (int)(c < 1 ? 1 : (c > 16 ? 16 : c));
+  const size_t gsz = sizeof(float) * (size_t)(in / 128) * 128 * 128;
+  size_t off = kHeader;
+  w.gpart = off;
+  off = align256(off + gsz * w.n_chunks);
+  w.G = off;
+  off = align256(off + gsz);
+  w.end = off;
+  return w;
+}
+
+uint32_t poll_cap() {
+  const char *f = getenv("AWQ_FAULT");
+  if (f && strcmp(f, "timeout") == 0) return 1u;  // test hook: every bounded wait gives up at once
+  return 1u << 24;
+}
+
+awq_status check_ws(void *ws, size_t ws_bytes, size_t need) {
+  if (!ws) return fail(AWQ_ERR_WORKSPACE, "workspace is NULL");
+  if (!aligned(ws, 256)) return fail(AWQ_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  if (ws_bytes < need)
+    return fail(AWQ_ERR_WORKSPACE, "workspace of %zu bytes is smaller than the %zu needed", ws_bytes,
+                need);
+  return AWQ_OK;
+}
+
+#define AWQ_TRY_CUDA(expr, what)                  \
+  do {                                            \
+    cudaError_t e_ = (expr);                      \
+    if (e_ != cudaSuccess) return cuda_fail(e_, what); \
+  } while (0)
+
+}  // namespace
+
+extern "C" {
+
+const char *awq_version(void) { return "awq-b200 0.1 (sm_100a)"; }
+
+const char *awq_last_error(void) { return g_err.c_str(); }
+
+size_t awq_workspace_size(int64_t T, int64_t in, int64_t out, const awq_config *cfg) {
+  if (check_cfg(cfg) != AWQ_OK) return 0;
+  if (check_shape(T, in, out, cfg) != AWQ_OK) return 0;
+  size_t need = scale_layout(T, in, out, cfg).end;
+  if (cfg->n_clip > 0) {
+    size_t c = clip_layout(T, in).end;
+    if (c > need) need = c;
+  }
+  return need;
+}
+
+awq_status awq_act_stats(const void *X, int64_t T, int64_t in, int64_t ldx, double *abar,
+                         awq_stream_t stream) {
+  g_err.clear();
+  if (T < 1 || T > (int64_t(1) << 22)) return fail(AWQ_ERR_INVALID_ARG, "T=%lld (1..2^22)", (long long)T);
+  if (in < 8 || in % 8 != 0) return fail(AWQ_ERR_INVALID_ARG, "in=%lld must be a multiple of 8", (long long)in);
+  awq_status st = check_x(X, in, ldx);
+  if (st != AWQ_OK) return st;
+  if (!abar || !aligned(abar, 8)) return fail(AWQ_ERR_INVALID_ARG, "abar is NULL or misaligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  ProfScope p("act_stats", s);
+  AWQ_TRY_CUDA(launch_act_stats(static_cast<const __half *>(X), T, in, ldx, abar,
+                                num_sms_current(), s),
+               "act_stats launch");
+  return AWQ_OK;
+}
+
+awq_status awq_scale_grid(const double *abar, int64_t in, int32_t n_alpha, float *s,
+                          awq_stream_t stream) {
+  g_err.clear();
+  if (!abar || !s) return fail(AWQ_ERR_INVALID_ARG, "abar or s is NULL");
+  if (in < 1 || in > (int64_t(1) << 24)) return fail(AWQ_ERR_INVALID_ARG, "in=%lld", (long long)in);
+  if (n_alpha < 1 || n_alpha > 64) return fail(AWQ_ERR_INVALID_ARG, "n_alpha=%d (1..64)", n_alpha);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  ProfScope p("scale_grid", st);
+  AWQ_TRY_CUDA(launch_scale_grid(abar, in, n_alpha, s, nullptr, st), "scale_grid launch");
+  return AWQ_OK;
+}
+
+awq_status awq_search_scale(const void *X, int64_t T, int64_t in, int64_t ldx, const void *W,
+                            int64_t out, const double *abar, const awq_config *cfg, void *ws,
+                            size_t ws_bytes, float *s_best, double *mse, int32_t *best_idx,
+                            awq_stream_t stream) {
+  g_err.clear();
+  awq_status st = check_cfg(cfg);
+  if (st != AWQ_OK) return st;
+  if ((st = check_shape(T, in, out, cfg)) != AWQ_OK) return st;
+  if ((st = check_x(X, in, ldx)) != AWQ_OK) return st;
+  if (!W || !aligned(W, 16)) return fail(AWQ_ERR_INVALID_ARG, "W is NULL or not 16-byte aligned");
+  if (!abar || !s_best || !mse || !best_idx) return fail(AWQ_ERR_INVALID_ARG, "an output pointer is NULL");
+  const ScaleWs L = scale_layout(T, in, out, cfg);
+  if ((st = check_ws(ws, ws_bytes, L.end)) != AWQ_OK) return st;
+  const int64_t tiles = (int64_t)L.num_m * L.nb_per_alpha * cfg->n_alpha;
+  if (tiles > INT32_MAX) return fail(AWQ_ERR_INVALID_ARG, "problem too large (%lld tiles)", (long long)tiles);
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t *base = static_cast<uint8_t *>(ws);
+  DevStatus *dst = reinterpret_cast<DevStatus *>(base);
+  float *s_grid = reinterpret_cast<float *>(base + L.s_grid);
+  float *inv_s = reinterpret_cast<float *>(base + L.inv_s);
+  __half *dW = reinterpret_cast<__half *>(base + L.dW);
+  double *partials = reinterpret_cast<double *>(base + L.partials);
+  const int nsm = num_sms_current();
+
+  // status of this call only: flags, site, exponent and max |W| start at zero
+  AWQ_TRY_CUDA(cudaMemsetAsync(dst, 0, sizeof(DevStatus), s), "workspace reset");
+  {
+    ProfScope p("wmax", s);
+    AWQ_TRY_CUDA(launch_wmax(static_cast<const __half *>(W), out * in, dst, nsm, s), "wmax launch");
+  }
+  {
+    ProfScope p("scale_grid", s);
+    AWQ_TRY_CUDA(launch_scale_grid(abar, in, cfg->n_alpha, s_grid, inv_s, s), "scale_grid launch");
+  }
+  {
+    ProfScope p("cand_quant", s);
+    AWQ_TRY_CUDA(launch_cand_quant(static_cast<const __half *>(W), out, in, L.out_pad, s_grid, inv_s,
+                                   cfg->n_alpha, cfg->group_size, cfg->w_bit, dst, dW, nsm, s),
+                 "cand_quant launch");
+  }
+  {
+    SearchGemmShape sh;
+    sh.T = T;
+    sh.in = in;
+    sh.rows_b = (int64_t)cfg->n_alpha * L.out_pad;
+    sh.num_m = L.num_m;
+    sh.num_n = (int)(sh.rows_b / kGemmBN);
+    sh.num_kb = (int)(in / kGemmBK);
+    ProfScope p("search_gemm", s);
+    AWQ_TRY_CUDA(launch_search_gemm(static_cast<const __half *>(X), ldx, dW, sh, partials, dst,
+                                    poll_cap(), nsm, s),
+                 "search_gemm launch");
+  }
+  {
+    ProfScope p("mse_argmin", s);
+    AWQ_TRY_CUDA(launch_mse_argmin(partials, cfg->n_alpha, L.nb_per_alpha, L.num_m, T, out, s_grid,
+                                   in, dst, mse, best_idx, s_best, s),
+                 "mse_argmin launch");
+  }
+  if (getenv("AWQ_SYNC_CHECK")) return awq_device_status(ws, stream);
+  return AWQ_OK;
+}
+
+awq_status awq_search_clip(const void *X, int64_t T, int64_t in, int64_t ldx, const void *W,
+                           int64_t out, const float *s, const awq_config *cfg, void *ws,
+                           size_t ws_bytes, uint8_t *clip_idx, float *err, awq_stream_t stream) {
+  g_err.clear();
+  awq_status st = check_cfg(cfg);
+  if (st != AWQ_OK) return st;
+  if (cfg->n_clip < 1) return fail(AWQ_ERR_INVALID_ARG, "n_clip=%d: clip search needs n_clip >= 1", cfg->n_clip);
+  if ((st = check_shape(T, in, out, cfg)) != AWQ_OK) return st;
+  if ((st = check_x(X, in, ldx)) != AWQ_OK) return st;
+  if (!W || !aligned(W, 16)) return fail(AWQ_ERR_INVALID_ARG, "W is NULL or not 16-byte aligned");
+  if (!clip_idx) return fail(AWQ_ERR_INVALID_ARG, "clip_idx is NULL");
+  if (s && !aligned(s, 16)) return fail(AWQ_ERR_INVALID_ARG, "s must be 16-byte aligned");
+  const ClipWs L = clip_layout(T, in);
+  if ((st = check_ws(ws, ws_bytes, L.end)) != AWQ_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  uint8_t *base = static_cast<uint8_t *>(ws);
+  float *gpart = reinterpret_cast<float *>(base + L.gpart);
+  float *Gk = reinterpret_cast<float *>(base + L.G);
+  AWQ_TRY_CUDA(cudaMemsetAsync(base, 0, sizeof(DevStatus), cs), "workspace reset");
+  {
+    ProfScope p("gram_blocks", cs);
+    AWQ_TRY_CUDA(launch_gram_blocks(static_cast<const __half *>(X), T, in, ldx, cfg->group_size,
+                                    L.n_chunks, gpart, Gk, cs),
+                 "gram_blocks launch");
+  }
+  {
+    ProfScope p("clip_eval", cs);
+    AWQ_TRY_CUDA(launch_clip_eval(static_cast<const __half *>(W), out, in, s, Gk, cfg->group_size,
+                                  cfg->w_bit, cfg->n_clip, cfg->clip_min, clip_idx, err, cs),
+                 "clip_eval launch");
+  }
+  return AWQ_OK;
+}
+
+awq_status awq_quant_pack(const void *W, int64_t out, int64_t in, const float *s,
+                          const uint8_t *clip_idx, const awq_config *cfg, int32_t *qweight,
+                          int32_t *qzeros, void *scales, awq_stream_t stream) {
+  g_err.clear();
+  awq_status st = check_cfg(cfg);
+  if (st != AWQ_OK) return st;
+  if ((st = check_shape(1, in, out, cfg)) != AWQ_OK) return st;
+  if (!W || !aligned(W, 16)) return fail(AWQ_ERR_INVALID_ARG, "W is NULL or not 16-byte aligned");
+  if (s && !aligned(s, 16)) return fail(AWQ_ERR_INVALID_ARG, "s must be 16-byte aligned");
+  if (clip_idx && cfg->n_clip < 1)
+    return fail(AWQ_ERR_INVALID_ARG, "clip_idx given but n_clip=%d", cfg->n_clip);
+  if (!qweight || !qzeros || !scales) return fail(AWQ_ERR_INVALID_ARG, "an output pointer is NULL");
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  ProfScope p("quant_pack", cs);
+  AWQ_TRY_CUDA(launch_quant_pack(static_cast<const __half *>(W), out, in, s, clip_idx,
+                                 cfg->group_size, cfg->w_bit, cfg->n_clip, cfg->clip_min, qweight,
+                                 qzeros, static_cast<__half *>(scales), cs),
+               "quant_pack launch");
+  return AWQ_OK;
+}
+
+awq_status awq_fold_inv_scale(void *v, int64_t rows, int64_t cols, const float *s,
+                              awq_stream_t stream) {
+  g_err.clear();
+  if (!v || !s) return fail(AWQ_ERR_INVALID_ARG, "v or s is NULL");
+  if (rows < 1 || cols < 1) return fail(AWQ_ERR_INVALID_ARG, "rows=%lld cols=%lld", (long long)rows, (long long)cols);
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  ProfScope p("fold", cs);
+  AWQ_TRY_CUDA(launch_fold(static_cast<__half *>(v), rows, cols, s, cs), "fold launch");
+  return AWQ_OK;
+}
+
+awq_status awq_device_status(void *ws, awq_stream_t stream) {
+  g_err.clear();
+  if (!ws || !aligned(ws, 256)) return fail(AWQ_ERR_WORKSPACE, "workspace is NULL or misaligned");
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  AWQ_TRY_CUDA(cudaStreamSynchronize(cs), "stream synchronize");
+  DevStatus h;
+  AWQ_TRY_CUDA(cudaMemcpy(&h, ws, sizeof(h), cudaMemcpyDeviceToHost), "status read");
+  const uint32_t zero[2] = {0, 0};
+  AWQ_TRY_CUDA(cudaMemcpy(ws, zero, sizeof(zero), cudaMemcpyHostToDevice), "status clear");
+  if (h.flags & kDevTimeout)
+    return fail(AWQ_ERR_TIMEOUT, "a bounded device wait ran out (site 0x%x)", h.where);
+  if (h.flags & kDevNonFinite) return fail(AWQ_ERR_NONFINITE, "a candidate score is not finite");
+  return AWQ_OK;
+}
+
+awq_status awq_profile_enable(int32_t on) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  g_prof_on = on != 0;
+  return AWQ_OK;
+}
+
+awq_status awq_profile_read(const char *name, double *total_ms, int64_t *launches) {
+  g_err.clear();
+  if (!name || !total_ms || !launches) return fail(AWQ_ERR_INVALID_ARG, "NULL argument");
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  double tot = 0.0;
+  int64_t n = 0;
+  for (const ProfRec &r : g_prof) {
+    if (strcmp(r.name, name) != 0) continue;
+    cudaError_t e = cudaEventSynchronize(r.b);
+    if (e != cudaSuccess) return cuda_fail(e, "event synchronize");
+    float ms = 0.0f;
+    e = cudaEventElapsedTime(&ms, r.a, r.b);
+    if (e != cudaSuccess) return cuda_fail(e, "event elapsed time");
+    tot += ms;
+    ++n;
+  }
+  *total_ms = tot;
+  *launches = n;
+  return AWQ_OK;
+}
+
+awq_status awq_profile_reset(void) {
+  std::lock_guard<std::mutex> lk(g_prof_mu);
+  for (const ProfRec &r : g_prof) {
+    cudaEventSynchronize(r.b);
+    g_ev_pool.push_back(r.a);
+    g_ev_pool.push_back(r.b);
+  }
+  g_prof.clear();
+  return AWQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,246 @@
+// Device-side building blocks shared by the AWQ kernels: the fp32 group
+// quantiser, the device status word, and thin inline-PTX wrappers for the
+// sm_100a features the scored GEMM uses (mbarrier, TMA, tcgen05/TMEM).
+#pragma once
+
+#include <cuda_fp16.h>
+#include <stdint.h>
+
+namespace awq {
+
+// ---------------------------------------------------------------------------
+// Device status word (first bytes of every workspace).
+// ---------------------------------------------------------------------------
+enum : uint32_t {
+  kDevOk = 0,
+  kDevTimeout = 1u << 0,    // a bounded wait ran out
+  kDevNonFinite = 1u << 1,  // a score was NaN or infinite
+};
+
+struct DevStatus {
+  uint32_t flags;     // kDev* bits, OR-ed by kernels
+  uint32_t where;     // code of the first wait that ran out (debug aid)
+  int32_t kscale;     // power-of-two exponent applied to the candidate errors
+  uint32_t wmax_bits; // bit pattern of max |W| (a non-negative float)
+};
+
+__device__ __forceinline__ void dev_fail(DevStatus *st, uint32_t flag, uint32_t where) {
+  if (st) {
+    atomicOr(&st->flags, flag);
+    atomicCAS(&st->where, 0u, where);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Group quantiser ("05 — AWQ" §5/§9: groups of g input channels, asymmetric
+// min/max with a zero point).  Every step is fp32, correctly rounded, with
+// round-half-to-even; the explicit _rn intrinsics keep the compiler from
+// contracting any of them into an FMA.
+// ---------------------------------------------------------------------------
+struct GroupQ {
+  float delta;  // step
+  float zero;   // zero point (integer valued)
+  float qmax;   // 2^b - 1
+  float rcp;    // RN(1/delta), used for the fast code path
+};
+
+// Range of one group after the optional clip ratio r32 (1 = no clip).
+__device__ __forceinline__ GroupQ group_params(float mx, float mn, float r32, float qmax) {
+  if (r32 != 1.0f) {
+    mx = __fmul_rn(r32, mx);
+    mn = __fmul_rn(r32, mn);
+  }
+  float d = fmaxf(__fsub_rn(mx, mn), 1e-5f);
+  GroupQ g;
+  g.delta = __fdiv_rn(d, qmax);
+  float z = rintf(__fdiv_rn(-mn, g.delta));
+  g.zero = fminf(fmaxf(z, 0.0f), qmax);
+  g.qmax = qmax;
+  g.rcp = __frcp_rn(g.delta);
+  return g;
+}
+
+// rne(RN32(wt / delta)) without a full division on the common path: y =
+// RN(wt * RN(1/delta)) is within 1.5 ulp of wt/delta, so unless y lies within
+// a few ulp of a half-integer both round to the same integer; otherwise (or
+// for very large quotients) fall back to the correctly rounded quotient.
+__device__ __forceinline__ float round_quotient(float wt, const GroupQ &g) {
+  float y = __fmul_rn(wt, g.rcp);
+  float ay = fabsf(y);
+  float h = __fadd_rn(floorf(y), 0.5f);
+  float dist = fabsf(__fsub_rn(y, h));
+  if (ay < 1048576.0f && dist > __fmul_rn(fmaxf(ay, 1.0f), 4.76837158203125e-07f /*2^-21*/)) {
+    return rintf(y);
+  }
+  return rintf(__fdiv_rn(wt, g.delta));
+}
+
+__device__ __forceinline__ float quant_code(float wt, const GroupQ &g) {
+  float q = __fadd_rn(round_quotient(wt, g), g.zero);
+  return fminf(fmaxf(q, 0.0f), g.qmax);
+}
+
+__device__ __forceinline__ float dequant(float q, const GroupQ &g) {
+  return __fmul_rn(__fsub_rn(q, g.zero), g.delta);
+}
+
+// ---------------------------------------------------------------------------
+// Bounded waits.  A wait that exceeds its poll budget records kDevTimeout and
+// returns false; callers stop issuing work and drain what is in flight.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Waits until the phase with `parity` of `bar` has completed.  Gives up after
+// `max_polls` polls or as soon as *abort is set; returns true on success.
+__device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity,
+                                                  uint32_t max_polls,
+                                                  volatile int *abort) {
+  for (uint32_t i = 0; i < max_polls; ++i) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (abort && *abort) return false;
+    if (i > 64) __nanosleep(32);
+  }
+  return false;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// TMA (cp.async.bulk.tensor), 2-D tiles, no multicast.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void tma_prefetch_desc(const void *tmap) {
+  asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
+}
+
+__device__ __forceinline__ void tma_load_2d(void *smem_dst, const void *tmap, uint64_t *bar,
+                                            int32_t x, int32_t y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// tcgen05 / TMEM.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void tmem_alloc(uint32_t *smem_result, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                   smem_u32(smem_result)),
+               "r"(ncols)
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::f16, one CTA.
+__device__ __forceinline__ void tc_mma_f16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                           uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// Arrives on `bar` once every tcgen05 operation this thread issued so far has
+// completed.
+__device__ __forceinline__ void tc_commit(uint64_t *bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+
+// 32 lanes x 32 consecutive fp32 columns: thread i of the warp gets lane
+// (base lane + i), columns [col, col + 32).
+__device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_ld_wait() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor for a K-major operand tile written by TMA
+// with 128-byte swizzling: rows of 64 fp16 (128 B), 8-row core groups 1024 B
+// apart.  Fields: start address >> 4 (bits 0-13), leading byte offset >> 4
+// (bits 16-29, unused for swizzled K-major, set to 1), stride byte offset >> 4
+// (bits 32-45), descriptor version 1 (bits 46-47), base offset 0, swizzle mode
+// 2 = 128B (bits 61-63).
+__device__ __forceinline__ uint64_t smem_desc_k_sw128(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((smem_addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1u << 16;
+  d |= (uint64_t)(1024u >> 4) << 32;
+  d |= (uint64_t)1u << 46;
+  d |= (uint64_t)2u << 61;
+  return d;
+}
+
+// Instruction descriptor, kind::f16: fp16 A and B (format 0), fp32 accumulator
+// (bits 4-5 = 1), both K-major, N >> 3 at bits 17-22, M >> 4 at bits 24-28.
+__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
+  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+}  // namespace awq

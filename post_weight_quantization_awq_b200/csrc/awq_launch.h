@@ -1,0 +1,78 @@
+// Internal launchers of the AWQ kernels (host side).  Every launcher only
+// enqueues work on `stream` and returns the launch error, if any.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "awq_device.cuh"
+
+namespace awq {
+
+__host__ __device__ constexpr int64_t i64min(int64_t a, int64_t b) { return a < b ? a : b; }
+__host__ __device__ constexpr int64_t i64max(int64_t a, int64_t b) { return a > b ? a : b; }
+
+// K1: abar (exact mean |x|).  abar doubles as the int64 accumulator.
+cudaError_t launch_act_stats(const __half *X, int64_t T, int64_t in, int64_t ldx, double *abar,
+                             int num_sms, cudaStream_t stream);
+
+// K2: s[i][j] = RN32(pow(max(abar_j, 1e-4), i/(n-1))); inv_s (optional) = RN(1/s).
+cudaError_t launch_scale_grid(const double *abar, int64_t in, int n_alpha, float *s, float *inv_s,
+                              cudaStream_t stream);
+
+// max |W| into st->wmax_bits (st->wmax_bits must be zero beforehand).
+cudaError_t launch_wmax(const __half *W, int64_t n, DevStatus *st, int num_sms, cudaStream_t stream);
+
+// K3: candidate effective errors dW[i][o][j] = RN16(2^k (deq/s - w)), rows
+// out..out_pad-1 zero.
+cudaError_t launch_cand_quant(const __half *W, int64_t out, int64_t in, int64_t out_pad,
+                              const float *s, const float *inv_s, int n_alpha, int group, int w_bit,
+                              const DevStatus *st, __half *dW, int num_sms, cudaStream_t stream);
+
+// K4: scored GEMM, partial sums of squares per (n-tile, m-tile, warp).
+struct SearchGemmShape {
+  int64_t T, in, rows_b;  // rows_b = n_alpha * out_pad
+  int num_m, num_n, num_kb;
+};
+cudaError_t launch_search_gemm(const __half *X, int64_t ldx, const __half *dW,
+                               const SearchGemmShape &sh, double *partials, DevStatus *st,
+                               uint32_t max_polls, int num_sms, cudaStream_t stream);
+constexpr int kGemmBM = 128, kGemmBN = 256, kGemmBK = 64;
+
+// K5: mse[i], best index, s_best.
+cudaError_t launch_mse_argmin(const double *partials, int n_alpha, int nb_per_alpha, int num_m,
+                              int64_t T, int64_t out, const float *s_grid, int64_t in,
+                              DevStatus *st, double *mse, int32_t *best_idx, float *s_best,
+                              cudaStream_t stream);
+
+// K6a: block Grams G[k] = X_k^T X_k (fp32), via per-chunk partials.
+cudaError_t launch_gram_blocks(const __half *X, int64_t T, int64_t in, int64_t ldx, int group,
+                               int n_chunks, float *partials, float *G, cudaStream_t stream);
+// K6b: clip choice per (row, group).
+cudaError_t launch_clip_eval(const __half *W, int64_t out, int64_t in, const float *s,
+                             const float *G, int group, int w_bit, int n_clip, float clip_min,
+                             uint8_t *clip_idx, float *err, cudaStream_t stream);
+
+// K7: final codes + packing.
+cudaError_t launch_quant_pack(const __half *W, int64_t out, int64_t in, const float *s,
+                              const uint8_t *clip_idx, int group, int w_bit, int n_clip,
+                              float clip_min, int32_t *qweight, int32_t *qzeros, __half *scales,
+                              cudaStream_t stream);
+
+// K8: v[j][:] = RN16(RN32(v[j][:]) / s_j).
+cudaError_t launch_fold(__half *v, int64_t rows, int64_t cols, const float *s, cudaStream_t stream);
+
+// Exponent k of the power-of-two factor applied to the candidate errors, from
+// max |W|: |deq/s - w| <= 2|w| (+ rounding), so 2 max|W| 2^k <= 2^14 keeps
+// every scaled error inside fp16 with a factor-4 margin.
+__host__ __device__ inline int kscale_from_wmax(float wmax) {
+  if (!(wmax > 0.0f)) return 0;
+  int e;
+  (void)frexpf(wmax, &e);  // wmax < 2^e
+  int k = 13 - e;
+  if (k > 60) k = 60;
+  if (k < -60) k = -60;
+  return k;
+}
+
+}  // namespace awq

@@ -1,0 +1,373 @@
+// HBM-bound kernels of the AWQ scale search: the activation statistic (K1),
+// the candidate scale grid (K2), max |W|, the candidate quantiser that writes
+// the tensor-core B operand (K3), final quantisation + packing (K7) and the
+// 1/s fold (K8).
+#include <cuda_fp16.h>
+#include <math.h>
+
+#include "awq_launch.h"
+
+namespace awq {
+
+// ---------------------------------------------------------------------------
+// K1 — abar_j = (sum_t |X_tj|) / T, exact  ("AWQ and Activation-Aware
+// Scaling", Scaling instead of protecting: abar is the per-channel mean
+// activation magnitude; "05 — AWQ" §4 step 1).
+//
+// Each thread owns 8 consecutive channels (one 16-byte load per token row) and
+// sums |x| over its share of a token chunk in fp64.  Every |x| is a multiple of
+// 2^-24 below 2^16, and a chunk holds at most 4096 tokens, so partial sums stay
+// below 2^29 and are exact in fp64.  Chunk sums are then converted to int64
+// units of 2^-24 (exact) and added with 64-bit integer atomics (exact, so the
+// order of arrival does not matter).  Block: 32 x 8 threads covering 256
+// channels x 8 token rows per step.
+// ---------------------------------------------------------------------------
+constexpr int kStatsChunk = 1024;  // tokens per block (<= 4096 keeps fp64 exact)
+
+__global__ void __launch_bounds__(256) act_stats_kernel(const __half *__restrict__ X, int64_t T,
+                                                        int64_t in, int64_t ldx,
+                                                        unsigned long long *__restrict__ acc) {
+  __shared__ double red[8][32][8];
+  const int tx = threadIdx.x, ty = threadIdx.y;
+  const int64_t c0 = ((int64_t)blockIdx.x * 32 + tx) * 8;  // first channel of this thread
+  const int64_t t_begin = (int64_t)blockIdx.y * kStatsChunk;
+  const int64_t t_end = min(T, t_begin + kStatsChunk);
+  double s[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) s[e] = 0.0;
+  if (c0 < in) {
+    int64_t t = t_begin + ty;
+    // four rows in flight per thread
+    for (; t + 24 < t_end; t += 32) {
+      uint4 v[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        v[u] = __ldcs(reinterpret_cast<const uint4 *>(X + (t + 8 * u) * ldx + c0));
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t w[4] = {v[u].x & 0x7FFF7FFFu, v[u].y & 0x7FFF7FFFu, v[u].z & 0x7FFF7FFFu,
+                               v[u].w & 0x7FFF7FFFu};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[h]));
+          s[2 * h] += (double)f.x;
+          s[2 * h + 1] += (double)f.y;
+        }
+      }
+    }
+    for (; t < t_end; t += 8) {
+      uint4 v = __ldcs(reinterpret_cast<const uint4 *>(X + t * ldx + c0));
+      const uint32_t w[4] = {v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu, v.z & 0x7FFF7FFFu,
+                             v.w & 0x7FFF7FFFu};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[h]));
+        s[2 * h] += (double)f.x;
+        s[2 * h + 1] += (double)f.y;
+      }
+    }
+  }
+#pragma unroll
+  for (int e = 0; e < 8; ++e) red[ty][tx][e] = s[e];
+  __syncthreads();
+  if (ty == 0 && c0 < in) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      double tot = 0.0;
+#pragma unroll
+      for (int r = 0; r < 8; ++r) tot += red[r][tx][e];
+      // exact: tot is a multiple of 2^-24 below 2^29
+      unsigned long long units = (unsigned long long)(tot * 16777216.0);
+      if (units) atomicAdd(&acc[c0 + e], units);
+    }
+  }
+}
+
+__global__ void act_stats_finish_kernel(double *abar, int64_t in, int64_t T) {
+  int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (j < in) {
+    long long units = reinterpret_cast<long long *>(abar)[j];
+    double S = __ll2double_rn(units) * 5.9604644775390625e-08;  // * 2^-24, exact
+    abar[j] = __ddiv_rn(S, (double)T);
+  }
+}
+
+cudaError_t launch_act_stats(const __half *X, int64_t T, int64_t in, int64_t ldx, double *abar,
+                             int num_sms, cudaStream_t stream) {
+  (void)num_sms;
+  cudaError_t e = cudaMemsetAsync(abar, 0, sizeof(double) * in, stream);
+  if (e != cudaSuccess) return e;
+  dim3 block(32, 8);
+  dim3 grid((unsigned)((in + 255) / 256), (unsigned)((T + kStatsChunk - 1) / kStatsChunk));
+  act_stats_kernel<<<grid, block, 0, stream>>>(X, T, in, ldx,
+                                               reinterpret_cast<unsigned long long *>(abar));
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  act_stats_finish_kernel<<<(unsigned)((in + 255) / 256), 256, 0, stream>>>(abar, in, T);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// K2 — s_ij = RN32(pow(max(abar_j, 1e-4), alpha_i)), alpha_i = i/(n-1)
+// ("AWQ and Activation-Aware Scaling": s = abar^alpha; "05 — AWQ" §4: ~20
+// values of alpha in [0, 1]).  pow is CUDA's double pow.
+// ---------------------------------------------------------------------------
+__global__ void scale_grid_kernel(const double *__restrict__ abar, int64_t in, int n_alpha,
+                                  float *__restrict__ s, float *__restrict__ inv_s) {
+  int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= in * n_alpha) return;
+  int i = (int)(idx / in);
+  int64_t j = idx - (int64_t)i * in;
+  double alpha = n_alpha > 1 ? __ddiv_rn((double)i, (double)(n_alpha - 1)) : 0.0;
+  double a = fmax(abar[j], 1e-4);
+  float v = __double2float_rn(pow(a, alpha));
+  s[idx] = v;
+  if (inv_s) inv_s[idx] = __frcp_rn(v);
+}
+
+cudaError_t launch_scale_grid(const double *abar, int64_t in, int n_alpha, float *s, float *inv_s,
+                              cudaStream_t stream) {
+  int64_t n = in * n_alpha;
+  scale_grid_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(abar, in, n_alpha, s, inv_s);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// max |W| (bit pattern of a non-negative float orders like an unsigned int).
+// ---------------------------------------------------------------------------
+__global__ void wmax_kernel(const __half *__restrict__ W, int64_t n, DevStatus *st) {
+  uint32_t m = 0;
+  const int64_t n8 = n / 8;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    uint4 v = __ldg(reinterpret_cast<const uint4 *>(W) + i);
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[h]));
+      m = max(m, __float_as_uint(fabsf(f.x)));
+      m = max(m, __float_as_uint(fabsf(f.y)));
+    }
+  }
+  for (int64_t i = n8 * 8 + (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x)
+    m = max(m, __float_as_uint(fabsf(__half2float(W[i]))));
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
+  if ((threadIdx.x & 31) == 0 && m) atomicMax(&st->wmax_bits, m);
+}
+
+cudaError_t launch_wmax(const __half *W, int64_t n, DevStatus *st, int num_sms,
+                        cudaStream_t stream) {
+  int64_t blocks = i64min((int64_t)num_sms * 4, (n / 8 + 255) / 256 + 1);
+  wmax_kernel<<<(unsigned)blocks, 256, 0, stream>>>(W, n, st);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// K3 — candidate quantiser ("05 — AWQ" §4: for each alpha apply the scaling
+// and quantize).  For candidate i, row o and group k it computes wt = s*w, the
+// group min/max by warp shuffles over the g/8 lanes that hold the group, the
+// step and zero point, the codes, deq = (q - z) delta, and writes the
+// effective error (deq/s - w) * 2^k as fp16: row (i * out_pad + o) of the
+// tensor-core B operand [n_alpha * out_pad, in].  Rows out..out_pad-1 of each
+// candidate are zero.  Each thread handles 8 consecutive channels (16-byte
+// loads and stores).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) cand_quant_kernel(
+    const __half *__restrict__ W, int64_t out, int64_t in, int64_t out_pad,
+    const float *__restrict__ s, const float *__restrict__ inv_s, int n_alpha, int group,
+    float qmax, const DevStatus *__restrict__ st, __half *__restrict__ dW) {
+  const int k = kscale_from_wmax(__uint_as_float(__ldg(&st->wmax_bits)));
+  const float two_k = ldexpf(1.0f, k);
+  const int lanes = group / 8;  // lanes per group (a power of two <= 32)
+  const int64_t items_per_row = in / 8;
+  const int64_t total = (int64_t)n_alpha * out_pad * items_per_row;  // multiple of 32
+  for (int64_t it = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; it < total;
+       it += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = it / items_per_row;
+    const int64_t j0 = (it - row * items_per_row) * 8;
+    const int a = (int)(row / out_pad);
+    const int64_t o = row - (int64_t)a * out_pad;
+    const bool live = o < out;
+    float w[8], sv[8], iv[8];
+    if (live) {
+      uint4 wv = __ldg(reinterpret_cast<const uint4 *>(W + o * in + j0));
+      const uint32_t wr[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&wr[h]));
+        w[2 * h] = f.x;
+        w[2 * h + 1] = f.y;
+      }
+      const float4 *sp = reinterpret_cast<const float4 *>(s + (int64_t)a * in + j0);
+      const float4 *ip = reinterpret_cast<const float4 *>(inv_s + (int64_t)a * in + j0);
+      float4 s0 = __ldg(sp), s1 = __ldg(sp + 1), i0 = __ldg(ip), i1 = __ldg(ip + 1);
+      sv[0] = s0.x; sv[1] = s0.y; sv[2] = s0.z; sv[3] = s0.w;
+      sv[4] = s1.x; sv[5] = s1.y; sv[6] = s1.z; sv[7] = s1.w;
+      iv[0] = i0.x; iv[1] = i0.y; iv[2] = i0.z; iv[3] = i0.w;
+      iv[4] = i1.x; iv[5] = i1.y; iv[6] = i1.z; iv[7] = i1.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) { w[e] = 0.0f; sv[e] = 1.0f; iv[e] = 1.0f; }
+    }
+    float wt[8];
+    float mx = -INFINITY, mn = INFINITY;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      wt[e] = __fmul_rn(sv[e], w[e]);
+      mx = fmaxf(mx, wt[e]);
+      mn = fminf(mn, wt[e]);
+    }
+    for (int off = lanes >> 1; off > 0; off >>= 1) {
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+    }
+    const GroupQ g = group_params(mx, mn, 1.0f, qmax);
+    uint32_t packed[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      float d2[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int e = 2 * h + u;
+        const float deq = dequant(quant_code(wt[e], g), g);
+        // (deq/s - w) 2^k; 2^k is exact, the product with 1/s is fp32 (the
+        // result is rounded to fp16 next)
+        d2[u] = fmaf(__fmul_rn(deq, two_k), iv[e], -__fmul_rn(w[e], two_k));
+        if (!live) d2[u] = 0.0f;
+      }
+      __half2 hv = __floats2half2_rn(d2[0], d2[1]);
+      packed[h] = *reinterpret_cast<uint32_t *>(&hv);
+    }
+    *reinterpret_cast<uint4 *>(dW + row * in + j0) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+  }
+}
+
+cudaError_t launch_cand_quant(const __half *W, int64_t out, int64_t in, int64_t out_pad,
+                              const float *s, const float *inv_s, int n_alpha, int group, int w_bit,
+                              const DevStatus *st, __half *dW, int num_sms, cudaStream_t stream) {
+  const int64_t total = (int64_t)n_alpha * out_pad * (in / 8);
+  int64_t blocks = i64min((int64_t)num_sms * 8, (total + 255) / 256);
+  cand_quant_kernel<<<(unsigned)blocks, 256, 0, stream>>>(W, out, in, out_pad, s, inv_s, n_alpha,
+                                                          group, (float)((1 << w_bit) - 1), st, dW);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// K7 — final codes with (s, clip ratio) and the pages' storage layout
+// ("05 — AWQ" §5): qweight [in, out/8] int32 with the code of output o in
+// nibble o%8 of word [j][o/8]; qzeros [in/g, out/8] likewise; scales
+// [in/g, out] fp16.  A block handles 128 output rows x one group of 128
+// input channels: warps quantise rows (one lane per 4 channels), codes go
+// through shared memory and are re-read transposed for packing, so every
+// global store is contiguous.
+// ---------------------------------------------------------------------------
+constexpr int kPackRows = 128;
+
+__device__ __forceinline__ float clip_ratio(int c, int n_clip, float clip_min) {
+  if (n_clip <= 1) return 1.0f;
+  double r = 1.0 - (double)c * (1.0 - (double)clip_min) / (double)(n_clip - 1);
+  return __double2float_rn(r);
+}
+
+__global__ void __launch_bounds__(256) quant_pack_kernel(
+    const __half *__restrict__ W, int64_t out, int64_t in, const float *__restrict__ s,
+    const uint8_t *__restrict__ clip_idx, int n_clip, float clip_min, float qmax,
+    int32_t *__restrict__ qweight, int32_t *__restrict__ qzeros, __half *__restrict__ scales) {
+  constexpr int G = 128;
+  __shared__ uint8_t codes[kPackRows][G + 4];
+  __shared__ uint8_t zeros[kPackRows];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int k = blockIdx.x;                       // group
+  const int64_t o0 = (int64_t)blockIdx.y * kPackRows;
+  const int64_t groups = in / G;
+  const int64_t j0 = (int64_t)k * G + lane * 4;
+  float sv[4] = {1.0f, 1.0f, 1.0f, 1.0f};
+  if (s) {
+    float4 f = __ldg(reinterpret_cast<const float4 *>(s + j0));
+    sv[0] = f.x; sv[1] = f.y; sv[2] = f.z; sv[3] = f.w;
+  }
+  for (int r = warp; r < kPackRows; r += 8) {
+    const int64_t o = o0 + r;
+    if (o >= out) break;
+    uint2 wv = __ldg(reinterpret_cast<const uint2 *>(W + o * in + j0));
+    float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&wv.x));
+    float2 b = __half22float2(*reinterpret_cast<const __half2 *>(&wv.y));
+    float wt[4] = {__fmul_rn(sv[0], a.x), __fmul_rn(sv[1], a.y), __fmul_rn(sv[2], b.x),
+                   __fmul_rn(sv[3], b.y)};
+    float mx = fmaxf(fmaxf(wt[0], wt[1]), fmaxf(wt[2], wt[3]));
+    float mn = fminf(fminf(wt[0], wt[1]), fminf(wt[2], wt[3]));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+    }
+    const float r32 = clip_idx ? clip_ratio(clip_idx[o * groups + k], n_clip, clip_min) : 1.0f;
+    const GroupQ g = group_params(mx, mn, r32, qmax);
+    uchar4 c4;
+    c4.x = (uint8_t)quant_code(wt[0], g);
+    c4.y = (uint8_t)quant_code(wt[1], g);
+    c4.z = (uint8_t)quant_code(wt[2], g);
+    c4.w = (uint8_t)quant_code(wt[3], g);
+    *reinterpret_cast<uchar4 *>(&codes[r][lane * 4]) = c4;
+    if (lane == 0) {
+      zeros[r] = (uint8_t)g.zero;
+      scales[(int64_t)k * out + o] = __float2half_rn(g.delta);
+    }
+  }
+  __syncthreads();
+  const int64_t words_per_row = out / 8;
+  const int rows_here = (int)i64min(kPackRows, out - o0);
+  const int o8_here = rows_here / 8;  // out % 8 == 0
+  for (int t = threadIdx.x; t < G * 16; t += 256) {
+    const int o8 = t & 15, jj = t >> 4;
+    if (o8 >= o8_here) continue;
+    uint32_t word = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) word |= (uint32_t)codes[o8 * 8 + e][jj] << (4 * e);
+    qweight[((int64_t)k * G + jj) * words_per_row + o0 / 8 + o8] = (int32_t)word;
+  }
+  if (threadIdx.x < o8_here) {
+    uint32_t word = 0;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) word |= (uint32_t)zeros[threadIdx.x * 8 + e] << (4 * e);
+    qzeros[(int64_t)k * words_per_row + o0 / 8 + threadIdx.x] = (int32_t)word;
+  }
+}
+
+cudaError_t launch_quant_pack(const __half *W, int64_t out, int64_t in, const float *s,
+                              const uint8_t *clip_idx, int group, int w_bit, int n_clip,
+                              float clip_min, int32_t *qweight, int32_t *qzeros, __half *scales,
+                              cudaStream_t stream) {
+  if (group != 128) return cudaErrorInvalidValue;
+  dim3 grid((unsigned)(in / group), (unsigned)((out + kPackRows - 1) / kPackRows));
+  quant_pack_kernel<<<grid, 256, 0, stream>>>(W, out, in, s, clip_idx, n_clip, clip_min,
+                                              (float)((1 << w_bit) - 1), qweight, qzeros, scales);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// K8 — fold 1/s into the preceding operation ("AWQ and Activation-Aware
+// Scaling": the activation-side division is absorbed by the preceding
+// normalisation's scale or linear layer): v[j][:] = RN16(RN32(v[j][:]) / s_j).
+// ---------------------------------------------------------------------------
+__global__ void fold_kernel(__half *__restrict__ v, int64_t rows, int64_t cols,
+                            const float *__restrict__ s) {
+  const int64_t n = rows * cols;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t j = i / cols;
+    v[i] = __float2half_rn(__fdiv_rn(__half2float(v[i]), s[j]));
+  }
+}
+
+cudaError_t launch_fold(__half *v, int64_t rows, int64_t cols, const float *s, cudaStream_t stream) {
+  const int64_t n = rows * cols;
+  int64_t blocks = i64min(4096, (n + 255) / 256);
+  if (blocks < 1) blocks = 1;
+  fold_kernel<<<(unsigned)blocks, 256, 0, stream>>>(v, rows, cols, s);
+  return cudaGetLastError();
+}
+
+}  // namespace awq

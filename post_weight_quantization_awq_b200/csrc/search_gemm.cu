@@ -1,0 +1,353 @@
+// K4 — the scored candidate GEMM of the AWQ alpha search, and K5, its
+// deterministic reduction and argmin.
+//
+// "05 — AWQ: Activation-Aware Weight Scaling" §4: for each alpha apply the
+// scaling, quantize, and measure the MSE against the fp16 output.  By the
+// scaling invariance of §3, (X diag(s)^-1) Qdeq^T - X W^T = X dW^T with
+// dW = Qdeq/s - W, so every candidate's error is one GEMM against the same X.
+// All n_alpha candidates are stacked along N (B = dW [n_alpha * out_pad, in])
+// and run as one persistent GEMM:  M = T tokens, N = n_alpha * out_pad,
+// K = in.  The epilogue squares and sums each accumulator tile straight out
+// of tensor memory, so no candidate output is ever written to HBM.
+//
+// sm_100a design, one CTA per SM (192 threads):
+//   warp 0      TMA producer: A tile 128x64 and B tile 256x64 (fp16, 128-byte
+//               swizzle) into a 4-stage shared-memory ring;
+//   warp 1      allocates 512 TMEM columns; one thread issues
+//               tcgen05.mma.cta_group::1.kind::f16 (M=128, N=256, K=16) into a
+//               double-buffered fp32 accumulator (2 x 256 columns) and commits
+//               stage/accumulator barriers;
+//   warps 2..5  epilogue: tcgen05.ld 32 lanes x 32 columns at a time, sum of
+//               squares in fp32 per row, fp64 warp reduction, one partial per
+//               (tile, warp) into HBM.
+// Tiles are visited in groups of `group_m` M-blocks so the A panels of a
+// group stay in L2 while all N-blocks stream past.  Every mbarrier wait is
+// bounded; a wait that runs out records kDevTimeout, raises a CTA-wide abort
+// flag, and every role drains its in-flight copies / MMAs before the CTA frees
+// its TMEM and exits.
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <math.h>
+
+#include "awq_launch.h"
+
+namespace awq {
+
+namespace {
+
+constexpr int BM = kGemmBM, BN = kGemmBN, BK = kGemmBK;
+constexpr int STAGES = 4;
+constexpr uint32_t A_BYTES = BM * BK * 2;  // 16 KiB
+constexpr uint32_t B_BYTES = BN * BK * 2;  // 32 KiB
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t IDESC = idesc_f16_f32(BM, BN);
+constexpr uint32_t DRAIN_POLLS = 1u << 22;
+constexpr int GROUP_M = 32;
+
+struct __align__(8) GemmSmemTail {
+  uint64_t full[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t tfull[2];
+  uint64_t tempty[2];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+constexpr size_t kGemmSmemBytes =
+    1024 /*alignment slack*/ + STAGES * (A_BYTES + B_BYTES) + sizeof(GemmSmemTail);
+
+__device__ __forceinline__ void tile_coords(int tile, int num_m, int num_n, int group_m,
+                                            int &m_blk, int &n_blk) {
+  const int per_group = group_m * num_n;
+  const int g = tile / per_group;
+  const int first_m = g * group_m;
+  const int gm = min(group_m, num_m - first_m);
+  const int local = tile - g * per_group;
+  m_blk = first_m + local % gm;
+  n_blk = local / gm;
+}
+
+__device__ __forceinline__ void raise_abort(GemmSmemTail *t, DevStatus *st, uint32_t where) {
+  dev_fail(st, kDevTimeout, where);
+  *reinterpret_cast<volatile int *>(&t->abort_flag) = 1;
+}
+
+}  // namespace
+
+__global__ void __launch_bounds__(192, 1)
+    search_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                       const __grid_constant__ CUtensorMap tmB, int num_m, int num_n, int num_kb,
+                       double *__restrict__ partials, DevStatus *st, uint32_t max_polls) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *sA = smem;
+  uint8_t *sB = smem + STAGES * A_BYTES;
+  GemmSmemTail *tail = reinterpret_cast<GemmSmemTail *>(sB + STAGES * B_BYTES);
+  volatile int *abort_flag = &tail->abort_flag;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int num_tiles = num_m * num_n;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&tail->full[s], 1);
+      mbar_init(&tail->empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tail->tfull[a], 1);
+      mbar_init(&tail->tempty[a], 4);  // one arrival per epilogue warp
+    }
+    mbar_init(&tail->mma_done, 1);
+    tail->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(&tail->tmem_base, TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tail->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued = 0, issued_parity = 0;  // per-stage: a fill is pending / its parity
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+        int m_blk, n_blk;
+        tile_coords(tile, num_m, num_n, GROUP_M, m_blk, n_blk);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait_bounded(&tail->empty[stage], phase ^ 1u, max_polls, abort_flag)) {
+            raise_abort(tail, st, 0x100u + stage);
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&tail->full[stage], A_BYTES + B_BYTES);
+          tma_load_2d(sA + stage * A_BYTES, &tmA, &tail->full[stage], kb * BK, m_blk * BM);
+          tma_load_2d(sB + stage * B_BYTES, &tmB, &tail->full[stage], kb * BK, n_blk * BN);
+          issued |= 1u << stage;
+          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok || *abort_flag) {
+        // Let every fill already issued land before the CTA can exit.
+        for (int s = 0; s < STAGES; ++s)
+          if (issued & (1u << s))
+            (void)mbar_wait_bounded(&tail->full[s], (issued_parity >> s) & 1u, DRAIN_POLLS,
+                                    nullptr);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true, issued_any = false;
+      int it = 0;
+      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++it) {
+        const int acc = it & 1;
+        const uint32_t acc_phase = (it >> 1) & 1;
+        if (!mbar_wait_bounded(&tail->tempty[acc], acc_phase ^ 1u, max_polls, abort_flag)) {
+          raise_abort(tail, st, 0x200u + acc);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait_bounded(&tail->full[stage], phase, max_polls, abort_flag)) {
+            raise_abort(tail, st, 0x300u + stage);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sA + stage * A_BYTES);
+          const uint32_t b_addr = smem_u32(sB + stage * B_BYTES);
+#pragma unroll
+          for (int k = 0; k < BK / 16; ++k) {
+            tc_mma_f16(d_tmem, smem_desc_k_sw128(a_addr + k * 32), smem_desc_k_sw128(b_addr + k * 32),
+                       IDESC, (kb | k) != 0 ? 1u : 0u);
+          }
+          issued_any = true;
+          tc_commit(&tail->empty[stage]);  // frees the stage once these MMAs finish
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(&tail->tfull[acc]);  // accumulator ready for the epilogue
+      }
+      if (issued_any) {
+        tc_commit(&tail->mma_done);
+        (void)mbar_wait_bounded(&tail->mma_done, 0, DRAIN_POLLS, nullptr);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    int it = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+      const int acc = it & 1;
+      const uint32_t acc_phase = (it >> 1) & 1;
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait_bounded(&tail->tfull[acc], acc_phase, max_polls, abort_flag);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) {
+        if (lane == 0) raise_abort(tail, st, 0x400u + acc);
+        break;
+      }
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+      float sum = 0.0f;
+#pragma unroll 1
+      for (int c = 0; c < BN; c += 32) {
+        float v[32];
+        tmem_ld_32x32b_x32(taddr + (uint32_t)c, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) sum = fmaf(v[i], v[i], sum);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tail->tempty[acc]);
+      double ds = (double)sum;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) ds += __shfl_xor_sync(0xffffffffu, ds, off);
+      if (lane == 0) {
+        int m_blk, n_blk;
+        tile_coords(tile, num_m, num_n, GROUP_M, m_blk, n_blk);
+        partials[((size_t)n_blk * num_m + m_blk) * 4 + q] = ds;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// Host side: tensor maps and launch.
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D fp16 tensor map over a row-major [rows, cols] matrix with row stride
+// `ld` elements, box [box_rows, 64 cols], 128-byte swizzle, zero fill.
+static cudaError_t make_tmap_f16(CUtensorMap *m, const void *base, int64_t rows, int64_t cols,
+                                 int64_t ld, uint32_t box_rows) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
+  cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
+cudaError_t launch_search_gemm(const __half *X, int64_t ldx, const __half *dW,
+                               const SearchGemmShape &sh, double *partials, DevStatus *st,
+                               uint32_t max_polls, int num_sms, cudaStream_t stream) {
+  CUtensorMap tmA, tmB;
+  cudaError_t e = make_tmap_f16(&tmA, X, sh.T, sh.in, ldx, BM);
+  if (e != cudaSuccess) return e;
+  e = make_tmap_f16(&tmB, dW, sh.rows_b, sh.in, sh.in, BN);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(search_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)kGemmSmemBytes);
+  if (e != cudaSuccess) return e;
+  const int tiles = sh.num_m * sh.num_n;
+  const int grid = tiles < num_sms ? tiles : num_sms;
+  search_gemm_kernel<<<grid, 192, kGemmSmemBytes, stream>>>(tmA, tmB, sh.num_m, sh.num_n,
+                                                            sh.num_kb, partials, st, max_polls);
+  return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// K5 — MSE_i = (sum of candidate i's partials) * 2^-2k / (T out), summed in a
+// fixed order (bitwise reproducible); best = first index of the smallest MSE;
+// s_best = s_grid[best].  One block.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024) mse_argmin_kernel(
+    const double *__restrict__ partials, int n_alpha, int nb_per_alpha, int num_m, int64_t T,
+    int64_t out, const float *__restrict__ s_grid, int64_t in, DevStatus *st,
+    double *__restrict__ mse, int32_t *__restrict__ best_idx, float *__restrict__ s_best) {
+  __shared__ double red[1024];
+  __shared__ int best_sh;
+  const int k = kscale_from_wmax(__uint_as_float(st->wmax_bits));
+  const size_t per = (size_t)nb_per_alpha * num_m * 4;
+  for (int i = 0; i < n_alpha; ++i) {
+    const double *p = partials + (size_t)i * per;
+    double acc = 0.0;
+    for (size_t idx = threadIdx.x; idx < per; idx += blockDim.x) acc += p[idx];
+    red[threadIdx.x] = acc;
+    __syncthreads();
+    for (int w = blockDim.x >> 1; w > 0; w >>= 1) {
+      if ((int)threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+      __syncthreads();
+    }
+    if (threadIdx.x == 0) mse[i] = ldexp(red[0], -2 * k) / ((double)T * (double)out);
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    int best = 0;
+    bool finite = true;
+    for (int i = 0; i < n_alpha; ++i) {
+      const double v = mse[i];
+      if (!isfinite(v)) finite = false;
+      if (v < mse[best]) best = i;
+    }
+    if (!finite) dev_fail(st, kDevNonFinite, 0x500u);
+    best_sh = best;
+    *best_idx = best;
+  }
+  __syncthreads();
+  const float *src = s_grid + (size_t)best_sh * in;
+  for (int64_t j = threadIdx.x; j < in; j += blockDim.x) s_best[j] = src[j];
+}
+
+cudaError_t launch_mse_argmin(const double *partials, int n_alpha, int nb_per_alpha, int num_m,
+                              int64_t T, int64_t out, const float *s_grid, int64_t in,
+                              DevStatus *st, double *mse, int32_t *best_idx, float *s_best,
+                              cudaStream_t stream) {
+  mse_argmin_kernel<<<1, 1024, 0, stream>>>(partials, n_alpha, nb_per_alpha, num_m, T, out, s_grid,
+                                            in, st, mse, best_idx, s_best);
+  return cudaGetLastError();
+}
+
+}  // namespace awq

@@ -1,0 +1,95 @@
+"""CPU-only checks of the C-ABI library: it loads, exports every function the
+header declares, and rejects bad arguments on the host before touching CUDA."""
+
+import ctypes
+
+import pytest
+
+import post_weight_quantization_awq_b200 as awq
+from post_weight_quantization_awq_b200 import abi
+
+
+def test_library_exports_every_header_function():
+    names = abi.header_functions()
+    assert {"awq_act_stats", "awq_search_scale", "awq_search_clip", "awq_quant_pack"} <= set(names)
+    for n in names:
+        assert hasattr(abi.LIB, n), n
+        assert abi.LIB[n] is not None
+
+
+def test_python_binding_has_the_abi_names():
+    for n in ("awq_act_stats", "awq_scale_grid", "awq_search_scale", "awq_search_clip",
+              "awq_quant_pack", "awq_fold_inv_scale", "awq_device_status", "awq_workspace_size"):
+        assert callable(getattr(awq, n)), n
+
+
+def test_version_string():
+    assert "sm_100a" in awq.version()
+
+
+def test_workspace_size_grows_with_the_problem():
+    cfg = awq.AwqConfig.make(n_alpha=20, n_clip=20)
+    a = awq.awq_workspace_size(65536, 4096, 4096, cfg)
+    b = awq.awq_workspace_size(65536, 4096, 8192, cfg)
+    # candidate operand alone: n_alpha * out * in fp16
+    assert a >= 20 * 4096 * 4096 * 2 and b > a
+    small = awq.awq_workspace_size(256, 512, 512, awq.AwqConfig.make(n_alpha=20))
+    assert 20 * 512 * 512 * 2 <= small < 40 * 2 ** 20
+
+
+@pytest.mark.parametrize("kw,shape,status", [
+    (dict(w_bit=5), (256, 512, 512), "AWQ_ERR_UNSUPPORTED"),
+    (dict(w_bit=0), (256, 512, 512), "AWQ_ERR_INVALID_ARG"),
+    (dict(group_size=64), (256, 512, 512), "AWQ_ERR_UNSUPPORTED"),
+    (dict(zero_point=0), (256, 512, 512), "AWQ_ERR_UNSUPPORTED"),
+    (dict(n_alpha=0), (256, 512, 512), "AWQ_ERR_INVALID_ARG"),
+    (dict(n_clip=65), (256, 512, 512), "AWQ_ERR_INVALID_ARG"),
+    (dict(clip_min=0.0), (256, 512, 512), "AWQ_ERR_INVALID_ARG"),
+    (dict(), (256, 500, 512), "AWQ_ERR_INVALID_ARG"),
+    (dict(), (256, 512, 12), "AWQ_ERR_INVALID_ARG"),
+    (dict(), (0, 512, 512), "AWQ_ERR_INVALID_ARG"),
+])
+def test_host_validation(kw, shape, status):
+    cfg = awq.AwqConfig.make(**kw)
+    with pytest.raises(awq.AwqError) as ei:
+        awq.awq_workspace_size(*shape, cfg)
+    assert "AWQ_ERR_INVALID_ARG" == ei.value.status_name or ei.value.status_name == status
+    # the calls report the precise status before any CUDA work
+    st = abi.LIB.awq_search_scale(16, shape[0], shape[1], shape[1], 16, shape[2], 16,
+                                  ctypes.byref(cfg), 256, 1 << 30, 16, 16, 16, None)
+    assert abi.STATUS[st] == status, abi.last_error()
+
+
+def test_null_and_misaligned_pointers_are_rejected():
+    cfg = awq.AwqConfig.make(n_clip=20)
+    L = abi.LIB
+    assert abi.STATUS[L.awq_act_stats(None, 16, 512, 512, 256, None)] == "AWQ_ERR_INVALID_ARG"
+    assert abi.STATUS[L.awq_act_stats(18, 16, 512, 512, 256, None)] == "AWQ_ERR_INVALID_ARG"  # misaligned X
+    assert abi.STATUS[L.awq_act_stats(16, 16, 512, 500, 256, None)] == "AWQ_ERR_INVALID_ARG"  # ldx < in
+    assert abi.STATUS[L.awq_act_stats(16, 16, 512, 516, 256, None)] == "AWQ_ERR_INVALID_ARG"  # ldx % 8
+    assert "ldx" in abi.last_error()
+    # workspace missing / misaligned / too small
+    for ws, nbytes in ((None, 1 << 30), (128, 1 << 30), (256, 1024)):
+        st = L.awq_search_scale(16, 256, 512, 512, 16, 512, 16, ctypes.byref(cfg), ws, nbytes,
+                                16, 16, 16, None)
+        assert abi.STATUS[st] == "AWQ_ERR_WORKSPACE"
+    st = L.awq_search_clip(16, 256, 512, 512, 16, 512, 16, ctypes.byref(awq.AwqConfig.make(n_clip=0)),
+                           256, 1 << 30, 16, None, None)
+    assert abi.STATUS[st] == "AWQ_ERR_INVALID_ARG" and "n_clip" in abi.last_error()
+    st = L.awq_quant_pack(16, 512, 512, None, 16, ctypes.byref(awq.AwqConfig.make(n_clip=0)),
+                          16, 16, 16, None)
+    assert abi.STATUS[st] == "AWQ_ERR_INVALID_ARG"
+    st = L.awq_quant_pack(16, 512, 512, None, None, ctypes.byref(cfg), None, 16, 16, None)
+    assert abi.STATUS[st] == "AWQ_ERR_INVALID_ARG"
+
+
+def test_errors_are_per_thread():
+    import threading
+    cfg = awq.AwqConfig.make(w_bit=7)
+    abi.LIB.awq_workspace_size(256, 512, 512, ctypes.byref(cfg))
+    mine = abi.last_error()
+    seen = []
+    t = threading.Thread(target=lambda: seen.append(abi.last_error()))
+    t.start()
+    t.join()
+    assert "w_bit" in mine and seen == [""]

@@ -1,0 +1,255 @@
+"""GPU parity: every step of the CUDA path, called through the C ABI, against
+the fp64 CPU oracle on the same seeded inputs.
+
+Bars: abar, the s grid, codes, zeros, qweight, qzeros and scales bit-exact;
+per-alpha MSE within 1e-3 relative; the selected alpha / clip index equal to
+the oracle's unless the oracle's scores of the two differ by < 1e-4 relative;
+clip errors within 1e-3 relative."""
+
+import numpy as np
+import pytest
+import torch
+
+import post_weight_quantization_awq_b200 as awq
+from oracle import awq_oracle as O
+from synthetic import OutlierSpec, heavy_tailed_activations, random_layer, workload_inputs
+
+from gpu_helpers import (MSE_RTOL, check_mse, check_selection, gpu_search, midpoint_report,
+                         need_cuda, to_dev)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _cuda():
+    need_cuda()
+
+
+# ------------------------------------------------------------------ K1
+@pytest.mark.parametrize("T,inn,ldx", [(1, 8, 8), (37, 136, 136), (1000, 520, 520), (4096 + 77, 1024, 1032),
+                                       (20000, 256, 256)])
+def test_act_stats_bitwise(T, inn, ldx):
+    X = heavy_tailed_activations(T, ldx, OutlierSpec(0.02, 20.0, 50.0), seed=T + inn)
+    X[0, :4] = torch.tensor([65504.0, -65504.0, 2 ** -24, -(2 ** -24)], dtype=torch.float16)
+    Xd = to_dev(X)[:, :inn]
+    abar = torch.empty(inn, dtype=torch.float64, device="cuda")
+    awq.awq_act_stats(Xd, abar)
+    want = O.act_stats(X[:, :inn].numpy())
+    got = abar.cpu().numpy()
+    assert np.array_equal(got, want), np.flatnonzero(got != want)[:10]
+
+
+# ------------------------------------------------------------------ K2
+@pytest.mark.parametrize("n_alpha", [1, 3, 20])
+def test_scale_grid_bitwise(n_alpha):
+    rng = np.random.default_rng(n_alpha)
+    abar = np.exp(rng.normal(0, 2, 4096))
+    abar[:4] = [0.0, 1e-9, 1.0, 300.0]
+    a_d = torch.from_numpy(abar).cuda()
+    s = torch.empty((n_alpha, 4096), dtype=torch.float32, device="cuda")
+    awq.awq_scale_grid(a_d, n_alpha, s)
+    got = s.cpu().numpy()
+    want = O.scale_grid(abar, O.alpha_grid(n_alpha))
+    assert np.array_equal(got, want), midpoint_report(abar, O.alpha_grid(n_alpha), got, want)
+
+
+# ------------------------------------------------------------------ K7
+def _gpu_pack(W, s, clip_idx, cfg):
+    out, inn = W.shape
+    g = cfg.group_size
+    qw = torch.empty((inn, out // 8), dtype=torch.int32, device="cuda")
+    qz = torch.empty((inn // g, out // 8), dtype=torch.int32, device="cuda")
+    sc = torch.empty((inn // g, out), dtype=torch.float16, device="cuda")
+    awq.awq_quant_pack(to_dev(W), None if s is None else torch.from_numpy(s).cuda(),
+                       None if clip_idx is None else torch.from_numpy(clip_idx).cuda(),
+                       cfg, qw, qz, sc)
+    torch.cuda.synchronize()
+    return qw.cpu().numpy(), qz.cpu().numpy(), sc.cpu().numpy()
+
+
+@pytest.mark.parametrize("out,inn,w_bit,use_s,use_clip", [
+    (8, 128, 4, False, False), (72, 384, 4, True, False), (136, 256, 3, True, True),
+    (512, 512, 4, True, True), (1000, 1024, 3, False, True)])
+def test_quant_pack_bitwise(out, inn, w_bit, use_s, use_clip):
+    X, W = random_layer(64, inn, out, seed=out + inn + w_bit)
+    s = O.scale_grid(O.act_stats(X.numpy()), O.alpha_grid(20))[13] if use_s else None
+    n_clip = 20 if use_clip else 0
+    clip_idx = (np.random.default_rng(out).integers(0, 20, size=(out, inn // 128)).astype(np.uint8)
+                if use_clip else None)
+    cfg = awq.AwqConfig.make(w_bit=w_bit, n_clip=n_clip)
+    got = _gpu_pack(W, s, clip_idx, cfg)
+    want = O.quant_pack(W.numpy(), s, clip_idx, w_bit, 128, max(n_clip, 1), 0.5)
+    for g_, w_, name in zip(got, want, ("qweight", "qzeros", "scales")):
+        assert np.array_equal(g_.view(np.uint8), w_.view(np.uint8)), name
+
+
+def test_quant_pack_hand_worked(golden):
+    hdr, rows = golden("pack_int4.txt")
+    W = np.zeros((8, 128), dtype=np.float16)
+    for o in range(8):
+        for j in range(8):
+            W[o, j] = ((o + j) % 16) - 8
+        W[o, 126], W[o, 127] = -8.0, 7.0
+    qw, qz, sc = _gpu_pack(torch.from_numpy(W), None, None, awq.AwqConfig.make())
+    for r in rows:
+        assert int(qw.view(np.uint32)[int(r[0]), 0]) == int(r[1], 16)
+    assert int(qz.view(np.uint32)[0, 0]) == int(hdr["qzeros_hex"], 16)
+    assert np.all(sc == np.float16(1.0))
+
+
+# ------------------------------------------------------------------ K2-K5
+SEARCH_CASES = [
+    # T, in, out, w_bit, n_alpha
+    (64, 128, 16, 4, 20),
+    (1, 128, 8, 4, 20),
+    (200, 384, 264, 3, 20),
+    (256, 512, 512, 4, 20),      # the tiny 512 x 512 linear workload's shapes
+    (2125, 1024, 768, 4, 20),    # > 1000 GEMM tiles: persistent schedule, both accumulators
+    (130, 256, 64, 4, 1),        # alpha = 0 only: plain RTN
+]
+
+
+@pytest.mark.parametrize("T,inn,out,w_bit,n_alpha", SEARCH_CASES)
+def test_search_scale_parity(T, inn, out, w_bit, n_alpha):
+    X, W = random_layer(T, inn, out, seed=T * 7 + inn + out)
+    cfg = awq.AwqConfig.make(w_bit=w_bit, n_alpha=n_alpha)
+    g = gpu_search(X, W, cfg)
+    Xn, Wn = X.numpy(), W.numpy()
+    abar = O.act_stats(Xn)
+    assert np.array_equal(g["abar"], abar)
+    mse, best, s_best, S = O.search_scale(Xn, Wn, abar, w_bit, 128, n_alpha)
+    check_mse(g["mse"], mse)
+    check_selection(g["best"], mse, "alpha")
+    assert np.array_equal(g["s_best"], S[g["best"]])
+
+
+def test_search_scale_strided_x_and_determinism():
+    X, W = random_layer(700, 640, 256, seed=5)
+    Xd = to_dev(X)
+    wide = torch.zeros((700, 768), dtype=torch.float16, device="cuda")
+    wide[:, 64:704] = Xd
+    Xv = wide[:, 64:704]                    # row stride 768, 128-byte aligned start
+    cfg = awq.AwqConfig.make()
+    ws = awq.alloc_workspace(700, 640, 256, cfg)
+    outs = []
+    for _ in range(2):
+        abar = torch.empty(640, dtype=torch.float64, device="cuda")
+        mse = torch.empty(20, dtype=torch.float64, device="cuda")
+        best = torch.empty(1, dtype=torch.int32, device="cuda")
+        s_best = torch.empty(640, dtype=torch.float32, device="cuda")
+        awq.awq_act_stats(Xv, abar)
+        awq.awq_search_scale(Xv, to_dev(W), abar, cfg, ws, s_best, mse, best)
+        awq.awq_device_status(ws)
+        outs.append(mse.cpu().numpy())
+    assert np.array_equal(outs[0], outs[1])  # fixed-order reductions: bitwise reproducible
+    mse_o, _, _, _ = O.search_scale(X.numpy(), W.numpy(), O.act_stats(X.numpy()), 4, 128, 20)
+    check_mse(outs[0], mse_o)
+
+
+def test_ties_keep_alpha_zero():
+    T, inn = 64, 256
+    X = torch.from_numpy(np.where(np.arange(T * inn).reshape(T, inn) % 2 == 0, 1.0, -1.0)
+                         .astype(np.float16))
+    _, W = random_layer(4, inn, 16, seed=3)
+    g = gpu_search(X, W, awq.AwqConfig.make())
+    assert np.all(g["mse"] == g["mse"][0]) and g["best"] == 0 and np.all(g["s_best"] == 1.0)
+
+
+# ------------------------------------------------------------------ K6
+def _gpu_clip(X, W, s, cfg, with_err=True):
+    Xd, Wd = to_dev(X), to_dev(W)
+    T, inn = Xd.shape
+    out = Wd.shape[0]
+    ws = awq.alloc_workspace(T, inn, out, cfg)
+    idx = torch.empty((out, inn // 128), dtype=torch.uint8, device="cuda")
+    err = torch.empty((out, inn // 128, cfg.n_clip), dtype=torch.float32, device="cuda") if with_err else None
+    awq.awq_search_clip(Xd, Wd, None if s is None else torch.from_numpy(s).cuda(), cfg, ws, idx, err)
+    torch.cuda.synchronize()
+    return idx.cpu().numpy(), (err.cpu().numpy() if with_err else None)
+
+
+@pytest.mark.parametrize("T,inn,out,w_bit,n_clip", [(300, 256, 40, 4, 20), (64, 128, 8, 3, 7),
+                                                     (1500, 512, 96, 3, 20), (33, 384, 24, 4, 1)])
+def test_search_clip_parity(T, inn, out, w_bit, n_clip):
+    X, W = random_layer(T, inn, out, seed=T + out + n_clip)
+    Xn, Wn = X.numpy(), W.numpy()
+    s = O.scale_grid(O.act_stats(Xn), O.alpha_grid(20))[10]
+    cfg = awq.AwqConfig.make(w_bit=w_bit, n_clip=n_clip)
+    idx, err = _gpu_clip(X, W, s, cfg)
+    idx_o, E = O.search_clip(Xn, Wn, s, w_bit, 128, n_clip, 0.5)
+    rel = np.abs(err - E) / np.maximum(np.abs(E), 1e-30)
+    assert rel.max() <= MSE_RTOL, rel.max()
+    for o, k in zip(*np.nonzero(idx != idx_o)):
+        check_selection(int(idx[o, k]), E[o, k], f"clip row {o} group {k}")
+    # s = None means s = 1
+    idx1, _ = _gpu_clip(X, W, None, cfg, with_err=False)
+    idx1_o, E1 = O.search_clip(Xn, Wn, None, w_bit, 128, n_clip, 0.5)
+    for o, k in zip(*np.nonzero(idx1 != idx1_o)):
+        check_selection(int(idx1[o, k]), E1[o, k], f"clip row {o} group {k}")
+
+
+def test_clip_hand_worked(golden):
+    """The hand-worked clip example, through the pack kernel with clip index 19."""
+    hdr, rows = golden("quant_group_clip.txt")
+    W = np.zeros((8, 128), dtype=np.float16)
+    for r in rows:
+        W[:, int(r[0])] = float(r[1])
+    idx = np.full((8, 1), int(hdr["clip_index"]), dtype=np.uint8)
+    qw, qz, sc = _gpu_pack(torch.from_numpy(W), None, idx, awq.AwqConfig.make(n_clip=int(hdr["n_clip"])))
+    q = O.unpack_nibbles(qw)
+    assert np.all(sc == np.float16(float(hdr["delta"])))
+    assert np.all(O.unpack_nibbles(qz) == int(hdr["zero"]))
+    for r in rows:
+        assert np.all(q[:, int(r[0])] == int(r[2]))
+
+
+# ------------------------------------------------------------------ full sizes
+def _layer_parity(X, W, w_bit, n_alpha, n_clip, rows=None):
+    """The whole path at full T and in; with `rows`, on that sample of output
+    rows (the same launch configuration with a smaller N)."""
+    if rows is not None:
+        W = W[rows]
+    cfg = awq.AwqConfig.make(w_bit=w_bit, n_alpha=n_alpha, n_clip=n_clip)
+    Xd, Wd = to_dev(X), to_dev(W)
+    ws = awq.alloc_workspace(Xd.shape[0], Xd.shape[1], Wd.shape[0], cfg)
+    res = awq.quantize_layer(Xd, Wd, cfg, ws=ws)
+    awq.awq_device_status(ws)
+    torch.cuda.synchronize()
+    Xn, Wn = X.numpy(), W.numpy()
+    abar = O.act_stats(Xn)
+    assert np.array_equal(res.abar.cpu().numpy(), abar)
+    mse, best, s_best, S = O.search_scale(Xn, Wn, abar, w_bit, 128, n_alpha)
+    g_mse = res.mse.cpu().numpy()
+    check_mse(g_mse, mse)
+    g_best = int(res.best_idx.item())
+    check_selection(g_best, mse, "alpha")
+    s = S[g_best]
+    assert np.array_equal(res.s_best.cpu().numpy(), s)
+    clip_idx = None
+    if n_clip:
+        clip_idx = res.clip_idx.cpu().numpy()
+        idx_o, E = O.search_clip(Xn, Wn, s, w_bit, 128, n_clip, 0.5)
+        for o, k in zip(*np.nonzero(clip_idx != idx_o)):
+            check_selection(int(clip_idx[o, k]), E[o, k], f"clip row {o} group {k}")
+    qw, qz, sc = O.quant_pack(Wn, s, clip_idx, w_bit, 128, max(n_clip, 1), 0.5)
+    assert np.array_equal(res.qweight.cpu().numpy(), qw)
+    assert np.array_equal(res.qzeros.cpu().numpy(), qz)
+    assert np.array_equal(res.scales.cpu().numpy().view(np.uint16), sc.view(np.uint16))
+    return g_mse, mse
+
+
+def test_full_q_proj_4096_workload():
+    """The Llama-7B-shaped q_proj workload at full size: X [65536 x 4096],
+    W [4096 x 4096], INT4 g128, 20 alphas, 20 clip ratios, packed."""
+    d = workload_inputs(1)
+    _, X, W = d["groups"][0]
+    _layer_parity(X, W, 4, 20, 20)
+
+
+def test_full_attention_int3_workload_sampled_rows():
+    """The 13B-shaped INT3 attention workload: full X [65536 x 5120]; qkv
+    [15360 x 5120] checked on a sample of 512 output rows (same T, in)."""
+    d = workload_inputs(3)
+    _, X, W = d["groups"][0]
+    rows = np.sort(np.random.default_rng(0).choice(W.shape[0], 512, replace=False))
+    _layer_parity(X, W, 3, 20, 20, rows=torch.from_numpy(rows))
