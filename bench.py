@@ -1,0 +1,394 @@
+#!/usr/bin/env python
+"""Benchmark of the AWQ per-layer scale search on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {awq,reference}]
+
+One step = the whole hot path for one layer of the Llama-7B-shaped q_proj
+workload (X [65536 x 4096] fp16 heavy-tailed, W [4096 x 4096], INT4 g128,
+20 alphas + 20 clip ratios, packed): awq_act_stats -> awq_search_scale ->
+awq_search_clip -> awq_quant_pack.  With N GPUs (torchrun, one process per
+GPU) every rank runs the same step on its own layer (independent seeds): weak
+scaling, no data-path collective.  Rank 0 prints one JSON line.
+
+--impl reference times the CPU oracle (the fp64 restatement of the method
+the tests check the CUDA path against) on the host cores, on a bounded
+sample of the same workload, extrapolated to ms per layer.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "AWQ search ms/layer & candidate-GEMM TFLOP/s on 1 B200; % of TC/HBM roofline"
+UNIT = "ms/layer"
+WORKLOAD_INDEX = 1  # Llama-7B-shaped q_proj
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNELS_PER_STEP = {  # kernels this library launches per step (memsets excluded)
+    "act_stats": 2, "wmax": 1, "scale_grid": 1, "cand_quant": 1, "search_gemm": 1,
+    "mse_argmin": 1, "gram_blocks": 2, "clip_eval": 1, "quant_pack": 1,
+}
+# ncu capture of the dominant kernel (q_proj workload, one launch), per launch;
+# None when the kernel changed after the capture.
+NCU_TRAFFIC_BYTES = None
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def workload_description(wl, T, inn, out):
+    return {
+        "workload": f"{wl.name}: {wl.description}",
+        "tokens": T, "in": inn, "out": out, "w_bit": wl.w_bit, "group_size": wl.group_size,
+        "n_alpha": wl.n_alpha, "n_clip": wl.n_clip,
+        "l2": "inputs larger than L2 (X is 512 MiB, candidate operand 640 MiB); no flush",
+    }
+
+
+# ---------------------------------------------------------------- distributed
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def init_dist(backend: str, world: int):
+    import datetime
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist if world > 1 else None
+
+
+def max_over_ranks(value: float, dist, device="cpu") -> float:
+    """Max of a per-rank float over all ranks (identity on one rank)."""
+    if dist is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(dist, device=None):
+    if dist is not None:
+        if device is not None and device != "cpu":
+            dist.barrier(device_ids=[device])
+        else:
+            dist.barrier()
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while the
+    timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        import tempfile
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.3)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                p = [x.strip() for x in line.split(",")]
+                if len(p) >= 9:
+                    rows.append(p)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        pw = [float(r[3]) for r in rows if r[3].replace(".", "", 1).isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        loaded = [r for r in rows if pw and float(r[3]) > 0.5 * max(pw)] if pw else rows
+        sm_load = [float(r[1]) for r in loaded if r[1].replace(".", "").isdigit()] or sm
+        return {"sm_mhz": statistics.median(sm_load) if sm_load else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(pw) if pw else None}
+
+
+# ---------------------------------------------------------------- oracle arm
+def oracle_layer_ms(X, W, wl, row_fraction: float):
+    """Times the CPU oracle on the workload with a sample of the output rows
+    and extrapolates to one full layer: phases whose cost does not depend on
+    the number of output rows (abar, X^T X, the block Grams) are timed in full,
+    the per-row phases (candidate quantisation and scoring, clip scoring,
+    packing) on round(row_fraction * out) rows and scaled by 1/row_fraction.
+    Returns (ms per layer, sample description)."""
+    import numpy as np
+    from oracle import awq_oracle as O
+    Xn, Wn = X.numpy(), W.numpy()
+    out = Wn.shape[0]
+    rows = max(8, int(round(out * row_fraction)) // 8 * 8)
+    Ws = Wn[:rows]
+    t = {}
+    t0 = time.perf_counter()
+    abar = O.act_stats(Xn)
+    t["act_stats"] = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    G = O.gram(Xn)
+    t["gram"] = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    mse, best, s, _ = O.search_scale(Xn, Ws, abar, wl.w_bit, wl.group_size, wl.n_alpha, G=G)
+    t["search"] = time.perf_counter() - t0
+    clip_idx = None
+    if wl.n_clip:
+        t0 = time.perf_counter()
+        Gk = O.block_grams(Xn, wl.group_size)
+        t["block_grams"] = time.perf_counter() - t0
+        t0 = time.perf_counter()
+        clip_idx, _ = O.search_clip(Xn, Ws, s, wl.w_bit, wl.group_size, wl.n_clip, 0.5, Gk=Gk)
+        t["clip"] = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    O.quant_pack(Ws, s, clip_idx, wl.w_bit, wl.group_size, max(wl.n_clip, 1), 0.5)
+    t["pack"] = time.perf_counter() - t0
+    scale = out / rows
+    fixed = t["act_stats"] + t["gram"] + t.get("block_grams", 0.0)
+    total = fixed + (t["search"] + t.get("clip", 0.0) + t["pack"]) * scale
+    sample = (f"oracle (numpy fp64, BLAS matmuls) on the full X [{Xn.shape[0]} x {Xn.shape[1]}] "
+              f"and {rows} of {out} output rows; abar, X^T X and the block Grams timed in full, the "
+              f"per-row phases (alpha search, clip search, packing) scaled by {scale:.0f}; "
+              f"phase seconds {json.dumps({k: round(v, 3) for k, v in t.items()})}")
+    return total * 1e3, sample
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if world > 1 and rank != 0:
+        return 0
+    from synthetic import WORKLOADS, workload_inputs
+    wl = WORKLOADS[WORKLOAD_INDEX]
+    d = workload_inputs(WORKLOAD_INDEX)
+    _, X, W = d["groups"][0]
+    vals, sample = [], ""
+    for i in range(args.warmup + args.steps):
+        ms, sample = oracle_layer_ms(X, W, wl, args.ref_row_fraction)
+        if i >= args.warmup:
+            vals.append(ms)
+    value = statistics.mean(vals)
+    cores = os.cpu_count()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": UNIT,
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(value, 3), "higher_is_better": False, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded heavy-tailed X, N(0,0.02) W)",
+        "config": workload_description(wl, X.shape[0], X.shape[1], W.shape[0]),
+        "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- CUDA arm
+def run_awq(args):
+    import torch
+    world, rank, local = dist_env()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the AWQ path has no CPU implementation)")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = init_dist("nccl", world)
+    import post_weight_quantization_awq_b200 as awq
+    from synthetic import WORKLOADS, heavy_tailed_activations, gaussian_weight, OutlierSpec
+
+    wl = WORKLOADS[WORKLOAD_INDEX]
+    T, inn, out = wl.T, 4096, 4096
+    # each rank quantises its own layer (weak scaling); rank 0 is the workload's seed
+    seed = wl.seed + 1000 * rank
+    X = heavy_tailed_activations(T, inn, OutlierSpec(0.01, 20.0, 50.0), seed)
+    W = gaussian_weight(out, inn, seed)
+    cfg = awq.AwqConfig.make(w_bit=wl.w_bit, group_size=wl.group_size, n_alpha=wl.n_alpha,
+                             n_clip=wl.n_clip, clip_min=0.5)
+    Xd, Wd = X.to(dev), W.to(dev)
+    ws = awq.alloc_workspace(T, inn, out, cfg, dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        return awq.quantize_layer(Xd, Wd, cfg, ws=ws)
+
+    # ---- device-timed region: inputs resident in HBM
+    for _ in range(args.warmup):
+        step()
+    awq.awq_device_status(ws)
+    torch.cuda.synchronize(dev)
+    awq.profile_reset()
+    awq.profile_enable(True)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier(dist, local)
+        torch.cuda.synchronize(dev)
+        ev0.record(stream)
+        for _ in range(args.steps):
+            res = step()
+        ev1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(dist, local)
+    awq.profile_enable(False)
+    awq.awq_device_status(ws)
+    ms_step = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, dist, dev)
+    kern = {}
+    for name in KERNELS_PER_STEP:
+        tot, n = awq.profile_read(name)
+        kern[name] = (tot / n if n else None, n)
+    awq.profile_reset()
+
+    # ---- end to end through the public API: pinned host buffers in, results out
+    Xh, Wh = X.pin_memory(), W.pin_memory()
+    Xe = torch.empty_like(Xd)
+    We = torch.empty_like(Wd)
+    g = wl.group_size
+    host_out = {
+        "qweight": torch.empty((inn, out // 8), dtype=torch.int32).pin_memory(),
+        "qzeros": torch.empty((inn // g, out // 8), dtype=torch.int32).pin_memory(),
+        "scales": torch.empty((inn // g, out), dtype=torch.float16).pin_memory(),
+        "s_best": torch.empty(inn, dtype=torch.float32).pin_memory(),
+        "mse": torch.empty(wl.n_alpha, dtype=torch.float64).pin_memory(),
+        "best_idx": torch.empty(1, dtype=torch.int32).pin_memory(),
+        "clip_idx": torch.empty((out, inn // g), dtype=torch.uint8).pin_memory(),
+    }
+
+    def e2e_step():
+        Xe.copy_(Xh, non_blocking=True)
+        We.copy_(Wh, non_blocking=True)
+        r = awq.quantize_layer(Xe, We, cfg, ws=ws)
+        for k, h in host_out.items():
+            h.copy_(getattr(r, k), non_blocking=True)
+
+    for _ in range(max(1, min(args.warmup, 2))):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    e_steps = max(1, min(args.steps, 5))
+    barrier(dist, local)
+    torch.cuda.synchronize(dev)
+    ev0.record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    ev1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dist, local)
+    ms_e2e = max_over_ranks(ev0.elapsed_time(ev1) / e_steps, dist, dev)
+    h2d = X.numel() * 2 + W.numel() * 2
+    d2h = sum(h.numel() * h.element_size() for h in host_out.values())
+
+    # ---- CPU baseline (rank 0 at N=1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        ms_cpu, sample = oracle_layer_ms(X, W, wl, args.ref_row_fraction)
+        cpu = {"value": round(ms_cpu, 1), "unit": UNIT, "cores": os.cpu_count(), "kind": "oracle",
+               "sample": sample}
+
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peaks, src = load_peaks()
+    flops = 2.0 * T * inn * out * wl.n_alpha
+    gemm_ms = kern["search_gemm"][0]
+    tflops = flops / (gemm_ms * 1e-3) / 1e12
+    peak = float(peaks.get("bf16_tflops_sustained") or peaks["bf16_tflops"])
+    launches = sum(KERNELS_PER_STEP.values()) * args.steps
+    hbm = float(peaks["hbm_gbs"])
+    per_kernel = {k: {"ms": round(v[0], 4) if v[0] is not None else None, "launches": v[1]}
+                  for k, v in kern.items()}
+    # algorithmic bytes of the HBM-bound kernels, per launch
+    hbm_bytes = {"act_stats": T * inn * 2, "cand_quant": out * inn * 2 * (1 + wl.n_alpha),
+                 "quant_pack": out * inn * 2 + out * inn // 2 + (inn // g) * out * 2.5}
+    hbm_frac = {k: round(b / (kern[k][0] * 1e-3) / 1e9 / hbm, 3) for k, b in hbm_bytes.items()
+                if kern[k][0]}
+    value = ms_step / world  # whole job: world layers per step
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 3),
+        "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "fp16",
+        "data": "synthetic (seeded heavy-tailed X, N(0,0.02) W)",
+        "config": workload_description(wl, T, inn, out),
+        "candidate_gemm_tflops": round(tflops, 1),
+        "roofline": {"kernel": "search_gemm", "bound": "tensor", "achieved": round(tflops, 1),
+                     "peak": peak, "unit": "TFLOP/s", "frac": round(tflops / peak, 3),
+                     "traffic": NCU_TRAFFIC_BYTES,
+                     "peak_source": f"{src} bf16 dense {'sustained' if 'bf16_tflops_sustained' in peaks else 'burst'} "
+                                    "(fp16 has the same nominal rate)",
+                     "algorithmic_flops_per_launch": flops},
+        "hbm_kernels": {"peak_gbs": hbm, "frac": hbm_frac, "bytes_per_launch": hbm_bytes},
+        "kernels": per_kernel,
+        "clocks": clk.summary(),
+        "e2e": {"value": round(ms_e2e / world, 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": e_steps},
+        "gpu_launches": launches,
+        "cpu_baseline": cpu,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=("awq", "reference"), default="awq")
+    ap.add_argument("--ref-row-fraction", type=float, default=0.125,
+                    help="share of output rows the oracle runs on (then scaled)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_awq(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

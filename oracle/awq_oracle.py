@@ -54,6 +54,7 @@ __all__ = [
     "mse_gram",
     "search_scale",
     "clip_ratios",
+    "block_grams",
     "search_clip",
     "quant_pack",
     "unpack_nibbles",
@@ -222,18 +223,27 @@ def clip_ratios(n_clip: int, clip_min: float) -> np.ndarray:
     return np.array([1.0 - c * (1.0 - cm) / (n_clip - 1) for c in range(n_clip)], dtype=np.float64)
 
 
+def block_grams(X: np.ndarray, group: int) -> list:
+    """G_k = X_k^T X_k (fp64) for every group k of g input channels."""
+    X64 = np.asarray(X, dtype=np.float64)
+    Gn = X64.shape[1] // group
+    return [X64[:, k * group:(k + 1) * group].T @ X64[:, k * group:(k + 1) * group] for k in range(Gn)]
+
+
 def search_clip(X: np.ndarray, W: np.ndarray, s: np.ndarray, w_bit: int, group: int,
-                n_clip: int, clip_min: float) -> Tuple[np.ndarray, np.ndarray]:
+                n_clip: int, clip_min: float, Gk: Optional[list] = None
+                ) -> Tuple[np.ndarray, np.ndarray]:
     """For every (row o, group k) pick the clip ratio whose fake-quantised
     group gives the smallest output error over all tokens,
     E_okc = sum_t (sum_{j in k} X_tj delta^(c)_oj)^2 = d^T (X_k^T X_k) d.
+    ``Gk`` may pass the block Grams of X already computed.
 
     Returns (clip_idx uint8 [out, in/g], E fp64 [out, in/g, n_clip])."""
     out, inn = W.shape
     Gn = inn // group
     r = clip_ratios(n_clip, clip_min).astype(np.float32)
-    X64 = np.asarray(X, dtype=np.float64)
-    Gk = [X64[:, k * group:(k + 1) * group].T @ X64[:, k * group:(k + 1) * group] for k in range(Gn)]
+    if Gk is None:
+        Gk = block_grams(X, group)
     E = np.empty((out, Gn, n_clip), dtype=np.float64)
     for c in range(n_clip):
         ratio = np.full((out, Gn), r[c], dtype=np.float32)
