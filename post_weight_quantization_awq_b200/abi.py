@@ -85,13 +85,35 @@ def _load() -> ctypes.CDLL:
             "(nvcc, sm_100a); there is no fallback implementation")
     lib = ctypes.CDLL(LIB_PATH)
     for name, (res, args) in _SIGNATURES.items():
-        fn = getattr(lib, name)
+        try:
+            fn = getattr(lib, name)
+        except AttributeError as e:
+            raise ImportError(f"{LIB_PATH} does not export {name}: rebuild it") from e
         fn.restype = res
         fn.argtypes = args
     return lib
 
 
-LIB = _load()
+class _Lib:
+    """libawq.so, loaded on first use (so that the build module can be
+    imported before the library exists); a missing or stale library raises
+    ImportError at the first call."""
+
+    _lib = None
+
+    def _get(self) -> ctypes.CDLL:
+        if _Lib._lib is None:
+            _Lib._lib = _load()
+        return _Lib._lib
+
+    def __getattr__(self, name):
+        return getattr(self._get(), name)
+
+    def __getitem__(self, name):
+        return self._get()[name]
+
+
+LIB = _Lib()
 
 
 def header_functions(path: str = HEADER_PATH):
