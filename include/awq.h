@@ -130,6 +130,33 @@ awq_status awq_search_clip(const void *X, int64_t T, int64_t in, int64_t ldx,
                            const awq_config *cfg, void *ws, size_t ws_bytes,
                            uint8_t *clip_idx, float *err, awq_stream_t stream);
 
+/* Allocation-free variant of awq_search_clip (the AWQ pages have no
+ * counterpart: this entry exists for callers, not for the method).  Some
+ * callers cannot allocate device memory while the search runs: a host
+ * framework that owns every device byte through its own pre-planned arena,
+ * or code that must not call cudaMalloc because that call can synchronise the
+ * device in the middle of its stream work.  This call takes no workspace and
+ * calls no cudaMalloc, cudaFree or allocating library routine: its scratch
+ * (the block Grams) lives in a static device array of 24 MiB inside this
+ * library, which every GPU that loads the library holds until the process
+ * exits.  Arguments and outputs are those of awq_search_clip, with these
+ * differences:
+ *   - in must be at most 16384; larger layers return AWQ_ERR_INVALID_ARG
+ *     (use awq_search_clip with a workspace);
+ *   - the first call on a device looks up the device address of the static
+ *     array (cudaGetSymbolAddress) with that device current; make that first
+ *     call before any stream capture;
+ *   - every call shares the one array, so calls that overlap on the GPU (on
+ *     different streams, or from different threads) race and must be
+ *     serialised by the caller.  Nothing in the array needs clearing: each
+ *     call writes every element it reads.
+ * Results equal awq_search_clip's up to the fp32 summation order of the block
+ * Grams (token chunks are summed in a different grouping). */
+awq_status awq_search_clip_noalloc(const void *X, int64_t T, int64_t in, int64_t ldx,
+                                   const void *W, int64_t out, const float *s,
+                                   const awq_config *cfg, uint8_t *clip_idx, float *err,
+                                   awq_stream_t stream);
+
 /* Final quantisation and packing ("05 — AWQ" §5 bit-level output format).
  *   s        device fp32 [in] or NULL (s = 1)
  *   clip_idx device uint8 [out, in/g] or NULL (ratio 1)

@@ -21,6 +21,7 @@ from .abi import (  # noqa: F401
     awq_quant_pack,
     awq_scale_grid,
     awq_search_clip,
+    awq_search_clip_noalloc,
     awq_search_scale,
     awq_workspace_size,
     header_functions,

@@ -68,6 +68,9 @@ _SIGNATURES = {
     "awq_search_clip": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_int64, c_void_p,
                                   POINTER(AwqConfig), c_void_p, c_size_t, c_void_p, c_void_p,
                                   c_void_p]),
+    "awq_search_clip_noalloc": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_int64,
+                                          c_void_p, POINTER(AwqConfig), c_void_p, c_void_p,
+                                          c_void_p]),
     "awq_quant_pack": (c_int32, [c_void_p, c_int64, c_int64, c_void_p, c_void_p, POINTER(AwqConfig),
                                  c_void_p, c_void_p, c_void_p, c_void_p]),
     "awq_fold_inv_scale": (c_int32, [c_void_p, c_int64, c_int64, c_void_p, c_void_p]),
@@ -178,6 +181,14 @@ def awq_search_clip(X, W, s, cfg: AwqConfig, ws, clip_idx, err=None, stream=None
         _ptr(X), X.shape[0], X.shape[1], X.stride(0), _ptr(W), W.shape[0], _ptr(s),
         ctypes.byref(cfg), _ptr(ws), ws.numel() * ws.element_size(), _ptr(clip_idx), _ptr(err),
         _stream(stream)))
+
+
+def awq_search_clip_noalloc(X, W, s, cfg: AwqConfig, clip_idx, err=None, stream=None) -> None:
+    """awq_search_clip without a workspace (scratch in the library's static
+    device array; in <= 16384; overlapping calls race)."""
+    _check("awq_search_clip_noalloc", LIB.awq_search_clip_noalloc(
+        _ptr(X), X.shape[0], X.shape[1], X.stride(0), _ptr(W), W.shape[0], _ptr(s),
+        ctypes.byref(cfg), _ptr(clip_idx), _ptr(err), _stream(stream)))
 
 
 def awq_quant_pack(W, s, clip_idx, cfg: AwqConfig, qweight, qzeros, scales, stream=None) -> None:

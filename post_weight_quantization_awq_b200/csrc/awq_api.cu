@@ -431,3 +431,85 @@ awq_status awq_profile_reset(void) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free clip search.
+//
+// Some callers cannot allocate device memory while they run this search: a
+// host framework that owns every device byte through its own pre-planned
+// arena (and forbids stray cudaMalloc calls that would fragment it or
+// overlap its budget), or code that must not call cudaMalloc because that
+// call can synchronise the whole device in the middle of its pipelined
+// stream work.  awq_search_clip_noalloc takes no workspace: its block-Gram
+// scratch lives in the file-scope device array below, sized for layers of up
+// to kNoAllocMaxIn input channels.  The array is part of this library's
+// module, so every GPU that loads the library holds it (24 MiB) until the
+// process exits.
+// ---------------------------------------------------------------------------
+namespace {
+constexpr int64_t kNoAllocMaxIn = 16384;  // up to 128 groups of 128 channels
+constexpr int kNoAllocChunks = 2;         // token chunks of the block-Gram partials
+constexpr size_t kNoAllocGroupFloats = 128 * 128;
+constexpr size_t kNoAllocFloats =
+    (size_t)(kNoAllocChunks + 1) * (size_t)(kNoAllocMaxIn / 128) * kNoAllocGroupFloats;
+
+std::mutex g_noalloc_mu;
+float *g_noalloc_ptr[64] = {};
+}  // namespace
+
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocFloats];
+
+extern "C" awq_status awq_search_clip_noalloc(const void *X, int64_t T, int64_t in, int64_t ldx,
+                                              const void *W, int64_t out, const float *s,
+                                              const awq_config *cfg, uint8_t *clip_idx, float *err,
+                                              awq_stream_t stream) {
+  g_err.clear();
+  awq_status st = check_cfg(cfg);
+  if (st != AWQ_OK) return st;
+  if (cfg->n_clip < 1) return fail(AWQ_ERR_INVALID_ARG, "n_clip=%d: clip search needs n_clip >= 1", cfg->n_clip);
+  if ((st = check_shape(T, in, out, cfg)) != AWQ_OK) return st;
+  if (in > kNoAllocMaxIn)
+    return fail(AWQ_ERR_INVALID_ARG,
+                "in=%lld exceeds the %lld input channels the allocation-free clip search's "
+                "static scratch holds; use awq_search_clip with a workspace",
+                (long long)in, (long long)kNoAllocMaxIn);
+  if ((st = check_x(X, in, ldx)) != AWQ_OK) return st;
+  if (!W || !aligned(W, 16)) return fail(AWQ_ERR_INVALID_ARG, "W is NULL or not 16-byte aligned");
+  if (!clip_idx) return fail(AWQ_ERR_INVALID_ARG, "clip_idx is NULL");
+  if (s && !aligned(s, 16)) return fail(AWQ_ERR_INVALID_ARG, "s must be 16-byte aligned");
+
+  // Device address of the static scratch, looked up once per device with that
+  // device current (the host-side symbol is not a device address).
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 64) return fail(AWQ_ERR_UNSUPPORTED, "device ordinal %d", dev);
+  float *scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+      void *p = nullptr;
+      e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static clip scratch)");
+      g_noalloc_ptr[dev] = static_cast<float *>(p);
+    }
+    scratch = g_noalloc_ptr[dev];
+  }
+
+  // Every scratch element a call reads is written earlier in the same call
+  // (all chunk partials of the groups in use, then their sums), so nothing
+  // has to be cleared between calls.
+  const int64_t c = (T + 1023) / 1024;
+  const int n_chunks = (int)(c < 1 ? 1 : (c > kNoAllocChunks ? kNoAllocChunks : c));
+  const size_t gsz = (size_t)(in / 128) * kNoAllocGroupFloats;
+  float *gpart = scratch;
+  float *Gk = scratch + gsz * (size_t)n_chunks;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  e = launch_gram_blocks(static_cast<const __half *>(X), T, in, ldx, cfg->group_size, n_chunks,
+                         gpart, Gk, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "gram_blocks launch");
+  e = launch_clip_eval(static_cast<const __half *>(W), out, in, s, Gk, cfg->group_size, cfg->w_bit,
+                       cfg->n_clip, cfg->clip_min, clip_idx, err, cs);
+  if (e != cudaSuccess) return cuda_fail(e, "clip_eval launch");
+  return AWQ_OK;
+}
