@@ -18,10 +18,11 @@ enum : uint32_t {
 };
 
 struct DevStatus {
-  uint32_t flags;     // kDev* bits, OR-ed by kernels
-  uint32_t where;     // code of the first wait that ran out (debug aid)
-  int32_t kscale;     // power-of-two exponent applied to the candidate errors
-  uint32_t wmax_bits; // bit pattern of max |W| (a non-negative float)
+  uint32_t flags;      // kDev* bits, OR-ed by kernels
+  uint32_t where;      // code of the first wait that ran out (debug aid)
+  int32_t kscale;      // power-of-two exponent applied to the candidate errors
+  uint32_t wmax_bits;  // bit pattern of max |W| (a non-negative float)
+  uint32_t mse_done;   // blocks of the MSE reduction that have finished
 };
 
 __device__ __forceinline__ void dev_fail(DevStatus *st, uint32_t flag, uint32_t where) {
@@ -38,10 +39,11 @@ __device__ __forceinline__ void dev_fail(DevStatus *st, uint32_t flag, uint32_t 
 // contracting any of them into an FMA.
 // ---------------------------------------------------------------------------
 struct GroupQ {
-  float delta;  // step
-  float zero;   // zero point (integer valued)
-  float qmax;   // 2^b - 1
-  float rcp;    // RN(1/delta), used for the fast code path
+  float delta;    // step
+  float zero;     // zero point (integer valued)
+  float qmax;     // 2^b - 1
+  float rcp;      // RN(1/delta), used for the fast code path
+  float half_lo;  // delta * (0.5 - 2^-16): remainders below it prove the fast code exact
 };
 
 // Range of one group after the optional clip ratio r32 (1 = no clip).
@@ -57,21 +59,21 @@ __device__ __forceinline__ GroupQ group_params(float mx, float mn, float r32, fl
   g.zero = fminf(fmaxf(z, 0.0f), qmax);
   g.qmax = qmax;
   g.rcp = __frcp_rn(g.delta);
+  g.half_lo = __fmul_rn(g.delta, 0.4999847412109375f /* 0.5 - 2^-16 */);
   return g;
 }
 
-// rne(RN32(wt / delta)) without a full division on the common path: y =
-// RN(wt * RN(1/delta)) is within 1.5 ulp of wt/delta, so unless y lies within
-// a few ulp of a half-integer both round to the same integer; otherwise (or
-// for very large quotients) fall back to the correctly rounded quotient.
+// rne(RN32(wt / delta)) without a division on the common path.  k = rne of
+// the approximate quotient wt * RN(1/delta); the remainder wt - k*delta comes
+// from one FMA (a single rounding).  If |remainder| < delta (0.5 - 2^-16) and
+// |k| < 64, then |wt/delta - k| < 0.5 - 2^-16 + 2^-22, and the fp32 rounding of
+// wt/delta moves it by at most 2^-24 * 64.5 < 2^-17, so RN32(wt/delta) is
+// strictly within 0.5 of k and rounds to k.  Otherwise the correctly rounded
+// quotient decides.
 __device__ __forceinline__ float round_quotient(float wt, const GroupQ &g) {
-  float y = __fmul_rn(wt, g.rcp);
-  float ay = fabsf(y);
-  float h = __fadd_rn(floorf(y), 0.5f);
-  float dist = fabsf(__fsub_rn(y, h));
-  if (ay < 1048576.0f && dist > __fmul_rn(fmaxf(ay, 1.0f), 4.76837158203125e-07f /*2^-21*/)) {
-    return rintf(y);
-  }
+  const float k = rintf(__fmul_rn(wt, g.rcp));
+  const float rem = fmaf(-k, g.delta, wt);
+  if (fabsf(rem) < g.half_lo && fabsf(k) < 64.0f) return k;
   return rintf(__fdiv_rn(wt, g.delta));
 }
 

@@ -171,45 +171,56 @@ cudaError_t launch_wmax(const __half *W, int64_t n, DevStatus *st, int num_sms,
 // step and zero point, the codes, deq = (q - z) delta, and writes the
 // effective error (deq/s - w) * 2^k as fp16: row (i * out_pad + o) of the
 // tensor-core B operand [n_alpha * out_pad, in].  Rows out..out_pad-1 of each
-// candidate are zero.  Each thread handles 8 consecutive channels (16-byte
-// loads and stores).
+// candidate are zero.
+// A block covers one candidate, 64 rows and a slab of 256 channels: lane l
+// owns channels 8l..8l+7 of the slab (16-byte loads and stores) and keeps
+// their s and 1/s in registers while its warp walks 8 of the 64 rows.
 // ---------------------------------------------------------------------------
+constexpr int kCandRows = 64;
+
 __global__ void __launch_bounds__(256) cand_quant_kernel(
     const __half *__restrict__ W, int64_t out, int64_t in, int64_t out_pad,
-    const float *__restrict__ s, const float *__restrict__ inv_s, int n_alpha, int group,
-    float qmax, const DevStatus *__restrict__ st, __half *__restrict__ dW) {
+    const float *__restrict__ s, const float *__restrict__ inv_s, int group, float qmax,
+    const DevStatus *__restrict__ st, __half *__restrict__ dW) {
   const int k = kscale_from_wmax(__uint_as_float(__ldg(&st->wmax_bits)));
   const float two_k = ldexpf(1.0f, k);
   const int lanes = group / 8;  // lanes per group (a power of two <= 32)
-  const int64_t items_per_row = in / 8;
-  const int64_t total = (int64_t)n_alpha * out_pad * items_per_row;  // multiple of 32
-  for (int64_t it = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; it < total;
-       it += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t row = it / items_per_row;
-    const int64_t j0 = (it - row * items_per_row) * 8;
-    const int a = (int)(row / out_pad);
-    const int64_t o = row - (int64_t)a * out_pad;
-    const bool live = o < out;
-    float w[8], sv[8], iv[8];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t j0 = (int64_t)blockIdx.x * 256 + lane * 8;
+  const bool j_ok = j0 < in;
+  const int rb_per_alpha = (int)(out_pad / kCandRows);
+  const int a = blockIdx.y / rb_per_alpha;
+  const int64_t o0 = (int64_t)(blockIdx.y - a * rb_per_alpha) * kCandRows;
+  float sv[8], iv[8];
+  if (j_ok) {
+    const float4 *sp = reinterpret_cast<const float4 *>(s + (int64_t)a * in + j0);
+    const float4 *ip = reinterpret_cast<const float4 *>(inv_s + (int64_t)a * in + j0);
+    const float4 s0 = __ldg(sp), s1 = __ldg(sp + 1), i0 = __ldg(ip), i1 = __ldg(ip + 1);
+    sv[0] = s0.x; sv[1] = s0.y; sv[2] = s0.z; sv[3] = s0.w;
+    sv[4] = s1.x; sv[5] = s1.y; sv[6] = s1.z; sv[7] = s1.w;
+    iv[0] = i0.x; iv[1] = i0.y; iv[2] = i0.z; iv[3] = i0.w;
+    iv[4] = i1.x; iv[5] = i1.y; iv[6] = i1.z; iv[7] = i1.w;
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) { sv[e] = 1.0f; iv[e] = 1.0f; }
+  }
+#pragma unroll 2
+  for (int r = warp; r < kCandRows; r += 8) {
+    const int64_t o = o0 + r;
+    const bool live = j_ok && o < out;
+    float w[8];
     if (live) {
-      uint4 wv = __ldg(reinterpret_cast<const uint4 *>(W + o * in + j0));
+      const uint4 wv = __ldg(reinterpret_cast<const uint4 *>(W + o * in + j0));
       const uint32_t wr[4] = {wv.x, wv.y, wv.z, wv.w};
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
-        float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&wr[h]));
+        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&wr[h]));
         w[2 * h] = f.x;
         w[2 * h + 1] = f.y;
       }
-      const float4 *sp = reinterpret_cast<const float4 *>(s + (int64_t)a * in + j0);
-      const float4 *ip = reinterpret_cast<const float4 *>(inv_s + (int64_t)a * in + j0);
-      float4 s0 = __ldg(sp), s1 = __ldg(sp + 1), i0 = __ldg(ip), i1 = __ldg(ip + 1);
-      sv[0] = s0.x; sv[1] = s0.y; sv[2] = s0.z; sv[3] = s0.w;
-      sv[4] = s1.x; sv[5] = s1.y; sv[6] = s1.z; sv[7] = s1.w;
-      iv[0] = i0.x; iv[1] = i0.y; iv[2] = i0.z; iv[3] = i0.w;
-      iv[4] = i1.x; iv[5] = i1.y; iv[6] = i1.z; iv[7] = i1.w;
     } else {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) { w[e] = 0.0f; sv[e] = 1.0f; iv[e] = 1.0f; }
+      for (int e = 0; e < 8; ++e) w[e] = 0.0f;
     }
     float wt[8];
     float mx = -INFINITY, mn = INFINITY;
@@ -224,6 +235,7 @@ __global__ void __launch_bounds__(256) cand_quant_kernel(
       mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
     }
     const GroupQ g = group_params(mx, mn, 1.0f, qmax);
+    const float dk = __fmul_rn(g.delta, two_k);  // exact: power-of-two scaling
     uint32_t packed[4];
 #pragma unroll
     for (int h = 0; h < 4; ++h) {
@@ -231,26 +243,27 @@ __global__ void __launch_bounds__(256) cand_quant_kernel(
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
         const int e = 2 * h + u;
-        const float deq = dequant(quant_code(wt[e], g), g);
-        // (deq/s - w) 2^k; 2^k is exact, the product with 1/s is fp32 (the
-        // result is rounded to fp16 next)
-        d2[u] = fmaf(__fmul_rn(deq, two_k), iv[e], -__fmul_rn(w[e], two_k));
-        if (!live) d2[u] = 0.0f;
+        const float qz = __fsub_rn(quant_code(wt[e], g), g.zero);
+        // 2^k (deq/s - w) with deq = (q - z) delta; the product with 1/s is
+        // fp32 (the result is rounded to fp16 next)
+        d2[u] = live ? fmaf(__fmul_rn(qz, dk), iv[e], -__fmul_rn(w[e], two_k)) : 0.0f;
       }
-      __half2 hv = __floats2half2_rn(d2[0], d2[1]);
-      packed[h] = *reinterpret_cast<uint32_t *>(&hv);
+      const __half2 hv = __floats2half2_rn(d2[0], d2[1]);
+      packed[h] = *reinterpret_cast<const uint32_t *>(&hv);
     }
-    *reinterpret_cast<uint4 *>(dW + row * in + j0) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+    if (j_ok)
+      *reinterpret_cast<uint4 *>(dW + ((int64_t)a * out_pad + o) * in + j0) =
+          make_uint4(packed[0], packed[1], packed[2], packed[3]);
   }
 }
 
 cudaError_t launch_cand_quant(const __half *W, int64_t out, int64_t in, int64_t out_pad,
                               const float *s, const float *inv_s, int n_alpha, int group, int w_bit,
                               const DevStatus *st, __half *dW, int num_sms, cudaStream_t stream) {
-  const int64_t total = (int64_t)n_alpha * out_pad * (in / 8);
-  int64_t blocks = i64min((int64_t)num_sms * 8, (total + 255) / 256);
-  cand_quant_kernel<<<(unsigned)blocks, 256, 0, stream>>>(W, out, in, out_pad, s, inv_s, n_alpha,
-                                                          group, (float)((1 << w_bit) - 1), st, dW);
+  (void)num_sms;
+  dim3 grid((unsigned)((in + 255) / 256), (unsigned)(n_alpha * (out_pad / kCandRows)));
+  cand_quant_kernel<<<grid, 256, 0, stream>>>(W, out, in, out_pad, s, inv_s, group,
+                                              (float)((1 << w_bit) - 1), st, dW);
   return cudaGetLastError();
 }
 

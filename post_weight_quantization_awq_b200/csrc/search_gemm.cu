@@ -299,38 +299,49 @@ cudaError_t launch_search_gemm(const __half *X, int64_t ldx, const __half *dW,
 }
 
 // ---------------------------------------------------------------------------
-// K5 — MSE_i = (sum of candidate i's partials) * 2^-2k / (T out), summed in a
-// fixed order (bitwise reproducible); best = first index of the smallest MSE;
-// s_best = s_grid[best].  One block.
+// K5 — MSE_i = (sum of candidate i's partials) * 2^-2k / (T out).  One block
+// per candidate sums its partials in a fixed order (bitwise reproducible);
+// the last block to finish picks best = the first index of the smallest MSE
+// and copies s_best = s_grid[best].
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024) mse_argmin_kernel(
     const double *__restrict__ partials, int n_alpha, int nb_per_alpha, int num_m, int64_t T,
     int64_t out, const float *__restrict__ s_grid, int64_t in, DevStatus *st,
     double *__restrict__ mse, int32_t *__restrict__ best_idx, float *__restrict__ s_best) {
   __shared__ double red[1024];
-  __shared__ int best_sh;
-  const int k = kscale_from_wmax(__uint_as_float(st->wmax_bits));
+  __shared__ int last_sh, best_sh;
+  const int i = blockIdx.x;
+  const int k = kscale_from_wmax(__uint_as_float(__ldcg(&st->wmax_bits)));
   const size_t per = (size_t)nb_per_alpha * num_m * 4;
-  for (int i = 0; i < n_alpha; ++i) {
-    const double *p = partials + (size_t)i * per;
-    double acc = 0.0;
-    for (size_t idx = threadIdx.x; idx < per; idx += blockDim.x) acc += p[idx];
-    red[threadIdx.x] = acc;
-    __syncthreads();
-    for (int w = blockDim.x >> 1; w > 0; w >>= 1) {
-      if ((int)threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
-      __syncthreads();
-    }
-    if (threadIdx.x == 0) mse[i] = ldexp(red[0], -2 * k) / ((double)T * (double)out);
+  const double *p = partials + (size_t)i * per;
+  double acc = 0.0;
+  for (size_t idx = threadIdx.x; idx < per; idx += blockDim.x) acc += __ldcg(p + idx);
+  red[threadIdx.x] = acc;
+  __syncthreads();
+  for (int w = blockDim.x >> 1; w > 0; w >>= 1) {
+    if ((int)threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
     __syncthreads();
   }
   if (threadIdx.x == 0) {
+    const double v = ldexp(red[0], -2 * k) / ((double)T * (double)out);
+    __stcg(mse + i, v);
+    __threadfence();
+    last_sh = atomicAdd(&st->mse_done, 1u) == (unsigned)(n_alpha - 1);
+  }
+  __syncthreads();
+  if (!last_sh) return;
+  if (threadIdx.x == 0) {
+    __threadfence();
     int best = 0;
-    bool finite = true;
-    for (int i = 0; i < n_alpha; ++i) {
-      const double v = mse[i];
+    double bv = __ldcg(mse);
+    bool finite = isfinite(bv);
+    for (int a = 1; a < n_alpha; ++a) {
+      const double v = __ldcg(mse + a);
       if (!isfinite(v)) finite = false;
-      if (v < mse[best]) best = i;
+      if (v < bv) {
+        bv = v;
+        best = a;
+      }
     }
     if (!finite) dev_fail(st, kDevNonFinite, 0x500u);
     best_sh = best;
@@ -345,8 +356,8 @@ cudaError_t launch_mse_argmin(const double *partials, int n_alpha, int nb_per_al
                               int64_t T, int64_t out, const float *s_grid, int64_t in,
                               DevStatus *st, double *mse, int32_t *best_idx, float *s_best,
                               cudaStream_t stream) {
-  mse_argmin_kernel<<<1, 1024, 0, stream>>>(partials, n_alpha, nb_per_alpha, num_m, T, out, s_grid,
-                                            in, st, mse, best_idx, s_best);
+  mse_argmin_kernel<<<n_alpha, 1024, 0, stream>>>(partials, n_alpha, nb_per_alpha, num_m, T, out,
+                                                  s_grid, in, st, mse, best_idx, s_best);
   return cudaGetLastError();
 }
 
