@@ -333,7 +333,8 @@ awq_status awq_search_clip(const void *X, int64_t T, int64_t in, int64_t ldx, co
   {
     ProfScope p("gram_blocks", cs);
     AWQ_TRY_CUDA(launch_gram_blocks(static_cast<const __half *>(X), T, in, ldx, cfg->group_size,
-                                    L.n_chunks, gpart, Gk, cs),
+                                    L.n_chunks, gpart, Gk, reinterpret_cast<DevStatus *>(base),
+                                    poll_cap(), cs),
                  "gram_blocks launch");
   }
   {
@@ -505,8 +506,9 @@ extern "C" awq_status awq_search_clip_noalloc(const void *X, int64_t T, int64_t 
   float *gpart = scratch;
   float *Gk = scratch + gsz * (size_t)n_chunks;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  // no status word here: a bounded wait that ran out leaves clip_idx unset
   e = launch_gram_blocks(static_cast<const __half *>(X), T, in, ldx, cfg->group_size, n_chunks,
-                         gpart, Gk, cs);
+                         gpart, Gk, nullptr, 1u << 24, cs);
   if (e != cudaSuccess) return cuda_fail(e, "gram_blocks launch");
   e = launch_clip_eval(static_cast<const __half *>(W), out, in, s, Gk, cfg->group_size, cfg->w_bit,
                        cfg->n_clip, cfg->clip_min, clip_idx, err, cs);

@@ -2,6 +2,7 @@
 // enqueues work on `stream` and returns the launch error, if any.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -39,15 +40,22 @@ cudaError_t launch_search_gemm(const __half *X, int64_t ldx, const __half *dW,
                                uint32_t max_polls, int num_sms, cudaStream_t stream);
 constexpr int kGemmBM = 128, kGemmBN = 256, kGemmBK = 64;
 
+// 2-D fp16 TMA descriptor over a row-major [rows, cols] matrix (row stride
+// `ld` elements), box [box_rows, box_cols], 128-byte swizzle, zero fill.
+cudaError_t make_tmap_f16_box(CUtensorMap *m, const void *base, int64_t rows, int64_t cols,
+                              int64_t ld, uint32_t box_cols, uint32_t box_rows);
+
 // K5: mse[i], best index, s_best.
 cudaError_t launch_mse_argmin(const double *partials, int n_alpha, int nb_per_alpha, int num_m,
                               int64_t T, int64_t out, const float *s_grid, int64_t in,
                               DevStatus *st, double *mse, int32_t *best_idx, float *s_best,
                               cudaStream_t stream);
 
-// K6a: block Grams G[k] = X_k^T X_k (fp32), via per-chunk partials.
+// K6a: block Grams G[k] = X_k^T X_k (fp32, tensor cores), via per-chunk
+// partials [n_chunks][in/g][g][g] summed in a fixed order.
 cudaError_t launch_gram_blocks(const __half *X, int64_t T, int64_t in, int64_t ldx, int group,
-                               int n_chunks, float *partials, float *G, cudaStream_t stream);
+                               int n_chunks, float *partials, float *G, DevStatus *st,
+                               uint32_t max_polls, cudaStream_t stream);
 // K6b: clip choice per (row, group).
 cudaError_t launch_clip_eval(const __half *W, int64_t out, int64_t in, const float *s,
                              const float *G, int group, int w_bit, int n_clip, float clip_min,

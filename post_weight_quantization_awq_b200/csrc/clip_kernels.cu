@@ -7,14 +7,15 @@
 // with d = deq_c/s - w over the group's g channels.  G_k does not depend on s
 // or on the row, so it is built once per call (K6a) and every (o, k, c) is a
 // 128-dimensional fp32 quadratic form (K6b).
-//   K6a  gram_blocks: fp32 FFMA over token chunks, one block per (group,
-//        chunk), 8x8 outputs per thread; chunk partials are summed in a fixed
-//        order by gram_reduce, so G is bitwise reproducible.
+//   K6a  gram_tc: tensor-core block Grams over token chunks, one CTA per
+//        (group, chunk); chunk partials are summed in a fixed order by
+//        gram_reduce, so G is bitwise reproducible.
 //   K6b  clip_eval: one block per (group, 16 rows) holds G_k in shared memory;
 //        a warp quantises one row for a batch of clip ratios, writes the error
 //        vectors to shared memory and evaluates y = G_k d for the whole batch
 //        (each G element read once per batch), then E = d . y by warp
 //        shuffles; the first c with the smallest E wins.
+#include <cuda.h>
 #include <cuda_fp16.h>
 #include <math.h>
 
@@ -24,83 +25,177 @@ namespace awq {
 
 namespace {
 constexpr int G = 128;          // group size handled by these kernels
-constexpr int GRAM_TT = 32;     // tokens staged per step
-constexpr int GRAM_PAD = 4;     // row padding of the staged tile (floats)
 constexpr int CLIP_ROWS = 16;   // rows per clip_eval block
 constexpr int CLIP_WARPS = 4;
 constexpr int CLIP_CB = 10;     // clip ratios per batch
 constexpr int GSTRIDE = G + 4;  // shared-memory row stride of G_k (floats)
 }  // namespace
 
-// Thread (ty, tx) of a 16x16 block owns rows {4ty..4ty+3, 64+4ty..64+4ty+3} and
-// the same split set of columns for tx, so float4 reads of a staged token row
-// are bank-conflict free.
-__global__ void __launch_bounds__(256) gram_blocks_kernel(const __half *__restrict__ X, int64_t T,
-                                                          int64_t ldx, int64_t chunk_tokens,
-                                                          int64_t n_groups,
-                                                          float *__restrict__ partials) {
-  __shared__ __align__(16) float xs[GRAM_TT][G + GRAM_PAD];
-  const int k = blockIdx.x;
-  const int chunk = blockIdx.y;
-  const int tid = threadIdx.x;
-  const int tx = tid & 15, ty = tid >> 4;
-  const int64_t t0 = (int64_t)chunk * chunk_tokens;
-  const int64_t t1 = min(T, t0 + chunk_tokens);
-  float acc[8][8];
-#pragma unroll
-  for (int a = 0; a < 8; ++a)
-#pragma unroll
-    for (int b = 0; b < 8; ++b) acc[a][b] = 0.0f;
+// ---------------------------------------------------------------------------
+// K6a — block Grams on the tensor cores.  One CTA per (group k, token chunk):
+// TMA brings X[t0:t0+64, 128k:128k+128] as two 64-channel boxes with 128-byte
+// swizzling (rows = tokens), which is the MN-major layout of X_k^T; the same
+// shared-memory tile is both the A (M = 128 channels) and the B (N = 128
+// channels) operand of tcgen05.mma kind::f16 (K = 16 tokens per instruction),
+// accumulating G_k = X_k^T X_k in fp32 in 128 TMEM columns.  fp16 products
+// are exact in fp32.  Warp 0 loads, warp 1 issues MMAs, warps 2..5 write the
+// 128 x 128 partial; chunk partials are summed in a fixed order afterwards.
+// ---------------------------------------------------------------------------
+namespace {
+constexpr int GT = 64;                          // tokens per stage
+constexpr int GSTAGES = 6;
+constexpr uint32_t GBOX_BYTES = 64 * GT * 2;    // 64 channels x 64 tokens fp16
+constexpr uint32_t GSTAGE_BYTES = 2 * GBOX_BYTES;
+constexpr uint32_t GDRAIN_POLLS = 1u << 22;
+// kind::f16, fp16 A/B, fp32 D, A and B MN-major, N = 128, M = 128
+constexpr uint32_t IDESC_GRAM =
+    (1u << 4) | (1u << 15) | (1u << 16) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
 
-  for (int64_t tb = t0; tb < t1; tb += GRAM_TT) {
-    // stage GRAM_TT rows x 128 channels (fp16 -> fp32); 256 threads x 16 values
-    {
-      const int r = tid >> 3;          // 0..31
-      const int c = (tid & 7) * 16;    // 0..112
-      const int64_t t = tb + r;
-      float v[16];
-      if (t < t1) {
-        const uint4 *p = reinterpret_cast<const uint4 *>(X + t * ldx + (int64_t)k * G + c);
-        uint4 a = __ldg(p), b = __ldg(p + 1);
-        const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-#pragma unroll
-        for (int h = 0; h < 8; ++h) {
-          float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[h]));
-          v[2 * h] = f.x;
-          v[2 * h + 1] = f.y;
-        }
-      } else {
-#pragma unroll
-        for (int h = 0; h < 16; ++h) v[h] = 0.0f;
-      }
-#pragma unroll
-      for (int h = 0; h < 16; h += 4)
-        *reinterpret_cast<float4 *>(&xs[r][c + h]) = make_float4(v[h], v[h + 1], v[h + 2], v[h + 3]);
+struct __align__(8) GramTail {
+  uint64_t full[GSTAGES];
+  uint64_t empty[GSTAGES];
+  uint64_t done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+constexpr size_t kGramSmemBytes = 1024 + GSTAGES * GSTAGE_BYTES + sizeof(GramTail);
+
+// MN-major operand with 128-byte swizzling: 64 channels (128 B) per token row,
+// 8-row core groups 1024 B apart (SBO), the second 64-channel half of the
+// group GBOX_BYTES further (LBO).
+__device__ __forceinline__ uint64_t smem_desc_mn_sw128(uint32_t addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((GBOX_BYTES >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)(1024u >> 4) << 32;
+  d |= (uint64_t)1u << 46;
+  d |= (uint64_t)2u << 61;
+  return d;
+}
+}  // namespace
+
+__global__ void __launch_bounds__(192, 1)
+    gram_tc_kernel(const __grid_constant__ CUtensorMap tmX, int64_t T, int64_t chunk_tokens,
+                   int64_t n_groups, float *__restrict__ partials, DevStatus *st,
+                   uint32_t max_polls) {
+  extern __shared__ uint8_t gsm_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(gsm_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  GramTail *tail = reinterpret_cast<GramTail *>(smem + GSTAGES * GSTAGE_BYTES);
+  volatile int *abort_flag = &tail->abort_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int k = blockIdx.x, chunk = blockIdx.y;
+  const int64_t t0 = (int64_t)chunk * chunk_tokens;
+  const int64_t t1 = i64min(T, t0 + chunk_tokens);
+  const int nsteps = (int)((t1 - t0 + GT - 1) / GT);  // >= 1 by construction of the chunks
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < GSTAGES; ++s) {
+      mbar_init(&tail->full[s], 1);
+      mbar_init(&tail->empty[s], 1);
     }
-    __syncthreads();
-#pragma unroll 4
-    for (int t = 0; t < GRAM_TT; ++t) {
-      const float4 a0 = *reinterpret_cast<const float4 *>(&xs[t][4 * ty]);
-      const float4 a1 = *reinterpret_cast<const float4 *>(&xs[t][64 + 4 * ty]);
-      const float4 b0 = *reinterpret_cast<const float4 *>(&xs[t][4 * tx]);
-      const float4 b1 = *reinterpret_cast<const float4 *>(&xs[t][64 + 4 * tx]);
-      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-#pragma unroll
-      for (int a = 0; a < 8; ++a)
-#pragma unroll
-        for (int b = 0; b < 8; ++b) acc[a][b] = fmaf(av[a], bv[b], acc[a][b]);
-    }
-    __syncthreads();
+    mbar_init(&tail->done, 1);
+    tail->abort_flag = 0;
+    fence_mbar_init();
   }
-  float *out = partials + ((int64_t)chunk * n_groups + k) * G * G;
+  if (warp == 0 && lane == 0) tma_prefetch_desc(&tmX);
+  if (warp == 1) {
+    tmem_alloc(&tail->tmem_base, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tail->tmem_base;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, issued = 0, issued_parity = 0;
+      bool ok = true;
+      for (int step = 0; step < nsteps; ++step) {
+        if (!mbar_wait_bounded(&tail->empty[stage], phase ^ 1u, max_polls, abort_flag)) {
+          dev_fail(st, kDevTimeout, 0x600u + stage);
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&tail->full[stage], GSTAGE_BYTES);
+        const int32_t y = (int32_t)(t0 + (int64_t)step * GT);
+        uint8_t *dst = smem + stage * GSTAGE_BYTES;
+        tma_load_2d(dst, &tmX, &tail->full[stage], k * 128, y);
+        tma_load_2d(dst + GBOX_BYTES, &tmX, &tail->full[stage], k * 128 + 64, y);
+        issued |= 1u << stage;
+        issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+        if (++stage == GSTAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok || *abort_flag)
+        for (int s = 0; s < GSTAGES; ++s)
+          if (issued & (1u << s))
+            (void)mbar_wait_bounded(&tail->full[s], (issued_parity >> s) & 1u, GDRAIN_POLLS, nullptr);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool issued_any = false, ok = true;
+      for (int step = 0; step < nsteps; ++step) {
+        if (!mbar_wait_bounded(&tail->full[stage], phase, max_polls, abort_flag)) {
+          dev_fail(st, kDevTimeout, 0x700u + stage);
+          *abort_flag = 1;
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t base = smem_u32(smem + stage * GSTAGE_BYTES);
 #pragma unroll
-  for (int a = 0; a < 8; ++a) {
-    const int row = (a < 4) ? (4 * ty + a) : (64 + 4 * ty + a - 4);
-    *reinterpret_cast<float4 *>(&out[row * G + 4 * tx]) =
-        make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
-    *reinterpret_cast<float4 *>(&out[row * G + 64 + 4 * tx]) =
-        make_float4(acc[a][4], acc[a][5], acc[a][6], acc[a][7]);
+        for (int ks = 0; ks < GT / 16; ++ks) {
+          const uint64_t d = smem_desc_mn_sw128(base + ks * 2048);  // 16 token rows per step
+          tc_mma_f16(tmem_base, d, d, IDESC_GRAM, (step | ks) != 0 ? 1u : 0u);
+        }
+        issued_any = true;
+        tc_commit(&tail->empty[stage]);
+        if (++stage == GSTAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (issued_any) tc_commit(&tail->done);
+      if (!ok && issued_any) (void)mbar_wait_bounded(&tail->done, 0, GDRAIN_POLLS, nullptr);
+    }
+  } else {
+    const int q = warp & 3;
+    int ok = 1;
+    if (lane == 0) ok = mbar_wait_bounded(&tail->done, 0, max_polls, abort_flag);
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    if (!ok) {
+      if (lane == 0) {
+        dev_fail(st, kDevTimeout, 0x800u);
+        *abort_flag = 1;
+      }
+    } else {
+      tc_fence_after();
+      const int row = q * 32 + lane;
+      float *dst = partials + (((int64_t)chunk * n_groups + k) * 128 + row) * 128;
+#pragma unroll 1
+      for (int c = 0; c < 128; c += 32) {
+        float v[32];
+        tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)c, v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int e = 0; e < 32; e += 4)
+          *reinterpret_cast<float4 *>(dst + c + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 128);
   }
 }
 
@@ -115,17 +210,29 @@ __global__ void gram_reduce_kernel(const float *__restrict__ partials, int n_chu
 }
 
 cudaError_t launch_gram_blocks(const __half *X, int64_t T, int64_t in, int64_t ldx, int group,
-                               int n_chunks, float *partials, float *Gout, cudaStream_t stream) {
+                               int n_chunks, float *partials, float *Gout, DevStatus *st,
+                               uint32_t max_polls, cudaStream_t stream) {
   if (group != G) return cudaErrorInvalidValue;
   const int64_t n_groups = in / G;
-  const int64_t chunk_tokens = (T + n_chunks - 1) / n_chunks;
-  dim3 grid((unsigned)n_groups, (unsigned)n_chunks);
-  gram_blocks_kernel<<<grid, 256, 0, stream>>>(X, T, ldx, chunk_tokens, n_groups, partials);
-  cudaError_t e = cudaGetLastError();
+  // chunks are whole multiples of GT tokens so that no TMA box straddles two
+  // chunks; only the last chunk ends at T (rows past T read as zero)
+  int64_t chunk_tokens = (T + n_chunks - 1) / n_chunks;
+  chunk_tokens = (chunk_tokens + GT - 1) / GT * GT;
+  const int eff_chunks = (int)((T + chunk_tokens - 1) / chunk_tokens);
+  CUtensorMap tm;
+  cudaError_t e = make_tmap_f16_box(&tm, X, T, in, ldx, 64, GT);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(gram_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)kGramSmemBytes);
+  if (e != cudaSuccess) return e;
+  dim3 grid((unsigned)n_groups, (unsigned)eff_chunks);
+  gram_tc_kernel<<<grid, 192, kGramSmemBytes, stream>>>(tm, T, chunk_tokens, n_groups, partials, st,
+                                                        max_polls);
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const int64_t n = n_groups * G * G;
   gram_reduce_kernel<<<(unsigned)i64min(4096, (n + 255) / 256), 256, 0, stream>>>(
-      partials, n_chunks, n, Gout);
+      partials, eff_chunks, n, Gout);
   return cudaGetLastError();
 }
 

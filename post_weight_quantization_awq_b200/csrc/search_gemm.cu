@@ -265,14 +265,14 @@ static EncodeTiledFn get_encode_fn() {
 }
 
 // 2-D fp16 tensor map over a row-major [rows, cols] matrix with row stride
-// `ld` elements, box [box_rows, 64 cols], 128-byte swizzle, zero fill.
-static cudaError_t make_tmap_f16(CUtensorMap *m, const void *base, int64_t rows, int64_t cols,
-                                 int64_t ld, uint32_t box_rows) {
+// `ld` elements, box [box_rows, box_cols], 128-byte swizzle, zero fill.
+cudaError_t make_tmap_f16_box(CUtensorMap *m, const void *base, int64_t rows, int64_t cols,
+                              int64_t ld, uint32_t box_cols, uint32_t box_rows) {
   EncodeTiledFn fn = get_encode_fn();
   if (!fn) return cudaErrorNotSupported;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)(ld * 2)};
-  cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+  cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, const_cast<void *>(base), dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -284,9 +284,9 @@ cudaError_t launch_search_gemm(const __half *X, int64_t ldx, const __half *dW,
                                const SearchGemmShape &sh, double *partials, DevStatus *st,
                                uint32_t max_polls, int num_sms, cudaStream_t stream) {
   CUtensorMap tmA, tmB;
-  cudaError_t e = make_tmap_f16(&tmA, X, sh.T, sh.in, ldx, BM);
+  cudaError_t e = make_tmap_f16_box(&tmA, X, sh.T, sh.in, ldx, BK, BM);
   if (e != cudaSuccess) return e;
-  e = make_tmap_f16(&tmB, dW, sh.rows_b, sh.in, sh.in, BN);
+  e = make_tmap_f16_box(&tmB, dW, sh.rows_b, sh.in, sh.in, BK, BN);
   if (e != cudaSuccess) return e;
   e = cudaFuncSetAttribute(search_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)kGemmSmemBytes);
