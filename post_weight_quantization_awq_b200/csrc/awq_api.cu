@@ -340,7 +340,9 @@ awq_status awq_search_clip(const void *X, int64_t T, int64_t in, int64_t ldx, co
   {
     ProfScope p("clip_eval", cs);
     AWQ_TRY_CUDA(launch_clip_eval(static_cast<const __half *>(W), out, in, s, Gk, cfg->group_size,
-                                  cfg->w_bit, cfg->n_clip, cfg->clip_min, clip_idx, err, cs),
+                                  cfg->w_bit, cfg->n_clip, cfg->clip_min, clip_idx, err,
+                                  reinterpret_cast<DevStatus *>(base), poll_cap(),
+                                  num_sms_current(), cs),
                  "clip_eval launch");
   }
   return AWQ_OK;
@@ -511,7 +513,8 @@ extern "C" awq_status awq_search_clip_noalloc(const void *X, int64_t T, int64_t 
                          gpart, Gk, nullptr, 1u << 24, cs);
   if (e != cudaSuccess) return cuda_fail(e, "gram_blocks launch");
   e = launch_clip_eval(static_cast<const __half *>(W), out, in, s, Gk, cfg->group_size, cfg->w_bit,
-                       cfg->n_clip, cfg->clip_min, clip_idx, err, cs);
+                       cfg->n_clip, cfg->clip_min, clip_idx, err, nullptr, 1u << 24,
+                       num_sms_current(), cs);
   if (e != cudaSuccess) return cuda_fail(e, "clip_eval launch");
   return AWQ_OK;
 }

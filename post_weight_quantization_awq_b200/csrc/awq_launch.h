@@ -56,10 +56,11 @@ cudaError_t launch_mse_argmin(const double *partials, int n_alpha, int nb_per_al
 cudaError_t launch_gram_blocks(const __half *X, int64_t T, int64_t in, int64_t ldx, int group,
                                int n_chunks, float *partials, float *G, DevStatus *st,
                                uint32_t max_polls, cudaStream_t stream);
-// K6b: clip choice per (row, group).
+// K6b: clip choice per (row, group), quadratic forms on the tensor cores.
 cudaError_t launch_clip_eval(const __half *W, int64_t out, int64_t in, const float *s,
                              const float *G, int group, int w_bit, int n_clip, float clip_min,
-                             uint8_t *clip_idx, float *err, cudaStream_t stream);
+                             uint8_t *clip_idx, float *err, DevStatus *st, uint32_t max_polls,
+                             int num_sms, cudaStream_t stream);
 
 // K7: final codes + packing.
 cudaError_t launch_quant_pack(const __half *W, int64_t out, int64_t in, const float *s,

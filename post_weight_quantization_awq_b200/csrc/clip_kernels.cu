@@ -10,11 +10,8 @@
 //   K6a  gram_tc: tensor-core block Grams over token chunks, one CTA per
 //        (group, chunk); chunk partials are summed in a fixed order by
 //        gram_reduce, so G is bitwise reproducible.
-//   K6b  clip_eval: one block per (group, 16 rows) holds G_k in shared memory;
-//        a warp quantises one row for a batch of clip ratios, writes the error
-//        vectors to shared memory and evaluates y = G_k d for the whole batch
-//        (each G element read once per batch), then E = d . y by warp
-//        shuffles; the first c with the smallest E wins.
+//   K6b  clip_tc: tensor-core quadratic forms, one CTA per (group, share of
+//        the rows); the first c with the smallest E wins.
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <math.h>
@@ -25,10 +22,6 @@ namespace awq {
 
 namespace {
 constexpr int G = 128;          // group size handled by these kernels
-constexpr int CLIP_ROWS = 16;   // rows per clip_eval block
-constexpr int CLIP_WARPS = 4;
-constexpr int CLIP_CB = 10;     // clip ratios per batch
-constexpr int GSTRIDE = G + 4;  // shared-memory row stride of G_k (floats)
 }  // namespace
 
 // ---------------------------------------------------------------------------
@@ -237,127 +230,339 @@ cudaError_t launch_gram_blocks(const __half *X, int64_t T, int64_t in, int64_t l
 }
 
 // ---------------------------------------------------------------------------
-// K6b
+// K6b — clip scoring on the tensor cores.
+//
+// With r_i = sqrt(G_ii), G~ = diag(r)^-1 G diag(r)^-1 (|G~_ij| <= 1, zero
+// where r vanishes) and d~ = diag(r) d (d = deq_c/s - w of one (row, group,
+// clip) candidate), E = d^T G d = d~^T G~ d~.  A CTA owns one group k: it
+// builds G~ once in shared memory as two fp16 parts (hi + lo, 22 significant
+// bits) and then walks tiles of 128 candidates = R rows x n_clip ratios.  For
+// each tile its threads quantise the candidates and write d~ (scaled by a
+// per-row power of two to sit inside fp16) as hi + lo parts into a K-major
+// 128-byte-swizzled tile; one thread issues
+//     Y = A_hi G~_hi + A_lo G~_hi + A_hi G~_lo
+// as tcgen05.mma kind::f16 (M = 128 candidates, N = 128, K = 128) into fp32
+// TMEM, and every thread dots its candidate's row of Y with its own d~, so no
+// cross-thread reduction is needed.  The dropped A_lo G~_lo term is 2^-22 of E.
 // ---------------------------------------------------------------------------
+namespace {
+constexpr int CT_THREADS = 512;
+constexpr int CT_MAXR = 32;                       // rows per tile at most
+constexpr uint32_t CT_ATOM = 128 * 128;           // bytes: 128 rows x 64 fp16
+constexpr uint32_t CT_OPND = 2 * CT_ATOM;         // one operand, K = 128
+constexpr int CT_RS = G + G / 32;                 // skewed row stride (floats)
+// kind::f16, fp16 A/B, fp32 D, K-major, N = 128, M = 128
+constexpr uint32_t IDESC_CLIP = (1u << 4) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+
+struct __align__(16) ClipSmem {
+  uint8_t a_hi[CT_OPND];
+  uint8_t a_lo[CT_OPND];
+  uint8_t b_hi[CT_OPND];
+  uint8_t b_lo[CT_OPND];
+  float wt[CT_MAXR][CT_RS];   // s_i w_i of the tile's rows (fp32, exact products)
+  float bw[CT_MAXR][CT_RS];   // r_i w_i 2^e_row
+  float s[G], ar[CT_RS], r[G];  // s_i, r_i / s_i (skewed), r_i = sqrt(G_ii)
+  float rmx[CT_MAXR], rmn[CT_MAXR];
+  int rexp[CT_MAXR];
+  float epart[4][128];
+  uint64_t mma_bar;
+  uint32_t tmem_base;
+  int abort_flag;  // a wait ran out: every thread leaves the tile loop together
+};
+constexpr size_t kClipSmemBytes = sizeof(ClipSmem) + 1024;
+
+// channel i of a skewed row: one extra float every 32 channels, so the four
+// threads that share a candidate (32 channels apart) hit different banks
+__device__ __forceinline__ int sk(int i) { return i + (i >> 5); }
+
+// byte offset of 16-byte chunk `c` (0..7) of row `row` inside a K-major
+// 128-byte-swizzled atom (8-row core groups of 1024 bytes)
+__device__ __forceinline__ uint32_t sw128_off(int row, int c) {
+  return (uint32_t)row * 128u + (uint32_t)((c ^ (row & 7)) << 4);
+}
+
+__device__ __forceinline__ void split_store8(uint8_t *hi, uint8_t *lo, uint32_t off, const float *v) {
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const __half2 hv = __floats2half2_rn(v[2 * e], v[2 * e + 1]);
+    const float2 hf = __half22float2(hv);
+    const __half2 lv = __floats2half2_rn(v[2 * e] - hf.x, v[2 * e + 1] - hf.y);
+    h[e] = *reinterpret_cast<const uint32_t *>(&hv);
+    l[e] = *reinterpret_cast<const uint32_t *>(&lv);
+  }
+  *reinterpret_cast<uint4 *>(hi + off) = make_uint4(h[0], h[1], h[2], h[3]);
+  *reinterpret_cast<uint4 *>(lo + off) = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __device__ __forceinline__ float clip_ratio_f(int c, int n_clip, float clip_min) {
   if (n_clip <= 1) return 1.0f;
   double r = 1.0 - (double)c * (1.0 - (double)clip_min) / (double)(n_clip - 1);
   return __double2float_rn(r);
 }
+}  // namespace
 
-__global__ void __launch_bounds__(CLIP_WARPS * 32) clip_eval_kernel(
+__global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
     const __half *__restrict__ W, int64_t out, int64_t in, const float *__restrict__ s,
-    const float *__restrict__ Gall, float qmax, int n_clip, float clip_min,
-    uint8_t *__restrict__ clip_idx, float *__restrict__ err) {
-  extern __shared__ __align__(16) float csm[];
-  float *Gs = csm;                                  // [G][GSTRIDE]
-  float *dsh = csm + G * GSTRIDE;                   // [warps][CLIP_CB][G]
-  const int k = blockIdx.x;
-  const int64_t o_base = (int64_t)blockIdx.y * CLIP_ROWS;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const float *__restrict__ Gall, float qmax, int n_clip, float clip_min, int rows_per_tile,
+    uint8_t *__restrict__ clip_idx, float *__restrict__ err, DevStatus *st, uint32_t max_polls) {
+  extern __shared__ uint8_t csm_raw[];
+  ClipSmem &S = *reinterpret_cast<ClipSmem *>(
+      (reinterpret_cast<uintptr_t>(csm_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t n_groups = in / G;
-  const float *Gk = Gall + (int64_t)k * G * G;
-  for (int i = threadIdx.x; i < G * G / 4; i += blockDim.x) {
-    const int r = (4 * i) / G, c = (4 * i) % G;
-    *reinterpret_cast<float4 *>(&Gs[r * GSTRIDE + c]) = __ldg(reinterpret_cast<const float4 *>(Gk) + i);
-  }
-  __syncthreads();
-  float *dw = dsh + warp * CLIP_CB * G;
-  // lane owns channels j = lane + 32 jj (jj = 0..3) of the group
-  float sv[4];
-#pragma unroll
-  for (int jj = 0; jj < 4; ++jj) sv[jj] = s ? s[(int64_t)k * G + lane + 32 * jj] : 1.0f;
+  const int R = rows_per_tile;
+  const int npairs = R * n_clip;  // <= 128
+  const int64_t n_tiles = (out + R - 1) / R;
+  // this CTA's share of the (group, row tile) items, group-major, so a CTA
+  // meets at most a few groups and builds each G~ once
+  const int64_t n_items = n_groups * n_tiles;
+  const int64_t item_begin = n_items * blockIdx.x / gridDim.x;
+  const int64_t item_end = n_items * (blockIdx.x + 1) / gridDim.x;
 
-  for (int r = warp; r < CLIP_ROWS; r += CLIP_WARPS) {
-    const int64_t o = o_base + r;
-    if (o >= out) break;
-    float w[4], wt[4];
-    float mx = -INFINITY, mn = INFINITY;
+  if (tid == 0) {
+    mbar_init(&S.mma_bar, 1);
+    S.abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&S.tmem_base, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = S.tmem_base;
+
+  uint32_t phase = 0;
+  bool committed = false;
+  int64_t k_cur = -1;
+  for (int64_t item = item_begin; item < item_end; ++item) {
+    const int64_t k = item / n_tiles;
+    const int64_t o0 = (item - k * n_tiles) * R;
+    if (k != k_cur) {
+      // ---- group set-up: s, r = sqrt(G_ii), r/s, then G~ = G_ij / (r_i r_j)
+      // as hi + lo fp16, K-major swizzled (row j, channel i)
+      k_cur = k;
+      const float *Gk = Gall + k * G * G;
+      if (tid < G) {
+        const float sv = s ? s[k * G + tid] : 1.0f;
+        const float rv = sqrtf(fmaxf(Gk[tid * G + tid], 0.0f));
+        S.s[tid] = sv;
+        S.r[tid] = rv;
+        S.ar[sk(tid)] = rv / sv;
+      }
+      __syncthreads();
+      const int j = tid >> 2, qq = tid & 3;  // row j, channels 32 qq .. 32 qq + 31
+      const float rj = S.r[j];
+      const float *grow = Gk + (int64_t)j * G + 32 * qq;
+#pragma unroll 1
+      for (int c = 0; c < 4; ++c) {
+        float v[8];
+        const float4 g0 = __ldg(reinterpret_cast<const float4 *>(grow + 8 * c));
+        const float4 g1 = __ldg(reinterpret_cast<const float4 *>(grow + 8 * c + 4));
+        const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
 #pragma unroll
-    for (int jj = 0; jj < 4; ++jj) {
-      w[jj] = __half2float(W[o * in + (int64_t)k * G + lane + 32 * jj]);
-      wt[jj] = __fmul_rn(sv[jj], w[jj]);
-      mx = fmaxf(mx, wt[jj]);
-      mn = fminf(mn, wt[jj]);
+        for (int e = 0; e < 8; ++e) {
+          const float den = rj * S.r[32 * qq + 8 * c + e];
+          v[e] = den > 0.0f ? gv[e] / den : 0.0f;
+        }
+        const int h = qq >> 1, cc = (qq & 1) * 4 + c;
+        split_store8(S.b_hi + h * CT_ATOM, S.b_lo + h * CT_ATOM, sw128_off(j, cc), v);
+      }
+      // (the fence before the first MMA of this group publishes these stores)
     }
+    // ---- rows of this tile: s w, range, exponent of the d~ scaling, r w 2^e
+    for (int rr = warp; rr < R; rr += CT_THREADS / 32) {
+      const int64_t o = o0 + rr;
+      float w4[4] = {0.f, 0.f, 0.f, 0.f};
+      if (o < out) {
+        const uint2 wv = __ldg(reinterpret_cast<const uint2 *>(W + o * in + k * G + 4 * lane));
+        const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&wv.x));
+        const float2 b = __half22float2(*reinterpret_cast<const __half2 *>(&wv.y));
+        w4[0] = a.x; w4[1] = a.y; w4[2] = b.x; w4[3] = b.y;
+      }
+      float mx = -INFINITY, mn = INFINITY, bmax = 0.0f, wt4[4];
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+      for (int e = 0; e < 4; ++e) {
+        const int i = 4 * lane + e;
+        wt4[e] = __fmul_rn(S.s[i], w4[e]);
+        mx = fmaxf(mx, wt4[e]);
+        mn = fminf(mn, wt4[e]);
+        bmax = fmaxf(bmax, S.r[i] * fabsf(w4[e]));
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+        bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, off));
+      }
+      // |d~_i| <= 2 r_i |w_i| (+ rounding): keep 2 bmax 2^e <= 2^14
+      int e2 = 0;
+      if (bmax > 0.0f) {
+        (void)frexpf(2.0f * bmax, &e2);
+        e2 = 14 - e2;
+      }
+      const float sc = ldexpf(1.0f, e2);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = 4 * lane + e;
+        S.wt[rr][sk(i)] = wt4[e];
+        S.bw[rr][sk(i)] = (S.r[i] * w4[e]) * sc;
+      }
+      if (lane == 0) {
+        S.rmx[rr] = mx;
+        S.rmn[rr] = mn;
+        S.rexp[rr] = e2;
+      }
     }
-    float best_e = INFINITY;
-    int best_c = 0;
-    for (int c0 = 0; c0 < n_clip; c0 += CLIP_CB) {
-      const int nb = min(CLIP_CB, n_clip - c0);
-      // error vectors of this batch -> shared memory
-      for (int cc = 0; cc < nb; ++cc) {
-        const GroupQ g = group_params(mx, mn, clip_ratio_f(c0 + cc, n_clip, clip_min), qmax);
+    __syncthreads();
+    // ---- candidates: thread (pair p, quarter qq) writes channels 32qq..32qq+31:
+    // d~_i 2^e = (q - z) (delta 2^e) (r_i / s_i) - r_i w_i 2^e
+    {
+      const int p = tid >> 2, qq = tid & 3;
+      const int rr = p / n_clip, c = p - rr * n_clip;
+      const bool valid = p < npairs && o0 + rr < out;
+      const int h = qq >> 1;
+      uint8_t *ahi = S.a_hi + h * CT_ATOM, *alo = S.a_lo + h * CT_ATOM;
+      if (valid) {
+        const GroupQ g = group_params(S.rmx[rr], S.rmn[rr], clip_ratio_f(c, n_clip, clip_min), qmax);
+        const float de = ldexpf(g.delta, S.rexp[rr]);  // exact power-of-two scaling
+        const float *wtr = S.wt[rr];
+        const float *bwr = S.bw[rr];
+#pragma unroll 1
+        for (int c4 = 0; c4 < 4; ++c4) {
+          float v[8];
+          const int i0 = 32 * qq + 8 * c4;
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-          const float deq = dequant(quant_code(wt[jj], g), g);
-          dw[cc * G + lane + 32 * jj] = __fsub_rn(__fdiv_rn(deq, sv[jj]), w[jj]);
+          for (int e = 0; e < 8; ++e) {
+            const int i = sk(i0 + e);
+            const float qz = __fsub_rn(quant_code(wtr[i], g), g.zero);
+            v[e] = fmaf(__fmul_rn(qz, de), S.ar[i], -bwr[i]);
+          }
+          split_store8(ahi, alo, sw128_off(p, (qq & 1) * 4 + c4), v);
+        }
+      } else {
+        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          *reinterpret_cast<uint4 *>(ahi + sw128_off(p, (qq & 1) * 4 + c4)) = z;
+          *reinterpret_cast<uint4 *>(alo + sw128_off(p, (qq & 1) * 4 + c4)) = z;
         }
       }
-      __syncwarp();
-      float y[4][CLIP_CB];
+    }
+    fence_async_smem();  // generic-proxy writes -> visible to the tensor cores
+    __syncthreads();
+    // ---- Y = A_hi B_hi + A_lo B_hi + A_hi B_lo
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t a_hi = smem_u32(S.a_hi), a_lo = smem_u32(S.a_lo);
+      const uint32_t b_hi = smem_u32(S.b_hi), b_lo = smem_u32(S.b_lo);
+      const uint32_t as[3] = {a_hi, a_lo, a_hi}, bs[3] = {b_hi, b_hi, b_lo};
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj)
+      for (int t = 0; t < 3; ++t)
 #pragma unroll
-        for (int cc = 0; cc < CLIP_CB; ++cc) y[jj][cc] = 0.0f;
-#pragma unroll 2
-      for (int i = 0; i < G; i += 4) {
-        float4 gr[4];
+        for (int ks = 0; ks < 8; ++ks) {
+          const uint32_t koff = (uint32_t)(ks >> 2) * CT_ATOM + (uint32_t)(ks & 3) * 32u;
+          tc_mma_f16(tmem_base, smem_desc_k_sw128(as[t] + koff), smem_desc_k_sw128(bs[t] + koff),
+                     IDESC_CLIP, (t | ks) != 0 ? 1u : 0u);
+        }
+      tc_commit(&S.mma_bar);
+    }
+    committed = true;
+    // ---- wait for Y, then E = d~ . y per candidate (warp: lane quarter q,
+    // column quarter cq)
+    int okw = 1;
+    if (lane == 0) okw = mbar_wait_bounded(&S.mma_bar, phase, max_polls, nullptr);
+    okw = __shfl_sync(0xffffffffu, okw, 0);
+    phase ^= 1u;
+    if (!okw) {
+      if (lane == 0) {
+        dev_fail(st, kDevTimeout, 0x900u);
+        *reinterpret_cast<volatile int *>(&S.abort_flag) = 1;
+      }
+    } else {
+      tc_fence_after();
+      const int q = warp & 3, cq = warp >> 2;
+      const int p = q * 32 + lane;
+      const uint8_t *ahi = S.a_hi + (cq >> 1) * CT_ATOM, *alo = S.a_lo + (cq >> 1) * CT_ATOM;
+      float y[32];
+      tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(32 * cq), y);
+      tmem_ld_wait();
+      float e = 0.0f;
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj)
-          gr[jj] = *reinterpret_cast<const float4 *>(&Gs[(lane + 32 * jj) * GSTRIDE + i]);
+      for (int cc = 0; cc < 4; ++cc) {
+        const int c = (cq & 1) * 4 + cc;
+        const uint4 hv = *reinterpret_cast<const uint4 *>(ahi + sw128_off(p, c));
+        const uint4 lv = *reinterpret_cast<const uint4 *>(alo + sw128_off(p, c));
+        const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w}, lw[4] = {lv.x, lv.y, lv.z, lv.w};
 #pragma unroll
-        for (int cc = 0; cc < CLIP_CB; ++cc) {
-          if (cc < nb) {
-            const float4 d = *reinterpret_cast<const float4 *>(&dw[cc * G + i]);
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-              float acc = y[jj][cc];
-              acc = fmaf(gr[jj].x, d.x, acc);
-              acc = fmaf(gr[jj].y, d.y, acc);
-              acc = fmaf(gr[jj].z, d.z, acc);
-              acc = fmaf(gr[jj].w, d.w, acc);
-              y[jj][cc] = acc;
-            }
+        for (int e2 = 0; e2 < 4; ++e2) {
+          const float2 fh = __half22float2(*reinterpret_cast<const __half2 *>(&hw[e2]));
+          const float2 fl = __half22float2(*reinterpret_cast<const __half2 *>(&lw[e2]));
+          e = fmaf(fh.x + fl.x, y[8 * cc + 2 * e2], e);
+          e = fmaf(fh.y + fl.y, y[8 * cc + 2 * e2 + 1], e);
+        }
+      }
+      S.epart[cq][p] = e;
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (*reinterpret_cast<volatile int *>(&S.abort_flag)) break;  // uniform across the CTA
+    // ---- per row: first clip index with the smallest E
+    if (tid < R) {
+      const int64_t o = o0 + tid;
+      if (o < out) {
+        const float unscale = ldexpf(1.0f, -2 * S.rexp[tid]);
+        float best = INFINITY;
+        int bc = 0;
+        for (int c = 0; c < n_clip; ++c) {
+          const int p = tid * n_clip + c;
+          const float ev =
+              ((S.epart[0][p] + S.epart[1][p]) + (S.epart[2][p] + S.epart[3][p])) * unscale;
+          if (err) err[(o * n_groups + k) * n_clip + c] = ev;
+          if (ev < best) {
+            best = ev;
+            bc = c;
           }
         }
+        clip_idx[o * n_groups + k] = (uint8_t)bc;
       }
-#pragma unroll
-      for (int cc = 0; cc < CLIP_CB; ++cc) {
-        if (cc < nb) {
-          float e = 0.0f;
-#pragma unroll
-          for (int jj = 0; jj < 4; ++jj) e = fmaf(dw[cc * G + lane + 32 * jj], y[jj][cc], e);
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) e += __shfl_xor_sync(0xffffffffu, e, off);
-          if (err && lane == 0) err[(o * n_groups + k) * n_clip + c0 + cc] = e;
-          if (e < best_e) {
-            best_e = e;
-            best_c = c0 + cc;
-          }
-        }
-      }
-      __syncwarp();
     }
-    if (lane == 0) clip_idx[o * n_groups + k] = (uint8_t)best_c;
+    __syncthreads();
+  }
+  // after an abort the last MMAs may still be running: let them finish
+  // (bounded) before the accumulator is freed
+  if (tid == 0 && committed && *reinterpret_cast<volatile int *>(&S.abort_flag))
+    (void)mbar_wait_bounded(&S.mma_bar, phase ^ 1u, 1u << 22, nullptr);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, 128);
   }
 }
 
 cudaError_t launch_clip_eval(const __half *W, int64_t out, int64_t in, const float *s,
                              const float *Gall, int group, int w_bit, int n_clip, float clip_min,
-                             uint8_t *clip_idx, float *err, cudaStream_t stream) {
-  if (group != G) return cudaErrorInvalidValue;
-  const size_t smem = sizeof(float) * ((size_t)G * GSTRIDE + (size_t)CLIP_WARPS * CLIP_CB * G);
-  cudaError_t e = cudaFuncSetAttribute(clip_eval_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+                             uint8_t *clip_idx, float *err, DevStatus *st, uint32_t max_polls,
+                             int num_sms, cudaStream_t stream) {
+  if (group != G || n_clip < 1 || n_clip > 128) return cudaErrorInvalidValue;
+  int R = 128 / n_clip;
+  if (R > CT_MAXR) R = CT_MAXR;
+  const int64_t n_items = (in / G) * ((out + R - 1) / R);
+  const int64_t ctas = i64min(num_sms, n_items);  // one CTA per SM (shared memory bound)
+  cudaError_t e = cudaFuncSetAttribute(clip_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kClipSmemBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)(in / G), (unsigned)((out + CLIP_ROWS - 1) / CLIP_ROWS));
-  clip_eval_kernel<<<grid, CLIP_WARPS * 32, smem, stream>>>(
-      W, out, in, s, Gall, (float)((1 << w_bit) - 1), n_clip, clip_min, clip_idx, err);
+  dim3 grid((unsigned)ctas);
+  clip_tc_kernel<<<grid, CT_THREADS, kClipSmemBytes, stream>>>(
+      W, out, in, s, Gall, (float)((1 << w_bit) - 1), n_clip, clip_min, R, clip_idx, err, st,
+      max_polls);
   return cudaGetLastError();
 }
 
