@@ -76,11 +76,13 @@ def init_dist(backend: str, world: int):
     return dist if world > 1 else None
 
 
-def max_over_ranks(value: float, dist, device="cpu") -> float:
-    """Max of a per-rank float over all ranks (identity on one rank)."""
+def max_over_ranks(value: float, dist) -> float:
+    """Max of a per-rank float over all ranks (identity on one rank).  The
+    scalar travels on the device the process group's backend uses."""
     if dist is None:
         return value
     import torch
+    device = "cuda" if dist.get_backend() == "nccl" else "cpu"
     t = torch.tensor([value], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
@@ -92,6 +94,41 @@ def barrier(dist, device=None):
             dist.barrier(device_ids=[device])
         else:
             dist.barrier()
+
+
+class CudaTimer:
+    """CUDA events on the stream the work is launched on."""
+
+    def __init__(self, torch, stream, device):
+        self.torch, self.stream, self.device = torch, stream, device
+        self.e0 = torch.cuda.Event(enable_timing=True)
+        self.e1 = torch.cuda.Event(enable_timing=True)
+
+    def sync(self):
+        self.torch.cuda.synchronize(self.device)
+
+    def start(self):
+        self.e0.record(self.stream)
+
+    def stop(self):
+        self.e1.record(self.stream)
+
+    def elapsed_ms(self):
+        return self.e0.elapsed_time(self.e1)
+
+
+def timed_steps(step, steps: int, dist, timer, barrier_device=None) -> float:
+    """Times exactly `steps` calls of `step` between a barrier + device sync on
+    both sides; returns the max over ranks of ms per step."""
+    barrier(dist, barrier_device)
+    timer.sync()
+    timer.start()
+    for _ in range(steps):
+        step()
+    timer.stop()
+    timer.sync()
+    barrier(dist, barrier_device)
+    return max_over_ranks(timer.elapsed_ms() / steps, dist)
 
 
 # ---------------------------------------------------------------- clocks
@@ -264,19 +301,11 @@ def run_awq(args):
     torch.cuda.synchronize(dev)
     awq.profile_reset()
     awq.profile_enable(True)
-    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    timer = CudaTimer(torch, stream, dev)
     with ClockSampler(local) as clk:
-        barrier(dist, local)
-        torch.cuda.synchronize(dev)
-        ev0.record(stream)
-        for _ in range(args.steps):
-            res = step()
-        ev1.record(stream)
-        torch.cuda.synchronize(dev)
-        barrier(dist, local)
+        ms_step = timed_steps(step, args.steps, dist, timer, local)
     awq.profile_enable(False)
     awq.awq_device_status(ws)
-    ms_step = max_over_ranks(ev0.elapsed_time(ev1) / args.steps, dist, dev)
     kern = {}
     for name in KERNELS_PER_STEP:
         tot, n = awq.profile_read(name)
@@ -309,15 +338,7 @@ def run_awq(args):
         e2e_step()
     torch.cuda.synchronize(dev)
     e_steps = max(1, min(args.steps, 5))
-    barrier(dist, local)
-    torch.cuda.synchronize(dev)
-    ev0.record(stream)
-    for _ in range(e_steps):
-        e2e_step()
-    ev1.record(stream)
-    torch.cuda.synchronize(dev)
-    barrier(dist, local)
-    ms_e2e = max_over_ranks(ev0.elapsed_time(ev1) / e_steps, dist, dev)
+    ms_e2e = timed_steps(e2e_step, e_steps, dist, timer, local)
     h2d = X.numel() * 2 + W.numel() * 2
     d2h = sum(h.numel() * h.element_size() for h in host_out.values())
 

@@ -253,3 +253,33 @@ def test_full_attention_int3_workload_sampled_rows():
     _, X, W = d["groups"][0]
     rows = np.sort(np.random.default_rng(0).choice(W.shape[0], 512, replace=False))
     _layer_parity(X, W, 3, 20, 20, rows=torch.from_numpy(rows))
+
+
+# ------------------------------------------------------------------ K8
+@pytest.mark.parametrize("rows,cols", [(4096, 1), (5120, 1), (4096, 4096), (136, 24)])
+def test_fold_inv_scale_bitwise(rows, cols):
+    """Folding 1/s into the preceding norm's gamma (cols = 1) or the preceding
+    linear's rows: RN16(RN32(v) / s), bit-exact."""
+    rng = np.random.default_rng(rows + cols)
+    v = rng.normal(0, 0.05 if cols > 1 else 1.0, (rows, cols)).astype(np.float16)
+    s = O.scale_grid(np.exp(rng.normal(0, 1.5, rows)), O.alpha_grid(20))[13]
+    vd = torch.from_numpy(v).cuda()
+    awq.awq_fold_inv_scale(vd, torch.from_numpy(s).cuda())
+    torch.cuda.synchronize()
+    want = O.fold_inv_scale(v[:, 0] if cols == 1 else v, s)
+    got = vd.cpu().numpy()
+    got = got[:, 0] if cols == 1 else got
+    assert np.array_equal(got.view(np.uint16), want.view(np.uint16))
+
+
+def test_mlp_workload_sampled():
+    """The Llama-7B-shaped MLP workload: gate|up [22016 x 4096] scaled jointly
+    on the full X (512 sampled output rows); down_proj [4096 x 11008] on its
+    SwiGLU input (a 8192-token sample, 512 sampled rows)."""
+    d = workload_inputs(2, device="cuda")
+    (_, X, Wgu), (_, Xd, Wd) = d["groups"]
+    rng = np.random.default_rng(2)
+    rows = torch.from_numpy(np.sort(rng.choice(Wgu.shape[0], 512, replace=False)))
+    _layer_parity(X, Wgu, 4, 20, 0, rows=rows)
+    rows_d = torch.from_numpy(np.sort(rng.choice(Wd.shape[0], 512, replace=False)))
+    _layer_parity(Xd[:8192].contiguous(), Wd, 4, 20, 0, rows=rows_d)

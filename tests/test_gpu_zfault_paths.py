@@ -1,0 +1,56 @@
+"""Device-side failure detection without a GPU fault: with AWQ_FAULT=timeout
+every bounded wait inside the tensor-core kernels gives up after one poll.
+The kernels then record AWQ_ERR_TIMEOUT in the workspace status word, let
+their in-flight copies and MMAs finish, free their tensor memory and return;
+the context stays usable and the next call is correct."""
+
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import post_weight_quantization_awq_b200 as awq
+from oracle import awq_oracle as O
+from synthetic import random_layer
+
+from gpu_helpers import check_mse, need_cuda
+
+pytestmark = pytest.mark.gpu
+
+
+def _search(X, W, cfg, ws):
+    abar = torch.empty(X.shape[1], dtype=torch.float64, device="cuda")
+    mse = torch.empty(cfg.n_alpha, dtype=torch.float64, device="cuda")
+    best = torch.empty(1, dtype=torch.int32, device="cuda")
+    s_best = torch.empty(X.shape[1], dtype=torch.float32, device="cuda")
+    awq.awq_act_stats(X, abar)
+    awq.awq_search_scale(X, W, abar, cfg, ws, s_best, mse, best)
+    return mse, s_best
+
+
+def test_bounded_waits_report_timeout_and_leave_the_context_usable(monkeypatch):
+    need_cuda()
+    X, W = random_layer(1500, 512, 512, seed=21)
+    Xd, Wd = X.cuda(), W.cuda()
+    cfg = awq.AwqConfig.make(n_clip=20)
+    ws = awq.alloc_workspace(1500, 512, 512, cfg)
+    idx = torch.empty((512, 4), dtype=torch.uint8, device="cuda")
+    monkeypatch.setenv("AWQ_FAULT", "timeout")
+    _search(Xd, Wd, cfg, ws)
+    with pytest.raises(awq.AwqError) as ei:
+        awq.awq_device_status(ws)
+    assert ei.value.status_name == "AWQ_ERR_TIMEOUT"
+    awq.awq_search_clip(Xd, Wd, None, cfg, ws, idx)
+    with pytest.raises(awq.AwqError) as ei:
+        awq.awq_device_status(ws)
+    assert ei.value.status_name == "AWQ_ERR_TIMEOUT"
+    monkeypatch.delenv("AWQ_FAULT")
+    # the same calls now complete and match the oracle
+    mse, _ = _search(Xd, Wd, cfg, ws)
+    awq.awq_device_status(ws)
+    Xn, Wn = X.numpy(), W.numpy()
+    mse_o, _, _, _ = O.search_scale(Xn, Wn, O.act_stats(Xn), 4, 128, 20)
+    check_mse(mse.cpu().numpy(), mse_o)
+    awq.awq_search_clip(Xd, Wd, None, cfg, ws, idx)
+    awq.awq_device_status(ws)
