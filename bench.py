@@ -378,6 +378,7 @@ def run_awq(args):
         "candidate_gemm_tflops": round(tflops, 1),
         "roofline": {"kernel": "search_gemm", "bound": "tensor", "achieved": round(tflops, 1),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(tflops / peak, 3),
+                     "frac_of_burst_peak": round(tflops / float(peaks["bf16_tflops"]), 3),
                      "traffic": NCU_TRAFFIC_BYTES,
                      "peak_source": f"{src} bf16 dense {'sustained' if 'bf16_tflops_sustained' in peaks else 'burst'} "
                                     "(fp16 has the same nominal rate)",
