@@ -42,9 +42,29 @@ struct GroupQ {
   float delta;    // step
   float zero;     // zero point (integer valued)
   float qmax;     // 2^b - 1
-  float rcp;      // RN(1/delta), used for the fast code path
-  float half_lo;  // delta * (0.5 - 2^-16): remainders below it prove the fast code exact
+  float rcp;      // approximate 1/delta: only proposes codes, never decides them
+  float half_lo;  // delta * (0.5 - 2^-16): remainders below it prove a code exact
 };
+
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+
+// rne(RN32(x / delta)) without a division on the common path.  k = rne of
+// the approximate quotient x * rcp; the remainder x - k*delta comes from one
+// FMA (a single rounding).  If |remainder| < delta (0.5 - 2^-16) and |k| < 64,
+// then |x/delta - k| < 0.5 - 2^-16 + 2^-22, and the fp32 rounding of x/delta
+// moves it by at most 2^-24 * 64.5 < 2^-17, so RN32(x/delta) is strictly within
+// 0.5 of k and rounds to k -- however k was proposed.  Otherwise the correctly
+// rounded quotient decides.
+__device__ __forceinline__ float round_quotient(float x, float delta, float rcp, float half_lo) {
+  const float k = rintf(__fmul_rn(x, rcp));
+  const float rem = fmaf(-k, delta, x);
+  if (fabsf(rem) < half_lo && fabsf(k) < 64.0f) return k;
+  return rintf(__fdiv_rn(x, delta));
+}
 
 // Range of one group after the optional clip ratio r32 (1 = no clip).
 __device__ __forceinline__ GroupQ group_params(float mx, float mn, float r32, float qmax) {
@@ -52,29 +72,37 @@ __device__ __forceinline__ GroupQ group_params(float mx, float mn, float r32, fl
     mx = __fmul_rn(r32, mx);
     mn = __fmul_rn(r32, mn);
   }
-  float d = fmaxf(__fsub_rn(mx, mn), 1e-5f);
+  const float d = fmaxf(__fsub_rn(mx, mn), 1e-5f);
   GroupQ g;
   g.delta = __fdiv_rn(d, qmax);
-  float z = rintf(__fdiv_rn(-mn, g.delta));
+  g.rcp = rcp_approx(g.delta);
+  g.half_lo = __fmul_rn(g.delta, 0.4999847412109375f /* 0.5 - 2^-16 */);
+  const float z = round_quotient(-mn, g.delta, g.rcp, g.half_lo);
   g.zero = fminf(fmaxf(z, 0.0f), qmax);
   g.qmax = qmax;
-  g.rcp = __frcp_rn(g.delta);
-  g.half_lo = __fmul_rn(g.delta, 0.4999847412109375f /* 0.5 - 2^-16 */);
   return g;
 }
 
-// rne(RN32(wt / delta)) without a division on the common path.  k = rne of
-// the approximate quotient wt * RN(1/delta); the remainder wt - k*delta comes
-// from one FMA (a single rounding).  If |remainder| < delta (0.5 - 2^-16) and
-// |k| < 64, then |wt/delta - k| < 0.5 - 2^-16 + 2^-22, and the fp32 rounding of
-// wt/delta moves it by at most 2^-24 * 64.5 < 2^-17, so RN32(wt/delta) is
-// strictly within 0.5 of k and rounds to k.  Otherwise the correctly rounded
-// quotient decides.
 __device__ __forceinline__ float round_quotient(float wt, const GroupQ &g) {
-  const float k = rintf(__fmul_rn(wt, g.rcp));
-  const float rem = fmaf(-k, g.delta, wt);
-  if (fabsf(rem) < g.half_lo && fabsf(k) < 64.0f) return k;
-  return rintf(__fdiv_rn(wt, g.delta));
+  return round_quotient(wt, g.delta, g.rcp, g.half_lo);
+}
+
+// (q - z) for two elements of one group, with Blackwell's packed fp32x2
+// arithmetic (each lane correctly rounded, so the values are those of the
+// scalar path): the same proven fast path, and the exact scalar path for both
+// elements whenever either fails the remainder test.
+__device__ __forceinline__ float2 quant_qz2(float2 wt, const GroupQ &g) {
+  const float2 y = __fmul2_rn(wt, make_float2(g.rcp, g.rcp));
+  float2 k = make_float2(rintf(y.x), rintf(y.y));
+  const float2 rem = __ffma2_rn(make_float2(-k.x, -k.y), make_float2(g.delta, g.delta), wt);
+  if (!(fmaxf(fabsf(rem.x), fabsf(rem.y)) < g.half_lo && fmaxf(fabsf(k.x), fabsf(k.y)) < 64.0f)) {
+    k.x = rintf(__fdiv_rn(wt.x, g.delta));
+    k.y = rintf(__fdiv_rn(wt.y, g.delta));
+  }
+  float2 q = __fadd2_rn(k, make_float2(g.zero, g.zero));
+  q.x = fminf(fmaxf(q.x, 0.0f), g.qmax);
+  q.y = fminf(fmaxf(q.y, 0.0f), g.qmax);
+  return __fadd2_rn(q, make_float2(-g.zero, -g.zero));
 }
 
 __device__ __forceinline__ float quant_code(float wt, const GroupQ &g) {

@@ -439,10 +439,14 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
           float v[8];
           const int i0 = 32 * qq + 8 * c4;
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int i = sk(i0 + e);
-            const float qz = __fsub_rn(quant_code(wtr[i], g), g.zero);
-            v[e] = fmaf(__fmul_rn(qz, de), S.ar[i], -bwr[i]);
+          for (int e = 0; e < 8; e += 2) {
+            const int i = sk(i0 + e);  // i0 + e and i0 + e + 1 stay in one 32-channel run
+            const float2 qz = quant_qz2(make_float2(wtr[i], wtr[i + 1]), g);
+            const float2 d2 = __ffma2_rn(__fmul2_rn(qz, make_float2(de, de)),
+                                         make_float2(S.ar[i], S.ar[i + 1]),
+                                         make_float2(-bwr[i], -bwr[i + 1]));
+            v[e] = d2.x;
+            v[e + 1] = d2.y;
           }
           split_store8(ahi, alo, sw128_off(p, (qq & 1) * 4 + c4), v);
         }

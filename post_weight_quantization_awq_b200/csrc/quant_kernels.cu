@@ -15,14 +15,26 @@ namespace awq {
 // activation magnitude; "05 — AWQ" §4 step 1).
 //
 // Each thread owns 8 consecutive channels (one 16-byte load per token row) and
-// sums |x| over its share of a token chunk in fp64.  Every |x| is a multiple of
-// 2^-24 below 2^16, and a chunk holds at most 4096 tokens, so partial sums stay
-// below 2^29 and are exact in fp64.  Chunk sums are then converted to int64
+// sums |x| over its share of a token chunk in fp64 (the fp16 -> fp32 step uses
+// integer operations, keeping the conversion unit for the fp32 -> fp64 step).
+// Every |x| is a multiple
+// of 2^-24 below 2^16, and a chunk holds at most 4096 tokens, so partial sums
+// stay below 2^29 and are exact in fp64.  Chunk sums are then converted to int64
 // units of 2^-24 (exact) and added with 64-bit integer atomics (exact, so the
 // order of arrival does not matter).  Block: 32 x 8 threads covering 256
 // channels x 8 token rows per step.
 // ---------------------------------------------------------------------------
 constexpr int kStatsChunk = 1024;  // tokens per block (<= 4096 keeps fp64 exact)
+
+// |x| of the two fp16 values packed in `w`, as fp32, without the conversion
+// unit: shifting a magnitude h = (e << 10) | m into fp32 position gives the
+// fp32 pattern of 2^(e-127) (1 + m/1024) (e >= 1) or of the fp32 subnormal
+// m 2^-136 (e = 0); one exact multiplication by 2^112 yields 2^(e-15)(1 + m/1024)
+// and m 2^-24, the fp16 values.  (fp32 subnormals are kept: no flush-to-zero.)
+__device__ __forceinline__ void abs_half2_alu(uint32_t w, float &lo, float &hi) {
+  lo = __fmul_rn(__uint_as_float((w << 13) & 0x0FFFE000u), 5.192296858534828e+33f /* 2^112 */);
+  hi = __fmul_rn(__uint_as_float((w >> 3) & 0x0FFFE000u), 5.192296858534828e+33f);
+}
 
 __global__ void __launch_bounds__(256) act_stats_kernel(const __half *__restrict__ X, int64_t T,
                                                         int64_t in, int64_t ldx,
@@ -32,9 +44,9 @@ __global__ void __launch_bounds__(256) act_stats_kernel(const __half *__restrict
   const int64_t c0 = ((int64_t)blockIdx.x * 32 + tx) * 8;  // first channel of this thread
   const int64_t t_begin = (int64_t)blockIdx.y * kStatsChunk;
   const int64_t t_end = min(T, t_begin + kStatsChunk);
-  double s[8];
+  double s64[8];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) s[e] = 0.0;
+  for (int e = 0; e < 8; ++e) s64[e] = 0.0;
   if (c0 < in) {
     int64_t t = t_begin + ty;
     // four rows in flight per thread
@@ -45,30 +57,30 @@ __global__ void __launch_bounds__(256) act_stats_kernel(const __half *__restrict
         v[u] = __ldcs(reinterpret_cast<const uint4 *>(X + (t + 8 * u) * ldx + c0));
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const uint32_t w[4] = {v[u].x & 0x7FFF7FFFu, v[u].y & 0x7FFF7FFFu, v[u].z & 0x7FFF7FFFu,
-                               v[u].w & 0x7FFF7FFFu};
+        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
         for (int h = 0; h < 4; ++h) {
-          float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[h]));
-          s[2 * h] += (double)f.x;
-          s[2 * h + 1] += (double)f.y;
+          float a, b;
+          abs_half2_alu(w[h], a, b);
+          s64[2 * h] += (double)a;
+          s64[2 * h + 1] += (double)b;
         }
       }
     }
     for (; t < t_end; t += 8) {
-      uint4 v = __ldcs(reinterpret_cast<const uint4 *>(X + t * ldx + c0));
-      const uint32_t w[4] = {v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu, v.z & 0x7FFF7FFFu,
-                             v.w & 0x7FFF7FFFu};
+      const uint4 v = __ldcs(reinterpret_cast<const uint4 *>(X + t * ldx + c0));
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
-        float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[h]));
-        s[2 * h] += (double)f.x;
-        s[2 * h + 1] += (double)f.y;
+        float a, b;
+        abs_half2_alu(w[h], a, b);
+        s64[2 * h] += (double)a;
+        s64[2 * h + 1] += (double)b;
       }
     }
   }
 #pragma unroll
-  for (int e = 0; e < 8; ++e) red[ty][tx][e] = s[e];
+  for (int e = 0; e < 8; ++e) red[ty][tx][e] = s64[e];
   __syncthreads();
   if (ty == 0 && c0 < in) {
 #pragma unroll
@@ -186,11 +198,11 @@ __global__ void __launch_bounds__(256) cand_quant_kernel(
   const float two_k = ldexpf(1.0f, k);
   const int lanes = group / 8;  // lanes per group (a power of two <= 32)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t j0 = (int64_t)blockIdx.x * 256 + lane * 8;
+  const int64_t j0 = (int64_t)blockIdx.y * 256 + lane * 8;
   const bool j_ok = j0 < in;
   const int rb_per_alpha = (int)(out_pad / kCandRows);
-  const int a = blockIdx.y / rb_per_alpha;
-  const int64_t o0 = (int64_t)(blockIdx.y - a * rb_per_alpha) * kCandRows;
+  const int a = (int)(blockIdx.x / rb_per_alpha);
+  const int64_t o0 = (int64_t)(blockIdx.x - (int64_t)a * rb_per_alpha) * kCandRows;
   float sv[8], iv[8];
   if (j_ok) {
     const float4 *sp = reinterpret_cast<const float4 *>(s + (int64_t)a * in + j0);
@@ -222,13 +234,13 @@ __global__ void __launch_bounds__(256) cand_quant_kernel(
 #pragma unroll
       for (int e = 0; e < 8; ++e) w[e] = 0.0f;
     }
-    float wt[8];
+    float2 wt[4];
     float mx = -INFINITY, mn = INFINITY;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      wt[e] = __fmul_rn(sv[e], w[e]);
-      mx = fmaxf(mx, wt[e]);
-      mn = fminf(mn, wt[e]);
+    for (int h = 0; h < 4; ++h) {
+      wt[h] = __fmul2_rn(make_float2(sv[2 * h], sv[2 * h + 1]), make_float2(w[2 * h], w[2 * h + 1]));
+      mx = fmaxf(mx, fmaxf(wt[h].x, wt[h].y));
+      mn = fminf(mn, fminf(wt[h].x, wt[h].y));
     }
     for (int off = lanes >> 1; off > 0; off >>= 1) {
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
@@ -239,16 +251,13 @@ __global__ void __launch_bounds__(256) cand_quant_kernel(
     uint32_t packed[4];
 #pragma unroll
     for (int h = 0; h < 4; ++h) {
-      float d2[2];
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        const int e = 2 * h + u;
-        const float qz = __fsub_rn(quant_code(wt[e], g), g.zero);
-        // 2^k (deq/s - w) with deq = (q - z) delta; the product with 1/s is
-        // fp32 (the result is rounded to fp16 next)
-        d2[u] = live ? fmaf(__fmul_rn(qz, dk), iv[e], -__fmul_rn(w[e], two_k)) : 0.0f;
-      }
-      const __half2 hv = __floats2half2_rn(d2[0], d2[1]);
+      // 2^k (deq/s - w) with deq = (q - z) delta; the product with 1/s is
+      // fp32 (the result is rounded to fp16 next)
+      const float2 qz = quant_qz2(wt[h], g);
+      float2 d2 = __ffma2_rn(__fmul2_rn(qz, make_float2(dk, dk)), make_float2(iv[2 * h], iv[2 * h + 1]),
+                             __fmul2_rn(make_float2(w[2 * h], w[2 * h + 1]), make_float2(-two_k, -two_k)));
+      if (!live) d2 = make_float2(0.0f, 0.0f);
+      const __half2 hv = __floats2half2_rn(d2.x, d2.y);
       packed[h] = *reinterpret_cast<const uint32_t *>(&hv);
     }
     if (j_ok)
@@ -261,7 +270,7 @@ cudaError_t launch_cand_quant(const __half *W, int64_t out, int64_t in, int64_t 
                               const float *s, const float *inv_s, int n_alpha, int group, int w_bit,
                               const DevStatus *st, __half *dW, int num_sms, cudaStream_t stream) {
   (void)num_sms;
-  dim3 grid((unsigned)((in + 255) / 256), (unsigned)(n_alpha * (out_pad / kCandRows)));
+  dim3 grid((unsigned)(n_alpha * (out_pad / kCandRows)), (unsigned)((in + 255) / 256));
   cand_quant_kernel<<<grid, 256, 0, stream>>>(W, out, in, out_pad, s, inv_s, group,
                                               (float)((1 << w_bit) - 1), st, dW);
   return cudaGetLastError();
@@ -276,7 +285,7 @@ cudaError_t launch_cand_quant(const __half *W, int64_t out, int64_t in, int64_t 
 // through shared memory and are re-read transposed for packing, so every
 // global store is contiguous.
 // ---------------------------------------------------------------------------
-constexpr int kPackRows = 128;
+constexpr int kPackRows = 64;
 
 __device__ __forceinline__ float clip_ratio(int c, int n_clip, float clip_min) {
   if (n_clip <= 1) return 1.0f;
@@ -284,31 +293,52 @@ __device__ __forceinline__ float clip_ratio(int c, int n_clip, float clip_min) {
   return __double2float_rn(r);
 }
 
+// A block handles 64 output rows x one group of 128 input channels: the whole
+// W tile is fetched with independent 16-byte loads into shared memory, warps
+// quantise 8 rows each (4 channels per lane), codes are re-read transposed for
+// packing so every global store is contiguous.
 __global__ void __launch_bounds__(256) quant_pack_kernel(
     const __half *__restrict__ W, int64_t out, int64_t in, const float *__restrict__ s,
     const uint8_t *__restrict__ clip_idx, int n_clip, float clip_min, float qmax,
     int32_t *__restrict__ qweight, int32_t *__restrict__ qzeros, __half *__restrict__ scales) {
   constexpr int G = 128;
+  __shared__ __align__(16) __half wsm[kPackRows][G + 8];
   __shared__ uint8_t codes[kPackRows][G + 4];
   __shared__ uint8_t zeros[kPackRows];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int k = blockIdx.x;                       // group
-  const int64_t o0 = (int64_t)blockIdx.y * kPackRows;
+  const int k = blockIdx.y;  // group
+  const int64_t o0 = (int64_t)blockIdx.x * kPackRows;
   const int64_t groups = in / G;
-  const int64_t j0 = (int64_t)k * G + lane * 4;
+  const int rows_here = (int)i64min(kPackRows, out - o0);
+  {
+    uint4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int c = threadIdx.x + 256 * u;  // 16-byte chunk: row c/16, channels 8*(c%16)
+      const int r = c >> 4;
+      v[u] = r < rows_here ? __ldg(reinterpret_cast<const uint4 *>(W + (o0 + r) * in + (int64_t)k * G +
+                                                                  8 * (c & 15)))
+                           : make_uint4(0u, 0u, 0u, 0u);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int c = threadIdx.x + 256 * u;
+      *reinterpret_cast<uint4 *>(&wsm[c >> 4][8 * (c & 15)]) = v[u];
+    }
+  }
   float sv[4] = {1.0f, 1.0f, 1.0f, 1.0f};
   if (s) {
-    float4 f = __ldg(reinterpret_cast<const float4 *>(s + j0));
+    const float4 f = __ldg(reinterpret_cast<const float4 *>(s + (int64_t)k * G + lane * 4));
     sv[0] = f.x; sv[1] = f.y; sv[2] = f.z; sv[3] = f.w;
   }
-  for (int r = warp; r < kPackRows; r += 8) {
+  __syncthreads();
+  for (int r = warp; r < rows_here; r += 8) {
     const int64_t o = o0 + r;
-    if (o >= out) break;
-    uint2 wv = __ldg(reinterpret_cast<const uint2 *>(W + o * in + j0));
-    float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&wv.x));
-    float2 b = __half22float2(*reinterpret_cast<const __half2 *>(&wv.y));
-    float wt[4] = {__fmul_rn(sv[0], a.x), __fmul_rn(sv[1], a.y), __fmul_rn(sv[2], b.x),
-                   __fmul_rn(sv[3], b.y)};
+    const uint2 wv = *reinterpret_cast<const uint2 *>(&wsm[r][lane * 4]);
+    const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&wv.x));
+    const float2 b = __half22float2(*reinterpret_cast<const __half2 *>(&wv.y));
+    const float wt[4] = {__fmul_rn(sv[0], a.x), __fmul_rn(sv[1], a.y), __fmul_rn(sv[2], b.x),
+                         __fmul_rn(sv[3], b.y)};
     float mx = fmaxf(fmaxf(wt[0], wt[1]), fmaxf(wt[2], wt[3]));
     float mn = fminf(fminf(wt[0], wt[1]), fminf(wt[2], wt[3]));
 #pragma unroll
@@ -331,10 +361,9 @@ __global__ void __launch_bounds__(256) quant_pack_kernel(
   }
   __syncthreads();
   const int64_t words_per_row = out / 8;
-  const int rows_here = (int)i64min(kPackRows, out - o0);
   const int o8_here = rows_here / 8;  // out % 8 == 0
-  for (int t = threadIdx.x; t < G * 16; t += 256) {
-    const int o8 = t & 15, jj = t >> 4;
+  for (int t = threadIdx.x; t < G * 8; t += 256) {
+    const int o8 = t & 7, jj = t >> 3;
     if (o8 >= o8_here) continue;
     uint32_t word = 0;
 #pragma unroll
@@ -354,7 +383,7 @@ cudaError_t launch_quant_pack(const __half *W, int64_t out, int64_t in, const fl
                               float clip_min, int32_t *qweight, int32_t *qzeros, __half *scales,
                               cudaStream_t stream) {
   if (group != 128) return cudaErrorInvalidValue;
-  dim3 grid((unsigned)(in / group), (unsigned)((out + kPackRows - 1) / kPackRows));
+  dim3 grid((unsigned)((out + kPackRows - 1) / kPackRows), (unsigned)(in / group));
   quant_pack_kernel<<<grid, 256, 0, stream>>>(W, out, in, s, clip_idx, n_clip, clip_min,
                                               (float)((1 << w_bit) - 1), qweight, qzeros, scales);
   return cudaGetLastError();
