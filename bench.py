@@ -37,9 +37,10 @@ KERNELS_PER_STEP = {  # kernels this library launches per step (memsets excluded
     "act_stats": 2, "wmax": 1, "scale_grid": 1, "cand_quant": 1, "search_gemm": 1,
     "mse_argmin": 1, "gram_blocks": 2, "clip_eval": 1, "quant_pack": 1,
 }
-# ncu capture of the dominant kernel (q_proj workload, one launch), per launch;
-# None when the kernel changed after the capture.
-NCU_TRAFFIC_BYTES = None
+# DRAM bytes (read + write) of one search_gemm_kernel launch on this workload,
+# from a one-pass ncu capture (profiles/search_gemm_q_proj_4096.md); to be
+# set to None whenever that kernel changes until it is captured again.
+NCU_TRAFFIC_BYTES = 11_290_000_000 + 9_940_000
 
 
 def load_peaks():
