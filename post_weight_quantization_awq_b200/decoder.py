@@ -1,0 +1,104 @@
+"""Layer-by-layer AWQ of a Llama-style decoder layer (the pages' offline
+pass: "AWQ and Activation-Aware Scaling", Why this is attractive: forward
+passes to collect statistics, then a small per-layer search).
+
+Per layer, for the four groups of linears that share an input
+(q|k|v, o, gate|up, down):
+  1. abar and the alpha search on the captured fp16 inputs (awq_act_stats,
+     awq_search_scale), all four groups before any weight changes;
+  2. fold 1/s into the operation feeding each group ("Scaling instead of
+     protecting": the activation-side division is absorbed by the preceding
+     normalisation's scale or linear layer): RMSNorm1 gamma <- qkv's s,
+     v_proj rows <- o's s, RMSNorm2 gamma <- gate|up's s, up_proj rows <-
+     down's s (awq_fold_inv_scale, in fp16);
+  3. clip search and packing of each group on the folded weights
+     (awq_search_clip, awq_quant_pack).
+Every step runs in the library's kernels; this module only orders the calls
+and slices the concatenated results.
+"""
+
+from __future__ import annotations
+
+import os
+from typing import Dict, Optional
+
+import torch
+
+from . import abi
+from .abi import AwqConfig
+
+GROUPS = (("qkv", ("q", "k", "v")), ("o", ("o",)), ("gate_up", ("gate", "up")), ("down", ("down",)))
+FOLDS = (("qkv", "gamma1"), ("o", "v"), ("gate_up", "gamma2"), ("down", "up"))
+
+
+def _search(X: torch.Tensor, W: torch.Tensor, cfg: AwqConfig, ws: torch.Tensor):
+    inn = X.shape[1]
+    dev = X.device
+    abar = torch.empty(inn, dtype=torch.float64, device=dev)
+    mse = torch.empty(cfg.n_alpha, dtype=torch.float64, device=dev)
+    best = torch.empty(1, dtype=torch.int32, device=dev)
+    s = torch.empty(inn, dtype=torch.float32, device=dev)
+    abi.awq_act_stats(X, abar)
+    abi.awq_search_scale(X, W, abar, cfg, ws, s, mse, best)
+    return {"abar": abar, "mse": mse, "best_idx": best, "s": s}
+
+
+def workspace_for_layer(captures: Dict[str, torch.Tensor], weights: Dict[str, torch.Tensor],
+                        cfg: AwqConfig) -> torch.Tensor:
+    need = 0
+    for g, names in GROUPS:
+        X = captures[g]
+        out = sum(weights[n].shape[0] for n in names)
+        need = max(need, abi.awq_workspace_size(X.shape[0], X.shape[1], out, cfg))
+    return torch.empty(need, dtype=torch.uint8, device=captures["qkv"].device)
+
+
+def quantize_layer_groups(captures: Dict[str, torch.Tensor], weights: Dict[str, torch.Tensor],
+                          cfg: AwqConfig, ws: Optional[torch.Tensor] = None) -> dict:
+    """AWQ of one decoder layer.  `weights` (fp16, [out, in]; gammas [hidden])
+    are modified in place by the folds.  Returns per group: abar, mse,
+    best_idx, s, clip_idx, qweight, qzeros, scales (concatenated along out for
+    joint groups) and per linear the (first, last) output rows."""
+    if ws is None:
+        ws = workspace_for_layer(captures, weights, cfg)
+    res = {}
+    cat = {g: (torch.cat([weights[n] for n in names], 0) if len(names) > 1 else weights[names[0]])
+           for g, names in GROUPS}
+    for g, _ in GROUPS:
+        res[g] = _search(captures[g], cat[g], cfg, ws)
+        abi.awq_device_status(ws)
+    for g, target in FOLDS:
+        abi.awq_fold_inv_scale(weights[target], res[g]["s"])
+    for g, names in GROUPS:
+        W = torch.cat([weights[n] for n in names], 0) if len(names) > 1 else weights[names[0]]
+        X = captures[g]
+        out, inn = W.shape
+        gsz = cfg.group_size
+        clip_idx = None
+        if cfg.n_clip > 0:
+            clip_idx = torch.empty((out, inn // gsz), dtype=torch.uint8, device=W.device)
+            abi.awq_search_clip(X, W, res[g]["s"], cfg, ws, clip_idx)
+            abi.awq_device_status(ws)
+        qweight = torch.empty((inn, out // 8), dtype=torch.int32, device=W.device)
+        qzeros = torch.empty((inn // gsz, out // 8), dtype=torch.int32, device=W.device)
+        scales = torch.empty((inn // gsz, out), dtype=torch.float16, device=W.device)
+        abi.awq_quant_pack(W, res[g]["s"], clip_idx, cfg, qweight, qzeros, scales)
+        rows, r0 = {}, 0
+        for n in names:
+            rows[n] = (r0, r0 + weights[n].shape[0])
+            r0 += weights[n].shape[0]
+        res[g].update({"clip_idx": clip_idx, "qweight": qweight, "qzeros": qzeros, "scales": scales,
+                       "rows": rows, "weights_folded": W})
+    return res
+
+
+def save_layer_checkpoint(path: str, layer: int, res: dict) -> None:
+    """Writes one layer's results atomically (temporary file, then rename)."""
+    state = {"layer": layer}
+    for g, _ in GROUPS:
+        r = res[g]
+        state[g] = {k: (v.cpu() if isinstance(v, torch.Tensor) else v) for k, v in r.items()
+                    if k not in ("weights_folded", "abar")}
+    tmp = path + ".tmp"
+    torch.save(state, tmp)
+    os.replace(tmp, path)

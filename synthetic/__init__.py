@@ -35,6 +35,10 @@ __all__ = [
     "Workload",
     "WORKLOADS",
     "workload_inputs",
+    "DecoderSpec",
+    "decoder_layer_weights",
+    "decoder_embeddings",
+    "decoder_layer_forward",
 ]
 
 
@@ -195,3 +199,99 @@ def random_layer(T: int, d_in: int, d_out: int, seed: int,
     X = heavy_tailed_activations(T, d_in, outliers, seed)
     W = gaussian_weight(d_out, d_in, seed, std=w_std)
     return X, W
+
+
+# ---------------------------------------------------------------------------
+# Synthetic Llama-2-7B-architecture decoder (random init) for layer-by-layer
+# calibration captures.  This is the model's fp16 forward pass (input
+# synthesis), not AWQ: hidden states propagate through the unmodified layer.
+# ---------------------------------------------------------------------------
+@dataclasses.dataclass(frozen=True)
+class DecoderSpec:
+    hidden: int = 4096
+    heads: int = 32
+    ffn: int = 11008
+    layers: int = 32
+    vocab: int = 32000
+    seq: int = 512
+    n_seq: int = 128
+    rope_theta: float = 10000.0
+    eps: float = 1e-5
+    w_std: float = 0.02
+    outliers: OutlierSpec = OutlierSpec(0.01, 20.0, 50.0)
+    seed: int = 4
+
+
+def decoder_layer_weights(spec: DecoderSpec, layer: int, device: str = "cpu") -> dict:
+    """fp16 weights of one decoder layer, N(0, w_std), nn.Linear layout
+    [out, in]; RMSNorm gammas are 1.  Drawn on `device` with a generator of
+    that device seeded from (spec.seed, layer), so a CUDA device gives the
+    same weights on every run of the same build."""
+    h, f = spec.hidden, spec.ffn
+    shapes = {"q": (h, h), "k": (h, h), "v": (h, h), "o": (h, h), "gate": (f, h), "up": (f, h),
+              "down": (h, f)}
+    g = torch.Generator(device=device)
+    g.manual_seed(spec.seed * 100_000 + layer)
+    w = {name: (spec.w_std * torch.randn(shp, generator=g, dtype=torch.float32, device=device)
+                ).to(torch.float16) for name, shp in shapes.items()}
+    w["gamma1"] = torch.ones(h, dtype=torch.float16, device=device)
+    w["gamma2"] = torch.ones(h, dtype=torch.float16, device=device)
+    return w
+
+
+def decoder_embeddings(spec: DecoderSpec, n_seq: Optional[int] = None, device: str = "cpu") -> torch.Tensor:
+    """Calibration input of layer 0: n_seq random token sequences of spec.seq
+    tokens looked up in a random N(0, w_std) embedding table whose outlier
+    channels are multiplied by U[lo, hi]; fp16 [n_seq * seq, hidden]."""
+    n_seq = spec.n_seq if n_seq is None else n_seq
+    g = _gen(spec.seed * 1_000_003 + 11)
+    ids = torch.randint(0, spec.vocab, (n_seq * spec.seq,), generator=g)
+    table = spec.w_std * torch.randn((spec.vocab, spec.hidden), generator=g, dtype=torch.float32)
+    n_out = int(round(spec.outliers.frac * spec.hidden))
+    idx = torch.randperm(spec.hidden, generator=g)[:n_out]
+    mult = spec.outliers.lo + (spec.outliers.hi - spec.outliers.lo) * torch.rand(n_out, generator=g)
+    table[:, idx] *= mult
+    return table.to(torch.float16)[ids].to(device)
+
+
+def _rms_norm(x: torch.Tensor, gamma: torch.Tensor, eps: float) -> torch.Tensor:
+    xf = x.float()
+    return (xf * torch.rsqrt(xf.pow(2).mean(-1, keepdim=True) + eps) * gamma.float()).to(torch.float16)
+
+
+def _rope(x: torch.Tensor, theta: float) -> torch.Tensor:
+    # x: [B, heads, S, d]
+    d = x.shape[-1]
+    pos = torch.arange(x.shape[-2], device=x.device, dtype=torch.float32)
+    inv = theta ** (-torch.arange(0, d, 2, device=x.device, dtype=torch.float32) / d)
+    ang = pos[:, None] * inv[None, :]
+    cos, sin = ang.cos(), ang.sin()
+    xf = x.float()
+    x1, x2 = xf[..., ::2], xf[..., 1::2]
+    out = torch.empty_like(xf)
+    out[..., ::2] = x1 * cos - x2 * sin
+    out[..., 1::2] = x1 * sin + x2 * cos
+    return out.to(torch.float16)
+
+
+@torch.no_grad()
+def decoder_layer_forward(x: torch.Tensor, w: dict, spec: DecoderSpec):
+    """One fp16 decoder layer (RMSNorm, RoPE causal attention, SwiGLU MLP).
+    Returns (captures, x_next) where captures holds the inputs of the four
+    linear groups: 'qkv' (RMSNorm1 output), 'o' (attention output), 'gate_up'
+    (RMSNorm2 output), 'down' (SiLU(gate) * up)."""
+    T, h = x.shape
+    B, S, H = T // spec.seq, spec.seq, spec.heads
+    d = h // H
+    a_in = _rms_norm(x, w["gamma1"], spec.eps)
+    q = (a_in @ w["q"].T).view(B, S, H, d).transpose(1, 2)
+    k = (a_in @ w["k"].T).view(B, S, H, d).transpose(1, 2)
+    v = (a_in @ w["v"].T).view(B, S, H, d).transpose(1, 2)
+    q, k = _rope(q, spec.rope_theta), _rope(k, spec.rope_theta)
+    att = torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=True)
+    o_in = att.transpose(1, 2).reshape(T, h).contiguous()
+    x = x + o_in @ w["o"].T
+    m_in = _rms_norm(x, w["gamma2"], spec.eps)
+    d_in = (torch.nn.functional.silu((m_in @ w["gate"].T).float()) * (m_in @ w["up"].T).float()).to(torch.float16)
+    x = x + d_in @ w["down"].T
+    return {"qkv": a_in, "o": o_in, "gate_up": m_in, "down": d_in.contiguous()}, x
