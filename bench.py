@@ -396,6 +396,58 @@ def run_awq(args):
     return 0
 
 
+def run_decoder(args):
+    """Times the layer-by-layer AWQ of the 32-layer Llama-2-7B-architecture
+    decoder (128 x 512 calibration tokens): per layer the four groups' alpha
+    searches, the folds, the clip searches and the packing.  The fp16 forward
+    that captures each layer's inputs is input synthesis and is not timed."""
+    import torch
+    import post_weight_quantization_awq_b200 as awq
+    from post_weight_quantization_awq_b200 import decoder
+    from synthetic import DecoderSpec, decoder_embeddings, decoder_layer_forward, decoder_layer_weights
+    world, rank, local = dist_env()
+    if world > 1:
+        raise SystemExit("--workload decoder runs on one GPU")
+    torch.cuda.set_device(local)
+    spec = DecoderSpec()
+    cfg = awq.AwqConfig.make(w_bit=4, n_alpha=20, n_clip=20, clip_min=0.5)
+    layers = min(args.steps, spec.layers)
+    x = decoder_embeddings(spec, device="cuda")
+    ws = None
+    times = []
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    for layer in range(layers):
+        w = decoder_layer_weights(spec, layer, device="cuda")
+        caps, x_next = decoder_layer_forward(x, w, spec)
+        if ws is None:
+            ws = decoder.workspace_for_layer(caps, w, cfg)
+            for _ in range(args.warmup):  # warm-up on copies of layer 0
+                decoder.quantize_layer_groups(caps, {k: v.clone() for k, v in w.items()}, cfg, ws)
+        torch.cuda.synchronize()
+        e0.record()
+        decoder.quantize_layer_groups(caps, w, cfg, ws)
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+        x = x_next
+    flops = 2.0 * spec.seq * spec.n_seq * cfg.n_alpha * spec.hidden * (
+        3 * spec.hidden + spec.hidden + 2 * spec.ffn) + 2.0 * spec.seq * spec.n_seq * cfg.n_alpha * spec.ffn * spec.hidden
+    ms = statistics.mean(times)
+    print(json.dumps({
+        "metric": METRIC, "value": round(ms, 3), "unit": UNIT, "n_gpus": 1, "steps": layers,
+        "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": False,
+        "scaling": "weak", "vs_baseline": None, "dtype": "fp16",
+        "data": "synthetic (random-init decoder, random token ids, outlier embedding channels)",
+        "config": {"workload": "llama2_7b_decoder_32_layers: hidden 4096, 32 heads, MLP 11008, "
+                               "128 x 512 calibration tokens, four groups per layer (q|k|v, o, gate|up, "
+                               "down), INT4 g128, 20 alphas + 20 clip ratios, folds, packed",
+                   "layers_timed": layers, "forward_capture": "untimed"},
+        "candidate_gemm_tflops": round(flops / (ms * 1e-3) / 1e12, 1),
+        "ms_per_layer_min_max": [round(min(times), 3), round(max(times), 3)],
+    }), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -405,11 +457,16 @@ def main(argv=None):
     ap.add_argument("--ref-row-fraction", type=float, default=0.125,
                     help="share of output rows the oracle runs on (then scaled)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workload", choices=("q_proj", "decoder"), default="q_proj",
+                    help="q_proj: the headline workload; decoder: the 32-layer decoder "
+                         "(--steps = layers timed)")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload == "decoder":
+        return run_decoder(args)
     return run_awq(args)
 
 

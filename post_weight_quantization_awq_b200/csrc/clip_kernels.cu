@@ -265,6 +265,7 @@ struct __align__(16) ClipSmem {
   float rmx[CT_MAXR], rmn[CT_MAXR];
   int rexp[CT_MAXR];
   float epart[4][128];
+  float ratio[128];  // clip ratio of each index
   uint64_t mma_bar;
   uint32_t tmem_base;
   int abort_flag;  // a wait ran out: every thread leaves the tile loop together
@@ -329,6 +330,7 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
     S.abort_flag = 0;
     fence_mbar_init();
   }
+  if (tid < n_clip) S.ratio[tid] = clip_ratio_f(tid, n_clip, clip_min);
   if (warp == 0) {
     tmem_alloc(&S.tmem_base, 128);
     tmem_relinquish();
@@ -430,7 +432,7 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
       const int h = qq >> 1;
       uint8_t *ahi = S.a_hi + h * CT_ATOM, *alo = S.a_lo + h * CT_ATOM;
       if (valid) {
-        const GroupQ g = group_params(S.rmx[rr], S.rmn[rr], clip_ratio_f(c, n_clip, clip_min), qmax);
+        const GroupQ g = group_params(S.rmx[rr], S.rmn[rr], S.ratio[c], qmax);
         const float de = ldexpf(g.delta, S.rexp[rr]);  // exact power-of-two scaling
         const float *wtr = S.wt[rr];
         const float *bwr = S.bw[rr];

@@ -305,7 +305,9 @@ __global__ void __launch_bounds__(256) quant_pack_kernel(
   __shared__ __align__(16) __half wsm[kPackRows][G + 8];
   __shared__ uint8_t codes[kPackRows][G + 4];
   __shared__ uint8_t zeros[kPackRows];
+  __shared__ float ratios[64];  // clip ratio of each index (n_clip <= 64)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (clip_idx && threadIdx.x < n_clip) ratios[threadIdx.x] = clip_ratio(threadIdx.x, n_clip, clip_min);
   const int k = blockIdx.y;  // group
   const int64_t o0 = (int64_t)blockIdx.x * kPackRows;
   const int64_t groups = in / G;
@@ -346,7 +348,7 @@ __global__ void __launch_bounds__(256) quant_pack_kernel(
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
       mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
     }
-    const float r32 = clip_idx ? clip_ratio(clip_idx[o * groups + k], n_clip, clip_min) : 1.0f;
+    const float r32 = clip_idx ? ratios[clip_idx[o * groups + k]] : 1.0f;
     const GroupQ g = group_params(mx, mn, r32, qmax);
     uchar4 c4;
     c4.x = (uint8_t)quant_code(wt[0], g);
