@@ -61,6 +61,16 @@ typedef enum {
   AWQ_ERR_NONFINITE = 6    /* a score came out NaN or infinite                */
 } awq_status;
 
+/* How awq_search_scale scores the candidates (both give the same MSE in exact
+ * arithmetic, by the scaling invariance of "05 — AWQ" §3):
+ *   AWQ_SEARCH_DIRECT  the scored GEMM ||X dW^T||^2 over all tokens
+ *                      (2 T in out n_alpha flops);
+ *   AWQ_SEARCH_GRAM    sum_o dW_o^T (X^T X) dW_o: G = X^T X once (T in^2 flops,
+ *                      symmetric), then one GEMM of the candidates against the
+ *                      normalised G held as fp16 hi + lo parts
+ *                      (4 in^2 out n_alpha flops). */
+enum { AWQ_SEARCH_DIRECT = 0, AWQ_SEARCH_GRAM = 1 };
+
 /* Quantisation and search settings; the first three fields are the pages'
  * quant_config ("05 — AWQ" §9: w_bit, q_group_size, zero_point). */
 typedef struct {
@@ -70,6 +80,7 @@ typedef struct {
   int32_t n_alpha;    /* alpha grid size, 1..64; alpha_i = i/(n_alpha-1) ("05 — AWQ" §4: ~20) */
   int32_t n_clip;     /* clip grid size, 0 = no clip search, else 1..64          */
   float clip_min;     /* smallest clip ratio, in (0, 1]; ("05 — AWQ" §4: 0.5)    */
+  int32_t search_form; /* AWQ_SEARCH_DIRECT (0, default) or AWQ_SEARCH_GRAM (1)   */
 } awq_config;
 
 /* Bytes of workspace needed by awq_search_scale and awq_search_clip for a
@@ -101,7 +112,8 @@ awq_status awq_scale_grid(const double *abar, int64_t in, int32_t n_alpha, float
  * scores MSE_i = mean over tokens and outputs of
  *   ((X diag(s_i)^-1) Qdeq(diag(s_i) W)^T - X W^T)^2,
  * evaluated as ||X dW_i^T||^2 / (T out) with dW_i = Qdeq/s_i - W (the
- * scaling invariance of "05 — AWQ" §3), on the tensor cores.
+ * scaling invariance of "05 — AWQ" §3), on the tensor cores; with
+ * cfg->search_form = AWQ_SEARCH_GRAM as sum_o dW_o^T (X^T X) dW_o / (T out).
  *   abar     device fp64 [in] from awq_act_stats
  *   s_best   device fp32 [in]      (output) s of the selected alpha
  *   mse      device fp64 [n_alpha] (output) MSE_i

@@ -37,9 +37,13 @@ class AwqError(RuntimeError):
         super().__init__(f"{func}: {self.status_name}: {message}")
 
 
+SEARCH_DIRECT, SEARCH_GRAM = 0, 1
+
+
 class AwqConfig(ctypes.Structure):
     """awq_config: w_bit, group_size, zero_point ("05 — AWQ" §9 quant_config),
-    n_alpha, n_clip, clip_min ("05 — AWQ" §4)."""
+    n_alpha, n_clip, clip_min ("05 — AWQ" §4), search_form (0 direct scored
+    GEMM, 1 Gram form)."""
 
     _fields_ = [
         ("w_bit", c_int32),
@@ -48,12 +52,14 @@ class AwqConfig(ctypes.Structure):
         ("n_alpha", c_int32),
         ("n_clip", c_int32),
         ("clip_min", c_float),
+        ("search_form", c_int32),
     ]
 
     @classmethod
-    def make(cls, w_bit=4, group_size=128, zero_point=1, n_alpha=20, n_clip=0, clip_min=0.5):
+    def make(cls, w_bit=4, group_size=128, zero_point=1, n_alpha=20, n_clip=0, clip_min=0.5,
+             search_form=0):
         return cls(int(w_bit), int(group_size), int(zero_point), int(n_alpha), int(n_clip),
-                   float(clip_min))
+                   float(clip_min), int(search_form))
 
 
 _SIGNATURES = {

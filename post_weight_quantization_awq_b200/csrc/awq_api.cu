@@ -109,6 +109,8 @@ awq_status check_cfg(const awq_config *cfg) {
     return fail(AWQ_ERR_INVALID_ARG, "n_clip=%d (0..64)", cfg->n_clip);
   if (!(cfg->clip_min > 0.0f && cfg->clip_min <= 1.0f))
     return fail(AWQ_ERR_INVALID_ARG, "clip_min=%g (must be in (0, 1])", (double)cfg->clip_min);
+  if (cfg->search_form != AWQ_SEARCH_DIRECT && cfg->search_form != AWQ_SEARCH_GRAM)
+    return fail(AWQ_ERR_INVALID_ARG, "search_form=%d (0 direct, 1 Gram)", cfg->search_form);
   return AWQ_OK;
 }
 
@@ -135,18 +137,25 @@ awq_status check_x(const void *X, int64_t in, int64_t ldx) {
 constexpr size_t kHeader = 256;
 
 struct ScaleWs {
-  size_t s_grid, inv_s, dW, partials, end;
+  size_t s_grid, inv_s, dW, partials, G, ghi, glo, r, end;
   int64_t out_pad;
   int num_m, nb_per_alpha;
+  size_t per_alpha;  // partials per candidate
 };
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// Direct form: candidates padded to the GEMM's 256-row N tiles, partials per
+// (n tile, m tile, warp).  Gram form: candidates padded to 128-row M tiles,
+// partials per (m tile, n tile, warp), plus G, G~ hi/lo and r.
 ScaleWs scale_layout(int64_t T, int64_t in, int64_t out, const awq_config *cfg) {
   ScaleWs w;
-  w.out_pad = round_up(out, kGemmBN);
+  const bool gram = cfg->search_form == AWQ_SEARCH_GRAM;
+  w.out_pad = round_up(out, gram ? 128 : kGemmBN);
   w.num_m = (int)((T + kGemmBM - 1) / kGemmBM);
   w.nb_per_alpha = (int)(w.out_pad / kGemmBN);
+  w.per_alpha = gram ? (size_t)(w.out_pad / 128) * (size_t)(in / 128) * 4
+                     : (size_t)w.nb_per_alpha * w.num_m * 4;
   size_t off = kHeader;
   w.s_grid = off;
   off = align256(off + sizeof(float) * (size_t)cfg->n_alpha * in);
@@ -155,7 +164,18 @@ ScaleWs scale_layout(int64_t T, int64_t in, int64_t out, const awq_config *cfg) 
   w.dW = off;
   off = align256(off + sizeof(__half) * (size_t)cfg->n_alpha * w.out_pad * in);
   w.partials = off;
-  off = align256(off + sizeof(double) * (size_t)cfg->n_alpha * w.nb_per_alpha * w.num_m * 4);
+  off = align256(off + sizeof(double) * (size_t)cfg->n_alpha * w.per_alpha);
+  w.G = w.ghi = w.glo = w.r = 0;
+  if (gram) {
+    w.G = off;
+    off = align256(off + sizeof(float) * (size_t)in * in);
+    w.ghi = off;
+    off = align256(off + sizeof(__half) * (size_t)in * in);
+    w.glo = off;
+    off = align256(off + sizeof(__half) * (size_t)in * in);
+    w.r = off;
+    off = align256(off + sizeof(float) * (size_t)in);
+  }
   w.end = off;
   return w;
 }
@@ -274,9 +294,19 @@ awq_status awq_search_scale(const void *X, int64_t T, int64_t in, int64_t ldx, c
 
   // status of this call only: flags, site, exponent and max |W| start at zero
   AWQ_TRY_CUDA(cudaMemsetAsync(dst, 0, sizeof(DevStatus), s), "workspace reset");
+  const bool gram = cfg->search_form == AWQ_SEARCH_GRAM;
+  float *r = gram ? reinterpret_cast<float *>(base + L.r) : nullptr;
+  if (gram) {
+    ProfScope p("gram_full", s);
+    AWQ_TRY_CUDA(launch_gram_full(static_cast<const __half *>(X), T, in, ldx,
+                                  reinterpret_cast<float *>(base + L.G), r,
+                                  reinterpret_cast<__half *>(base + L.ghi),
+                                  reinterpret_cast<__half *>(base + L.glo), dst, poll_cap(), s),
+                 "gram_full launch");
+  }
   {
     ProfScope p("wmax", s);
-    AWQ_TRY_CUDA(launch_wmax(static_cast<const __half *>(W), out * in, dst, nsm, s), "wmax launch");
+    AWQ_TRY_CUDA(launch_wmax(static_cast<const __half *>(W), out * in, in, r, dst, nsm, s), "wmax launch");
   }
   {
     ProfScope p("scale_grid", s);
@@ -284,11 +314,18 @@ awq_status awq_search_scale(const void *X, int64_t T, int64_t in, int64_t ldx, c
   }
   {
     ProfScope p("cand_quant", s);
-    AWQ_TRY_CUDA(launch_cand_quant(static_cast<const __half *>(W), out, in, L.out_pad, s_grid, inv_s,
+    AWQ_TRY_CUDA(launch_cand_quant(static_cast<const __half *>(W), out, in, L.out_pad, s_grid, inv_s, r,
                                    cfg->n_alpha, cfg->group_size, cfg->w_bit, dst, dW, nsm, s),
                  "cand_quant launch");
   }
-  {
+  if (gram) {
+    ProfScope p("gram_score", s);
+    AWQ_TRY_CUDA(launch_gram_score(dW, (int64_t)cfg->n_alpha * L.out_pad, in,
+                                   reinterpret_cast<const __half *>(base + L.ghi),
+                                   reinterpret_cast<const __half *>(base + L.glo), partials, dst,
+                                   poll_cap(), nsm, s),
+                 "gram_score launch");
+  } else {
     SearchGemmShape sh;
     sh.T = T;
     sh.in = in;
@@ -303,8 +340,8 @@ awq_status awq_search_scale(const void *X, int64_t T, int64_t in, int64_t ldx, c
   }
   {
     ProfScope p("mse_argmin", s);
-    AWQ_TRY_CUDA(launch_mse_argmin(partials, cfg->n_alpha, L.nb_per_alpha, L.num_m, T, out, s_grid,
-                                   in, dst, mse, best_idx, s_best, s),
+    AWQ_TRY_CUDA(launch_mse_argmin(partials, cfg->n_alpha, L.per_alpha, T, out, s_grid, in, dst, mse,
+                                   best_idx, s_best, s),
                  "mse_argmin launch");
   }
   if (getenv("AWQ_SYNC_CHECK")) return awq_device_status(ws, stream);

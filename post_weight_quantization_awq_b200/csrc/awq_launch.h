@@ -21,14 +21,16 @@ cudaError_t launch_act_stats(const __half *X, int64_t T, int64_t in, int64_t ldx
 cudaError_t launch_scale_grid(const double *abar, int64_t in, int n_alpha, float *s, float *inv_s,
                               cudaStream_t stream);
 
-// max |W| into st->wmax_bits (st->wmax_bits must be zero beforehand).
-cudaError_t launch_wmax(const __half *W, int64_t n, DevStatus *st, int num_sms, cudaStream_t stream);
+// max |W| (r == NULL) or max r_j |W_oj| into st->wmax_bits (zero beforehand).
+cudaError_t launch_wmax(const __half *W, int64_t n, int64_t in, const float *r, DevStatus *st,
+                        int num_sms, cudaStream_t stream);
 
-// K3: candidate effective errors dW[i][o][j] = RN16(2^k (deq/s - w)), rows
-// out..out_pad-1 zero.
+// K3: candidate effective errors dW[i][o][j] = RN16(2^k r_j (deq/s - w))
+// (r = NULL: r_j = 1), rows out..out_pad-1 zero.
 cudaError_t launch_cand_quant(const __half *W, int64_t out, int64_t in, int64_t out_pad,
-                              const float *s, const float *inv_s, int n_alpha, int group, int w_bit,
-                              const DevStatus *st, __half *dW, int num_sms, cudaStream_t stream);
+                              const float *s, const float *inv_s, const float *r, int n_alpha,
+                              int group, int w_bit, const DevStatus *st, __half *dW, int num_sms,
+                              cudaStream_t stream);
 
 // K4: scored GEMM, partial sums of squares per (n-tile, m-tile, warp).
 struct SearchGemmShape {
@@ -45,11 +47,20 @@ constexpr int kGemmBM = 128, kGemmBN = 256, kGemmBK = 64;
 cudaError_t make_tmap_f16_box(CUtensorMap *m, const void *base, int64_t rows, int64_t cols,
                               int64_t ld, uint32_t box_cols, uint32_t box_rows);
 
-// K5: mse[i], best index, s_best.
-cudaError_t launch_mse_argmin(const double *partials, int n_alpha, int nb_per_alpha, int num_m,
-                              int64_t T, int64_t out, const float *s_grid, int64_t in,
-                              DevStatus *st, double *mse, int32_t *best_idx, float *s_best,
-                              cudaStream_t stream);
+// K5: mse[i] from `per_alpha` contiguous partials per candidate, best index, s_best.
+cudaError_t launch_mse_argmin(const double *partials, int n_alpha, size_t per_alpha, int64_t T,
+                              int64_t out, const float *s_grid, int64_t in, DevStatus *st,
+                              double *mse, int32_t *best_idx, float *s_best, cudaStream_t stream);
+
+// Gram form: G = X^T X (fp32 [in][in]), r = sqrt(diag G), G~ hi/lo fp16 [in][in].
+cudaError_t launch_gram_full(const __half *X, int64_t T, int64_t in, int64_t ldx, float *G, float *r,
+                             __half *ghi, __half *glo, DevStatus *st, uint32_t max_polls,
+                             cudaStream_t stream);
+// Gram form scoring: partials[(m_blk * (in/128) + n_blk) * 4 + warp] of
+// d~ (G~_hi + G~_lo) . d~ over 128 x 128 tiles; rows % 128 == 0.
+cudaError_t launch_gram_score(const __half *dW, int64_t rows, int64_t in, const __half *ghi,
+                              const __half *glo, double *partials, DevStatus *st, uint32_t max_polls,
+                              int num_sms, cudaStream_t stream);
 
 // K6a: block Grams G[k] = X_k^T X_k (fp32, tensor cores), via per-chunk
 // partials [n_chunks][in/g][g][g] summed in a fixed order.

@@ -147,32 +147,38 @@ cudaError_t launch_scale_grid(const double *abar, int64_t in, int n_alpha, float
 // ---------------------------------------------------------------------------
 // max |W| (bit pattern of a non-negative float orders like an unsigned int).
 // ---------------------------------------------------------------------------
-__global__ void wmax_kernel(const __half *__restrict__ W, int64_t n, DevStatus *st) {
+// max |W| (r == NULL) or max_oj r_j |W_oj| (bit pattern of a non-negative
+// float orders like an unsigned int).
+__global__ void wmax_kernel(const __half *__restrict__ W, int64_t n, int64_t in,
+                            const float *__restrict__ r, DevStatus *st) {
   uint32_t m = 0;
-  const int64_t n8 = n / 8;
+  const int64_t n8 = n / 8;  // in % 8 == 0: the 8 values of a vector share a row
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8;
        i += (int64_t)gridDim.x * blockDim.x) {
     uint4 v = __ldg(reinterpret_cast<const uint4 *>(W) + i);
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    const int64_t j0 = (i * 8) % in;
 #pragma unroll
     for (int h = 0; h < 4; ++h) {
       float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&w[h]));
-      m = max(m, __float_as_uint(fabsf(f.x)));
-      m = max(m, __float_as_uint(fabsf(f.y)));
+      float a = fabsf(f.x), b = fabsf(f.y);
+      if (r) {
+        a *= __ldg(r + j0 + 2 * h);
+        b *= __ldg(r + j0 + 2 * h + 1);
+      }
+      m = max(m, __float_as_uint(a));
+      m = max(m, __float_as_uint(b));
     }
   }
-  for (int64_t i = n8 * 8 + (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
-       i += (int64_t)gridDim.x * blockDim.x)
-    m = max(m, __float_as_uint(fabsf(__half2float(W[i]))));
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, off));
   if ((threadIdx.x & 31) == 0 && m) atomicMax(&st->wmax_bits, m);
 }
 
-cudaError_t launch_wmax(const __half *W, int64_t n, DevStatus *st, int num_sms,
-                        cudaStream_t stream) {
+cudaError_t launch_wmax(const __half *W, int64_t n, int64_t in, const float *r, DevStatus *st,
+                        int num_sms, cudaStream_t stream) {
   int64_t blocks = i64min((int64_t)num_sms * 4, (n / 8 + 255) / 256 + 1);
-  wmax_kernel<<<(unsigned)blocks, 256, 0, stream>>>(W, n, st);
+  wmax_kernel<<<(unsigned)blocks, 256, 0, stream>>>(W, n, in, r, st);
   return cudaGetLastError();
 }
 
@@ -192,8 +198,8 @@ constexpr int kCandRows = 64;
 
 __global__ void __launch_bounds__(256) cand_quant_kernel(
     const __half *__restrict__ W, int64_t out, int64_t in, int64_t out_pad,
-    const float *__restrict__ s, const float *__restrict__ inv_s, int group, float qmax,
-    const DevStatus *__restrict__ st, __half *__restrict__ dW) {
+    const float *__restrict__ s, const float *__restrict__ inv_s, const float *__restrict__ rch,
+    int group, float qmax, const DevStatus *__restrict__ st, __half *__restrict__ dW) {
   const int k = kscale_from_wmax(__uint_as_float(__ldg(&st->wmax_bits)));
   const float two_k = ldexpf(1.0f, k);
   const int lanes = group / 8;  // lanes per group (a power of two <= 32)
@@ -203,7 +209,7 @@ __global__ void __launch_bounds__(256) cand_quant_kernel(
   const int rb_per_alpha = (int)(out_pad / kCandRows);
   const int a = (int)(blockIdx.x / rb_per_alpha);
   const int64_t o0 = (int64_t)(blockIdx.x - (int64_t)a * rb_per_alpha) * kCandRows;
-  float sv[8], iv[8];
+  float sv[8], iv[8], rv[8] = {1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f};
   if (j_ok) {
     const float4 *sp = reinterpret_cast<const float4 *>(s + (int64_t)a * in + j0);
     const float4 *ip = reinterpret_cast<const float4 *>(inv_s + (int64_t)a * in + j0);
@@ -212,6 +218,14 @@ __global__ void __launch_bounds__(256) cand_quant_kernel(
     sv[4] = s1.x; sv[5] = s1.y; sv[6] = s1.z; sv[7] = s1.w;
     iv[0] = i0.x; iv[1] = i0.y; iv[2] = i0.z; iv[3] = i0.w;
     iv[4] = i1.x; iv[5] = i1.y; iv[6] = i1.z; iv[7] = i1.w;
+    if (rch) {  // Gram form: d~ = r_j (deq/s - w)
+      const float4 r0 = __ldg(reinterpret_cast<const float4 *>(rch + j0));
+      const float4 r1 = __ldg(reinterpret_cast<const float4 *>(rch + j0) + 1);
+      rv[0] = r0.x; rv[1] = r0.y; rv[2] = r0.z; rv[3] = r0.w;
+      rv[4] = r1.x; rv[5] = r1.y; rv[6] = r1.z; rv[7] = r1.w;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) iv[e] *= rv[e];
+    }
   } else {
 #pragma unroll
     for (int e = 0; e < 8; ++e) { sv[e] = 1.0f; iv[e] = 1.0f; }
@@ -255,7 +269,8 @@ __global__ void __launch_bounds__(256) cand_quant_kernel(
       // fp32 (the result is rounded to fp16 next)
       const float2 qz = quant_qz2(wt[h], g);
       float2 d2 = __ffma2_rn(__fmul2_rn(qz, make_float2(dk, dk)), make_float2(iv[2 * h], iv[2 * h + 1]),
-                             __fmul2_rn(make_float2(w[2 * h], w[2 * h + 1]), make_float2(-two_k, -two_k)));
+                             __fmul2_rn(make_float2(w[2 * h], w[2 * h + 1]),
+                                        make_float2(-two_k * rv[2 * h], -two_k * rv[2 * h + 1])));
       if (!live) d2 = make_float2(0.0f, 0.0f);
       const __half2 hv = __floats2half2_rn(d2.x, d2.y);
       packed[h] = *reinterpret_cast<const uint32_t *>(&hv);
@@ -267,11 +282,12 @@ __global__ void __launch_bounds__(256) cand_quant_kernel(
 }
 
 cudaError_t launch_cand_quant(const __half *W, int64_t out, int64_t in, int64_t out_pad,
-                              const float *s, const float *inv_s, int n_alpha, int group, int w_bit,
-                              const DevStatus *st, __half *dW, int num_sms, cudaStream_t stream) {
+                              const float *s, const float *inv_s, const float *r, int n_alpha,
+                              int group, int w_bit, const DevStatus *st, __half *dW, int num_sms,
+                              cudaStream_t stream) {
   (void)num_sms;
   dim3 grid((unsigned)(n_alpha * (out_pad / kCandRows)), (unsigned)((in + 255) / 256));
-  cand_quant_kernel<<<grid, 256, 0, stream>>>(W, out, in, out_pad, s, inv_s, group,
+  cand_quant_kernel<<<grid, 256, 0, stream>>>(W, out, in, out_pad, s, inv_s, r, group,
                                               (float)((1 << w_bit) - 1), st, dW);
   return cudaGetLastError();
 }

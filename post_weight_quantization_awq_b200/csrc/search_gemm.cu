@@ -299,20 +299,20 @@ cudaError_t launch_search_gemm(const __half *X, int64_t ldx, const __half *dW,
 }
 
 // ---------------------------------------------------------------------------
-// K5 — MSE_i = (sum of candidate i's partials) * 2^-2k / (T out).  One block
+// K5 — MSE_i = (sum of candidate i's `per` partials, stored contiguously)
+// * 2^-2k / (T out).  One block
 // per candidate sums its partials in a fixed order (bitwise reproducible);
 // the last block to finish picks best = the first index of the smallest MSE
 // and copies s_best = s_grid[best].
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024) mse_argmin_kernel(
-    const double *__restrict__ partials, int n_alpha, int nb_per_alpha, int num_m, int64_t T,
+    const double *__restrict__ partials, int n_alpha, size_t per, int64_t T,
     int64_t out, const float *__restrict__ s_grid, int64_t in, DevStatus *st,
     double *__restrict__ mse, int32_t *__restrict__ best_idx, float *__restrict__ s_best) {
   __shared__ double red[1024];
   __shared__ int last_sh, best_sh;
   const int i = blockIdx.x;
   const int k = kscale_from_wmax(__uint_as_float(__ldcg(&st->wmax_bits)));
-  const size_t per = (size_t)nb_per_alpha * num_m * 4;
   const double *p = partials + (size_t)i * per;
   double acc = 0.0;
   for (size_t idx = threadIdx.x; idx < per; idx += blockDim.x) acc += __ldcg(p + idx);
@@ -352,12 +352,11 @@ __global__ void __launch_bounds__(1024) mse_argmin_kernel(
   for (int64_t j = threadIdx.x; j < in; j += blockDim.x) s_best[j] = src[j];
 }
 
-cudaError_t launch_mse_argmin(const double *partials, int n_alpha, int nb_per_alpha, int num_m,
-                              int64_t T, int64_t out, const float *s_grid, int64_t in,
-                              DevStatus *st, double *mse, int32_t *best_idx, float *s_best,
-                              cudaStream_t stream) {
-  mse_argmin_kernel<<<n_alpha, 1024, 0, stream>>>(partials, n_alpha, nb_per_alpha, num_m, T, out,
-                                                  s_grid, in, st, mse, best_idx, s_best);
+cudaError_t launch_mse_argmin(const double *partials, int n_alpha, size_t per_alpha, int64_t T,
+                              int64_t out, const float *s_grid, int64_t in, DevStatus *st,
+                              double *mse, int32_t *best_idx, float *s_best, cudaStream_t stream) {
+  mse_argmin_kernel<<<n_alpha, 1024, 0, stream>>>(partials, n_alpha, per_alpha, T, out, s_grid, in,
+                                                  st, mse, best_idx, s_best);
   return cudaGetLastError();
 }
 

@@ -283,3 +283,31 @@ def test_mlp_workload_sampled():
     _layer_parity(X, Wgu, 4, 20, 0, rows=rows)
     rows_d = torch.from_numpy(np.sort(rng.choice(Wd.shape[0], 512, replace=False)))
     _layer_parity(Xd[:8192].contiguous(), Wd, 4, 20, 0, rows=rows_d)
+
+
+# ------------------------------------------------------------------ Gram form
+@pytest.mark.parametrize("T,inn,out,w_bit", [(64, 128, 16, 4), (200, 384, 264, 3), (256, 512, 512, 4),
+                                             (2125, 1024, 768, 4)])
+def test_search_scale_gram_form_parity(T, inn, out, w_bit):
+    """The Gram-form search (sum_o dW_o^T X^T X dW_o, normalised G in fp16
+    hi + lo) against the oracle's MSE curve and selection."""
+    X, W = random_layer(T, inn, out, seed=T * 7 + inn + out)
+    cfg = awq.AwqConfig.make(w_bit=w_bit, search_form=awq.abi.SEARCH_GRAM)
+    g = gpu_search(X, W, cfg)
+    Xn, Wn = X.numpy(), W.numpy()
+    mse, _, _, S = O.search_scale(Xn, Wn, O.act_stats(Xn), w_bit, 128, 20)
+    check_mse(g["mse"], mse)
+    check_selection(g["best"], mse, "alpha (Gram form)")
+    assert np.array_equal(g["s_best"], S[g["best"]])
+
+
+def test_gram_form_matches_direct_form_full_q_proj():
+    """Both scoring forms on the full q_proj workload agree within the MSE bar
+    and pick the same alpha (unless tied within 1e-4)."""
+    d = workload_inputs(1)
+    _, X, W = d["groups"][0]
+    a = gpu_search(X, W, awq.AwqConfig.make())
+    b = gpu_search(X, W, awq.AwqConfig.make(search_form=awq.abi.SEARCH_GRAM))
+    rel = np.abs(a["mse"] - b["mse"]) / a["mse"]
+    assert rel.max() <= MSE_RTOL, rel.max()
+    check_selection(b["best"], a["mse"], "alpha (Gram vs direct)")
