@@ -343,6 +343,42 @@ def run_awq(args):
     h2d = X.numel() * 2 + W.numel() * 2
     d2h = sum(h.numel() * h.element_size() for h in host_out.values())
 
+    # ---- the Gram-form search on the same layer (same MSE, fewer flops), its
+    # own timing and flop count; the headline value above is the direct form
+    gram = None
+    if not args.no_gram_form:
+        cfg_g = awq.AwqConfig.make(w_bit=wl.w_bit, group_size=wl.group_size, n_alpha=wl.n_alpha,
+                                   n_clip=wl.n_clip, clip_min=0.5, search_form=awq.abi.SEARCH_GRAM)
+        ws_g = awq.alloc_workspace(T, inn, out, cfg_g, dev)
+
+        def step_g():
+            return awq.quantize_layer(Xd, Wd, cfg_g, ws=ws_g)
+
+        for _ in range(args.warmup):
+            step_g()
+        awq.awq_device_status(ws_g)
+        awq.profile_reset()
+        awq.profile_enable(True)
+        ms_g = timed_steps(step_g, args.steps, dist, timer, local)
+        awq.profile_enable(False)
+        awq.awq_device_status(ws_g)
+        kg = {}
+        for name in ("gram_full", "gram_score"):
+            tot, n = awq.profile_read(name)
+            kg[name] = tot / n if n else None
+        awq.profile_reset()
+        del ws_g
+        nb = (inn + 255) // 256  # G: the nb(nb+1)/2 upper 256x256 block pairs; scores: hi and lo
+        out128 = (out + 127) // 128 * 128
+        nt = inn // 128  # scores: the nt(nt+1)/2 upper 128-blocks of G~, hi and lo
+        flops_g = (2.0 * T * 256 * 256 * (nb * (nb + 1) // 2)
+                   + 2.0 * 2 * 128 * 128 * (nt * (nt + 1) // 2) * out128 * wl.n_alpha)
+        gram = {"value": round(ms_g / world, 3), "unit": UNIT, "ms_per_step": round(ms_g, 3),
+                "kernels_ms": {k: round(v, 4) for k, v in kg.items() if v},
+                "executed_flops_per_step": flops_g,
+                "note": "same MSE as the direct form (X^T X once, candidates scored against its "
+                        "normalised fp16 hi+lo form); flops counted as executed, not the direct form's"}
+
     # ---- CPU baseline (rank 0 at N=1 only)
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -391,6 +427,7 @@ def run_awq(args):
                 "d2h_bytes_per_step": d2h, "steps": e_steps},
         "gpu_launches": launches,
         "cpu_baseline": cpu,
+        "gram_form": gram,
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -457,6 +494,8 @@ def main(argv=None):
     ap.add_argument("--ref-row-fraction", type=float, default=0.125,
                     help="share of output rows the oracle runs on (then scaled)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-gram-form", action="store_true",
+                    help="skip the extra measurement of the Gram-form search")
     ap.add_argument("--workload", choices=("q_proj", "decoder"), default="q_proj",
                     help="q_proj: the headline workload; decoder: the 32-layer decoder "
                          "(--steps = layers timed)")

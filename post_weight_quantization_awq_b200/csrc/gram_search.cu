@@ -12,10 +12,11 @@
 // accumulator row with the matching tile of d~ itself.
 //
 //   gram_full_kernel   G = X^T X (fp32) on the tensor cores, one CTA per
-//                      128 x 128 block pair (bi <= bj), mirrored store;
+//                      256 x 256 block pair (bi <= bj), mirrored store;
 //   gram_norm_kernel   r and the hi/lo parts of G~;
-//   gram_score_kernel  persistent warp-specialised GEMM + dot epilogue, one
-//                      partial per (tile, warp).
+//   gram_score_kernel  persistent warp-specialised GEMM + dot epilogue over
+//                      the 128-block upper triangle of G~, one partial per
+//                      (tile, warp).
 #include <cuda.h>
 #include <cuda_fp16.h>
 #include <math.h>
@@ -26,14 +27,15 @@ namespace awq {
 
 namespace {
 constexpr int GF_T = 64;                          // tokens per stage
-constexpr int GF_STAGES = 6;
-constexpr uint32_t GF_BOX = 64 * GF_T * 2;        // 64 channels x 64 tokens fp16
-constexpr uint32_t GF_HALF = 2 * GF_BOX;          // one 128-channel panel
-constexpr uint32_t GF_STAGE = 2 * GF_HALF;        // A panel + B panel
+constexpr int GF_STAGES = 3;
+constexpr uint32_t GF_BOX = 64 * GF_T * 2;        // 64 channels x 64 tokens fp16 (8 KiB)
+constexpr uint32_t GF_A = 2 * GF_BOX;             // one 128-channel A half
+constexpr uint32_t GF_B = 4 * GF_BOX;             // the 256-channel B panel
+constexpr uint32_t GF_STAGE = 2 * GF_A + GF_B;    // 64 KiB
 constexpr uint32_t GF_DRAIN = 1u << 22;
-// kind::f16, fp16 A/B, fp32 D, A and B MN-major, N = 128, M = 128
+// kind::f16, fp16 A/B, fp32 D, A and B MN-major, N = 256, M = 128
 constexpr uint32_t IDESC_GF =
-    (1u << 4) | (1u << 15) | (1u << 16) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+    (1u << 4) | (1u << 15) | (1u << 16) | ((256u >> 3) << 17) | ((128u >> 4) << 24);
 
 struct __align__(8) GramFullTail {
   uint64_t full[GF_STAGES];
@@ -44,10 +46,13 @@ struct __align__(8) GramFullTail {
 };
 constexpr size_t kGramFullSmem = 1024 + GF_STAGES * GF_STAGE + sizeof(GramFullTail);
 
+// MN-major operand with 128-byte swizzling: 64 channels (128 B) per token row,
+// 8-row core groups 1024 B apart (SBO), consecutive 64-channel boxes GF_BOX
+// apart (LBO).
 __device__ __forceinline__ uint64_t desc_mn_sw128(uint32_t addr) {
   uint64_t d = 0;
   d |= (uint64_t)((addr >> 4) & 0x3FFFu);
-  d |= (uint64_t)((GF_BOX >> 4) & 0x3FFFu) << 16;  // second 64-channel half of the panel
+  d |= (uint64_t)((GF_BOX >> 4) & 0x3FFFu) << 16;
   d |= (uint64_t)(1024u >> 4) << 32;
   d |= (uint64_t)1u << 46;
   d |= (uint64_t)2u << 61;
@@ -68,6 +73,9 @@ __device__ __forceinline__ void tri_pair(int t, int nb, int &bi, int &bj) {
 }
 }  // namespace
 
+// One CTA per pair (BI <= BJ) of 256-channel blocks: A = X[:, 256 BI ...] as
+// two 128-channel halves (two TMEM accumulators of 256 columns), B =
+// X[:, 256 BJ ... + 256]; channels past `in` read as zero and are not stored.
 __global__ void __launch_bounds__(192, 1)
     gram_full_kernel(const __grid_constant__ CUtensorMap tmX, int64_t T, int nb,
                      float *__restrict__ G, int64_t in, DevStatus *st, uint32_t max_polls) {
@@ -92,7 +100,7 @@ __global__ void __launch_bounds__(192, 1)
   }
   if (warp == 0 && lane == 0) tma_prefetch_desc(&tmX);
   if (warp == 1) {
-    tmem_alloc(&tail->tmem_base, 128);
+    tmem_alloc(&tail->tmem_base, 512);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -115,10 +123,11 @@ __global__ void __launch_bounds__(192, 1)
         mbar_arrive_expect_tx(&tail->full[stage], GF_STAGE);
         const int32_t y = step * GF_T;
         uint8_t *dst = smem + stage * GF_STAGE;
-        tma_load_2d(dst, &tmX, &tail->full[stage], bi * 128, y);
-        tma_load_2d(dst + GF_BOX, &tmX, &tail->full[stage], bi * 128 + 64, y);
-        tma_load_2d(dst + GF_HALF, &tmX, &tail->full[stage], bj * 128, y);
-        tma_load_2d(dst + GF_HALF + GF_BOX, &tmX, &tail->full[stage], bj * 128 + 64, y);
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          tma_load_2d(dst + b * GF_BOX, &tmX, &tail->full[stage], bi * 256 + 64 * b, y);
+          tma_load_2d(dst + 2 * GF_A + b * GF_BOX, &tmX, &tail->full[stage], bj * 256 + 64 * b, y);
+        }
         issued |= 1u << stage;
         issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
         if (++stage == GF_STAGES) {
@@ -146,9 +155,13 @@ __global__ void __launch_bounds__(192, 1)
         tc_fence_after();
         const uint32_t base = smem_u32(smem + stage * GF_STAGE);
 #pragma unroll
-        for (int ks = 0; ks < GF_T / 16; ++ks)
-          tc_mma_f16(tmem_base, desc_mn_sw128(base + ks * 2048), desc_mn_sw128(base + GF_HALF + ks * 2048),
-                     IDESC_GF, (step | ks) != 0 ? 1u : 0u);
+        for (int ks = 0; ks < GF_T / 16; ++ks) {
+          const uint64_t bd = desc_mn_sw128(base + 2 * GF_A + ks * 2048);  // 16 token rows per step
+#pragma unroll
+          for (int h = 0; h < 2; ++h)
+            tc_mma_f16(tmem_base + h * 256, desc_mn_sw128(base + h * GF_A + ks * 2048), bd, IDESC_GF,
+                       (step | ks) != 0 ? 1u : 0u);
+        }
         issued_any = true;
         tc_commit(&tail->empty[stage]);
         if (++stage == GF_STAGES) {
@@ -171,19 +184,25 @@ __global__ void __launch_bounds__(192, 1)
       }
     } else {
       tc_fence_after();
-      const int m = q * 32 + lane;  // row within the block (channel bi*128 + m)
-      float *row = G + (int64_t)(bi * 128 + m) * in + bj * 128;
 #pragma unroll 1
-      for (int c = 0; c < 128; c += 32) {
-        float v[32];
-        tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)c, v);
-        tmem_ld_wait();
+      for (int h = 0; h < 2; ++h) {
+        const int64_t gi = (int64_t)bi * 256 + h * 128 + q * 32 + lane;  // this thread's channel
+#pragma unroll 1
+        for (int c = 0; c < 256; c += 32) {
+          float v[32];
+          tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * 256 + c), v);
+          tmem_ld_wait();
+          const int64_t gj0 = (int64_t)bj * 256 + c;
+          if (gi < in && gj0 < in) {  // in % 128 == 0: a 32-column run is all in or all out
+            float *row = G + gi * in + gj0;
 #pragma unroll
-        for (int e = 0; e < 32; e += 4)
-          *reinterpret_cast<float4 *>(row + c + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
-        if (bi != bj) {  // mirrored block: column m of rows bj*128 + c + e
+            for (int e = 0; e < 32; e += 4)
+              *reinterpret_cast<float4 *>(row + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
+            if (bi != bj) {  // mirrored block: column gi of rows gj0 + e
 #pragma unroll
-          for (int e = 0; e < 32; ++e) G[(int64_t)(bj * 128 + c + e) * in + bi * 128 + m] = v[e];
+              for (int e = 0; e < 32; ++e) G[(gj0 + e) * in + gi] = v[e];
+            }
+          }
         }
       }
     }
@@ -192,12 +211,16 @@ __global__ void __launch_bounds__(192, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, 128);
+    tmem_dealloc(tmem_base, 512);
   }
 }
 
 // r_j = sqrt(G_jj); G~_ij = G_ij / (r_i r_j) (0 where r_i r_j = 0) as fp16
 // hi + lo parts, row-major [in][in] (row j, channel i: the K-major B operand).
+// Because G~ is symmetric, the scores only read the 128-block upper triangle:
+// d^T G~ d = sum_J d_J^T G~_JJ d_J + 2 sum_{J<I} d_J^T G~_JI d_I, so blocks
+// right of the diagonal are stored doubled (exact) and blocks left of it are
+// never read (stored as zero).
 __global__ void gram_norm_kernel(const float *__restrict__ G, int64_t in, float *__restrict__ r,
                                  __half *__restrict__ ghi, __half *__restrict__ glo) {
   const int64_t n = in * in;
@@ -207,7 +230,9 @@ __global__ void gram_norm_kernel(const float *__restrict__ G, int64_t in, float 
     const float rj = sqrtf(fmaxf(__ldg(G + j * in + j), 0.0f));
     const float ri = sqrtf(fmaxf(__ldg(G + i * in + i), 0.0f));
     const float den = ri * rj;
-    const float v = den > 0.0f ? __ldg(G + idx) / den : 0.0f;
+    const int64_t bi = i >> 7, bj = j >> 7;
+    float v = den > 0.0f ? __ldg(G + idx) / den : 0.0f;
+    v = bi > bj ? 2.0f * v : (bi < bj ? 0.0f : v);
     const __half h = __float2half_rn(v);
     ghi[idx] = h;
     glo[idx] = __float2half_rn(v - __half2float(h));
@@ -218,7 +243,7 @@ __global__ void gram_norm_kernel(const float *__restrict__ G, int64_t in, float 
 cudaError_t launch_gram_full(const __half *X, int64_t T, int64_t in, int64_t ldx, float *G, float *r,
                              __half *ghi, __half *glo, DevStatus *st, uint32_t max_polls,
                              cudaStream_t stream) {
-  const int nb = (int)(in / 128);
+  const int nb = (int)((in + 255) / 256);
   CUtensorMap tm;
   cudaError_t e = make_tmap_f16_box(&tm, X, T, in, ldx, 64, GF_T);
   if (e != cudaSuccess) return e;
@@ -330,7 +355,7 @@ __global__ void __launch_bounds__(192, 1)
         tma_load_2d(sc + acc * SC + SC_ATOM, &tmA, &tail->cfull[acc], n_blk * SN + 64, m_blk * SM_);
         c_issued |= 1u << acc;
         c_parity = (c_parity & ~(1u << acc)) | (acc_phase << acc);
-        for (int kb = 0; kb < num_kb; ++kb) {
+        for (int kb = n_blk * (SN / SK); kb < num_kb; ++kb) {  // upper triangle of G~ only
           if (!mbar_wait_bounded(&tail->empty[stage], phase ^ 1u, max_polls, abort_flag)) {
             dev_fail(st, kDevTimeout, 0xD00u + stage);
             *abort_flag = 1;
@@ -367,6 +392,7 @@ __global__ void __launch_bounds__(192, 1)
       for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++it) {
         const int acc = it & 1;
         const uint32_t acc_phase = (it >> 1) & 1;
+        const int kb0 = (tile % num_n) * (SN / SK);
         if (!mbar_wait_bounded(&tail->tempty[acc], acc_phase ^ 1u, max_polls, abort_flag)) {
           dev_fail(st, kDevTimeout, 0xE00u + acc);
           *abort_flag = 1;
@@ -374,7 +400,7 @@ __global__ void __launch_bounds__(192, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * SN;
-        for (int kb = 0; kb < num_kb; ++kb) {
+        for (int kb = kb0; kb < num_kb; ++kb) {
           if (!mbar_wait_bounded(&tail->full[stage], phase, max_polls, abort_flag)) {
             dev_fail(st, kDevTimeout, 0xE10u + stage);
             *abort_flag = 1;
@@ -386,7 +412,8 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
           for (int k = 0; k < SK / 16; ++k) {
             const uint64_t ad = smem_desc_k_sw128(a + k * 32);
-            tc_mma_f16(d_tmem, ad, smem_desc_k_sw128(a + SA + k * 32), IDESC_S, (kb | k) != 0 ? 1u : 0u);
+            tc_mma_f16(d_tmem, ad, smem_desc_k_sw128(a + SA + k * 32), IDESC_S,
+                       (kb != kb0 || k != 0) ? 1u : 0u);
             tc_mma_f16(d_tmem, ad, smem_desc_k_sw128(a + SA + SB + k * 32), IDESC_S, 1u);
           }
           issued_any = true;
