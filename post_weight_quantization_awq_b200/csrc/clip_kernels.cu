@@ -263,7 +263,7 @@ struct __align__(16) ClipSmem {
   float bw[CT_MAXR][CT_RS];   // r_i w_i 2^e_row
   float s[G], ar[CT_RS], r[G];  // s_i, r_i / s_i (skewed), r_i = sqrt(G_ii)
   float rmx[CT_MAXR], rmn[CT_MAXR];
-  int rexp[CT_MAXR];
+  int rexp[2][CT_MAXR];  // per-row exponent; the argmin of a tile reads it during the next tile
   float epart[4][128];
   float ratio[128];  // clip ratio of each index
   uint64_t mma_bar;
@@ -343,6 +343,54 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
   uint32_t phase = 0;
   bool committed = false;
   int64_t k_cur = -1;
+  constexpr int kRowWarps = 12;  // warps 0..11 run the row pass; warps 12..15 the argmin
+  // W rows of the next tile, loaded by the row-pass warps one tile ahead
+  uint2 wpre[3] = {make_uint2(0u, 0u), make_uint2(0u, 0u), make_uint2(0u, 0u)};
+  auto load_rows = [&](int64_t it) {
+    const int64_t kk = it / n_tiles, oo = (it - kk * n_tiles) * R;
+#pragma unroll
+    for (int m = 0; m < 3; ++m) {
+      const int rr = warp + kRowWarps * m;
+      const int64_t o = oo + rr;
+      wpre[m] = (rr < R && o < out)
+                    ? __ldg(reinterpret_cast<const uint2 *>(W + o * in + kk * G + 4 * lane))
+                    : make_uint2(0u, 0u);
+    }
+  };
+  // first clip index with the smallest E of each row of a finished tile;
+  // four threads per row scan every fourth ratio, then combine (ties keep
+  // the lower index)
+  auto argmin_rows = [&](int64_t kk, int64_t oo, int b) {
+    const int t = tid - kRowWarps * 32, rr = t >> 2, part = t & 3;
+    const bool row_ok = rr < R && oo + rr < out;
+    float best = INFINITY;
+    int bc = 1 << 30;
+    if (row_ok) {
+      const float unscale = ldexpf(1.0f, -2 * S.rexp[b][rr]);
+      for (int c = part; c < n_clip; c += 4) {
+        const int p = rr * n_clip + c;
+        const float ev = ((S.epart[0][p] + S.epart[1][p]) + (S.epart[2][p] + S.epart[3][p])) * unscale;
+        if (err) err[((oo + rr) * n_groups + kk) * n_clip + c] = ev;
+        if (ev < best) {
+          best = ev;
+          bc = c;
+        }
+      }
+    }
+#pragma unroll
+    for (int off = 1; off < 4; off <<= 1) {
+      const float ob = __shfl_xor_sync(0xffffffffu, best, off);
+      const int oc = __shfl_xor_sync(0xffffffffu, bc, off);
+      if (ob < best || (ob == best && oc < bc)) {
+        best = ob;
+        bc = oc;
+      }
+    }
+    if (row_ok && part == 0) clip_idx[(oo + rr) * n_groups + kk] = (uint8_t)bc;
+  };
+  if (warp < kRowWarps && item_begin < item_end) load_rows(item_begin);
+  int64_t k_prev = -1, o0_prev = 0;
+  int buf = 0;
   for (int64_t item = item_begin; item < item_end; ++item) {
     const int64_t k = item / n_tiles;
     const int64_t o0 = (item - k * n_tiles) * R;
@@ -378,49 +426,53 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
       }
       // (the fence before the first MMA of this group publishes these stores)
     }
-    // ---- rows of this tile: s w, range, exponent of the d~ scaling, r w 2^e
-    for (int rr = warp; rr < R; rr += CT_THREADS / 32) {
-      const int64_t o = o0 + rr;
-      float w4[4] = {0.f, 0.f, 0.f, 0.f};
-      if (o < out) {
-        const uint2 wv = __ldg(reinterpret_cast<const uint2 *>(W + o * in + k * G + 4 * lane));
+    if (warp < kRowWarps) {
+      // ---- rows of this tile: s w, range, exponent of the d~ scaling, r w 2^e
+#pragma unroll
+      for (int m = 0; m < 3; ++m) {
+        const int rr = warp + kRowWarps * m;
+        if (rr >= R) break;
+        const uint2 wv = wpre[m];
         const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&wv.x));
         const float2 b = __half22float2(*reinterpret_cast<const __half2 *>(&wv.y));
-        w4[0] = a.x; w4[1] = a.y; w4[2] = b.x; w4[3] = b.y;
-      }
-      float mx = -INFINITY, mn = INFINITY, bmax = 0.0f, wt4[4];
+        const float w4[4] = {a.x, a.y, b.x, b.y};
+        float mx = -INFINITY, mn = INFINITY, bmax = 0.0f, wt4[4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int i = 4 * lane + e;
-        wt4[e] = __fmul_rn(S.s[i], w4[e]);
-        mx = fmaxf(mx, wt4[e]);
-        mn = fminf(mn, wt4[e]);
-        bmax = fmaxf(bmax, S.r[i] * fabsf(w4[e]));
-      }
+        for (int e = 0; e < 4; ++e) {
+          const int i = 4 * lane + e;
+          wt4[e] = __fmul_rn(S.s[i], w4[e]);
+          mx = fmaxf(mx, wt4[e]);
+          mn = fminf(mn, wt4[e]);
+          bmax = fmaxf(bmax, S.r[i] * fabsf(w4[e]));
+        }
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
-        bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, off));
-      }
-      // |d~_i| <= 2 r_i |w_i| (+ rounding): keep 2 bmax 2^e <= 2^14
-      int e2 = 0;
-      if (bmax > 0.0f) {
-        (void)frexpf(2.0f * bmax, &e2);
-        e2 = 14 - e2;
-      }
-      const float sc = ldexpf(1.0f, e2);
+        for (int off = 16; off > 0; off >>= 1) {
+          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+          mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+          bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, off));
+        }
+        // |d~_i| <= 2 r_i |w_i| (+ rounding): keep 2 bmax 2^e <= 2^14
+        int e2 = 0;
+        if (bmax > 0.0f) {
+          (void)frexpf(2.0f * bmax, &e2);
+          e2 = 14 - e2;
+        }
+        const float sc = ldexpf(1.0f, e2);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int i = 4 * lane + e;
-        S.wt[rr][sk(i)] = wt4[e];
-        S.bw[rr][sk(i)] = (S.r[i] * w4[e]) * sc;
+        for (int e = 0; e < 4; ++e) {
+          const int i = 4 * lane + e;
+          S.wt[rr][sk(i)] = wt4[e];
+          S.bw[rr][sk(i)] = (S.r[i] * w4[e]) * sc;
+        }
+        if (lane == 0) {
+          S.rmx[rr] = mx;
+          S.rmn[rr] = mn;
+          S.rexp[buf][rr] = e2;
+        }
       }
-      if (lane == 0) {
-        S.rmx[rr] = mx;
-        S.rmn[rr] = mn;
-        S.rexp[rr] = e2;
-      }
+      if (item + 1 < item_end) load_rows(item + 1);
+    } else if (k_prev >= 0) {
+      argmin_rows(k_prev, o0_prev, buf ^ 1);  // the previous tile, overlapping this row pass
     }
     __syncthreads();
     // ---- candidates: thread (pair p, quarter qq) writes channels 32qq..32qq+31:
@@ -433,7 +485,7 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
       uint8_t *ahi = S.a_hi + h * CT_ATOM, *alo = S.a_lo + h * CT_ATOM;
       if (valid) {
         const GroupQ g = group_params(S.rmx[rr], S.rmn[rr], S.ratio[c], qmax);
-        const float de = ldexpf(g.delta, S.rexp[rr]);  // exact power-of-two scaling
+        const float de = ldexpf(g.delta, S.rexp[buf][rr]);  // exact power-of-two scaling
         const float *wtr = S.wt[rr];
         const float *bwr = S.bw[rr];
 #pragma unroll 1
@@ -519,28 +571,12 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
     tc_fence_before();
     __syncthreads();
     if (*reinterpret_cast<volatile int *>(&S.abort_flag)) break;  // uniform across the CTA
-    // ---- per row: first clip index with the smallest E
-    if (tid < R) {
-      const int64_t o = o0 + tid;
-      if (o < out) {
-        const float unscale = ldexpf(1.0f, -2 * S.rexp[tid]);
-        float best = INFINITY;
-        int bc = 0;
-        for (int c = 0; c < n_clip; ++c) {
-          const int p = tid * n_clip + c;
-          const float ev =
-              ((S.epart[0][p] + S.epart[1][p]) + (S.epart[2][p] + S.epart[3][p])) * unscale;
-          if (err) err[(o * n_groups + k) * n_clip + c] = ev;
-          if (ev < best) {
-            best = ev;
-            bc = c;
-          }
-        }
-        clip_idx[o * n_groups + k] = (uint8_t)bc;
-      }
-    }
-    __syncthreads();
+    k_prev = k;
+    o0_prev = o0;
+    buf ^= 1;
   }
+  if (!*reinterpret_cast<volatile int *>(&S.abort_flag) && k_prev >= 0 && warp >= kRowWarps)
+    argmin_rows(k_prev, o0_prev, buf ^ 1);  // the last tile
   // after an abort the last MMAs may still be running: let them finish
   // (bounded) before the accumulator is freed
   if (tid == 0 && committed && *reinterpret_cast<volatile int *>(&S.abort_flag))
