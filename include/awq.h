@@ -75,7 +75,9 @@ enum { AWQ_SEARCH_DIRECT = 0, AWQ_SEARCH_GRAM = 1 };
  * quant_config ("05 — AWQ" §9: w_bit, q_group_size, zero_point). */
 typedef struct {
   int32_t w_bit;      /* 3 or 4                                                  */
-  int32_t group_size; /* 128 (the pages' g); must divide in                      */
+  int32_t group_size; /* 128 (the pages' g), or 32 / 64 ("AWQ and Activation-Aware
+                         Scaling", When it breaks, contrasts g = 32); must divide in;
+                         the clip search handles g = 128 only */
   int32_t zero_point; /* 1 = asymmetric min/max with zero point (only mode)      */
   int32_t n_alpha;    /* alpha grid size, 1..64; alpha_i = i/(n_alpha-1) ("05 — AWQ" §4: ~20) */
   int32_t n_clip;     /* clip grid size, 0 = no clip search, else 1..64          */
@@ -118,7 +120,8 @@ awq_status awq_scale_grid(const double *abar, int64_t in, int32_t n_alpha, float
  *   s_best   device fp32 [in]      (output) s of the selected alpha
  *   mse      device fp64 [n_alpha] (output) MSE_i
  *   best_idx device int32 [1]      (output) first index of the smallest MSE
- * Requires in % 64 == 0, out % 8 == 0, ldx % 8 == 0. */
+ * Requires out % 8 == 0, ldx % 8 == 0, and in % 64 == 0 (direct form) or
+ * in % 128 == 0 (Gram form). */
 awq_status awq_search_scale(const void *X, int64_t T, int64_t in, int64_t ldx,
                             const void *W, int64_t out, const double *abar,
                             const awq_config *cfg, void *ws, size_t ws_bytes,

@@ -99,8 +99,8 @@ awq_status check_cfg(const awq_config *cfg) {
   if (cfg->w_bit != 3 && cfg->w_bit != 4)
     return fail(AWQ_ERR_UNSUPPORTED, "w_bit=%d (3 or 4 supported)", cfg->w_bit);
   if (cfg->group_size <= 0) return fail(AWQ_ERR_INVALID_ARG, "group_size=%d", cfg->group_size);
-  if (cfg->group_size != 128)
-    return fail(AWQ_ERR_UNSUPPORTED, "group_size=%d (128 supported)", cfg->group_size);
+  if (cfg->group_size != 32 && cfg->group_size != 64 && cfg->group_size != 128)
+    return fail(AWQ_ERR_UNSUPPORTED, "group_size=%d (32, 64 or 128 supported)", cfg->group_size);
   if (cfg->zero_point != 1)
     return fail(AWQ_ERR_UNSUPPORTED, "zero_point=%d (asymmetric, 1, supported)", cfg->zero_point);
   if (cfg->n_alpha < 1 || cfg->n_alpha > 64)
@@ -232,7 +232,7 @@ size_t awq_workspace_size(int64_t T, int64_t in, int64_t out, const awq_config *
   if (check_cfg(cfg) != AWQ_OK) return 0;
   if (check_shape(T, in, out, cfg) != AWQ_OK) return 0;
   size_t need = scale_layout(T, in, out, cfg).end;
-  if (cfg->n_clip > 0) {
+  if (cfg->n_clip > 0 && cfg->group_size == 128) {
     size_t c = clip_layout(T, in).end;
     if (c > need) need = c;
   }
@@ -278,6 +278,10 @@ awq_status awq_search_scale(const void *X, int64_t T, int64_t in, int64_t ldx, c
   if ((st = check_x(X, in, ldx)) != AWQ_OK) return st;
   if (!W || !aligned(W, 16)) return fail(AWQ_ERR_INVALID_ARG, "W is NULL or not 16-byte aligned");
   if (!abar || !s_best || !mse || !best_idx) return fail(AWQ_ERR_INVALID_ARG, "an output pointer is NULL");
+  if (in % (cfg->search_form == AWQ_SEARCH_GRAM ? 128 : 64) != 0)
+    return fail(AWQ_ERR_UNSUPPORTED, "in=%lld: the %s search needs in %% %d == 0", (long long)in,
+                cfg->search_form == AWQ_SEARCH_GRAM ? "Gram-form" : "direct",
+                cfg->search_form == AWQ_SEARCH_GRAM ? 128 : 64);
   const ScaleWs L = scale_layout(T, in, out, cfg);
   if ((st = check_ws(ws, ws_bytes, L.end)) != AWQ_OK) return st;
   const int64_t tiles = (int64_t)L.num_m * L.nb_per_alpha * cfg->n_alpha;
@@ -355,6 +359,8 @@ awq_status awq_search_clip(const void *X, int64_t T, int64_t in, int64_t ldx, co
   awq_status st = check_cfg(cfg);
   if (st != AWQ_OK) return st;
   if (cfg->n_clip < 1) return fail(AWQ_ERR_INVALID_ARG, "n_clip=%d: clip search needs n_clip >= 1", cfg->n_clip);
+  if (cfg->group_size != 128)
+    return fail(AWQ_ERR_UNSUPPORTED, "group_size=%d: the clip search handles groups of 128", cfg->group_size);
   if ((st = check_shape(T, in, out, cfg)) != AWQ_OK) return st;
   if ((st = check_x(X, in, ldx)) != AWQ_OK) return st;
   if (!W || !aligned(W, 16)) return fail(AWQ_ERR_INVALID_ARG, "W is NULL or not 16-byte aligned");
@@ -507,6 +513,8 @@ extern "C" awq_status awq_search_clip_noalloc(const void *X, int64_t T, int64_t 
   awq_status st = check_cfg(cfg);
   if (st != AWQ_OK) return st;
   if (cfg->n_clip < 1) return fail(AWQ_ERR_INVALID_ARG, "n_clip=%d: clip search needs n_clip >= 1", cfg->n_clip);
+  if (cfg->group_size != 128)
+    return fail(AWQ_ERR_UNSUPPORTED, "group_size=%d: the clip search handles groups of 128", cfg->group_size);
   if ((st = check_shape(T, in, out, cfg)) != AWQ_OK) return st;
   if (in > kNoAllocMaxIn)
     return fail(AWQ_ERR_INVALID_ARG,

@@ -309,34 +309,40 @@ __device__ __forceinline__ float clip_ratio(int c, int n_clip, float clip_min) {
   return __double2float_rn(r);
 }
 
-// A block handles 64 output rows x one group of 128 input channels: the whole
-// W tile is fetched with independent 16-byte loads into shared memory, warps
-// quantise 8 rows each (4 channels per lane), codes are re-read transposed for
-// packing so every global store is contiguous.
+// A block handles 64 output rows x a tile of 128 input channels (the last
+// tile may be narrower; g in {32, 64, 128} divides both): the W tile is
+// fetched with independent 16-byte loads into shared memory, warps quantise
+// 8 rows each (4 channels per lane, a group's g/4 lanes reduce its range by
+// shuffles), codes are re-read transposed for packing so every global store
+// is contiguous.
+constexpr int kPackTile = 128;
+
 __global__ void __launch_bounds__(256) quant_pack_kernel(
-    const __half *__restrict__ W, int64_t out, int64_t in, const float *__restrict__ s,
+    const __half *__restrict__ W, int64_t out, int64_t in, int group, const float *__restrict__ s,
     const uint8_t *__restrict__ clip_idx, int n_clip, float clip_min, float qmax,
     int32_t *__restrict__ qweight, int32_t *__restrict__ qzeros, __half *__restrict__ scales) {
-  constexpr int G = 128;
-  __shared__ __align__(16) __half wsm[kPackRows][G + 8];
-  __shared__ uint8_t codes[kPackRows][G + 4];
-  __shared__ uint8_t zeros[kPackRows];
+  constexpr int TC = kPackTile;
+  __shared__ __align__(16) __half wsm[kPackRows][TC + 8];
+  __shared__ uint8_t codes[kPackRows][TC + 4];
+  __shared__ uint8_t zeros[kPackRows][TC / 32];
   __shared__ float ratios[64];  // clip ratio of each index (n_clip <= 64)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (clip_idx && threadIdx.x < n_clip) ratios[threadIdx.x] = clip_ratio(threadIdx.x, n_clip, clip_min);
-  const int k = blockIdx.y;  // group
+  const int64_t j_tile = (int64_t)blockIdx.y * TC;              // first channel of the tile
+  const int cols = (int)i64min(TC, in - j_tile);                // channels in this tile
   const int64_t o0 = (int64_t)blockIdx.x * kPackRows;
-  const int64_t groups = in / G;
+  const int64_t groups = in / group;
   const int rows_here = (int)i64min(kPackRows, out - o0);
+  const int gl = group / 4;                                     // lanes per group
   {
     uint4 v[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int c = threadIdx.x + 256 * u;  // 16-byte chunk: row c/16, channels 8*(c%16)
-      const int r = c >> 4;
-      v[u] = r < rows_here ? __ldg(reinterpret_cast<const uint4 *>(W + (o0 + r) * in + (int64_t)k * G +
-                                                                  8 * (c & 15)))
-                           : make_uint4(0u, 0u, 0u, 0u);
+      const int r = c >> 4, cc = 8 * (c & 15);
+      v[u] = (r < rows_here && cc < cols)
+                 ? __ldg(reinterpret_cast<const uint4 *>(W + (o0 + r) * in + j_tile + cc))
+                 : make_uint4(0u, 0u, 0u, 0u);
     }
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
@@ -344,11 +350,14 @@ __global__ void __launch_bounds__(256) quant_pack_kernel(
       *reinterpret_cast<uint4 *>(&wsm[c >> 4][8 * (c & 15)]) = v[u];
     }
   }
+  const bool lane_ok = lane * 4 < cols;
   float sv[4] = {1.0f, 1.0f, 1.0f, 1.0f};
-  if (s) {
-    const float4 f = __ldg(reinterpret_cast<const float4 *>(s + (int64_t)k * G + lane * 4));
+  if (s && lane_ok) {
+    const float4 f = __ldg(reinterpret_cast<const float4 *>(s + j_tile + lane * 4));
     sv[0] = f.x; sv[1] = f.y; sv[2] = f.z; sv[3] = f.w;
   }
+  const int gi = (lane * 4) / group;                            // group within the tile
+  const int64_t kg = j_tile / group + gi;                       // global group index
   __syncthreads();
   for (int r = warp; r < rows_here; r += 8) {
     const int64_t o = o0 + r;
@@ -359,12 +368,12 @@ __global__ void __launch_bounds__(256) quant_pack_kernel(
                          __fmul_rn(sv[3], b.y)};
     float mx = fmaxf(fmaxf(wt[0], wt[1]), fmaxf(wt[2], wt[3]));
     float mn = fminf(fminf(wt[0], wt[1]), fminf(wt[2], wt[3]));
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
+    for (int off = gl >> 1; off > 0; off >>= 1) {
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
       mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
     }
-    const float r32 = clip_idx ? ratios[clip_idx[o * groups + k]] : 1.0f;
+    if (!lane_ok) continue;  // past the last channel (its lanes form whole groups)
+    const float r32 = clip_idx ? ratios[clip_idx[o * groups + kg]] : 1.0f;
     const GroupQ g = group_params(mx, mn, r32, qmax);
     uchar4 c4;
     c4.x = (uint8_t)quant_code(wt[0], g);
@@ -372,27 +381,30 @@ __global__ void __launch_bounds__(256) quant_pack_kernel(
     c4.z = (uint8_t)quant_code(wt[2], g);
     c4.w = (uint8_t)quant_code(wt[3], g);
     *reinterpret_cast<uchar4 *>(&codes[r][lane * 4]) = c4;
-    if (lane == 0) {
-      zeros[r] = (uint8_t)g.zero;
-      scales[(int64_t)k * out + o] = __float2half_rn(g.delta);
+    if ((lane & (gl - 1)) == 0) {  // first lane of the group
+      zeros[r][gi] = (uint8_t)g.zero;
+      scales[kg * out + o] = __float2half_rn(g.delta);
     }
   }
   __syncthreads();
   const int64_t words_per_row = out / 8;
   const int o8_here = rows_here / 8;  // out % 8 == 0
-  for (int t = threadIdx.x; t < G * 8; t += 256) {
+  for (int t = threadIdx.x; t < cols * 8; t += 256) {
     const int o8 = t & 7, jj = t >> 3;
     if (o8 >= o8_here) continue;
     uint32_t word = 0;
 #pragma unroll
     for (int e = 0; e < 8; ++e) word |= (uint32_t)codes[o8 * 8 + e][jj] << (4 * e);
-    qweight[((int64_t)k * G + jj) * words_per_row + o0 / 8 + o8] = (int32_t)word;
+    qweight[(j_tile + jj) * words_per_row + o0 / 8 + o8] = (int32_t)word;
   }
-  if (threadIdx.x < o8_here) {
+  const int g_here = cols / group;
+  for (int t = threadIdx.x; t < g_here * 8; t += 256) {
+    const int o8 = t & 7, gg = t >> 3;
+    if (o8 >= o8_here) continue;
     uint32_t word = 0;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) word |= (uint32_t)zeros[threadIdx.x * 8 + e] << (4 * e);
-    qzeros[(int64_t)k * words_per_row + o0 / 8 + threadIdx.x] = (int32_t)word;
+    for (int e = 0; e < 8; ++e) word |= (uint32_t)zeros[o8 * 8 + e][gg] << (4 * e);
+    qzeros[(j_tile / group + gg) * words_per_row + o0 / 8 + o8] = (int32_t)word;
   }
 }
 
@@ -400,9 +412,9 @@ cudaError_t launch_quant_pack(const __half *W, int64_t out, int64_t in, const fl
                               const uint8_t *clip_idx, int group, int w_bit, int n_clip,
                               float clip_min, int32_t *qweight, int32_t *qzeros, __half *scales,
                               cudaStream_t stream) {
-  if (group != 128) return cudaErrorInvalidValue;
-  dim3 grid((unsigned)((out + kPackRows - 1) / kPackRows), (unsigned)(in / group));
-  quant_pack_kernel<<<grid, 256, 0, stream>>>(W, out, in, s, clip_idx, n_clip, clip_min,
+  if (group != 32 && group != 64 && group != 128) return cudaErrorInvalidValue;
+  dim3 grid((unsigned)((out + kPackRows - 1) / kPackRows), (unsigned)((in + kPackTile - 1) / kPackTile));
+  quant_pack_kernel<<<grid, 256, 0, stream>>>(W, out, in, group, s, clip_idx, n_clip, clip_min,
                                               (float)((1 << w_bit) - 1), qweight, qzeros, scales);
   return cudaGetLastError();
 }

@@ -40,7 +40,7 @@ def test_workspace_size_grows_with_the_problem():
 @pytest.mark.parametrize("kw,shape,status", [
     (dict(w_bit=5), (256, 512, 512), "AWQ_ERR_UNSUPPORTED"),
     (dict(w_bit=0), (256, 512, 512), "AWQ_ERR_INVALID_ARG"),
-    (dict(group_size=64), (256, 512, 512), "AWQ_ERR_UNSUPPORTED"),
+    (dict(group_size=96), (256, 576, 512), "AWQ_ERR_UNSUPPORTED"),
     (dict(zero_point=0), (256, 512, 512), "AWQ_ERR_UNSUPPORTED"),
     (dict(n_alpha=0), (256, 512, 512), "AWQ_ERR_INVALID_ARG"),
     (dict(n_clip=65), (256, 512, 512), "AWQ_ERR_INVALID_ARG"),
@@ -93,3 +93,19 @@ def test_errors_are_per_thread():
     t.start()
     t.join()
     assert "w_bit" in mine and seen == [""]
+
+
+def test_group_sizes_and_clip_limits():
+    """Groups of 32/64/128 for the search and packing; the clip search handles
+    128 only and says so before touching CUDA."""
+    for g in (32, 64, 128):
+        assert awq.awq_workspace_size(256, 512, 512, awq.AwqConfig.make(group_size=g)) > 0
+    cfg = awq.AwqConfig.make(group_size=64, n_clip=20)
+    st = abi.LIB.awq_search_clip(16, 256, 512, 512, 16, 512, None, ctypes.byref(cfg), 256, 1 << 30,
+                                 16, None, None)
+    assert abi.STATUS[st] == "AWQ_ERR_UNSUPPORTED" and "128" in abi.last_error()
+    # Gram form needs in % 128 == 0
+    cfg = awq.AwqConfig.make(group_size=64, search_form=abi.SEARCH_GRAM)
+    st = abi.LIB.awq_search_scale(16, 256, 192, 192, 16, 64, 16, ctypes.byref(cfg), 256, 1 << 30,
+                                  16, 16, 16, None)
+    assert abi.STATUS[st] == "AWQ_ERR_UNSUPPORTED" and "Gram" in abi.last_error()

@@ -311,3 +311,36 @@ def test_gram_form_matches_direct_form_full_q_proj():
     rel = np.abs(a["mse"] - b["mse"]) / a["mse"]
     assert rel.max() <= MSE_RTOL, rel.max()
     check_selection(b["best"], a["mse"], "alpha (Gram vs direct)")
+
+
+# ------------------------------------------------------------------ group sizes 32 / 64
+@pytest.mark.parametrize("T,inn,out,w_bit,group,form", [
+    (300, 256, 72, 4, 32, 0), (1200, 640, 264, 3, 64, 0), (500, 384, 136, 4, 32, 1), (257, 512, 512, 4, 64, 1)])
+def test_search_scale_other_group_sizes(T, inn, out, w_bit, group, form):
+    """Groups of 32 and 64 input channels ("AWQ and Activation-Aware Scaling",
+    When it breaks: the gain narrows at g = 32), both scoring forms."""
+    X, W = random_layer(T, inn, out, seed=T + inn + group)
+    cfg = awq.AwqConfig.make(w_bit=w_bit, group_size=group, search_form=form)
+    g = gpu_search(X, W, cfg)
+    Xn, Wn = X.numpy(), W.numpy()
+    mse, _, _, S = O.search_scale(Xn, Wn, O.act_stats(Xn), w_bit, group, 20)
+    check_mse(g["mse"], mse)
+    check_selection(g["best"], mse, f"alpha g={group}")
+    assert np.array_equal(g["s_best"], S[g["best"]])
+
+
+@pytest.mark.parametrize("out,inn,w_bit,group", [(72, 96, 4, 32), (136, 320, 3, 64), (512, 4096, 4, 32),
+                                                 (64, 192, 4, 64)])
+def test_quant_pack_other_group_sizes(out, inn, w_bit, group):
+    X, W = random_layer(16, inn, out, seed=out + inn)
+    s = O.scale_grid(O.act_stats(X.numpy()), O.alpha_grid(20))[11]
+    cfg = awq.AwqConfig.make(w_bit=w_bit, group_size=group)
+    qw = torch.empty((inn, out // 8), dtype=torch.int32, device="cuda")
+    qz = torch.empty((inn // group, out // 8), dtype=torch.int32, device="cuda")
+    sc = torch.empty((inn // group, out), dtype=torch.float16, device="cuda")
+    awq.awq_quant_pack(to_dev(W), torch.from_numpy(s).cuda(), None, cfg, qw, qz, sc)
+    torch.cuda.synchronize()
+    want = O.quant_pack(W.numpy(), s, None, w_bit, group)
+    for g_, w_, name in zip((qw.cpu().numpy(), qz.cpu().numpy(), sc.cpu().numpy()), want,
+                            ("qweight", "qzeros", "scales")):
+        assert np.array_equal(g_.view(np.uint8), w_.view(np.uint8)), name

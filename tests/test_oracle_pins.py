@@ -119,8 +119,8 @@ def _nearest_code_bruteforce(wt, delta, z, qmax):
     return best, margin
 
 
-@pytest.mark.parametrize("w_bit", [3, 4])
-def test_alpha0_is_plain_rtn_nearest_grid_point(w_bit):
+@pytest.mark.parametrize("w_bit,group", [(3, 128), (4, 128), (4, 32), (3, 64)])
+def test_alpha0_is_plain_rtn_nearest_grid_point(w_bit, group):
     """alpha = 0 reduces to plain round-to-nearest ("AWQ and Activation-Aware
     Scaling", Scaling instead of protecting): codes are the nearest in-range
     grid point, checked by exhaustive search in exact arithmetic."""
@@ -128,14 +128,14 @@ def test_alpha0_is_plain_rtn_nearest_grid_point(w_bit):
     abar = O.act_stats(X.numpy())
     S = O.scale_grid(abar, O.alpha_grid(20))
     Wn = W.numpy()
-    q0 = O.quantize_groups(Wn, S[0], 128, w_bit)
-    qr = O.quantize_groups(Wn, None, 128, w_bit)
+    q0 = O.quantize_groups(Wn, S[0], group, w_bit)
+    qr = O.quantize_groups(Wn, None, group, w_bit)
     assert np.array_equal(q0["q"], qr["q"]) and np.array_equal(q0["delta"], qr["delta"])
     qmax = 2 ** w_bit - 1
     checked = 0
     for o in range(Wn.shape[0]):
         for j in range(Wn.shape[1]):
-            k = j // 128
+            k = j // group
             code, margin = _nearest_code_bruteforce(qr["wt"][o, j], qr["delta"][o, k], int(qr["z"][o, k]), qmax)
             if margin < Fraction(1, 2 ** 18):
                 continue  # the fp32 quotient may round across a half-integer
@@ -356,6 +356,10 @@ def test_pack_roundtrip_and_storage_bits(golden):
     bits = 8.0 * (qw.nbytes + qz.nbytes + sc.nbytes) / Wg.numel()
     assert bits == float(hdr["bits_per_weight"])
     assert round(bits, 3) == float(hdr["printed"])
+    # the same closed form, 4 + 16/g + 4/g, at the other group sizes
+    for gs in (32, 64):
+        qw, qz, sc = O.quant_pack(Wg.numpy(), None, None, 4, gs)
+        assert 8.0 * (qw.nbytes + qz.nbytes + sc.nbytes) / Wg.numel() == 4 + 16 / gs + 4 / gs
 
 
 def test_fold_keeps_the_product():
