@@ -246,35 +246,32 @@ cudaError_t launch_gram_blocks(const __half *X, int64_t T, int64_t in, int64_t l
 // cross-thread reduction is needed.  The dropped A_lo G~_lo term is 2^-22 of E.
 // ---------------------------------------------------------------------------
 namespace {
-constexpr int CT_THREADS = 512;
+constexpr int CW_PROD = 8;                        // producer warps 0..7
+constexpr int CW_MMA = 8;                         // MMA warp
+constexpr int CW_EPI = 9;                         // epilogue warps 9..12
+constexpr int CT_THREADS = 13 * 32;
 constexpr int CT_MAXR = 32;                       // rows per tile at most
 constexpr uint32_t CT_ATOM = 128 * 128;           // bytes: 128 rows x 64 fp16
 constexpr uint32_t CT_OPND = 2 * CT_ATOM;         // one operand, K = 128
-constexpr int CT_RS = G + G / 32;                 // skewed row stride (floats)
 // kind::f16, fp16 A/B, fp32 D, K-major, N = 128, M = 128
 constexpr uint32_t IDESC_CLIP = (1u << 4) | ((128u >> 3) << 17) | ((128u >> 4) << 24);
+constexpr uint32_t CT_DRAIN = 1u << 22;
 
 struct __align__(16) ClipSmem {
-  uint8_t a_hi[CT_OPND];
-  uint8_t a_lo[CT_OPND];
-  uint8_t b_hi[CT_OPND];
+  uint8_t a_hi[2][CT_OPND];  // candidates of two tiles in flight
+  uint8_t a_lo[2][CT_OPND];
+  uint8_t b_hi[CT_OPND];     // G~ of the current group
   uint8_t b_lo[CT_OPND];
-  float wt[CT_MAXR][CT_RS];   // s_i w_i of the tile's rows (fp32, exact products)
-  float bw[CT_MAXR][CT_RS];   // r_i w_i 2^e_row
-  float s[G], ar[CT_RS], r[G];  // s_i, r_i / s_i (skewed), r_i = sqrt(G_ii)
-  float rmx[CT_MAXR], rmn[CT_MAXR];
-  int rexp[2][CT_MAXR];  // per-row exponent; the argmin of a tile reads it during the next tile
-  float epart[4][128];
+  float s[G], ar[G], r[G];  // s_i, r_i / s_i, r_i = sqrt(G_ii)
+  int rexp[2][CT_MAXR];
+  float epart[2][128];
   float ratio[128];  // clip ratio of each index
-  uint64_t mma_bar;
+  uint64_t a_full[2], a_empty[2], acc_full[2], acc_empty[2], mma_done;
   uint32_t tmem_base;
-  int abort_flag;  // a wait ran out: every thread leaves the tile loop together
+  int prod_ok, epi_ok;  // outcome of a group's wait, broadcast through its named barrier
+  int abort_flag;
 };
 constexpr size_t kClipSmemBytes = sizeof(ClipSmem) + 1024;
-
-// channel i of a skewed row: one extra float every 32 channels, so the four
-// threads that share a candidate (32 channels apart) hit different banks
-__device__ __forceinline__ int sk(int i) { return i + (i >> 5); }
 
 // byte offset of 16-byte chunk `c` (0..7) of row `row` inside a K-major
 // 128-byte-swizzled atom (8-row core groups of 1024 bytes)
@@ -300,6 +297,10 @@ __device__ __forceinline__ void fence_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+__device__ __forceinline__ void named_bar(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 __device__ __forceinline__ float clip_ratio_f(int c, int n_clip, float clip_min) {
   if (n_clip <= 1) return 1.0f;
   double r = 1.0 - (double)c * (1.0 - (double)clip_min) / (double)(n_clip - 1);
@@ -307,6 +308,9 @@ __device__ __forceinline__ float clip_ratio_f(int c, int n_clip, float clip_min)
 }
 }  // namespace
 
+// Warp-specialised pipeline over (group, row tile) items, two tiles in
+// flight: producers (warps 0-7) build tile t's candidates while the MMA warp
+// runs tile t-1 and the epilogue warps (9-12) score and pick tile t-2.
 __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
     const __half *__restrict__ W, int64_t out, int64_t in, const float *__restrict__ s,
     const float *__restrict__ Gall, float qmax, int n_clip, float clip_min, int rows_per_tile,
@@ -314,10 +318,10 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
   extern __shared__ uint8_t csm_raw[];
   ClipSmem &S = *reinterpret_cast<ClipSmem *>(
       (reinterpret_cast<uintptr_t>(csm_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  volatile int *abort_flag = &S.abort_flag;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int64_t n_groups = in / G;
   const int R = rows_per_tile;
-  const int npairs = R * n_clip;  // <= 128
   const int64_t n_tiles = (out + R - 1) / R;
   // this CTA's share of the (group, row tile) items, group-major, so a CTA
   // meets at most a few groups and builds each G~ once
@@ -326,13 +330,19 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
   const int64_t item_end = n_items * (blockIdx.x + 1) / gridDim.x;
 
   if (tid == 0) {
-    mbar_init(&S.mma_bar, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&S.a_full[b], CW_PROD);
+      mbar_init(&S.a_empty[b], 4);
+      mbar_init(&S.acc_full[b], 1);
+      mbar_init(&S.acc_empty[b], 4);
+    }
+    mbar_init(&S.mma_done, 1);
     S.abort_flag = 0;
     fence_mbar_init();
   }
   if (tid < n_clip) S.ratio[tid] = clip_ratio_f(tid, n_clip, clip_min);
-  if (warp == 0) {
-    tmem_alloc(&S.tmem_base, 128);
+  if (warp == CW_MMA) {
+    tmem_alloc(&S.tmem_base, 256);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -340,252 +350,314 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
   tc_fence_after();
   const uint32_t tmem_base = S.tmem_base;
 
-  uint32_t phase = 0;
-  bool committed = false;
-  int64_t k_cur = -1;
-  constexpr int kRowWarps = 12;  // warps 0..11 run the row pass; warps 12..15 the argmin
-  // W rows of the next tile, loaded by the row-pass warps one tile ahead
-  uint2 wpre[3] = {make_uint2(0u, 0u), make_uint2(0u, 0u), make_uint2(0u, 0u)};
-  auto load_rows = [&](int64_t it) {
-    const int64_t kk = it / n_tiles, oo = (it - kk * n_tiles) * R;
+  if (warp < CW_PROD) {
+    // ================================================================ producers
+    // Work unit: (row rr, 16-byte chunk ch of 8 channels, split sp of the
+    // clip ratios).  A thread keeps its chunk's s, r and r/s in registers
+    // for the whole group, reduces its row's range over the 16 lanes that
+    // share the row, and walks ratios sp, sp + nsp, ... < n_clip; lane l of
+    // the 16 computes the group parameters of its split's l-th ratio once,
+    // and the others take them by shuffle.
+    const int ptid = tid;  // 0..255
+    const int ch = ptid & 15;
+    const int nrc = 16 * R;                          // (row, chunk) slots
+    const int nsp = nrc >= CW_PROD * 32 ? 1 : (CW_PROD * 32) / nrc;
+    const int nunits = nrc * nsp;                    // a multiple of 16, <= 512
+    const int cper = (n_clip + nsp - 1) / nsp;       // ratios per split, <= 16
+    int64_t k_cur = -1;
+    float sv[8], rv[8], av[8];                       // s_i, r_i, r_i / s_i of the chunk
+    uint4 wpre[2];
+    auto load_rows = [&](int64_t it) {
+      const int64_t kk = it / n_tiles, oo = (it - kk * n_tiles) * R;
 #pragma unroll
-    for (int m = 0; m < 3; ++m) {
-      const int rr = warp + kRowWarps * m;
-      const int64_t o = oo + rr;
-      wpre[m] = (rr < R && o < out)
-                    ? __ldg(reinterpret_cast<const uint2 *>(W + o * in + kk * G + 4 * lane))
-                    : make_uint2(0u, 0u);
-    }
-  };
-  // first clip index with the smallest E of each row of a finished tile;
-  // four threads per row scan every fourth ratio, then combine (ties keep
-  // the lower index)
-  auto argmin_rows = [&](int64_t kk, int64_t oo, int b) {
-    const int t = tid - kRowWarps * 32, rr = t >> 2, part = t & 3;
-    const bool row_ok = rr < R && oo + rr < out;
-    float best = INFINITY;
-    int bc = 1 << 30;
-    if (row_ok) {
-      const float unscale = ldexpf(1.0f, -2 * S.rexp[b][rr]);
-      for (int c = part; c < n_clip; c += 4) {
-        const int p = rr * n_clip + c;
-        const float ev = ((S.epart[0][p] + S.epart[1][p]) + (S.epart[2][p] + S.epart[3][p])) * unscale;
-        if (err) err[((oo + rr) * n_groups + kk) * n_clip + c] = ev;
-        if (ev < best) {
-          best = ev;
-          bc = c;
+      for (int pass = 0; pass < 2; ++pass) {
+        const int u = warp * 32 + pass * CW_PROD * 32 + lane;
+        const int rr = (u >> 4) % R;
+        const int64_t o = oo + rr;
+        wpre[pass] = (u < nunits && o < out)
+                         ? __ldg(reinterpret_cast<const uint4 *>(W + o * in + kk * G + 8 * ch))
+                         : make_uint4(0u, 0u, 0u, 0u);
+      }
+    };
+    if (item_begin < item_end) load_rows(item_begin);
+    for (int64_t item = item_begin; item < item_end; ++item) {
+      const int t = (int)(item - item_begin);
+      const int b = t & 1;
+      const int64_t k = item / n_tiles;
+      const bool new_group = k != k_cur;
+      // buffer b is free once tile t-2 is scored; a new G~ also needs tile t-1 done
+      if (ptid == 0) {
+        int ok = mbar_wait_bounded(&S.a_empty[b], ((t >> 1) & 1) ^ 1u, max_polls, abort_flag);
+        if (ok && new_group && t >= 1)
+          ok = mbar_wait_bounded(&S.a_empty[b ^ 1], ((t - 1) >> 1) & 1, max_polls, abort_flag);
+        if (!ok) {
+          dev_fail(st, kDevTimeout, 0x910u);
+          *abort_flag = 1;
         }
+        S.prod_ok = ok;
       }
-    }
-#pragma unroll
-    for (int off = 1; off < 4; off <<= 1) {
-      const float ob = __shfl_xor_sync(0xffffffffu, best, off);
-      const int oc = __shfl_xor_sync(0xffffffffu, bc, off);
-      if (ob < best || (ob == best && oc < bc)) {
-        best = ob;
-        bc = oc;
-      }
-    }
-    if (row_ok && part == 0) clip_idx[(oo + rr) * n_groups + kk] = (uint8_t)bc;
-  };
-  if (warp < kRowWarps && item_begin < item_end) load_rows(item_begin);
-  int64_t k_prev = -1, o0_prev = 0;
-  int buf = 0;
-  for (int64_t item = item_begin; item < item_end; ++item) {
-    const int64_t k = item / n_tiles;
-    const int64_t o0 = (item - k * n_tiles) * R;
-    if (k != k_cur) {
-      // ---- group set-up: s, r = sqrt(G_ii), r/s, then G~ = G_ij / (r_i r_j)
-      // as hi + lo fp16, K-major swizzled (row j, channel i)
-      k_cur = k;
-      const float *Gk = Gall + k * G * G;
-      if (tid < G) {
-        const float sv = s ? s[k * G + tid] : 1.0f;
-        const float rv = sqrtf(fmaxf(Gk[tid * G + tid], 0.0f));
-        S.s[tid] = sv;
-        S.r[tid] = rv;
-        S.ar[sk(tid)] = rv / sv;
-      }
-      __syncthreads();
-      const int j = tid >> 2, qq = tid & 3;  // row j, channels 32 qq .. 32 qq + 31
-      const float rj = S.r[j];
-      const float *grow = Gk + (int64_t)j * G + 32 * qq;
+      named_bar(1, CW_PROD * 32);
+      if (!S.prod_ok) break;
+      if (new_group) {
+        // ---- group set-up: s, r = sqrt(G_ii), r/s, then G~ = G_ij / (r_i r_j)
+        // as hi + lo fp16, K-major swizzled (row j, channel i)
+        k_cur = k;
+        const float *Gk = Gall + k * G * G;
+        if (ptid < G) {
+          const float s0 = s ? s[k * G + ptid] : 1.0f;
+          const float r0 = sqrtf(fmaxf(Gk[ptid * G + ptid], 0.0f));
+          S.s[ptid] = s0;
+          S.r[ptid] = r0;
+          S.ar[ptid] = r0 / s0;
+        }
+        named_bar(1, CW_PROD * 32);
+        // row j, channels 64 h .. 64 h + 63; a warp shares h, so its
+        // swizzled 16-byte stores fall in distinct banks
+        const int j = ptid & 127, h = ptid >> 7;
+        const float rj = S.r[j];
+        const float *grow = Gk + (int64_t)j * G + 64 * h;
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        float v[8];
-        const float4 g0 = __ldg(reinterpret_cast<const float4 *>(grow + 8 * c));
-        const float4 g1 = __ldg(reinterpret_cast<const float4 *>(grow + 8 * c + 4));
-        const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+        for (int c = 0; c < 8; ++c) {
+          float v[8];
+          const float4 g0 = __ldg(reinterpret_cast<const float4 *>(grow + 8 * c));
+          const float4 g1 = __ldg(reinterpret_cast<const float4 *>(grow + 8 * c + 4));
+          const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float den = rj * S.r[64 * h + 8 * c + e];
+            v[e] = den > 0.0f ? gv[e] / den : 0.0f;
+          }
+          split_store8(S.b_hi + h * CT_ATOM, S.b_lo + h * CT_ATOM, sw128_off(j, c), v);
+        }
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          const float den = rj * S.r[32 * qq + 8 * c + e];
-          v[e] = den > 0.0f ? gv[e] / den : 0.0f;
+          sv[e] = S.s[8 * ch + e];
+          rv[e] = S.r[8 * ch + e];
+          av[e] = S.ar[8 * ch + e];
         }
-        const int h = qq >> 1, cc = (qq & 1) * 4 + c;
-        split_store8(S.b_hi + h * CT_ATOM, S.b_lo + h * CT_ATOM, sw128_off(j, cc), v);
       }
-      // (the fence before the first MMA of this group publishes these stores)
-    }
-    if (warp < kRowWarps) {
-      // ---- rows of this tile: s w, range, exponent of the d~ scaling, r w 2^e
+#pragma unroll 1
+      for (int pass = 0; pass < 2; ++pass) {
+        const int ub = warp * 32 + pass * CW_PROD * 32;  // warp-uniform
+        if (ub >= nunits) break;
+        const int u = ub + lane;
+        const bool live = u < nunits;
+        const int rr = (u >> 4) % R, sp = (u >> 4) / R;
+        // ---- this row's range (s w) and the exponent of the d~ scaling
+        const uint4 wv = pass ? wpre[1] : wpre[0];  // no dynamic register indexing
+        const uint32_t wr[4] = {wv.x, wv.y, wv.z, wv.w};
+        float2 wt[4];
+        float mx = -INFINITY, mn = INFINITY, bmax = 0.0f;
 #pragma unroll
-      for (int m = 0; m < 3; ++m) {
-        const int rr = warp + kRowWarps * m;
-        if (rr >= R) break;
-        const uint2 wv = wpre[m];
-        const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&wv.x));
-        const float2 b = __half22float2(*reinterpret_cast<const __half2 *>(&wv.y));
-        const float w4[4] = {a.x, a.y, b.x, b.y};
-        float mx = -INFINITY, mn = INFINITY, bmax = 0.0f, wt4[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int i = 4 * lane + e;
-          wt4[e] = __fmul_rn(S.s[i], w4[e]);
-          mx = fmaxf(mx, wt4[e]);
-          mn = fminf(mn, wt4[e]);
-          bmax = fmaxf(bmax, S.r[i] * fabsf(w4[e]));
+        for (int h = 0; h < 4; ++h) {
+          const float2 w2 = __half22float2(*reinterpret_cast<const __half2 *>(&wr[h]));
+          wt[h] = __fmul2_rn(make_float2(sv[2 * h], sv[2 * h + 1]), w2);
+          mx = fmaxf(mx, fmaxf(wt[h].x, wt[h].y));
+          mn = fminf(mn, fminf(wt[h].x, wt[h].y));
+          bmax = fmaxf(bmax, fmaxf(rv[2 * h] * fabsf(w2.x), rv[2 * h + 1] * fabsf(w2.y)));
         }
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
+        for (int off = 8; off > 0; off >>= 1) {
           mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
           mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
           bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, off));
         }
-        // |d~_i| <= 2 r_i |w_i| (+ rounding): keep 2 bmax 2^e <= 2^14
+        // |d~_i| <= r_i |w_i| (+ rounding): keep 2 bmax 2^e <= 2^14
         int e2 = 0;
         if (bmax > 0.0f) {
           (void)frexpf(2.0f * bmax, &e2);
           e2 = 14 - e2;
         }
+        if (live && ch == 0 && sp == 0) S.rexp[b][rr] = e2;
         const float sc = ldexpf(1.0f, e2);
+        float2 ae[4];  // (r_i / s_i) 2^e, exact power-of-two scaling
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int i = 4 * lane + e;
-          S.wt[rr][sk(i)] = wt4[e];
-          S.bw[rr][sk(i)] = (S.r[i] * w4[e]) * sc;
+        for (int h = 0; h < 4; ++h) ae[h] = __fmul2_rn(make_float2(av[2 * h], av[2 * h + 1]), make_float2(sc, sc));
+        // ---- parameters of ratio sp + nsp * (lane % 16), computed once
+        GroupQ gq;
+        {
+          const int cl = sp + nsp * ch;
+          gq = group_params(mx, mn, S.ratio[cl < n_clip ? cl : 0], qmax);
+          // every quotient of the group stays below 63 in magnitude, which the
+          // remainder test below needs; otherwise force the exact path
+          if (!(fmaxf(fabsf(mx), fabsf(mn)) * gq.rcp < 63.0f)) gq.half_lo = -1.0f;
         }
-        if (lane == 0) {
-          S.rmx[rr] = mx;
-          S.rmn[rr] = mn;
-          S.rexp[buf][rr] = e2;
+        const int p0 = rr * n_clip;
+        uint8_t *ahi = S.a_hi[b] + (ch >> 3) * CT_ATOM, *alo = S.a_lo[b] + (ch >> 3) * CT_ATOM;
+#pragma unroll 1
+        for (int jc = 0; jc < cper; ++jc) {
+          const float dl = __shfl_sync(0xffffffffu, gq.delta, jc, 16);
+          const float rc = __shfl_sync(0xffffffffu, gq.rcp, jc, 16);
+          const float hl = __shfl_sync(0xffffffffu, gq.half_lo, jc, 16);
+          const float zz = __shfl_sync(0xffffffffu, gq.zero, jc, 16);
+          const int c = sp + nsp * jc;
+          if (!live || c >= n_clip) continue;
+          // (q - z) = clamp(rne(wt / delta), -z, qmax - z), proposed from the
+          // approximate reciprocal and proven by the remainder
+          float2 kq[4];
+          float rmax = 0.0f;
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const float2 y = __fmul2_rn(wt[h], make_float2(rc, rc));
+            kq[h] = make_float2(rintf(y.x), rintf(y.y));
+            const float2 rem = __ffma2_rn(make_float2(-kq[h].x, -kq[h].y), make_float2(dl, dl), wt[h]);
+            rmax = fmaxf(rmax, fmaxf(fabsf(rem.x), fabsf(rem.y)));
+          }
+          if (!(rmax < hl)) {
+#pragma unroll
+            for (int h = 0; h < 4; ++h)
+              kq[h] = make_float2(rintf(__fdiv_rn(wt[h].x, dl)), rintf(__fdiv_rn(wt[h].y, dl)));
+          }
+          const float lo = -zz, hi = qmax - zz;
+          float v[8];
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            const float2 qz = make_float2(fminf(fmaxf(kq[h].x, lo), hi), fminf(fmaxf(kq[h].y, lo), hi));
+            // d~ 2^e = ((q - z) delta - s w) (r / s) 2^e
+            const float2 tq = __ffma2_rn(qz, make_float2(dl, dl), make_float2(-wt[h].x, -wt[h].y));
+            const float2 d2 = __fmul2_rn(tq, ae[h]);
+            v[2 * h] = d2.x;
+            v[2 * h + 1] = d2.y;
+          }
+          split_store8(ahi, alo, sw128_off(p0 + c, ch & 7), v);
         }
       }
       if (item + 1 < item_end) load_rows(item + 1);
-    } else if (k_prev >= 0) {
-      argmin_rows(k_prev, o0_prev, buf ^ 1);  // the previous tile, overlapping this row pass
+      fence_async_smem();  // generic-proxy writes (A and, on a new group, B) -> tensor cores
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.a_full[b]);
     }
-    __syncthreads();
-    // ---- candidates: thread (pair p, quarter qq) writes channels 32qq..32qq+31:
-    // d~_i 2^e = (q - z) (delta 2^e) (r_i / s_i) - r_i w_i 2^e
-    {
-      const int p = tid >> 2, qq = tid & 3;
-      const int rr = p / n_clip, c = p - rr * n_clip;
-      const bool valid = p < npairs && o0 + rr < out;
-      const int h = qq >> 1;
-      uint8_t *ahi = S.a_hi + h * CT_ATOM, *alo = S.a_lo + h * CT_ATOM;
-      if (valid) {
-        const GroupQ g = group_params(S.rmx[rr], S.rmn[rr], S.ratio[c], qmax);
-        const float de = ldexpf(g.delta, S.rexp[buf][rr]);  // exact power-of-two scaling
-        const float *wtr = S.wt[rr];
-        const float *bwr = S.bw[rr];
-#pragma unroll 1
-        for (int c4 = 0; c4 < 4; ++c4) {
-          float v[8];
-          const int i0 = 32 * qq + 8 * c4;
+  } else if (warp == CW_MMA) {
+    // ================================================================ MMA issuer
+    if (lane == 0) {
+      bool issued_any = false;
+      for (int64_t item = item_begin; item < item_end; ++item) {
+        const int t = (int)(item - item_begin);
+        const int b = t & 1;
+        const uint32_t ph = (t >> 1) & 1;
+        if (!mbar_wait_bounded(&S.a_full[b], ph, max_polls, abort_flag) ||
+            !mbar_wait_bounded(&S.acc_empty[b], ph ^ 1u, max_polls, abort_flag)) {
+          dev_fail(st, kDevTimeout, 0x920u);
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        // Y = A_hi B_hi + A_lo B_hi + A_hi B_lo
+        const uint32_t a_hi = smem_u32(S.a_hi[b]), a_lo = smem_u32(S.a_lo[b]);
+        const uint32_t b_hi = smem_u32(S.b_hi), b_lo = smem_u32(S.b_lo);
+        const uint32_t as[3] = {a_hi, a_lo, a_hi}, bs[3] = {b_hi, b_hi, b_lo};
+        const uint32_t d = tmem_base + (uint32_t)(b * 128);
 #pragma unroll
-          for (int e = 0; e < 8; e += 2) {
-            const int i = sk(i0 + e);  // i0 + e and i0 + e + 1 stay in one 32-channel run
-            const float2 qz = quant_qz2(make_float2(wtr[i], wtr[i + 1]), g);
-            const float2 d2 = __ffma2_rn(__fmul2_rn(qz, make_float2(de, de)),
-                                         make_float2(S.ar[i], S.ar[i + 1]),
-                                         make_float2(-bwr[i], -bwr[i + 1]));
-            v[e] = d2.x;
-            v[e + 1] = d2.y;
+        for (int tt = 0; tt < 3; ++tt)
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t koff = (uint32_t)(ks >> 2) * CT_ATOM + (uint32_t)(ks & 3) * 32u;
+            tc_mma_f16(d, smem_desc_k_sw128(as[tt] + koff), smem_desc_k_sw128(bs[tt] + koff),
+                       IDESC_CLIP, (tt | ks) != 0 ? 1u : 0u);
           }
-          split_store8(ahi, alo, sw128_off(p, (qq & 1) * 4 + c4), v);
-        }
-      } else {
-        const uint4 z = make_uint4(0u, 0u, 0u, 0u);
-#pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          *reinterpret_cast<uint4 *>(ahi + sw128_off(p, (qq & 1) * 4 + c4)) = z;
-          *reinterpret_cast<uint4 *>(alo + sw128_off(p, (qq & 1) * 4 + c4)) = z;
-        }
+        tc_commit(&S.acc_full[b]);
+        issued_any = true;
+      }
+      if (issued_any) {
+        tc_commit(&S.mma_done);
+        (void)mbar_wait_bounded(&S.mma_done, 0, CT_DRAIN, nullptr);
       }
     }
-    fence_async_smem();  // generic-proxy writes -> visible to the tensor cores
-    __syncthreads();
-    // ---- Y = A_hi B_hi + A_lo B_hi + A_hi B_lo
-    if (tid == 0) {
+  } else {
+    // ================================================================ epilogue
+    const int etid = tid - CW_EPI * 32;  // 0..127
+    const int q = warp & 3;              // TMEM lane quarter of this warp
+    const int p = q * 32 + lane;         // candidate (accumulator row)
+    for (int64_t item = item_begin; item < item_end; ++item) {
+      const int t = (int)(item - item_begin);
+      const int b = t & 1;
+      const uint32_t ph = (t >> 1) & 1;
+      const int64_t k = item / n_tiles;
+      const int64_t o0 = (item - k * n_tiles) * R;
+      if (etid == 0) {
+        // acc_full: the products are in TMEM; a_full (already complete) makes
+        // the producers' plain stores of A and the row data visible here
+        const int ok = mbar_wait_bounded(&S.acc_full[b], ph, max_polls, abort_flag) &&
+                       mbar_wait_bounded(&S.a_full[b], ph, max_polls, abort_flag);
+        if (!ok) {
+          dev_fail(st, kDevTimeout, 0x930u);
+          *abort_flag = 1;
+        }
+        S.epi_ok = ok;
+      }
+      named_bar(2, 128);
+      if (!S.epi_ok) break;
       tc_fence_after();
-      const uint32_t a_hi = smem_u32(S.a_hi), a_lo = smem_u32(S.a_lo);
-      const uint32_t b_hi = smem_u32(S.b_hi), b_lo = smem_u32(S.b_lo);
-      const uint32_t as[3] = {a_hi, a_lo, a_hi}, bs[3] = {b_hi, b_hi, b_lo};
+      // E = d~ . y over the 128 columns of this candidate's accumulator row
+      float2 e2a = make_float2(0.0f, 0.0f), e2b = make_float2(0.0f, 0.0f);
+#pragma unroll 1
+      for (int cb = 0; cb < 4; ++cb) {
+        float y[32];
+        tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * 128 + 32 * cb), y);
+        tmem_ld_wait();
+        const uint8_t *ahi = S.a_hi[b] + (cb >> 1) * CT_ATOM, *alo = S.a_lo[b] + (cb >> 1) * CT_ATOM;
 #pragma unroll
-      for (int t = 0; t < 3; ++t)
+        for (int cc = 0; cc < 4; ++cc) {
+          const int c = (cb & 1) * 4 + cc;
+          const uint4 hv = *reinterpret_cast<const uint4 *>(ahi + sw128_off(p, c));
+          const uint4 lv = *reinterpret_cast<const uint4 *>(alo + sw128_off(p, c));
+          const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w}, lw[4] = {lv.x, lv.y, lv.z, lv.w};
 #pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-          const uint32_t koff = (uint32_t)(ks >> 2) * CT_ATOM + (uint32_t)(ks & 3) * 32u;
-          tc_mma_f16(tmem_base, smem_desc_k_sw128(as[t] + koff), smem_desc_k_sw128(bs[t] + koff),
-                     IDESC_CLIP, (t | ks) != 0 ? 1u : 0u);
-        }
-      tc_commit(&S.mma_bar);
-    }
-    committed = true;
-    // ---- wait for Y, then E = d~ . y per candidate (warp: lane quarter q,
-    // column quarter cq)
-    int okw = 1;
-    if (lane == 0) okw = mbar_wait_bounded(&S.mma_bar, phase, max_polls, nullptr);
-    okw = __shfl_sync(0xffffffffu, okw, 0);
-    phase ^= 1u;
-    if (!okw) {
-      if (lane == 0) {
-        dev_fail(st, kDevTimeout, 0x900u);
-        *reinterpret_cast<volatile int *>(&S.abort_flag) = 1;
-      }
-    } else {
-      tc_fence_after();
-      const int q = warp & 3, cq = warp >> 2;
-      const int p = q * 32 + lane;
-      const uint8_t *ahi = S.a_hi + (cq >> 1) * CT_ATOM, *alo = S.a_lo + (cq >> 1) * CT_ATOM;
-      float y[32];
-      tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(32 * cq), y);
-      tmem_ld_wait();
-      float e = 0.0f;
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        const int c = (cq & 1) * 4 + cc;
-        const uint4 hv = *reinterpret_cast<const uint4 *>(ahi + sw128_off(p, c));
-        const uint4 lv = *reinterpret_cast<const uint4 *>(alo + sw128_off(p, c));
-        const uint32_t hw[4] = {hv.x, hv.y, hv.z, hv.w}, lw[4] = {lv.x, lv.y, lv.z, lv.w};
-#pragma unroll
-        for (int e2 = 0; e2 < 4; ++e2) {
-          const float2 fh = __half22float2(*reinterpret_cast<const __half2 *>(&hw[e2]));
-          const float2 fl = __half22float2(*reinterpret_cast<const __half2 *>(&lw[e2]));
-          e = fmaf(fh.x + fl.x, y[8 * cc + 2 * e2], e);
-          e = fmaf(fh.y + fl.y, y[8 * cc + 2 * e2 + 1], e);
+          for (int x = 0; x < 4; ++x) {
+            const float2 fh = __half22float2(*reinterpret_cast<const __half2 *>(&hw[x]));
+            const float2 fl = __half22float2(*reinterpret_cast<const __half2 *>(&lw[x]));
+            const float2 yy = make_float2(y[8 * cc + 2 * x], y[8 * cc + 2 * x + 1]);
+            if (x & 1)
+              e2b = __ffma2_rn(__fadd2_rn(fh, fl), yy, e2b);
+            else
+              e2a = __ffma2_rn(__fadd2_rn(fh, fl), yy, e2a);
+          }
         }
       }
-      S.epart[cq][p] = e;
+      const float e = (e2a.x + e2b.x) + (e2a.y + e2b.y);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.acc_empty[b]);
+      S.epart[b][p] = e;
+      named_bar(2, 128);
+      // ---- per row: first clip index with the smallest E; four threads per
+      // row scan every fourth ratio, then combine (ties keep the lower index)
+      {
+        const int rr = etid >> 2, part = etid & 3;
+        const bool row_ok = rr < R && o0 + rr < out;
+        float best = INFINITY;
+        int bc = 1 << 30;
+        if (row_ok) {
+          const float unscale = ldexpf(1.0f, -2 * S.rexp[b][rr]);
+          for (int c = part; c < n_clip; c += 4) {
+            const float ev = S.epart[b][rr * n_clip + c] * unscale;
+            if (err) err[((o0 + rr) * n_groups + k) * n_clip + c] = ev;
+            if (ev < best) {
+              best = ev;
+              bc = c;
+            }
+          }
+        }
+#pragma unroll
+        for (int off = 1; off < 4; off <<= 1) {
+          const float ob = __shfl_xor_sync(0xffffffffu, best, off);
+          const int oc = __shfl_xor_sync(0xffffffffu, bc, off);
+          if (ob < best || (ob == best && oc < bc)) {
+            best = ob;
+            bc = oc;
+          }
+        }
+        if (row_ok && part == 0) clip_idx[(o0 + rr) * n_groups + k] = (uint8_t)bc;
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.a_empty[b]);  // A, rows and partial sums of tile t reusable
     }
-    tc_fence_before();
-    __syncthreads();
-    if (*reinterpret_cast<volatile int *>(&S.abort_flag)) break;  // uniform across the CTA
-    k_prev = k;
-    o0_prev = o0;
-    buf ^= 1;
   }
-  if (!*reinterpret_cast<volatile int *>(&S.abort_flag) && k_prev >= 0 && warp >= kRowWarps)
-    argmin_rows(k_prev, o0_prev, buf ^ 1);  // the last tile
-  // after an abort the last MMAs may still be running: let them finish
-  // (bounded) before the accumulator is freed
-  if (tid == 0 && committed && *reinterpret_cast<volatile int *>(&S.abort_flag))
-    (void)mbar_wait_bounded(&S.mma_bar, phase ^ 1u, 1u << 22, nullptr);
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == CW_MMA) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, 128);
+    tmem_dealloc(tmem_base, 256);
   }
 }
 
