@@ -23,6 +23,9 @@ Sources (web pages about AWQ, Lin et al.):
 Readings where the pages are silent (each also listed in the design notes):
   * group-wise asymmetric min/max quantisation of g consecutive INPUT channels
     of one output row; zero point rounded and clamped to [0, 2^b - 1];
+  * without a zero point ([P4] §9 zero_point = False; [P4] §3 describes the
+    symmetric scheme only by its half-step error): step = max |wt| /
+    (2^(b-1) - 1), codes centred on z = 2^(b-1) in the same unsigned nibble;
   * every float step of the quantiser in fp32, correctly rounded, with
     round-half-to-even; guards d >= 1e-5 and abar >= 1e-4;
   * alpha_i = i / (n_alpha - 1); clip ratio r_c = 1 - c (1 - r_min)/(n_clip - 1)
@@ -112,14 +115,18 @@ def scale_grid(abar: np.ndarray, alphas: np.ndarray) -> np.ndarray:
 #     ([P4] §5 layout, §9 zero_point / q_group_size / w_bit)
 # --------------------------------------------------------------------------
 def quantize_groups(W: np.ndarray, s: Optional[np.ndarray], group: int, w_bit: int,
-                    ratio: Optional[np.ndarray] = None) -> dict:
+                    ratio: Optional[np.ndarray] = None, zero_point: bool = True) -> dict:
     """Quantise every (row o, group k) of diag(s) W, all in fp32.
 
     W [out, in] fp16; s [in] fp32 (None = 1); ratio [out, in/g] fp32 (None = 1).
     Per group: wt = RN32(s w); mx, mn = max, min of wt (each scaled by the
-    ratio when one is given); d = max(mx - mn, 1e-5); delta = d / (2^b - 1);
-    z = clamp(rne(-mn / delta), 0, 2^b - 1); q = clamp(rne(wt / delta) + z,
-    0, 2^b - 1); deq = (q - z) delta.
+    ratio when one is given); then
+      zero_point (asymmetric, [P4] §9 zero_point = True):
+        d = max(mx - mn, 1e-5); delta = d / (2^b - 1);
+        z = clamp(rne(-mn / delta), 0, 2^b - 1);
+      no zero point (the symmetric scheme of [P4] §3, codes centred on 0):
+        d = max(|mx|, |mn|, 1e-5); delta = d / (2^(b-1) - 1); z = 2^(b-1);
+    q = clamp(rne(wt / delta) + z, 0, 2^b - 1); deq = (q - z) delta.
 
     Returns dict with q uint8 [out, in], z uint8 [out, in/g], delta fp32
     [out, in/g], deq fp32 [out, in], wt fp32 [out, in]."""
@@ -138,9 +145,14 @@ def quantize_groups(W: np.ndarray, s: Optional[np.ndarray], group: int, w_bit: i
         r = np.asarray(ratio, dtype=np.float32)
         mx = r * mx
         mn = r * mn
-    d = np.maximum(mx - mn, RANGE_FLOOR)
-    delta = d / qmax
-    z = np.clip(np.rint(-mn / delta), np.float32(0), qmax)
+    if zero_point:
+        d = np.maximum(mx - mn, RANGE_FLOOR)
+        delta = d / qmax
+        z = np.clip(np.rint(-mn / delta), np.float32(0), qmax)
+    else:
+        d = np.maximum(np.maximum(np.abs(mx), np.abs(mn)), RANGE_FLOOR)
+        delta = d / np.float32(2 ** (w_bit - 1) - 1)
+        z = np.full(delta.shape, np.float32(2 ** (w_bit - 1)), dtype=np.float32)
     q = np.clip(np.rint(wt3 / delta[:, :, None]) + z[:, :, None], np.float32(0), qmax)
     deq = (q - z[:, :, None]) * delta[:, :, None]
     assert wt.dtype == np.float32 and delta.dtype == np.float32 and deq.dtype == np.float32
@@ -191,8 +203,8 @@ def mse_gram(G: np.ndarray, delta: np.ndarray, T: int) -> float:
 
 
 def search_scale(X: np.ndarray, W: np.ndarray, abar: np.ndarray, w_bit: int, group: int,
-                 n_alpha: int, form: str = "gram", G: Optional[np.ndarray] = None
-                 ) -> Tuple[np.ndarray, int, np.ndarray, np.ndarray]:
+                 n_alpha: int, form: str = "gram", G: Optional[np.ndarray] = None,
+                 zero_point: bool = True) -> Tuple[np.ndarray, int, np.ndarray, np.ndarray]:
     """alpha-grid search ([P1], [P4] §4).
 
     For every alpha_i: s_i = abar^alpha_i, fake-quantise diag(s_i) W, score
@@ -205,7 +217,7 @@ def search_scale(X: np.ndarray, W: np.ndarray, abar: np.ndarray, w_bit: int, gro
         G = gram(X)
     mse = np.empty(n_alpha, dtype=np.float64)
     for i in range(n_alpha):
-        qd = quantize_groups(W, S[i], group, w_bit)
+        qd = quantize_groups(W, S[i], group, w_bit, zero_point=zero_point)
         delta = effective_error(W, S[i], qd["deq"])
         mse[i] = mse_gram(G, delta, T) if form == "gram" else mse_direct(X, delta)
     best = int(np.argmin(mse))  # first index attaining the minimum
@@ -231,8 +243,8 @@ def block_grams(X: np.ndarray, group: int) -> list:
 
 
 def search_clip(X: np.ndarray, W: np.ndarray, s: np.ndarray, w_bit: int, group: int,
-                n_clip: int, clip_min: float, Gk: Optional[list] = None
-                ) -> Tuple[np.ndarray, np.ndarray]:
+                n_clip: int, clip_min: float, Gk: Optional[list] = None,
+                zero_point: bool = True) -> Tuple[np.ndarray, np.ndarray]:
     """For every (row o, group k) pick the clip ratio whose fake-quantised
     group gives the smallest output error over all tokens,
     E_okc = sum_t (sum_{j in k} X_tj delta^(c)_oj)^2 = d^T (X_k^T X_k) d.
@@ -247,7 +259,7 @@ def search_clip(X: np.ndarray, W: np.ndarray, s: np.ndarray, w_bit: int, group: 
     E = np.empty((out, Gn, n_clip), dtype=np.float64)
     for c in range(n_clip):
         ratio = np.full((out, Gn), r[c], dtype=np.float32)
-        qd = quantize_groups(W, s, group, w_bit, ratio)
+        qd = quantize_groups(W, s, group, w_bit, ratio, zero_point)
         delta = effective_error(W, s, qd["deq"]).reshape(out, Gn, group)
         for k in range(Gn):
             dk = delta[:, k, :]
@@ -260,11 +272,12 @@ def search_clip(X: np.ndarray, W: np.ndarray, s: np.ndarray, w_bit: int, group: 
 # D8  final codes and packing                                ([P4] §5)
 # --------------------------------------------------------------------------
 def quant_pack(W: np.ndarray, s: Optional[np.ndarray], clip_idx: Optional[np.ndarray],
-               w_bit: int, group: int, n_clip: int = 1, clip_min: float = 0.5
-               ) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
+               w_bit: int, group: int, n_clip: int = 1, clip_min: float = 0.5,
+               zero_point: bool = True) -> Tuple[np.ndarray, np.ndarray, np.ndarray]:
     """Final codes with (s, r_clip) and the pages' storage layout:
     qweight [in, out/8] int32 with q[o, j] in nibble (o mod 8) of word
-    [j, o // 8]; qzeros [in/g, out/8] int32 likewise for z[o, k];
+    [j, o // 8]; qzeros [in/g, out/8] int32 likewise for z[o, k] (without a
+    zero point every z is 2^(b-1), so (q - z) scale dequantises either kind);
     scales [in/g, out] fp16 = RN16(delta[o, k])."""
     out, inn = W.shape
     assert out % 8 == 0
@@ -272,7 +285,7 @@ def quant_pack(W: np.ndarray, s: Optional[np.ndarray], clip_idx: Optional[np.nda
     if clip_idx is not None:
         r = clip_ratios(n_clip, clip_min).astype(np.float32)
         ratio = r[np.asarray(clip_idx, dtype=np.int64)]
-    qd = quantize_groups(W, s, group, w_bit, ratio)
+    qd = quantize_groups(W, s, group, w_bit, ratio, zero_point)
     q = qd["q"].astype(np.uint32)
     z = qd["z"].astype(np.uint32)
     qweight = np.zeros((inn, out // 8), dtype=np.uint32)

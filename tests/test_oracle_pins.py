@@ -81,16 +81,21 @@ def test_scale_grid_closed_forms():
 # --------------------------------------------------------------------------
 # D4  quantiser
 # --------------------------------------------------------------------------
-@pytest.mark.parametrize("name", ["quant_group_int4.txt", "quant_group_int3.txt", "quant_group_clip.txt"])
+HAND_WORKED = ["quant_group_int4.txt", "quant_group_int3.txt", "quant_group_clip.txt",
+               "quant_group_sym_int4.txt", "quant_group_sym_int3.txt", "quant_group_sym_clip.txt"]
+
+
+@pytest.mark.parametrize("name", HAND_WORKED)
 def test_quantiser_hand_worked(golden, name):
     hdr, rows = golden(name)
     g, b = int(hdr["group"]), int(hdr["w_bit"])
+    zp = bool(int(hdr.get("zero_point", 1)))
     W = _group_row({int(r[0]): float(r[1]) for r in rows}, g)
     ratio = None
     if "clip_index" in hdr:
         r = O.clip_ratios(int(hdr["n_clip"]), 0.5)[int(hdr["clip_index"])]
         ratio = np.full((1, 1), np.float32(r), dtype=np.float32)
-    qd = O.quantize_groups(W, None, g, b, ratio)
+    qd = O.quantize_groups(W, None, g, b, ratio, zero_point=zp)
     assert qd["delta"][0, 0] == np.float32(float(hdr["delta"]))
     assert int(qd["z"][0, 0]) == int(hdr["zero"])
     for r in rows:
@@ -119,8 +124,9 @@ def _nearest_code_bruteforce(wt, delta, z, qmax):
     return best, margin
 
 
-@pytest.mark.parametrize("w_bit,group", [(3, 128), (4, 128), (4, 32), (3, 64)])
-def test_alpha0_is_plain_rtn_nearest_grid_point(w_bit, group):
+@pytest.mark.parametrize("w_bit,group,zp", [(3, 128, True), (4, 128, True), (4, 32, True),
+                                             (3, 64, True), (4, 128, False), (3, 32, False)])
+def test_alpha0_is_plain_rtn_nearest_grid_point(w_bit, group, zp):
     """alpha = 0 reduces to plain round-to-nearest ("AWQ and Activation-Aware
     Scaling", Scaling instead of protecting): codes are the nearest in-range
     grid point, checked by exhaustive search in exact arithmetic."""
@@ -128,8 +134,8 @@ def test_alpha0_is_plain_rtn_nearest_grid_point(w_bit, group):
     abar = O.act_stats(X.numpy())
     S = O.scale_grid(abar, O.alpha_grid(20))
     Wn = W.numpy()
-    q0 = O.quantize_groups(Wn, S[0], group, w_bit)
-    qr = O.quantize_groups(Wn, None, group, w_bit)
+    q0 = O.quantize_groups(Wn, S[0], group, w_bit, zero_point=zp)
+    qr = O.quantize_groups(Wn, None, group, w_bit, zero_point=zp)
     assert np.array_equal(q0["q"], qr["q"]) and np.array_equal(q0["delta"], qr["delta"])
     qmax = 2 ** w_bit - 1
     checked = 0
@@ -161,6 +167,39 @@ def test_half_step_bound(w_bit):
         assert np.all(err <= bound)
 
 
+@pytest.mark.parametrize("w_bit", [3, 4])
+def test_half_step_bound_without_zero_point(w_bit):
+    """The symmetric scheme of "05 — AWQ" §3: every weight's rounding error
+    is at most half a step, with no clamping at ratio 1 and no condition on the
+    group's range (one-signed groups included); the codes stay in
+    [1, 2^b - 1], symmetric about z = 2^(b-1)."""
+    X, W = random_layer(64, 512, 64, seed=3)
+    Wn = W.numpy().copy()
+    Wn[:8] = np.abs(Wn[:8])  # one-signed rows
+    abar = O.act_stats(X.numpy())
+    S = O.scale_grid(abar, O.alpha_grid(20))
+    for i in (0, 7, 19):
+        qd = O.quantize_groups(Wn, S[i], 128, w_bit, zero_point=False)
+        err = np.abs(qd["deq"].astype(np.float64) - qd["wt"]).reshape(64, 4, 128)
+        bound = qd["delta"].astype(np.float64)[:, :, None] * (0.5 + 2.0 ** -18)
+        assert np.all(err <= bound)
+        assert np.all(qd["z"] == 2 ** (w_bit - 1))
+        assert qd["q"].min() >= 1 and qd["q"].max() <= 2 ** w_bit - 1
+        m = np.abs(qd["wt"]).reshape(64, 4, 128).max(2)
+        assert np.array_equal(qd["delta"], (m / np.float32(2 ** (w_bit - 1) - 1)).astype(np.float32))
+
+
+def test_constant_group_guard_without_zero_point():
+    W = _group_row({}, 128, fill=0.25)
+    qd = O.quantize_groups(W, None, 128, 4, zero_point=False)
+    assert qd["delta"][0, 0] == np.float32(np.float32(0.25) / np.float32(7))
+    assert np.all(qd["q"] == 15) and int(qd["z"][0, 0]) == 8
+    W0 = _group_row({}, 128, fill=0.0)
+    qd0 = O.quantize_groups(W0, None, 128, 4, zero_point=False)
+    assert qd0["delta"][0, 0] == np.float32(np.float32(1e-5) / np.float32(7))
+    assert np.all(qd0["q"] == 8) and np.all(qd0["deq"] == 0.0)
+
+
 def test_one_signed_group_clamps():
     """A group with min > 0: the zero point clamps to 0 and codes clamp to
     2^b - 1 (the range is not widened to include 0)."""
@@ -181,15 +220,16 @@ def test_constant_group_guard():
     assert int(qd["z"][0, 0]) == 0 and np.all(qd["q"] == 15)
 
 
-@pytest.mark.parametrize("k", [-3, 4])
-def test_power_of_two_scale_invariance(k):
+@pytest.mark.parametrize("k,zp", [(-3, True), (4, True), (-5, False), (3, False)])
+def test_power_of_two_scale_invariance(k, zp):
     """s -> 2^k s leaves codes and zeros unchanged and scales delta by 2^k
     exactly (every fp32 step commutes with an exact power-of-two scaling)."""
     X, W = random_layer(32, 256, 16, seed=5)
     abar = O.act_stats(X.numpy())
     s = O.scale_grid(abar, O.alpha_grid(20))[12]
-    a = O.quantize_groups(W.numpy(), s, 128, 4)
-    b = O.quantize_groups(W.numpy(), (s * np.float32(2.0 ** k)).astype(np.float32), 128, 4)
+    a = O.quantize_groups(W.numpy(), s, 128, 4, zero_point=zp)
+    b = O.quantize_groups(W.numpy(), (s * np.float32(2.0 ** k)).astype(np.float32), 128, 4,
+                          zero_point=zp)
     assert np.array_equal(a["q"], b["q"]) and np.array_equal(a["z"], b["z"])
     assert np.array_equal(a["delta"] * np.float32(2.0 ** k), b["delta"])
 
@@ -242,14 +282,16 @@ def test_mse_forms_match_pure_python_definition():
         assert O.mse_gram(O.gram(Xn), delta, Xn.shape[0]) == pytest.approx(want, rel=1e-10)
 
 
-@pytest.mark.parametrize("T,inn,out,w_bit", [(64, 128, 16, 4), (48, 256, 8, 3), (33, 256, 16, 4)])
-def test_search_bruteforce_tiny(T, inn, out, w_bit):
+@pytest.mark.parametrize("T,inn,out,w_bit,zp", [(64, 128, 16, 4, True), (48, 256, 8, 3, True),
+                                                (33, 256, 16, 4, True), (40, 256, 8, 4, False),
+                                                (24, 128, 16, 3, False)])
+def test_search_bruteforce_tiny(T, inn, out, w_bit, zp):
     X, W = random_layer(T, inn, out, seed=T + inn + out + w_bit)
     Xn, Wn = X.numpy(), W.numpy()
     abar = O.act_stats(Xn)
-    mse, best, s_best, S = O.search_scale(Xn, Wn, abar, w_bit, 128, 20, form="direct")
-    mse_g, best_g, _, _ = O.search_scale(Xn, Wn, abar, w_bit, 128, 20, form="gram")
-    lit = np.array([_literal_mse(Xn, Wn, S[i], O.quantize_groups(Wn, S[i], 128, w_bit)["deq"])
+    mse, best, s_best, S = O.search_scale(Xn, Wn, abar, w_bit, 128, 20, form="direct", zero_point=zp)
+    mse_g, best_g, _, _ = O.search_scale(Xn, Wn, abar, w_bit, 128, 20, form="gram", zero_point=zp)
+    lit = np.array([_literal_mse(Xn, Wn, S[i], O.quantize_groups(Wn, S[i], 128, w_bit, zero_point=zp)["deq"])
                     for i in range(20)])
     assert np.allclose(mse, lit, rtol=1e-10, atol=0)
     assert np.allclose(mse_g, lit, rtol=1e-10, atol=0)
@@ -299,16 +341,17 @@ def test_clip_ratio_one_is_unclipped():
         assert np.array_equal(a[key], b[key])
 
 
-def test_clip_search_bruteforce_tokens():
+@pytest.mark.parametrize("zp", [True, False])
+def test_clip_search_bruteforce_tokens(zp):
     T, inn, out, nc = 40, 256, 8, 6
     X, W = random_layer(T, inn, out, seed=13)
     Xn, Wn = X.numpy(), W.numpy()
     s = O.scale_grid(O.act_stats(Xn), O.alpha_grid(20))[8]
-    idx, E = O.search_clip(Xn, Wn, s, 4, 128, nc, 0.5)
+    idx, E = O.search_clip(Xn, Wn, s, 4, 128, nc, 0.5, zero_point=zp)
     r = O.clip_ratios(nc, 0.5).astype(np.float32)
     X64 = Xn.astype(np.float64)
     for c in range(nc):
-        qd = O.quantize_groups(Wn, s, 128, 4, np.full((out, 2), r[c], np.float32))
+        qd = O.quantize_groups(Wn, s, 128, 4, np.full((out, 2), r[c], np.float32), zero_point=zp)
         for o in range(out):
             for k in range(2):
                 sl = slice(128 * k, 128 * (k + 1))
@@ -377,3 +420,22 @@ def test_fold_keeps_the_product():
     # the subnormal range), carried back through the multiplication by s
     err = np.abs(r2.astype(np.float64) * s[:, None] - rows.astype(np.float64))
     assert np.all(err <= 2.0 ** -11 * np.abs(rows.astype(np.float64)) * 1.001 + 2.0 ** -25 * s[:, None])
+
+
+@pytest.mark.parametrize("w_bit", [3, 4])
+def test_pack_without_zero_point(w_bit):
+    """Without a zero point every qzeros nibble holds 2^(b-1) (0x88888888 per
+    word at INT4), the codes round-trip, and (q - z) scale gives back the
+    fp32 dequantised weights up to the fp16 rounding of the scale."""
+    X, W = random_layer(16, 256, 32, seed=17)
+    Wn = W.numpy()
+    s = O.scale_grid(O.act_stats(X.numpy()), O.alpha_grid(20))[6]
+    qw, qz, sc = O.quant_pack(Wn, s, None, w_bit, 128, zero_point=False)
+    nib = 2 ** (w_bit - 1)
+    assert np.all(O.unpack_nibbles(qz) == nib)
+    assert np.all(qz.view(np.uint32) == np.uint32(int(("%x" % nib) * 8, 16)))
+    q = O.unpack_nibbles(qw).astype(np.int64)  # [out, in]
+    qd = O.quantize_groups(Wn, s, 128, w_bit, zero_point=False)
+    assert np.array_equal(q, qd["q"])
+    deq16 = (q - nib) * np.repeat(sc.T.astype(np.float64), 128, axis=1)
+    assert np.allclose(deq16, qd["deq"], rtol=2.0 ** -10, atol=0)
