@@ -78,7 +78,12 @@ typedef struct {
   int32_t group_size; /* 128 (the pages' g), or 32 / 64 ("AWQ and Activation-Aware
                          Scaling", When it breaks, contrasts g = 32); must divide in;
                          the clip search handles g = 128 only */
-  int32_t zero_point; /* 1 = asymmetric min/max with zero point (only mode)      */
+  int32_t zero_point; /* 1 = asymmetric: step (max - min)/(2^b - 1), zero point
+                         z = clamp(rne(-min/step), 0, 2^b - 1) ("05 — AWQ" §9
+                         zero_point = True).  0 = symmetric, the scheme of
+                         "05 — AWQ" §3: step max|w|/(2^(b-1) - 1), z = 2^(b-1)
+                         for every group, so codes lie in [0, 2^b - 1] centred on
+                         z and qzeros holds 2^(b-1) in every nibble           */
   int32_t n_alpha;    /* alpha grid size, 1..64; alpha_i = i/(n_alpha-1) ("05 — AWQ" §4: ~20) */
   int32_t n_clip;     /* clip grid size, 0 = no clip search, else 1..64          */
   float clip_min;     /* smallest clip ratio, in (0, 1]; ("05 — AWQ" §4: 0.5)    */

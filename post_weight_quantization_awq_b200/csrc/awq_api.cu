@@ -101,8 +101,8 @@ awq_status check_cfg(const awq_config *cfg) {
   if (cfg->group_size <= 0) return fail(AWQ_ERR_INVALID_ARG, "group_size=%d", cfg->group_size);
   if (cfg->group_size != 32 && cfg->group_size != 64 && cfg->group_size != 128)
     return fail(AWQ_ERR_UNSUPPORTED, "group_size=%d (32, 64 or 128 supported)", cfg->group_size);
-  if (cfg->zero_point != 1)
-    return fail(AWQ_ERR_UNSUPPORTED, "zero_point=%d (asymmetric, 1, supported)", cfg->zero_point);
+  if (cfg->zero_point != 0 && cfg->zero_point != 1)
+    return fail(AWQ_ERR_INVALID_ARG, "zero_point=%d (1 asymmetric, 0 symmetric)", cfg->zero_point);
   if (cfg->n_alpha < 1 || cfg->n_alpha > 64)
     return fail(AWQ_ERR_INVALID_ARG, "n_alpha=%d (1..64)", cfg->n_alpha);
   if (cfg->n_clip < 0 || cfg->n_clip > 64)
@@ -319,7 +319,8 @@ awq_status awq_search_scale(const void *X, int64_t T, int64_t in, int64_t ldx, c
   {
     ProfScope p("cand_quant", s);
     AWQ_TRY_CUDA(launch_cand_quant(static_cast<const __half *>(W), out, in, L.out_pad, s_grid, inv_s, r,
-                                   cfg->n_alpha, cfg->group_size, cfg->w_bit, dst, dW, nsm, s),
+                                   cfg->n_alpha, cfg->group_size, cfg->w_bit, cfg->zero_point, dst,
+                                   dW, nsm, s),
                  "cand_quant launch");
   }
   if (gram) {
@@ -383,7 +384,7 @@ awq_status awq_search_clip(const void *X, int64_t T, int64_t in, int64_t ldx, co
   {
     ProfScope p("clip_eval", cs);
     AWQ_TRY_CUDA(launch_clip_eval(static_cast<const __half *>(W), out, in, s, Gk, cfg->group_size,
-                                  cfg->w_bit, cfg->n_clip, cfg->clip_min, clip_idx, err,
+                                  cfg->w_bit, cfg->zero_point, cfg->n_clip, cfg->clip_min, clip_idx, err,
                                   reinterpret_cast<DevStatus *>(base), poll_cap(),
                                   num_sms_current(), cs),
                  "clip_eval launch");
@@ -406,7 +407,8 @@ awq_status awq_quant_pack(const void *W, int64_t out, int64_t in, const float *s
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   ProfScope p("quant_pack", cs);
   AWQ_TRY_CUDA(launch_quant_pack(static_cast<const __half *>(W), out, in, s, clip_idx,
-                                 cfg->group_size, cfg->w_bit, cfg->n_clip, cfg->clip_min, qweight,
+                                 cfg->group_size, cfg->w_bit, cfg->zero_point, cfg->n_clip,
+                                 cfg->clip_min, qweight,
                                  qzeros, static_cast<__half *>(scales), cs),
                "quant_pack launch");
   return AWQ_OK;
@@ -558,7 +560,7 @@ extern "C" awq_status awq_search_clip_noalloc(const void *X, int64_t T, int64_t 
                          gpart, Gk, nullptr, 1u << 24, cs);
   if (e != cudaSuccess) return cuda_fail(e, "gram_blocks launch");
   e = launch_clip_eval(static_cast<const __half *>(W), out, in, s, Gk, cfg->group_size, cfg->w_bit,
-                       cfg->n_clip, cfg->clip_min, clip_idx, err, nullptr, 1u << 24,
+                       cfg->zero_point, cfg->n_clip, cfg->clip_min, clip_idx, err, nullptr, 1u << 24,
                        num_sms_current(), cs);
   if (e != cudaSuccess) return cuda_fail(e, "clip_eval launch");
   return AWQ_OK;

@@ -67,19 +67,31 @@ __device__ __forceinline__ float round_quotient(float x, float delta, float rcp,
 }
 
 // Range of one group after the optional clip ratio r32 (1 = no clip).
-__device__ __forceinline__ GroupQ group_params(float mx, float mn, float r32, float qmax) {
+// Asymmetric (zero point): delta = max(mx - mn, 1e-5) / (2^b - 1) and
+// z = clamp(rne(-mn / delta), 0, 2^b - 1).  Symmetric (sym, no zero point):
+// delta = max(|mx|, |mn|, 1e-5) / (2^(b-1) - 1) and z = 2^(b-1), so codes
+// are centred on z in the same unsigned range [0, 2^b - 1].
+__device__ __forceinline__ GroupQ group_params(float mx, float mn, float r32, float qmax, bool sym) {
   if (r32 != 1.0f) {
     mx = __fmul_rn(r32, mx);
     mn = __fmul_rn(r32, mn);
   }
-  const float d = fmaxf(__fsub_rn(mx, mn), 1e-5f);
   GroupQ g;
+  g.qmax = qmax;
+  if (sym) {
+    const float d = fmaxf(fmaxf(fabsf(mx), fabsf(mn)), 1e-5f);
+    g.delta = __fdiv_rn(d, 0.5f * (qmax - 1.0f));  // 2^(b-1) - 1, exact
+    g.rcp = rcp_approx(g.delta);
+    g.half_lo = __fmul_rn(g.delta, 0.4999847412109375f /* 0.5 - 2^-16 */);
+    g.zero = 0.5f * (qmax + 1.0f);  // 2^(b-1), exact
+    return g;
+  }
+  const float d = fmaxf(__fsub_rn(mx, mn), 1e-5f);
   g.delta = __fdiv_rn(d, qmax);
   g.rcp = rcp_approx(g.delta);
   g.half_lo = __fmul_rn(g.delta, 0.4999847412109375f /* 0.5 - 2^-16 */);
   const float z = round_quotient(-mn, g.delta, g.rcp, g.half_lo);
   g.zero = fminf(fmaxf(z, 0.0f), qmax);
-  g.qmax = qmax;
   return g;
 }
 

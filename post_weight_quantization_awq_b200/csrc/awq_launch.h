@@ -26,11 +26,12 @@ cudaError_t launch_wmax(const __half *W, int64_t n, int64_t in, const float *r, 
                         int num_sms, cudaStream_t stream);
 
 // K3: candidate effective errors dW[i][o][j] = RN16(2^k r_j (deq/s - w))
-// (r = NULL: r_j = 1), rows out..out_pad-1 zero.
+// (r = NULL: r_j = 1), rows out..out_pad-1 zero.  zero_point = 0 quantises
+// symmetrically (step max|w|/(2^(b-1)-1), z = 2^(b-1)).
 cudaError_t launch_cand_quant(const __half *W, int64_t out, int64_t in, int64_t out_pad,
                               const float *s, const float *inv_s, const float *r, int n_alpha,
-                              int group, int w_bit, const DevStatus *st, __half *dW, int num_sms,
-                              cudaStream_t stream);
+                              int group, int w_bit, int zero_point, const DevStatus *st, __half *dW,
+                              int num_sms, cudaStream_t stream);
 
 // K4: scored GEMM, partial sums of squares per (n-tile, m-tile, warp).
 struct SearchGemmShape {
@@ -69,15 +70,15 @@ cudaError_t launch_gram_blocks(const __half *X, int64_t T, int64_t in, int64_t l
                                uint32_t max_polls, cudaStream_t stream);
 // K6b: clip choice per (row, group), quadratic forms on the tensor cores.
 cudaError_t launch_clip_eval(const __half *W, int64_t out, int64_t in, const float *s,
-                             const float *G, int group, int w_bit, int n_clip, float clip_min,
-                             uint8_t *clip_idx, float *err, DevStatus *st, uint32_t max_polls,
-                             int num_sms, cudaStream_t stream);
+                             const float *G, int group, int w_bit, int zero_point, int n_clip,
+                             float clip_min, uint8_t *clip_idx, float *err, DevStatus *st,
+                             uint32_t max_polls, int num_sms, cudaStream_t stream);
 
 // K7: final codes + packing.
 cudaError_t launch_quant_pack(const __half *W, int64_t out, int64_t in, const float *s,
-                              const uint8_t *clip_idx, int group, int w_bit, int n_clip,
-                              float clip_min, int32_t *qweight, int32_t *qzeros, __half *scales,
-                              cudaStream_t stream);
+                              const uint8_t *clip_idx, int group, int w_bit, int zero_point,
+                              int n_clip, float clip_min, int32_t *qweight, int32_t *qzeros,
+                              __half *scales, cudaStream_t stream);
 
 // K8: v[j][:] = RN16(RN32(v[j][:]) / s_j).
 cudaError_t launch_fold(__half *v, int64_t rows, int64_t cols, const float *s, cudaStream_t stream);

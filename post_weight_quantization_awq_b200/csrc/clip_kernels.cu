@@ -313,7 +313,7 @@ __device__ __forceinline__ float clip_ratio_f(int c, int n_clip, float clip_min)
 // runs tile t-1 and the epilogue warps (9-12) score and pick tile t-2.
 __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
     const __half *__restrict__ W, int64_t out, int64_t in, const float *__restrict__ s,
-    const float *__restrict__ Gall, float qmax, int n_clip, float clip_min, int rows_per_tile,
+    const float *__restrict__ Gall, float qmax, int sym, int n_clip, float clip_min, int rows_per_tile,
     uint8_t *__restrict__ clip_idx, float *__restrict__ err, DevStatus *st, uint32_t max_polls) {
   extern __shared__ uint8_t csm_raw[];
   ClipSmem &S = *reinterpret_cast<ClipSmem *>(
@@ -477,7 +477,7 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
         GroupQ gq;
         {
           const int cl = sp + nsp * ch;
-          gq = group_params(mx, mn, S.ratio[cl < n_clip ? cl : 0], qmax);
+          gq = group_params(mx, mn, S.ratio[cl < n_clip ? cl : 0], qmax, sym != 0);
           // every quotient of the group stays below 63 in magnitude, which the
           // remainder test below needs; otherwise force the exact path
           if (!(fmaxf(fabsf(mx), fabsf(mn)) * gq.rcp < 63.0f)) gq.half_lo = -1.0f;
@@ -662,9 +662,9 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
 }
 
 cudaError_t launch_clip_eval(const __half *W, int64_t out, int64_t in, const float *s,
-                             const float *Gall, int group, int w_bit, int n_clip, float clip_min,
-                             uint8_t *clip_idx, float *err, DevStatus *st, uint32_t max_polls,
-                             int num_sms, cudaStream_t stream) {
+                             const float *Gall, int group, int w_bit, int zero_point, int n_clip,
+                             float clip_min, uint8_t *clip_idx, float *err, DevStatus *st,
+                             uint32_t max_polls, int num_sms, cudaStream_t stream) {
   if (group != G || n_clip < 1 || n_clip > 128) return cudaErrorInvalidValue;
   int R = 128 / n_clip;
   if (R > CT_MAXR) R = CT_MAXR;
@@ -675,7 +675,8 @@ cudaError_t launch_clip_eval(const __half *W, int64_t out, int64_t in, const flo
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)ctas);
   clip_tc_kernel<<<grid, CT_THREADS, kClipSmemBytes, stream>>>(
-      W, out, in, s, Gall, (float)((1 << w_bit) - 1), n_clip, clip_min, R, clip_idx, err, st,
+      W, out, in, s, Gall, (float)((1 << w_bit) - 1), zero_point ? 0 : 1, n_clip, clip_min, R,
+      clip_idx, err, st,
       max_polls);
   return cudaGetLastError();
 }

@@ -199,7 +199,7 @@ constexpr int kCandRows = 64;
 __global__ void __launch_bounds__(256) cand_quant_kernel(
     const __half *__restrict__ W, int64_t out, int64_t in, int64_t out_pad,
     const float *__restrict__ s, const float *__restrict__ inv_s, const float *__restrict__ rch,
-    int group, float qmax, const DevStatus *__restrict__ st, __half *__restrict__ dW) {
+    int group, float qmax, int sym, const DevStatus *__restrict__ st, __half *__restrict__ dW) {
   const int k = kscale_from_wmax(__uint_as_float(__ldg(&st->wmax_bits)));
   const float two_k = ldexpf(1.0f, k);
   const int lanes = group / 8;  // lanes per group (a power of two <= 32)
@@ -260,7 +260,7 @@ __global__ void __launch_bounds__(256) cand_quant_kernel(
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
       mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
     }
-    const GroupQ g = group_params(mx, mn, 1.0f, qmax);
+    const GroupQ g = group_params(mx, mn, 1.0f, qmax, sym != 0);
     const float dk = __fmul_rn(g.delta, two_k);  // exact: power-of-two scaling
     uint32_t packed[4];
 #pragma unroll
@@ -283,12 +283,12 @@ __global__ void __launch_bounds__(256) cand_quant_kernel(
 
 cudaError_t launch_cand_quant(const __half *W, int64_t out, int64_t in, int64_t out_pad,
                               const float *s, const float *inv_s, const float *r, int n_alpha,
-                              int group, int w_bit, const DevStatus *st, __half *dW, int num_sms,
-                              cudaStream_t stream) {
+                              int group, int w_bit, int zero_point, const DevStatus *st, __half *dW,
+                              int num_sms, cudaStream_t stream) {
   (void)num_sms;
   dim3 grid((unsigned)(n_alpha * (out_pad / kCandRows)), (unsigned)((in + 255) / 256));
   cand_quant_kernel<<<grid, 256, 0, stream>>>(W, out, in, out_pad, s, inv_s, r, group,
-                                              (float)((1 << w_bit) - 1), st, dW);
+                                              (float)((1 << w_bit) - 1), zero_point ? 0 : 1, st, dW);
   return cudaGetLastError();
 }
 
@@ -319,7 +319,7 @@ constexpr int kPackTile = 128;
 
 __global__ void __launch_bounds__(256) quant_pack_kernel(
     const __half *__restrict__ W, int64_t out, int64_t in, int group, const float *__restrict__ s,
-    const uint8_t *__restrict__ clip_idx, int n_clip, float clip_min, float qmax,
+    const uint8_t *__restrict__ clip_idx, int n_clip, float clip_min, float qmax, int sym,
     int32_t *__restrict__ qweight, int32_t *__restrict__ qzeros, __half *__restrict__ scales) {
   constexpr int TC = kPackTile;
   __shared__ __align__(16) __half wsm[kPackRows][TC + 8];
@@ -374,7 +374,7 @@ __global__ void __launch_bounds__(256) quant_pack_kernel(
     }
     if (!lane_ok) continue;  // past the last channel (its lanes form whole groups)
     const float r32 = clip_idx ? ratios[clip_idx[o * groups + kg]] : 1.0f;
-    const GroupQ g = group_params(mx, mn, r32, qmax);
+    const GroupQ g = group_params(mx, mn, r32, qmax, sym != 0);
     uchar4 c4;
     c4.x = (uint8_t)quant_code(wt[0], g);
     c4.y = (uint8_t)quant_code(wt[1], g);
@@ -409,13 +409,14 @@ __global__ void __launch_bounds__(256) quant_pack_kernel(
 }
 
 cudaError_t launch_quant_pack(const __half *W, int64_t out, int64_t in, const float *s,
-                              const uint8_t *clip_idx, int group, int w_bit, int n_clip,
-                              float clip_min, int32_t *qweight, int32_t *qzeros, __half *scales,
-                              cudaStream_t stream) {
+                              const uint8_t *clip_idx, int group, int w_bit, int zero_point,
+                              int n_clip, float clip_min, int32_t *qweight, int32_t *qzeros,
+                              __half *scales, cudaStream_t stream) {
   if (group != 32 && group != 64 && group != 128) return cudaErrorInvalidValue;
   dim3 grid((unsigned)((out + kPackRows - 1) / kPackRows), (unsigned)((in + kPackTile - 1) / kPackTile));
   quant_pack_kernel<<<grid, 256, 0, stream>>>(W, out, in, group, s, clip_idx, n_clip, clip_min,
-                                              (float)((1 << w_bit) - 1), qweight, qzeros, scales);
+                                              (float)((1 << w_bit) - 1), zero_point ? 0 : 1,
+                                              qweight, qzeros, scales);
   return cudaGetLastError();
 }
 

@@ -41,7 +41,7 @@ def test_workspace_size_grows_with_the_problem():
     (dict(w_bit=5), (256, 512, 512), "AWQ_ERR_UNSUPPORTED"),
     (dict(w_bit=0), (256, 512, 512), "AWQ_ERR_INVALID_ARG"),
     (dict(group_size=96), (256, 576, 512), "AWQ_ERR_UNSUPPORTED"),
-    (dict(zero_point=0), (256, 512, 512), "AWQ_ERR_UNSUPPORTED"),
+    (dict(zero_point=2), (256, 512, 512), "AWQ_ERR_INVALID_ARG"),
     (dict(n_alpha=0), (256, 512, 512), "AWQ_ERR_INVALID_ARG"),
     (dict(n_clip=65), (256, 512, 512), "AWQ_ERR_INVALID_ARG"),
     (dict(clip_min=0.0), (256, 512, 512), "AWQ_ERR_INVALID_ARG"),
