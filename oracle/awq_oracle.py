@@ -54,6 +54,7 @@ __all__ = [
     "effective_error",
     "gram",
     "mse_direct",
+    "mse_fp16_output",
     "mse_gram",
     "search_scale",
     "clip_ratios",
@@ -196,6 +197,29 @@ def mse_direct(X: np.ndarray, delta: np.ndarray) -> float:
     return total / (T * delta.shape[0])
 
 
+def mse_fp16_output(X: np.ndarray, W: np.ndarray, s: Optional[np.ndarray],
+                    deq: np.ndarray) -> float:
+    """The literal reading of [P4] §4, "measure MSE against the fp16 output":
+    the candidate's weights deq/s (fp32 quotient) and the reference output
+    X W^T (exact) are each rounded to fp16, and the mean squared difference of
+    X (deq/s)^T and that fp16 output is taken in fp64.  It differs from the
+    exact score (mse_direct of effective_error) only through the two fp16
+    roundings."""
+    X64 = np.asarray(X, dtype=np.float64)
+    W64 = np.asarray(W, dtype=np.float64)
+    d32 = np.asarray(deq, dtype=np.float32)
+    B = d32 if s is None else d32 / np.asarray(s, dtype=np.float32)[None, :]
+    B64 = B.astype(np.float16).astype(np.float64)
+    T = X64.shape[0]
+    total = 0.0
+    for t0 in range(0, T, 4096):
+        Xb = X64[t0:t0 + 4096]
+        Y16 = (Xb @ W64.T).astype(np.float16).astype(np.float64)
+        E = Xb @ B64.T - Y16
+        total += float(np.sum(E * E))
+    return total / (T * W64.shape[0])
+
+
 def mse_gram(G: np.ndarray, delta: np.ndarray, T: int) -> float:
     """(1 / (T out)) sum_o delta_o^T G delta_o, fp64 (Gram form; equal to the
     direct form in exact arithmetic since sum_t (x_t . d)^2 = d^T X^T X d)."""
@@ -209,6 +233,8 @@ def search_scale(X: np.ndarray, W: np.ndarray, abar: np.ndarray, w_bit: int, gro
 
     For every alpha_i: s_i = abar^alpha_i, fake-quantise diag(s_i) W, score
     MSE_i of (X diag(s_i)^-1) Qdeq^T against X W^T; keep the first argmin.
+    form "gram" / "direct" score against the exact X W^T; "fp16_output"
+    against its fp16 rounding (mse_fp16_output).
     Returns (mse fp64 [n_alpha], best index, s_best fp32 [in], s grid)."""
     alphas = alpha_grid(n_alpha)
     S = scale_grid(abar, alphas)
@@ -218,6 +244,9 @@ def search_scale(X: np.ndarray, W: np.ndarray, abar: np.ndarray, w_bit: int, gro
     mse = np.empty(n_alpha, dtype=np.float64)
     for i in range(n_alpha):
         qd = quantize_groups(W, S[i], group, w_bit, zero_point=zero_point)
+        if form == "fp16_output":
+            mse[i] = mse_fp16_output(X, W, S[i], qd["deq"])
+            continue
         delta = effective_error(W, S[i], qd["deq"])
         mse[i] = mse_gram(G, delta, T) if form == "gram" else mse_direct(X, delta)
     best = int(np.argmin(mse))  # first index attaining the minimum

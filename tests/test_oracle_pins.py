@@ -282,6 +282,57 @@ def test_mse_forms_match_pure_python_definition():
         assert O.mse_gram(O.gram(Xn), delta, Xn.shape[0]) == pytest.approx(want, rel=1e-10)
 
 
+def test_fp16_output_score_is_exact_when_nothing_rounds():
+    """The fp16-output reading of "05 — AWQ" §4 equals the exact score when the
+    candidate weights and X W^T are fp16-representable: X in {-2..2}, W on a
+    1/8 grid spanning [-1, 0.875] (so delta = 1.875 / 15 = 1/8 and deq = W),
+    outputs multiples of 1/8 below 2^8."""
+    rng = np.random.default_rng(21)
+    T, inn, out = 24, 128, 16
+    X = rng.integers(-2, 3, size=(T, inn)).astype(np.float16)
+    W = (rng.integers(-8, 8, size=(out, inn)) / 8.0).astype(np.float16)
+    W[:, 0], W[:, 1] = -1.0, 0.875
+    qd = O.quantize_groups(W, None, 128, 4)
+    assert np.all(qd["delta"] == np.float32(0.125)) and np.array_equal(qd["deq"], W.astype(np.float32))
+    # perturb a few weights off the grid so the exact score is not zero
+    W2 = W.copy()
+    W2[:, 5] += np.float16(1.0 / 64)
+    qd2 = O.quantize_groups(W2, None, 128, 4)
+    exact = O.mse_direct(X, O.effective_error(W2, None, qd2["deq"]))
+    assert exact > 0
+    assert O.mse_fp16_output(X, W2, None, qd2["deq"]) == exact
+
+
+def _ulp16(v):
+    """Spacing of fp16 numbers around |v| (subnormal spacing 2^-24 below 2^-14)."""
+    a = np.abs(np.asarray(v, dtype=np.float64))
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -14)))
+    return np.exp2(e - 10)
+
+
+def test_fp16_output_score_within_half_ulp_bound():
+    """|sqrt(N MSE16) - sqrt(N MSE)| <= || X u_B^T + u_Y ||_F, u being half an
+    fp16 ulp of each rounded candidate weight and reference output: the only
+    difference from the exact score is the two roundings (triangle
+    inequality), whatever the scale s."""
+    X, W = random_layer(40, 256, 24, seed=23)
+    Xn, Wn = X.numpy(), W.numpy()
+    abar = O.act_stats(Xn)
+    S = O.scale_grid(abar, O.alpha_grid(20))
+    X64, W64 = Xn.astype(np.float64), Wn.astype(np.float64)
+    N = Xn.shape[0] * Wn.shape[0]
+    for i in (0, 9, 19):
+        qd = O.quantize_groups(Wn, S[i], 128, 4)
+        exact = O.mse_direct(Xn, O.effective_error(Wn, S[i], qd["deq"]))
+        m16 = O.mse_fp16_output(Xn, Wn, S[i], qd["deq"])
+        B = qd["deq"] / S[i][None, :]
+        uB = _ulp16(B) / 2 * (1 + 2.0 ** -20)
+        uY = _ulp16(X64 @ W64.T) / 2
+        bound = np.sqrt(np.sum((np.abs(X64) @ uB.T + uY) ** 2))
+        assert abs(np.sqrt(N * m16) - np.sqrt(N * exact)) <= bound
+        assert m16 != exact  # the roundings are there
+
+
 @pytest.mark.parametrize("T,inn,out,w_bit,zp", [(64, 128, 16, 4, True), (48, 256, 8, 3, True),
                                                 (33, 256, 16, 4, True), (40, 256, 8, 4, False),
                                                 (24, 128, 16, 3, False)])
