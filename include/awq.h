@@ -61,15 +61,23 @@ typedef enum {
   AWQ_ERR_NONFINITE = 6    /* a score came out NaN or infinite                */
 } awq_status;
 
-/* How awq_search_scale scores the candidates (both give the same MSE in exact
+/* How awq_search_scale scores the candidates (all give the same MSE in exact
  * arithmetic, by the scaling invariance of "05 — AWQ" §3):
- *   AWQ_SEARCH_DIRECT  the scored GEMM ||X dW^T||^2 over all tokens
- *                      (2 T in out n_alpha flops);
- *   AWQ_SEARCH_GRAM    sum_o dW_o^T (X^T X) dW_o: G = X^T X once (T in^2 flops,
- *                      symmetric), then one GEMM of the candidates against the
- *                      normalised G held as fp16 hi + lo parts
- *                      (4 in^2 out n_alpha flops). */
-enum { AWQ_SEARCH_DIRECT = 0, AWQ_SEARCH_GRAM = 1 };
+ *   AWQ_SEARCH_DIRECT   the scored GEMM ||X dW^T||^2 over all tokens, dW =
+ *                       Qdeq/s - W held as fp16 x 2^k (2 T in out n_alpha flops);
+ *   AWQ_SEARCH_GRAM     sum_o dW_o^T (X^T X) dW_o: G = X^T X once (T in^2 flops,
+ *                       symmetric), then one GEMM of the candidates against the
+ *                       normalised G held as fp16 hi + lo parts
+ *                       (4 in^2 out n_alpha flops);
+ *   AWQ_SEARCH_CACHED_Y the literal reading of "05 — AWQ" §4 ("measure MSE
+ *                       against the fp16 output"): Y = RN16(X W^T) once into the
+ *                       workspace, then one GEMM of X against the candidate
+ *                       weights RN16(Qdeq/s) whose epilogue subtracts the cached
+ *                       Y tile and sums the squares (2 T in out (n_alpha + 1)
+ *                       flops; the 1/s of the activation side is folded into
+ *                       the candidate weights so that every candidate shares
+ *                       one staged X tile). */
+enum { AWQ_SEARCH_DIRECT = 0, AWQ_SEARCH_GRAM = 1, AWQ_SEARCH_CACHED_Y = 2 };
 
 /* Quantisation and search settings; the first three fields are the pages'
  * quant_config ("05 — AWQ" §9: w_bit, q_group_size, zero_point). */
@@ -87,7 +95,8 @@ typedef struct {
   int32_t n_alpha;    /* alpha grid size, 1..64; alpha_i = i/(n_alpha-1) ("05 — AWQ" §4: ~20) */
   int32_t n_clip;     /* clip grid size, 0 = no clip search, else 1..64          */
   float clip_min;     /* smallest clip ratio, in (0, 1]; ("05 — AWQ" §4: 0.5)    */
-  int32_t search_form; /* AWQ_SEARCH_DIRECT (0, default) or AWQ_SEARCH_GRAM (1)   */
+  int32_t search_form; /* AWQ_SEARCH_DIRECT (0, default), AWQ_SEARCH_GRAM (1) or
+                          AWQ_SEARCH_CACHED_Y (2)                                */
 } awq_config;
 
 /* Bytes of workspace needed by awq_search_scale and awq_search_clip for a
@@ -120,13 +129,16 @@ awq_status awq_scale_grid(const double *abar, int64_t in, int32_t n_alpha, float
  *   ((X diag(s_i)^-1) Qdeq(diag(s_i) W)^T - X W^T)^2,
  * evaluated as ||X dW_i^T||^2 / (T out) with dW_i = Qdeq/s_i - W (the
  * scaling invariance of "05 — AWQ" §3), on the tensor cores; with
- * cfg->search_form = AWQ_SEARCH_GRAM as sum_o dW_o^T (X^T X) dW_o / (T out).
+ * cfg->search_form = AWQ_SEARCH_GRAM as sum_o dW_o^T (X^T X) dW_o / (T out);
+ * with AWQ_SEARCH_CACHED_Y as ||X RN16(Qdeq/s_i)^T - RN16(X W^T)||^2 / (T out)
+ * (the workspace then also holds Y: ceil(T/128) * 128 x round_up(out, 256)
+ * fp16).
  *   abar     device fp64 [in] from awq_act_stats
  *   s_best   device fp32 [in]      (output) s of the selected alpha
  *   mse      device fp64 [n_alpha] (output) MSE_i
  *   best_idx device int32 [1]      (output) first index of the smallest MSE
- * Requires out % 8 == 0, ldx % 8 == 0, and in % 64 == 0 (direct form) or
- * in % 128 == 0 (Gram form). */
+ * Requires out % 8 == 0, ldx % 8 == 0, and in % 64 == 0 (direct and cached-Y
+ * forms) or in % 128 == 0 (Gram form). */
 awq_status awq_search_scale(const void *X, int64_t T, int64_t in, int64_t ldx,
                             const void *W, int64_t out, const double *abar,
                             const awq_config *cfg, void *ws, size_t ws_bytes,

@@ -37,7 +37,7 @@ class AwqError(RuntimeError):
         super().__init__(f"{func}: {self.status_name}: {message}")
 
 
-SEARCH_DIRECT, SEARCH_GRAM = 0, 1
+SEARCH_DIRECT, SEARCH_GRAM, SEARCH_CACHED_Y = 0, 1, 2
 
 
 class AwqConfig(ctypes.Structure):

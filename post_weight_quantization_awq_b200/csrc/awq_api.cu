@@ -109,8 +109,10 @@ awq_status check_cfg(const awq_config *cfg) {
     return fail(AWQ_ERR_INVALID_ARG, "n_clip=%d (0..64)", cfg->n_clip);
   if (!(cfg->clip_min > 0.0f && cfg->clip_min <= 1.0f))
     return fail(AWQ_ERR_INVALID_ARG, "clip_min=%g (must be in (0, 1])", (double)cfg->clip_min);
-  if (cfg->search_form != AWQ_SEARCH_DIRECT && cfg->search_form != AWQ_SEARCH_GRAM)
-    return fail(AWQ_ERR_INVALID_ARG, "search_form=%d (0 direct, 1 Gram)", cfg->search_form);
+  if (cfg->search_form != AWQ_SEARCH_DIRECT && cfg->search_form != AWQ_SEARCH_GRAM &&
+      cfg->search_form != AWQ_SEARCH_CACHED_Y)
+    return fail(AWQ_ERR_INVALID_ARG, "search_form=%d (0 direct, 1 Gram, 2 cached fp16 output)",
+                cfg->search_form);
   return AWQ_OK;
 }
 
@@ -137,7 +139,7 @@ awq_status check_x(const void *X, int64_t in, int64_t ldx) {
 constexpr size_t kHeader = 256;
 
 struct ScaleWs {
-  size_t s_grid, inv_s, dW, partials, G, ghi, glo, r, end;
+  size_t s_grid, inv_s, dW, partials, G, ghi, glo, r, Y, end;
   int64_t out_pad;
   int num_m, nb_per_alpha;
   size_t per_alpha;  // partials per candidate
@@ -151,6 +153,7 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 ScaleWs scale_layout(int64_t T, int64_t in, int64_t out, const awq_config *cfg) {
   ScaleWs w;
   const bool gram = cfg->search_form == AWQ_SEARCH_GRAM;
+  const bool cached_y = cfg->search_form == AWQ_SEARCH_CACHED_Y;
   w.out_pad = round_up(out, gram ? 128 : kGemmBN);
   w.num_m = (int)((T + kGemmBM - 1) / kGemmBM);
   w.nb_per_alpha = (int)(w.out_pad / kGemmBN);
@@ -165,7 +168,11 @@ ScaleWs scale_layout(int64_t T, int64_t in, int64_t out, const awq_config *cfg) 
   off = align256(off + sizeof(__half) * (size_t)cfg->n_alpha * w.out_pad * in);
   w.partials = off;
   off = align256(off + sizeof(double) * (size_t)cfg->n_alpha * w.per_alpha);
-  w.G = w.ghi = w.glo = w.r = 0;
+  w.G = w.ghi = w.glo = w.r = w.Y = 0;
+  if (cached_y) {  // Y = RN16(X W^T), padded to whole 128-token and 256-column tiles
+    w.Y = off;
+    off = align256(off + sizeof(__half) * (size_t)w.num_m * kGemmBM * (size_t)w.out_pad);
+  }
   if (gram) {
     w.G = off;
     off = align256(off + sizeof(float) * (size_t)in * in);
@@ -299,7 +306,16 @@ awq_status awq_search_scale(const void *X, int64_t T, int64_t in, int64_t ldx, c
   // status of this call only: flags, site, exponent and max |W| start at zero
   AWQ_TRY_CUDA(cudaMemsetAsync(dst, 0, sizeof(DevStatus), s), "workspace reset");
   const bool gram = cfg->search_form == AWQ_SEARCH_GRAM;
+  const bool cached_y = cfg->search_form == AWQ_SEARCH_CACHED_Y;
   float *r = gram ? reinterpret_cast<float *>(base + L.r) : nullptr;
+  __half *Y = cached_y ? reinterpret_cast<__half *>(base + L.Y) : nullptr;
+  if (cached_y) {
+    ProfScope p("ref_output", s);
+    AWQ_TRY_CUDA(launch_ref_output(static_cast<const __half *>(X), T, in, ldx,
+                                   static_cast<const __half *>(W), out, L.out_pad, Y, dst,
+                                   poll_cap(), nsm, s),
+                 "ref_output launch");
+  }
   if (gram) {
     ProfScope p("gram_full", s);
     AWQ_TRY_CUDA(launch_gram_full(static_cast<const __half *>(X), T, in, ldx,
@@ -308,7 +324,7 @@ awq_status awq_search_scale(const void *X, int64_t T, int64_t in, int64_t ldx, c
                                   reinterpret_cast<__half *>(base + L.glo), dst, poll_cap(), s),
                  "gram_full launch");
   }
-  {
+  if (!cached_y) {  // the candidate errors' power-of-two scaling
     ProfScope p("wmax", s);
     AWQ_TRY_CUDA(launch_wmax(static_cast<const __half *>(W), out * in, in, r, dst, nsm, s), "wmax launch");
   }
@@ -319,8 +335,8 @@ awq_status awq_search_scale(const void *X, int64_t T, int64_t in, int64_t ldx, c
   {
     ProfScope p("cand_quant", s);
     AWQ_TRY_CUDA(launch_cand_quant(static_cast<const __half *>(W), out, in, L.out_pad, s_grid, inv_s, r,
-                                   cfg->n_alpha, cfg->group_size, cfg->w_bit, cfg->zero_point, dst,
-                                   dW, nsm, s),
+                                   cfg->n_alpha, cfg->group_size, cfg->w_bit, cfg->zero_point,
+                                   cached_y ? 1 : 0, dst, dW, nsm, s),
                  "cand_quant launch");
   }
   if (gram) {
@@ -339,8 +355,8 @@ awq_status awq_search_scale(const void *X, int64_t T, int64_t in, int64_t ldx, c
     sh.num_n = (int)(sh.rows_b / kGemmBN);
     sh.num_kb = (int)(in / kGemmBK);
     ProfScope p("search_gemm", s);
-    AWQ_TRY_CUDA(launch_search_gemm(static_cast<const __half *>(X), ldx, dW, sh, partials, dst,
-                                    poll_cap(), nsm, s),
+    AWQ_TRY_CUDA(launch_search_gemm(static_cast<const __half *>(X), ldx, dW, sh, partials, Y,
+                                    L.out_pad, dst, poll_cap(), nsm, s),
                  "search_gemm launch");
   }
   {

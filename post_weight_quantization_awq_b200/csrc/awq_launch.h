@@ -27,20 +27,30 @@ cudaError_t launch_wmax(const __half *W, int64_t n, int64_t in, const float *r, 
 
 // K3: candidate effective errors dW[i][o][j] = RN16(2^k r_j (deq/s - w))
 // (r = NULL: r_j = 1), rows out..out_pad-1 zero.  zero_point = 0 quantises
-// symmetrically (step max|w|/(2^(b-1)-1), z = 2^(b-1)).
+// symmetrically (step max|w|/(2^(b-1)-1), z = 2^(b-1)).  weights_only: the
+// candidate weights RN16(deq/s) themselves (no 2^k, no - w).
 cudaError_t launch_cand_quant(const __half *W, int64_t out, int64_t in, int64_t out_pad,
                               const float *s, const float *inv_s, const float *r, int n_alpha,
-                              int group, int w_bit, int zero_point, const DevStatus *st, __half *dW,
-                              int num_sms, cudaStream_t stream);
+                              int group, int w_bit, int zero_point, int weights_only,
+                              const DevStatus *st, __half *dW, int num_sms, cudaStream_t stream);
 
 // K4: scored GEMM, partial sums of squares per (n-tile, m-tile, warp).
 struct SearchGemmShape {
   int64_t T, in, rows_b;  // rows_b = n_alpha * out_pad
   int num_m, num_n, num_kb;
 };
+// Y == NULL: partials of sum acc^2 (dW = candidate errors).  Y != NULL: partials
+// of sum (acc - Y)^2 with the cached fp16 output Y [num_m * 128, ldy], the
+// columns of N tile n being (n * 256) mod ldy (dW = candidate weights Qdeq/s).
 cudaError_t launch_search_gemm(const __half *X, int64_t ldx, const __half *dW,
-                               const SearchGemmShape &sh, double *partials, DevStatus *st,
-                               uint32_t max_polls, int num_sms, cudaStream_t stream);
+                               const SearchGemmShape &sh, double *partials, const __half *Y,
+                               int64_t ldy, DevStatus *st, uint32_t max_polls, int num_sms,
+                               cudaStream_t stream);
+// Reference output Y = RN16(X W^T) into Y [ceil(T/128) * 128, out_pad] (padding
+// rows and columns come out zero); out_pad % 256 == 0, in % 64 == 0.
+cudaError_t launch_ref_output(const __half *X, int64_t T, int64_t in, int64_t ldx, const __half *W,
+                              int64_t out, int64_t out_pad, __half *Y, DevStatus *st,
+                              uint32_t max_polls, int num_sms, cudaStream_t stream);
 constexpr int kGemmBM = 128, kGemmBN = 256, kGemmBK = 64;
 
 // 2-D fp16 TMA descriptor over a row-major [rows, cols] matrix (row stride

@@ -199,9 +199,11 @@ constexpr int kCandRows = 64;
 __global__ void __launch_bounds__(256) cand_quant_kernel(
     const __half *__restrict__ W, int64_t out, int64_t in, int64_t out_pad,
     const float *__restrict__ s, const float *__restrict__ inv_s, const float *__restrict__ rch,
-    int group, float qmax, int sym, const DevStatus *__restrict__ st, __half *__restrict__ dW) {
-  const int k = kscale_from_wmax(__uint_as_float(__ldg(&st->wmax_bits)));
+    int group, float qmax, int sym, int weights_only, const DevStatus *__restrict__ st,
+    __half *__restrict__ dW) {
+  const int k = weights_only ? 0 : kscale_from_wmax(__uint_as_float(__ldg(&st->wmax_bits)));
   const float two_k = ldexpf(1.0f, k);
+  const float wneg = weights_only ? 0.0f : -two_k;  // coefficient of w
   const int lanes = group / 8;  // lanes per group (a power of two <= 32)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t j0 = (int64_t)blockIdx.y * 256 + lane * 8;
@@ -265,12 +267,12 @@ __global__ void __launch_bounds__(256) cand_quant_kernel(
     uint32_t packed[4];
 #pragma unroll
     for (int h = 0; h < 4; ++h) {
-      // 2^k (deq/s - w) with deq = (q - z) delta; the product with 1/s is
-      // fp32 (the result is rounded to fp16 next)
+      // 2^k (deq/s - w) with deq = (q - z) delta (weights_only: deq/s); the
+      // product with 1/s is fp32 (the result is rounded to fp16 next)
       const float2 qz = quant_qz2(wt[h], g);
       float2 d2 = __ffma2_rn(__fmul2_rn(qz, make_float2(dk, dk)), make_float2(iv[2 * h], iv[2 * h + 1]),
                              __fmul2_rn(make_float2(w[2 * h], w[2 * h + 1]),
-                                        make_float2(-two_k * rv[2 * h], -two_k * rv[2 * h + 1])));
+                                        make_float2(wneg * rv[2 * h], wneg * rv[2 * h + 1])));
       if (!live) d2 = make_float2(0.0f, 0.0f);
       const __half2 hv = __floats2half2_rn(d2.x, d2.y);
       packed[h] = *reinterpret_cast<const uint32_t *>(&hv);
@@ -283,12 +285,13 @@ __global__ void __launch_bounds__(256) cand_quant_kernel(
 
 cudaError_t launch_cand_quant(const __half *W, int64_t out, int64_t in, int64_t out_pad,
                               const float *s, const float *inv_s, const float *r, int n_alpha,
-                              int group, int w_bit, int zero_point, const DevStatus *st, __half *dW,
-                              int num_sms, cudaStream_t stream) {
+                              int group, int w_bit, int zero_point, int weights_only,
+                              const DevStatus *st, __half *dW, int num_sms, cudaStream_t stream) {
   (void)num_sms;
   dim3 grid((unsigned)(n_alpha * (out_pad / kCandRows)), (unsigned)((in + 255) / 256));
   cand_quant_kernel<<<grid, 256, 0, stream>>>(W, out, in, out_pad, s, inv_s, r, group,
-                                              (float)((1 << w_bit) - 1), zero_point ? 0 : 1, st, dW);
+                                              (float)((1 << w_bit) - 1), zero_point ? 0 : 1,
+                                              weights_only, st, dW);
   return cudaGetLastError();
 }
 

@@ -43,6 +43,7 @@ constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t IDESC = idesc_f16_f32(BM, BN);
 constexpr uint32_t DRAIN_POLLS = 1u << 22;
 constexpr int GROUP_M = 32;
+constexpr int kEpiSse = 0, kEpiStoreY = 1, kEpiSubY = 2;
 
 struct __align__(8) GemmSmemTail {
   uint64_t full[STAGES];
@@ -75,10 +76,19 @@ __device__ __forceinline__ void raise_abort(GemmSmemTail *t, DevStatus *st, uint
 
 }  // namespace
 
+// Epilogue of one accumulator tile (a 128-token x 256-column block of the
+// product of X with the B rows):
+//   kEpiSse    sum of squares (B = candidate errors dW: X dW^T is the error);
+//   kEpiStoreY the tile rounded to fp16 into Y [tokens, ldy] (B = W: the
+//              reference output Y = X W^T, computed once);
+//   kEpiSubY   sum of (acc - Y)^2 with the cached fp16 Y (B = candidate
+//              weights Qdeq/s: the literal "MSE against the fp16 output").
+template <int EPI>
 __global__ void __launch_bounds__(192, 1)
     search_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                        const __grid_constant__ CUtensorMap tmB, int num_m, int num_n, int num_kb,
-                       double *__restrict__ partials, DevStatus *st, uint32_t max_polls) {
+                       double *__restrict__ partials, __half *__restrict__ Y, int64_t ldy,
+                       int64_t y_cols, DevStatus *st, uint32_t max_polls) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -211,26 +221,64 @@ __global__ void __launch_bounds__(192, 1)
         break;
       }
       tc_fence_after();
+      int m_blk, n_blk;
+      tile_coords(tile, num_m, num_n, GROUP_M, m_blk, n_blk);
       const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
+      // this thread's accumulator row is token m_blk * BM + 32 q + lane
+      const size_t yrow = (size_t)(m_blk * BM + q * 32 + lane) * (size_t)ldy;
       float sum = 0.0f;
 #pragma unroll 1
       for (int c = 0; c < BN; c += 32) {
         float v[32];
-        tmem_ld_32x32b_x32(taddr + (uint32_t)c, v);
-        tmem_ld_wait();
+        if constexpr (EPI == kEpiSubY) {
+          // fetch the cached fp16 outputs first, so their latency overlaps the TMEM read
+          const uint4 *yp = reinterpret_cast<const uint4 *>(
+              Y + yrow + (size_t)(((int64_t)n_blk * BN) % y_cols) + c);
+          uint4 yv[4];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) sum = fmaf(v[i], v[i], sum);
+          for (int u = 0; u < 4; ++u) yv[u] = __ldg(yp + u);
+          tmem_ld_32x32b_x32(taddr + (uint32_t)c, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const uint32_t yw[4] = {yv[u].x, yv[u].y, yv[u].z, yv[u].w};
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const float2 yf = __half22float2(*reinterpret_cast<const __half2 *>(&yw[h]));
+              const float d0 = v[8 * u + 2 * h] - yf.x, d1 = v[8 * u + 2 * h + 1] - yf.y;
+              sum = fmaf(d0, d0, sum);
+              sum = fmaf(d1, d1, sum);
+            }
+          }
+        } else {
+          tmem_ld_32x32b_x32(taddr + (uint32_t)c, v);
+          tmem_ld_wait();
+          if constexpr (EPI == kEpiStoreY) {
+            uint4 *yp = reinterpret_cast<uint4 *>(Y + yrow + (size_t)n_blk * BN + c);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              uint32_t hw[4];
+#pragma unroll
+              for (int h = 0; h < 4; ++h) {
+                const __half2 hv = __floats2half2_rn(v[8 * u + 2 * h], v[8 * u + 2 * h + 1]);
+                hw[h] = *reinterpret_cast<const uint32_t *>(&hv);
+              }
+              yp[u] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) sum = fmaf(v[i], v[i], sum);
+          }
+        }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tail->tempty[acc]);
-      double ds = (double)sum;
+      if constexpr (EPI != kEpiStoreY) {
+        double ds = (double)sum;
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) ds += __shfl_xor_sync(0xffffffffu, ds, off);
-      if (lane == 0) {
-        int m_blk, n_blk;
-        tile_coords(tile, num_m, num_n, GROUP_M, m_blk, n_blk);
-        partials[((size_t)n_blk * num_m + m_blk) * 4 + q] = ds;
+        for (int off = 16; off > 0; off >>= 1) ds += __shfl_xor_sync(0xffffffffu, ds, off);
+        if (lane == 0) partials[((size_t)n_blk * num_m + m_blk) * 4 + q] = ds;
       }
     }
   }
@@ -280,22 +328,56 @@ cudaError_t make_tmap_f16_box(CUtensorMap *m, const void *base, int64_t rows, in
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+template <int EPI>
+static cudaError_t launch_gemm_epi(const CUtensorMap &tmA, const CUtensorMap &tmB,
+                                   const SearchGemmShape &sh, double *partials, __half *Y,
+                                   int64_t ldy, int64_t y_cols, DevStatus *st, uint32_t max_polls,
+                                   int num_sms, cudaStream_t stream) {
+  cudaError_t e = cudaFuncSetAttribute(search_gemm_kernel<EPI>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)kGemmSmemBytes);
+  if (e != cudaSuccess) return e;
+  const int tiles = sh.num_m * sh.num_n;
+  const int grid = tiles < num_sms ? tiles : num_sms;
+  search_gemm_kernel<EPI><<<grid, 192, kGemmSmemBytes, stream>>>(
+      tmA, tmB, sh.num_m, sh.num_n, sh.num_kb, partials, Y, ldy, y_cols, st, max_polls);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_search_gemm(const __half *X, int64_t ldx, const __half *dW,
-                               const SearchGemmShape &sh, double *partials, DevStatus *st,
-                               uint32_t max_polls, int num_sms, cudaStream_t stream) {
+                               const SearchGemmShape &sh, double *partials, const __half *Y,
+                               int64_t ldy, DevStatus *st, uint32_t max_polls, int num_sms,
+                               cudaStream_t stream) {
   CUtensorMap tmA, tmB;
   cudaError_t e = make_tmap_f16_box(&tmA, X, sh.T, sh.in, ldx, BK, BM);
   if (e != cudaSuccess) return e;
   e = make_tmap_f16_box(&tmB, dW, sh.rows_b, sh.in, sh.in, BK, BN);
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(search_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)kGemmSmemBytes);
+  if (Y)
+    return launch_gemm_epi<kEpiSubY>(tmA, tmB, sh, partials, const_cast<__half *>(Y), ldy, ldy, st,
+                                     max_polls, num_sms, stream);
+  return launch_gemm_epi<kEpiSse>(tmA, tmB, sh, partials, nullptr, 0, 1, st, max_polls, num_sms,
+                                  stream);
+}
+
+cudaError_t launch_ref_output(const __half *X, int64_t T, int64_t in, int64_t ldx, const __half *W,
+                              int64_t out, int64_t out_pad, __half *Y, DevStatus *st,
+                              uint32_t max_polls, int num_sms, cudaStream_t stream) {
+  if (out_pad % BN != 0 || in % BK != 0) return cudaErrorInvalidValue;
+  CUtensorMap tmA, tmB;
+  cudaError_t e = make_tmap_f16_box(&tmA, X, T, in, ldx, BK, BM);
   if (e != cudaSuccess) return e;
-  const int tiles = sh.num_m * sh.num_n;
-  const int grid = tiles < num_sms ? tiles : num_sms;
-  search_gemm_kernel<<<grid, 192, kGemmSmemBytes, stream>>>(tmA, tmB, sh.num_m, sh.num_n,
-                                                            sh.num_kb, partials, st, max_polls);
-  return cudaGetLastError();
+  e = make_tmap_f16_box(&tmB, W, out, in, in, BK, BN);  // rows >= out read as zeros
+  if (e != cudaSuccess) return e;
+  SearchGemmShape sh;
+  sh.T = T;
+  sh.in = in;
+  sh.rows_b = out;
+  sh.num_m = (int)((T + BM - 1) / BM);
+  sh.num_n = (int)(out_pad / BN);
+  sh.num_kb = (int)(in / BK);
+  return launch_gemm_epi<kEpiStoreY>(tmA, tmB, sh, nullptr, Y, out_pad, out_pad, st, max_polls,
+                                     num_sms, stream);
 }
 
 // ---------------------------------------------------------------------------

@@ -2,7 +2,7 @@
 (ncu) and quick timing.
 
     python -m post_weight_quantization_awq_b200.run_case --op search --tokens 16384 \
-        --in 4096 --out 4096 [--alphas 20] [--clips 20] [--bits 4] [--repeat 3] [--form gram]
+        --in 4096 --out 4096 [--alphas 20] [--clips 20] [--bits 4] [--repeat 3] [--form gram|cached_y]
 
 --op is one of: stats, search, clip, pack, layer (all four calls).  Inputs
 follow the heavy-tailed recipe of the synthetic module (1% outlier channels
@@ -36,14 +36,15 @@ def main(argv=None) -> int:
     ap.add_argument("--bits", type=int, default=4)
     ap.add_argument("--repeat", type=int, default=3)
     ap.add_argument("--seed", type=int, default=1)
-    ap.add_argument("--form", choices=("direct", "gram"), default="direct",
+    ap.add_argument("--form", choices=("direct", "gram", "cached_y"), default="direct",
                     help="alpha-search scoring form")
     a = ap.parse_args(argv)
 
     X = heavy_tailed_activations(a.tokens, a.inn, OutlierSpec(0.01, 20.0, 50.0), a.seed).cuda()
     W = gaussian_weight(a.out, a.inn, a.seed).cuda()
     cfg = awq.AwqConfig.make(w_bit=a.bits, n_alpha=a.alphas, n_clip=a.clips,
-                             search_form=awq.abi.SEARCH_GRAM if a.form == "gram" else 0)
+                             search_form={"direct": awq.abi.SEARCH_DIRECT, "gram": awq.abi.SEARCH_GRAM,
+                                          "cached_y": awq.abi.SEARCH_CACHED_Y}[a.form])
     ws = awq.alloc_workspace(a.tokens, a.inn, a.out, cfg)
     abar = torch.empty(a.inn, dtype=torch.float64, device="cuda")
     mse = torch.empty(a.alphas, dtype=torch.float64, device="cuda")
