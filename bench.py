@@ -40,7 +40,7 @@ KERNELS_PER_STEP = {  # kernels this library launches per step (memsets excluded
 # DRAM bytes (read + write) of one search_gemm_kernel launch on this workload,
 # from a one-pass ncu capture (profiles/search_gemm_q_proj_4096.md); to be
 # set to None whenever that kernel changes until it is captured again.
-NCU_TRAFFIC_BYTES = 11_290_000_000 + 9_940_000
+NCU_TRAFFIC_BYTES = None
 
 
 def load_peaks():
@@ -343,31 +343,51 @@ def run_awq(args):
     h2d = X.numel() * 2 + W.numel() * 2
     d2h = sum(h.numel() * h.element_size() for h in host_out.values())
 
+    def time_form(search_form, names):
+        """ms per step of the whole layer with another scoring form, and the
+        average per-launch ms of the named kernels."""
+        cfg_f = awq.AwqConfig.make(w_bit=wl.w_bit, group_size=wl.group_size, n_alpha=wl.n_alpha,
+                                   n_clip=wl.n_clip, clip_min=0.5, search_form=search_form)
+        ws_f = awq.alloc_workspace(T, inn, out, cfg_f, dev)
+
+        def step_f():
+            return awq.quantize_layer(Xd, Wd, cfg_f, ws=ws_f)
+
+        for _ in range(args.warmup):
+            step_f()
+        awq.awq_device_status(ws_f)
+        awq.profile_reset()
+        awq.profile_enable(True)
+        ms_f = timed_steps(step_f, args.steps, dist, timer, local)
+        awq.profile_enable(False)
+        awq.awq_device_status(ws_f)
+        kf = {}
+        for name in names:
+            tot, n = awq.profile_read(name)
+            kf[name] = tot / n if n else None
+        awq.profile_reset()
+        del ws_f
+        return ms_f, kf
+
+    # ---- the literal fp16-output form on the same layer: Y = RN16(X W^T) once,
+    # then every candidate's output scored against it in the GEMM's epilogue
+    cached = None
+    if not args.no_cached_form:
+        ms_c, kc = time_form(awq.abi.SEARCH_CACHED_Y, ("ref_output", "search_gemm"))
+        flops_c = 2.0 * T * inn * out * (wl.n_alpha + 1)
+        gemm_c = (kc["ref_output"] or 0.0) + (kc["search_gemm"] or 0.0)
+        cached = {"value": round(ms_c / world, 3), "unit": UNIT, "ms_per_step": round(ms_c, 3),
+                  "kernels_ms": {k: round(v, 4) for k, v in kc.items() if v},
+                  "algorithmic_flops_per_step": flops_c,
+                  "gemm_tflops": round(flops_c / (gemm_c * 1e-3) / 1e12, 1) if gemm_c else None,
+                  "note": "scores against the cached fp16 output RN16(X W^T) (one extra GEMM "
+                          "with a store epilogue); candidates RN16(Qdeq/s)"}
+
     # ---- the Gram-form search on the same layer (same MSE, fewer flops), its
     # own timing and flop count; the headline value above is the direct form
     gram = None
     if not args.no_gram_form:
-        cfg_g = awq.AwqConfig.make(w_bit=wl.w_bit, group_size=wl.group_size, n_alpha=wl.n_alpha,
-                                   n_clip=wl.n_clip, clip_min=0.5, search_form=awq.abi.SEARCH_GRAM)
-        ws_g = awq.alloc_workspace(T, inn, out, cfg_g, dev)
-
-        def step_g():
-            return awq.quantize_layer(Xd, Wd, cfg_g, ws=ws_g)
-
-        for _ in range(args.warmup):
-            step_g()
-        awq.awq_device_status(ws_g)
-        awq.profile_reset()
-        awq.profile_enable(True)
-        ms_g = timed_steps(step_g, args.steps, dist, timer, local)
-        awq.profile_enable(False)
-        awq.awq_device_status(ws_g)
-        kg = {}
-        for name in ("gram_full", "gram_score"):
-            tot, n = awq.profile_read(name)
-            kg[name] = tot / n if n else None
-        awq.profile_reset()
-        del ws_g
+        ms_g, kg = time_form(awq.abi.SEARCH_GRAM, ("gram_full", "gram_score"))
         nb = (inn + 255) // 256  # G: the nb(nb+1)/2 upper 256x256 block pairs; scores: hi and lo
         out128 = (out + 127) // 128 * 128
         nt = inn // 128  # scores: the nt(nt+1)/2 upper 128-blocks of G~, hi and lo
@@ -428,6 +448,7 @@ def run_awq(args):
         "gpu_launches": launches,
         "cpu_baseline": cpu,
         "gram_form": gram,
+        "cached_output_form": cached,
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -496,6 +517,8 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-gram-form", action="store_true",
                     help="skip the extra measurement of the Gram-form search")
+    ap.add_argument("--no-cached-form", action="store_true",
+                    help="skip the extra measurement of the cached fp16-output form")
     ap.add_argument("--workload", choices=("q_proj", "decoder"), default="q_proj",
                     help="q_proj: the headline workload; decoder: the 32-layer decoder "
                          "(--steps = layers timed)")
