@@ -209,6 +209,56 @@ awq_status awq_quant_pack(const void *W, int64_t out, int64_t in, const float *s
 awq_status awq_fold_inv_scale(void *v, int64_t rows, int64_t cols, const float *s,
                               awq_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Token sharding of one layer over several GPUs.  Every statistic the search
+ * needs is a sum over tokens: the exact |x| sums behind abar, each alpha's
+ * squared error, and the clip search's block Grams.  Each rank computes its
+ * tokens' part with the calls below, the caller sums the parts over ranks
+ * (an all-reduce; the library itself never communicates), and the finishing
+ * calls turn the sums into the results the single-GPU calls give.  Every rank
+ * needs the full W.
+ * ------------------------------------------------------------------------ */
+
+/* sums_j = sum_t |X_tj| of these tokens in units of 2^-24: exact int64
+ * (every fp16 is an integer multiple of 2^-24), so sums add exactly across
+ * ranks.  X as in awq_act_stats; sums device int64 [in], overwritten. */
+awq_status awq_act_sums(const void *X, int64_t T, int64_t in, int64_t ldx, int64_t *sums,
+                        awq_stream_t stream);
+
+/* abar_j = RN64(RN64(sums_j 2^-24) / T_total) from the summed sums: the same
+ * bits awq_act_stats gives on all T_total tokens.  sums may alias abar. */
+awq_status awq_act_stats_finish(const int64_t *sums, int64_t T_total, int64_t in, double *abar,
+                                awq_stream_t stream);
+
+/* Unnormalised squared errors of these tokens for every alpha,
+ *   sse_i = sum_{t in this shard} sum_o (candidate i's output error)^2,
+ * in the scoring form cfg->search_form (each form's sum splits over tokens;
+ * the Gram form builds X^T X of these tokens).  abar must be the global abar
+ * (awq_act_stats_finish) so that every rank scores the same candidates.
+ * Arguments and workspace as awq_search_scale; sse device fp64 [n_alpha]. */
+awq_status awq_search_scale_sse(const void *X, int64_t T, int64_t in, int64_t ldx, const void *W,
+                                int64_t out, const double *abar, const awq_config *cfg, void *ws,
+                                size_t ws_bytes, double *sse, awq_stream_t stream);
+
+/* The selection from the summed sse: mse_i = sse_i / (T_total out), best_idx =
+ * the first index of the smallest, s_best = RN32(pow(max(abar_j, 1e-4),
+ * alpha_best)) (the grid's value).  ws: at least 256 bytes (status word). */
+awq_status awq_select_scale(const double *sse, int64_t T_total, int64_t in, int64_t out,
+                            const double *abar, const awq_config *cfg, void *ws, size_t ws_bytes,
+                            float *s_best, double *mse, int32_t *best_idx, awq_stream_t stream);
+
+/* Block Grams of these tokens, G[k] = X_k^T X_k for every group k of 128 input
+ * channels: device fp32 [in/128][128][128] (output).  in % 128 == 0,
+ * cfg->group_size == 128; workspace as awq_search_clip (the same size). */
+awq_status awq_block_grams(const void *X, int64_t T, int64_t in, int64_t ldx, const awq_config *cfg,
+                           void *ws, size_t ws_bytes, float *G, awq_stream_t stream);
+
+/* The clip-ratio search of awq_search_clip from block Grams G (summed over
+ * ranks) instead of X.  ws: at least 256 bytes (status word). */
+awq_status awq_search_clip_grams(const void *W, int64_t out, int64_t in, const float *s,
+                                 const float *G, const awq_config *cfg, void *ws, size_t ws_bytes,
+                                 uint8_t *clip_idx, float *err, awq_stream_t stream);
+
 /* Synchronises `stream`, then returns and clears the device status recorded in
  * workspace `ws` (AWQ_OK, AWQ_ERR_TIMEOUT or AWQ_ERR_NONFINITE). */
 awq_status awq_device_status(void *ws, awq_stream_t stream);

@@ -16,13 +16,19 @@ from .abi import (  # noqa: F401
     AwqConfig,
     AwqError,
     awq_act_stats,
+    awq_act_stats_finish,
+    awq_act_sums,
+    awq_block_grams,
     awq_device_status,
     awq_fold_inv_scale,
     awq_quant_pack,
     awq_scale_grid,
     awq_search_clip,
+    awq_search_clip_grams,
     awq_search_clip_noalloc,
     awq_search_scale,
+    awq_search_scale_sse,
+    awq_select_scale,
     awq_workspace_size,
     header_functions,
     last_error,

@@ -80,6 +80,18 @@ _SIGNATURES = {
     "awq_quant_pack": (c_int32, [c_void_p, c_int64, c_int64, c_void_p, c_void_p, POINTER(AwqConfig),
                                  c_void_p, c_void_p, c_void_p, c_void_p]),
     "awq_fold_inv_scale": (c_int32, [c_void_p, c_int64, c_int64, c_void_p, c_void_p]),
+    "awq_act_sums": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_void_p]),
+    "awq_act_stats_finish": (c_int32, [c_void_p, c_int64, c_int64, c_void_p, c_void_p]),
+    "awq_search_scale_sse": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_int64,
+                                       c_void_p, POINTER(AwqConfig), c_void_p, c_size_t, c_void_p,
+                                       c_void_p]),
+    "awq_select_scale": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, POINTER(AwqConfig),
+                                   c_void_p, c_size_t, c_void_p, c_void_p, c_void_p, c_void_p]),
+    "awq_block_grams": (c_int32, [c_void_p, c_int64, c_int64, c_int64, POINTER(AwqConfig), c_void_p,
+                                  c_size_t, c_void_p, c_void_p]),
+    "awq_search_clip_grams": (c_int32, [c_void_p, c_int64, c_int64, c_void_p, c_void_p,
+                                        POINTER(AwqConfig), c_void_p, c_size_t, c_void_p, c_void_p,
+                                        c_void_p]),
     "awq_device_status": (c_int32, [c_void_p, c_void_p]),
     "awq_profile_enable": (c_int32, [c_int32]),
     "awq_profile_read": (c_int32, [c_char_p, POINTER(c_double), POINTER(c_int64)]),
@@ -208,6 +220,42 @@ def awq_fold_inv_scale(v, s, stream=None) -> None:
     cols = v.numel() // rows
     _check("awq_fold_inv_scale", LIB.awq_fold_inv_scale(_ptr(v), rows, cols, _ptr(s),
                                                         _stream(stream)))
+
+
+def awq_act_sums(X, sums, stream=None) -> None:
+    """Exact sums of |X| over these tokens, int64 [in] in units of 2^-24."""
+    _check("awq_act_sums", LIB.awq_act_sums(_ptr(X), X.shape[0], X.shape[1], X.stride(0),
+                                            _ptr(sums), _stream(stream)))
+
+
+def awq_act_stats_finish(sums, T_total: int, abar, stream=None) -> None:
+    _check("awq_act_stats_finish", LIB.awq_act_stats_finish(_ptr(sums), int(T_total), sums.shape[0],
+                                                            _ptr(abar), _stream(stream)))
+
+
+def awq_search_scale_sse(X, W, abar, cfg: AwqConfig, ws, sse, stream=None) -> None:
+    _check("awq_search_scale_sse", LIB.awq_search_scale_sse(
+        _ptr(X), X.shape[0], X.shape[1], X.stride(0), _ptr(W), W.shape[0], _ptr(abar),
+        ctypes.byref(cfg), _ptr(ws), ws.numel() * ws.element_size(), _ptr(sse), _stream(stream)))
+
+
+def awq_select_scale(sse, T_total: int, out: int, abar, cfg: AwqConfig, ws, s_best, mse, best_idx,
+                     stream=None) -> None:
+    _check("awq_select_scale", LIB.awq_select_scale(
+        _ptr(sse), int(T_total), abar.shape[0], int(out), _ptr(abar), ctypes.byref(cfg), _ptr(ws),
+        ws.numel() * ws.element_size(), _ptr(s_best), _ptr(mse), _ptr(best_idx), _stream(stream)))
+
+
+def awq_block_grams(X, cfg: AwqConfig, ws, G, stream=None) -> None:
+    _check("awq_block_grams", LIB.awq_block_grams(
+        _ptr(X), X.shape[0], X.shape[1], X.stride(0), ctypes.byref(cfg), _ptr(ws),
+        ws.numel() * ws.element_size(), _ptr(G), _stream(stream)))
+
+
+def awq_search_clip_grams(W, s, G, cfg: AwqConfig, ws, clip_idx, err=None, stream=None) -> None:
+    _check("awq_search_clip_grams", LIB.awq_search_clip_grams(
+        _ptr(W), W.shape[0], W.shape[1], _ptr(s), _ptr(G), ctypes.byref(cfg), _ptr(ws),
+        ws.numel() * ws.element_size(), _ptr(clip_idx), _ptr(err), _stream(stream)))
 
 
 def awq_device_status(ws, stream=None) -> None:

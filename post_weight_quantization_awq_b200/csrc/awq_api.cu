@@ -274,17 +274,21 @@ awq_status awq_scale_grid(const double *abar, int64_t in, int32_t n_alpha, float
   return AWQ_OK;
 }
 
-awq_status awq_search_scale(const void *X, int64_t T, int64_t in, int64_t ldx, const void *W,
-                            int64_t out, const double *abar, const awq_config *cfg, void *ws,
-                            size_t ws_bytes, float *s_best, double *mse, int32_t *best_idx,
-                            awq_stream_t stream) {
-  g_err.clear();
+namespace {
+// The alpha search up to the candidate scores.  sse == NULL: MSE, best and
+// s_best (awq_search_scale); otherwise the unnormalised sums of squared errors
+// of these tokens into sse [n_alpha] (awq_search_scale_sse).
+awq_status search_scale_impl(const void *X, int64_t T, int64_t in, int64_t ldx, const void *W,
+                             int64_t out, const double *abar, const awq_config *cfg, void *ws,
+                             size_t ws_bytes, float *s_best, double *mse, int32_t *best_idx,
+                             double *sse, awq_stream_t stream) {
   awq_status st = check_cfg(cfg);
   if (st != AWQ_OK) return st;
   if ((st = check_shape(T, in, out, cfg)) != AWQ_OK) return st;
   if ((st = check_x(X, in, ldx)) != AWQ_OK) return st;
   if (!W || !aligned(W, 16)) return fail(AWQ_ERR_INVALID_ARG, "W is NULL or not 16-byte aligned");
-  if (!abar || !s_best || !mse || !best_idx) return fail(AWQ_ERR_INVALID_ARG, "an output pointer is NULL");
+  if (!abar || (!sse && (!s_best || !mse || !best_idx)))
+    return fail(AWQ_ERR_INVALID_ARG, "an output pointer is NULL");
   if (in % (cfg->search_form == AWQ_SEARCH_GRAM ? 128 : 64) != 0)
     return fail(AWQ_ERR_UNSUPPORTED, "in=%lld: the %s search needs in %% %d == 0", (long long)in,
                 cfg->search_form == AWQ_SEARCH_GRAM ? "Gram-form" : "direct",
@@ -361,11 +365,81 @@ awq_status awq_search_scale(const void *X, int64_t T, int64_t in, int64_t ldx, c
   }
   {
     ProfScope p("mse_argmin", s);
-    AWQ_TRY_CUDA(launch_mse_argmin(partials, cfg->n_alpha, L.per_alpha, T, out, s_grid, in, dst, mse,
-                                   best_idx, s_best, s),
-                 "mse_argmin launch");
+    if (sse)  // T = out = 1: the plain sums of squared errors
+      AWQ_TRY_CUDA(launch_mse_argmin(partials, cfg->n_alpha, L.per_alpha, 1, 1, s_grid, in, dst, sse,
+                                     nullptr, nullptr, s),
+                   "mse_argmin launch");
+    else
+      AWQ_TRY_CUDA(launch_mse_argmin(partials, cfg->n_alpha, L.per_alpha, T, out, s_grid, in, dst,
+                                     mse, best_idx, s_best, s),
+                   "mse_argmin launch");
   }
   if (getenv("AWQ_SYNC_CHECK")) return awq_device_status(ws, stream);
+  return AWQ_OK;
+}
+}  // namespace
+
+awq_status awq_search_scale(const void *X, int64_t T, int64_t in, int64_t ldx, const void *W,
+                            int64_t out, const double *abar, const awq_config *cfg, void *ws,
+                            size_t ws_bytes, float *s_best, double *mse, int32_t *best_idx,
+                            awq_stream_t stream) {
+  g_err.clear();
+  return search_scale_impl(X, T, in, ldx, W, out, abar, cfg, ws, ws_bytes, s_best, mse, best_idx,
+                           nullptr, stream);
+}
+
+awq_status awq_search_scale_sse(const void *X, int64_t T, int64_t in, int64_t ldx, const void *W,
+                                int64_t out, const double *abar, const awq_config *cfg, void *ws,
+                                size_t ws_bytes, double *sse, awq_stream_t stream) {
+  g_err.clear();
+  if (!sse) return fail(AWQ_ERR_INVALID_ARG, "sse is NULL");
+  return search_scale_impl(X, T, in, ldx, W, out, abar, cfg, ws, ws_bytes, nullptr, nullptr, nullptr,
+                           sse, stream);
+}
+
+awq_status awq_select_scale(const double *sse, int64_t T_total, int64_t in, int64_t out,
+                            const double *abar, const awq_config *cfg, void *ws, size_t ws_bytes,
+                            float *s_best, double *mse, int32_t *best_idx, awq_stream_t stream) {
+  g_err.clear();
+  awq_status st = check_cfg(cfg);
+  if (st != AWQ_OK) return st;
+  if ((st = check_shape(T_total, in, out, cfg)) != AWQ_OK) return st;
+  if (!sse || !abar || !s_best || !mse || !best_idx)
+    return fail(AWQ_ERR_INVALID_ARG, "a pointer argument is NULL");
+  if ((st = check_ws(ws, ws_bytes, kHeader)) != AWQ_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  DevStatus *dst = static_cast<DevStatus *>(ws);
+  AWQ_TRY_CUDA(cudaMemsetAsync(dst, 0, sizeof(DevStatus), s), "workspace reset");
+  ProfScope p("select_scale", s);
+  AWQ_TRY_CUDA(launch_select_scale(sse, cfg->n_alpha, T_total, out, abar, in, dst, mse, best_idx,
+                                   s_best, s),
+               "select_scale launch");
+  return AWQ_OK;
+}
+
+awq_status awq_act_sums(const void *X, int64_t T, int64_t in, int64_t ldx, int64_t *sums,
+                        awq_stream_t stream) {
+  g_err.clear();
+  if (T < 1 || T > (int64_t(1) << 22)) return fail(AWQ_ERR_INVALID_ARG, "T=%lld (1..2^22)", (long long)T);
+  if (in < 8 || in % 8 != 0) return fail(AWQ_ERR_INVALID_ARG, "in=%lld must be a multiple of 8", (long long)in);
+  awq_status st = check_x(X, in, ldx);
+  if (st != AWQ_OK) return st;
+  if (!sums || !aligned(sums, 8)) return fail(AWQ_ERR_INVALID_ARG, "sums is NULL or misaligned");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  ProfScope p("act_stats", s);
+  AWQ_TRY_CUDA(launch_act_sums(static_cast<const __half *>(X), T, in, ldx, sums, s), "act_sums launch");
+  return AWQ_OK;
+}
+
+awq_status awq_act_stats_finish(const int64_t *sums, int64_t T_total, int64_t in, double *abar,
+                                awq_stream_t stream) {
+  g_err.clear();
+  if (T_total < 1 || T_total > (int64_t(1) << 22))
+    return fail(AWQ_ERR_INVALID_ARG, "T_total=%lld (1..2^22)", (long long)T_total);
+  if (in < 1) return fail(AWQ_ERR_INVALID_ARG, "in=%lld", (long long)in);
+  if (!sums || !abar) return fail(AWQ_ERR_INVALID_ARG, "sums or abar is NULL");
+  AWQ_TRY_CUDA(launch_act_finish(sums, in, T_total, abar, static_cast<cudaStream_t>(stream)),
+               "act_finish launch");
   return AWQ_OK;
 }
 
@@ -405,6 +479,57 @@ awq_status awq_search_clip(const void *X, int64_t T, int64_t in, int64_t ldx, co
                                   num_sms_current(), cs),
                  "clip_eval launch");
   }
+  return AWQ_OK;
+}
+
+awq_status awq_block_grams(const void *X, int64_t T, int64_t in, int64_t ldx, const awq_config *cfg,
+                           void *ws, size_t ws_bytes, float *G, awq_stream_t stream) {
+  g_err.clear();
+  awq_status st = check_cfg(cfg);
+  if (st != AWQ_OK) return st;
+  if (cfg->group_size != 128)
+    return fail(AWQ_ERR_UNSUPPORTED, "group_size=%d: block Grams of groups of 128 only", cfg->group_size);
+  if (T < 1 || T > (int64_t(1) << 22)) return fail(AWQ_ERR_INVALID_ARG, "T=%lld (1..2^22)", (long long)T);
+  if (in < 128 || in % 128 != 0 || in > (int64_t(1) << 20))
+    return fail(AWQ_ERR_INVALID_ARG, "in=%lld must be a positive multiple of 128", (long long)in);
+  if ((st = check_x(X, in, ldx)) != AWQ_OK) return st;
+  if (!G || !aligned(G, 16)) return fail(AWQ_ERR_INVALID_ARG, "G is NULL or not 16-byte aligned");
+  const ClipWs L = clip_layout(T, in);
+  if ((st = check_ws(ws, ws_bytes, L.end)) != AWQ_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  uint8_t *base = static_cast<uint8_t *>(ws);
+  AWQ_TRY_CUDA(cudaMemsetAsync(base, 0, sizeof(DevStatus), cs), "workspace reset");
+  ProfScope p("gram_blocks", cs);
+  AWQ_TRY_CUDA(launch_gram_blocks(static_cast<const __half *>(X), T, in, ldx, cfg->group_size,
+                                  L.n_chunks, reinterpret_cast<float *>(base + L.gpart), G,
+                                  reinterpret_cast<DevStatus *>(base), poll_cap(), cs),
+               "gram_blocks launch");
+  return AWQ_OK;
+}
+
+awq_status awq_search_clip_grams(const void *W, int64_t out, int64_t in, const float *s,
+                                 const float *G, const awq_config *cfg, void *ws, size_t ws_bytes,
+                                 uint8_t *clip_idx, float *err, awq_stream_t stream) {
+  g_err.clear();
+  awq_status st = check_cfg(cfg);
+  if (st != AWQ_OK) return st;
+  if (cfg->n_clip < 1) return fail(AWQ_ERR_INVALID_ARG, "n_clip=%d: clip search needs n_clip >= 1", cfg->n_clip);
+  if (cfg->group_size != 128)
+    return fail(AWQ_ERR_UNSUPPORTED, "group_size=%d: the clip search handles groups of 128", cfg->group_size);
+  if ((st = check_shape(1, in, out, cfg)) != AWQ_OK) return st;
+  if (!W || !aligned(W, 16)) return fail(AWQ_ERR_INVALID_ARG, "W is NULL or not 16-byte aligned");
+  if (!G || !aligned(G, 16)) return fail(AWQ_ERR_INVALID_ARG, "G is NULL or not 16-byte aligned");
+  if (!clip_idx) return fail(AWQ_ERR_INVALID_ARG, "clip_idx is NULL");
+  if (s && !aligned(s, 16)) return fail(AWQ_ERR_INVALID_ARG, "s must be 16-byte aligned");
+  if ((st = check_ws(ws, ws_bytes, kHeader)) != AWQ_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  uint8_t *base = static_cast<uint8_t *>(ws);
+  AWQ_TRY_CUDA(cudaMemsetAsync(base, 0, sizeof(DevStatus), cs), "workspace reset");
+  ProfScope p("clip_eval", cs);
+  AWQ_TRY_CUDA(launch_clip_eval(static_cast<const __half *>(W), out, in, s, G, cfg->group_size,
+                                cfg->w_bit, cfg->zero_point, cfg->n_clip, cfg->clip_min, clip_idx, err,
+                                reinterpret_cast<DevStatus *>(base), poll_cap(), num_sms_current(), cs),
+               "clip_eval launch");
   return AWQ_OK;
 }
 

@@ -17,6 +17,18 @@ __host__ __device__ constexpr int64_t i64max(int64_t a, int64_t b) { return a > 
 cudaError_t launch_act_stats(const __half *X, int64_t T, int64_t in, int64_t ldx, double *abar,
                              int num_sms, cudaStream_t stream);
 
+// Token-sharded K1: exact sums of |X| in units of 2^-24 into sums [in]
+// (overwritten), and abar = RN64(RN64(sums 2^-24) / T) from summed sums.
+cudaError_t launch_act_sums(const __half *X, int64_t T, int64_t in, int64_t ldx, int64_t *sums,
+                            cudaStream_t stream);
+cudaError_t launch_act_finish(const int64_t *sums, int64_t in, int64_t T, double *abar,
+                              cudaStream_t stream);
+
+// Token-sharded K5: mse = sse / (T out), best, s_best = s grid row of best.
+cudaError_t launch_select_scale(const double *sse, int n_alpha, int64_t T, int64_t out,
+                                const double *abar, int64_t in, DevStatus *st, double *mse,
+                                int32_t *best_idx, float *s_best, cudaStream_t stream);
+
 // K2: s[i][j] = RN32(pow(max(abar_j, 1e-4), i/(n-1))); inv_s (optional) = RN(1/s).
 cudaError_t launch_scale_grid(const double *abar, int64_t in, int n_alpha, float *s, float *inv_s,
                               cudaStream_t stream);

@@ -95,28 +95,42 @@ __global__ void __launch_bounds__(256) act_stats_kernel(const __half *__restrict
   }
 }
 
-__global__ void act_stats_finish_kernel(double *abar, int64_t in, int64_t T) {
+// abar_j = RN64(RN64(units_j 2^-24) / T); `units` may alias `abar` (each
+// thread reads its element before writing it).
+__global__ void act_stats_finish_kernel(const long long *units, double *abar, int64_t in, int64_t T) {
   int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (j < in) {
-    long long units = reinterpret_cast<long long *>(abar)[j];
-    double S = __ll2double_rn(units) * 5.9604644775390625e-08;  // * 2^-24, exact
+    const long long u = units[j];
+    double S = __ll2double_rn(u) * 5.9604644775390625e-08;  // * 2^-24, exact
     abar[j] = __ddiv_rn(S, (double)T);
   }
+}
+
+cudaError_t launch_act_sums(const __half *X, int64_t T, int64_t in, int64_t ldx, int64_t *sums,
+                            cudaStream_t stream) {
+  cudaError_t e = cudaMemsetAsync(sums, 0, sizeof(int64_t) * in, stream);
+  if (e != cudaSuccess) return e;
+  dim3 block(32, 8);
+  dim3 grid((unsigned)((in + 255) / 256), (unsigned)((T + kStatsChunk - 1) / kStatsChunk));
+  act_stats_kernel<<<grid, block, 0, stream>>>(X, T, in, ldx,
+                                               reinterpret_cast<unsigned long long *>(sums));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_act_finish(const int64_t *sums, int64_t in, int64_t T, double *abar,
+                              cudaStream_t stream) {
+  act_stats_finish_kernel<<<(unsigned)((in + 255) / 256), 256, 0, stream>>>(
+      reinterpret_cast<const long long *>(sums), abar, in, T);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_act_stats(const __half *X, int64_t T, int64_t in, int64_t ldx, double *abar,
                              int num_sms, cudaStream_t stream) {
   (void)num_sms;
-  cudaError_t e = cudaMemsetAsync(abar, 0, sizeof(double) * in, stream);
+  // abar's storage holds the int64 sums until the finish kernel converts them
+  cudaError_t e = launch_act_sums(X, T, in, ldx, reinterpret_cast<int64_t *>(abar), stream);
   if (e != cudaSuccess) return e;
-  dim3 block(32, 8);
-  dim3 grid((unsigned)((in + 255) / 256), (unsigned)((T + kStatsChunk - 1) / kStatsChunk));
-  act_stats_kernel<<<grid, block, 0, stream>>>(X, T, in, ldx,
-                                               reinterpret_cast<unsigned long long *>(abar));
-  e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
-  act_stats_finish_kernel<<<(unsigned)((in + 255) / 256), 256, 0, stream>>>(abar, in, T);
-  return cudaGetLastError();
+  return launch_act_finish(reinterpret_cast<const int64_t *>(abar), in, T, abar, stream);
 }
 
 // ---------------------------------------------------------------------------
@@ -124,17 +138,63 @@ cudaError_t launch_act_stats(const __half *X, int64_t T, int64_t in, int64_t ldx
 // ("AWQ and Activation-Aware Scaling": s = abar^alpha; "05 — AWQ" §4: ~20
 // values of alpha in [0, 1]).  pow is CUDA's double pow.
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ float scale_value(double abar_j, int i, int n_alpha) {
+  const double alpha = n_alpha > 1 ? __ddiv_rn((double)i, (double)(n_alpha - 1)) : 0.0;
+  return __double2float_rn(pow(fmax(abar_j, 1e-4), alpha));
+}
+
 __global__ void scale_grid_kernel(const double *__restrict__ abar, int64_t in, int n_alpha,
                                   float *__restrict__ s, float *__restrict__ inv_s) {
   int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= in * n_alpha) return;
   int i = (int)(idx / in);
   int64_t j = idx - (int64_t)i * in;
-  double alpha = n_alpha > 1 ? __ddiv_rn((double)i, (double)(n_alpha - 1)) : 0.0;
-  double a = fmax(abar[j], 1e-4);
-  float v = __double2float_rn(pow(a, alpha));
+  const float v = scale_value(abar[j], i, n_alpha);
   s[idx] = v;
   if (inv_s) inv_s[idx] = __frcp_rn(v);
+}
+
+// The selection step of a token-sharded search: MSE_i = sse_i / (T out) from
+// the summed squared errors of all shards, best = the first index of the
+// smallest, s_best = the grid's s of that alpha.  Every block finds best on
+// its own (n_alpha <= 64 values); block 0 writes mse and best_idx.
+__global__ void select_scale_kernel(const double *__restrict__ sse, int n_alpha, int64_t T,
+                                    int64_t out, const double *__restrict__ abar, int64_t in,
+                                    DevStatus *st, double *__restrict__ mse,
+                                    int32_t *__restrict__ best_idx, float *__restrict__ s_best) {
+  __shared__ int best_sh;
+  if (threadIdx.x == 0) {
+    const double norm = (double)T * (double)out;
+    int best = 0;
+    double bv = sse[0] / norm;
+    bool finite = isfinite(bv);
+    if (blockIdx.x == 0) mse[0] = bv;
+    for (int a = 1; a < n_alpha; ++a) {
+      const double v = sse[a] / norm;
+      if (blockIdx.x == 0) mse[a] = v;
+      if (!isfinite(v)) finite = false;
+      if (v < bv) {
+        bv = v;
+        best = a;
+      }
+    }
+    if (blockIdx.x == 0) {
+      *best_idx = best;
+      if (!finite) dev_fail(st, kDevNonFinite, 0x510u);
+    }
+    best_sh = best;
+  }
+  __syncthreads();
+  const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (j < in) s_best[j] = scale_value(abar[j], best_sh, n_alpha);
+}
+
+cudaError_t launch_select_scale(const double *sse, int n_alpha, int64_t T, int64_t out,
+                                const double *abar, int64_t in, DevStatus *st, double *mse,
+                                int32_t *best_idx, float *s_best, cudaStream_t stream) {
+  select_scale_kernel<<<(unsigned)((in + 255) / 256), 256, 0, stream>>>(
+      sse, n_alpha, T, out, abar, in, st, mse, best_idx, s_best);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_scale_grid(const double *abar, int64_t in, int n_alpha, float *s, float *inv_s,

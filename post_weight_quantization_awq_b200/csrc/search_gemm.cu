@@ -385,7 +385,8 @@ cudaError_t launch_ref_output(const __half *X, int64_t T, int64_t in, int64_t ld
 // * 2^-2k / (T out).  One block
 // per candidate sums its partials in a fixed order (bitwise reproducible);
 // the last block to finish picks best = the first index of the smallest MSE
-// and copies s_best = s_grid[best].
+// and copies s_best = s_grid[best].  With best_idx = s_best = NULL it only
+// writes the sums (T = out = 1 gives the unnormalised SSE of these tokens).
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(1024) mse_argmin_kernel(
     const double *__restrict__ partials, int n_alpha, size_t per, int64_t T,
@@ -427,9 +428,10 @@ __global__ void __launch_bounds__(1024) mse_argmin_kernel(
     }
     if (!finite) dev_fail(st, kDevNonFinite, 0x500u);
     best_sh = best;
-    *best_idx = best;
+    if (best_idx) *best_idx = best;
   }
   __syncthreads();
+  if (!s_best) return;  // partial sums only (token-sharded search)
   const float *src = s_grid + (size_t)best_sh * in;
   for (int64_t j = threadIdx.x; j < in; j += blockDim.x) s_best[j] = src[j];
 }
