@@ -427,7 +427,8 @@ awq_status awq_act_sums(const void *X, int64_t T, int64_t in, int64_t ldx, int64
   if (!sums || !aligned(sums, 8)) return fail(AWQ_ERR_INVALID_ARG, "sums is NULL or misaligned");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   ProfScope p("act_stats", s);
-  AWQ_TRY_CUDA(launch_act_sums(static_cast<const __half *>(X), T, in, ldx, sums, s), "act_sums launch");
+  AWQ_TRY_CUDA(launch_act_sums(static_cast<const __half *>(X), T, in, ldx, sums, num_sms_current(), s),
+               "act_sums launch");
   return AWQ_OK;
 }
 

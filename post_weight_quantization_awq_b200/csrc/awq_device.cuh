@@ -71,7 +71,11 @@ __device__ __forceinline__ float round_quotient(float x, float delta, float rcp,
 // z = clamp(rne(-mn / delta), 0, 2^b - 1).  Symmetric (sym, no zero point):
 // delta = max(|mx|, |mn|, 1e-5) / (2^(b-1) - 1) and z = 2^(b-1), so codes
 // are centred on z in the same unsigned range [0, 2^b - 1].
-__device__ __forceinline__ GroupQ group_params(float mx, float mn, float r32, float qmax, bool sym) {
+// `guard` is the floor on the range (1e-5; 1e-5 2^k when every value of the
+// group carries an exact factor 2^k, which leaves codes and zero points
+// unchanged and scales delta by exactly 2^k).
+__device__ __forceinline__ GroupQ group_params(float mx, float mn, float r32, float qmax, bool sym,
+                                               float guard = 1e-5f) {
   if (r32 != 1.0f) {
     mx = __fmul_rn(r32, mx);
     mn = __fmul_rn(r32, mn);
@@ -79,14 +83,14 @@ __device__ __forceinline__ GroupQ group_params(float mx, float mn, float r32, fl
   GroupQ g;
   g.qmax = qmax;
   if (sym) {
-    const float d = fmaxf(fmaxf(fabsf(mx), fabsf(mn)), 1e-5f);
+    const float d = fmaxf(fmaxf(fabsf(mx), fabsf(mn)), guard);
     g.delta = __fdiv_rn(d, 0.5f * (qmax - 1.0f));  // 2^(b-1) - 1, exact
     g.rcp = rcp_approx(g.delta);
     g.half_lo = __fmul_rn(g.delta, 0.4999847412109375f /* 0.5 - 2^-16 */);
     g.zero = 0.5f * (qmax + 1.0f);  // 2^(b-1), exact
     return g;
   }
-  const float d = fmaxf(__fsub_rn(mx, mn), 1e-5f);
+  const float d = fmaxf(__fsub_rn(mx, mn), guard);
   g.delta = __fdiv_rn(d, qmax);
   g.rcp = rcp_approx(g.delta);
   g.half_lo = __fmul_rn(g.delta, 0.4999847412109375f /* 0.5 - 2^-16 */);
@@ -115,6 +119,47 @@ __device__ __forceinline__ float2 quant_qz2(float2 wt, const GroupQ &g) {
   q.x = fminf(fmaxf(q.x, 0.0f), g.qmax);
   q.y = fminf(fmaxf(q.y, 0.0f), g.qmax);
   return __fadd2_rn(q, make_float2(-g.zero, -g.zero));
+}
+
+// rne(y) for |y| < 2^22 with two fp32 additions (FMA pipe): y + 1.5 2^23 lies
+// in (2^23, 2^24), where the spacing is 1, so its rounding is 1.5 2^23 +
+// rne(y) (ties to even, 1.5 2^23 being even), and removing 1.5 2^23 is exact.
+__device__ __forceinline__ float2 rne2_small(float2 y) {
+  const float2 m = make_float2(12582912.0f, 12582912.0f);
+  return __fadd2_rn(__fadd2_rn(y, m), make_float2(-12582912.0f, -12582912.0f));
+}
+
+// (q - z) = clamp(rne(RN32(wt/delta)), -z, qmax - z) for 2 NP values of one
+// group whose quotients all lie below 63 in magnitude (the caller checks
+// max|wt| * rcp < 63 for the group, else passes half_lo = -1): proposed by
+// the approximate reciprocal and the small-number rounding, proven by one
+// remainder test for all of them (see round_quotient), decided by the
+// correctly rounded division otherwise.
+template <int NP>
+__device__ __forceinline__ void quant_qz_pairs(const float2 (&wt)[NP], const GroupQ &g,
+                                               float2 (&qz)[NP]) {
+  const float2 rc = make_float2(g.rcp, g.rcp), dl = make_float2(g.delta, g.delta);
+  float rmax = 0.0f;
+#pragma unroll
+  for (int h = 0; h < NP; ++h) {
+    qz[h] = rne2_small(__fmul2_rn(wt[h], rc));
+    const float2 rem = __ffma2_rn(make_float2(-qz[h].x, -qz[h].y), dl, wt[h]);
+    rmax = fmaxf(rmax, fmaxf(fabsf(rem.x), fabsf(rem.y)));
+  }
+  if (!(rmax < g.half_lo)) {
+#pragma unroll
+    for (int h = 0; h < NP; ++h)
+      qz[h] = make_float2(rintf(__fdiv_rn(wt[h].x, g.delta)), rintf(__fdiv_rn(wt[h].y, g.delta)));
+  }
+  const float lo = -g.zero, hi = g.qmax - g.zero;  // exact (small integers)
+#pragma unroll
+  for (int h = 0; h < NP; ++h)
+    qz[h] = make_float2(fminf(fmaxf(qz[h].x, lo), hi), fminf(fmaxf(qz[h].y, lo), hi));
+}
+
+// the group check of quant_qz_pairs: every |wt| <= max(|mx|, |mn|)
+__device__ __forceinline__ void fast_path_check(GroupQ &g, float mx, float mn) {
+  if (!(fmaxf(fabsf(mx), fabsf(mn)) * g.rcp < 63.0f)) g.half_lo = -1.0f;
 }
 
 __device__ __forceinline__ float quant_code(float wt, const GroupQ &g) {

@@ -20,7 +20,7 @@ cudaError_t launch_act_stats(const __half *X, int64_t T, int64_t in, int64_t ldx
 // Token-sharded K1: exact sums of |X| in units of 2^-24 into sums [in]
 // (overwritten), and abar = RN64(RN64(sums 2^-24) / T) from summed sums.
 cudaError_t launch_act_sums(const __half *X, int64_t T, int64_t in, int64_t ldx, int64_t *sums,
-                            cudaStream_t stream);
+                            int num_sms, cudaStream_t stream);
 cudaError_t launch_act_finish(const int64_t *sums, int64_t in, int64_t T, double *abar,
                               cudaStream_t stream);
 

@@ -498,8 +498,7 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
           float rmax = 0.0f;
 #pragma unroll
           for (int h = 0; h < 4; ++h) {
-            const float2 y = __fmul2_rn(wt[h], make_float2(rc, rc));
-            kq[h] = make_float2(rintf(y.x), rintf(y.y));
+            kq[h] = rne2_small(__fmul2_rn(wt[h], make_float2(rc, rc)));
             const float2 rem = __ffma2_rn(make_float2(-kq[h].x, -kq[h].y), make_float2(dl, dl), wt[h]);
             rmax = fmaxf(rmax, fmaxf(fabsf(rem.x), fabsf(rem.y)));
           }

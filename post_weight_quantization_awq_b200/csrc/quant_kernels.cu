@@ -14,84 +14,77 @@ namespace awq {
 // Scaling", Scaling instead of protecting: abar is the per-channel mean
 // activation magnitude; "05 — AWQ" §4 step 1).
 //
-// Each thread owns 8 consecutive channels (one 16-byte load per token row) and
-// sums |x| over its share of a token chunk in fp64 (the fp16 -> fp32 step uses
-// integer operations, keeping the conversion unit for the fp32 -> fp64 step).
-// Every |x| is a multiple
-// of 2^-24 below 2^16, and a chunk holds at most 4096 tokens, so partial sums
-// stay below 2^29 and are exact in fp64.  Chunk sums are then converted to int64
-// units of 2^-24 (exact) and added with 64-bit integer atomics (exact, so the
-// order of arrival does not matter).  Block: 32 x 8 threads covering 256
-// channels x 8 token rows per step.
+// A block sweeps whole token rows (contiguous bytes, good DRAM locality):
+// thread i owns channels 8i..8i+7 of the block's column range and keeps
+// kStatsDepth rows of 16-byte loads in flight in a register ring.  The grid
+// is one wave: column tiles x row splits = SMs x resident blocks.
+//
+// Exact sums without a conversion unit: for an fp16 magnitude h = (e << 10) | m,
+// the fp64 whose high word is h << 10 (low word 0) is 2^(e-1023)(1 + m/1024)
+// for e >= 1 and the subnormal m 2^-1032 for e = 0, i.e. |x| 2^-1008 exactly.
+// These are multiples of 2^-1032 below 2^-992, so fp64 sums of up to 4096 of
+// them (< 2^-980) are exact; every 4096 rows the sum is scaled by 2^1008 2^24
+// (exact) into int64 units of 2^-24 held in registers, and the block's units
+// go to the result with one 64-bit integer atomic per channel (exact in any
+// order).
 // ---------------------------------------------------------------------------
-constexpr int kStatsChunk = 1024;  // tokens per block (<= 4096 keeps fp64 exact)
+constexpr int kStatsDepth = 4;        // rows of loads in flight per thread
+constexpr int kStatsExactRows = 4096;  // rows per exact fp64 partial (multiple of kStatsDepth)
 
-// |x| of the two fp16 values packed in `w`, as fp32, without the conversion
-// unit: shifting a magnitude h = (e << 10) | m into fp32 position gives the
-// fp32 pattern of 2^(e-127) (1 + m/1024) (e >= 1) or of the fp32 subnormal
-// m 2^-136 (e = 0); one exact multiplication by 2^112 yields 2^(e-15)(1 + m/1024)
-// and m 2^-24, the fp16 values.  (fp32 subnormals are kept: no flush-to-zero.)
-__device__ __forceinline__ void abs_half2_alu(uint32_t w, float &lo, float &hi) {
-  lo = __fmul_rn(__uint_as_float((w << 13) & 0x0FFFE000u), 5.192296858534828e+33f /* 2^112 */);
-  hi = __fmul_rn(__uint_as_float((w >> 3) & 0x0FFFE000u), 5.192296858534828e+33f);
+__device__ __forceinline__ double mag_scaled(uint32_t hi_word) {
+  return __hiloint2double((int)hi_word, 0);
 }
 
-__global__ void __launch_bounds__(256) act_stats_kernel(const __half *__restrict__ X, int64_t T,
-                                                        int64_t in, int64_t ldx,
-                                                        unsigned long long *__restrict__ acc) {
-  __shared__ double red[8][32][8];
-  const int tx = threadIdx.x, ty = threadIdx.y;
-  const int64_t c0 = ((int64_t)blockIdx.x * 32 + tx) * 8;  // first channel of this thread
-  const int64_t t_begin = (int64_t)blockIdx.y * kStatsChunk;
-  const int64_t t_end = min(T, t_begin + kStatsChunk);
-  double s64[8];
+__global__ void __launch_bounds__(1024) act_stats_kernel(const __half *__restrict__ X, int64_t T,
+                                                         int64_t in, int64_t ldx,
+                                                         int64_t rows_per_block,
+                                                         unsigned long long *__restrict__ acc) {
+  const int64_t c0 = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8;
+  const int64_t t0 = (int64_t)blockIdx.y * rows_per_block;
+  const int64_t t1 = min(T, t0 + rows_per_block);
+  if (c0 >= in || t0 >= t1) return;  // no block-wide synchronisation below
+  const __half *p = X + c0;
+  double sb[8];
+  unsigned long long units[8];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) s64[e] = 0.0;
-  if (c0 < in) {
-    int64_t t = t_begin + ty;
-    // four rows in flight per thread
-    for (; t + 24 < t_end; t += 32) {
-      uint4 v[4];
+  for (int e = 0; e < 8; ++e) {
+    sb[e] = 0.0;
+    units[e] = 0ull;
+  }
+  uint4 v[kStatsDepth];
 #pragma unroll
-      for (int u = 0; u < 4; ++u)
-        v[u] = __ldcs(reinterpret_cast<const uint4 *>(X + (t + 8 * u) * ldx + c0));
+  for (int u = 0; u < kStatsDepth; ++u)
+    v[u] = t0 + u < t1 ? __ldcs(reinterpret_cast<const uint4 *>(p + (t0 + u) * ldx))
+                       : make_uint4(0u, 0u, 0u, 0u);
+  int since = 0;
+  for (int64_t t = t0; t < t1; t += kStatsDepth) {
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-#pragma unroll
-        for (int h = 0; h < 4; ++h) {
-          float a, b;
-          abs_half2_alu(w[h], a, b);
-          s64[2 * h] += (double)a;
-          s64[2 * h + 1] += (double)b;
-        }
-      }
-    }
-    for (; t < t_end; t += 8) {
-      const uint4 v = __ldcs(reinterpret_cast<const uint4 *>(X + t * ldx + c0));
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    for (int u = 0; u < kStatsDepth; ++u) {
+      // rows past t1 were loaded as zeros and add nothing
+      const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
       for (int h = 0; h < 4; ++h) {
-        float a, b;
-        abs_half2_alu(w[h], a, b);
-        s64[2 * h] += (double)a;
-        s64[2 * h + 1] += (double)b;
+        sb[2 * h] += mag_scaled((w[h] << 10) & 0x01FFFC00u);
+        sb[2 * h + 1] += mag_scaled((w[h] >> 6) & 0x01FFFC00u);
       }
+      const int64_t nx = t + u + kStatsDepth;
+      v[u] = nx < t1 ? __ldcs(reinterpret_cast<const uint4 *>(p + nx * ldx))
+                     : make_uint4(0u, 0u, 0u, 0u);
+    }
+    since += kStatsDepth;
+    if (since == kStatsExactRows) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        units[e] += __double2ull_rn(__dmul_rn(__dmul_rn(sb[e], 0x1p1008), 0x1p24));
+        sb[e] = 0.0;
+      }
+      since = 0;
     }
   }
 #pragma unroll
-  for (int e = 0; e < 8; ++e) red[ty][tx][e] = s64[e];
-  __syncthreads();
-  if (ty == 0 && c0 < in) {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      double tot = 0.0;
-#pragma unroll
-      for (int r = 0; r < 8; ++r) tot += red[r][tx][e];
-      // exact: tot is a multiple of 2^-24 below 2^29
-      unsigned long long units = (unsigned long long)(tot * 16777216.0);
-      if (units) atomicAdd(&acc[c0 + e], units);
-    }
+  for (int e = 0; e < 8; ++e) {
+    units[e] += __double2ull_rn(__dmul_rn(__dmul_rn(sb[e], 0x1p1008), 0x1p24));
+    if (units[e]) atomicAdd(&acc[c0 + e], units[e]);
   }
 }
 
@@ -107,13 +100,20 @@ __global__ void act_stats_finish_kernel(const long long *units, double *abar, in
 }
 
 cudaError_t launch_act_sums(const __half *X, int64_t T, int64_t in, int64_t ldx, int64_t *sums,
-                            cudaStream_t stream) {
+                            int num_sms, cudaStream_t stream) {
   cudaError_t e = cudaMemsetAsync(sums, 0, sizeof(int64_t) * in, stream);
   if (e != cudaSuccess) return e;
-  dim3 block(32, 8);
-  dim3 grid((unsigned)((in + 255) / 256), (unsigned)((T + kStatsChunk - 1) / kStatsChunk));
-  act_stats_kernel<<<grid, block, 0, stream>>>(X, T, in, ldx,
-                                               reinterpret_cast<unsigned long long *>(sums));
+  // column tiles of at most 1024 threads x 8 channels, split evenly
+  const int64_t vec = in / 8;
+  const int64_t ntiles = (vec + 1023) / 1024;
+  const int64_t nthr = ((vec + ntiles - 1) / ntiles + 31) / 32 * 32;
+  const int64_t per_sm = i64max(1, 2048 / nthr);  // resident blocks per SM (64 registers)
+  int64_t splits = i64max(1, i64min(T, (int64_t)(num_sms > 0 ? num_sms : 148) * per_sm / ntiles));
+  const int64_t rows = (T + splits - 1) / splits;
+  splits = (T + rows - 1) / rows;
+  dim3 grid((unsigned)ntiles, (unsigned)splits);
+  act_stats_kernel<<<grid, (unsigned)nthr, 0, stream>>>(X, T, in, ldx, rows,
+                                                        reinterpret_cast<unsigned long long *>(sums));
   return cudaGetLastError();
 }
 
@@ -126,9 +126,8 @@ cudaError_t launch_act_finish(const int64_t *sums, int64_t in, int64_t T, double
 
 cudaError_t launch_act_stats(const __half *X, int64_t T, int64_t in, int64_t ldx, double *abar,
                              int num_sms, cudaStream_t stream) {
-  (void)num_sms;
   // abar's storage holds the int64 sums until the finish kernel converts them
-  cudaError_t e = launch_act_sums(X, T, in, ldx, reinterpret_cast<int64_t *>(abar), stream);
+  cudaError_t e = launch_act_sums(X, T, in, ldx, reinterpret_cast<int64_t *>(abar), num_sms, stream);
   if (e != cudaSuccess) return e;
   return launch_act_finish(reinterpret_cast<const int64_t *>(abar), in, T, abar, stream);
 }
@@ -261,9 +260,14 @@ __global__ void __launch_bounds__(256) cand_quant_kernel(
     const float *__restrict__ s, const float *__restrict__ inv_s, const float *__restrict__ rch,
     int group, float qmax, int sym, int weights_only, const DevStatus *__restrict__ st,
     __half *__restrict__ dW) {
+  // Everything runs on s 2^k: codes and zero points are those of s (power-of-
+  // two invariance), delta comes out times 2^k, and the candidate error
+  // (deq - s w) 2^k (r / s) needs one FFMA2 and one FMUL2 per pair.  It drops
+  // the rounding residual (RN32(s w)/s - w) 2^k, below 2^-22 of the error
+  // it is added to, far under the fp16 rounding that follows.
   const int k = weights_only ? 0 : kscale_from_wmax(__uint_as_float(__ldg(&st->wmax_bits)));
   const float two_k = ldexpf(1.0f, k);
-  const float wneg = weights_only ? 0.0f : -two_k;  // coefficient of w
+  const float guard = __fmul_rn(1e-5f, two_k);  // exact
   const int lanes = group / 8;  // lanes per group (a power of two <= 32)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t j0 = (int64_t)blockIdx.y * 256 + lane * 8;
@@ -271,50 +275,47 @@ __global__ void __launch_bounds__(256) cand_quant_kernel(
   const int rb_per_alpha = (int)(out_pad / kCandRows);
   const int a = (int)(blockIdx.x / rb_per_alpha);
   const int64_t o0 = (int64_t)(blockIdx.x - (int64_t)a * rb_per_alpha) * kCandRows;
-  float sv[8], iv[8], rv[8] = {1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f, 1.f};
+  float2 sk[4], iv[4];  // s 2^k and r / s of this lane's 8 channels
   if (j_ok) {
     const float4 *sp = reinterpret_cast<const float4 *>(s + (int64_t)a * in + j0);
     const float4 *ip = reinterpret_cast<const float4 *>(inv_s + (int64_t)a * in + j0);
     const float4 s0 = __ldg(sp), s1 = __ldg(sp + 1), i0 = __ldg(ip), i1 = __ldg(ip + 1);
-    sv[0] = s0.x; sv[1] = s0.y; sv[2] = s0.z; sv[3] = s0.w;
-    sv[4] = s1.x; sv[5] = s1.y; sv[6] = s1.z; sv[7] = s1.w;
-    iv[0] = i0.x; iv[1] = i0.y; iv[2] = i0.z; iv[3] = i0.w;
-    iv[4] = i1.x; iv[5] = i1.y; iv[6] = i1.z; iv[7] = i1.w;
+    const float2 tk = make_float2(two_k, two_k);
+    sk[0] = __fmul2_rn(make_float2(s0.x, s0.y), tk);
+    sk[1] = __fmul2_rn(make_float2(s0.z, s0.w), tk);
+    sk[2] = __fmul2_rn(make_float2(s1.x, s1.y), tk);
+    sk[3] = __fmul2_rn(make_float2(s1.z, s1.w), tk);
+    iv[0] = make_float2(i0.x, i0.y);
+    iv[1] = make_float2(i0.z, i0.w);
+    iv[2] = make_float2(i1.x, i1.y);
+    iv[3] = make_float2(i1.z, i1.w);
     if (rch) {  // Gram form: d~ = r_j (deq/s - w)
       const float4 r0 = __ldg(reinterpret_cast<const float4 *>(rch + j0));
       const float4 r1 = __ldg(reinterpret_cast<const float4 *>(rch + j0) + 1);
-      rv[0] = r0.x; rv[1] = r0.y; rv[2] = r0.z; rv[3] = r0.w;
-      rv[4] = r1.x; rv[5] = r1.y; rv[6] = r1.z; rv[7] = r1.w;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) iv[e] *= rv[e];
+      iv[0] = __fmul2_rn(iv[0], make_float2(r0.x, r0.y));
+      iv[1] = __fmul2_rn(iv[1], make_float2(r0.z, r0.w));
+      iv[2] = __fmul2_rn(iv[2], make_float2(r1.x, r1.y));
+      iv[3] = __fmul2_rn(iv[3], make_float2(r1.z, r1.w));
     }
   } else {
 #pragma unroll
-    for (int e = 0; e < 8; ++e) { sv[e] = 1.0f; iv[e] = 1.0f; }
+    for (int h = 0; h < 4; ++h) {
+      sk[h] = make_float2(two_k, two_k);
+      iv[h] = make_float2(1.0f, 1.0f);
+    }
   }
 #pragma unroll 2
   for (int r = warp; r < kCandRows; r += 8) {
     const int64_t o = o0 + r;
     const bool live = j_ok && o < out;
-    float w[8];
-    if (live) {
-      const uint4 wv = __ldg(reinterpret_cast<const uint4 *>(W + o * in + j0));
-      const uint32_t wr[4] = {wv.x, wv.y, wv.z, wv.w};
-#pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        const float2 f = __half22float2(*reinterpret_cast<const __half2 *>(&wr[h]));
-        w[2 * h] = f.x;
-        w[2 * h + 1] = f.y;
-      }
-    } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) w[e] = 0.0f;
-    }
+    uint4 wv = make_uint4(0u, 0u, 0u, 0u);
+    if (live) wv = __ldg(reinterpret_cast<const uint4 *>(W + o * in + j0));
+    const uint32_t wr[4] = {wv.x, wv.y, wv.z, wv.w};
     float2 wt[4];
     float mx = -INFINITY, mn = INFINITY;
 #pragma unroll
     for (int h = 0; h < 4; ++h) {
-      wt[h] = __fmul2_rn(make_float2(sv[2 * h], sv[2 * h + 1]), make_float2(w[2 * h], w[2 * h + 1]));
+      wt[h] = __fmul2_rn(sk[h], __half22float2(*reinterpret_cast<const __half2 *>(&wr[h])));
       mx = fmaxf(mx, fmaxf(wt[h].x, wt[h].y));
       mn = fminf(mn, fminf(wt[h].x, wt[h].y));
     }
@@ -322,18 +323,19 @@ __global__ void __launch_bounds__(256) cand_quant_kernel(
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
       mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
     }
-    const GroupQ g = group_params(mx, mn, 1.0f, qmax, sym != 0);
-    const float dk = __fmul_rn(g.delta, two_k);  // exact: power-of-two scaling
+    GroupQ g = group_params(mx, mn, 1.0f, qmax, sym != 0, guard);
+    fast_path_check(g, mx, mn);
+    float2 qz[4];
+    quant_qz_pairs<4>(wt, g, qz);
+    const float2 dl = make_float2(g.delta, g.delta);
     uint32_t packed[4];
 #pragma unroll
     for (int h = 0; h < 4; ++h) {
-      // 2^k (deq/s - w) with deq = (q - z) delta (weights_only: deq/s); the
-      // product with 1/s is fp32 (the result is rounded to fp16 next)
-      const float2 qz = quant_qz2(wt[h], g);
-      float2 d2 = __ffma2_rn(__fmul2_rn(qz, make_float2(dk, dk)), make_float2(iv[2 * h], iv[2 * h + 1]),
-                             __fmul2_rn(make_float2(w[2 * h], w[2 * h + 1]),
-                                        make_float2(wneg * rv[2 * h], wneg * rv[2 * h + 1])));
-      if (!live) d2 = make_float2(0.0f, 0.0f);
+      // error form: (deq - s w) 2^k (r / s); weights only: deq / s
+      const float2 t = weights_only ? __fmul2_rn(qz[h], dl)
+                                    : __ffma2_rn(qz[h], dl, make_float2(-wt[h].x, -wt[h].y));
+      // rows past `out` and channels past `in` hold w = 0, which gives 0 here
+      const float2 d2 = __fmul2_rn(t, iv[h]);
       const __half2 hv = __floats2half2_rn(d2.x, d2.y);
       packed[h] = *reinterpret_cast<const uint32_t *>(&hv);
     }
@@ -427,22 +429,24 @@ __global__ void __launch_bounds__(256) quant_pack_kernel(
     const uint2 wv = *reinterpret_cast<const uint2 *>(&wsm[r][lane * 4]);
     const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&wv.x));
     const float2 b = __half22float2(*reinterpret_cast<const __half2 *>(&wv.y));
-    const float wt[4] = {__fmul_rn(sv[0], a.x), __fmul_rn(sv[1], a.y), __fmul_rn(sv[2], b.x),
-                         __fmul_rn(sv[3], b.y)};
-    float mx = fmaxf(fmaxf(wt[0], wt[1]), fmaxf(wt[2], wt[3]));
-    float mn = fminf(fminf(wt[0], wt[1]), fminf(wt[2], wt[3]));
+    const float2 wt[2] = {__fmul2_rn(make_float2(sv[0], sv[1]), a), __fmul2_rn(make_float2(sv[2], sv[3]), b)};
+    float mx = fmaxf(fmaxf(wt[0].x, wt[0].y), fmaxf(wt[1].x, wt[1].y));
+    float mn = fminf(fminf(wt[0].x, wt[0].y), fminf(wt[1].x, wt[1].y));
     for (int off = gl >> 1; off > 0; off >>= 1) {
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
       mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
     }
     if (!lane_ok) continue;  // past the last channel (its lanes form whole groups)
     const float r32 = clip_idx ? ratios[clip_idx[o * groups + kg]] : 1.0f;
-    const GroupQ g = group_params(mx, mn, r32, qmax, sym != 0);
-    uchar4 c4;
-    c4.x = (uint8_t)quant_code(wt[0], g);
-    c4.y = (uint8_t)quant_code(wt[1], g);
-    c4.z = (uint8_t)quant_code(wt[2], g);
-    c4.w = (uint8_t)quant_code(wt[3], g);
+    GroupQ g = group_params(mx, mn, r32, qmax, sym != 0);
+    fast_path_check(g, mx, mn);  // mx, mn: the unclipped extremes, which bound every |wt|
+    float2 qz[2];
+    quant_qz_pairs<2>(wt, g, qz);
+    uchar4 c4;  // q = (q - z) + z, exact small integers
+    c4.x = (uint8_t)__fadd_rn(qz[0].x, g.zero);
+    c4.y = (uint8_t)__fadd_rn(qz[0].y, g.zero);
+    c4.z = (uint8_t)__fadd_rn(qz[1].x, g.zero);
+    c4.w = (uint8_t)__fadd_rn(qz[1].y, g.zero);
     *reinterpret_cast<uchar4 *>(&codes[r][lane * 4]) = c4;
     if ((lane & (gl - 1)) == 0) {  // first lane of the group
       zeros[r][gi] = (uint8_t)g.zero;
