@@ -382,7 +382,7 @@ __device__ __forceinline__ float clip_ratio(int c, int n_clip, float clip_min) {
 // is contiguous.
 constexpr int kPackTile = 128;
 
-__global__ void __launch_bounds__(256) quant_pack_kernel(
+__global__ void __launch_bounds__(256, 6) quant_pack_kernel(
     const __half *__restrict__ W, int64_t out, int64_t in, int group, const float *__restrict__ s,
     const uint8_t *__restrict__ clip_idx, int n_clip, float clip_min, float qmax, int sym,
     int32_t *__restrict__ qweight, int32_t *__restrict__ qzeros, __half *__restrict__ scales) {
