@@ -246,10 +246,11 @@ cudaError_t launch_gram_blocks(const __half *X, int64_t T, int64_t in, int64_t l
 // cross-thread reduction is needed.  The dropped A_lo G~_lo term is 2^-22 of E.
 // ---------------------------------------------------------------------------
 namespace {
-constexpr int CW_PROD = 8;                        // producer warps 0..7
-constexpr int CW_MMA = 8;                         // MMA warp
-constexpr int CW_EPI = 9;                         // epilogue warps 9..12
-constexpr int CT_THREADS = 13 * 32;
+constexpr int CW_PROD = 12;                       // producer warps 0..11
+constexpr int CW_MMA = 12;                        // MMA warp
+constexpr int CW_EPI = 13;                        // epilogue warps 13..16
+constexpr int CW_NEPI = 4;                        // one per TMEM lane quarter
+constexpr int CT_THREADS = (CW_EPI + CW_NEPI) * 32;  // 17 warps: up to 120 registers
 constexpr int CT_MAXR = 32;                       // rows per tile at most
 constexpr uint32_t CT_ATOM = 128 * 128;           // bytes: 128 rows x 64 fp16
 constexpr uint32_t CT_OPND = 2 * CT_ATOM;         // one operand, K = 128
@@ -309,8 +310,9 @@ __device__ __forceinline__ float clip_ratio_f(int c, int n_clip, float clip_min)
 }  // namespace
 
 // Warp-specialised pipeline over (group, row tile) items, two tiles in
-// flight: producers (warps 0-7) build tile t's candidates while the MMA warp
-// runs tile t-1 and the epilogue warps (9-12) score and pick tile t-2.
+// flight: producers (warps 0-11, three per SM sub-partition) build tile t's
+// candidates while the MMA warp runs tile t-1 and the epilogue warps (13-16)
+// score and pick tile t-2.
 __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
     const __half *__restrict__ W, int64_t out, int64_t in, const float *__restrict__ s,
     const float *__restrict__ Gall, float qmax, int sym, int n_clip, float clip_min, int rows_per_tile,
@@ -332,9 +334,9 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
   if (tid == 0) {
     for (int b = 0; b < 2; ++b) {
       mbar_init(&S.a_full[b], CW_PROD);
-      mbar_init(&S.a_empty[b], 4);
+      mbar_init(&S.a_empty[b], CW_NEPI);
       mbar_init(&S.acc_full[b], 1);
-      mbar_init(&S.acc_empty[b], 4);
+      mbar_init(&S.acc_empty[b], CW_NEPI);
     }
     mbar_init(&S.mma_done, 1);
     S.abort_flag = 0;
@@ -358,7 +360,7 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
     // share the row, and walks ratios sp, sp + nsp, ... < n_clip; lane l of
     // the 16 computes the group parameters of its split's l-th ratio once,
     // and the others take them by shuffle.
-    const int ptid = tid;  // 0..255
+    const int ptid = tid;  // 0..CW_PROD*32-1
     const int ch = ptid & 15;
     const int nrc = 16 * R;                          // (row, chunk) slots
     const int nsp = nrc >= CW_PROD * 32 ? 1 : (CW_PROD * 32) / nrc;
@@ -411,13 +413,13 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
           S.ar[ptid] = r0 / s0;
         }
         named_bar(1, CW_PROD * 32);
-        // row j, channels 64 h .. 64 h + 63; a warp shares h, so its
-        // swizzled 16-byte stores fall in distinct banks
+        // row j, channels 64 h .. 64 h + 63 (threads 0..255); a warp shares h,
+        // so its swizzled 16-byte stores fall in distinct banks
         const int j = ptid & 127, h = ptid >> 7;
         const float rj = S.r[j];
         const float *grow = Gk + (int64_t)j * G + 64 * h;
 #pragma unroll 1
-        for (int c = 0; c < 8; ++c) {
+        for (int c = 0; c < (ptid < 256 ? 8 : 0); ++c) {
           float v[8];
           const float4 g0 = __ldg(reinterpret_cast<const float4 *>(grow + 8 * c));
           const float4 g1 = __ldg(reinterpret_cast<const float4 *>(grow + 8 * c + 4));
@@ -484,14 +486,14 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
         }
         const int p0 = rr * n_clip;
         uint8_t *ahi = S.a_hi[b] + (ch >> 3) * CT_ATOM, *alo = S.a_lo[b] + (ch >> 3) * CT_ATOM;
-#pragma unroll 1
-        for (int jc = 0; jc < cper; ++jc) {
+#pragma unroll 2
+        for (int jc = 0; jc < cper; ++jc) {  // two ratios interleaved: more independent work
           const float dl = __shfl_sync(0xffffffffu, gq.delta, jc, 16);
           const float rc = __shfl_sync(0xffffffffu, gq.rcp, jc, 16);
           const float hl = __shfl_sync(0xffffffffu, gq.half_lo, jc, 16);
           const float zz = __shfl_sync(0xffffffffu, gq.zero, jc, 16);
           const int c = sp + nsp * jc;
-          if (!live || c >= n_clip) continue;
+          const bool store = live && c < n_clip;  // past n_clip: lane 0's ratio, not stored
           // (q - z) = clamp(rne(wt / delta), -z, qmax - z), proposed from the
           // approximate reciprocal and proven by the remainder
           float2 kq[4];
@@ -518,7 +520,7 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
             v[2 * h] = d2.x;
             v[2 * h + 1] = d2.y;
           }
-          split_store8(ahi, alo, sw128_off(p0 + c, ch & 7), v);
+          if (store) split_store8(ahi, alo, sw128_off(p0 + c, ch & 7), v);
         }
       }
       if (item + 1 < item_end) load_rows(item + 1);
@@ -584,7 +586,7 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
         }
         S.epi_ok = ok;
       }
-      named_bar(2, 128);
+      named_bar(2, CW_NEPI * 32);
       if (!S.epi_ok) break;
       tc_fence_after();
       // E = d~ . y over the 128 columns of this candidate's accumulator row
@@ -618,16 +620,22 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.acc_empty[b]);
       S.epart[b][p] = e;
-      named_bar(2, 128);
+      // the argmin below needs only epart (this group's) and its row's
+      // exponent: take the exponent now and release A, the row data and the
+      // buffer to the producers as soon as every dot is done
+      const int rr = etid >> 2, part = etid & 3;
+      const int rexp_row = S.rexp[b][rr];  // rr < 32
+      named_bar(2, CW_NEPI * 32);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.a_empty[b]);
       // ---- per row: first clip index with the smallest E; four threads per
       // row scan every fourth ratio, then combine (ties keep the lower index)
       {
-        const int rr = etid >> 2, part = etid & 3;
         const bool row_ok = rr < R && o0 + rr < out;
         float best = INFINITY;
         int bc = 1 << 30;
         if (row_ok) {
-          const float unscale = ldexpf(1.0f, -2 * S.rexp[b][rr]);
+          const float unscale = ldexpf(1.0f, -2 * rexp_row);
           for (int c = part; c < n_clip; c += 4) {
             const float ev = S.epart[b][rr * n_clip + c] * unscale;
             if (err) err[((o0 + rr) * n_groups + k) * n_clip + c] = ev;
@@ -648,8 +656,6 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
         }
         if (row_ok && part == 0) clip_idx[(o0 + rr) * n_groups + k] = (uint8_t)bc;
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&S.a_empty[b]);  // A, rows and partial sums of tile t reusable
     }
   }
   tc_fence_before();
