@@ -62,6 +62,8 @@ __all__ = [
     "search_clip",
     "quant_pack",
     "unpack_nibbles",
+    "dequant_packed",
+    "w4a16_matmul",
     "fold_inv_scale",
 ]
 
@@ -335,6 +337,30 @@ def unpack_nibbles(words: np.ndarray) -> np.ndarray:
     for e in range(8):
         q[e::8, :] = ((u >> np.uint32(4 * e)) & np.uint32(0xF)).T.astype(np.uint8)
     return q
+
+
+# --------------------------------------------------------------------------
+# The step after the path: a W4A16 product on the packed output  ([P4] §5
+# layout; the pages' inference kernels dequantise the weights on the fly)
+# --------------------------------------------------------------------------
+def dequant_packed(qweight: np.ndarray, qzeros: np.ndarray, scales: np.ndarray,
+                   group: int) -> np.ndarray:
+    """fp16 weights [out, in] of a packed layer: RN16((q - z) * scale), with q
+    from qweight [in, out/8], z from qzeros [in/g, out/8] and scale from
+    scales [in/g, out].  (q - z) * scale is exact in fp32 (a small integer times
+    an fp16), so the one rounding is the final RN16."""
+    q = unpack_nibbles(qweight).astype(np.float32)                        # [out, in]
+    z = np.repeat(unpack_nibbles(qzeros).astype(np.float32), group, axis=1)
+    sc = np.repeat(np.asarray(scales).astype(np.float32).T, group, axis=1)
+    return ((q - z) * sc).astype(np.float16)
+
+
+def w4a16_matmul(X: np.ndarray, qweight: np.ndarray, qzeros: np.ndarray, scales: np.ndarray,
+                 group: int) -> np.ndarray:
+    """Y = X Wd^T in fp64 with Wd = dequant_packed(...) (the GPU accumulates in
+    fp32 and rounds Y to fp16)."""
+    Wd = dequant_packed(qweight, qzeros, scales, group).astype(np.float64)
+    return np.asarray(X, dtype=np.float64) @ Wd.T
 
 
 # --------------------------------------------------------------------------

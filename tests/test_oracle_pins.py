@@ -490,3 +490,37 @@ def test_pack_without_zero_point(w_bit):
     assert np.array_equal(q, qd["q"])
     deq16 = (q - nib) * np.repeat(sc.T.astype(np.float64), 128, axis=1)
     assert np.allclose(deq16, qd["deq"], rtol=2.0 ** -10, atol=0)
+
+
+# --------------------------------------------------------------------------
+# The W4A16 product on the packed output
+# --------------------------------------------------------------------------
+def test_w4a16_exact_on_the_hand_worked_packing(golden):
+    """The hand-worked packing example has step 1 and zero 8, so the packed
+    weights dequantise to W itself; with integer X the product is exact."""
+    W = np.zeros((16, 128), dtype=np.float16)
+    for o in range(16):
+        for j in range(8):
+            W[o, j] = ((o + j) % 16) - 8
+        W[o, 126], W[o, 127] = -8.0, 7.0
+    qw, qz, sc = O.quant_pack(W, None, None, 4, 128)
+    assert np.all(sc == np.float16(1.0))
+    assert np.array_equal(O.dequant_packed(qw, qz, sc, 128), W)
+    X = np.random.default_rng(3).integers(-3, 4, size=(9, 128)).astype(np.float16)
+    want = X.astype(np.int64) @ W.astype(np.int64).T
+    assert np.array_equal(O.w4a16_matmul(X, qw, qz, sc, 128), want.astype(np.float64))
+
+
+@pytest.mark.parametrize("w_bit,group,zp", [(4, 128, True), (3, 64, True), (4, 32, False)])
+def test_w4a16_weights_within_half_a_step(w_bit, group, zp):
+    """Dequantised packed weights sit within half a step of the weights they
+    came from (s = 1, no clip, groups spanning 0), up to the fp16 rounding of
+    the stored step and of the product."""
+    _, W = random_layer(4, 256, 32, seed=19)
+    Wn = W.numpy()
+    qw, qz, sc = O.quant_pack(Wn, None, None, w_bit, group, zero_point=zp)
+    Wd = O.dequant_packed(qw, qz, sc, group).astype(np.float64)
+    step = np.repeat(sc.astype(np.float64).T, group, axis=1)
+    qmax = 2 ** w_bit - 1
+    bound = step * (0.5 + qmax * 2.0 ** -11) + np.abs(Wd) * 2.0 ** -11
+    assert np.all(np.abs(Wd - Wn.astype(np.float64)) <= bound)
