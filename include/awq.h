@@ -259,6 +259,25 @@ awq_status awq_search_clip_grams(const void *W, int64_t out, int64_t in, const f
                                  const float *G, const awq_config *cfg, void *ws, size_t ws_bytes,
                                  uint8_t *clip_idx, float *err, awq_stream_t stream);
 
+/* W4A16 GEMM on the packed output, the step after the search ("05 — AWQ" §5
+ * layout; the weights are dequantised on the fly inside the GEMM, as the
+ * pages describe for AWQ's inference kernels):
+ *   Y[t][o] = RN16( sum_j X[t][j] Wd[o][j] ),  Wd[o][j] = RN16((q - z) scale)
+ * with q the 4-bit code of (o, j) (nibble o % 8 of qweight[j][o/8]), z that of
+ * qzeros[j/g][o/8] and scale = scales[j/g][o]; fp32 accumulation on the tensor
+ * cores.  INT3 codes use the same nibbles.
+ *   X        device fp16 [T, in], row stride ldx
+ *   qweight  device int32 [in, out/8]; qzeros int32 [in/g, out/8]; scales fp16 [in/g, out]
+ *   Y        device fp16 [T, out] (output), row stride ldy (multiple of 8)
+ *   ws       at least 256 bytes (status word)
+ * Uses cfg->group_size (32, 64 or 128); requires in % 64 == 0 and out % 32 == 0
+ * (the packed words of a row are staged by TMA, whose row stride must be a
+ * multiple of 16 bytes). */
+awq_status awq_w4a16_gemm(const void *X, int64_t T, int64_t in, int64_t ldx, const int32_t *qweight,
+                          const int32_t *qzeros, const void *scales, int64_t out,
+                          const awq_config *cfg, void *Y, int64_t ldy, void *ws, size_t ws_bytes,
+                          awq_stream_t stream);
+
 /* Synchronises `stream`, then returns and clears the device status recorded in
  * workspace `ws` (AWQ_OK, AWQ_ERR_TIMEOUT or AWQ_ERR_NONFINITE). */
 awq_status awq_device_status(void *ws, awq_stream_t stream);

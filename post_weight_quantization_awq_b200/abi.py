@@ -80,6 +80,9 @@ _SIGNATURES = {
     "awq_quant_pack": (c_int32, [c_void_p, c_int64, c_int64, c_void_p, c_void_p, POINTER(AwqConfig),
                                  c_void_p, c_void_p, c_void_p, c_void_p]),
     "awq_fold_inv_scale": (c_int32, [c_void_p, c_int64, c_int64, c_void_p, c_void_p]),
+    "awq_w4a16_gemm": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_void_p, c_void_p,
+                                 c_int64, POINTER(AwqConfig), c_void_p, c_int64, c_void_p, c_size_t,
+                                 c_void_p]),
     "awq_act_sums": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_void_p]),
     "awq_act_stats_finish": (c_int32, [c_void_p, c_int64, c_int64, c_void_p, c_void_p]),
     "awq_search_scale_sse": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_int64,
@@ -256,6 +259,14 @@ def awq_search_clip_grams(W, s, G, cfg: AwqConfig, ws, clip_idx, err=None, strea
     _check("awq_search_clip_grams", LIB.awq_search_clip_grams(
         _ptr(W), W.shape[0], W.shape[1], _ptr(s), _ptr(G), ctypes.byref(cfg), _ptr(ws),
         ws.numel() * ws.element_size(), _ptr(clip_idx), _ptr(err), _stream(stream)))
+
+
+def awq_w4a16_gemm(X, qweight, qzeros, scales, cfg: AwqConfig, Y, ws, stream=None) -> None:
+    """Y [T, out] fp16 = X [T, in] times the packed weights, dequantised on the fly."""
+    _check("awq_w4a16_gemm", LIB.awq_w4a16_gemm(
+        _ptr(X), X.shape[0], X.shape[1], X.stride(0), _ptr(qweight), _ptr(qzeros), _ptr(scales),
+        Y.shape[1], ctypes.byref(cfg), _ptr(Y), Y.stride(0), _ptr(ws), ws.numel() * ws.element_size(),
+        _stream(stream)))
 
 
 def awq_device_status(ws, stream=None) -> None:

@@ -556,6 +556,35 @@ awq_status awq_quant_pack(const void *W, int64_t out, int64_t in, const float *s
   return AWQ_OK;
 }
 
+awq_status awq_w4a16_gemm(const void *X, int64_t T, int64_t in, int64_t ldx, const int32_t *qweight,
+                          const int32_t *qzeros, const void *scales, int64_t out,
+                          const awq_config *cfg, void *Y, int64_t ldy, void *ws, size_t ws_bytes,
+                          awq_stream_t stream) {
+  g_err.clear();
+  awq_status st = check_cfg(cfg);
+  if (st != AWQ_OK) return st;
+  if ((st = check_shape(T, in, out, cfg)) != AWQ_OK) return st;
+  if (in % 64 != 0 || out % 32 != 0)
+    return fail(AWQ_ERR_UNSUPPORTED, "in=%lld, out=%lld: the W4A16 GEMM needs in %% 64 == 0 and out %% 32 == 0",
+                (long long)in, (long long)out);
+  if ((st = check_x(X, in, ldx)) != AWQ_OK) return st;
+  if (!qweight || !qzeros || !scales || !aligned(qweight, 16) || !aligned(qzeros, 16) || !aligned(scales, 16))
+    return fail(AWQ_ERR_INVALID_ARG, "qweight, qzeros and scales must be non-NULL and 16-byte aligned");
+  if (!Y || !aligned(Y, 16)) return fail(AWQ_ERR_INVALID_ARG, "Y is NULL or not 16-byte aligned");
+  if (ldy < out || ldy % 8 != 0)
+    return fail(AWQ_ERR_INVALID_ARG, "ldy=%lld must be >= out and a multiple of 8", (long long)ldy);
+  if ((st = check_ws(ws, ws_bytes, kHeader)) != AWQ_OK) return st;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  DevStatus *dst = static_cast<DevStatus *>(ws);
+  AWQ_TRY_CUDA(cudaMemsetAsync(dst, 0, sizeof(DevStatus), cs), "workspace reset");
+  ProfScope p("w4a16_gemm", cs);
+  AWQ_TRY_CUDA(launch_w4a16_gemm(static_cast<const __half *>(X), T, in, ldx, qweight, qzeros,
+                                 static_cast<const __half *>(scales), out, cfg->group_size,
+                                 static_cast<__half *>(Y), ldy, dst, poll_cap(), num_sms_current(), cs),
+               "w4a16_gemm launch");
+  return AWQ_OK;
+}
+
 awq_status awq_fold_inv_scale(void *v, int64_t rows, int64_t cols, const float *s,
                               awq_stream_t stream) {
   g_err.clear();

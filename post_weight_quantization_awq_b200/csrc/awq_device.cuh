@@ -212,6 +212,34 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t parity
   return false;
 }
 
+// try_wait with a suspend-time hint: the thread sleeps until the phase
+// completes or about `ns` nanoseconds pass, instead of spinning (spinning
+// warps take issue slots from the warps that do the work).
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for waits expected to be long (a role idle for most of a
+// tile): max_polls is scaled down by 64, each poll sleeping up to ~1 us, so
+// the bound in time stays that of mbar_wait_bounded.
+__device__ __forceinline__ bool mbar_wait_long(uint64_t *bar, uint32_t parity, uint32_t max_polls,
+                                               volatile int *abort) {
+  const uint32_t polls = (max_polls >> 6) + 1;
+  for (uint32_t i = 0; i < polls; ++i) {
+    if (mbar_try_wait_sleep(bar, parity, 1000u)) return true;
+    if (abort && *abort) return false;
+  }
+  return false;
+}
+
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }

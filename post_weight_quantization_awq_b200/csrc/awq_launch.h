@@ -69,6 +69,9 @@ constexpr int kGemmBM = 128, kGemmBN = 256, kGemmBK = 64;
 // `ld` elements), box [box_rows, box_cols], 128-byte swizzle, zero fill.
 cudaError_t make_tmap_f16_box(CUtensorMap *m, const void *base, int64_t rows, int64_t cols,
                               int64_t ld, uint32_t box_cols, uint32_t box_rows);
+// The same for int32 elements (row stride a multiple of 4), no swizzle.
+cudaError_t make_tmap_i32_box(CUtensorMap *m, const void *base, int64_t rows, int64_t cols,
+                              int64_t ld, uint32_t box_cols, uint32_t box_rows);
 
 // K5: mse[i] from `per_alpha` contiguous partials per candidate, best index, s_best.
 cudaError_t launch_mse_argmin(const double *partials, int n_alpha, size_t per_alpha, int64_t T,
@@ -101,6 +104,13 @@ cudaError_t launch_quant_pack(const __half *W, int64_t out, int64_t in, const fl
                               const uint8_t *clip_idx, int group, int w_bit, int zero_point,
                               int n_clip, float clip_min, int32_t *qweight, int32_t *qzeros,
                               __half *scales, cudaStream_t stream);
+
+// W4A16 GEMM on the packed output: Y = RN16(X Wd^T), Wd = RN16((q - z) scale);
+// in % 64 == 0, out % 32 == 0, group in {32, 64, 128}.
+cudaError_t launch_w4a16_gemm(const __half *X, int64_t T, int64_t in, int64_t ldx,
+                              const int32_t *qweight, const int32_t *qzeros, const __half *scales,
+                              int64_t out, int group, __half *Y, int64_t ldy, DevStatus *st,
+                              uint32_t max_polls, int num_sms, cudaStream_t stream);
 
 // K8: v[j][:] = RN16(RN32(v[j][:]) / s_j).
 cudaError_t launch_fold(__half *v, int64_t rows, int64_t cols, const float *s, cudaStream_t stream);

@@ -344,6 +344,22 @@ static cudaError_t launch_gemm_epi(const CUtensorMap &tmA, const CUtensorMap &tm
   return cudaGetLastError();
 }
 
+// 2-D int32 tensor map over a row-major [rows, cols] matrix (row stride `ld`
+// elements, a multiple of 4), box [box_rows, box_cols], no swizzle, zero fill.
+cudaError_t make_tmap_i32_box(CUtensorMap *m, const void *base, int64_t rows, int64_t cols,
+                              int64_t ld, uint32_t box_cols, uint32_t box_rows) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return cudaErrorNotSupported;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(ld * 4)};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_INT32, 2, const_cast<void *>(base), dims, strides, box,
+                  estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 cudaError_t launch_search_gemm(const __half *X, int64_t ldx, const __half *dW,
                                const SearchGemmShape &sh, double *partials, const __half *Y,
                                int64_t ldy, DevStatus *st, uint32_t max_polls, int num_sms,

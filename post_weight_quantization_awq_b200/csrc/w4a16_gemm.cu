@@ -1,0 +1,422 @@
+// W4A16 GEMM on the packed output of the search: the step after the path,
+// in which a layer's fp16 activations meet its 4-bit weights ("05 — AWQ:
+// Activation-Aware Weight Scaling" §5: qweight [in, out/8] int32 with output o
+// in nibble o % 8, qzeros [in/g, out/8], scales fp16 [in/g, out]; "AWQ and
+// Activation-Aware Scaling" / the papermap summary: the weights are
+// dequantised on the fly inside the GEMM).
+//
+//   Y[t][o] = RN16( sum_j X[t][j] * Wd[o][j] ),  Wd[o][j] = RN16((q - z) * scale)
+//
+// with q = the code of (o, j), z the zero of (o, j/g), scale = scales[j/g][o]:
+// the fp16 weights a consumer multiplies.  fp32 accumulation on the tensor
+// cores.
+//
+// sm_100a design, one CTA per SM (448 threads), persistent over 128 x 256
+// output tiles:
+//   warp 0      TMA loads of the 128 x 64 X tile (K-major, 128-byte swizzle)
+//               and of the 64 x 32 block of packed words behind the B tile;
+//   warps 6..13 dequantise the 64 x 256 weight tile: each thread turns int32
+//               words (8 outputs of one input channel each) into 16-byte
+//               chunks of an MN-major 128-byte-swizzled B tile — the packed
+//               layout is input-major, which is exactly MN-major for B, so no
+//               transpose is needed.  Within a chunk the outputs sit in the
+//               order 0,4,1,5,2,6,3,7 (what two mask operations per pair give);
+//               the accumulator columns carry the same order and the epilogue
+//               puts them back when it packs Y.  The words come from shared
+//               memory (staged by TMA with the X tile), zero points and
+//               scales from L1/L2 one step ahead;
+//   warp 1      one thread issues tcgen05.mma kind::f16 (M = 128, N = 256,
+//               K = 16) into a double-buffered TMEM accumulator;
+//   warps 2..5  read the accumulator (tcgen05.ld), round to fp16 and store Y.
+// Four pipeline stages of (16 + 32 + 8) KiB.  Every mbarrier wait is bounded; on a
+// timeout the CTA records kDevTimeout, drains its copies and MMAs, frees TMEM
+// and exits.
+#include <cuda.h>
+#include <cuda_fp16.h>
+
+#include "awq_launch.h"
+
+namespace awq {
+
+namespace {
+constexpr int QBM = 128, QBN = 256, QBK = 64, QSTAGES = 4;
+constexpr uint32_t QA_BYTES = QBM * QBK * 2;   // 16 KiB
+constexpr uint32_t QB_BOX = QBK * 128;         // 64 input channels x 64 outputs (8 KiB)
+constexpr uint32_t QB_BYTES = 4 * QB_BOX;      // 32 KiB
+constexpr uint32_t QW_BYTES = QBK * (QBN / 8) * 4;  // packed words of a B tile (8 KiB)
+constexpr uint32_t QTMEM_COLS = 512;
+constexpr int QGROUP_M = 16;
+constexpr int QW_DEQ = 6;                      // first dequantising warp
+constexpr int QN_DEQ = 8;                      // dequantising warps (two per sub-partition)
+constexpr int Q_WORDS = QBK * (QBN / 8) / (QN_DEQ * 32);  // words per thread per K tile (8)
+constexpr int Q_THREADS = (QW_DEQ + QN_DEQ) * 32;         // 448: up to 128 registers
+constexpr uint32_t Q_DRAIN = 1u << 22;
+// kind::f16, fp16 A/B, fp32 D, A K-major, B MN-major, N = 256, M = 128
+constexpr uint32_t IDESC_Q = (1u << 4) | (1u << 16) | ((uint32_t)(QBN >> 3) << 17) |
+                             ((uint32_t)(QBM >> 4) << 24);
+
+struct __align__(8) QTail {
+  uint64_t ld[QSTAGES];     // TMA bytes of the X tile and the packed words
+  uint64_t full[QSTAGES];   // one arrival per dequantising warp
+  uint64_t empty[QSTAGES];  // MMA commit
+  uint64_t tfull[2], tempty[2], mma_done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+constexpr size_t kQSmemBytes = 1024 + QSTAGES * (QA_BYTES + QB_BYTES + QW_BYTES) + sizeof(QTail);
+
+// MN-major B with 128-byte swizzling: 64 outputs (128 B) per input-channel row,
+// 8-row core groups 1024 B apart (SBO), 64-output boxes QB_BOX apart (LBO).
+__device__ __forceinline__ uint64_t desc_b_mn(uint32_t addr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((QB_BOX >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)(1024u >> 4) << 32;
+  d |= (uint64_t)1u << 46;
+  d |= (uint64_t)2u << 61;
+  return d;
+}
+
+__device__ __forceinline__ void q_tile_coords(int tile, int num_m, int num_n, int &m_blk, int &n_blk) {
+  const int per_group = QGROUP_M * num_n;
+  const int g = tile / per_group;
+  const int first_m = g * QGROUP_M;
+  const int gm = min(QGROUP_M, num_m - first_m);
+  const int local = tile - g * per_group;
+  m_blk = first_m + local % gm;
+  n_blk = local / gm;
+}
+
+// fp16 pairs {1024 + nibble p, 1024 + nibble p + 4}, p = 0..3, of a word
+__device__ __forceinline__ void nib_pairs(uint32_t w, __half2 (&h)[4]) {
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    const uint32_t bits = ((w >> (4 * p)) & 0x000F000Fu) | 0x64006400u;
+    h[p] = *reinterpret_cast<const __half2 *>(&bits);
+  }
+}
+
+// scales of outputs (p, p + 4), p = 0..3, from 8 consecutive fp16 scales
+__device__ __forceinline__ void scale_pairs(uint4 sc, __half2 (&h)[4]) {
+  const uint32_t lo[2] = {sc.x, sc.y}, hi[2] = {sc.z, sc.w};
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    // half p of the first four, half p of the last four
+    const uint32_t a = lo[p >> 1], b = hi[p >> 1];
+    const uint32_t bits = __byte_perm(a, b, (p & 1) ? 0x7632u : 0x5410u);
+    h[p] = *reinterpret_cast<const __half2 *>(&bits);
+  }
+}
+
+// 8 weights RN16((q - z) * scale) of one word in the order 0,4,1,5,2,6,3,7;
+// (1024 + q) - (1024 + z) is exact
+__device__ __forceinline__ uint4 dequant_word(uint32_t w, const __half2 (&zp)[4], const __half2 (&sp)[4]) {
+  __half2 qp[4];
+  nib_pairs(w, qp);
+  uint32_t o[4];
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    const __half2 r = __hmul2(__hsub2(qp[p], zp[p]), sp[p]);
+    o[p] = *reinterpret_cast<const uint32_t *>(&r);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+__device__ __forceinline__ void q_abort(QTail *t, DevStatus *st, uint32_t where) {
+  dev_fail(st, kDevTimeout, where);
+  *reinterpret_cast<volatile int *>(&t->abort_flag) = 1;
+}
+}  // namespace
+
+__global__ void __launch_bounds__(Q_THREADS, 1) w4a16_gemm_kernel(
+    const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+    const int32_t *__restrict__ qzeros, const __half *__restrict__ scales, int64_t T, int64_t out,
+    int group, int num_m, int num_n, int num_kb, __half *__restrict__ Y, int64_t ldy,
+    DevStatus *st, uint32_t max_polls) {
+  extern __shared__ uint8_t q_smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(q_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t *sA = smem;
+  uint8_t *sB = smem + QSTAGES * QA_BYTES;
+  uint8_t *sW = sB + QSTAGES * QB_BYTES;
+  QTail *tail = reinterpret_cast<QTail *>(sW + QSTAGES * QW_BYTES);
+  volatile int *abort_flag = &tail->abort_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int num_tiles = num_m * num_n;
+  const int64_t words = out / 8;  // int32 words per qweight / qzeros row
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < QSTAGES; ++s) {
+      mbar_init(&tail->ld[s], 1);
+      mbar_init(&tail->full[s], QN_DEQ);
+      mbar_init(&tail->empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tail->tfull[a], 1);
+      mbar_init(&tail->tempty[a], 4);
+    }
+    mbar_init(&tail->mma_done, 1);
+    tail->abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmX);
+    tma_prefetch_desc(&tmW);
+  }
+  if (warp == 1) {
+    tmem_alloc(&tail->tmem_base, QTMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = tail->tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ X by TMA
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, issued = 0, issued_parity = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+        int m_blk, n_blk;
+        q_tile_coords(tile, num_m, num_n, m_blk, n_blk);
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait_long(&tail->empty[stage], phase ^ 1u, max_polls, abort_flag)) {
+            q_abort(tail, st, 0xD00u + stage);
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&tail->ld[stage], QA_BYTES + QW_BYTES);
+          tma_load_2d(sA + stage * QA_BYTES, &tmX, &tail->ld[stage], kb * QBK, m_blk * QBM);
+          tma_load_2d(sW + stage * QW_BYTES, &tmW, &tail->ld[stage], n_blk * (QBN / 8), kb * QBK);
+          issued |= 1u << stage;
+          issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == QSTAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok || *abort_flag)
+        for (int s = 0; s < QSTAGES; ++s)
+          if (issued & (1u << s))
+            (void)mbar_wait_bounded(&tail->ld[s], (issued_parity >> s) & 1u, Q_DRAIN, nullptr);
+    }
+  } else if (warp >= QW_DEQ) {
+    // ------------------------------------------------------------ dequantise W
+    const int dt = threadIdx.x - QW_DEQ * 32;  // 0..255
+    const int col = dt & 31;                   // word column: outputs 8 col .. 8 col + 7
+    const int row0 = dt >> 5;                  // input-channel rows row0 + 8 i (so k & 7 = row0)
+    const uint32_t chunk_off = (uint32_t)(col >> 3) * QB_BOX + (uint32_t)row0 * 128u +
+                               ((uint32_t)((col & 7) ^ row0) << 4);
+    int stage = 0;
+    uint32_t phase = 0;
+    // the (tile, K step) sequence of this CTA, one step ahead for the word loads
+    int tile = blockIdx.x, kb = 0;
+    auto word_col = [&](int tl) {  // this thread's qweight column in tile tl
+      int m_blk, n_blk;
+      q_tile_coords(tl, num_m, num_n, m_blk, n_blk);
+      return (int64_t)n_blk * (QBN / 8) + col;
+    };
+    // zero words and scales of one K step: rows 0..31 of the step use group
+    // h = 0, rows 32..63 group h = 1 (the same group unless g = 32); loaded one
+    // step ahead (the packed words themselves arrive by TMA with the X tile)
+    uint32_t znext[2];
+    uint4 snext[2];
+    auto load_zs = [&](int64_t wc, int k_blk) {
+      const bool ok_c = wc < words;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int64_t gi = ((int64_t)k_blk * QBK + 32 * h) / group;
+        znext[h] = ok_c ? (uint32_t)__ldg(qzeros + gi * words + wc) : 0u;
+        snext[h] = ok_c ? __ldg(reinterpret_cast<const uint4 *>(scales + gi * out + 8 * wc))
+                        : make_uint4(0u, 0u, 0u, 0u);
+      }
+    };
+    int64_t wcol = tile < num_tiles ? word_col(tile) : 0;
+    if (tile < num_tiles) load_zs(wcol, 0);
+    bool ok = true;
+    while (ok && tile < num_tiles) {
+      uint32_t zw[2];
+      uint4 sc[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        zw[h] = znext[h];
+        sc[h] = snext[h];
+      }
+      int ntile = tile, nkb = kb + 1;
+      int64_t nwcol = wcol;
+      if (nkb == num_kb) {
+        nkb = 0;
+        ntile += gridDim.x;
+        nwcol = ntile < num_tiles ? word_col(ntile) : 0;
+      }
+      if (ntile < num_tiles) load_zs(nwcol, nkb);
+      __half2 zp[2][4], sp[2][4];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        nib_pairs(zw[h], zp[h]);
+        scale_pairs(sc[h], sp[h]);
+      }
+      // the stage's X tile and packed words have landed (which also means the
+      // MMAs that last read this stage are done: the loads waited for them)
+      int got = 1;
+      if (lane == 0) got = mbar_wait_long(&tail->ld[stage], phase, max_polls, abort_flag);
+      got = __shfl_sync(0xffffffffu, got, 0);
+      if (!got) {
+        if (lane == 0) q_abort(tail, st, 0xD10u + stage);
+        ok = false;
+        break;
+      }
+      // words past `out` were filled with zeros by TMA; their zeros and scales
+      // are zero too, so they give 0
+      const uint32_t *wsrc = reinterpret_cast<const uint32_t *>(sW + stage * QW_BYTES) + row0 * 32 + col;
+      uint8_t *bst = sB + stage * QB_BYTES + chunk_off;
+      // all eight words first: the B stores below may not be reordered above
+      // loads the compiler cannot prove disjoint, so loads come first explicitly
+      uint32_t wv[Q_WORDS];
+#pragma unroll
+      for (int i = 0; i < Q_WORDS; ++i) wv[i] = wsrc[i * 8 * 32];
+#pragma unroll
+      for (int i = 0; i < Q_WORDS; ++i) {
+        // row row0 + 8 i lies in 0..31 for i < 4 and in 32..63 for i >= 4
+        const uint4 v = dequant_word(wv[i], zp[i < 4 ? 0 : 1], sp[i < 4 ? 0 : 1]);
+        *reinterpret_cast<uint4 *>(bst + i * 8 * 128) = v;  // row row0 + 8 i, same swizzle
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tail->full[stage]);
+      if (++stage == QSTAGES) {
+        stage = 0;
+        phase ^= 1u;
+      }
+      tile = ntile;
+      kb = nkb;
+      wcol = nwcol;
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true, issued_any = false;
+      int it = 0;
+      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++it) {
+        const int acc = it & 1;
+        const uint32_t acc_phase = (it >> 1) & 1;
+        if (!mbar_wait_long(&tail->tempty[acc], acc_phase ^ 1u, max_polls, abort_flag)) {
+          q_abort(tail, st, 0xD20u + acc);
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * QBN;
+        for (int kb = 0; kb < num_kb; ++kb) {
+          if (!mbar_wait_long(&tail->full[stage], phase, max_polls, abort_flag) ||
+              !mbar_wait_bounded(&tail->ld[stage], phase, max_polls, abort_flag)) {  // X tile
+            q_abort(tail, st, 0xD30u + stage);
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_u32(sA + stage * QA_BYTES);
+          const uint32_t b_addr = smem_u32(sB + stage * QB_BYTES);
+#pragma unroll
+          for (int k = 0; k < QBK / 16; ++k)
+            tc_mma_f16(d_tmem, smem_desc_k_sw128(a_addr + k * 32), desc_b_mn(b_addr + k * 2048),
+                       IDESC_Q, (kb | k) != 0 ? 1u : 0u);
+          issued_any = true;
+          tc_commit(&tail->empty[stage]);
+          if (++stage == QSTAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(&tail->tfull[acc]);
+      }
+      if (issued_any) {
+        tc_commit(&tail->mma_done);
+        (void)mbar_wait_bounded(&tail->mma_done, 0, Q_DRAIN, nullptr);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2..5)
+    const int q = warp & 3;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
+      const int acc = it & 1;
+      const uint32_t acc_phase = (it >> 1) & 1;
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait_long(&tail->tfull[acc], acc_phase, max_polls, abort_flag);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) {
+        if (lane == 0) q_abort(tail, st, 0xD40u + acc);
+        break;
+      }
+      tc_fence_after();
+      int m_blk, n_blk;
+      q_tile_coords(tile, num_m, num_n, m_blk, n_blk);
+      const int64_t t_row = (int64_t)m_blk * QBM + q * 32 + lane;
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * QBN);
+#pragma unroll 1
+      for (int c = 0; c < QBN; c += 32) {
+        float v[32];
+        tmem_ld_32x32b_x32(taddr + (uint32_t)c, v);
+        tmem_ld_wait();
+        const int64_t o0 = (int64_t)n_blk * QBN + c;
+        if (t_row < T) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            if (o0 + 8 * u >= out) break;  // out % 8 == 0
+            // accumulator column 8u + 2p holds output 8u + p, column 8u + 2p + 1 output 8u + p + 4
+            uint32_t hw[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const int e0 = 2 * h, e1 = 2 * h + 1;  // outputs of this half2
+              const int c0 = e0 < 4 ? 2 * e0 : 2 * (e0 - 4) + 1, c1 = e1 < 4 ? 2 * e1 : 2 * (e1 - 4) + 1;
+              const __half2 hv = __floats2half2_rn(v[8 * u + c0], v[8 * u + c1]);
+              hw[h] = *reinterpret_cast<const uint32_t *>(&hv);
+            }
+            *reinterpret_cast<uint4 *>(Y + t_row * ldy + o0 + 8 * u) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tail->tempty[acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, QTMEM_COLS);
+  }
+}
+
+cudaError_t launch_w4a16_gemm(const __half *X, int64_t T, int64_t in, int64_t ldx,
+                              const int32_t *qweight, const int32_t *qzeros, const __half *scales,
+                              int64_t out, int group, __half *Y, int64_t ldy, DevStatus *st,
+                              uint32_t max_polls, int num_sms, cudaStream_t stream) {
+  if (in % QBK != 0 || out % 32 != 0 || group % 32 != 0) return cudaErrorInvalidValue;
+  CUtensorMap tmX, tmW;
+  cudaError_t e = make_tmap_f16_box(&tmX, X, T, in, ldx, QBK, QBM);
+  if (e != cudaSuccess) return e;
+  e = make_tmap_i32_box(&tmW, qweight, in, out / 8, out / 8, QBN / 8, QBK);  // words past out/8 read 0
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(w4a16_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)kQSmemBytes);
+  if (e != cudaSuccess) return e;
+  const int num_m = (int)((T + QBM - 1) / QBM);
+  const int num_n = (int)((out + QBN - 1) / QBN);
+  const int tiles = num_m * num_n;
+  const int grid = tiles < num_sms ? tiles : num_sms;
+  w4a16_gemm_kernel<<<grid, Q_THREADS, kQSmemBytes, stream>>>(
+      tmX, tmW, qzeros, scales, T, out, group, num_m, num_n, (int)(in / QBK), Y, ldy, st,
+      max_polls);
+  return cudaGetLastError();
+}
+
+}  // namespace awq

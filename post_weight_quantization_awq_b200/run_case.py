@@ -4,7 +4,8 @@
     python -m post_weight_quantization_awq_b200.run_case --op search --tokens 16384 \
         --in 4096 --out 4096 [--alphas 20] [--clips 20] [--bits 4] [--repeat 3] [--form gram|cached_y]
 
---op is one of: stats, search, clip, pack, layer (all four calls).  Inputs
+--op is one of: stats, search, clip, pack, layer (all four calls), w4a16 (the
+GEMM on the packed output, Y = X Wd^T with Wd dequantised on the fly).  Inputs
 follow the heavy-tailed recipe of the synthetic module (1% outlier channels
 x U[20, 50], W ~ N(0, 0.02)).  Prints the CUDA-event time of the last repeat.
 """
@@ -27,7 +28,7 @@ def main(argv=None) -> int:
     from synthetic import OutlierSpec, gaussian_weight, heavy_tailed_activations
 
     ap = argparse.ArgumentParser()
-    ap.add_argument("--op", choices=("stats", "search", "clip", "pack", "layer"), required=True)
+    ap.add_argument("--op", choices=("stats", "search", "clip", "pack", "layer", "w4a16"), required=True)
     ap.add_argument("--tokens", type=int, default=16384)
     ap.add_argument("--in", dest="inn", type=int, default=4096)
     ap.add_argument("--out", type=int, default=4096)
@@ -56,6 +57,10 @@ def main(argv=None) -> int:
     qz = torch.empty((a.inn // g, a.out // 8), dtype=torch.int32, device="cuda")
     sc = torch.empty((a.inn // g, a.out), dtype=torch.float16, device="cuda")
     awq.awq_act_stats(X, abar)
+    if a.op == "w4a16":
+        awq.awq_quant_pack(W, s_best, None, cfg, qw, qz, sc)
+        Y = torch.empty((a.tokens, a.out), dtype=torch.float16, device="cuda")
+        ws16 = torch.empty(256, dtype=torch.uint8, device="cuda")
 
     def once():
         if a.op == "stats":
@@ -66,6 +71,8 @@ def main(argv=None) -> int:
             awq.awq_search_clip(X, W, s_best, cfg, ws, clip_idx)
         elif a.op == "pack":
             awq.awq_quant_pack(W, s_best, clip_idx if a.clips else None, cfg, qw, qz, sc)
+        elif a.op == "w4a16":
+            awq.awq_w4a16_gemm(X, qw, qz, sc, cfg, Y, ws16)
         else:
             awq.quantize_layer(X, W, cfg, ws=ws)
 
@@ -76,7 +83,11 @@ def main(argv=None) -> int:
         e1.record()
     torch.cuda.synchronize()
     awq.awq_device_status(ws)
-    print(f"{a.op}: T={a.tokens} in={a.inn} out={a.out} last call {e0.elapsed_time(e1):.3f} ms")
+    ms = e0.elapsed_time(e1)
+    extra = ""
+    if a.op == "w4a16":
+        extra = f", {2.0 * a.tokens * a.inn * a.out / (ms * 1e-3) / 1e12:.1f} TFLOP/s"
+    print(f"{a.op}: T={a.tokens} in={a.inn} out={a.out} last call {ms:.3f} ms{extra}")
     return 0
 
 

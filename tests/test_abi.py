@@ -109,3 +109,12 @@ def test_group_sizes_and_clip_limits():
     st = abi.LIB.awq_search_scale(16, 256, 192, 192, 16, 64, 16, ctypes.byref(cfg), 256, 1 << 30,
                                   16, 16, 16, None)
     assert abi.STATUS[st] == "AWQ_ERR_UNSUPPORTED" and "Gram" in abi.last_error()
+
+
+def test_w4a16_shape_limits():
+    """The W4A16 GEMM states its limits before touching CUDA."""
+    cfg = awq.AwqConfig.make()
+    st = abi.LIB.awq_w4a16_gemm(16, 256, 512, 512, 16, 16, 16, 264, ctypes.byref(cfg), 16, 264, 256, 1024, None)
+    assert abi.STATUS[st] == "AWQ_ERR_UNSUPPORTED" and "out % 32" in abi.last_error()
+    st = abi.LIB.awq_w4a16_gemm(16, 256, 512, 512, 16, 16, 16, 256, ctypes.byref(cfg), 16, 200, 256, 1024, None)
+    assert abi.STATUS[st] == "AWQ_ERR_INVALID_ARG" and "ldy" in abi.last_error()

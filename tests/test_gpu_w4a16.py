@@ -1,0 +1,106 @@
+"""GPU parity of the W4A16 GEMM on the packed output (the step after the
+search; "05 — AWQ: Activation-Aware Weight Scaling" §5 layout, weights
+dequantised on the fly): Y = RN16(X Wd^T) with Wd = RN16((q - z) scale),
+against the oracle's fp64 product of the same fp16 weights.  Bound per output:
+half an fp16 ulp of the result plus 2^-11 sum_j |X_tj| |Wd_oj| for the fp32
+accumulation of up to 4096 products (two roundings per addition at most)."""
+
+import numpy as np
+import pytest
+import torch
+
+import post_weight_quantization_awq_b200 as awq
+from oracle import awq_oracle as O
+from synthetic import OutlierSpec, heavy_tailed_activations, random_layer, workload_inputs
+
+from gpu_helpers import need_cuda, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _cuda():
+    need_cuda()
+
+
+def _ulp16(v):
+    a = np.abs(np.asarray(v, dtype=np.float64))
+    return np.exp2(np.floor(np.log2(np.maximum(a, 2.0 ** -14))) - 10)
+
+
+def _gpu_w4a16(X, qw, qz, sc, cfg):
+    Xd = to_dev(X)
+    T, out = Xd.shape[0], sc.shape[1]
+    Y = torch.empty((T, out), dtype=torch.float16, device="cuda")
+    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    awq.awq_w4a16_gemm(Xd, torch.from_numpy(qw).cuda(), torch.from_numpy(qz).cuda(),
+                       torch.from_numpy(np.ascontiguousarray(sc)).cuda(), cfg, Y, ws)
+    awq.awq_device_status(ws)
+    torch.cuda.synchronize()
+    return Y.cpu().numpy()
+
+
+def _check(Yg, X, qw, qz, sc, group):
+    Xn = np.asarray(X, dtype=np.float64)
+    Yo = O.w4a16_matmul(X, qw, qz, sc, group)
+    Wd = np.abs(O.dequant_packed(qw, qz, sc, group).astype(np.float64))
+    acc = np.abs(Xn) @ Wd.T * 2.0 ** -11
+    tol = 0.5 * _ulp16(np.abs(Yo) + acc) + acc
+    err = np.abs(Yg.astype(np.float64) - Yo)
+    assert np.all(err <= tol), (err.max(), np.unravel_index(np.argmax(err - tol), err.shape))
+
+
+def test_w4a16_exact_integer_case():
+    """Step 1, zero 8, integer X: every sum is an integer below 2^11, so the
+    fp32 accumulation and the fp16 output are exact."""
+    W = np.zeros((288, 256), dtype=np.float16)
+    rng = np.random.default_rng(7)
+    W[:] = rng.integers(-8, 8, size=W.shape)
+    W[:, 0], W[:, 1], W[:, 128], W[:, 129] = -8.0, 7.0, -8.0, 7.0  # step 1, zero 8 in both groups
+    qw, qz, sc = O.quant_pack(W, None, None, 4, 128)
+    assert np.all(sc == np.float16(1.0))
+    X = rng.integers(-2, 3, size=(300, 256)).astype(np.float16)
+    Yg = _gpu_w4a16(torch.from_numpy(X), qw, qz, sc, awq.AwqConfig.make())
+    want = X.astype(np.int64) @ W.astype(np.int64).T
+    assert np.array_equal(Yg.astype(np.int64), want)
+
+
+@pytest.mark.parametrize("T,inn,out,w_bit,group,zp", [
+    (200, 384, 288, 4, 128, 1), (1, 512, 160, 3, 64, 1), (300, 256, 96, 4, 32, 1),
+    (2000, 1024, 768, 4, 128, 1), (129, 640, 544, 3, 128, 0)])
+def test_w4a16_parity(T, inn, out, w_bit, group, zp):
+    X, W = random_layer(T, inn, out, seed=T + inn + out + group)
+    Wn = W.numpy()
+    s = O.scale_grid(O.act_stats(X.numpy()), O.alpha_grid(20))[9]
+    qw, qz, sc = O.quant_pack(Wn, s, None, w_bit, group, zero_point=bool(zp))
+    # the layer's input after the fold: X / s, as fp16
+    Xs = (X.numpy().astype(np.float32) / s[None, :]).astype(np.float16)
+    cfg = awq.AwqConfig.make(w_bit=w_bit, group_size=group, zero_point=zp)
+    Yg = _gpu_w4a16(torch.from_numpy(Xs), qw, qz, sc, cfg)
+    _check(Yg, Xs, qw, qz, sc, group)
+
+
+def test_w4a16_on_the_searched_q_proj_layer():
+    """The full q_proj workload: search, clip and pack on the GPU, then the
+    W4A16 GEMM of X / s* (T = 65536, in = out = 4096) against the oracle on
+    256 sampled tokens; and its output error against the fp16 X W^T stays
+    the quantisation error the search measured."""
+    d = workload_inputs(1)
+    _, X, W = d["groups"][0]
+    cfg = awq.AwqConfig.make(w_bit=4, n_alpha=20, n_clip=20)
+    Xd, Wd = to_dev(X), to_dev(W)
+    res = awq.quantize_layer(Xd, Wd, cfg)
+    Xs = (Xd.float() / res.s_best[None, :]).half()  # the fold of 1/s* into the input
+    Y = torch.empty((Xd.shape[0], Wd.shape[0]), dtype=torch.float16, device="cuda")
+    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    awq.awq_w4a16_gemm(Xs, res.qweight, res.qzeros, res.scales, cfg, Y, ws)
+    awq.awq_device_status(ws)
+    torch.cuda.synchronize()
+    rows = np.sort(np.random.default_rng(1).choice(Xd.shape[0], 256, replace=False))
+    qw, qz, sc = res.qweight.cpu().numpy(), res.qzeros.cpu().numpy(), res.scales.cpu().numpy()
+    _check(Y[torch.from_numpy(rows).cuda()].cpu().numpy(), Xs[torch.from_numpy(rows).cuda()].cpu().numpy(),
+           qw, qz, sc, 128)
+    # the packed layer reproduces X W^T to the searched error level
+    Yref = Xd[torch.from_numpy(rows).cuda()].float() @ Wd.float().T
+    mse = float(((Y[torch.from_numpy(rows).cuda()].float() - Yref) ** 2).mean())
+    assert mse < 1.5 * float(res.mse.min()) + 1e-6, (mse, float(res.mse.min()))
