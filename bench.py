@@ -40,7 +40,7 @@ KERNELS_PER_STEP = {  # kernels this library launches per step (memsets excluded
 # DRAM bytes (read + write) of one search_gemm_kernel launch on this workload,
 # from a one-pass ncu capture (profiles/search_gemm_q_proj_4096.md); to be
 # set to None whenever that kernel changes until it is captured again.
-NCU_TRAFFIC_BYTES = 11_290_000_000 + 9_690_000
+NCU_TRAFFIC_BYTES = None  # re-captured after the wait change
 
 
 def load_peaks():
@@ -369,6 +369,30 @@ def run_awq(args):
         del ws_f
         return ms_f, kf
 
+    # ---- the step after the search: the W4A16 GEMM on this layer's packed
+    # output, fed the folded input X / s* (its own timing and flops)
+    w4a16 = None
+    if not args.no_w4a16:
+        r = awq.quantize_layer(Xd, Wd, cfg, ws=ws)
+        Xs = (Xd.float() / r.s_best[None, :]).half()
+        Yq = torch.empty((T, out), dtype=torch.float16, device=dev)
+        ws_q = torch.empty(256, dtype=torch.uint8, device=dev)
+
+        def step_q():
+            awq.awq_w4a16_gemm(Xs, r.qweight, r.qzeros, r.scales, cfg, Yq, ws_q)
+
+        for _ in range(args.warmup):
+            step_q()
+        awq.awq_device_status(ws_q)
+        ms_q = timed_steps(step_q, args.steps, dist, timer, local)
+        awq.awq_device_status(ws_q)
+        flops_q = 2.0 * T * inn * out
+        w4a16 = {"ms": round(ms_q, 4), "tflops": round(flops_q / (ms_q * 1e-3) / 1e12, 1),
+                 "flops": flops_q,
+                 "note": "Y = X Wd^T with Wd dequantised on the fly from qweight/qzeros/scales; "
+                         "T x in x out of the layer above"}
+        del Xs, Yq
+
     # ---- the literal fp16-output form on the same layer: Y = RN16(X W^T) once,
     # then every candidate's output scored against it in the GEMM's epilogue
     cached = None
@@ -449,6 +473,7 @@ def run_awq(args):
         "cpu_baseline": cpu,
         "gram_form": gram,
         "cached_output_form": cached,
+        "w4a16_gemm": w4a16,
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -519,6 +544,8 @@ def main(argv=None):
                     help="skip the extra measurement of the Gram-form search")
     ap.add_argument("--no-cached-form", action="store_true",
                     help="skip the extra measurement of the cached fp16-output form")
+    ap.add_argument("--no-w4a16", action="store_true",
+                    help="skip the measurement of the W4A16 GEMM on the packed output")
     ap.add_argument("--workload", choices=("q_proj", "decoder"), default="q_proj",
                     help="q_proj: the headline workload; decoder: the 32-layer decoder "
                          "(--steps = layers timed)")

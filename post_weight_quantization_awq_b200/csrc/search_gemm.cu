@@ -137,7 +137,7 @@ __global__ void __launch_bounds__(192, 1)
         int m_blk, n_blk;
         tile_coords(tile, num_m, num_n, GROUP_M, m_blk, n_blk);
         for (int kb = 0; kb < num_kb; ++kb) {
-          if (!mbar_wait_bounded(&tail->empty[stage], phase ^ 1u, max_polls, abort_flag)) {
+          if (!mbar_wait_long(&tail->empty[stage], phase ^ 1u, max_polls, abort_flag)) {
             raise_abort(tail, st, 0x100u + stage);
             ok = false;
             break;
@@ -214,7 +214,7 @@ __global__ void __launch_bounds__(192, 1)
       const int acc = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
       int ok = 1;
-      if (lane == 0) ok = mbar_wait_bounded(&tail->tfull[acc], acc_phase, max_polls, abort_flag);
+      if (lane == 0) ok = mbar_wait_long(&tail->tfull[acc], acc_phase, max_polls, abort_flag);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) {
         if (lane == 0) raise_abort(tail, st, 0x400u + acc);
