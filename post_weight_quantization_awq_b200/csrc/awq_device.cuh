@@ -80,22 +80,20 @@ __device__ __forceinline__ GroupQ group_params(float mx, float mn, float r32, fl
     mx = __fmul_rn(r32, mx);
     mn = __fmul_rn(r32, mn);
   }
+  // one division for both kinds: range and divisor are chosen, not branched
   GroupQ g;
   g.qmax = qmax;
-  if (sym) {
-    const float d = fmaxf(fmaxf(fabsf(mx), fabsf(mn)), guard);
-    g.delta = __fdiv_rn(d, 0.5f * (qmax - 1.0f));  // 2^(b-1) - 1, exact
-    g.rcp = rcp_approx(g.delta);
-    g.half_lo = __fmul_rn(g.delta, 0.4999847412109375f /* 0.5 - 2^-16 */);
-    g.zero = 0.5f * (qmax + 1.0f);  // 2^(b-1), exact
-    return g;
-  }
-  const float d = fmaxf(__fsub_rn(mx, mn), guard);
-  g.delta = __fdiv_rn(d, qmax);
+  const float range = sym ? fmaxf(fabsf(mx), fabsf(mn)) : __fsub_rn(mx, mn);
+  const float divisor = sym ? 0.5f * (qmax - 1.0f) : qmax;  // 2^(b-1) - 1 or 2^b - 1, exact
+  g.delta = __fdiv_rn(fmaxf(range, guard), divisor);
   g.rcp = rcp_approx(g.delta);
   g.half_lo = __fmul_rn(g.delta, 0.4999847412109375f /* 0.5 - 2^-16 */);
-  const float z = round_quotient(-mn, g.delta, g.rcp, g.half_lo);
-  g.zero = fminf(fmaxf(z, 0.0f), qmax);
+  if (sym) {
+    g.zero = 0.5f * (qmax + 1.0f);  // 2^(b-1), exact
+  } else {
+    const float z = round_quotient(-mn, g.delta, g.rcp, g.half_lo);
+    g.zero = fminf(fmaxf(z, 0.0f), qmax);
+  }
   return g;
 }
 

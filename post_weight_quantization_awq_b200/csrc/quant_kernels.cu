@@ -255,10 +255,11 @@ cudaError_t launch_wmax(const __half *W, int64_t n, int64_t in, const float *r, 
 // ---------------------------------------------------------------------------
 constexpr int kCandRows = 64;
 
+template <int group>  // 32, 64 or 128: the range shuffles unroll
 __global__ void __launch_bounds__(256) cand_quant_kernel(
     const __half *__restrict__ W, int64_t out, int64_t in, int64_t out_pad,
     const float *__restrict__ s, const float *__restrict__ inv_s, const float *__restrict__ rch,
-    int group, float qmax, int sym, int weights_only, const DevStatus *__restrict__ st,
+    float qmax, int sym, int weights_only, const DevStatus *__restrict__ st,
     __half *__restrict__ dW) {
   // Everything runs on s 2^k: codes and zero points are those of s (power-of-
   // two invariance), delta comes out times 2^k, and the candidate error
@@ -268,7 +269,7 @@ __global__ void __launch_bounds__(256) cand_quant_kernel(
   const int k = weights_only ? 0 : kscale_from_wmax(__uint_as_float(__ldg(&st->wmax_bits)));
   const float two_k = ldexpf(1.0f, k);
   const float guard = __fmul_rn(1e-5f, two_k);  // exact
-  const int lanes = group / 8;  // lanes per group (a power of two <= 32)
+  constexpr int lanes = group / 8;  // lanes per group (a power of two <= 16)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t j0 = (int64_t)blockIdx.y * 256 + lane * 8;
   const bool j_ok = j0 < in;
@@ -319,6 +320,7 @@ __global__ void __launch_bounds__(256) cand_quant_kernel(
       mx = fmaxf(mx, fmaxf(wt[h].x, wt[h].y));
       mn = fminf(mn, fminf(wt[h].x, wt[h].y));
     }
+#pragma unroll
     for (int off = lanes >> 1; off > 0; off >>= 1) {
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
       mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
@@ -351,9 +353,10 @@ cudaError_t launch_cand_quant(const __half *W, int64_t out, int64_t in, int64_t 
                               const DevStatus *st, __half *dW, int num_sms, cudaStream_t stream) {
   (void)num_sms;
   dim3 grid((unsigned)(n_alpha * (out_pad / kCandRows)), (unsigned)((in + 255) / 256));
-  cand_quant_kernel<<<grid, 256, 0, stream>>>(W, out, in, out_pad, s, inv_s, r, group,
-                                              (float)((1 << w_bit) - 1), zero_point ? 0 : 1,
-                                              weights_only, st, dW);
+  if (group != 32 && group != 64 && group != 128) return cudaErrorInvalidValue;
+  auto kern = group == 32 ? cand_quant_kernel<32> : group == 64 ? cand_quant_kernel<64> : cand_quant_kernel<128>;
+  kern<<<grid, 256, 0, stream>>>(W, out, in, out_pad, s, inv_s, r, (float)((1 << w_bit) - 1),
+                                 zero_point ? 0 : 1, weights_only, st, dW);
   return cudaGetLastError();
 }
 
@@ -382,8 +385,9 @@ __device__ __forceinline__ float clip_ratio(int c, int n_clip, float clip_min) {
 // is contiguous.
 constexpr int kPackTile = 128;
 
+template <int group>  // 32, 64 or 128: divisions and the shuffle loop become constants
 __global__ void __launch_bounds__(256, 6) quant_pack_kernel(
-    const __half *__restrict__ W, int64_t out, int64_t in, int group, const float *__restrict__ s,
+    const __half *__restrict__ W, int64_t out, int64_t in, const float *__restrict__ s,
     const uint8_t *__restrict__ clip_idx, int n_clip, float clip_min, float qmax, int sym,
     int32_t *__restrict__ qweight, int32_t *__restrict__ qzeros, __half *__restrict__ scales) {
   constexpr int TC = kPackTile;
@@ -398,7 +402,7 @@ __global__ void __launch_bounds__(256, 6) quant_pack_kernel(
   const int64_t o0 = (int64_t)blockIdx.x * kPackRows;
   const int64_t groups = in / group;
   const int rows_here = (int)i64min(kPackRows, out - o0);
-  const int gl = group / 4;                                     // lanes per group
+  constexpr int gl = group / 4;                                 // lanes per group
   {
     uint4 v[4];
 #pragma unroll
@@ -429,24 +433,25 @@ __global__ void __launch_bounds__(256, 6) quant_pack_kernel(
     const uint2 wv = *reinterpret_cast<const uint2 *>(&wsm[r][lane * 4]);
     const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&wv.x));
     const float2 b = __half22float2(*reinterpret_cast<const __half2 *>(&wv.y));
-    const float2 wt[2] = {__fmul2_rn(make_float2(sv[0], sv[1]), a), __fmul2_rn(make_float2(sv[2], sv[3]), b)};
-    float mx = fmaxf(fmaxf(wt[0].x, wt[0].y), fmaxf(wt[1].x, wt[1].y));
-    float mn = fminf(fminf(wt[0].x, wt[0].y), fminf(wt[1].x, wt[1].y));
+    const float wt[4] = {__fmul_rn(sv[0], a.x), __fmul_rn(sv[1], a.y), __fmul_rn(sv[2], b.x),
+                         __fmul_rn(sv[3], b.y)};
+    float mx = fmaxf(fmaxf(wt[0], wt[1]), fmaxf(wt[2], wt[3]));
+    float mn = fminf(fminf(wt[0], wt[1]), fminf(wt[2], wt[3]));
+#pragma unroll
     for (int off = gl >> 1; off > 0; off >>= 1) {
       mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
       mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
     }
     if (!lane_ok) continue;  // past the last channel (its lanes form whole groups)
     const float r32 = clip_idx ? ratios[clip_idx[o * groups + kg]] : 1.0f;
-    GroupQ g = group_params(mx, mn, r32, qmax, sym != 0);
-    fast_path_check(g, mx, mn);  // mx, mn: the unclipped extremes, which bound every |wt|
-    float2 qz[2];
-    quant_qz_pairs<2>(wt, g, qz);
-    uchar4 c4;  // q = (q - z) + z, exact small integers
-    c4.x = (uint8_t)__fadd_rn(qz[0].x, g.zero);
-    c4.y = (uint8_t)__fadd_rn(qz[0].y, g.zero);
-    c4.z = (uint8_t)__fadd_rn(qz[1].x, g.zero);
-    c4.w = (uint8_t)__fadd_rn(qz[1].y, g.zero);
+    // four values per lane: the scalar quantiser (the batched fast path of the
+    // candidate kernels costs more than it saves at this width)
+    const GroupQ g = group_params(mx, mn, r32, qmax, sym != 0);
+    uchar4 c4;
+    c4.x = (uint8_t)quant_code(wt[0], g);
+    c4.y = (uint8_t)quant_code(wt[1], g);
+    c4.z = (uint8_t)quant_code(wt[2], g);
+    c4.w = (uint8_t)quant_code(wt[3], g);
     *reinterpret_cast<uchar4 *>(&codes[r][lane * 4]) = c4;
     if ((lane & (gl - 1)) == 0) {  // first lane of the group
       zeros[r][gi] = (uint8_t)g.zero;
@@ -481,9 +486,9 @@ cudaError_t launch_quant_pack(const __half *W, int64_t out, int64_t in, const fl
                               __half *scales, cudaStream_t stream) {
   if (group != 32 && group != 64 && group != 128) return cudaErrorInvalidValue;
   dim3 grid((unsigned)((out + kPackRows - 1) / kPackRows), (unsigned)((in + kPackTile - 1) / kPackTile));
-  quant_pack_kernel<<<grid, 256, 0, stream>>>(W, out, in, group, s, clip_idx, n_clip, clip_min,
-                                              (float)((1 << w_bit) - 1), zero_point ? 0 : 1,
-                                              qweight, qzeros, scales);
+  auto kern = group == 32 ? quant_pack_kernel<32> : group == 64 ? quant_pack_kernel<64> : quant_pack_kernel<128>;
+  kern<<<grid, 256, 0, stream>>>(W, out, in, s, clip_idx, n_clip, clip_min, (float)((1 << w_bit) - 1),
+                                 zero_point ? 0 : 1, qweight, qzeros, scales);
   return cudaGetLastError();
 }
 
