@@ -54,7 +54,7 @@ typedef void *awq_stream_t; /* a cudaStream_t */
 typedef enum {
   AWQ_OK = 0,
   AWQ_ERR_INVALID_ARG = 1, /* a size, stride, pointer or alignment is wrong   */
-  AWQ_ERR_UNSUPPORTED = 2, /* a valid setting this build does not implement   */
+  AWQ_ERR_UNSUPPORTED = 2, /* a valid setting the library does not implement  */
   AWQ_ERR_WORKSPACE = 3,   /* workspace missing, misaligned or too small      */
   AWQ_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed               */
   AWQ_ERR_TIMEOUT = 5,     /* a bounded device-side wait ran out              */
