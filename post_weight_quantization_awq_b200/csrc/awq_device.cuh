@@ -225,17 +225,25 @@ __device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t pari
   return ok != 0;
 }
 
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
 // Bounded wait for waits expected to be long (a role idle for most of a
-// tile): max_polls is scaled down by 64, each poll sleeping up to ~1 us, so
-// the bound in time stays that of mbar_wait_bounded.
+// tile): each poll sleeps until the phase completes or up to ~1 us, and the
+// bound is in time, max_polls x 64 ns (about 1 s for the default 2^24; one
+// poll when max_polls is 1), since how long a hinted poll sleeps varies.
 __device__ __forceinline__ bool mbar_wait_long(uint64_t *bar, uint32_t parity, uint32_t max_polls,
                                                volatile int *abort) {
-  const uint32_t polls = (max_polls >> 6) + 1;
-  for (uint32_t i = 0; i < polls; ++i) {
+  const uint64_t limit_ns = (uint64_t)max_polls * 64u;
+  const uint64_t t0 = global_ns();
+  for (;;) {
     if (mbar_try_wait_sleep(bar, parity, 1000u)) return true;
     if (abort && *abort) return false;
+    if (global_ns() - t0 > limit_ns) return false;
   }
-  return false;
 }
 
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {

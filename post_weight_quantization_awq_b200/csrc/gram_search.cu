@@ -114,7 +114,7 @@ __global__ void __launch_bounds__(192, 1)
       uint32_t phase = 0, issued = 0, issued_parity = 0;
       bool ok = true;
       for (int step = 0; step < nsteps; ++step) {
-        if (!mbar_wait_bounded(&tail->empty[stage], phase ^ 1u, max_polls, abort_flag)) {
+        if (!mbar_wait_long(&tail->empty[stage], phase ^ 1u, max_polls, abort_flag)) {
           dev_fail(st, kDevTimeout, 0xA00u + stage);
           *abort_flag = 1;
           ok = false;
@@ -175,7 +175,7 @@ __global__ void __launch_bounds__(192, 1)
   } else {
     const int q = warp & 3;
     int ok = 1;
-    if (lane == 0) ok = mbar_wait_bounded(&tail->done, 0, max_polls, abort_flag);
+    if (lane == 0) ok = mbar_wait_long(&tail->done, 0, max_polls, abort_flag);
     ok = __shfl_sync(0xffffffffu, ok, 0);
     if (!ok) {
       if (lane == 0) {
@@ -345,7 +345,7 @@ __global__ void __launch_bounds__(192, 1)
         const int acc = it & 1;
         const uint32_t acc_phase = (it >> 1) & 1;
         // C tile: d~[m rows][n columns], read by the epilogue
-        if (!mbar_wait_bounded(&tail->cempty[acc], acc_phase ^ 1u, max_polls, abort_flag)) {
+        if (!mbar_wait_long(&tail->cempty[acc], acc_phase ^ 1u, max_polls, abort_flag)) {
           dev_fail(st, kDevTimeout, 0xD10u + acc);
           *abort_flag = 1;
           break;
@@ -356,7 +356,7 @@ __global__ void __launch_bounds__(192, 1)
         c_issued |= 1u << acc;
         c_parity = (c_parity & ~(1u << acc)) | (acc_phase << acc);
         for (int kb = n_blk * (SN / SK); kb < num_kb; ++kb) {  // upper triangle of G~ only
-          if (!mbar_wait_bounded(&tail->empty[stage], phase ^ 1u, max_polls, abort_flag)) {
+          if (!mbar_wait_long(&tail->empty[stage], phase ^ 1u, max_polls, abort_flag)) {
             dev_fail(st, kDevTimeout, 0xD00u + stage);
             *abort_flag = 1;
             ok = false;
@@ -439,7 +439,7 @@ __global__ void __launch_bounds__(192, 1)
       const uint32_t acc_phase = (it >> 1) & 1;
       int ok = 1;
       if (lane == 0)
-        ok = mbar_wait_bounded(&tail->tfull[acc], acc_phase, max_polls, abort_flag) &&
+        ok = mbar_wait_long(&tail->tfull[acc], acc_phase, max_polls, abort_flag) &&
              mbar_wait_bounded(&tail->cfull[acc], acc_phase, max_polls, abort_flag);
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) {

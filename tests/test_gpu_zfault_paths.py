@@ -54,3 +54,48 @@ def test_bounded_waits_report_timeout_and_leave_the_context_usable(monkeypatch):
     check_mse(mse.cpu().numpy(), mse_o)
     awq.awq_search_clip(Xd, Wd, None, cfg, ws, idx)
     awq.awq_device_status(ws)
+
+
+def test_timeouts_in_the_gram_cached_and_w4a16_kernels(monkeypatch):
+    """The same for the Gram-form and cached-output searches and for the W4A16
+    GEMM.  The W4A16 roles that idle for long stretches wait with a suspend
+    hint, so one poll may already see the phase complete: there the test
+    accepts either status, and checks that nothing hangs and the next call is
+    exact."""
+    need_cuda()
+    X, W = random_layer(600, 512, 256, seed=22)
+    Xd, Wd = X.cuda(), W.cuda()
+    Xn, Wn = X.numpy(), W.numpy()
+    qw, qz, sc = (torch.from_numpy(a).cuda() for a in O.quant_pack(Wn, None, None, 4, 128))
+    Y = torch.empty((600, 256), dtype=torch.float16, device="cuda")
+    ws16 = torch.empty(256, dtype=torch.uint8, device="cuda")
+    cfgs = {form: awq.AwqConfig.make(search_form=form)
+            for form in (awq.abi.SEARCH_GRAM, awq.abi.SEARCH_CACHED_Y)}
+    wss = {form: awq.alloc_workspace(600, 512, 256, cfg) for form, cfg in cfgs.items()}
+    monkeypatch.setenv("AWQ_FAULT", "timeout")
+    for form, cfg in cfgs.items():
+        _search(Xd, Wd, cfg, wss[form])
+        with pytest.raises(awq.AwqError) as ei:
+            awq.awq_device_status(wss[form])
+        assert ei.value.status_name == "AWQ_ERR_TIMEOUT", form
+    awq.awq_w4a16_gemm(Xd, qw, qz, sc, cfgs[awq.abi.SEARCH_GRAM], Y, ws16)
+    try:
+        awq.awq_device_status(ws16)
+    except awq.AwqError as e:
+        assert e.status_name == "AWQ_ERR_TIMEOUT"
+    monkeypatch.delenv("AWQ_FAULT")
+    mse_o, _, _, _ = O.search_scale(Xn, Wn, O.act_stats(Xn), 4, 128, 20, form="direct")
+    mse_y, _, _, _ = O.search_scale(Xn, Wn, O.act_stats(Xn), 4, 128, 20, form="fp16_output")
+    for form, cfg in cfgs.items():
+        mse, _ = _search(Xd, Wd, cfg, wss[form])
+        awq.awq_device_status(wss[form])
+        check_mse(mse.cpu().numpy(), mse_o if form == awq.abi.SEARCH_GRAM else mse_y)
+    awq.awq_w4a16_gemm(Xd, qw, qz, sc, cfgs[awq.abi.SEARCH_GRAM], Y, ws16)
+    awq.awq_device_status(ws16)
+    Y1 = Y.clone()
+    awq.awq_w4a16_gemm(Xd, qw, qz, sc, cfgs[awq.abi.SEARCH_GRAM], Y, ws16)
+    awq.awq_device_status(ws16)
+    torch.cuda.synchronize()
+    assert torch.isfinite(Y.float()).all() and torch.equal(Y, Y1)
+    Yo = O.w4a16_matmul(Xn, qw.cpu().numpy(), qz.cpu().numpy(), sc.cpu().numpy(), 128)
+    assert np.allclose(Y.cpu().numpy().astype(np.float64), Yo, rtol=2e-3, atol=1e-2)
