@@ -40,7 +40,7 @@ KERNELS_PER_STEP = {  # kernels this library launches per step (memsets excluded
 # DRAM bytes (read + write) of one search_gemm_kernel launch on this workload,
 # from a one-pass ncu capture (profiles/search_gemm_q_proj_4096.md); to be
 # set to None whenever that kernel changes until it is captured again.
-NCU_TRAFFIC_BYTES = 11_290_000_000 + 9_600_000
+NCU_TRAFFIC_BYTES = 11_300_000_000 + 10_080_000
 
 
 def load_peaks():
