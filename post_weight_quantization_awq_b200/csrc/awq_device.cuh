@@ -101,24 +101,6 @@ __device__ __forceinline__ float round_quotient(float wt, const GroupQ &g) {
   return round_quotient(wt, g.delta, g.rcp, g.half_lo);
 }
 
-// (q - z) for two elements of one group, with Blackwell's packed fp32x2
-// arithmetic (each lane correctly rounded, so the values are those of the
-// scalar path): the same proven fast path, and the exact scalar path for both
-// elements whenever either fails the remainder test.
-__device__ __forceinline__ float2 quant_qz2(float2 wt, const GroupQ &g) {
-  const float2 y = __fmul2_rn(wt, make_float2(g.rcp, g.rcp));
-  float2 k = make_float2(rintf(y.x), rintf(y.y));
-  const float2 rem = __ffma2_rn(make_float2(-k.x, -k.y), make_float2(g.delta, g.delta), wt);
-  if (!(fmaxf(fabsf(rem.x), fabsf(rem.y)) < g.half_lo && fmaxf(fabsf(k.x), fabsf(k.y)) < 64.0f)) {
-    k.x = rintf(__fdiv_rn(wt.x, g.delta));
-    k.y = rintf(__fdiv_rn(wt.y, g.delta));
-  }
-  float2 q = __fadd2_rn(k, make_float2(g.zero, g.zero));
-  q.x = fminf(fmaxf(q.x, 0.0f), g.qmax);
-  q.y = fminf(fmaxf(q.y, 0.0f), g.qmax);
-  return __fadd2_rn(q, make_float2(-g.zero, -g.zero));
-}
-
 // rne(y) for |y| < 2^22 with two fp32 additions (FMA pipe): y + 1.5 2^23 lies
 // in (2^23, 2^24), where the spacing is 1, so its rounding is 1.5 2^23 +
 // rne(y) (ties to even, 1.5 2^23 being even), and removing 1.5 2^23 is exact.
@@ -165,9 +147,6 @@ __device__ __forceinline__ float quant_code(float wt, const GroupQ &g) {
   return fminf(fmaxf(q, 0.0f), g.qmax);
 }
 
-__device__ __forceinline__ float dequant(float q, const GroupQ &g) {
-  return __fmul_rn(__fsub_rn(q, g.zero), g.delta);
-}
 
 // ---------------------------------------------------------------------------
 // Bounded waits.  A wait that exceeds its poll budget records kDevTimeout and

@@ -118,3 +118,41 @@ def test_w4a16_shape_limits():
     assert abi.STATUS[st] == "AWQ_ERR_UNSUPPORTED" and "out % 32" in abi.last_error()
     st = abi.LIB.awq_w4a16_gemm(16, 256, 512, 512, 16, 16, 16, 256, ctypes.byref(cfg), 16, 200, 256, 1024, None)
     assert abi.STATUS[st] == "AWQ_ERR_INVALID_ARG" and "ldy" in abi.last_error()
+
+
+def test_sharding_calls_check_their_arguments():
+    """The token-sharding calls reject bad arguments on the host, before any
+    CUDA work, with the status the header states."""
+    L = abi.LIB
+    cfg = awq.AwqConfig.make(n_clip=20)
+    S = abi.STATUS
+    assert S[L.awq_act_sums(16, 256, 512, 512, None, None)] == "AWQ_ERR_INVALID_ARG"
+    assert S[L.awq_act_sums(16, 256, 512, 512, 12, None)] == "AWQ_ERR_INVALID_ARG"  # sums misaligned
+    assert S[L.awq_act_sums(16, 0, 512, 512, 16, None)] == "AWQ_ERR_INVALID_ARG"   # no tokens
+    assert S[L.awq_act_stats_finish(16, 0, 512, 16, None)] == "AWQ_ERR_INVALID_ARG"
+    assert S[L.awq_act_stats_finish(None, 10, 512, 16, None)] == "AWQ_ERR_INVALID_ARG"
+    st = L.awq_search_scale_sse(16, 256, 512, 512, 16, 512, 16, ctypes.byref(cfg), 256, 1 << 30, None, None)
+    assert S[st] == "AWQ_ERR_INVALID_ARG" and "sse" in abi.last_error()
+    st = L.awq_select_scale(16, 256, 512, 512, 16, ctypes.byref(cfg), 256, 128, 16, 16, 16, None)
+    assert S[st] == "AWQ_ERR_WORKSPACE"
+    st = L.awq_block_grams(16, 256, 512, 512, ctypes.byref(awq.AwqConfig.make(group_size=64)), 256, 1 << 30,
+                           16, None)
+    assert S[st] == "AWQ_ERR_UNSUPPORTED"
+    st = L.awq_block_grams(16, 256, 320, 320, ctypes.byref(cfg), 256, 1 << 30, 16, None)
+    assert S[st] == "AWQ_ERR_INVALID_ARG"
+    st = L.awq_search_clip_grams(16, 512, 512, 16, 16, ctypes.byref(awq.AwqConfig.make(n_clip=0)),
+                                 256, 1024, 16, None, None)
+    assert S[st] == "AWQ_ERR_INVALID_ARG" and "n_clip" in abi.last_error()
+    st = L.awq_search_clip_grams(16, 512, 512, 16, None, ctypes.byref(cfg), 256, 1024, 16, None, None)
+    assert S[st] == "AWQ_ERR_INVALID_ARG" and "G" in abi.last_error()
+
+
+def test_search_forms_and_zero_point_are_validated():
+    for kw, status in ((dict(search_form=3), "AWQ_ERR_INVALID_ARG"), (dict(zero_point=-1), "AWQ_ERR_INVALID_ARG")):
+        with pytest.raises(awq.AwqError) as ei:
+            awq.awq_workspace_size(256, 512, 512, awq.AwqConfig.make(**kw))
+        assert ei.value.status_name == status
+    # the cached-output form needs room for the cached output: more workspace than the error form
+    a = awq.awq_workspace_size(1000, 512, 512, awq.AwqConfig.make())
+    b = awq.awq_workspace_size(1000, 512, 512, awq.AwqConfig.make(search_form=abi.SEARCH_CACHED_Y))
+    assert b - a >= 1024 * 512 * 2
