@@ -11,9 +11,10 @@
 // the fp16 weights a consumer multiplies.  fp32 accumulation on the tensor
 // cores.
 //
-// sm_100a design, one CTA per SM (448 threads), persistent over 128 x 256
-// output tiles:
-//   warp 0      TMA loads of the 128 x 64 X tile (K-major, 128-byte swizzle)
+// sm_100a design, one CTA per SM (448 threads), persistent over 256 x 256
+// output tiles (two M = 128 accumulators share every dequantised B tile, which
+// halves the conversion work per flop):
+//   warp 0      TMA loads of the 256 x 64 X tile (K-major, 128-byte swizzle)
 //               and of the 64 x 32 block of packed words behind the B tile;
 //   warps 6..13 dequantise the 64 x 256 weight tile: each thread turns int32
 //               words (8 outputs of one input channel each) into 16-byte
@@ -26,9 +27,10 @@
 //               memory (staged by TMA with the X tile), zero points and
 //               scales from L1/L2 one step ahead;
 //   warp 1      one thread issues tcgen05.mma kind::f16 (M = 128, N = 256,
-//               K = 16) into a double-buffered TMEM accumulator;
-//   warps 2..5  read the accumulator (tcgen05.ld), round to fp16 and store Y.
-// Four pipeline stages of (16 + 32 + 8) KiB.  Every mbarrier wait is bounded; on a
+//               K = 16), two per K step, into the two halves of TMEM;
+//   warps 2..5  read the accumulators (tcgen05.ld), round to fp16 and store Y
+//               (the next tile's MMAs wait for them: TMEM holds one tile).
+// Three pipeline stages of (32 + 32 + 8) KiB.  Every mbarrier wait is bounded; on a
 // timeout the CTA records kDevTimeout, drains its copies and MMAs, frees TMEM
 // and exits.
 #include <cuda.h>
@@ -39,8 +41,9 @@
 namespace awq {
 
 namespace {
-constexpr int QBM = 128, QBN = 256, QBK = 64, QSTAGES = 4;
-constexpr uint32_t QA_BYTES = QBM * QBK * 2;   // 16 KiB
+constexpr int QBM = 256, QMM = 128, QBN = 256, QBK = 64, QSTAGES = 3;  // CTA rows, MMA rows
+constexpr uint32_t QA_BYTES = QBM * QBK * 2;   // 32 KiB
+constexpr uint32_t QA_HALF = QMM * QBK * 2;    // rows 128..255 of the X tile start here
 constexpr uint32_t QB_BOX = QBK * 128;         // 64 input channels x 64 outputs (8 KiB)
 constexpr uint32_t QB_BYTES = 4 * QB_BOX;      // 32 KiB
 constexpr uint32_t QW_BYTES = QBK * (QBN / 8) * 4;  // packed words of a B tile (8 KiB)
@@ -53,7 +56,7 @@ constexpr int Q_THREADS = (QW_DEQ + QN_DEQ) * 32;         // 448: up to 128 regi
 constexpr uint32_t Q_DRAIN = 1u << 22;
 // kind::f16, fp16 A/B, fp32 D, A K-major, B MN-major, N = 256, M = 128
 constexpr uint32_t IDESC_Q = (1u << 4) | (1u << 16) | ((uint32_t)(QBN >> 3) << 17) |
-                             ((uint32_t)(QBM >> 4) << 24);
+                             ((uint32_t)(QMM >> 4) << 24);
 
 struct __align__(8) QTail {
   uint64_t ld[QSTAGES];     // TMA bytes of the X tile and the packed words
@@ -303,14 +306,14 @@ __global__ void __launch_bounds__(Q_THREADS, 1) w4a16_gemm_kernel(
       bool ok = true, issued_any = false;
       int it = 0;
       for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++it) {
-        const int acc = it & 1;
-        const uint32_t acc_phase = (it >> 1) & 1;
+        const int acc = 0;  // one tile in TMEM: columns 0..255 rows 0..127, 256..511 rows 128..255
+        const uint32_t acc_phase = it & 1;
         if (!mbar_wait_long(&tail->tempty[acc], acc_phase ^ 1u, max_polls, abort_flag)) {
           q_abort(tail, st, 0xD20u + acc);
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * QBN;
+        const uint32_t d_tmem = tmem_base;
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait_long(&tail->full[stage], phase, max_polls, abort_flag) ||
               !mbar_wait_bounded(&tail->ld[stage], phase, max_polls, abort_flag)) {  // X tile
@@ -322,9 +325,13 @@ __global__ void __launch_bounds__(Q_THREADS, 1) w4a16_gemm_kernel(
           const uint32_t a_addr = smem_u32(sA + stage * QA_BYTES);
           const uint32_t b_addr = smem_u32(sB + stage * QB_BYTES);
 #pragma unroll
-          for (int k = 0; k < QBK / 16; ++k)
-            tc_mma_f16(d_tmem, smem_desc_k_sw128(a_addr + k * 32), desc_b_mn(b_addr + k * 2048),
-                       IDESC_Q, (kb | k) != 0 ? 1u : 0u);
+          for (int k = 0; k < QBK / 16; ++k) {
+            const uint64_t bd = desc_b_mn(b_addr + k * 2048);
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+              tc_mma_f16(d_tmem + h * QBN, smem_desc_k_sw128(a_addr + h * QA_HALF + k * 32), bd, IDESC_Q,
+                         (kb | k) != 0 ? 1u : 0u);
+          }
           issued_any = true;
           tc_commit(&tail->empty[stage]);
           if (++stage == QSTAGES) {
@@ -345,8 +352,8 @@ __global__ void __launch_bounds__(Q_THREADS, 1) w4a16_gemm_kernel(
     const int q = warp & 3;
     int it = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
-      const int acc = it & 1;
-      const uint32_t acc_phase = (it >> 1) & 1;
+      const int acc = 0;
+      const uint32_t acc_phase = it & 1;
       int ok = 1;
       if (lane == 0) ok = mbar_wait_long(&tail->tfull[acc], acc_phase, max_polls, abort_flag);
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -357,12 +364,12 @@ __global__ void __launch_bounds__(Q_THREADS, 1) w4a16_gemm_kernel(
       tc_fence_after();
       int m_blk, n_blk;
       q_tile_coords(tile, num_m, num_n, m_blk, n_blk);
-      const int64_t t_row = (int64_t)m_blk * QBM + q * 32 + lane;
-      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * QBN);
 #pragma unroll 1
-      for (int c = 0; c < QBN; c += 32) {
+      for (int c2 = 0; c2 < 2 * QBN; c2 += 32) {
+        const int h = c2 / QBN, c = c2 % QBN;  // accumulator half (rows 128 h ..) and column
+        const int64_t t_row = (int64_t)m_blk * QBM + h * QMM + q * 32 + lane;
         float v[32];
-        tmem_ld_32x32b_x32(taddr + (uint32_t)c, v);
+        tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)c2, v);
         tmem_ld_wait();
         const int64_t o0 = (int64_t)n_blk * QBN + c;
         if (t_row < T) {
