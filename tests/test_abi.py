@@ -156,3 +156,15 @@ def test_search_forms_and_zero_point_are_validated():
     a = awq.awq_workspace_size(1000, 512, 512, awq.AwqConfig.make())
     b = awq.awq_workspace_size(1000, 512, 512, awq.AwqConfig.make(search_form=abi.SEARCH_CACHED_Y))
     assert b - a >= 1024 * 512 * 2
+
+
+def test_binding_constants_match_the_header():
+    """Status codes and scoring forms in the binding are the header's."""
+    import re
+    text = open(abi.HEADER_PATH).read()
+    for name, val in re.findall(r"\b(AWQ_(?:OK|ERR_[A-Z_]+))\s*=\s*(\d+)", text):
+        assert abi.STATUS[int(val)] == name, name
+    forms = dict(re.findall(r"\b(AWQ_SEARCH_[A-Z_]+)\s*=\s*(\d+)", text))
+    assert int(forms["AWQ_SEARCH_DIRECT"]) == abi.SEARCH_DIRECT
+    assert int(forms["AWQ_SEARCH_GRAM"]) == abi.SEARCH_GRAM
+    assert int(forms["AWQ_SEARCH_CACHED_Y"]) == abi.SEARCH_CACHED_Y
