@@ -22,11 +22,23 @@
  *   - Arguments are checked on the host before anything is launched; a failed
  *     check returns AWQ_ERR_INVALID_ARG or AWQ_ERR_UNSUPPORTED and has no side
  *     effect.  awq_last_error() returns a message for the calling thread.
- *   - Device-side failures (a bounded wait in a kernel that ran out) are
- *     recorded in a status word inside the workspace; awq_device_status()
- *     synchronises the stream and reports and clears it.  Every call that
- *     takes a workspace clears that word first, so it describes the latest
- *     such call.
+ *   - Device-side failures (a bounded wait in a kernel that ran out, a
+ *     non-finite score) are recorded in a status word inside the workspace;
+ *     awq_device_status() synchronises the stream and reports and clears it.
+ *     Every call that takes a workspace clears that word first, so it
+ *     describes the latest such call.  The calls that take no workspace
+ *     (awq_quant_pack, awq_search_clip_noalloc) record theirs in one status
+ *     word of the library per device instead, which keeps every failure
+ *     until awq_device_status(NULL, stream) reads and clears it.
+ *   - With the environment variable AWQ_SYNC_CHECK set, the searches, the
+ *     packing and the allocation-free clip search synchronise before
+ *     returning and return the device status themselves.
+ *   - Fault injection for tests, environment variable AWQ_FAULT (read at
+ *     every call): "timeout" makes every bounded device wait give up after
+ *     one poll; "alloc" refuses every workspace (AWQ_ERR_WORKSPACE, and
+ *     awq_workspace_size returns 0); "launch" fails every call after its
+ *     argument checks and before any CUDA call (AWQ_ERR_CUDA); "nonfinite"
+ *     makes the alpha selection see non-finite scores (AWQ_ERR_NONFINITE).
  *   - X is [T, in] fp16, token-major, row stride ldx >= in elements (ldx a
  *     multiple of 8).  W is [out, in] fp16, row-major and contiguous, laid out
  *     like nn.Linear.  Linears that share one input and one scale (q|k|v,
@@ -162,6 +174,31 @@ awq_status awq_search_clip(const void *X, int64_t T, int64_t in, int64_t ldx,
                            const awq_config *cfg, void *ws, size_t ws_bytes,
                            uint8_t *clip_idx, float *err, awq_stream_t stream);
 
+/* Inspection form of the alpha search's candidate quantiser: the codes of
+ * every candidate of awq_search_scale's grid, produced by the same kernel and
+ * quantisation steps that build the search's scored operand ("05 — AWQ" §4:
+ * for each alpha apply the scaling and quantize).  For candidate i, row o and
+ * group k of diag(s_i) W:
+ *   q     device uint8 [n_alpha, out, in]      codes in [0, 2^b - 1]
+ *   z     device uint8 [n_alpha, out, in/g]    zero points
+ *   delta device fp32  [n_alpha, out, in/g]    steps
+ * abar as for awq_search_scale; ws as for awq_search_scale (the first
+ * 2 n_alpha in fp32 values of it are used).  Requires in % 64 == 0. */
+awq_status awq_candidate_codes(const void *W, int64_t out, int64_t in, const double *abar,
+                               const awq_config *cfg, void *ws, size_t ws_bytes, uint8_t *q,
+                               uint8_t *z, float *delta, awq_stream_t stream);
+
+/* awq_search_clip_grams, which also stores the codes of every clip candidate
+ * as its quantiser makes them (inspection form of "05 — AWQ" §4's optional
+ * clipping):
+ *   q device uint8 [out, n_clip, in]     codes of (row o, ratio c, channel j)
+ *   z device uint8 [out, n_clip, in/128] zero points of (o, c, group k)
+ * The search's own outputs (clip_idx, err) are those of awq_search_clip_grams. */
+awq_status awq_clip_candidate_codes(const void *W, int64_t out, int64_t in, const float *s,
+                                    const float *G, const awq_config *cfg, void *ws,
+                                    size_t ws_bytes, uint8_t *clip_idx, float *err, uint8_t *q,
+                                    uint8_t *z, awq_stream_t stream);
+
 /* Allocation-free variant of awq_search_clip (the AWQ pages have no
  * counterpart: this entry exists for callers, not for the method).  Some
  * callers cannot allocate device memory while the search runs: a host
@@ -181,9 +218,15 @@ awq_status awq_search_clip(const void *X, int64_t T, int64_t in, int64_t ldx,
  *   - every call shares the one array, so calls that overlap on the GPU (on
  *     different streams, or from different threads) race and must be
  *     serialised by the caller.  Nothing in the array needs clearing: each
- *     call writes every element it reads.
- * Results equal awq_search_clip's up to the fp32 summation order of the block
- * Grams (token chunks are summed in a different grouping). */
+ *     call writes every element it reads;
+ *   - a device-side failure (a bounded wait that ran out) is recorded in the
+ *     library's status word: read it with awq_device_status(NULL, stream)
+ *     (or set AWQ_SYNC_CHECK); after AWQ_ERR_TIMEOUT, clip_idx and err of
+ *     that call are not to be used.
+ * The Grams are summed over min(16, ceil(T/1024), 384/(in/128) - 1) token
+ * chunks; where that equals awq_search_clip's min(16, ceil(T/1024)) (every
+ * in <= 2048) the results are identical, otherwise they equal up to the
+ * fp32 summation order of the block Grams. */
 awq_status awq_search_clip_noalloc(const void *X, int64_t T, int64_t in, int64_t ldx,
                                    const void *W, int64_t out, const float *s,
                                    const awq_config *cfg, uint8_t *clip_idx, float *err,
@@ -195,7 +238,10 @@ awq_status awq_search_clip_noalloc(const void *X, int64_t T, int64_t in, int64_t
  *   qweight  device int32 [in, out/8]:   code of (o, j) in bits 4(o%8)..+3 of [j][o/8]
  *   qzeros   device int32 [in/g, out/8]: zero of (o, k) in bits 4(o%8)..+3 of [k][o/8]
  *   scales   device fp16 [in/g, out]:    RN16(delta of (o, k))
- * INT3 codes use the same 4-bit container. */
+ * INT3 codes use the same 4-bit container.  A clip index >= cfg->n_clip is
+ * an error found on the device: that group gets codes and zero point 0 and a
+ * NaN scale, and the library's status word records AWQ_ERR_INVALID_ARG
+ * (awq_device_status(NULL, stream)). */
 awq_status awq_quant_pack(const void *W, int64_t out, int64_t in, const float *s,
                           const uint8_t *clip_idx, const awq_config *cfg,
                           int32_t *qweight, int32_t *qzeros, void *scales,
@@ -279,7 +325,10 @@ awq_status awq_w4a16_gemm(const void *X, int64_t T, int64_t in, int64_t ldx, con
                           awq_stream_t stream);
 
 /* Synchronises `stream`, then returns and clears the device status recorded in
- * workspace `ws` (AWQ_OK, AWQ_ERR_TIMEOUT or AWQ_ERR_NONFINITE). */
+ * workspace `ws` (AWQ_OK, AWQ_ERR_TIMEOUT or AWQ_ERR_NONFINITE).  With
+ * ws = NULL: the library's status word of the current device, which the calls
+ * without a workspace use (AWQ_OK, AWQ_ERR_TIMEOUT from
+ * awq_search_clip_noalloc, AWQ_ERR_INVALID_ARG from awq_quant_pack). */
 awq_status awq_device_status(void *ws, awq_stream_t stream);
 
 /* Message describing the last failure on the calling thread ("" if none). */

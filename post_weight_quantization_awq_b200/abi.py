@@ -77,6 +77,11 @@ _SIGNATURES = {
     "awq_search_clip_noalloc": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_int64,
                                           c_void_p, POINTER(AwqConfig), c_void_p, c_void_p,
                                           c_void_p]),
+    "awq_candidate_codes": (c_int32, [c_void_p, c_int64, c_int64, c_void_p, POINTER(AwqConfig),
+                                      c_void_p, c_size_t, c_void_p, c_void_p, c_void_p, c_void_p]),
+    "awq_clip_candidate_codes": (c_int32, [c_void_p, c_int64, c_int64, c_void_p, c_void_p,
+                                           POINTER(AwqConfig), c_void_p, c_size_t, c_void_p,
+                                           c_void_p, c_void_p, c_void_p, c_void_p]),
     "awq_quant_pack": (c_int32, [c_void_p, c_int64, c_int64, c_void_p, c_void_p, POINTER(AwqConfig),
                                  c_void_p, c_void_p, c_void_p, c_void_p]),
     "awq_fold_inv_scale": (c_int32, [c_void_p, c_int64, c_int64, c_void_p, c_void_p]),
@@ -145,7 +150,7 @@ def header_functions(path: str = HEADER_PATH):
     with open(path) as f:
         text = f.read()
     text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-    return sorted(set(re.findall(r"\b(awq_[a-z_]+)\s*\(", text)))
+    return sorted(set(re.findall(r"\b(awq_[a-z0-9_]+)\s*\(", text)))
 
 
 def version() -> str:
@@ -261,6 +266,23 @@ def awq_search_clip_grams(W, s, G, cfg: AwqConfig, ws, clip_idx, err=None, strea
         ws.numel() * ws.element_size(), _ptr(clip_idx), _ptr(err), _stream(stream)))
 
 
+def awq_candidate_codes(W, abar, cfg: AwqConfig, ws, q, z, delta, stream=None) -> None:
+    """Codes q uint8 [n_alpha, out, in], zero points z uint8 and steps delta
+    fp32 [n_alpha, out, in/g] of every candidate of the alpha search."""
+    _check("awq_candidate_codes", LIB.awq_candidate_codes(
+        _ptr(W), W.shape[0], W.shape[1], _ptr(abar), ctypes.byref(cfg), _ptr(ws),
+        ws.numel() * ws.element_size(), _ptr(q), _ptr(z), _ptr(delta), _stream(stream)))
+
+
+def awq_clip_candidate_codes(W, s, G, cfg: AwqConfig, ws, clip_idx, err, q, z, stream=None) -> None:
+    """awq_search_clip_grams that also stores the clip candidates' codes q
+    uint8 [out, n_clip, in] and zero points z uint8 [out, n_clip, in/128]."""
+    _check("awq_clip_candidate_codes", LIB.awq_clip_candidate_codes(
+        _ptr(W), W.shape[0], W.shape[1], _ptr(s), _ptr(G), ctypes.byref(cfg), _ptr(ws),
+        ws.numel() * ws.element_size(), _ptr(clip_idx), _ptr(err), _ptr(q), _ptr(z),
+        _stream(stream)))
+
+
 def awq_w4a16_gemm(X, qweight, qzeros, scales, cfg: AwqConfig, Y, ws, stream=None) -> None:
     """Y [T, out] fp16 = X [T, in] times the packed weights, dequantised on the fly."""
     _check("awq_w4a16_gemm", LIB.awq_w4a16_gemm(
@@ -270,6 +292,9 @@ def awq_w4a16_gemm(X, qweight, qzeros, scales, cfg: AwqConfig, Y, ws, stream=Non
 
 
 def awq_device_status(ws, stream=None) -> None:
+    """Raises AwqError if the device status in workspace ``ws`` records a
+    failure; ws=None reads the library's own status word (the calls that take
+    no workspace: awq_quant_pack, awq_search_clip_noalloc)."""
     _check("awq_device_status", LIB.awq_device_status(_ptr(ws), _stream(stream)))
 
 

@@ -11,6 +11,8 @@
 #include <string>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "awq.h"
 #include "awq_launch.h"
 
@@ -77,6 +79,7 @@ struct ProfScope {
   cudaStream_t s;
   cudaEvent_t a = nullptr;
   ProfScope(const char *n, cudaStream_t st) : name(n), s(st) {
+    nvtxRangePushA(n);  // a no-op unless a profiler is attached
     std::lock_guard<std::mutex> lk(g_prof_mu);
     if (g_prof_on) {
       a = take_event();
@@ -84,6 +87,7 @@ struct ProfScope {
     }
   }
   ~ProfScope() {
+    nvtxRangePop();
     if (!a) return;
     std::lock_guard<std::mutex> lk(g_prof_mu);
     cudaEvent_t b = take_event();
@@ -206,13 +210,38 @@ ClipWs clip_layout(int64_t T, int64_t in) {
   return w;
 }
 
-uint32_t poll_cap() {
+// Fault injection for tests (environment variable AWQ_FAULT, read at every
+// call): "timeout" makes every bounded device wait give up after one poll;
+// "alloc" makes the workspace unobtainable (awq_workspace_size returns 0 and
+// every workspace is refused); "launch" fails every call that would launch,
+// after its argument checks and before any CUDA call; "nonfinite" makes the
+// alpha selection see non-finite scores (the MSE is divided by zero tokens).
+enum class Fault { kNone, kTimeout, kAlloc, kLaunch, kNonFinite };
+
+Fault fault_mode() {
   const char *f = getenv("AWQ_FAULT");
-  if (f && strcmp(f, "timeout") == 0) return 1u;  // test hook: every bounded wait gives up at once
-  return 1u << 24;
+  if (!f) return Fault::kNone;
+  if (strcmp(f, "timeout") == 0) return Fault::kTimeout;
+  if (strcmp(f, "alloc") == 0) return Fault::kAlloc;
+  if (strcmp(f, "launch") == 0) return Fault::kLaunch;
+  if (strcmp(f, "nonfinite") == 0) return Fault::kNonFinite;
+  return Fault::kNone;
+}
+
+uint32_t poll_cap() {
+  return fault_mode() == Fault::kTimeout ? 1u : 1u << 24;
+}
+
+// AWQ_OK, or the injected launch failure
+awq_status launch_gate() {
+  if (fault_mode() == Fault::kLaunch)
+    return fail(AWQ_ERR_CUDA, "injected launch failure (AWQ_FAULT=launch)");
+  return AWQ_OK;
 }
 
 awq_status check_ws(void *ws, size_t ws_bytes, size_t need) {
+  if (fault_mode() == Fault::kAlloc)
+    return fail(AWQ_ERR_WORKSPACE, "injected allocation failure (AWQ_FAULT=alloc)");
   if (!ws) return fail(AWQ_ERR_WORKSPACE, "workspace is NULL");
   if (!aligned(ws, 256)) return fail(AWQ_ERR_WORKSPACE, "workspace must be 256-byte aligned");
   if (ws_bytes < need)
@@ -220,6 +249,12 @@ awq_status check_ws(void *ws, size_t ws_bytes, size_t need) {
                 need);
   return AWQ_OK;
 }
+
+#define AWQ_LAUNCH_GATE()                   \
+  do {                                      \
+    const awq_status g_ = launch_gate();    \
+    if (g_ != AWQ_OK) return g_;            \
+  } while (0)
 
 #define AWQ_TRY_CUDA(expr, what)                  \
   do {                                            \
@@ -236,6 +271,11 @@ const char *awq_version(void) { return "awq-b200 0.1 (sm_100a)"; }
 const char *awq_last_error(void) { return g_err.c_str(); }
 
 size_t awq_workspace_size(int64_t T, int64_t in, int64_t out, const awq_config *cfg) {
+  g_err.clear();
+  if (fault_mode() == Fault::kAlloc) {
+    fail(AWQ_ERR_WORKSPACE, "injected allocation failure (AWQ_FAULT=alloc)");
+    return 0;
+  }
   if (check_cfg(cfg) != AWQ_OK) return 0;
   if (check_shape(T, in, out, cfg) != AWQ_OK) return 0;
   size_t need = scale_layout(T, in, out, cfg).end;
@@ -254,6 +294,7 @@ awq_status awq_act_stats(const void *X, int64_t T, int64_t in, int64_t ldx, doub
   awq_status st = check_x(X, in, ldx);
   if (st != AWQ_OK) return st;
   if (!abar || !aligned(abar, 8)) return fail(AWQ_ERR_INVALID_ARG, "abar is NULL or misaligned");
+  AWQ_LAUNCH_GATE();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   ProfScope p("act_stats", s);
   AWQ_TRY_CUDA(launch_act_stats(static_cast<const __half *>(X), T, in, ldx, abar,
@@ -268,6 +309,7 @@ awq_status awq_scale_grid(const double *abar, int64_t in, int32_t n_alpha, float
   if (!abar || !s) return fail(AWQ_ERR_INVALID_ARG, "abar or s is NULL");
   if (in < 1 || in > (int64_t(1) << 24)) return fail(AWQ_ERR_INVALID_ARG, "in=%lld", (long long)in);
   if (n_alpha < 1 || n_alpha > 64) return fail(AWQ_ERR_INVALID_ARG, "n_alpha=%d (1..64)", n_alpha);
+  AWQ_LAUNCH_GATE();
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   ProfScope p("scale_grid", st);
   AWQ_TRY_CUDA(launch_scale_grid(abar, in, n_alpha, s, nullptr, st), "scale_grid launch");
@@ -297,6 +339,7 @@ awq_status search_scale_impl(const void *X, int64_t T, int64_t in, int64_t ldx, 
   if ((st = check_ws(ws, ws_bytes, L.end)) != AWQ_OK) return st;
   const int64_t tiles = (int64_t)L.num_m * L.nb_per_alpha * cfg->n_alpha;
   if (tiles > INT32_MAX) return fail(AWQ_ERR_INVALID_ARG, "problem too large (%lld tiles)", (long long)tiles);
+  AWQ_LAUNCH_GATE();
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint8_t *base = static_cast<uint8_t *>(ws);
@@ -365,13 +408,15 @@ awq_status search_scale_impl(const void *X, int64_t T, int64_t in, int64_t ldx, 
   }
   {
     ProfScope p("mse_argmin", s);
+    // AWQ_FAULT=nonfinite: normalising by zero tokens makes every score non-finite
+    const int64_t t_norm = fault_mode() == Fault::kNonFinite ? 0 : (sse ? 1 : T);
     if (sse)  // T = out = 1: the plain sums of squared errors
-      AWQ_TRY_CUDA(launch_mse_argmin(partials, cfg->n_alpha, L.per_alpha, 1, 1, s_grid, in, dst, sse,
-                                     nullptr, nullptr, s),
+      AWQ_TRY_CUDA(launch_mse_argmin(partials, cfg->n_alpha, L.per_alpha, t_norm, 1, s_grid, in, dst,
+                                     sse, nullptr, nullptr, s),
                    "mse_argmin launch");
     else
-      AWQ_TRY_CUDA(launch_mse_argmin(partials, cfg->n_alpha, L.per_alpha, T, out, s_grid, in, dst,
-                                     mse, best_idx, s_best, s),
+      AWQ_TRY_CUDA(launch_mse_argmin(partials, cfg->n_alpha, L.per_alpha, t_norm, out, s_grid, in,
+                                     dst, mse, best_idx, s_best, s),
                    "mse_argmin launch");
   }
   if (getenv("AWQ_SYNC_CHECK")) return awq_device_status(ws, stream);
@@ -407,11 +452,13 @@ awq_status awq_select_scale(const double *sse, int64_t T_total, int64_t in, int6
   if (!sse || !abar || !s_best || !mse || !best_idx)
     return fail(AWQ_ERR_INVALID_ARG, "a pointer argument is NULL");
   if ((st = check_ws(ws, ws_bytes, kHeader)) != AWQ_OK) return st;
+  AWQ_LAUNCH_GATE();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   DevStatus *dst = static_cast<DevStatus *>(ws);
   AWQ_TRY_CUDA(cudaMemsetAsync(dst, 0, sizeof(DevStatus), s), "workspace reset");
   ProfScope p("select_scale", s);
-  AWQ_TRY_CUDA(launch_select_scale(sse, cfg->n_alpha, T_total, out, abar, in, dst, mse, best_idx,
+  const int64_t t_norm = fault_mode() == Fault::kNonFinite ? 0 : T_total;  // see Fault
+  AWQ_TRY_CUDA(launch_select_scale(sse, cfg->n_alpha, t_norm, out, abar, in, dst, mse, best_idx,
                                    s_best, s),
                "select_scale launch");
   return AWQ_OK;
@@ -425,6 +472,7 @@ awq_status awq_act_sums(const void *X, int64_t T, int64_t in, int64_t ldx, int64
   awq_status st = check_x(X, in, ldx);
   if (st != AWQ_OK) return st;
   if (!sums || !aligned(sums, 8)) return fail(AWQ_ERR_INVALID_ARG, "sums is NULL or misaligned");
+  AWQ_LAUNCH_GATE();
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   ProfScope p("act_stats", s);
   AWQ_TRY_CUDA(launch_act_sums(static_cast<const __half *>(X), T, in, ldx, sums, num_sms_current(), s),
@@ -439,6 +487,7 @@ awq_status awq_act_stats_finish(const int64_t *sums, int64_t T_total, int64_t in
     return fail(AWQ_ERR_INVALID_ARG, "T_total=%lld (1..2^22)", (long long)T_total);
   if (in < 1) return fail(AWQ_ERR_INVALID_ARG, "in=%lld", (long long)in);
   if (!sums || !abar) return fail(AWQ_ERR_INVALID_ARG, "sums or abar is NULL");
+  AWQ_LAUNCH_GATE();
   AWQ_TRY_CUDA(launch_act_finish(sums, in, T_total, abar, static_cast<cudaStream_t>(stream)),
                "act_finish launch");
   return AWQ_OK;
@@ -460,6 +509,7 @@ awq_status awq_search_clip(const void *X, int64_t T, int64_t in, int64_t ldx, co
   if (s && !aligned(s, 16)) return fail(AWQ_ERR_INVALID_ARG, "s must be 16-byte aligned");
   const ClipWs L = clip_layout(T, in);
   if ((st = check_ws(ws, ws_bytes, L.end)) != AWQ_OK) return st;
+  AWQ_LAUNCH_GATE();
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   uint8_t *base = static_cast<uint8_t *>(ws);
   float *gpart = reinterpret_cast<float *>(base + L.gpart);
@@ -497,6 +547,7 @@ awq_status awq_block_grams(const void *X, int64_t T, int64_t in, int64_t ldx, co
   if (!G || !aligned(G, 16)) return fail(AWQ_ERR_INVALID_ARG, "G is NULL or not 16-byte aligned");
   const ClipWs L = clip_layout(T, in);
   if ((st = check_ws(ws, ws_bytes, L.end)) != AWQ_OK) return st;
+  AWQ_LAUNCH_GATE();
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   uint8_t *base = static_cast<uint8_t *>(ws);
   AWQ_TRY_CUDA(cudaMemsetAsync(base, 0, sizeof(DevStatus), cs), "workspace reset");
@@ -523,6 +574,7 @@ awq_status awq_search_clip_grams(const void *W, int64_t out, int64_t in, const f
   if (!clip_idx) return fail(AWQ_ERR_INVALID_ARG, "clip_idx is NULL");
   if (s && !aligned(s, 16)) return fail(AWQ_ERR_INVALID_ARG, "s must be 16-byte aligned");
   if ((st = check_ws(ws, ws_bytes, kHeader)) != AWQ_OK) return st;
+  AWQ_LAUNCH_GATE();
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   uint8_t *base = static_cast<uint8_t *>(ws);
   AWQ_TRY_CUDA(cudaMemsetAsync(base, 0, sizeof(DevStatus), cs), "workspace reset");
@@ -530,6 +582,71 @@ awq_status awq_search_clip_grams(const void *W, int64_t out, int64_t in, const f
   AWQ_TRY_CUDA(launch_clip_eval(static_cast<const __half *>(W), out, in, s, G, cfg->group_size,
                                 cfg->w_bit, cfg->zero_point, cfg->n_clip, cfg->clip_min, clip_idx, err,
                                 reinterpret_cast<DevStatus *>(base), poll_cap(), num_sms_current(), cs),
+               "clip_eval launch");
+  return AWQ_OK;
+}
+
+awq_status awq_candidate_codes(const void *W, int64_t out, int64_t in, const double *abar,
+                               const awq_config *cfg, void *ws, size_t ws_bytes, uint8_t *q,
+                               uint8_t *z, float *delta, awq_stream_t stream) {
+  g_err.clear();
+  awq_status st = check_cfg(cfg);
+  if (st != AWQ_OK) return st;
+  if ((st = check_shape(1, in, out, cfg)) != AWQ_OK) return st;
+  if (in % 64 != 0) return fail(AWQ_ERR_UNSUPPORTED, "in=%lld: needs in %% 64 == 0", (long long)in);
+  if (!W || !aligned(W, 16)) return fail(AWQ_ERR_INVALID_ARG, "W is NULL or not 16-byte aligned");
+  if (!abar || !q || !z || !delta) return fail(AWQ_ERR_INVALID_ARG, "a pointer argument is NULL");
+  if (!aligned(q, 8)) return fail(AWQ_ERR_INVALID_ARG, "q must be 8-byte aligned");
+  // the s grid and 1/s as the direct-form search lays them out
+  awq_config c = *cfg;
+  c.search_form = AWQ_SEARCH_DIRECT;
+  const ScaleWs L = scale_layout(1, in, out, &c);
+  if ((st = check_ws(ws, ws_bytes, L.dW)) != AWQ_OK) return st;
+  AWQ_LAUNCH_GATE();
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  uint8_t *base = static_cast<uint8_t *>(ws);
+  DevStatus *dst = reinterpret_cast<DevStatus *>(base);
+  float *s_grid = reinterpret_cast<float *>(base + L.s_grid);
+  float *inv_s = reinterpret_cast<float *>(base + L.inv_s);
+  const int nsm = num_sms_current();
+  AWQ_TRY_CUDA(cudaMemsetAsync(dst, 0, sizeof(DevStatus), cs), "workspace reset");
+  AWQ_TRY_CUDA(launch_wmax(static_cast<const __half *>(W), out * in, in, nullptr, dst, nsm, cs),
+               "wmax launch");
+  AWQ_TRY_CUDA(launch_scale_grid(abar, in, cfg->n_alpha, s_grid, inv_s, cs), "scale_grid launch");
+  ProfScope p("cand_codes", cs);
+  AWQ_TRY_CUDA(launch_cand_codes(static_cast<const __half *>(W), out, in, L.out_pad,
+                                 s_grid, inv_s, cfg->n_alpha, cfg->group_size, cfg->w_bit,
+                                 cfg->zero_point, dst, q, z, delta, cs),
+               "cand_codes launch");
+  return AWQ_OK;
+}
+
+awq_status awq_clip_candidate_codes(const void *W, int64_t out, int64_t in, const float *s,
+                                    const float *G, const awq_config *cfg, void *ws,
+                                    size_t ws_bytes, uint8_t *clip_idx, float *err, uint8_t *q,
+                                    uint8_t *z, awq_stream_t stream) {
+  g_err.clear();
+  awq_status st = check_cfg(cfg);
+  if (st != AWQ_OK) return st;
+  if (cfg->n_clip < 1) return fail(AWQ_ERR_INVALID_ARG, "n_clip=%d: clip search needs n_clip >= 1", cfg->n_clip);
+  if (cfg->group_size != 128)
+    return fail(AWQ_ERR_UNSUPPORTED, "group_size=%d: the clip search handles groups of 128", cfg->group_size);
+  if ((st = check_shape(1, in, out, cfg)) != AWQ_OK) return st;
+  if (!W || !aligned(W, 16)) return fail(AWQ_ERR_INVALID_ARG, "W is NULL or not 16-byte aligned");
+  if (!G || !aligned(G, 16)) return fail(AWQ_ERR_INVALID_ARG, "G is NULL or not 16-byte aligned");
+  if (!clip_idx || !q || !z) return fail(AWQ_ERR_INVALID_ARG, "clip_idx, q or z is NULL");
+  if (!aligned(q, 8)) return fail(AWQ_ERR_INVALID_ARG, "q must be 8-byte aligned");
+  if (s && !aligned(s, 16)) return fail(AWQ_ERR_INVALID_ARG, "s must be 16-byte aligned");
+  if ((st = check_ws(ws, ws_bytes, kHeader)) != AWQ_OK) return st;
+  AWQ_LAUNCH_GATE();
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  uint8_t *base = static_cast<uint8_t *>(ws);
+  AWQ_TRY_CUDA(cudaMemsetAsync(base, 0, sizeof(DevStatus), cs), "workspace reset");
+  ProfScope p("clip_eval", cs);
+  AWQ_TRY_CUDA(launch_clip_eval(static_cast<const __half *>(W), out, in, s, G, cfg->group_size,
+                                cfg->w_bit, cfg->zero_point, cfg->n_clip, cfg->clip_min, clip_idx, err,
+                                reinterpret_cast<DevStatus *>(base), poll_cap(), num_sms_current(), cs,
+                                q, z),
                "clip_eval launch");
   return AWQ_OK;
 }
@@ -546,6 +663,7 @@ awq_status awq_quant_pack(const void *W, int64_t out, int64_t in, const float *s
   if (clip_idx && cfg->n_clip < 1)
     return fail(AWQ_ERR_INVALID_ARG, "clip_idx given but n_clip=%d", cfg->n_clip);
   if (!qweight || !qzeros || !scales) return fail(AWQ_ERR_INVALID_ARG, "an output pointer is NULL");
+  AWQ_LAUNCH_GATE();
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   ProfScope p("quant_pack", cs);
   AWQ_TRY_CUDA(launch_quant_pack(static_cast<const __half *>(W), out, in, s, clip_idx,
@@ -553,6 +671,7 @@ awq_status awq_quant_pack(const void *W, int64_t out, int64_t in, const float *s
                                  cfg->clip_min, qweight,
                                  qzeros, static_cast<__half *>(scales), cs),
                "quant_pack launch");
+  if (getenv("AWQ_SYNC_CHECK")) return awq_device_status(nullptr, stream);
   return AWQ_OK;
 }
 
@@ -574,6 +693,7 @@ awq_status awq_w4a16_gemm(const void *X, int64_t T, int64_t in, int64_t ldx, con
   if (ldy < out || ldy % 8 != 0)
     return fail(AWQ_ERR_INVALID_ARG, "ldy=%lld must be >= out and a multiple of 8", (long long)ldy);
   if ((st = check_ws(ws, ws_bytes, kHeader)) != AWQ_OK) return st;
+  AWQ_LAUNCH_GATE();
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   DevStatus *dst = static_cast<DevStatus *>(ws);
   AWQ_TRY_CUDA(cudaMemsetAsync(dst, 0, sizeof(DevStatus), cs), "workspace reset");
@@ -590,6 +710,7 @@ awq_status awq_fold_inv_scale(void *v, int64_t rows, int64_t cols, const float *
   g_err.clear();
   if (!v || !s) return fail(AWQ_ERR_INVALID_ARG, "v or s is NULL");
   if (rows < 1 || cols < 1) return fail(AWQ_ERR_INVALID_ARG, "rows=%lld cols=%lld", (long long)rows, (long long)cols);
+  AWQ_LAUNCH_GATE();
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   ProfScope p("fold", cs);
   AWQ_TRY_CUDA(launch_fold(static_cast<__half *>(v), rows, cols, s, cs), "fold launch");
@@ -598,16 +719,23 @@ awq_status awq_fold_inv_scale(void *v, int64_t rows, int64_t cols, const float *
 
 awq_status awq_device_status(void *ws, awq_stream_t stream) {
   g_err.clear();
-  if (!ws || !aligned(ws, 256)) return fail(AWQ_ERR_WORKSPACE, "workspace is NULL or misaligned");
+  if (ws && !aligned(ws, 256)) return fail(AWQ_ERR_WORKSPACE, "workspace is misaligned");
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   AWQ_TRY_CUDA(cudaStreamSynchronize(cs), "stream synchronize");
   DevStatus h;
-  AWQ_TRY_CUDA(cudaMemcpy(&h, ws, sizeof(h), cudaMemcpyDeviceToHost), "status read");
-  const uint32_t zero[2] = {0, 0};
-  AWQ_TRY_CUDA(cudaMemcpy(ws, zero, sizeof(zero), cudaMemcpyHostToDevice), "status clear");
+  if (ws) {
+    AWQ_TRY_CUDA(cudaMemcpy(&h, ws, sizeof(h), cudaMemcpyDeviceToHost), "status read");
+    const uint32_t zero[2] = {0, 0};
+    AWQ_TRY_CUDA(cudaMemcpy(ws, zero, sizeof(zero), cudaMemcpyHostToDevice), "status clear");
+  } else {  // the library's own word, used by the calls that take no workspace
+    AWQ_TRY_CUDA(lib_status_read_clear(&h), "library status read");
+  }
   if (h.flags & kDevTimeout)
     return fail(AWQ_ERR_TIMEOUT, "a bounded device wait ran out (site 0x%x)", h.where);
   if (h.flags & kDevNonFinite) return fail(AWQ_ERR_NONFINITE, "a candidate score is not finite");
+  if (h.flags & kDevBadIndex)
+    return fail(AWQ_ERR_INVALID_ARG,
+                "awq_quant_pack was given a clip index >= n_clip (those groups got a NaN scale)");
   return AWQ_OK;
 }
 
@@ -660,20 +788,26 @@ awq_status awq_profile_reset(void) {
 // overlap its budget), or code that must not call cudaMalloc because that
 // call can synchronise the whole device in the middle of its pipelined
 // stream work.  awq_search_clip_noalloc takes no workspace: its block-Gram
-// scratch lives in the file-scope device array below, sized for layers of up
-// to kNoAllocMaxIn input channels.  The array is part of this library's
-// module, so every GPU that loads the library holds it (24 MiB) until the
-// process exits.
+// scratch lives in the file-scope device array below, which holds 384 blocks
+// of 128 x 128 fp32 (24 MiB): the Grams of up to kNoAllocMaxIn / 128 groups
+// plus the per-chunk partials of as many token chunks as the rest holds.
+// The array is part of this library's module, so every GPU that loads the
+// library holds it until the process exits.  Device-side failures go to the
+// library's status word (the one awq_quant_pack uses), read with
+// awq_device_status(NULL, stream).
 // ---------------------------------------------------------------------------
 namespace {
 constexpr int64_t kNoAllocMaxIn = 16384;  // up to 128 groups of 128 channels
-constexpr int kNoAllocChunks = 2;         // token chunks of the block-Gram partials
+constexpr int64_t kNoAllocBlocks = 384;   // 128 x 128 fp32 blocks in the array
 constexpr size_t kNoAllocGroupFloats = 128 * 128;
-constexpr size_t kNoAllocFloats =
-    (size_t)(kNoAllocChunks + 1) * (size_t)(kNoAllocMaxIn / 128) * kNoAllocGroupFloats;
+constexpr size_t kNoAllocFloats = (size_t)kNoAllocBlocks * kNoAllocGroupFloats;
 
+struct NoAllocDev {
+  float *scratch;
+  DevStatus *status;
+};
 std::mutex g_noalloc_mu;
-float *g_noalloc_ptr[64] = {};
+NoAllocDev g_noalloc_dev[64] = {};
 }  // namespace
 
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocFloats];
@@ -698,41 +832,60 @@ extern "C" awq_status awq_search_clip_noalloc(const void *X, int64_t T, int64_t 
   if (!W || !aligned(W, 16)) return fail(AWQ_ERR_INVALID_ARG, "W is NULL or not 16-byte aligned");
   if (!clip_idx) return fail(AWQ_ERR_INVALID_ARG, "clip_idx is NULL");
   if (s && !aligned(s, 16)) return fail(AWQ_ERR_INVALID_ARG, "s must be 16-byte aligned");
+  AWQ_LAUNCH_GATE();
 
-  // Device address of the static scratch, looked up once per device with that
-  // device current (the host-side symbol is not a device address).
+  // Device addresses of the static scratch and of the status word, looked up
+  // once per device with that device current (the host-side symbols are not
+  // device addresses).
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
   if (dev < 0 || dev >= 64) return fail(AWQ_ERR_UNSUPPORTED, "device ordinal %d", dev);
-  float *scratch = nullptr;
+  NoAllocDev nd;
   {
     std::lock_guard<std::mutex> lk(g_noalloc_mu);
-    if (!g_noalloc_ptr[dev]) {
+    if (!g_noalloc_dev[dev].scratch) {
       void *p = nullptr;
       e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
       if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(static clip scratch)");
-      g_noalloc_ptr[dev] = static_cast<float *>(p);
+      DevStatus *sp = nullptr;
+      e = lib_status_address(&sp);
+      if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(library status word)");
+      g_noalloc_dev[dev].status = sp;
+      g_noalloc_dev[dev].scratch = static_cast<float *>(p);
     }
-    scratch = g_noalloc_ptr[dev];
+    nd = g_noalloc_dev[dev];
   }
 
-  // Every scratch element a call reads is written earlier in the same call
-  // (all chunk partials of the groups in use, then their sums), so nothing
-  // has to be cleared between calls.
-  const int64_t c = (T + 1023) / 1024;
-  const int n_chunks = (int)(c < 1 ? 1 : (c > kNoAllocChunks ? kNoAllocChunks : c));
-  const size_t gsz = (size_t)(in / 128) * kNoAllocGroupFloats;
-  float *gpart = scratch;
-  float *Gk = scratch + gsz * (size_t)n_chunks;
+  // Token chunks of the block-Gram partials: as many as the workspace form
+  // uses (up to 16, one per 1024 tokens) while chunks + 1 sets of the layer's
+  // group blocks fit in the array.  Every scratch element a call reads is
+  // written earlier in the same call when no wait runs out (all chunk
+  // partials of the groups in use, then their sums); after a timeout the
+  // status word says so and clip_idx is not to be used.
+  const int64_t groups = in / 128;
+  const int64_t fit = kNoAllocBlocks / groups - 1;  // >= 2 for in <= kNoAllocMaxIn
+  int64_t c = (T + 1023) / 1024;
+  if (c > 16) c = 16;
+  if (c > fit) c = fit;
+  const int n_chunks = (int)(c < 1 ? 1 : c);
+  const size_t gsz = (size_t)groups * kNoAllocGroupFloats;
+  float *gpart = nd.scratch;
+  float *Gk = nd.scratch + gsz * (size_t)n_chunks;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
-  // no status word here: a bounded wait that ran out leaves clip_idx unset
-  e = launch_gram_blocks(static_cast<const __half *>(X), T, in, ldx, cfg->group_size, n_chunks,
-                         gpart, Gk, nullptr, 1u << 24, cs);
-  if (e != cudaSuccess) return cuda_fail(e, "gram_blocks launch");
-  e = launch_clip_eval(static_cast<const __half *>(W), out, in, s, Gk, cfg->group_size, cfg->w_bit,
-                       cfg->zero_point, cfg->n_clip, cfg->clip_min, clip_idx, err, nullptr, 1u << 24,
-                       num_sms_current(), cs);
-  if (e != cudaSuccess) return cuda_fail(e, "clip_eval launch");
+  {
+    ProfScope p("gram_blocks", cs);
+    e = launch_gram_blocks(static_cast<const __half *>(X), T, in, ldx, cfg->group_size, n_chunks,
+                           gpart, Gk, nd.status, poll_cap(), cs);
+    if (e != cudaSuccess) return cuda_fail(e, "gram_blocks launch");
+  }
+  {
+    ProfScope p("clip_eval", cs);
+    e = launch_clip_eval(static_cast<const __half *>(W), out, in, s, Gk, cfg->group_size, cfg->w_bit,
+                         cfg->zero_point, cfg->n_clip, cfg->clip_min, clip_idx, err, nd.status,
+                         poll_cap(), num_sms_current(), cs);
+    if (e != cudaSuccess) return cuda_fail(e, "clip_eval launch");
+  }
+  if (getenv("AWQ_SYNC_CHECK")) return awq_device_status(nullptr, stream);
   return AWQ_OK;
 }

@@ -15,6 +15,7 @@ enum : uint32_t {
   kDevOk = 0,
   kDevTimeout = 1u << 0,    // a bounded wait ran out
   kDevNonFinite = 1u << 1,  // a score was NaN or infinite
+  kDevBadIndex = 1u << 2,   // a clip index passed to the packing was >= n_clip
 };
 
 struct DevStatus {

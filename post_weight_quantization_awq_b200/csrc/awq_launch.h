@@ -46,6 +46,13 @@ cudaError_t launch_cand_quant(const __half *W, int64_t out, int64_t in, int64_t 
                               int group, int w_bit, int zero_point, int weights_only,
                               const DevStatus *st, __half *dW, int num_sms, cudaStream_t stream);
 
+// K3, inspection form: the candidates' codes q [n_alpha, out, in], zero
+// points z and steps delta [n_alpha, out, in/group] (direct-form k).
+cudaError_t launch_cand_codes(const __half *W, int64_t out, int64_t in, int64_t out_pad,
+                              const float *s, const float *inv_s, int n_alpha, int group, int w_bit,
+                              int zero_point, const DevStatus *st, uint8_t *q, uint8_t *z,
+                              float *delta, cudaStream_t stream);
+
 // K4: scored GEMM, partial sums of squares per (n-tile, m-tile, warp).
 struct SearchGemmShape {
   int64_t T, in, rows_b;  // rows_b = n_alpha * out_pad
@@ -97,13 +104,19 @@ cudaError_t launch_gram_blocks(const __half *X, int64_t T, int64_t in, int64_t l
 cudaError_t launch_clip_eval(const __half *W, int64_t out, int64_t in, const float *s,
                              const float *G, int group, int w_bit, int zero_point, int n_clip,
                              float clip_min, uint8_t *clip_idx, float *err, DevStatus *st,
-                             uint32_t max_polls, int num_sms, cudaStream_t stream);
+                             uint32_t max_polls, int num_sms, cudaStream_t stream,
+                             uint8_t *cand_q = nullptr, uint8_t *cand_z = nullptr);
 
 // K7: final codes + packing.
 cudaError_t launch_quant_pack(const __half *W, int64_t out, int64_t in, const float *s,
                               const uint8_t *clip_idx, int group, int w_bit, int zero_point,
                               int n_clip, float clip_min, int32_t *qweight, int32_t *qzeros,
                               __half *scales, cudaStream_t stream);
+
+// The status word of the calls that take no workspace: its device address on
+// the current device, and a synchronous read that clears it.
+cudaError_t lib_status_address(DevStatus **p);
+cudaError_t lib_status_read_clear(DevStatus *h);
 
 // W4A16 GEMM on the packed output: Y = RN16(X Wd^T), Wd = RN16((q - z) scale);
 // in % 64 == 0, out % 32 == 0, group in {32, 64, 128}.

@@ -313,10 +313,15 @@ __device__ __forceinline__ float clip_ratio_f(int c, int n_clip, float clip_min)
 // flight: producers (warps 0-11, three per SM sub-partition) build tile t's
 // candidates while the MMA warp runs tile t-1 and the epilogue warps (13-16)
 // score and pick tile t-2.
+// kCodes: the producers also store every candidate's codes q [out, n_clip, in]
+// and zero points z [out, n_clip, in/128] (the inspection form; the search
+// itself is unchanged).
+template <bool kCodes>
 __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
     const __half *__restrict__ W, int64_t out, int64_t in, const float *__restrict__ s,
     const float *__restrict__ Gall, float qmax, int sym, int n_clip, float clip_min, int rows_per_tile,
-    uint8_t *__restrict__ clip_idx, float *__restrict__ err, DevStatus *st, uint32_t max_polls) {
+    uint8_t *__restrict__ clip_idx, float *__restrict__ err, DevStatus *st, uint32_t max_polls,
+    uint8_t *__restrict__ cq, uint8_t *__restrict__ cz) {
   extern __shared__ uint8_t csm_raw[];
   ClipSmem &S = *reinterpret_cast<ClipSmem *>(
       (reinterpret_cast<uintptr_t>(csm_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -521,6 +526,21 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
             v[2 * h + 1] = d2.y;
           }
           if (store) split_store8(ahi, alo, sw128_off(p0 + c, ch & 7), v);
+          if constexpr (kCodes) {
+            const int64_t o = (item - k * n_tiles) * R + rr;
+            if (store && o < out) {
+              uint32_t cw[2] = {0u, 0u};
+#pragma unroll
+              for (int h = 0; h < 4; ++h) {
+                const float qa = fminf(fmaxf(kq[h].x, lo), hi) + zz;
+                const float qb = fminf(fmaxf(kq[h].y, lo), hi) + zz;
+                cw[h >> 1] |= ((uint32_t)qa << (16 * (h & 1))) | ((uint32_t)qb << (16 * (h & 1) + 8));
+              }
+              *reinterpret_cast<uint2 *>(cq + (o * n_clip + c) * in + k * G + 8 * ch) =
+                  make_uint2(cw[0], cw[1]);
+              if (ch == 0) cz[(o * n_clip + c) * n_groups + k] = (uint8_t)zz;
+            }
+          }
         }
       }
       if (item + 1 < item_end) load_rows(item + 1);
@@ -669,20 +689,21 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
 cudaError_t launch_clip_eval(const __half *W, int64_t out, int64_t in, const float *s,
                              const float *Gall, int group, int w_bit, int zero_point, int n_clip,
                              float clip_min, uint8_t *clip_idx, float *err, DevStatus *st,
-                             uint32_t max_polls, int num_sms, cudaStream_t stream) {
+                             uint32_t max_polls, int num_sms, cudaStream_t stream, uint8_t *cq,
+                             uint8_t *cz) {
   if (group != G || n_clip < 1 || n_clip > 128) return cudaErrorInvalidValue;
   int R = 128 / n_clip;
   if (R > CT_MAXR) R = CT_MAXR;
   const int64_t n_items = (in / G) * ((out + R - 1) / R);
   const int64_t ctas = i64min(num_sms, n_items);  // one CTA per SM (shared memory bound)
-  cudaError_t e = cudaFuncSetAttribute(clip_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  auto kern = cq ? clip_tc_kernel<true> : clip_tc_kernel<false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kClipSmemBytes);
   if (e != cudaSuccess) return e;
   dim3 grid((unsigned)ctas);
-  clip_tc_kernel<<<grid, CT_THREADS, kClipSmemBytes, stream>>>(
+  kern<<<grid, CT_THREADS, kClipSmemBytes, stream>>>(
       W, out, in, s, Gall, (float)((1 << w_bit) - 1), zero_point ? 0 : 1, n_clip, clip_min, R,
-      clip_idx, err, st,
-      max_polls);
+      clip_idx, err, st, max_polls, cq, cz);
   return cudaGetLastError();
 }
 

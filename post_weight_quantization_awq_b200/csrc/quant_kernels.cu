@@ -255,12 +255,17 @@ cudaError_t launch_wmax(const __half *W, int64_t n, int64_t in, const float *r, 
 // ---------------------------------------------------------------------------
 constexpr int kCandRows = 64;
 
-template <int group>  // 32, 64 or 128: the range shuffles unroll
+// kCodes: instead of the B operand, the same candidates' codes q [n_alpha,
+// out, in], zero points z and steps delta [n_alpha, out, in/group] (delta of
+// s, i.e. the s 2^k step times 2^-k, exact) -- the inspection form of the
+// kernel, with every quantisation step shared with the operand form.
+template <int group, bool kCodes>  // group 32, 64 or 128: the range shuffles unroll
 __global__ void __launch_bounds__(256) cand_quant_kernel(
     const __half *__restrict__ W, int64_t out, int64_t in, int64_t out_pad,
     const float *__restrict__ s, const float *__restrict__ inv_s, const float *__restrict__ rch,
     float qmax, int sym, int weights_only, const DevStatus *__restrict__ st,
-    __half *__restrict__ dW) {
+    __half *__restrict__ dW, uint8_t *__restrict__ cq, uint8_t *__restrict__ cz,
+    float *__restrict__ cdelta) {
   // Everything runs on s 2^k: codes and zero points are those of s (power-of-
   // two invariance), delta comes out times 2^k, and the candidate error
   // (deq - s w) 2^k (r / s) needs one FFMA2 and one FMUL2 per pair.  It drops
@@ -329,6 +334,24 @@ __global__ void __launch_bounds__(256) cand_quant_kernel(
     fast_path_check(g, mx, mn);
     float2 qz[4];
     quant_qz_pairs<4>(wt, g, qz);
+    if constexpr (kCodes) {
+      if (live) {
+        uint32_t b[2] = {0u, 0u};
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          // q = (q - z) + z, small exact integers in [0, qmax]
+          b[h >> 1] |= (uint32_t)__fadd_rn(qz[h].x, g.zero) << (16 * (h & 1));
+          b[h >> 1] |= (uint32_t)__fadd_rn(qz[h].y, g.zero) << (16 * (h & 1) + 8);
+        }
+        *reinterpret_cast<uint2 *>(cq + ((int64_t)a * out + o) * in + j0) = make_uint2(b[0], b[1]);
+        if ((lane & (lanes - 1)) == 0) {
+          const int64_t gi = ((int64_t)a * out + o) * (in / group) + j0 / group;
+          cz[gi] = (uint8_t)g.zero;
+          cdelta[gi] = ldexpf(g.delta, -k);
+        }
+      }
+      continue;
+    }
     const float2 dl = make_float2(g.delta, g.delta);
     uint32_t packed[4];
 #pragma unroll
@@ -354,9 +377,26 @@ cudaError_t launch_cand_quant(const __half *W, int64_t out, int64_t in, int64_t 
   (void)num_sms;
   dim3 grid((unsigned)(n_alpha * (out_pad / kCandRows)), (unsigned)((in + 255) / 256));
   if (group != 32 && group != 64 && group != 128) return cudaErrorInvalidValue;
-  auto kern = group == 32 ? cand_quant_kernel<32> : group == 64 ? cand_quant_kernel<64> : cand_quant_kernel<128>;
+  auto kern = group == 32   ? cand_quant_kernel<32, false>
+              : group == 64 ? cand_quant_kernel<64, false>
+                            : cand_quant_kernel<128, false>;
   kern<<<grid, 256, 0, stream>>>(W, out, in, out_pad, s, inv_s, r, (float)((1 << w_bit) - 1),
-                                 zero_point ? 0 : 1, weights_only, st, dW);
+                                 zero_point ? 0 : 1, weights_only, st, dW, nullptr, nullptr,
+                                 nullptr);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_cand_codes(const __half *W, int64_t out, int64_t in, int64_t out_pad,
+                              const float *s, const float *inv_s, int n_alpha, int group, int w_bit,
+                              int zero_point, const DevStatus *st, uint8_t *q, uint8_t *z,
+                              float *delta, cudaStream_t stream) {
+  dim3 grid((unsigned)(n_alpha * (out_pad / kCandRows)), (unsigned)((in + 255) / 256));
+  if (group != 32 && group != 64 && group != 128) return cudaErrorInvalidValue;
+  auto kern = group == 32   ? cand_quant_kernel<32, true>
+              : group == 64 ? cand_quant_kernel<64, true>
+                            : cand_quant_kernel<128, true>;
+  kern<<<grid, 256, 0, stream>>>(W, out, in, out_pad, s, inv_s, nullptr, (float)((1 << w_bit) - 1),
+                                 zero_point ? 0 : 1, 0, st, nullptr, q, z, delta);
   return cudaGetLastError();
 }
 
@@ -370,6 +410,25 @@ cudaError_t launch_cand_quant(const __half *W, int64_t out, int64_t in, int64_t 
 // global store is contiguous.
 // ---------------------------------------------------------------------------
 constexpr int kPackRows = 64;
+
+// Status word of the calls that take no workspace (awq_quant_pack,
+// awq_search_clip_noalloc): one per device, zero at load, OR-ed by kernels,
+// read and cleared by the host (lib_status_read_clear).
+static __device__ DevStatus g_lib_status;
+
+cudaError_t lib_status_address(DevStatus **p) {
+  void *a = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&a, g_lib_status);
+  *p = static_cast<DevStatus *>(a);
+  return e;
+}
+
+cudaError_t lib_status_read_clear(DevStatus *h) {
+  cudaError_t e = cudaMemcpyFromSymbol(h, g_lib_status, sizeof(DevStatus));
+  if (e != cudaSuccess) return e;
+  const DevStatus zero = {};
+  return cudaMemcpyToSymbol(g_lib_status, &zero, sizeof(DevStatus));
+}
 
 __device__ __forceinline__ float clip_ratio(int c, int n_clip, float clip_min) {
   if (n_clip <= 1) return 1.0f;
@@ -443,19 +502,32 @@ __global__ void __launch_bounds__(256, 6) quant_pack_kernel(
       mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
     }
     if (!lane_ok) continue;  // past the last channel (its lanes form whole groups)
-    const float r32 = clip_idx ? ratios[clip_idx[o * groups + kg]] : 1.0f;
+    // an index past the clip grid is the caller's error: that group gets codes
+    // and zero 0 and a NaN scale, and the library status word records it
+    float r32 = 1.0f;
+    bool bad = false;
+    if (clip_idx) {
+      const int ci = clip_idx[o * groups + kg];
+      if (ci < n_clip)
+        r32 = ratios[ci];
+      else
+        bad = true;
+    }
     // four values per lane: the scalar quantiser (the batched fast path of the
     // candidate kernels costs more than it saves at this width)
     const GroupQ g = group_params(mx, mn, r32, qmax, sym != 0);
-    uchar4 c4;
-    c4.x = (uint8_t)quant_code(wt[0], g);
-    c4.y = (uint8_t)quant_code(wt[1], g);
-    c4.z = (uint8_t)quant_code(wt[2], g);
-    c4.w = (uint8_t)quant_code(wt[3], g);
+    uchar4 c4 = make_uchar4(0, 0, 0, 0);
+    if (!bad) {
+      c4.x = (uint8_t)quant_code(wt[0], g);
+      c4.y = (uint8_t)quant_code(wt[1], g);
+      c4.z = (uint8_t)quant_code(wt[2], g);
+      c4.w = (uint8_t)quant_code(wt[3], g);
+    }
     *reinterpret_cast<uchar4 *>(&codes[r][lane * 4]) = c4;
     if ((lane & (gl - 1)) == 0) {  // first lane of the group
-      zeros[r][gi] = (uint8_t)g.zero;
-      scales[kg * out + o] = __float2half_rn(g.delta);
+      zeros[r][gi] = bad ? (uint8_t)0 : (uint8_t)g.zero;
+      scales[kg * out + o] = bad ? __ushort_as_half((unsigned short)0x7E00u) : __float2half_rn(g.delta);
+      if (bad) dev_fail(&g_lib_status, kDevBadIndex, 0x4B0u);
     }
   }
   __syncthreads();

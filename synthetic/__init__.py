@@ -29,6 +29,8 @@ import torch
 
 __all__ = [
     "OutlierSpec",
+    "EDGE_PATTERNS",
+    "edge_layer",
     "heavy_tailed_activations",
     "gaussian_weight",
     "swiglu_activations",
@@ -199,6 +201,65 @@ def random_layer(T: int, d_in: int, d_out: int, seed: int,
     X = heavy_tailed_activations(T, d_in, outliers, seed)
     W = gaussian_weight(d_out, d_in, seed, std=w_std)
     return X, W
+
+
+# Weight-group patterns of edge_layer (name, description):
+EDGE_PATTERNS = (
+    ("normal", "N(0, 0.02)"),
+    ("pos_narrow", "0.5 + 0.001 U: one-signed, range far below the values"),
+    ("neg_narrow", "-0.25 - 0.0005 U: one-signed negative, narrow"),
+    ("pos_wide", "0.01 + 0.02 U: one-signed, range wider than the offset"),
+    ("const", "the constant 0.03"),
+    ("zero", "all zeros"),
+    ("const_pow2", "the constant -0.0625"),
+    ("tiny", "1e-4 N(0, 1): partly fp16 subnormals"),
+    ("spike", "N(0, 0.02) with one weight set to 0.3"),
+)
+
+
+def edge_layer(T: int, d_in: int, d_out: int, seed: int, group: int = 128
+               ) -> Tuple[torch.Tensor, torch.Tensor]:
+    """An (X, W) pair that reaches the quantiser's and the search's special
+    cases, for edge-case tests.
+
+    X is heavy_tailed_activations with dead channels: columns 0..2 are zero
+    (mean |x| = 0), columns group+1..group+3 (if present) are ~1e-5 (mean |x|
+    below 1e-4), and, when d_in >= 3 group, the whole group 2 is zero.
+    W has one pattern of EDGE_PATTERNS per (row o, group k), pattern number
+    (5 o + 3 k) mod 9, so every group column and every row meets several."""
+    X = heavy_tailed_activations(T, d_in, OutlierSpec(0.01, 20.0, 50.0), seed)
+    X[:, 0:3] = 0
+    if d_in >= 2 * group:
+        tiny = torch.randn((T, 3), generator=_gen(seed + 11)) * 1e-5
+        X[:, group + 1:group + 4] = tiny.to(torch.float16)
+    if d_in >= 3 * group:
+        X[:, 2 * group:3 * group] = 0
+    n_groups = d_in // group
+    W = torch.randn((d_out, d_in), generator=_gen(seed + 12)) * 0.02
+    u = torch.rand((d_out, d_in), generator=_gen(seed + 13))
+    z = torch.randn((d_out, d_in), generator=_gen(seed + 14))
+    pos = torch.randint(0, group, (d_out, n_groups), generator=_gen(seed + 15))
+    for o in range(d_out):
+        for k in range(n_groups):
+            sl = slice(k * group, (k + 1) * group)
+            p = EDGE_PATTERNS[(5 * o + 3 * k) % len(EDGE_PATTERNS)][0]
+            if p == "pos_narrow":
+                W[o, sl] = 0.5 + 0.001 * u[o, sl]
+            elif p == "neg_narrow":
+                W[o, sl] = -0.25 - 0.0005 * u[o, sl]
+            elif p == "pos_wide":
+                W[o, sl] = 0.01 + 0.02 * u[o, sl]
+            elif p == "const":
+                W[o, sl] = 0.03
+            elif p == "zero":
+                W[o, sl] = 0.0
+            elif p == "const_pow2":
+                W[o, sl] = -0.0625
+            elif p == "tiny":
+                W[o, sl] = 1e-4 * z[o, sl]
+            elif p == "spike":
+                W[o, k * group + int(pos[o, k])] = 0.3
+    return X, W.to(torch.float16)
 
 
 # ---------------------------------------------------------------------------

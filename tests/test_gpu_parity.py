@@ -188,9 +188,11 @@ def test_search_clip_parity(T, inn, out, w_bit, n_clip):
         check_selection(int(idx1[o, k]), E1[o, k], f"clip row {o} group {k}")
 
 
-def test_clip_hand_worked(golden):
-    """The hand-worked clip example, through the pack kernel with clip index 19."""
-    hdr, rows = golden("quant_group_clip.txt")
+@pytest.mark.parametrize("name", ["quant_group_clip.txt", "quant_group_clip_interior.txt"])
+def test_clip_hand_worked(golden, name):
+    """The hand-worked clip examples (ratio index 19, and the interior index 8
+    whose codes are all round-half-even ties), through the pack kernel."""
+    hdr, rows = golden(name)
     W = np.zeros((8, 128), dtype=np.float16)
     for r in rows:
         W[:, int(r[0])] = float(r[1])
@@ -270,6 +272,19 @@ def test_fold_inv_scale_bitwise(rows, cols):
     got = vd.cpu().numpy()
     got = got[:, 0] if cols == 1 else got
     assert np.array_equal(got.view(np.uint16), want.view(np.uint16))
+
+
+def test_fold_rounding_chain_hand_worked(golden):
+    """The fixture where RN16(RN32(v)/s) lands on an fp16 tie (two roundings)
+    and the single rounding or the reciprocal product would give the other
+    neighbour: the fold kernel gives the fixture's bits."""
+    hdr, _ = golden("fold_rounding.txt")
+    v = np.full((8, 4), int(hdr["v_hex"], 16), dtype=np.uint16).view(np.float16)
+    s = np.full(8, int(hdr["s_hex"], 16), dtype=np.uint32).view(np.float32)
+    vd = torch.from_numpy(v).cuda()
+    awq.awq_fold_inv_scale(vd, torch.from_numpy(s).cuda())
+    torch.cuda.synchronize()
+    assert np.all(vd.cpu().numpy().view(np.uint16) == int(hdr["folded_hex"], 16))
 
 
 def test_mlp_workload_sampled():

@@ -65,6 +65,58 @@ def test_w4a16_exact_integer_case():
     assert np.array_equal(Yg.astype(np.int64), want)
 
 
+def _random_packed(inn, out, group, rng, pow2_scales):
+    """qweight / qzeros / scales with random codes and zero points; scales
+    2^e (e in -4..2) or random fp16 values in [2^-8, 4)."""
+    q = rng.integers(0, 16, size=(out, inn)).astype(np.uint32)
+    z = rng.integers(0, 16, size=(out, inn // group)).astype(np.uint32)
+    qw = np.zeros((inn, out // 8), dtype=np.uint32)
+    qz = np.zeros((inn // group, out // 8), dtype=np.uint32)
+    for e in range(8):
+        qw |= q[e::8, :].T << np.uint32(4 * e)
+        qz |= z[e::8, :].T << np.uint32(4 * e)
+    if pow2_scales:
+        sc = np.exp2(rng.integers(-4, 3, size=(inn // group, out))).astype(np.float16)
+    else:
+        sc = np.exp2(rng.uniform(-8, 2, size=(inn // group, out))).astype(np.float16)
+    return qw.view(np.int32), qz.view(np.int32), sc
+
+
+@pytest.mark.parametrize("group", [128, 64, 32])
+def test_w4a16_exact_pow2_scales(group):
+    """Power-of-two scales, zero points across 0..15, integer X in [-3, 3]:
+    every dequantised weight (q - z) 2^e is exact, every product and every
+    fp32 partial sum is a multiple of 2^-4 below 2^20, so the fp32 sum is the
+    exact sum and Y = RN16 of it, bit for bit."""
+    rng = np.random.default_rng(group)
+    inn, out, T = 512, 288, 333
+    qw, qz, sc = _random_packed(inn, out, group, rng, pow2_scales=True)
+    X = rng.integers(-3, 4, size=(T, inn)).astype(np.float16)
+    Yg = _gpu_w4a16(torch.from_numpy(X), qw, qz, sc, awq.AwqConfig.make(group_size=group))
+    want = O.w4a16_matmul(X, qw, qz, sc, group).astype(np.float16)
+    assert np.array_equal(Yg.view(np.uint16), want.view(np.uint16))
+
+
+@pytest.mark.parametrize("group", [128, 32])
+def test_w4a16_dequantised_weights_bitwise(group):
+    """Any fp16 scale: with one-hot rows of X (row t has a single 1 at input
+    channel t), Y[t, o] is one dequantised weight, RN16((q - z) scale), so
+    the on-the-fly conversion (subtract the zero, multiply by the scale, one
+    fp16 rounding) is compared bit for bit with the oracle's dequant_packed."""
+    rng = np.random.default_rng(100 + group)
+    inn, out = 256, 160
+    qw, qz, sc = _random_packed(inn, out, group, rng, pow2_scales=False)
+    X = np.eye(inn, dtype=np.float16)
+    Yg = _gpu_w4a16(torch.from_numpy(X), qw, qz, sc, awq.AwqConfig.make(group_size=group))
+    Wd = O.dequant_packed(qw, qz, sc, group)  # [out, in] fp16
+    assert np.array_equal(Yg.view(np.uint16), Wd.T.view(np.uint16))
+    # the scales were not powers of two: the fp16 product did round somewhere
+    exact = (O.unpack_nibbles(qw).astype(np.float64) -
+             np.repeat(O.unpack_nibbles(qz).astype(np.float64), group, axis=1)) * \
+        np.repeat(sc.astype(np.float64).T, group, axis=1)
+    assert np.any(Wd.astype(np.float64) != exact)
+
+
 @pytest.mark.parametrize("T,inn,out,w_bit,group,zp", [
     (200, 384, 288, 4, 128, 1), (1, 512, 160, 3, 64, 1), (300, 256, 96, 4, 32, 1),
     (2000, 1024, 768, 4, 128, 1), (129, 640, 544, 3, 128, 0)])

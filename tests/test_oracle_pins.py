@@ -82,6 +82,7 @@ def test_scale_grid_closed_forms():
 # D4  quantiser
 # --------------------------------------------------------------------------
 HAND_WORKED = ["quant_group_int4.txt", "quant_group_int3.txt", "quant_group_clip.txt",
+               "quant_group_clip_interior.txt",
                "quant_group_sym_int4.txt", "quant_group_sym_int3.txt", "quant_group_sym_clip.txt"]
 
 
@@ -380,6 +381,55 @@ def test_clip_ratio_grid():
     r = O.clip_ratios(20, 0.5)
     assert r[0] == 1.0 and r[-1] == 0.5 and np.all(np.diff(r) < 0)
     assert list(O.clip_ratios(1, 0.5)) == [1.0]
+
+
+def _rn32_exact(x: Fraction) -> Fraction:
+    """Round-half-to-even of a positive rational to the fp32 grid (normal
+    range), in exact arithmetic."""
+    e = math.floor(math.log2(x))
+    while Fraction(2) ** e > x:
+        e -= 1
+    while Fraction(2) ** (e + 1) <= x:
+        e += 1
+    m = x / Fraction(2) ** (e - 23)
+    fl = m.numerator // m.denominator
+    rem = m - fl
+    if rem > Fraction(1, 2) or (rem == Fraction(1, 2) and fl % 2 == 1):
+        fl += 1
+    return fl * Fraction(2) ** (e - 23)
+
+
+@pytest.mark.parametrize("n_clip,clip_min", [(20, 0.5), (7, 0.5), (2, 0.5)])
+def test_clip_ratio_grid_closed_form(n_clip, clip_min):
+    """Every ratio of the grid, interior ones included, is the fp32 rounding
+    of the exact 1 - c (1 - clip_min)/(n_clip - 1) ("05 — AWQ" §4: ratios of
+    0.5 - 1.0).  At 20 ratios an fp32 evaluation of the formula, or an fp32
+    linspace, misses it at c = 8, 11, 15, 17 (one ulp)."""
+    r = O.clip_ratios(n_clip, clip_min).astype(np.float32)
+    cm = Fraction(float(np.float32(clip_min)))
+    for c in range(n_clip):
+        want = _rn32_exact(1 - c * (1 - cm) / (n_clip - 1))
+        assert Fraction(float(r[c])) == want, (c, float(r[c]), float(want))
+    if n_clip == 20:
+        lin = np.linspace(np.float32(1), np.float32(0.5), 20, dtype=np.float32)
+        f32 = np.float32(1) - np.arange(20, dtype=np.float32) * np.float32(0.5) / np.float32(19)
+        assert sorted(set(np.flatnonzero(lin != r)) | set(np.flatnonzero(f32 != r))) == [8, 11, 15, 17]
+
+
+def test_fold_rounding_chain_hand_worked(golden):
+    """The fold rounds the quotient to fp32, then to fp16; the fixture's value
+    sits where one rounding, or the product with a rounded reciprocal, gives
+    the other fp16 neighbour."""
+    hdr, _ = golden("fold_rounding.txt")
+    v = np.array([int(hdr["v_hex"], 16)], dtype=np.uint16).view(np.float16)
+    s = np.array([int(hdr["s_hex"], 16)], dtype=np.uint32).view(np.float32)
+    got = O.fold_inv_scale(v, s).view(np.uint16)[0]
+    assert got == int(hdr["folded_hex"], 16)
+    one = np.float16(Fraction(float(v[0])) / Fraction(float(s[0])))  # RN16 of the exact quotient
+    assert abs(Fraction(float(v[0])) / Fraction(float(s[0])) - Fraction(float(one))) < Fraction(1, 2 ** 14)
+    assert one.view(np.uint16) == int(hdr["one_rounding_hex"], 16)
+    rec = np.float16(np.float32(v[0]) * (np.float32(1) / s[0]))
+    assert rec.view(np.uint16) == int(hdr["reciprocal_hex"], 16)
 
 
 def test_clip_ratio_one_is_unclipped():
