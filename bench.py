@@ -11,8 +11,8 @@ GPU) every rank runs the same step on its own layer (independent seeds): weak
 scaling, no data-path collective.  Rank 0 prints one JSON line.
 
 --impl reference times the CPU oracle (the fp64 restatement of the method
-the tests check the CUDA path against) on the host cores, on a bounded
-sample of the same workload, extrapolated to ms per layer.
+the tests check the CUDA path against) on the host cores: each step is one
+whole layer of the same workload (about 15-20 s on 16 cores).
 """
 
 from __future__ import annotations
@@ -37,10 +37,42 @@ KERNELS_PER_STEP = {  # kernels this library launches per step (memsets excluded
     "act_stats": 2, "wmax": 1, "scale_grid": 1, "cand_quant": 1, "search_gemm": 1,
     "mse_argmin": 1, "gram_blocks": 2, "clip_eval": 1, "quant_pack": 1,
 }
-# DRAM bytes (read + write) of one search_gemm_kernel launch on this workload,
-# from a one-pass ncu capture (profiles/search_gemm_q_proj_4096.md); to be
-# set to None whenever that kernel changes until it is captured again.
-NCU_TRAFFIC_BYTES = 11_300_000_000 + 10_080_000
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one
+# search_gemm_kernel launch on this workload, from a one-pass ncu capture of
+# the command below, together with the SHA-256 of the kernel's sources at
+# capture time.  The figure is reported only while the sources still hash to
+# that digest; after any change to them the line carries traffic = null until
+# the kernel is captured again.
+NCU_TRAFFIC = {
+    "bytes": None,
+    "sources_sha256": None,
+    "command": ("ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none "
+                "-k regex:search_gemm -s 5 -c 1 python bench.py --steps 1 --warmup 5 "
+                "--no-cpu-baseline --no-gram-form --no-cached-form --no-w4a16"),
+}
+TRAFFIC_SOURCES = ("post_weight_quantization_awq_b200/csrc/search_gemm.cu",
+                   "post_weight_quantization_awq_b200/csrc/awq_device.cuh",
+                   "post_weight_quantization_awq_b200/csrc/awq_launch.h")
+
+
+def traffic_sources_digest() -> str:
+    """SHA-256 over the sources the scored-GEMM kernel is compiled from."""
+    import hashlib
+    h = hashlib.sha256()
+    for rel in TRAFFIC_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
+def ncu_traffic():
+    """(bytes per launch, note): the recorded capture if it describes the
+    kernel as built now, else (None, why)."""
+    if NCU_TRAFFIC["bytes"] is None:
+        return None, "not captured for the current kernel"
+    if NCU_TRAFFIC["sources_sha256"] != traffic_sources_digest():
+        return None, "kernel sources changed since the capture"
+    return NCU_TRAFFIC["bytes"], "ncu capture of the current kernel sources: " + NCU_TRAFFIC["command"]
 
 
 def load_peaks():
@@ -194,12 +226,13 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- oracle arm
-def oracle_layer_ms(X, W, wl, row_fraction: float):
-    """Times the CPU oracle on the workload with a sample of the output rows
-    and extrapolates to one full layer: phases whose cost does not depend on
-    the number of output rows (abar, X^T X, the block Grams) are timed in full,
-    the per-row phases (candidate quantisation and scoring, clip scoring,
-    packing) on round(row_fraction * out) rows and scaled by 1/row_fraction.
+def oracle_layer_ms(X, W, wl, row_fraction: float = 1.0):
+    """Times the CPU oracle on one layer of the workload: abar, X^T X, the
+    alpha search, the block Grams, the clip search and the packing, in that
+    order.  With row_fraction = 1 (the default) this is the whole layer, timed
+    as it runs; with row_fraction < 1 the per-row phases run on
+    round(row_fraction * out) rows and are scaled by 1/row_fraction (the
+    row-independent phases are still timed in full).
     Returns (ms per layer, sample description)."""
     import numpy as np
     from oracle import awq_oracle as O
@@ -231,10 +264,15 @@ def oracle_layer_ms(X, W, wl, row_fraction: float):
     scale = out / rows
     fixed = t["act_stats"] + t["gram"] + t.get("block_grams", 0.0)
     total = fixed + (t["search"] + t.get("clip", 0.0) + t["pack"]) * scale
-    sample = (f"oracle (numpy fp64, BLAS matmuls) on the full X [{Xn.shape[0]} x {Xn.shape[1]}] "
-              f"and {rows} of {out} output rows; abar, X^T X and the block Grams timed in full, the "
-              f"per-row phases (alpha search, clip search, packing) scaled by {scale:.0f}; "
-              f"phase seconds {json.dumps({k: round(v, 3) for k, v in t.items()})}")
+    phases = json.dumps({k: round(v, 3) for k, v in t.items()})
+    if rows == out:
+        sample = (f"oracle (numpy fp64, BLAS matmuls) on the whole layer, timed as it runs: "
+                  f"X [{Xn.shape[0]} x {Xn.shape[1]}], all {out} output rows; phase seconds {phases}")
+    else:
+        sample = (f"oracle (numpy fp64, BLAS matmuls) on the full X [{Xn.shape[0]} x {Xn.shape[1]}] "
+                  f"and {rows} of {out} output rows; abar, X^T X and the block Grams timed in full, "
+                  f"the per-row phases (alpha search, clip search, packing) scaled by {scale:.0f}; "
+                  f"phase seconds {phases}")
     return total * 1e3, sample
 
 
@@ -450,6 +488,7 @@ def run_awq(args):
     hbm_frac = {k: round(b / (kern[k][0] * 1e-3) / 1e9 / hbm, 3) for k, b in hbm_bytes.items()
                 if kern[k][0]}
     value = ms_step / world  # whole job: world layers per step
+    traffic = ncu_traffic()
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 3),
@@ -460,7 +499,7 @@ def run_awq(args):
         "roofline": {"kernel": "search_gemm", "bound": "tensor", "achieved": round(tflops, 1),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(tflops / peak, 3),
                      "frac_of_burst_peak": round(tflops / float(peaks["bf16_tflops"]), 3),
-                     "traffic": NCU_TRAFFIC_BYTES,
+                     "traffic": traffic[0], "traffic_note": traffic[1],
                      "peak_source": f"{src} bf16 dense {'sustained' if 'bf16_tflops_sustained' in peaks else 'burst'} "
                                     "(fp16 has the same nominal rate)",
                      "algorithmic_flops_per_launch": flops},
@@ -483,50 +522,81 @@ def run_decoder(args):
     """Times the layer-by-layer AWQ of the 32-layer Llama-2-7B-architecture
     decoder (128 x 512 calibration tokens): per layer the four groups' alpha
     searches, the folds, the clip searches and the packing.  The fp16 forward
-    that captures each layer's inputs is input synthesis and is not timed."""
+    that captures each layer's inputs is input synthesis and is not timed.
+    --steps = layers quantised by the whole job (at most 32).  With N GPUs the
+    layers split into N contiguous blocks (decoder.layer_block), one per rank,
+    with no collective on the data path: each rank runs the untimed fp16
+    forward up to its first layer, then quantises its block, each layer timed
+    with CUDA events; the job's time is the max over ranks of the summed layer
+    times (strong scaling: the layer count is fixed)."""
     import torch
     import post_weight_quantization_awq_b200 as awq
     from post_weight_quantization_awq_b200 import decoder
     from synthetic import DecoderSpec, decoder_embeddings, decoder_layer_forward, decoder_layer_weights
     world, rank, local = dist_env()
-    if world > 1:
-        raise SystemExit("--workload decoder runs on one GPU")
     torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = init_dist("nccl", world)
     spec = DecoderSpec()
     cfg = awq.AwqConfig.make(w_bit=4, n_alpha=20, n_clip=20, clip_min=0.5)
     layers = min(args.steps, spec.layers)
-    x = decoder_embeddings(spec, device="cuda")
+    block = decoder.layer_block(rank, world, layers)
+    x = decoder_embeddings(spec, device=dev)
+    with torch.no_grad():  # untimed: the fp16 forward up to this rank's first layer
+        for layer in range(block.start):
+            w = decoder_layer_weights(spec, layer, device=dev)
+            _, x = decoder_layer_forward(x, w, spec)
     ws = None
-    times = []
+    times, summaries = [], []
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    for layer in range(layers):
-        w = decoder_layer_weights(spec, layer, device="cuda")
-        caps, x_next = decoder_layer_forward(x, w, spec)
-        if ws is None:
-            ws = decoder.workspace_for_layer(caps, w, cfg)
-            for _ in range(args.warmup):  # warm-up on copies of layer 0
-                decoder.quantize_layer_groups(caps, {k: v.clone() for k, v in w.items()}, cfg, ws)
-        torch.cuda.synchronize()
-        e0.record()
-        decoder.quantize_layer_groups(caps, w, cfg, ws)
-        e1.record()
-        torch.cuda.synchronize()
-        times.append(e0.elapsed_time(e1))
-        x = x_next
-    flops = 2.0 * spec.seq * spec.n_seq * cfg.n_alpha * spec.hidden * (
+    barrier(dist, local)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        for layer in block:
+            w = decoder_layer_weights(spec, layer, device=dev)
+            caps, x_next = decoder_layer_forward(x, w, spec)
+            if ws is None:
+                ws = decoder.workspace_for_layer(caps, w, cfg)
+                for _ in range(args.warmup):  # warm-up on copies of the first layer
+                    decoder.quantize_layer_groups(caps, {k: v.clone() for k, v in w.items()}, cfg, ws)
+            torch.cuda.synchronize(dev)
+            e0.record()
+            res = decoder.quantize_layer_groups(caps, w, cfg, ws)
+            e1.record()
+            torch.cuda.synchronize(dev)
+            times.append(e0.elapsed_time(e1))
+            summaries.append(decoder.layer_summary(layer, res))
+            x = x_next
+    barrier(dist, local)
+    torch.cuda.synchronize(dev)
+    rank_ms = sum(times)
+    job_ms = max_over_ranks(rank_ms, dist)
+    all_layers = decoder.gather_summaries(summaries, dist)
+    if dist is not None:
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    flops_layer = 2.0 * spec.seq * spec.n_seq * cfg.n_alpha * spec.hidden * (
         3 * spec.hidden + spec.hidden + 2 * spec.ffn) + 2.0 * spec.seq * spec.n_seq * cfg.n_alpha * spec.ffn * spec.hidden
-    ms = statistics.mean(times)
+    value = job_ms / layers  # whole job: ms per layer
     print(json.dumps({
-        "metric": METRIC, "value": round(ms, 3), "unit": UNIT, "n_gpus": 1, "steps": layers,
-        "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": False,
-        "scaling": "weak", "vs_baseline": None, "dtype": "fp16",
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": layers,
+        "warmup": args.warmup, "ms_per_step": round(job_ms / max(1, len(block)), 3),
+        "higher_is_better": False, "scaling": "strong" if world > 1 else "weak",
+        "vs_baseline": None, "dtype": "fp16",
         "data": "synthetic (random-init decoder, random token ids, outlier embedding channels)",
         "config": {"workload": "llama2_7b_decoder_32_layers: hidden 4096, 32 heads, MLP 11008, "
                                "128 x 512 calibration tokens, four groups per layer (q|k|v, o, gate|up, "
                                "down), INT4 g128, 20 alphas + 20 clip ratios, folds, packed",
-                   "layers_timed": layers, "forward_capture": "untimed"},
-        "candidate_gemm_tflops": round(flops / (ms * 1e-3) / 1e12, 1),
-        "ms_per_layer_min_max": [round(min(times), 3), round(max(times), 3)],
+                   "layers": layers, "parallelism": f"layer blocks over {world} GPU(s)",
+                   "forward_capture": "untimed",
+                   "timing": "CUDA events around each layer's quantisation, summed per rank, "
+                             "max over ranks"},
+        "candidate_gemm_tflops": round(flops_layer * layers / (job_ms * 1e-3) / 1e12, 1),
+        "rank0_ms_per_layer_min_max": [round(min(times), 3), round(max(times), 3)] if times else None,
+        "clocks": clk.summary(),
+        "layers_summary": [{"layer": d["layer"], **{g: d[g]["best_idx"] for g in ("qkv", "o", "gate_up", "down")}}
+                           for d in all_layers],
     }), flush=True)
     return 0
 
@@ -537,8 +607,9 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=("awq", "reference"), default="awq")
-    ap.add_argument("--ref-row-fraction", type=float, default=0.125,
-                    help="share of output rows the oracle runs on (then scaled)")
+    ap.add_argument("--ref-row-fraction", type=float, default=1.0,
+                    help="share of output rows the oracle runs on (1 = the whole layer; "
+                         "below 1 the per-row phases are scaled up)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-gram-form", action="store_true",
                     help="skip the extra measurement of the Gram-form search")

@@ -96,8 +96,7 @@ enum { AWQ_SEARCH_DIRECT = 0, AWQ_SEARCH_GRAM = 1, AWQ_SEARCH_CACHED_Y = 2 };
 typedef struct {
   int32_t w_bit;      /* 3 or 4                                                  */
   int32_t group_size; /* 128 (the pages' g), or 32 / 64 ("AWQ and Activation-Aware
-                         Scaling", When it breaks, contrasts g = 32); must divide in;
-                         the clip search handles g = 128 only */
+                         Scaling", When it breaks, contrasts g = 32); must divide in */
   int32_t zero_point; /* 1 = asymmetric: step (max - min)/(2^b - 1), zero point
                          z = clamp(rne(-min/step), 0, 2^b - 1) ("05 — AWQ" §9
                          zero_point = True).  0 = symmetric, the scheme of
@@ -164,11 +163,13 @@ awq_status awq_search_scale(const void *X, int64_t T, int64_t in, int64_t ldx,
  * group's own output error over all tokens,
  *   E_okc = sum_t (sum_{j in k} X_tj (deq_c,oj / s_j - W_oj))^2
  *         = d^T (X_k^T X_k) d,
- * evaluated with an fp32 block Gram X_k^T X_k and fp32 quadratic forms.
+ * evaluated with an fp32 block Gram X_k^T X_k and fp32 quadratic forms (the
+ * Grams of 128-channel blocks, whose diagonal g x g blocks are the groups'
+ * when g = 32 or 64).
  *   s        device fp32 [in] (normally s_best); NULL means s = 1
  *   clip_idx device uint8 [out, in/g] (output)
  *   err      device fp32 [out, in/g, n_clip] (output, optional, may be NULL)
- * Requires cfg->n_clip >= 1. */
+ * Requires cfg->n_clip >= 1 and in % 128 == 0. */
 awq_status awq_search_clip(const void *X, int64_t T, int64_t in, int64_t ldx,
                            const void *W, int64_t out, const float *s,
                            const awq_config *cfg, void *ws, size_t ws_bytes,
@@ -192,7 +193,7 @@ awq_status awq_candidate_codes(const void *W, int64_t out, int64_t in, const dou
  * as its quantiser makes them (inspection form of "05 — AWQ" §4's optional
  * clipping):
  *   q device uint8 [out, n_clip, in]     codes of (row o, ratio c, channel j)
- *   z device uint8 [out, n_clip, in/128] zero points of (o, c, group k)
+ *   z device uint8 [out, n_clip, in/g]   zero points of (o, c, group k)
  * The search's own outputs (clip_idx, err) are those of awq_search_clip_grams. */
 awq_status awq_clip_candidate_codes(const void *W, int64_t out, int64_t in, const float *s,
                                     const float *G, const awq_config *cfg, void *ws,
@@ -293,9 +294,10 @@ awq_status awq_select_scale(const double *sse, int64_t T_total, int64_t in, int6
                             const double *abar, const awq_config *cfg, void *ws, size_t ws_bytes,
                             float *s_best, double *mse, int32_t *best_idx, awq_stream_t stream);
 
-/* Block Grams of these tokens, G[k] = X_k^T X_k for every group k of 128 input
- * channels: device fp32 [in/128][128][128] (output).  in % 128 == 0,
- * cfg->group_size == 128; workspace as awq_search_clip (the same size). */
+/* Block Grams of these tokens, G[k] = X_k^T X_k for every block k of 128 input
+ * channels (any cfg->group_size: groups of 32 or 64 are the diagonal blocks):
+ * device fp32 [in/128][128][128] (output).  in % 128 == 0; workspace as
+ * awq_search_clip (the same size). */
 awq_status awq_block_grams(const void *X, int64_t T, int64_t in, int64_t ldx, const awq_config *cfg,
                            void *ws, size_t ws_bytes, float *G, awq_stream_t stream);
 

@@ -131,6 +131,14 @@ awq_status check_shape(int64_t T, int64_t in, int64_t out, const awq_config *cfg
   return AWQ_OK;
 }
 
+// The clip search works on 128-channel blocks (their Grams hold every group
+// of 32, 64 or 128 channels of the block on the diagonal).
+awq_status check_clip_in(int64_t in) {
+  if (in % 128 != 0)
+    return fail(AWQ_ERR_UNSUPPORTED, "in=%lld: the clip search needs in %% 128 == 0", (long long)in);
+  return AWQ_OK;
+}
+
 awq_status check_x(const void *X, int64_t in, int64_t ldx) {
   if (!X) return fail(AWQ_ERR_INVALID_ARG, "X is NULL");
   if (!aligned(X, 16)) return fail(AWQ_ERR_INVALID_ARG, "X must be 16-byte aligned");
@@ -279,7 +287,7 @@ size_t awq_workspace_size(int64_t T, int64_t in, int64_t out, const awq_config *
   if (check_cfg(cfg) != AWQ_OK) return 0;
   if (check_shape(T, in, out, cfg) != AWQ_OK) return 0;
   size_t need = scale_layout(T, in, out, cfg).end;
-  if (cfg->n_clip > 0 && cfg->group_size == 128) {
+  if (cfg->n_clip > 0 && in % 128 == 0) {
     size_t c = clip_layout(T, in).end;
     if (c > need) need = c;
   }
@@ -500,9 +508,8 @@ awq_status awq_search_clip(const void *X, int64_t T, int64_t in, int64_t ldx, co
   awq_status st = check_cfg(cfg);
   if (st != AWQ_OK) return st;
   if (cfg->n_clip < 1) return fail(AWQ_ERR_INVALID_ARG, "n_clip=%d: clip search needs n_clip >= 1", cfg->n_clip);
-  if (cfg->group_size != 128)
-    return fail(AWQ_ERR_UNSUPPORTED, "group_size=%d: the clip search handles groups of 128", cfg->group_size);
   if ((st = check_shape(T, in, out, cfg)) != AWQ_OK) return st;
+  if ((st = check_clip_in(in)) != AWQ_OK) return st;
   if ((st = check_x(X, in, ldx)) != AWQ_OK) return st;
   if (!W || !aligned(W, 16)) return fail(AWQ_ERR_INVALID_ARG, "W is NULL or not 16-byte aligned");
   if (!clip_idx) return fail(AWQ_ERR_INVALID_ARG, "clip_idx is NULL");
@@ -538,8 +545,6 @@ awq_status awq_block_grams(const void *X, int64_t T, int64_t in, int64_t ldx, co
   g_err.clear();
   awq_status st = check_cfg(cfg);
   if (st != AWQ_OK) return st;
-  if (cfg->group_size != 128)
-    return fail(AWQ_ERR_UNSUPPORTED, "group_size=%d: block Grams of groups of 128 only", cfg->group_size);
   if (T < 1 || T > (int64_t(1) << 22)) return fail(AWQ_ERR_INVALID_ARG, "T=%lld (1..2^22)", (long long)T);
   if (in < 128 || in % 128 != 0 || in > (int64_t(1) << 20))
     return fail(AWQ_ERR_INVALID_ARG, "in=%lld must be a positive multiple of 128", (long long)in);
@@ -566,9 +571,8 @@ awq_status awq_search_clip_grams(const void *W, int64_t out, int64_t in, const f
   awq_status st = check_cfg(cfg);
   if (st != AWQ_OK) return st;
   if (cfg->n_clip < 1) return fail(AWQ_ERR_INVALID_ARG, "n_clip=%d: clip search needs n_clip >= 1", cfg->n_clip);
-  if (cfg->group_size != 128)
-    return fail(AWQ_ERR_UNSUPPORTED, "group_size=%d: the clip search handles groups of 128", cfg->group_size);
   if ((st = check_shape(1, in, out, cfg)) != AWQ_OK) return st;
+  if ((st = check_clip_in(in)) != AWQ_OK) return st;
   if (!W || !aligned(W, 16)) return fail(AWQ_ERR_INVALID_ARG, "W is NULL or not 16-byte aligned");
   if (!G || !aligned(G, 16)) return fail(AWQ_ERR_INVALID_ARG, "G is NULL or not 16-byte aligned");
   if (!clip_idx) return fail(AWQ_ERR_INVALID_ARG, "clip_idx is NULL");
@@ -629,9 +633,8 @@ awq_status awq_clip_candidate_codes(const void *W, int64_t out, int64_t in, cons
   awq_status st = check_cfg(cfg);
   if (st != AWQ_OK) return st;
   if (cfg->n_clip < 1) return fail(AWQ_ERR_INVALID_ARG, "n_clip=%d: clip search needs n_clip >= 1", cfg->n_clip);
-  if (cfg->group_size != 128)
-    return fail(AWQ_ERR_UNSUPPORTED, "group_size=%d: the clip search handles groups of 128", cfg->group_size);
   if ((st = check_shape(1, in, out, cfg)) != AWQ_OK) return st;
+  if ((st = check_clip_in(in)) != AWQ_OK) return st;
   if (!W || !aligned(W, 16)) return fail(AWQ_ERR_INVALID_ARG, "W is NULL or not 16-byte aligned");
   if (!G || !aligned(G, 16)) return fail(AWQ_ERR_INVALID_ARG, "G is NULL or not 16-byte aligned");
   if (!clip_idx || !q || !z) return fail(AWQ_ERR_INVALID_ARG, "clip_idx, q or z is NULL");
@@ -820,9 +823,8 @@ extern "C" awq_status awq_search_clip_noalloc(const void *X, int64_t T, int64_t 
   awq_status st = check_cfg(cfg);
   if (st != AWQ_OK) return st;
   if (cfg->n_clip < 1) return fail(AWQ_ERR_INVALID_ARG, "n_clip=%d: clip search needs n_clip >= 1", cfg->n_clip);
-  if (cfg->group_size != 128)
-    return fail(AWQ_ERR_UNSUPPORTED, "group_size=%d: the clip search handles groups of 128", cfg->group_size);
   if ((st = check_shape(T, in, out, cfg)) != AWQ_OK) return st;
+  if ((st = check_clip_in(in)) != AWQ_OK) return st;
   if (in > kNoAllocMaxIn)
     return fail(AWQ_ERR_INVALID_ARG,
                 "in=%lld exceeds the %lld input channels the allocation-free clip search's "

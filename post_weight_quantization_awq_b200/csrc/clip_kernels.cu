@@ -205,7 +205,8 @@ __global__ void gram_reduce_kernel(const float *__restrict__ partials, int n_chu
 cudaError_t launch_gram_blocks(const __half *X, int64_t T, int64_t in, int64_t ldx, int group,
                                int n_chunks, float *partials, float *Gout, DevStatus *st,
                                uint32_t max_polls, cudaStream_t stream) {
-  if (group != G) return cudaErrorInvalidValue;
+  (void)group;  // the block Grams are of 128-channel blocks whatever the quantisation group
+  if (in % G != 0) return cudaErrorInvalidValue;
   const int64_t n_groups = in / G;
   // chunks are whole multiples of GT tokens so that no TMA box straddles two
   // chunks; only the last chunk ends at T (rows past T read as zero)
@@ -265,7 +266,7 @@ struct __align__(16) ClipSmem {
   uint8_t b_lo[CT_OPND];
   float s[G], ar[G], r[G];  // s_i, r_i / s_i, r_i = sqrt(G_ii)
   int rexp[2][CT_MAXR];
-  float epart[2][128];
+  float epart[2][4][128];  // per buffer, per group of the block, per candidate
   float ratio[128];  // clip ratio of each index
   uint64_t a_full[2], a_empty[2], acc_full[2], acc_empty[2], mma_done;
   uint32_t tmem_base;
@@ -313,10 +314,16 @@ __device__ __forceinline__ float clip_ratio_f(int c, int n_clip, float clip_min)
 // flight: producers (warps 0-11, three per SM sub-partition) build tile t's
 // candidates while the MMA warp runs tile t-1 and the epilogue warps (13-16)
 // score and pick tile t-2.
+// GS: the quantisation group (32, 64 or 128 channels).  A CTA item is still a
+// 128-channel block of one row tile: for GS < 128 the block holds 128/GS
+// groups, G~ keeps only their diagonal GS x GS blocks (the group's own
+// output error, no cross-group terms), and the epilogue's dot products are
+// taken per GS-column segment, so one candidate row (row, ratio) scores that
+// ratio for every group of the block at once.
 // kCodes: the producers also store every candidate's codes q [out, n_clip, in]
-// and zero points z [out, n_clip, in/128] (the inspection form; the search
+// and zero points z [out, n_clip, in/GS] (the inspection form; the search
 // itself is unchanged).
-template <bool kCodes>
+template <int GS, bool kCodes>
 __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
     const __half *__restrict__ W, int64_t out, int64_t in, const float *__restrict__ s,
     const float *__restrict__ Gall, float qmax, int sym, int n_clip, float clip_min, int rows_per_tile,
@@ -327,12 +334,15 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
       (reinterpret_cast<uintptr_t>(csm_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   volatile int *abort_flag = &S.abort_flag;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int64_t n_groups = in / G;
+  constexpr int GPB = G / GS;        // quantisation groups per 128-channel block
+  constexpr int CPG = GS / 8;        // 8-channel chunks per group
+  const int64_t n_blocks = in / G;
+  const int64_t n_groups = in / GS;  // groups of the outputs clip_idx, err, cz
   const int R = rows_per_tile;
   const int64_t n_tiles = (out + R - 1) / R;
   // this CTA's share of the (group, row tile) items, group-major, so a CTA
   // meets at most a few groups and builds each G~ once
-  const int64_t n_items = n_groups * n_tiles;
+  const int64_t n_items = n_blocks * n_tiles;
   const int64_t item_begin = n_items * blockIdx.x / gridDim.x;
   const int64_t item_end = n_items * (blockIdx.x + 1) / gridDim.x;
 
@@ -431,8 +441,10 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
           const float gv[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
-            const float den = rj * S.r[64 * h + 8 * c + e];
-            v[e] = den > 0.0f ? gv[e] / den : 0.0f;
+            const int i = 64 * h + 8 * c + e;
+            const float den = rj * S.r[i];
+            // only the group's own block (every entry when GS = 128)
+            v[e] = (den > 0.0f && (i / GS) == (j / GS)) ? gv[e] / den : 0.0f;
           }
           split_store8(S.b_hi + h * CT_ATOM, S.b_lo + h * CT_ATOM, sw128_off(j, c), v);
         }
@@ -463,10 +475,13 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
           mn = fminf(mn, fminf(wt[h].x, wt[h].y));
           bmax = fmaxf(bmax, fmaxf(rv[2 * h] * fabsf(w2.x), rv[2 * h + 1] * fabsf(w2.y)));
         }
+        // the group's range over its CPG lanes, the row's bmax over all 16
 #pragma unroll
         for (int off = 8; off > 0; off >>= 1) {
-          mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-          mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+          if (off < CPG) {
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+          }
           bmax = fmaxf(bmax, __shfl_xor_sync(0xffffffffu, bmax, off));
         }
         // |d~_i| <= r_i |w_i| (+ rounding): keep 2 bmax 2^e <= 2^14
@@ -480,9 +495,10 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
         float2 ae[4];  // (r_i / s_i) 2^e, exact power-of-two scaling
 #pragma unroll
         for (int h = 0; h < 4; ++h) ae[h] = __fmul2_rn(make_float2(av[2 * h], av[2 * h + 1]), make_float2(sc, sc));
-        // ---- parameters of ratio sp + nsp * (lane % 16), computed once
+        // ---- GS = 128: parameters of ratio sp + nsp * (lane % 16), computed
+        // once and shared by shuffle; smaller groups compute their own below
         GroupQ gq;
-        {
+        if constexpr (GS == 128) {
           const int cl = sp + nsp * ch;
           gq = group_params(mx, mn, S.ratio[cl < n_clip ? cl : 0], qmax, sym != 0);
           // every quotient of the group stays below 63 in magnitude, which the
@@ -493,11 +509,21 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
         uint8_t *ahi = S.a_hi[b] + (ch >> 3) * CT_ATOM, *alo = S.a_lo[b] + (ch >> 3) * CT_ATOM;
 #pragma unroll 2
         for (int jc = 0; jc < cper; ++jc) {  // two ratios interleaved: more independent work
-          const float dl = __shfl_sync(0xffffffffu, gq.delta, jc, 16);
-          const float rc = __shfl_sync(0xffffffffu, gq.rcp, jc, 16);
-          const float hl = __shfl_sync(0xffffffffu, gq.half_lo, jc, 16);
-          const float zz = __shfl_sync(0xffffffffu, gq.zero, jc, 16);
           const int c = sp + nsp * jc;
+          float dl, rc, hl, zz;
+          if constexpr (GS == 128) {
+            dl = __shfl_sync(0xffffffffu, gq.delta, jc, 16);
+            rc = __shfl_sync(0xffffffffu, gq.rcp, jc, 16);
+            hl = __shfl_sync(0xffffffffu, gq.half_lo, jc, 16);
+            zz = __shfl_sync(0xffffffffu, gq.zero, jc, 16);
+          } else {
+            GroupQ g2 = group_params(mx, mn, S.ratio[c < n_clip ? c : 0], qmax, sym != 0);
+            if (!(fmaxf(fabsf(mx), fabsf(mn)) * g2.rcp < 63.0f)) g2.half_lo = -1.0f;
+            dl = g2.delta;
+            rc = g2.rcp;
+            hl = g2.half_lo;
+            zz = g2.zero;
+          }
           const bool store = live && c < n_clip;  // past n_clip: lane 0's ratio, not stored
           // (q - z) = clamp(rne(wt / delta), -z, qmax - z), proposed from the
           // approximate reciprocal and proven by the remainder
@@ -538,7 +564,7 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
               }
               *reinterpret_cast<uint2 *>(cq + (o * n_clip + c) * in + k * G + 8 * ch) =
                   make_uint2(cw[0], cw[1]);
-              if (ch == 0) cz[(o * n_clip + c) * n_groups + k] = (uint8_t)zz;
+              if (ch % CPG == 0) cz[(o * n_clip + c) * n_groups + k * GPB + ch / CPG] = (uint8_t)zz;
             }
           }
         }
@@ -612,7 +638,7 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
       // E = d~ . y over the 128 columns of this candidate's accumulator row
       float2 e2a = make_float2(0.0f, 0.0f), e2b = make_float2(0.0f, 0.0f);
 #pragma unroll 1
-      for (int cb = 0; cb < 4; ++cb) {
+      for (int cb = 0; cb < 4; ++cb) {  // 32 columns each; a group ends every GS / 32
         float y[32];
         tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(b * 128 + 32 * cb), y);
         tmem_ld_wait();
@@ -634,31 +660,38 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
               e2a = __ffma2_rn(__fadd2_rn(fh, fl), yy, e2a);
           }
         }
+        if (((cb + 1) * 32) % GS == 0) {  // this candidate's E for group cb * 32 / GS
+          S.epart[b][(cb * 32) / GS][p] = (e2a.x + e2b.x) + (e2a.y + e2b.y);
+          e2a = make_float2(0.0f, 0.0f);
+          e2b = make_float2(0.0f, 0.0f);
+        }
       }
-      const float e = (e2a.x + e2b.x) + (e2a.y + e2b.y);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.acc_empty[b]);
-      S.epart[b][p] = e;
-      // the argmin below needs only epart (this group's) and its row's
+      // the argmin below needs only epart (this block's) and its row's
       // exponent: take the exponent now and release A, the row data and the
-      // buffer to the producers as soon as every dot is done
-      const int rr = etid >> 2, part = etid & 3;
+      // buffer to the producers as soon as every dot is done.  TPP threads
+      // share one (row, group) pair.
+      constexpr int TPP = 4 / GPB;
+      const int pair = etid / TPP, part = etid % TPP;
+      const int rr = pair / GPB, kk = pair % GPB;
       const int rexp_row = S.rexp[b][rr];  // rr < 32
       named_bar(2, CW_NEPI * 32);
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.a_empty[b]);
-      // ---- per row: first clip index with the smallest E; four threads per
-      // row scan every fourth ratio, then combine (ties keep the lower index)
+      // ---- per (row, group): first clip index with the smallest E; the pair's
+      // threads scan every TPP-th ratio, then combine (ties keep the lower index)
       {
         const bool row_ok = rr < R && o0 + rr < out;
+        const int64_t gk = k * GPB + kk;  // group index along in
         float best = INFINITY;
         int bc = 1 << 30;
         if (row_ok) {
           const float unscale = ldexpf(1.0f, -2 * rexp_row);
-          for (int c = part; c < n_clip; c += 4) {
-            const float ev = S.epart[b][rr * n_clip + c] * unscale;
-            if (err) err[((o0 + rr) * n_groups + k) * n_clip + c] = ev;
+          for (int c = part; c < n_clip; c += TPP) {
+            const float ev = S.epart[b][kk][rr * n_clip + c] * unscale;
+            if (err) err[((o0 + rr) * n_groups + gk) * n_clip + c] = ev;
             if (ev < best) {
               best = ev;
               bc = c;
@@ -666,7 +699,7 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
           }
         }
 #pragma unroll
-        for (int off = 1; off < 4; off <<= 1) {
+        for (int off = 1; off < TPP; off <<= 1) {
           const float ob = __shfl_xor_sync(0xffffffffu, best, off);
           const int oc = __shfl_xor_sync(0xffffffffu, bc, off);
           if (ob < best || (ob == best && oc < bc)) {
@@ -674,7 +707,7 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
             bc = oc;
           }
         }
-        if (row_ok && part == 0) clip_idx[(o0 + rr) * n_groups + k] = (uint8_t)bc;
+        if (row_ok && part == 0) clip_idx[(o0 + rr) * n_groups + gk] = (uint8_t)bc;
       }
     }
   }
@@ -691,12 +724,15 @@ cudaError_t launch_clip_eval(const __half *W, int64_t out, int64_t in, const flo
                              float clip_min, uint8_t *clip_idx, float *err, DevStatus *st,
                              uint32_t max_polls, int num_sms, cudaStream_t stream, uint8_t *cq,
                              uint8_t *cz) {
-  if (group != G || n_clip < 1 || n_clip > 128) return cudaErrorInvalidValue;
+  if ((group != 32 && group != 64 && group != G) || in % G != 0 || n_clip < 1 || n_clip > 128)
+    return cudaErrorInvalidValue;
   int R = 128 / n_clip;
   if (R > CT_MAXR) R = CT_MAXR;
   const int64_t n_items = (in / G) * ((out + R - 1) / R);
   const int64_t ctas = i64min(num_sms, n_items);  // one CTA per SM (shared memory bound)
-  auto kern = cq ? clip_tc_kernel<true> : clip_tc_kernel<false>;
+  auto kern = group == 32   ? (cq ? clip_tc_kernel<32, true> : clip_tc_kernel<32, false>)
+              : group == 64 ? (cq ? clip_tc_kernel<64, true> : clip_tc_kernel<64, false>)
+                            : (cq ? clip_tc_kernel<128, true> : clip_tc_kernel<128, false>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kClipSmemBytes);
   if (e != cudaSuccess) return e;

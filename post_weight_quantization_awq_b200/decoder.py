@@ -102,3 +102,43 @@ def save_layer_checkpoint(path: str, layer: int, res: dict) -> None:
     tmp = path + ".tmp"
     torch.save(state, tmp)
     os.replace(tmp, path)
+
+
+# ---------------------------------------------------------------------------
+# Several GPUs: every layer's search is independent once its fp16 inputs are
+# known (the calibration states propagate through the unmodified layers), so
+# the layers split into contiguous blocks, one per rank, with no collective on
+# the data path.  A rank computes the fp16 forward up to its first layer
+# (input synthesis), then quantises its block.
+# ---------------------------------------------------------------------------
+def layer_block(rank: int, world: int, n_layers: int) -> range:
+    """Contiguous block of layers of `rank` out of `world`: the first
+    n_layers % world ranks take one layer more.  Blocks are disjoint, in
+    order, and cover range(n_layers)."""
+    if world < 1 or not 0 <= rank < world or n_layers < 0:
+        raise ValueError(f"rank {rank} of {world}, {n_layers} layers")
+    base, extra = divmod(n_layers, world)
+    start = rank * base + min(rank, extra)
+    return range(start, start + base + (1 if rank < extra else 0))
+
+
+def layer_summary(layer: int, res: dict) -> dict:
+    """What a rank reports about one quantised layer: per group the selected
+    alpha index, the smallest MSE and a checksum of the packed weights."""
+    out = {"layer": layer}
+    for g, _ in GROUPS:
+        r = res[g]
+        out[g] = {"best_idx": int(r["best_idx"].item()), "mse": float(r["mse"].min().item()),
+                  "qweight_sum": int(r["qweight"].to(torch.int64).sum().item())}
+    return out
+
+
+def gather_summaries(summaries: list, dist=None) -> list:
+    """All ranks' layer summaries, ordered by layer (an all_gather of Python
+    objects over the process group; a single process returns its own)."""
+    if dist is None:
+        return sorted(summaries, key=lambda d: d["layer"])
+    parts = [None] * dist.get_world_size()
+    dist.all_gather_object(parts, summaries)
+    return sorted((s for p in parts for s in p), key=lambda d: d["layer"])
+

@@ -75,7 +75,7 @@ class LibraryShardOps:
     def clip_from_grams(self, W, s_best, G, cfg, ws):
         import torch
         out, inn = W.shape
-        clip_idx = torch.empty((out, inn // 128), dtype=torch.uint8, device=self.device)
+        clip_idx = torch.empty((out, inn // cfg.group_size), dtype=torch.uint8, device=self.device)
         abi.awq_search_clip_grams(W, s_best, G, cfg, ws, clip_idx)
         abi.awq_device_status(ws)
         return clip_idx

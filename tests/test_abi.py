@@ -96,12 +96,16 @@ def test_errors_are_per_thread():
 
 
 def test_group_sizes_and_clip_limits():
-    """Groups of 32/64/128 for the search and packing; the clip search handles
-    128 only and says so before touching CUDA."""
+    """Groups of 32/64/128 for the search, the clip search and packing; the
+    clip search works on 128-channel blocks and says so before touching CUDA
+    when in is not a multiple of 128."""
     for g in (32, 64, 128):
         assert awq.awq_workspace_size(256, 512, 512, awq.AwqConfig.make(group_size=g)) > 0
+        # the clip search's block Grams are counted for every group size
+        assert (awq.awq_workspace_size(256, 512, 512, awq.AwqConfig.make(group_size=g, n_clip=20))
+                >= 256 + 4 * 128 * 128 * 4)
     cfg = awq.AwqConfig.make(group_size=64, n_clip=20)
-    st = abi.LIB.awq_search_clip(16, 256, 512, 512, 16, 512, None, ctypes.byref(cfg), 256, 1 << 30,
+    st = abi.LIB.awq_search_clip(16, 256, 576, 576, 16, 512, None, ctypes.byref(cfg), 256, 1 << 30,
                                  16, None, None)
     assert abi.STATUS[st] == "AWQ_ERR_UNSUPPORTED" and "128" in abi.last_error()
     # Gram form needs in % 128 == 0
@@ -135,9 +139,6 @@ def test_sharding_calls_check_their_arguments():
     assert S[st] == "AWQ_ERR_INVALID_ARG" and "sse" in abi.last_error()
     st = L.awq_select_scale(16, 256, 512, 512, 16, ctypes.byref(cfg), 256, 128, 16, 16, 16, None)
     assert S[st] == "AWQ_ERR_WORKSPACE"
-    st = L.awq_block_grams(16, 256, 512, 512, ctypes.byref(awq.AwqConfig.make(group_size=64)), 256, 1 << 30,
-                           16, None)
-    assert S[st] == "AWQ_ERR_UNSUPPORTED"
     st = L.awq_block_grams(16, 256, 320, 320, ctypes.byref(cfg), 256, 1 << 30, 16, None)
     assert S[st] == "AWQ_ERR_INVALID_ARG"
     st = L.awq_search_clip_grams(16, 512, 512, 16, 16, ctypes.byref(awq.AwqConfig.make(n_clip=0)),

@@ -89,9 +89,10 @@ def gpu_clip_codes(X, W, s, cfg):
     ws = awq.alloc_workspace(T, inn, out, cfg)
     G = torch.empty((inn // 128, 128, 128), dtype=torch.float32, device="cuda")
     awq.awq_block_grams(Xd, cfg, ws, G)
-    idx = torch.empty((out, inn // 128), dtype=torch.uint8, device="cuda")
+    g = cfg.group_size
+    idx = torch.empty((out, inn // g), dtype=torch.uint8, device="cuda")
     q = torch.empty((out, cfg.n_clip, inn), dtype=torch.uint8, device="cuda")
-    z = torch.empty((out, cfg.n_clip, inn // 128), dtype=torch.uint8, device="cuda")
+    z = torch.empty((out, cfg.n_clip, inn // g), dtype=torch.uint8, device="cuda")
     sd = None if s is None else torch.from_numpy(s).cuda()
     awq.awq_clip_candidate_codes(Wd, sd, G, cfg, ws, idx, None, q, z)
     awq.awq_device_status(ws)
@@ -107,31 +108,35 @@ def check_clip_codes(X, W, s, cfg):
     q, z = gpu_clip_codes(X, W, s, cfg)
     Wn = W.numpy()
     out, inn = Wn.shape
+    g = cfg.group_size
     r = O.clip_ratios(cfg.n_clip, cfg.clip_min).astype(np.float32)
     for c in range(cfg.n_clip):
-        ratio = np.full((out, inn // 128), r[c], dtype=np.float32)
-        ref = O.quantize_groups(Wn, s, 128, cfg.w_bit, ratio, zero_point=bool(cfg.zero_point))
+        ratio = np.full((out, inn // g), r[c], dtype=np.float32)
+        ref = O.quantize_groups(Wn, s, g, cfg.w_bit, ratio, zero_point=bool(cfg.zero_point))
         bad = np.argwhere(q[:, c, :] != ref["q"])
         assert bad.size == 0, (c, bad[:5])
         assert np.array_equal(z[:, c, :], ref["z"]), c
 
 
-@pytest.mark.parametrize("T,inn,out,w_bit,n_clip,zp", [
-    (300, 256, 40, 4, 20, 1), (64, 128, 8, 3, 7, 1), (500, 512, 96, 3, 20, 1), (100, 384, 24, 4, 1, 1),
-    (200, 256, 72, 4, 20, 0)])
-def test_clip_candidate_codes_bitwise(T, inn, out, w_bit, n_clip, zp):
+@pytest.mark.parametrize("T,inn,out,w_bit,n_clip,zp,group", [
+    (300, 256, 40, 4, 20, 1, 128), (64, 128, 8, 3, 7, 1, 128), (500, 512, 96, 3, 20, 1, 128),
+    (100, 384, 24, 4, 1, 1, 128), (200, 256, 72, 4, 20, 0, 128), (300, 256, 40, 4, 20, 1, 32),
+    (200, 384, 72, 3, 20, 0, 64)])
+def test_clip_candidate_codes_bitwise(T, inn, out, w_bit, n_clip, zp, group):
     X, W = random_layer(T, inn, out, seed=T + out + n_clip)
     s = O.scale_grid(O.act_stats(X.numpy()), O.alpha_grid(20))[10]
-    cfg = awq.AwqConfig.make(w_bit=w_bit, n_clip=n_clip, zero_point=zp)
+    cfg = awq.AwqConfig.make(w_bit=w_bit, n_clip=n_clip, zero_point=zp, group_size=group)
     check_clip_codes(X, W, s, cfg)
     check_clip_codes(X, W, None, cfg)
 
 
-@pytest.mark.parametrize("w_bit,zp", [(4, 1), (3, 1), (4, 0)])
-def test_clip_candidate_codes_edge_layer(w_bit, zp):
-    X, W = edge_layer(300, 4 * 128, 136, seed=40 + w_bit + zp)
+@pytest.mark.parametrize("w_bit,zp,group", [(4, 1, 128), (3, 1, 128), (4, 0, 128), (4, 1, 32),
+                                            (3, 0, 64)])
+def test_clip_candidate_codes_edge_layer(w_bit, zp, group):
+    X, W = edge_layer(300, 4 * 128, 136, seed=40 + w_bit + zp, group=group)
     s = O.scale_grid(O.act_stats(X.numpy()), O.alpha_grid(20))[15]
-    check_clip_codes(X, W, s, awq.AwqConfig.make(w_bit=w_bit, n_clip=20, zero_point=zp))
+    check_clip_codes(X, W, s, awq.AwqConfig.make(w_bit=w_bit, n_clip=20, zero_point=zp,
+                                                 group_size=group))
 
 
 def test_clip_candidate_codes_q_proj_rows():

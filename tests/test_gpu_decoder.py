@@ -1,7 +1,7 @@
 """The 32-layer Llama-2-7B-architecture decoder workload: layer-by-layer AWQ
 (four groups per layer, INT4 g128, 20 alphas + 20 clip ratios, folds, packing)
 with the calibration hidden states propagated through the fp16 layers, at
-16 x 512 calibration tokens.  On sampled layers every output is checked
+the workload's 128 x 512 = 65536 calibration tokens.  On sampled layers every output is checked
 against the CPU oracle: abar, s, folds and packing bit-exact on the whole
 layer; clip choices on sampled rows; and the alpha search, run through the
 same C ABI on sampled rows of the same captured inputs, against the oracle's
@@ -59,7 +59,7 @@ def _check_layer(caps, w_orig, w_folded, res, cfg, rng):
 
 def test_llama7b_decoder_layer_by_layer(tmp_path):
     need_cuda()
-    spec = DecoderSpec(n_seq=16)
+    spec = DecoderSpec()  # 128 sequences x 512 tokens
     cfg = awq.AwqConfig.make(w_bit=4, n_alpha=20, n_clip=20, clip_min=0.5)
     rng = np.random.default_rng(5)
     x = decoder_embeddings(spec, device="cuda")

@@ -442,20 +442,21 @@ def test_clip_ratio_one_is_unclipped():
         assert np.array_equal(a[key], b[key])
 
 
-@pytest.mark.parametrize("zp", [True, False])
-def test_clip_search_bruteforce_tokens(zp):
+@pytest.mark.parametrize("zp,group", [(True, 128), (False, 128), (True, 32), (False, 64)])
+def test_clip_search_bruteforce_tokens(zp, group):
     T, inn, out, nc = 40, 256, 8, 6
     X, W = random_layer(T, inn, out, seed=13)
     Xn, Wn = X.numpy(), W.numpy()
     s = O.scale_grid(O.act_stats(Xn), O.alpha_grid(20))[8]
-    idx, E = O.search_clip(Xn, Wn, s, 4, 128, nc, 0.5, zero_point=zp)
+    idx, E = O.search_clip(Xn, Wn, s, 4, group, nc, 0.5, zero_point=zp)
     r = O.clip_ratios(nc, 0.5).astype(np.float32)
     X64 = Xn.astype(np.float64)
+    ng = inn // group
     for c in range(nc):
-        qd = O.quantize_groups(Wn, s, 128, 4, np.full((out, 2), r[c], np.float32), zero_point=zp)
+        qd = O.quantize_groups(Wn, s, group, 4, np.full((out, ng), r[c], np.float32), zero_point=zp)
         for o in range(out):
-            for k in range(2):
-                sl = slice(128 * k, 128 * (k + 1))
+            for k in range(ng):
+                sl = slice(group * k, group * (k + 1))
                 d = qd["deq"][o, sl].astype(np.float64) / s[sl].astype(np.float64) - Wn[o, sl].astype(np.float64)
                 e = float(np.sum((X64[:, sl] @ d) ** 2))
                 assert E[o, k, c] == pytest.approx(e, rel=1e-10)
