@@ -20,7 +20,7 @@ Sources (web pages about AWQ, Lin et al.):
        [in/g, out/8] int32, scales fp16 [in/g, out], g = 128, 4.156 bits/weight;
        §9 (quant_config): zero_point = True, q_group_size = 128, w_bit = 4.
 
-Readings where the pages are silent (each also listed in the design notes):
+Readings where the pages are silent:
   * group-wise asymmetric min/max quantisation of g consecutive INPUT channels
     of one output row; zero point rounded and clamped to [0, 2^b - 1];
   * without a zero point ([P4] §9 zero_point = False; [P4] §3 describes the

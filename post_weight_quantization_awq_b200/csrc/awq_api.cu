@@ -96,6 +96,12 @@ struct ProfScope {
   }
 };
 
+// NVTX range around one C-ABI call (a no-op unless a profiler is attached)
+struct NvtxCall {
+  explicit NvtxCall(const char *name) { nvtxRangePushA(name); }
+  ~NvtxCall() { nvtxRangePop(); }
+};
+
 // ------------------------------------------------------------ validation
 awq_status check_cfg(const awq_config *cfg) {
   if (!cfg) return fail(AWQ_ERR_INVALID_ARG, "cfg is NULL");
@@ -280,6 +286,7 @@ const char *awq_last_error(void) { return g_err.c_str(); }
 
 size_t awq_workspace_size(int64_t T, int64_t in, int64_t out, const awq_config *cfg) {
   g_err.clear();
+  NvtxCall nvtx_call_(__func__);
   if (fault_mode() == Fault::kAlloc) {
     fail(AWQ_ERR_WORKSPACE, "injected allocation failure (AWQ_FAULT=alloc)");
     return 0;
@@ -297,6 +304,7 @@ size_t awq_workspace_size(int64_t T, int64_t in, int64_t out, const awq_config *
 awq_status awq_act_stats(const void *X, int64_t T, int64_t in, int64_t ldx, double *abar,
                          awq_stream_t stream) {
   g_err.clear();
+  NvtxCall nvtx_call_(__func__);
   if (T < 1 || T > (int64_t(1) << 22)) return fail(AWQ_ERR_INVALID_ARG, "T=%lld (1..2^22)", (long long)T);
   if (in < 8 || in % 8 != 0) return fail(AWQ_ERR_INVALID_ARG, "in=%lld must be a multiple of 8", (long long)in);
   awq_status st = check_x(X, in, ldx);
@@ -314,6 +322,7 @@ awq_status awq_act_stats(const void *X, int64_t T, int64_t in, int64_t ldx, doub
 awq_status awq_scale_grid(const double *abar, int64_t in, int32_t n_alpha, float *s,
                           awq_stream_t stream) {
   g_err.clear();
+  NvtxCall nvtx_call_(__func__);
   if (!abar || !s) return fail(AWQ_ERR_INVALID_ARG, "abar or s is NULL");
   if (in < 1 || in > (int64_t(1) << 24)) return fail(AWQ_ERR_INVALID_ARG, "in=%lld", (long long)in);
   if (n_alpha < 1 || n_alpha > 64) return fail(AWQ_ERR_INVALID_ARG, "n_alpha=%d (1..64)", n_alpha);
@@ -437,6 +446,7 @@ awq_status awq_search_scale(const void *X, int64_t T, int64_t in, int64_t ldx, c
                             size_t ws_bytes, float *s_best, double *mse, int32_t *best_idx,
                             awq_stream_t stream) {
   g_err.clear();
+  NvtxCall nvtx_call_(__func__);
   return search_scale_impl(X, T, in, ldx, W, out, abar, cfg, ws, ws_bytes, s_best, mse, best_idx,
                            nullptr, stream);
 }
@@ -445,6 +455,7 @@ awq_status awq_search_scale_sse(const void *X, int64_t T, int64_t in, int64_t ld
                                 int64_t out, const double *abar, const awq_config *cfg, void *ws,
                                 size_t ws_bytes, double *sse, awq_stream_t stream) {
   g_err.clear();
+  NvtxCall nvtx_call_(__func__);
   if (!sse) return fail(AWQ_ERR_INVALID_ARG, "sse is NULL");
   return search_scale_impl(X, T, in, ldx, W, out, abar, cfg, ws, ws_bytes, nullptr, nullptr, nullptr,
                            sse, stream);
@@ -454,6 +465,7 @@ awq_status awq_select_scale(const double *sse, int64_t T_total, int64_t in, int6
                             const double *abar, const awq_config *cfg, void *ws, size_t ws_bytes,
                             float *s_best, double *mse, int32_t *best_idx, awq_stream_t stream) {
   g_err.clear();
+  NvtxCall nvtx_call_(__func__);
   awq_status st = check_cfg(cfg);
   if (st != AWQ_OK) return st;
   if ((st = check_shape(T_total, in, out, cfg)) != AWQ_OK) return st;
@@ -475,6 +487,7 @@ awq_status awq_select_scale(const double *sse, int64_t T_total, int64_t in, int6
 awq_status awq_act_sums(const void *X, int64_t T, int64_t in, int64_t ldx, int64_t *sums,
                         awq_stream_t stream) {
   g_err.clear();
+  NvtxCall nvtx_call_(__func__);
   if (T < 1 || T > (int64_t(1) << 22)) return fail(AWQ_ERR_INVALID_ARG, "T=%lld (1..2^22)", (long long)T);
   if (in < 8 || in % 8 != 0) return fail(AWQ_ERR_INVALID_ARG, "in=%lld must be a multiple of 8", (long long)in);
   awq_status st = check_x(X, in, ldx);
@@ -491,6 +504,7 @@ awq_status awq_act_sums(const void *X, int64_t T, int64_t in, int64_t ldx, int64
 awq_status awq_act_stats_finish(const int64_t *sums, int64_t T_total, int64_t in, double *abar,
                                 awq_stream_t stream) {
   g_err.clear();
+  NvtxCall nvtx_call_(__func__);
   if (T_total < 1 || T_total > (int64_t(1) << 22))
     return fail(AWQ_ERR_INVALID_ARG, "T_total=%lld (1..2^22)", (long long)T_total);
   if (in < 1) return fail(AWQ_ERR_INVALID_ARG, "in=%lld", (long long)in);
@@ -505,6 +519,7 @@ awq_status awq_search_clip(const void *X, int64_t T, int64_t in, int64_t ldx, co
                            int64_t out, const float *s, const awq_config *cfg, void *ws,
                            size_t ws_bytes, uint8_t *clip_idx, float *err, awq_stream_t stream) {
   g_err.clear();
+  NvtxCall nvtx_call_(__func__);
   awq_status st = check_cfg(cfg);
   if (st != AWQ_OK) return st;
   if (cfg->n_clip < 1) return fail(AWQ_ERR_INVALID_ARG, "n_clip=%d: clip search needs n_clip >= 1", cfg->n_clip);
@@ -543,6 +558,7 @@ awq_status awq_search_clip(const void *X, int64_t T, int64_t in, int64_t ldx, co
 awq_status awq_block_grams(const void *X, int64_t T, int64_t in, int64_t ldx, const awq_config *cfg,
                            void *ws, size_t ws_bytes, float *G, awq_stream_t stream) {
   g_err.clear();
+  NvtxCall nvtx_call_(__func__);
   awq_status st = check_cfg(cfg);
   if (st != AWQ_OK) return st;
   if (T < 1 || T > (int64_t(1) << 22)) return fail(AWQ_ERR_INVALID_ARG, "T=%lld (1..2^22)", (long long)T);
@@ -568,6 +584,7 @@ awq_status awq_search_clip_grams(const void *W, int64_t out, int64_t in, const f
                                  const float *G, const awq_config *cfg, void *ws, size_t ws_bytes,
                                  uint8_t *clip_idx, float *err, awq_stream_t stream) {
   g_err.clear();
+  NvtxCall nvtx_call_(__func__);
   awq_status st = check_cfg(cfg);
   if (st != AWQ_OK) return st;
   if (cfg->n_clip < 1) return fail(AWQ_ERR_INVALID_ARG, "n_clip=%d: clip search needs n_clip >= 1", cfg->n_clip);
@@ -594,6 +611,7 @@ awq_status awq_candidate_codes(const void *W, int64_t out, int64_t in, const dou
                                const awq_config *cfg, void *ws, size_t ws_bytes, uint8_t *q,
                                uint8_t *z, float *delta, awq_stream_t stream) {
   g_err.clear();
+  NvtxCall nvtx_call_(__func__);
   awq_status st = check_cfg(cfg);
   if (st != AWQ_OK) return st;
   if ((st = check_shape(1, in, out, cfg)) != AWQ_OK) return st;
@@ -630,6 +648,7 @@ awq_status awq_clip_candidate_codes(const void *W, int64_t out, int64_t in, cons
                                     size_t ws_bytes, uint8_t *clip_idx, float *err, uint8_t *q,
                                     uint8_t *z, awq_stream_t stream) {
   g_err.clear();
+  NvtxCall nvtx_call_(__func__);
   awq_status st = check_cfg(cfg);
   if (st != AWQ_OK) return st;
   if (cfg->n_clip < 1) return fail(AWQ_ERR_INVALID_ARG, "n_clip=%d: clip search needs n_clip >= 1", cfg->n_clip);
@@ -658,6 +677,7 @@ awq_status awq_quant_pack(const void *W, int64_t out, int64_t in, const float *s
                           const uint8_t *clip_idx, const awq_config *cfg, int32_t *qweight,
                           int32_t *qzeros, void *scales, awq_stream_t stream) {
   g_err.clear();
+  NvtxCall nvtx_call_(__func__);
   awq_status st = check_cfg(cfg);
   if (st != AWQ_OK) return st;
   if ((st = check_shape(1, in, out, cfg)) != AWQ_OK) return st;
@@ -683,6 +703,7 @@ awq_status awq_w4a16_gemm(const void *X, int64_t T, int64_t in, int64_t ldx, con
                           const awq_config *cfg, void *Y, int64_t ldy, void *ws, size_t ws_bytes,
                           awq_stream_t stream) {
   g_err.clear();
+  NvtxCall nvtx_call_(__func__);
   awq_status st = check_cfg(cfg);
   if (st != AWQ_OK) return st;
   if ((st = check_shape(T, in, out, cfg)) != AWQ_OK) return st;
@@ -711,6 +732,7 @@ awq_status awq_w4a16_gemm(const void *X, int64_t T, int64_t in, int64_t ldx, con
 awq_status awq_fold_inv_scale(void *v, int64_t rows, int64_t cols, const float *s,
                               awq_stream_t stream) {
   g_err.clear();
+  NvtxCall nvtx_call_(__func__);
   if (!v || !s) return fail(AWQ_ERR_INVALID_ARG, "v or s is NULL");
   if (rows < 1 || cols < 1) return fail(AWQ_ERR_INVALID_ARG, "rows=%lld cols=%lld", (long long)rows, (long long)cols);
   AWQ_LAUNCH_GATE();
@@ -722,6 +744,7 @@ awq_status awq_fold_inv_scale(void *v, int64_t rows, int64_t cols, const float *
 
 awq_status awq_device_status(void *ws, awq_stream_t stream) {
   g_err.clear();
+  NvtxCall nvtx_call_(__func__);
   if (ws && !aligned(ws, 256)) return fail(AWQ_ERR_WORKSPACE, "workspace is misaligned");
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   AWQ_TRY_CUDA(cudaStreamSynchronize(cs), "stream synchronize");
@@ -750,6 +773,7 @@ awq_status awq_profile_enable(int32_t on) {
 
 awq_status awq_profile_read(const char *name, double *total_ms, int64_t *launches) {
   g_err.clear();
+  NvtxCall nvtx_call_(__func__);
   if (!name || !total_ms || !launches) return fail(AWQ_ERR_INVALID_ARG, "NULL argument");
   std::lock_guard<std::mutex> lk(g_prof_mu);
   double tot = 0.0;
@@ -820,6 +844,7 @@ extern "C" awq_status awq_search_clip_noalloc(const void *X, int64_t T, int64_t 
                                               const awq_config *cfg, uint8_t *clip_idx, float *err,
                                               awq_stream_t stream) {
   g_err.clear();
+  NvtxCall nvtx_call_(__func__);
   awq_status st = check_cfg(cfg);
   if (st != AWQ_OK) return st;
   if (cfg->n_clip < 1) return fail(AWQ_ERR_INVALID_ARG, "n_clip=%d: clip search needs n_clip >= 1", cfg->n_clip);

@@ -138,6 +138,19 @@ __device__ __forceinline__ void quant_qz_pairs(const float2 (&wt)[NP], const Gro
     qz[h] = make_float2(fminf(fmaxf(qz[h].x, lo), hi), fminf(fmaxf(qz[h].y, lo), hi));
 }
 
+// Three-input max / min (one instruction on sm_100a; same NaN rule as fmaxf).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+__device__ __forceinline__ float fmin3(float a, float b, float c) {
+  float r;
+  asm("min.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
 // the group check of quant_qz_pairs: every |wt| <= max(|mx|, |mn|)
 __device__ __forceinline__ void fast_path_check(GroupQ &g, float mx, float mn) {
   if (!(fmaxf(fabsf(mx), fabsf(mn)) * g.rcp < 63.0f)) g.half_lo = -1.0f;

@@ -251,9 +251,67 @@ cudaError_t launch_wmax(const __half *W, int64_t n, int64_t in, const float *r, 
 // candidate are zero.
 // A block covers one candidate, 64 rows and a slab of 256 channels: lane l
 // owns channels 8l..8l+7 of the slab (16-byte loads and stores) and keeps
-// their s and 1/s in registers while its warp walks 8 of the 64 rows.
+// their s and 1/s in registers; each warp holds 8 rows in registers, reduces
+// their 8 group ranges together (a transposing butterfly: every lane ends
+// with whole ranges of its own rows), computes each group's step and zero
+// point on one lane instead of all of its lanes, and quantises the rows with
+// the parameters taken by shuffle.
 // ---------------------------------------------------------------------------
 constexpr int kCandRows = 64;
+constexpr int kCandWarpRows = 8;  // rows per warp: 8 warps x 8 rows
+
+// Transposing butterfly for the group ranges of N rows over the 2 * OFF lanes
+// of a group: each round exchanges half of the rows a lane carries with its
+// partner (xor OFF) and keeps the max / min of the other half, so the rows
+// carried halve while the lanes reduced over double; once one row is left the
+// rounds are plain butterflies.  Lane l ends with rows held_by_lane / held_at.
+template <int N, int OFF>
+__device__ __forceinline__ void transpose_reduce(float (&mx)[kCandWarpRows], float (&mn)[kCandWarpRows],
+                                                 int lane) {
+  if constexpr (OFF >= 1) {
+    if constexpr (N > 1) {
+      const bool up = (lane & OFF) != 0;
+#pragma unroll
+      for (int i = 0; i < N / 2; ++i) {
+        const float sx = up ? mx[i] : mx[i + N / 2], sn = up ? mn[i] : mn[i + N / 2];
+        const float kx = up ? mx[i + N / 2] : mx[i], kn = up ? mn[i + N / 2] : mn[i];
+        mx[i] = fmaxf(kx, __shfl_xor_sync(0xffffffffu, sx, OFF));
+        mn[i] = fminf(kn, __shfl_xor_sync(0xffffffffu, sn, OFF));
+      }
+      transpose_reduce<N / 2, OFF / 2>(mx, mn, lane);
+    } else {
+      mx[0] = fmaxf(mx[0], __shfl_xor_sync(0xffffffffu, mx[0], OFF));
+      mn[0] = fminf(mn[0], __shfl_xor_sync(0xffffffffu, mn[0], OFF));
+      transpose_reduce<1, OFF / 2>(mx, mn, lane);
+    }
+  }
+}
+
+// After transpose_reduce<N, L/2> over groups of L lanes: the lane (within the
+// group) and the element that hold row r.  Round k (OFF = L/2, L/4, ...)
+// keeps the upper half of the N_k rows on lanes with bit OFF set.
+template <int L, int N>
+__device__ __forceinline__ constexpr int held_by_lane(int r) {
+  int lane = 0, n = N, base = 0;
+  for (int off = L / 2; off >= 1 && n > 1; off /= 2) {
+    if (r - base >= n / 2) {
+      lane |= off;
+      base += n / 2;
+    }
+    n /= 2;
+  }
+  return lane;
+}
+
+template <int L, int N>
+__device__ __forceinline__ constexpr int held_at(int r) {
+  int n = N, base = 0;
+  for (int off = L / 2; off >= 1 && n > 1; off /= 2) {
+    if (r - base >= n / 2) base += n / 2;
+    n /= 2;
+  }
+  return r - base;
+}
 
 // kCodes: instead of the B operand, the same candidates' codes q [n_alpha,
 // out, in], zero points z and steps delta [n_alpha, out, in/group] (delta of
@@ -310,55 +368,112 @@ __global__ void __launch_bounds__(256) cand_quant_kernel(
       iv[h] = make_float2(1.0f, 1.0f);
     }
   }
-#pragma unroll 2
-  for (int r = warp; r < kCandRows; r += 8) {
-    const int64_t o = o0 + r;
-    const bool live = j_ok && o < out;
-    uint4 wv = make_uint4(0u, 0u, 0u, 0u);
-    if (live) wv = __ldg(reinterpret_cast<const uint4 *>(W + o * in + j0));
-    const uint32_t wr[4] = {wv.x, wv.y, wv.z, wv.w};
-    float2 wt[4];
-    float mx = -INFINITY, mn = INFINITY;
+  // ---- pass 1: this warp's 8 rows (o0 + 8 warp .. + 7) into registers, and
+  // this lane's share of each row's group range
+  uint4 wv[kCandWarpRows];
+  float mx[kCandWarpRows], mn[kCandWarpRows];
+  const int64_t orow = o0 + (int64_t)warp * kCandWarpRows;
+#pragma unroll
+  for (int r = 0; r < kCandWarpRows; ++r) {
+    const bool live = j_ok && orow + r < out;
+    wv[r] = live ? __ldg(reinterpret_cast<const uint4 *>(W + (orow + r) * in + j0))
+                 : make_uint4(0u, 0u, 0u, 0u);
+  }
+#pragma unroll
+  for (int r = 0; r < kCandWarpRows; ++r) {
+    const uint32_t wr[4] = {wv[r].x, wv[r].y, wv[r].z, wv[r].w};
+    float m = -INFINITY, n = INFINITY;
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+      const float2 t = __fmul2_rn(sk[h], __half22float2(*reinterpret_cast<const __half2 *>(&wr[h])));
+      m = fmax3(m, t.x, t.y);
+      n = fmin3(n, t.x, t.y);
+    }
+    mx[r] = m;
+    mn[r] = n;
+  }
+  // ---- whole-group ranges: a transposing butterfly over the group's lanes
+  // leaves each lane kCandWarpRows / lanes rows (one row, on two lanes, when
+  // lanes = 16), and each lane computes the step, zero point, fast-path bound
+  // and clamp need of its rows once
+  transpose_reduce<kCandWarpRows, lanes / 2>(mx, mn, lane);
+  constexpr int kHeld = kCandWarpRows >= lanes ? kCandWarpRows / lanes : 1;
+  float pd[kHeld], pr[kHeld], ph[kHeld];
+  int pz[kHeld];
+#pragma unroll
+  for (int i = 0; i < kHeld; ++i) {
+    GroupQ g = group_params(mx[i], mn[i], 1.0f, qmax, sym != 0, guard);
+    fast_path_check(g, mx[i], mn[i]);
+    // every code of the group lies between those of its extremes (the
+    // quantiser is monotonic): the clamp is needed only if one leaves [0, qmax]
+    const float qhi = __fadd_rn(round_quotient(mx[i], g), g.zero);
+    const float qlo = __fadd_rn(round_quotient(mn[i], g), g.zero);
+    const bool clamp = !(qlo >= 0.0f && qhi <= g.qmax);
+    pd[i] = g.delta;
+    pr[i] = g.rcp;
+    ph[i] = g.half_lo;
+    pz[i] = (int)g.zero | (clamp ? 256 : 0);
+  }
+  // ---- pass 2: per row, the group's parameters from the lane that holds
+  // them, then codes proposed by the approximate reciprocal (one FMA rounds
+  // the product to an integer), proven by the remainder test, decided by the
+  // correctly rounded division otherwise; the clamp only where needed
+  const float2 M = make_float2(12582912.0f, 12582912.0f);  // 1.5 2^23
+#pragma unroll
+  for (int r = 0; r < kCandWarpRows; ++r) {
+    const int src = held_by_lane<lanes, kCandWarpRows>(r), el = held_at<lanes, kCandWarpRows>(r);
+    const float dl = __shfl_sync(0xffffffffu, pd[el], src, lanes);
+    const float rc = __shfl_sync(0xffffffffu, pr[el], src, lanes);
+    const float hl = __shfl_sync(0xffffffffu, ph[el], src, lanes);
+    const int zf = __shfl_sync(0xffffffffu, pz[el], src, lanes);
+    const float zero = (float)(zf & 255);
+    const int64_t o = orow + r;
+    const uint32_t wr[4] = {wv[r].x, wv[r].y, wv[r].z, wv[r].w};
+    float2 wt[4], qz[4];
+    float rmax = 0.0f;
 #pragma unroll
     for (int h = 0; h < 4; ++h) {
       wt[h] = __fmul2_rn(sk[h], __half22float2(*reinterpret_cast<const __half2 *>(&wr[h])));
-      mx = fmaxf(mx, fmaxf(wt[h].x, wt[h].y));
-      mn = fminf(mn, fminf(wt[h].x, wt[h].y));
+      qz[h] = __fadd2_rn(__ffma2_rn(wt[h], make_float2(rc, rc), M), make_float2(-M.x, -M.y));
+      const float2 rem = __ffma2_rn(make_float2(-qz[h].x, -qz[h].y), make_float2(dl, dl), wt[h]);
+      rmax = fmax3(rmax, fabsf(rem.x), fabsf(rem.y));
     }
+    if (!(rmax < hl)) {
 #pragma unroll
-    for (int off = lanes >> 1; off > 0; off >>= 1) {
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
+      for (int h = 0; h < 4; ++h)
+        qz[h] = make_float2(rintf(__fdiv_rn(wt[h].x, dl)), rintf(__fdiv_rn(wt[h].y, dl)));
     }
-    GroupQ g = group_params(mx, mn, 1.0f, qmax, sym != 0, guard);
-    fast_path_check(g, mx, mn);
-    float2 qz[4];
-    quant_qz_pairs<4>(wt, g, qz);
+    if (zf & 256) {
+      const float lo = -zero, hi = qmax - zero;  // exact (small integers)
+#pragma unroll
+      for (int h = 0; h < 4; ++h)
+        qz[h] = make_float2(fminf(fmaxf(qz[h].x, lo), hi), fminf(fmaxf(qz[h].y, lo), hi));
+    }
     if constexpr (kCodes) {
-      if (live) {
-        uint32_t b[2] = {0u, 0u};
+      if (j_ok && o < out) {
+        uint32_t bq[2] = {0u, 0u};
 #pragma unroll
         for (int h = 0; h < 4; ++h) {
           // q = (q - z) + z, small exact integers in [0, qmax]
-          b[h >> 1] |= (uint32_t)__fadd_rn(qz[h].x, g.zero) << (16 * (h & 1));
-          b[h >> 1] |= (uint32_t)__fadd_rn(qz[h].y, g.zero) << (16 * (h & 1) + 8);
+          bq[h >> 1] |= (uint32_t)__fadd_rn(qz[h].x, zero) << (16 * (h & 1));
+          bq[h >> 1] |= (uint32_t)__fadd_rn(qz[h].y, zero) << (16 * (h & 1) + 8);
         }
-        *reinterpret_cast<uint2 *>(cq + ((int64_t)a * out + o) * in + j0) = make_uint2(b[0], b[1]);
+        *reinterpret_cast<uint2 *>(cq + ((int64_t)a * out + o) * in + j0) = make_uint2(bq[0], bq[1]);
         if ((lane & (lanes - 1)) == 0) {
           const int64_t gi = ((int64_t)a * out + o) * (in / group) + j0 / group;
-          cz[gi] = (uint8_t)g.zero;
-          cdelta[gi] = ldexpf(g.delta, -k);
+          cz[gi] = (uint8_t)zero;
+          cdelta[gi] = ldexpf(dl, -k);
         }
       }
       continue;
     }
-    const float2 dl = make_float2(g.delta, g.delta);
+    const float2 dl2 = make_float2(dl, dl);
     uint32_t packed[4];
 #pragma unroll
     for (int h = 0; h < 4; ++h) {
       // error form: (deq - s w) 2^k (r / s); weights only: deq / s
-      const float2 t = weights_only ? __fmul2_rn(qz[h], dl)
-                                    : __ffma2_rn(qz[h], dl, make_float2(-wt[h].x, -wt[h].y));
+      const float2 t = weights_only ? __fmul2_rn(qz[h], dl2)
+                                    : __ffma2_rn(qz[h], dl2, make_float2(-wt[h].x, -wt[h].y));
       // rows past `out` and channels past `in` hold w = 0, which gives 0 here
       const float2 d2 = __fmul2_rn(t, iv[h]);
       const __half2 hv = __floats2half2_rn(d2.x, d2.y);

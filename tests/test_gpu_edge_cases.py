@@ -152,12 +152,12 @@ def test_injected_nonfinite_in_token_sharded_selection(monkeypatch):
     mse = torch.empty(20, dtype=torch.float64, device="cuda")
     best = torch.empty(1, dtype=torch.int32, device="cuda")
     monkeypatch.setenv("AWQ_FAULT", "nonfinite")
-    awq.awq_select_scale(sse, 1000, 512, 264, abar, cfg, ws, s_best, mse, best)
+    awq.awq_select_scale(sse, 1000, 264, abar, cfg, ws, s_best, mse, best)
     with pytest.raises(awq.AwqError) as ei:
         awq.awq_device_status(ws)
     assert ei.value.status_name == "AWQ_ERR_NONFINITE"
     monkeypatch.delenv("AWQ_FAULT")
-    awq.awq_select_scale(sse, 1000, 512, 264, abar, cfg, ws, s_best, mse, best)
+    awq.awq_select_scale(sse, 1000, 264, abar, cfg, ws, s_best, mse, best)
     awq.awq_device_status(ws)
 
 
