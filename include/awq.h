@@ -317,7 +317,10 @@ awq_status awq_search_clip_grams(const void *W, int64_t out, int64_t in, const f
  *   X        device fp16 [T, in], row stride ldx
  *   qweight  device int32 [in, out/8]; qzeros int32 [in/g, out/8]; scales fp16 [in/g, out]
  *   Y        device fp16 [T, out] (output), row stride ldy (multiple of 8)
- *   ws       at least 256 bytes (status word)
+ *   ws       at least 256 bytes (status word); with awq_w4a16_workspace_size()
+ *            bytes, few tokens (output tiles filling under half of the SMs)
+ *            are computed with split-K: fp32 partial sums of K ranges in the
+ *            workspace, added in a fixed order and rounded to fp16 once
  * Uses cfg->group_size (32, 64 or 128); requires in % 64 == 0 and out % 32 == 0
  * (the packed words of a row are staged by TMA, whose row stride must be a
  * multiple of 16 bytes). */
@@ -325,6 +328,10 @@ awq_status awq_w4a16_gemm(const void *X, int64_t T, int64_t in, int64_t ldx, con
                           const int32_t *qzeros, const void *scales, int64_t out,
                           const awq_config *cfg, void *Y, int64_t ldy, void *ws, size_t ws_bytes,
                           awq_stream_t stream);
+
+/* Workspace bytes with which awq_w4a16_gemm uses split-K for this shape (256
+ * when it would not split).  Returns 0 when the arguments are invalid. */
+size_t awq_w4a16_workspace_size(int64_t T, int64_t in, int64_t out, const awq_config *cfg);
 
 /* Synchronises `stream`, then returns and clears the device status recorded in
  * workspace `ws` (AWQ_OK, AWQ_ERR_TIMEOUT or AWQ_ERR_NONFINITE).  With

@@ -32,6 +32,7 @@ from .abi import (  # noqa: F401
     awq_search_scale_sse,
     awq_select_scale,
     awq_w4a16_gemm,
+    awq_w4a16_workspace_size,
     awq_workspace_size,
     header_functions,
     last_error,

@@ -88,6 +88,7 @@ _SIGNATURES = {
     "awq_w4a16_gemm": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_void_p, c_void_p,
                                  c_int64, POINTER(AwqConfig), c_void_p, c_int64, c_void_p, c_size_t,
                                  c_void_p]),
+    "awq_w4a16_workspace_size": (c_size_t, [c_int64, c_int64, c_int64, POINTER(AwqConfig)]),
     "awq_act_sums": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_void_p]),
     "awq_act_stats_finish": (c_int32, [c_void_p, c_int64, c_int64, c_void_p, c_void_p]),
     "awq_search_scale_sse": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_int64,
@@ -289,6 +290,14 @@ def awq_w4a16_gemm(X, qweight, qzeros, scales, cfg: AwqConfig, Y, ws, stream=Non
         _ptr(X), X.shape[0], X.shape[1], X.stride(0), _ptr(qweight), _ptr(qzeros), _ptr(scales),
         Y.shape[1], ctypes.byref(cfg), _ptr(Y), Y.stride(0), _ptr(ws), ws.numel() * ws.element_size(),
         _stream(stream)))
+
+
+def awq_w4a16_workspace_size(T: int, inn: int, out: int, cfg: AwqConfig) -> int:
+    """Workspace bytes that let awq_w4a16_gemm split K for few tokens."""
+    n = LIB.awq_w4a16_workspace_size(T, inn, out, ctypes.byref(cfg))
+    if n == 0:
+        raise AwqError("awq_w4a16_workspace_size", 1, last_error())
+    return int(n)
 
 
 def awq_device_status(ws, stream=None) -> None:

@@ -242,6 +242,11 @@ Fault fault_mode() {
   return Fault::kNone;
 }
 
+// status word plus the fp32 partial sums [splits][T][out] of a split-K W4A16 GEMM
+size_t w4a16_ws_bytes(int64_t T, int64_t out, int splits) {
+  return kHeader + align256(sizeof(float) * (size_t)splits * (size_t)T * (size_t)out);
+}
+
 uint32_t poll_cap() {
   return fault_mode() == Fault::kTimeout ? 1u : 1u << 24;
 }
@@ -720,13 +725,31 @@ awq_status awq_w4a16_gemm(const void *X, int64_t T, int64_t in, int64_t ldx, con
   AWQ_LAUNCH_GATE();
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   DevStatus *dst = static_cast<DevStatus *>(ws);
+  // split-K for few tokens, when the workspace holds the fp32 partial sums
+  int splits = w4a16_splits(T, in, out, num_sms_current());
+  if (splits > 1 && ws_bytes < w4a16_ws_bytes(T, out, splits)) splits = 1;
+  float *partials = splits > 1 ? reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + kHeader) : nullptr;
   AWQ_TRY_CUDA(cudaMemsetAsync(dst, 0, sizeof(DevStatus), cs), "workspace reset");
   ProfScope p("w4a16_gemm", cs);
   AWQ_TRY_CUDA(launch_w4a16_gemm(static_cast<const __half *>(X), T, in, ldx, qweight, qzeros,
                                  static_cast<const __half *>(scales), out, cfg->group_size,
-                                 static_cast<__half *>(Y), ldy, dst, poll_cap(), num_sms_current(), cs),
+                                 static_cast<__half *>(Y), ldy, partials, splits, dst, poll_cap(),
+                                 num_sms_current(), cs),
                "w4a16_gemm launch");
   return AWQ_OK;
+}
+
+size_t awq_w4a16_workspace_size(int64_t T, int64_t in, int64_t out, const awq_config *cfg) {
+  g_err.clear();
+  NvtxCall nvtx_call_(__func__);
+  if (fault_mode() == Fault::kAlloc) {
+    fail(AWQ_ERR_WORKSPACE, "injected allocation failure (AWQ_FAULT=alloc)");
+    return 0;
+  }
+  if (check_cfg(cfg) != AWQ_OK) return 0;
+  if (check_shape(T, in, out, cfg) != AWQ_OK) return 0;
+  const int splits = w4a16_splits(T, in, out, num_sms_current());
+  return splits > 1 ? w4a16_ws_bytes(T, out, splits) : kHeader;
 }
 
 awq_status awq_fold_inv_scale(void *v, int64_t rows, int64_t cols, const float *s,

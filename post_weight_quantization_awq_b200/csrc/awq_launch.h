@@ -120,10 +120,17 @@ cudaError_t lib_status_read_clear(DevStatus *h);
 
 // W4A16 GEMM on the packed output: Y = RN16(X Wd^T), Wd = RN16((q - z) scale);
 // in % 64 == 0, out % 32 == 0, group in {32, 64, 128}.
+// splits > 1: split-K over `splits` K ranges, fp32 partial sums in
+// partials [splits][T][out], then a fixed-order reduction into Y.
 cudaError_t launch_w4a16_gemm(const __half *X, int64_t T, int64_t in, int64_t ldx,
                               const int32_t *qweight, const int32_t *qzeros, const __half *scales,
-                              int64_t out, int group, __half *Y, int64_t ldy, DevStatus *st,
-                              uint32_t max_polls, int num_sms, cudaStream_t stream);
+                              int64_t out, int group, __half *Y, int64_t ldy, float *partials,
+                              int splits, DevStatus *st, uint32_t max_polls, int num_sms,
+                              cudaStream_t stream);
+// The split count the W4A16 GEMM uses when its workspace allows: 1 when the
+// output tiles fill at least half of the SMs, else enough K splits (each of
+// at least 4 K steps of 64 channels) to occupy them.
+int w4a16_splits(int64_t T, int64_t in, int64_t out, int num_sms);
 
 // K8: v[j][:] = RN16(RN32(v[j][:]) / s_j).
 cudaError_t launch_fold(__half *v, int64_t rows, int64_t cols, const float *s, cudaStream_t stream);

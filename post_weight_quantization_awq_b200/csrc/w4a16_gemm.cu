@@ -90,6 +90,16 @@ __device__ __forceinline__ void q_tile_coords(int tile, int num_m, int num_n, in
   n_blk = local / gm;
 }
 
+// Split-K: tile = (output tile, K split), split fastest; split sp of S covers
+// K steps [sp num_kb / S, (sp + 1) num_kb / S).
+__device__ __forceinline__ void q_tile_split(int tile, int num_m, int num_n, int splits, int num_kb,
+                                             int &m_blk, int &n_blk, int &sp, int &kb0, int &kb1) {
+  sp = tile % splits;
+  q_tile_coords(tile / splits, num_m, num_n, m_blk, n_blk);
+  kb0 = (int)((int64_t)sp * num_kb / splits);
+  kb1 = (int)((int64_t)(sp + 1) * num_kb / splits);
+}
+
 // fp16 pairs {1024 + nibble p, 1024 + nibble p + 4}, p = 0..3, of a word
 __device__ __forceinline__ void nib_pairs(uint32_t w, __half2 (&h)[4]) {
 #pragma unroll
@@ -134,8 +144,8 @@ __device__ __forceinline__ void q_abort(QTail *t, DevStatus *st, uint32_t where)
 __global__ void __launch_bounds__(Q_THREADS, 1) w4a16_gemm_kernel(
     const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
     const int32_t *__restrict__ qzeros, const __half *__restrict__ scales, int64_t T, int64_t out,
-    int group, int num_m, int num_n, int num_kb, __half *__restrict__ Y, int64_t ldy,
-    DevStatus *st, uint32_t max_polls) {
+    int group, int num_m, int num_n, int num_kb, int splits, __half *__restrict__ Y, int64_t ldy,
+    float *__restrict__ partials, DevStatus *st, uint32_t max_polls) {
   extern __shared__ uint8_t q_smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(q_smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -145,7 +155,7 @@ __global__ void __launch_bounds__(Q_THREADS, 1) w4a16_gemm_kernel(
   QTail *tail = reinterpret_cast<QTail *>(sW + QSTAGES * QW_BYTES);
   volatile int *abort_flag = &tail->abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int num_tiles = num_m * num_n;
+  const int num_tiles = num_m * num_n * splits;
   const int64_t words = out / 8;  // int32 words per qweight / qzeros row
 
   if (threadIdx.x == 0) {
@@ -182,9 +192,9 @@ __global__ void __launch_bounds__(Q_THREADS, 1) w4a16_gemm_kernel(
       uint32_t phase = 0, issued = 0, issued_parity = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-        int m_blk, n_blk;
-        q_tile_coords(tile, num_m, num_n, m_blk, n_blk);
-        for (int kb = 0; kb < num_kb; ++kb) {
+        int m_blk, n_blk, sp, kb0, kb1;
+        q_tile_split(tile, num_m, num_n, splits, num_kb, m_blk, n_blk, sp, kb0, kb1);
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait_long(&tail->empty[stage], phase ^ 1u, max_polls, abort_flag)) {
             q_abort(tail, st, 0xD00u + stage);
             ok = false;
@@ -216,10 +226,11 @@ __global__ void __launch_bounds__(Q_THREADS, 1) w4a16_gemm_kernel(
     int stage = 0;
     uint32_t phase = 0;
     // the (tile, K step) sequence of this CTA, one step ahead for the word loads
-    int tile = blockIdx.x, kb = 0;
-    auto word_col = [&](int tl) {  // this thread's qweight column in tile tl
-      int m_blk, n_blk;
-      q_tile_coords(tl, num_m, num_n, m_blk, n_blk);
+    int tile = blockIdx.x, kb = 0, kb_end = 0;
+    // this thread's qweight column in tile tl, and the tile's K steps
+    auto word_col = [&](int tl, int &k0, int &k1) {
+      int m_blk, n_blk, sp;
+      q_tile_split(tl, num_m, num_n, splits, num_kb, m_blk, n_blk, sp, k0, k1);
       return (int64_t)n_blk * (QBN / 8) + col;
     };
     // zero words and scales of one K step: rows 0..31 of the step use group
@@ -237,8 +248,8 @@ __global__ void __launch_bounds__(Q_THREADS, 1) w4a16_gemm_kernel(
                         : make_uint4(0u, 0u, 0u, 0u);
       }
     };
-    int64_t wcol = tile < num_tiles ? word_col(tile) : 0;
-    if (tile < num_tiles) load_zs(wcol, 0);
+    int64_t wcol = tile < num_tiles ? word_col(tile, kb, kb_end) : 0;
+    if (tile < num_tiles) load_zs(wcol, kb);
     bool ok = true;
     while (ok && tile < num_tiles) {
       uint32_t zw[2];
@@ -248,12 +259,11 @@ __global__ void __launch_bounds__(Q_THREADS, 1) w4a16_gemm_kernel(
         zw[h] = znext[h];
         sc[h] = snext[h];
       }
-      int ntile = tile, nkb = kb + 1;
+      int ntile = tile, nkb = kb + 1, nkb_end = kb_end;
       int64_t nwcol = wcol;
-      if (nkb == num_kb) {
-        nkb = 0;
+      if (nkb == kb_end) {
         ntile += gridDim.x;
-        nwcol = ntile < num_tiles ? word_col(ntile) : 0;
+        nwcol = ntile < num_tiles ? word_col(ntile, nkb, nkb_end) : 0;
       }
       if (ntile < num_tiles) load_zs(nwcol, nkb);
       __half2 zp[2][4], sp[2][4];
@@ -296,6 +306,7 @@ __global__ void __launch_bounds__(Q_THREADS, 1) w4a16_gemm_kernel(
       }
       tile = ntile;
       kb = nkb;
+      kb_end = nkb_end;
       wcol = nwcol;
     }
   } else if (warp == 1) {
@@ -314,7 +325,9 @@ __global__ void __launch_bounds__(Q_THREADS, 1) w4a16_gemm_kernel(
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base;
-        for (int kb = 0; kb < num_kb; ++kb) {
+        int m_blk, n_blk, sp, kb0, kb1;
+        q_tile_split(tile, num_m, num_n, splits, num_kb, m_blk, n_blk, sp, kb0, kb1);
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait_long(&tail->full[stage], phase, max_polls, abort_flag) ||
               !mbar_wait_bounded(&tail->ld[stage], phase, max_polls, abort_flag)) {  // X tile
             q_abort(tail, st, 0xD30u + stage);
@@ -330,7 +343,7 @@ __global__ void __launch_bounds__(Q_THREADS, 1) w4a16_gemm_kernel(
 #pragma unroll
             for (int h = 0; h < 2; ++h)
               tc_mma_f16(d_tmem + h * QBN, smem_desc_k_sw128(a_addr + h * QA_HALF + k * 32), bd, IDESC_Q,
-                         (kb | k) != 0 ? 1u : 0u);
+                         (kb != kb0 || k != 0) ? 1u : 0u);
           }
           issued_any = true;
           tc_commit(&tail->empty[stage]);
@@ -362,8 +375,8 @@ __global__ void __launch_bounds__(Q_THREADS, 1) w4a16_gemm_kernel(
         break;
       }
       tc_fence_after();
-      int m_blk, n_blk;
-      q_tile_coords(tile, num_m, num_n, m_blk, n_blk);
+      int m_blk, n_blk, sp, kb0, kb1;
+      q_tile_split(tile, num_m, num_n, splits, num_kb, m_blk, n_blk, sp, kb0, kb1);
 #pragma unroll 1
       for (int c2 = 0; c2 < 2 * QBN; c2 += 32) {
         const int h = c2 / QBN, c = c2 % QBN;  // accumulator half (rows 128 h ..) and column
@@ -372,7 +385,19 @@ __global__ void __launch_bounds__(Q_THREADS, 1) w4a16_gemm_kernel(
         tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)c2, v);
         tmem_ld_wait();
         const int64_t o0 = (int64_t)n_blk * QBN + c;
-        if (t_row < T) {
+        if (partials && t_row < T) {
+          // split-K: this split's fp32 sums, in output order, for the reduction
+          float *prow = partials + ((int64_t)sp * T + t_row) * out + o0;
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            if (o0 + 8 * u >= out) break;  // out % 8 == 0
+            // accumulator column 8u + 2p holds output 8u + p, column 8u + 2p + 1 output 8u + p + 4
+            const float4 lo = make_float4(v[8 * u + 0], v[8 * u + 2], v[8 * u + 4], v[8 * u + 6]);
+            const float4 hi = make_float4(v[8 * u + 1], v[8 * u + 3], v[8 * u + 5], v[8 * u + 7]);
+            *reinterpret_cast<float4 *>(prow + 8 * u) = lo;
+            *reinterpret_cast<float4 *>(prow + 8 * u + 4) = hi;
+          }
+        } else if (t_row < T) {
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
             if (o0 + 8 * u >= out) break;  // out % 8 == 0
@@ -403,11 +428,47 @@ __global__ void __launch_bounds__(Q_THREADS, 1) w4a16_gemm_kernel(
   }
 }
 
+// Y[t][o] = RN16(sum over splits s of partials[s][t][o]), the splits added in
+// order (a fixed summation order: the result does not depend on scheduling).
+__global__ void w4a16_splitk_reduce_kernel(const float *__restrict__ partials, int splits, int64_t T,
+                                           int64_t out, __half *__restrict__ Y, int64_t ldy) {
+  const int64_t n4 = T * out / 4;  // out % 8 == 0
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    float4 acc = __ldcs(reinterpret_cast<const float4 *>(partials) + i);
+    for (int sp = 1; sp < splits; ++sp) {
+      const float4 v = __ldcs(reinterpret_cast<const float4 *>(partials + (int64_t)sp * T * out) + i);
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
+    }
+    const int64_t e = 4 * i, t = e / out, o = e - t * out;
+    const __half2 a = __floats2half2_rn(acc.x, acc.y), b = __floats2half2_rn(acc.z, acc.w);
+    uint2 pk;
+    pk.x = *reinterpret_cast<const uint32_t *>(&a);
+    pk.y = *reinterpret_cast<const uint32_t *>(&b);
+    *reinterpret_cast<uint2 *>(Y + t * ldy + o) = pk;
+  }
+}
+
+int w4a16_splits(int64_t T, int64_t in, int64_t out, int num_sms) {
+  const int64_t tiles = ((T + QBM - 1) / QBM) * ((out + QBN - 1) / QBN);
+  const int64_t num_kb = in / QBK;
+  if (tiles * 2 > num_sms || num_kb < 8) return 1;
+  // enough splits to fill the SMs, each with at least 4 K steps
+  int64_t s = num_sms / tiles;
+  if (s > num_kb / 4) s = num_kb / 4;
+  return (int)(s < 1 ? 1 : s);
+}
+
 cudaError_t launch_w4a16_gemm(const __half *X, int64_t T, int64_t in, int64_t ldx,
                               const int32_t *qweight, const int32_t *qzeros, const __half *scales,
-                              int64_t out, int group, __half *Y, int64_t ldy, DevStatus *st,
-                              uint32_t max_polls, int num_sms, cudaStream_t stream) {
+                              int64_t out, int group, __half *Y, int64_t ldy, float *partials,
+                              int splits, DevStatus *st, uint32_t max_polls, int num_sms,
+                              cudaStream_t stream) {
   if (in % QBK != 0 || out % 32 != 0 || group % 32 != 0) return cudaErrorInvalidValue;
+  if (splits < 1 || splits > in / QBK || (splits > 1 && !partials)) return cudaErrorInvalidValue;
   CUtensorMap tmX, tmW;
   cudaError_t e = make_tmap_f16_box(&tmX, X, T, in, ldx, QBK, QBM);
   if (e != cudaSuccess) return e;
@@ -418,11 +479,17 @@ cudaError_t launch_w4a16_gemm(const __half *X, int64_t T, int64_t in, int64_t ld
   if (e != cudaSuccess) return e;
   const int num_m = (int)((T + QBM - 1) / QBM);
   const int num_n = (int)((out + QBN - 1) / QBN);
-  const int tiles = num_m * num_n;
+  const int tiles = num_m * num_n * splits;
   const int grid = tiles < num_sms ? tiles : num_sms;
   w4a16_gemm_kernel<<<grid, Q_THREADS, kQSmemBytes, stream>>>(
-      tmX, tmW, qzeros, scales, T, out, group, num_m, num_n, (int)(in / QBK), Y, ldy, st,
-      max_polls);
+      tmX, tmW, qzeros, scales, T, out, group, num_m, num_n, (int)(in / QBK), splits, Y, ldy,
+      splits > 1 ? partials : nullptr, st, max_polls);
+  e = cudaGetLastError();
+  if (e != cudaSuccess || splits == 1) return e;
+  const int64_t n4 = T * out / 4;
+  const int64_t blocks = i64min((int64_t)num_sms * 8, (n4 + 255) / 256);
+  w4a16_splitk_reduce_kernel<<<(unsigned)(blocks < 1 ? 1 : blocks), 256, 0, stream>>>(
+      partials, splits, T, out, Y, ldy);
   return cudaGetLastError();
 }
 

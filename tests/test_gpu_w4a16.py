@@ -28,11 +28,14 @@ def _ulp16(v):
     return np.exp2(np.floor(np.log2(np.maximum(a, 2.0 ** -14))) - 10)
 
 
-def _gpu_w4a16(X, qw, qz, sc, cfg):
+def _gpu_w4a16(X, qw, qz, sc, cfg, split_ws=False):
+    """split_ws: a workspace of awq_w4a16_workspace_size() bytes (split-K for
+    few tokens); otherwise the 256-byte minimum (never splits)."""
     Xd = to_dev(X)
     T, out = Xd.shape[0], sc.shape[1]
     Y = torch.empty((T, out), dtype=torch.float16, device="cuda")
-    ws = torch.empty(256, dtype=torch.uint8, device="cuda")
+    n = awq.awq_w4a16_workspace_size(T, Xd.shape[1], out, cfg) if split_ws else 256
+    ws = torch.empty(n, dtype=torch.uint8, device="cuda")
     awq.awq_w4a16_gemm(Xd, torch.from_numpy(qw).cuda(), torch.from_numpy(qz).cuda(),
                        torch.from_numpy(np.ascontiguousarray(sc)).cuda(), cfg, Y, ws)
     awq.awq_device_status(ws)
@@ -156,3 +159,29 @@ def test_w4a16_on_the_searched_q_proj_layer():
     Yref = Xd[torch.from_numpy(rows).cuda()].float() @ Wd.float().T
     mse = float(((Y[torch.from_numpy(rows).cuda()].float() - Yref) ** 2).mean())
     assert mse < 1.5 * float(res.mse.min()) + 1e-6, (mse, float(res.mse.min()))
+
+
+@pytest.mark.parametrize("T", [1, 16, 100, 300])
+def test_w4a16_split_k_for_few_tokens(T):
+    """Few tokens leave most SMs without an output tile: with the workspace
+    awq_w4a16_workspace_size() asks for, K is split and the fp32 partial sums
+    are added in a fixed order.  Exact sums stay exact (bit-equal to the
+    unsplit GEMM and the oracle); a searched layer stays within the bound."""
+    cfg = awq.AwqConfig.make()
+    inn, out = 4096, 1024
+    assert awq.awq_w4a16_workspace_size(T, inn, out, cfg) > 256  # this shape splits
+    assert awq.awq_w4a16_workspace_size(65536, inn, out, cfg) == 256
+    rng = np.random.default_rng(T)
+    qw, qz, sc = _random_packed(inn, out, 128, rng, pow2_scales=True)
+    X = rng.integers(-3, 4, size=(T, inn)).astype(np.float16)
+    a = _gpu_w4a16(torch.from_numpy(X), qw, qz, sc, cfg, split_ws=True)
+    b = _gpu_w4a16(torch.from_numpy(X), qw, qz, sc, cfg, split_ws=False)
+    want = O.w4a16_matmul(X, qw, qz, sc, 128).astype(np.float16)
+    assert np.array_equal(a.view(np.uint16), want.view(np.uint16))
+    assert np.array_equal(b.view(np.uint16), want.view(np.uint16))
+    Xr, W = random_layer(T, inn, out, seed=T + 5)
+    s = O.scale_grid(O.act_stats(Xr.numpy()), O.alpha_grid(20))[9]
+    qw, qz, sc = O.quant_pack(W.numpy(), s, None, 4, 128)
+    Xs = (Xr.numpy().astype(np.float32) / s[None, :]).astype(np.float16)
+    _check(_gpu_w4a16(torch.from_numpy(Xs), qw, qz, sc, cfg, split_ws=True), Xs, qw, qz, sc, 128)
+
