@@ -44,24 +44,29 @@ KERNELS_PER_STEP = {  # kernels this library launches per step (memsets excluded
 # that digest; after any change to them the line carries traffic = null until
 # the kernel is captured again.
 NCU_TRAFFIC = {
-    "bytes": None,
-    "sources_sha256": None,
+    "bytes": 11_301_274_368 + 9_137_152,  # read + write, one launch at 65536 tokens
+    "sources_sha256": "aca2aec1256dde43bb8269898f7055072f8ad9a5ff3bb62c30e7bdc71bfdf28f",
     "command": ("ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none "
                 "-k regex:search_gemm -s 5 -c 1 python bench.py --steps 1 --warmup 5 "
                 "--no-cpu-baseline --no-gram-form --no-cached-form --no-w4a16"),
 }
 TRAFFIC_SOURCES = ("post_weight_quantization_awq_b200/csrc/search_gemm.cu",
-                   "post_weight_quantization_awq_b200/csrc/awq_device.cuh",
-                   "post_weight_quantization_awq_b200/csrc/awq_launch.h")
+                   "post_weight_quantization_awq_b200/csrc/awq_device.cuh")
+TILE_HEADER = "post_weight_quantization_awq_b200/csrc/awq_launch.h"
 
 
 def traffic_sources_digest() -> str:
-    """SHA-256 over the sources the scored-GEMM kernel is compiled from."""
+    """SHA-256 over the sources the scored-GEMM kernel is compiled from: its
+    file, the device header, and the line of the launch header that fixes its
+    tile shape."""
     import hashlib
     h = hashlib.sha256()
     for rel in TRAFFIC_SOURCES:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
+    with open(os.path.join(ROOT, TILE_HEADER)) as f:
+        tile = [ln for ln in f.read().splitlines() if "kGemmBM" in ln and "constexpr" in ln]
+    h.update("\n".join(tile).encode())
     return h.hexdigest()
 
 
@@ -429,7 +434,28 @@ def run_awq(args):
                  "flops": flops_q,
                  "note": "Y = X Wd^T with Wd dequantised on the fly from qweight/qzeros/scales; "
                          "T x in x out of the layer above"}
-        del Xs, Yq
+        # decode-sized: 16 tokens, split-K through the workspace the library asks for
+        td = 16
+        Xt = Xs[:td].contiguous()
+        Yt = torch.empty((td, out), dtype=torch.float16, device=dev)
+        ws_t = torch.empty(awq.awq_w4a16_workspace_size(td, inn, out, cfg), dtype=torch.uint8,
+                           device=dev)
+
+        def step_t():
+            awq.awq_w4a16_gemm(Xt, r.qweight, r.qzeros, r.scales, cfg, Yt, ws_t)
+
+        for _ in range(args.warmup):
+            step_t()
+        awq.awq_device_status(ws_t)
+        ms_t = timed_steps(step_t, max(args.steps, 20), dist, timer, local)
+        awq.awq_device_status(ws_t)
+        wbytes = inn * out // 2 + (inn // g) * out * 2 + (inn // g) * out // 2  # codes, scales, zeros
+        w4a16["decode_16_tokens"] = {
+            "ms": round(ms_t, 4), "weight_bytes": wbytes,
+            "gbs": round(wbytes / (ms_t * 1e-3) / 1e9, 1),
+            "note": "T = 16: bound by reading the packed weights; K split over the SMs "
+                    "(awq_w4a16_workspace_size), L2-resident after the first step"}
+        del Xs, Yq, Xt, Yt, ws_t
 
     # ---- the literal fp16-output form on the same layer: Y = RN16(X W^T) once,
     # then every candidate's output scored against it in the GEMM's epilogue

@@ -259,6 +259,7 @@ cudaError_t launch_wmax(const __half *W, int64_t n, int64_t in, const float *r, 
 // ---------------------------------------------------------------------------
 constexpr int kCandRows = 64;
 constexpr int kCandWarpRows = 8;  // rows per warp: 8 warps x 8 rows
+constexpr int kCandBatch = 4;     // rows a warp holds in registers at a time
 
 // Transposing butterfly for the group ranges of N rows over the 2 * OFF lanes
 // of a group: each round exchanges half of the rows a lane carries with its
@@ -266,7 +267,7 @@ constexpr int kCandWarpRows = 8;  // rows per warp: 8 warps x 8 rows
 // carried halve while the lanes reduced over double; once one row is left the
 // rounds are plain butterflies.  Lane l ends with rows held_by_lane / held_at.
 template <int N, int OFF>
-__device__ __forceinline__ void transpose_reduce(float (&mx)[kCandWarpRows], float (&mn)[kCandWarpRows],
+__device__ __forceinline__ void transpose_reduce(float (&mx)[kCandBatch], float (&mn)[kCandBatch],
                                                  int lane) {
   if constexpr (OFF >= 1) {
     if constexpr (N > 1) {
@@ -318,7 +319,7 @@ __device__ __forceinline__ constexpr int held_at(int r) {
 // s, i.e. the s 2^k step times 2^-k, exact) -- the inspection form of the
 // kernel, with every quantisation step shared with the operand form.
 template <int group, bool kCodes>  // group 32, 64 or 128: the range shuffles unroll
-__global__ void __launch_bounds__(256) cand_quant_kernel(
+__global__ void __launch_bounds__(256, 3) cand_quant_kernel(
     const __half *__restrict__ W, int64_t out, int64_t in, int64_t out_pad,
     const float *__restrict__ s, const float *__restrict__ inv_s, const float *__restrict__ rch,
     float qmax, int sym, int weights_only, const DevStatus *__restrict__ st,
@@ -368,19 +369,21 @@ __global__ void __launch_bounds__(256) cand_quant_kernel(
       iv[h] = make_float2(1.0f, 1.0f);
     }
   }
-  // ---- pass 1: this warp's 8 rows (o0 + 8 warp .. + 7) into registers, and
-  // this lane's share of each row's group range
-  uint4 wv[kCandWarpRows];
-  float mx[kCandWarpRows], mn[kCandWarpRows];
-  const int64_t orow = o0 + (int64_t)warp * kCandWarpRows;
+  // ---- the warp's 8 rows (o0 + 8 warp .. + 7) in batches of kCandBatch rows
+  // held in registers: pass 1 takes this lane's share of each row's group range
+#pragma unroll 1
+  for (int bt = 0; bt < kCandWarpRows / kCandBatch; ++bt) {
+  uint4 wv[kCandBatch];
+  float mx[kCandBatch], mn[kCandBatch];
+  const int64_t orow = o0 + (int64_t)warp * kCandWarpRows + bt * kCandBatch;
 #pragma unroll
-  for (int r = 0; r < kCandWarpRows; ++r) {
+  for (int r = 0; r < kCandBatch; ++r) {
     const bool live = j_ok && orow + r < out;
     wv[r] = live ? __ldg(reinterpret_cast<const uint4 *>(W + (orow + r) * in + j0))
                  : make_uint4(0u, 0u, 0u, 0u);
   }
 #pragma unroll
-  for (int r = 0; r < kCandWarpRows; ++r) {
+  for (int r = 0; r < kCandBatch; ++r) {
     const uint32_t wr[4] = {wv[r].x, wv[r].y, wv[r].z, wv[r].w};
     float m = -INFINITY, n = INFINITY;
 #pragma unroll
@@ -393,11 +396,11 @@ __global__ void __launch_bounds__(256) cand_quant_kernel(
     mn[r] = n;
   }
   // ---- whole-group ranges: a transposing butterfly over the group's lanes
-  // leaves each lane kCandWarpRows / lanes rows (one row, on two lanes, when
-  // lanes = 16), and each lane computes the step, zero point, fast-path bound
-  // and clamp need of its rows once
-  transpose_reduce<kCandWarpRows, lanes / 2>(mx, mn, lane);
-  constexpr int kHeld = kCandWarpRows >= lanes ? kCandWarpRows / lanes : 1;
+  // leaves each lane kCandBatch / lanes rows (or one row shared by several
+  // lanes), and each lane computes the step, zero point, fast-path bound and
+  // clamp need of its rows once
+  transpose_reduce<kCandBatch, lanes / 2>(mx, mn, lane);
+  constexpr int kHeld = kCandBatch >= lanes ? kCandBatch / lanes : 1;
   float pd[kHeld], pr[kHeld], ph[kHeld];
   int pz[kHeld];
 #pragma unroll
@@ -420,8 +423,8 @@ __global__ void __launch_bounds__(256) cand_quant_kernel(
   // correctly rounded division otherwise; the clamp only where needed
   const float2 M = make_float2(12582912.0f, 12582912.0f);  // 1.5 2^23
 #pragma unroll
-  for (int r = 0; r < kCandWarpRows; ++r) {
-    const int src = held_by_lane<lanes, kCandWarpRows>(r), el = held_at<lanes, kCandWarpRows>(r);
+  for (int r = 0; r < kCandBatch; ++r) {
+    const int src = held_by_lane<lanes, kCandBatch>(r), el = held_at<lanes, kCandBatch>(r);
     const float dl = __shfl_sync(0xffffffffu, pd[el], src, lanes);
     const float rc = __shfl_sync(0xffffffffu, pr[el], src, lanes);
     const float hl = __shfl_sync(0xffffffffu, ph[el], src, lanes);
@@ -482,6 +485,7 @@ __global__ void __launch_bounds__(256) cand_quant_kernel(
     if (j_ok)
       *reinterpret_cast<uint4 *>(dW + ((int64_t)a * out_pad + o) * in + j0) =
           make_uint4(packed[0], packed[1], packed[2], packed[3]);
+  }
   }
 }
 
