@@ -10,16 +10,21 @@
 // K = in.  The epilogue squares and sums each accumulator tile straight out
 // of tensor memory, so no candidate output is ever written to HBM.
 //
-// sm_100a design, one CTA per SM (192 threads):
-//   warp 0      TMA producer: A tile 128x64 and B tile 256x64 (fp16, 128-byte
-//               swizzle) into a 4-stage shared-memory ring;
-//   warp 1      allocates 512 TMEM columns; one thread issues
-//               tcgen05.mma.cta_group::1.kind::f16 (M=128, N=256, K=16) into a
-//               double-buffered fp32 accumulator (2 x 256 columns) and commits
-//               stage/accumulator barriers;
+// sm_100a design, one CTA per SM (192 threads), 256 x 256 output tiles:
+//   warp 0      TMA producer: A tile 256x64 and B tile 256x64 (fp16, 128-byte
+//               swizzle) into a 3-stage shared-memory ring;
+//   warp 1      allocates 512 TMEM columns; one thread issues two
+//               tcgen05.mma.cta_group::1.kind::f16 (M=128, N=256, K=16) per K
+//               slice, one per 128-row half of the A tile, both against the one
+//               B tile, into the two halves of TMEM, and commits stage and
+//               accumulator barriers (TMEM holds one tile: the next tile's
+//               MMAs wait for the epilogue);
 //   warps 2..5  epilogue: tcgen05.ld 32 lanes x 32 columns at a time, sum of
 //               squares in fp32 per row, fp64 warp reduction, one partial per
-//               (tile, warp) into HBM.
+//               (128-row block, N tile, warp) into HBM.
+// Sharing each B tile between two M halves halves the B traffic from L2 to
+// shared memory per flop; under the power cap that bought 4 % more
+// throughput than 128 x 256 tiles with a double-buffered accumulator.
 // Tiles are visited in groups of `group_m` M-blocks so the A panels of a
 // group stay in L2 while all N-blocks stream past.  Every mbarrier wait is
 // bounded; a wait that runs out records kDevTimeout, raises a CTA-wide abort
@@ -36,13 +41,15 @@ namespace awq {
 namespace {
 
 constexpr int BM = kGemmBM, BN = kGemmBN, BK = kGemmBK;
-constexpr int STAGES = 4;
-constexpr uint32_t A_BYTES = BM * BK * 2;  // 16 KiB
+constexpr int STAGES = 3;
+constexpr int BM2 = 2 * BM;                  // CTA tile rows: two M = 128 accumulators
+constexpr uint32_t A_HALF = BM * BK * 2;     // 16 KiB: rows 128..255 of an A tile start here
+constexpr uint32_t A_BYTES = BM2 * BK * 2;   // 32 KiB
 constexpr uint32_t B_BYTES = BN * BK * 2;  // 32 KiB
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t IDESC = idesc_f16_f32(BM, BN);
 constexpr uint32_t DRAIN_POLLS = 1u << 22;
-constexpr int GROUP_M = 32;
+constexpr int GROUP_M = 16;  // 256-row M blocks per group: 4096 rows of A in L2
 constexpr int kEpiSse = 0, kEpiStoreY = 1, kEpiSubY = 2;
 
 struct __align__(8) GemmSmemTail {
@@ -98,7 +105,8 @@ __global__ void __launch_bounds__(192, 1)
   volatile int *abort_flag = &tail->abort_flag;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int num_tiles = num_m * num_n;
+  const int num_m2 = (num_m + 1) / 2;  // 256-row M blocks (num_m counts 128-row blocks)
+  const int num_tiles = num_m2 * num_n;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
@@ -135,7 +143,7 @@ __global__ void __launch_bounds__(192, 1)
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
         int m_blk, n_blk;
-        tile_coords(tile, num_m, num_n, GROUP_M, m_blk, n_blk);
+        tile_coords(tile, num_m2, num_n, GROUP_M, m_blk, n_blk);
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait_long(&tail->empty[stage], phase ^ 1u, max_polls, abort_flag)) {
             raise_abort(tail, st, 0x100u + stage);
@@ -143,7 +151,7 @@ __global__ void __launch_bounds__(192, 1)
             break;
           }
           mbar_arrive_expect_tx(&tail->full[stage], A_BYTES + B_BYTES);
-          tma_load_2d(sA + stage * A_BYTES, &tmA, &tail->full[stage], kb * BK, m_blk * BM);
+          tma_load_2d(sA + stage * A_BYTES, &tmA, &tail->full[stage], kb * BK, m_blk * BM2);
           tma_load_2d(sB + stage * B_BYTES, &tmB, &tail->full[stage], kb * BK, n_blk * BN);
           issued |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
@@ -169,14 +177,14 @@ __global__ void __launch_bounds__(192, 1)
       bool ok = true, issued_any = false;
       int it = 0;
       for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x, ++it) {
-        const int acc = it & 1;
-        const uint32_t acc_phase = (it >> 1) & 1;
+        const int acc = 0;  // TMEM holds one 256 x 256 tile: columns 0..255 rows 0..127, 256..511 rows 128..255
+        const uint32_t acc_phase = it & 1;
         if (!mbar_wait_bounded(&tail->tempty[acc], acc_phase ^ 1u, max_polls, abort_flag)) {
           raise_abort(tail, st, 0x200u + acc);
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * BN;
+        const uint32_t d_tmem = tmem_base;
         for (int kb = 0; kb < num_kb; ++kb) {
           if (!mbar_wait_bounded(&tail->full[stage], phase, max_polls, abort_flag)) {
             raise_abort(tail, st, 0x300u + stage);
@@ -188,8 +196,11 @@ __global__ void __launch_bounds__(192, 1)
           const uint32_t b_addr = smem_u32(sB + stage * B_BYTES);
 #pragma unroll
           for (int k = 0; k < BK / 16; ++k) {
-            tc_mma_f16(d_tmem, smem_desc_k_sw128(a_addr + k * 32), smem_desc_k_sw128(b_addr + k * 32),
-                       IDESC, (kb | k) != 0 ? 1u : 0u);
+            const uint64_t bd = smem_desc_k_sw128(b_addr + k * 32);
+#pragma unroll
+            for (int h = 0; h < 2; ++h)  // both row halves share the B tile
+              tc_mma_f16(d_tmem + h * BN, smem_desc_k_sw128(a_addr + h * A_HALF + k * 32), bd, IDESC,
+                         (kb | k) != 0 ? 1u : 0u);
           }
           issued_any = true;
           tc_commit(&tail->empty[stage]);  // frees the stage once these MMAs finish
@@ -211,8 +222,8 @@ __global__ void __launch_bounds__(192, 1)
     const int q = warp & 3;  // TMEM lane quarter this warp may access
     int it = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
-      const int acc = it & 1;
-      const uint32_t acc_phase = (it >> 1) & 1;
+      const int acc = 0;
+      const uint32_t acc_phase = it & 1;
       int ok = 1;
       if (lane == 0) ok = mbar_wait_long(&tail->tfull[acc], acc_phase, max_polls, abort_flag);
       ok = __shfl_sync(0xffffffffu, ok, 0);
@@ -222,63 +233,74 @@ __global__ void __launch_bounds__(192, 1)
       }
       tc_fence_after();
       int m_blk, n_blk;
-      tile_coords(tile, num_m, num_n, GROUP_M, m_blk, n_blk);
-      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN);
-      // this thread's accumulator row is token m_blk * BM + 32 q + lane
-      const size_t yrow = (size_t)(m_blk * BM + q * 32 + lane) * (size_t)ldy;
-      float sum = 0.0f;
+      tile_coords(tile, num_m2, num_n, GROUP_M, m_blk, n_blk);
+      float sums[2] = {0.0f, 0.0f};
 #pragma unroll 1
-      for (int c = 0; c < BN; c += 32) {
-        float v[32];
-        if constexpr (EPI == kEpiSubY) {
-          // fetch the cached fp16 outputs first, so their latency overlaps the TMEM read
-          const uint4 *yp = reinterpret_cast<const uint4 *>(
-              Y + yrow + (size_t)(((int64_t)n_blk * BN) % y_cols) + c);
-          uint4 yv[4];
+      for (int h = 0; h < 2; ++h) {
+        const int m128 = 2 * m_blk + h;  // 128-row block of this half
+        if (m128 >= num_m) break;        // the last tile's second half lies past T (and past Y)
+        const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * BN);
+        // this thread's accumulator row is token 128 m128 + 32 q + lane
+        const size_t yrow = (size_t)(m128 * BM + q * 32 + lane) * (size_t)ldy;
+        float sum = 0.0f;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 32) {
+          float v[32];
+          if constexpr (EPI == kEpiSubY) {
+            // fetch the cached fp16 outputs first, so their latency overlaps the TMEM read
+            const uint4 *yp = reinterpret_cast<const uint4 *>(
+                Y + yrow + (size_t)(((int64_t)n_blk * BN) % y_cols) + c);
+            uint4 yv[4];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) yv[u] = __ldg(yp + u);
-          tmem_ld_32x32b_x32(taddr + (uint32_t)c, v);
-          tmem_ld_wait();
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const uint32_t yw[4] = {yv[u].x, yv[u].y, yv[u].z, yv[u].w};
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-              const float2 yf = __half22float2(*reinterpret_cast<const __half2 *>(&yw[h]));
-              const float d0 = v[8 * u + 2 * h] - yf.x, d1 = v[8 * u + 2 * h + 1] - yf.y;
-              sum = fmaf(d0, d0, sum);
-              sum = fmaf(d1, d1, sum);
-            }
-          }
-        } else {
-          tmem_ld_32x32b_x32(taddr + (uint32_t)c, v);
-          tmem_ld_wait();
-          if constexpr (EPI == kEpiStoreY) {
-            uint4 *yp = reinterpret_cast<uint4 *>(Y + yrow + (size_t)n_blk * BN + c);
+            for (int u = 0; u < 4; ++u) yv[u] = __ldg(yp + u);
+            tmem_ld_32x32b_x32(taddr + (uint32_t)c, v);
+            tmem_ld_wait();
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
-              uint32_t hw[4];
+              const uint32_t yw[4] = {yv[u].x, yv[u].y, yv[u].z, yv[u].w};
 #pragma unroll
-              for (int h = 0; h < 4; ++h) {
-                const __half2 hv = __floats2half2_rn(v[8 * u + 2 * h], v[8 * u + 2 * h + 1]);
-                hw[h] = *reinterpret_cast<const uint32_t *>(&hv);
+              for (int e = 0; e < 4; ++e) {
+                const float2 yf = __half22float2(*reinterpret_cast<const __half2 *>(&yw[e]));
+                const float d0 = v[8 * u + 2 * e] - yf.x, d1 = v[8 * u + 2 * e + 1] - yf.y;
+                sum = fmaf(d0, d0, sum);
+                sum = fmaf(d1, d1, sum);
               }
-              yp[u] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
             }
           } else {
+            tmem_ld_32x32b_x32(taddr + (uint32_t)c, v);
+            tmem_ld_wait();
+            if constexpr (EPI == kEpiStoreY) {
+              uint4 *yp = reinterpret_cast<uint4 *>(Y + yrow + (size_t)n_blk * BN + c);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) sum = fmaf(v[i], v[i], sum);
+              for (int u = 0; u < 4; ++u) {
+                uint32_t hw[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                  const __half2 hv = __floats2half2_rn(v[8 * u + 2 * e], v[8 * u + 2 * e + 1]);
+                  hw[e] = *reinterpret_cast<const uint32_t *>(&hv);
+                }
+                yp[u] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) sum = fmaf(v[i], v[i], sum);
+            }
           }
         }
+        sums[h] = sum;
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tail->tempty[acc]);
       if constexpr (EPI != kEpiStoreY) {
-        double ds = (double)sum;
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) ds += __shfl_xor_sync(0xffffffffu, ds, off);
-        if (lane == 0) partials[((size_t)n_blk * num_m + m_blk) * 4 + q] = ds;
+        for (int h = 0; h < 2; ++h) {
+          double ds = (double)sums[h];
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) ds += __shfl_xor_sync(0xffffffffu, ds, off);
+          const int m128 = 2 * m_blk + h;
+          if (lane == 0 && m128 < num_m) partials[((size_t)n_blk * num_m + m128) * 4 + q] = ds;
+        }
       }
     }
   }
@@ -337,7 +359,7 @@ static cudaError_t launch_gemm_epi(const CUtensorMap &tmA, const CUtensorMap &tm
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kGemmSmemBytes);
   if (e != cudaSuccess) return e;
-  const int tiles = sh.num_m * sh.num_n;
+  const int tiles = ((sh.num_m + 1) / 2) * sh.num_n;  // 256-row tiles
   const int grid = tiles < num_sms ? tiles : num_sms;
   search_gemm_kernel<EPI><<<grid, 192, kGemmSmemBytes, stream>>>(
       tmA, tmB, sh.num_m, sh.num_n, sh.num_kb, partials, Y, ldy, y_cols, st, max_polls);
@@ -365,7 +387,7 @@ cudaError_t launch_search_gemm(const __half *X, int64_t ldx, const __half *dW,
                                int64_t ldy, DevStatus *st, uint32_t max_polls, int num_sms,
                                cudaStream_t stream) {
   CUtensorMap tmA, tmB;
-  cudaError_t e = make_tmap_f16_box(&tmA, X, sh.T, sh.in, ldx, BK, BM);
+  cudaError_t e = make_tmap_f16_box(&tmA, X, sh.T, sh.in, ldx, BK, BM2);
   if (e != cudaSuccess) return e;
   e = make_tmap_f16_box(&tmB, dW, sh.rows_b, sh.in, sh.in, BK, BN);
   if (e != cudaSuccess) return e;
@@ -381,7 +403,7 @@ cudaError_t launch_ref_output(const __half *X, int64_t T, int64_t in, int64_t ld
                               uint32_t max_polls, int num_sms, cudaStream_t stream) {
   if (out_pad % BN != 0 || in % BK != 0) return cudaErrorInvalidValue;
   CUtensorMap tmA, tmB;
-  cudaError_t e = make_tmap_f16_box(&tmA, X, T, in, ldx, BK, BM);
+  cudaError_t e = make_tmap_f16_box(&tmA, X, T, in, ldx, BK, BM2);
   if (e != cudaSuccess) return e;
   e = make_tmap_f16_box(&tmB, W, out, in, in, BK, BN);  // rows >= out read as zeros
   if (e != cudaSuccess) return e;

@@ -53,6 +53,7 @@ constexpr int QW_DEQ = 6;                      // first dequantising warp
 constexpr int QN_DEQ = 8;                      // dequantising warps (two per sub-partition)
 constexpr int Q_WORDS = QBK * (QBN / 8) / (QN_DEQ * 32);  // words per thread per K tile (8)
 constexpr int Q_THREADS = (QW_DEQ + QN_DEQ) * 32;         // 448: up to 128 registers
+static_assert(QN_DEQ % 8 == 0 && Q_WORDS % 2 == 0 && QN_DEQ * Q_WORDS == QBK, "dequant split");
 constexpr uint32_t Q_DRAIN = 1u << 22;
 // kind::f16, fp16 A/B, fp32 D, A K-major, B MN-major, N = 256, M = 128
 constexpr uint32_t IDESC_Q = (1u << 4) | (1u << 16) | ((uint32_t)(QBN >> 3) << 17) |
@@ -220,9 +221,10 @@ __global__ void __launch_bounds__(Q_THREADS, 1) w4a16_gemm_kernel(
     // ------------------------------------------------------------ dequantise W
     const int dt = threadIdx.x - QW_DEQ * 32;  // 0..255
     const int col = dt & 31;                   // word column: outputs 8 col .. 8 col + 7
-    const int row0 = dt >> 5;                  // input-channel rows row0 + 8 i (so k & 7 = row0)
+    const int row0 = dt >> 5;                  // input-channel rows row0 + QN_DEQ i
+    // (QN_DEQ is a multiple of 8, so every row of this thread has k & 7 = row0 & 7)
     const uint32_t chunk_off = (uint32_t)(col >> 3) * QB_BOX + (uint32_t)row0 * 128u +
-                               ((uint32_t)((col & 7) ^ row0) << 4);
+                               ((uint32_t)((col & 7) ^ (row0 & 7)) << 4);
     int stage = 0;
     uint32_t phase = 0;
     // the (tile, K step) sequence of this CTA, one step ahead for the word loads
@@ -290,12 +292,14 @@ __global__ void __launch_bounds__(Q_THREADS, 1) w4a16_gemm_kernel(
       // loads the compiler cannot prove disjoint, so loads come first explicitly
       uint32_t wv[Q_WORDS];
 #pragma unroll
-      for (int i = 0; i < Q_WORDS; ++i) wv[i] = wsrc[i * 8 * 32];
+      for (int i = 0; i < Q_WORDS; ++i) wv[i] = wsrc[i * QN_DEQ * 32];
 #pragma unroll
       for (int i = 0; i < Q_WORDS; ++i) {
-        // row row0 + 8 i lies in 0..31 for i < 4 and in 32..63 for i >= 4
-        const uint4 v = dequant_word(wv[i], zp[i < 4 ? 0 : 1], sp[i < 4 ? 0 : 1]);
-        *reinterpret_cast<uint4 *>(bst + i * 8 * 128) = v;  // row row0 + 8 i, same swizzle
+        // row row0 + QN_DEQ i lies in 0..31 (zero and scale group h = 0) for the
+        // first half of i and in 32..63 (h = 1) for the second
+        constexpr int kHalf = Q_WORDS / 2;
+        const uint4 v = dequant_word(wv[i], zp[i < kHalf ? 0 : 1], sp[i < kHalf ? 0 : 1]);
+        *reinterpret_cast<uint4 *>(bst + i * QN_DEQ * 128) = v;  // row row0 + QN_DEQ i, same swizzle
       }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       __syncwarp();
