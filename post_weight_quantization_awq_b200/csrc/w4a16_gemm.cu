@@ -42,6 +42,7 @@ namespace awq {
 
 namespace {
 constexpr int QBM = 256, QMM = 128, QBN = 256, QBK = 64, QSTAGES = 3;  // CTA rows, MMA rows
+constexpr int QW_STAGES = 4;  // packed-word stages: their own ring, refilled as soon as read
 constexpr uint32_t QA_BYTES = QBM * QBK * 2;   // 32 KiB
 constexpr uint32_t QA_HALF = QMM * QBK * 2;    // rows 128..255 of the X tile start here
 constexpr uint32_t QB_BOX = QBK * 128;         // 64 input channels x 64 outputs (8 KiB)
@@ -49,10 +50,11 @@ constexpr uint32_t QB_BYTES = 4 * QB_BOX;      // 32 KiB
 constexpr uint32_t QW_BYTES = QBK * (QBN / 8) * 4;  // packed words of a B tile (8 KiB)
 constexpr uint32_t QTMEM_COLS = 512;
 constexpr int QGROUP_M = 16;
-constexpr int QW_DEQ = 6;                      // first dequantising warp
+constexpr int QW_WPROD = 6;                    // the packed words' TMA producer
+constexpr int QW_DEQ = 7;                      // first dequantising warp
 constexpr int QN_DEQ = 8;                      // dequantising warps (two per sub-partition)
 constexpr int Q_WORDS = QBK * (QBN / 8) / (QN_DEQ * 32);  // words per thread per K tile (8)
-constexpr int Q_THREADS = (QW_DEQ + QN_DEQ) * 32;         // 448: up to 128 registers
+constexpr int Q_THREADS = (QW_DEQ + QN_DEQ) * 32;         // 480: up to 136 registers
 static_assert(QN_DEQ % 8 == 0 && Q_WORDS % 2 == 0 && QN_DEQ * Q_WORDS == QBK, "dequant split");
 constexpr uint32_t Q_DRAIN = 1u << 22;
 // kind::f16, fp16 A/B, fp32 D, A K-major, B MN-major, N = 256, M = 128
@@ -60,14 +62,18 @@ constexpr uint32_t IDESC_Q = (1u << 4) | (1u << 16) | ((uint32_t)(QBN >> 3) << 1
                              ((uint32_t)(QMM >> 4) << 24);
 
 struct __align__(8) QTail {
-  uint64_t ld[QSTAGES];     // TMA bytes of the X tile and the packed words
-  uint64_t full[QSTAGES];   // one arrival per dequantising warp
-  uint64_t empty[QSTAGES];  // MMA commit
+  uint64_t ld[QSTAGES];       // TMA bytes of the X tile
+  uint64_t full[QSTAGES];     // the B tile: one arrival per dequantising warp
+  uint64_t empty[QSTAGES];    // MMA commit: X and B of the stage are free
+  uint64_t wld[QW_STAGES];    // TMA bytes of the packed words
+  uint64_t wempty[QW_STAGES]; // words read: one arrival per dequantising warp
   uint64_t tfull[2], tempty[2], mma_done;
   uint32_t tmem_base;
   int abort_flag;
 };
-constexpr size_t kQSmemBytes = 1024 + QSTAGES * (QA_BYTES + QB_BYTES + QW_BYTES) + sizeof(QTail);
+constexpr size_t kQSmemBytes =
+    1024 + QSTAGES * (QA_BYTES + QB_BYTES) + QW_STAGES * QW_BYTES + sizeof(QTail);
+static_assert(kQSmemBytes <= 232448, "shared memory per CTA");
 
 // MN-major B with 128-byte swizzling: 64 outputs (128 B) per input-channel row,
 // 8-row core groups 1024 B apart (SBO), 64-output boxes QB_BOX apart (LBO).
@@ -153,7 +159,7 @@ __global__ void __launch_bounds__(Q_THREADS, 1) w4a16_gemm_kernel(
   uint8_t *sA = smem;
   uint8_t *sB = smem + QSTAGES * QA_BYTES;
   uint8_t *sW = sB + QSTAGES * QB_BYTES;
-  QTail *tail = reinterpret_cast<QTail *>(sW + QSTAGES * QW_BYTES);
+  QTail *tail = reinterpret_cast<QTail *>(sW + QW_STAGES * QW_BYTES);
   volatile int *abort_flag = &tail->abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int num_tiles = num_m * num_n * splits;
@@ -165,6 +171,10 @@ __global__ void __launch_bounds__(Q_THREADS, 1) w4a16_gemm_kernel(
       mbar_init(&tail->full[s], QN_DEQ);
       mbar_init(&tail->empty[s], 1);
     }
+    for (int s = 0; s < QW_STAGES; ++s) {
+      mbar_init(&tail->wld[s], 1);
+      mbar_init(&tail->wempty[s], QN_DEQ);
+    }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tail->tfull[a], 1);
       mbar_init(&tail->tempty[a], 4);
@@ -173,10 +183,8 @@ __global__ void __launch_bounds__(Q_THREADS, 1) w4a16_gemm_kernel(
     tail->abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tmX);
-    tma_prefetch_desc(&tmW);
-  }
+  if (warp == 0 && lane == 0) tma_prefetch_desc(&tmX);
+  if (warp == QW_WPROD && lane == 0) tma_prefetch_desc(&tmW);
   if (warp == 1) {
     tmem_alloc(&tail->tmem_base, QTMEM_COLS);
     tmem_relinquish();
@@ -201,9 +209,8 @@ __global__ void __launch_bounds__(Q_THREADS, 1) w4a16_gemm_kernel(
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&tail->ld[stage], QA_BYTES + QW_BYTES);
+          mbar_arrive_expect_tx(&tail->ld[stage], QA_BYTES);
           tma_load_2d(sA + stage * QA_BYTES, &tmX, &tail->ld[stage], kb * QBK, m_blk * QBM);
-          tma_load_2d(sW + stage * QW_BYTES, &tmW, &tail->ld[stage], n_blk * (QBN / 8), kb * QBK);
           issued |= 1u << stage;
           issued_parity = (issued_parity & ~(1u << stage)) | (phase << stage);
           if (++stage == QSTAGES) {
@@ -217,6 +224,38 @@ __global__ void __launch_bounds__(Q_THREADS, 1) w4a16_gemm_kernel(
           if (issued & (1u << s))
             (void)mbar_wait_bounded(&tail->ld[s], (issued_parity >> s) & 1u, Q_DRAIN, nullptr);
     }
+  } else if (warp == QW_WPROD) {
+    // ------------------------------------------------------------ packed words by TMA
+    // Their own ring: a slot is refilled as soon as the dequantising warps have
+    // read it, so the words of a step land long before its B slot frees.
+    if (lane == 0) {
+      int ws = 0;
+      uint32_t wphase = 0, issued = 0, issued_parity = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
+        int m_blk, n_blk, sp, kb0, kb1;
+        q_tile_split(tile, num_m, num_n, splits, num_kb, m_blk, n_blk, sp, kb0, kb1);
+        for (int kb = kb0; kb < kb1; ++kb) {
+          if (!mbar_wait_long(&tail->wempty[ws], wphase ^ 1u, max_polls, abort_flag)) {
+            q_abort(tail, st, 0xD50u + ws);
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&tail->wld[ws], QW_BYTES);
+          tma_load_2d(sW + ws * QW_BYTES, &tmW, &tail->wld[ws], n_blk * (QBN / 8), kb * QBK);
+          issued |= 1u << ws;
+          issued_parity = (issued_parity & ~(1u << ws)) | (wphase << ws);
+          if (++ws == QW_STAGES) {
+            ws = 0;
+            wphase ^= 1u;
+          }
+        }
+      }
+      if (!ok || *abort_flag)
+        for (int s = 0; s < QW_STAGES; ++s)
+          if (issued & (1u << s))
+            (void)mbar_wait_bounded(&tail->wld[s], (issued_parity >> s) & 1u, Q_DRAIN, nullptr);
+    }
   } else if (warp >= QW_DEQ) {
     // ------------------------------------------------------------ dequantise W
     const int dt = threadIdx.x - QW_DEQ * 32;  // 0..255
@@ -225,8 +264,8 @@ __global__ void __launch_bounds__(Q_THREADS, 1) w4a16_gemm_kernel(
     // (QN_DEQ is a multiple of 8, so every row of this thread has k & 7 = row0 & 7)
     const uint32_t chunk_off = (uint32_t)(col >> 3) * QB_BOX + (uint32_t)row0 * 128u +
                                ((uint32_t)((col & 7) ^ (row0 & 7)) << 4);
-    int stage = 0;
-    uint32_t phase = 0;
+    int stage = 0, ws = 0;
+    uint32_t phase = 0, wphase = 0;
     // the (tile, K step) sequence of this CTA, one step ahead for the word loads
     int tile = blockIdx.x, kb = 0, kb_end = 0;
     // this thread's qweight column in tile tl, and the tile's K steps
@@ -274,10 +313,12 @@ __global__ void __launch_bounds__(Q_THREADS, 1) w4a16_gemm_kernel(
         nib_pairs(zw[h], zp[h]);
         scale_pairs(sc[h], sp[h]);
       }
-      // the stage's X tile and packed words have landed (which also means the
-      // MMAs that last read this stage are done: the loads waited for them)
+      // the step's packed words have landed, and the MMAs that last read this
+      // B slot are done
       int got = 1;
-      if (lane == 0) got = mbar_wait_long(&tail->ld[stage], phase, max_polls, abort_flag);
+      if (lane == 0)
+        got = mbar_wait_long(&tail->wld[ws], wphase, max_polls, abort_flag) &&
+              mbar_wait_long(&tail->empty[stage], phase ^ 1u, max_polls, abort_flag);
       got = __shfl_sync(0xffffffffu, got, 0);
       if (!got) {
         if (lane == 0) q_abort(tail, st, 0xD10u + stage);
@@ -286,7 +327,7 @@ __global__ void __launch_bounds__(Q_THREADS, 1) w4a16_gemm_kernel(
       }
       // words past `out` were filled with zeros by TMA; their zeros and scales
       // are zero too, so they give 0
-      const uint32_t *wsrc = reinterpret_cast<const uint32_t *>(sW + stage * QW_BYTES) + row0 * 32 + col;
+      const uint32_t *wsrc = reinterpret_cast<const uint32_t *>(sW + ws * QW_BYTES) + row0 * 32 + col;
       uint8_t *bst = sB + stage * QB_BYTES + chunk_off;
       // all eight words first: the B stores below may not be reordered above
       // loads the compiler cannot prove disjoint, so loads come first explicitly
@@ -303,10 +344,17 @@ __global__ void __launch_bounds__(Q_THREADS, 1) w4a16_gemm_kernel(
       }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tail->full[stage]);
+      if (lane == 0) {
+        mbar_arrive(&tail->wempty[ws]);  // every word of the slot was used above
+        mbar_arrive(&tail->full[stage]);
+      }
       if (++stage == QSTAGES) {
         stage = 0;
         phase ^= 1u;
+      }
+      if (++ws == QW_STAGES) {
+        ws = 0;
+        wphase ^= 1u;
       }
       tile = ntile;
       kb = nkb;

@@ -8,6 +8,7 @@ last on purpose: if it fails, a run that stops at the first failure has
 already run every other test.  It passes both alone and after the others."""
 
 import ctypes
+import gc
 
 import numpy as np
 import pytest
@@ -67,6 +68,7 @@ def test_noalloc_matches_workspace_entry_twice(T, inn, out, exact):
     for call in range(2):
         idx.fill_(255)
         err.fill_(float("nan"))
+        gc.collect()
         torch.cuda.synchronize()
         before = (torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated(),
                   torch.cuda.memory_reserved())
@@ -74,9 +76,10 @@ def test_noalloc_matches_workspace_entry_twice(T, inn, out, exact):
         awq.awq_device_status(None)  # no device-side failure recorded
         after = (torch.cuda.mem_get_info()[0], torch.cuda.memory_allocated(),
                  torch.cuda.memory_reserved())
-        # nothing was allocated through torch; after the first call's set-up,
-        # no device memory at all
-        assert after[1:] == before[1:], (call, before, after)
+        # torch's allocator did not grow (the call allocates nothing through it;
+        # unrelated tensors may be freed meanwhile); after the first call's
+        # set-up, the device's free memory did not shrink either
+        assert after[1] <= before[1] and after[2] <= before[2], (call, before, after)
         if call == 1:
             assert after[0] >= before[0], (before, after)
         got_idx, got_err = idx.cpu().numpy(), err.cpu().numpy()
