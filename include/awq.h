@@ -317,10 +317,14 @@ awq_status awq_search_clip_grams(const void *W, int64_t out, int64_t in, const f
  *   X        device fp16 [T, in], row stride ldx
  *   qweight  device int32 [in, out/8]; qzeros int32 [in/g, out/8]; scales fp16 [in/g, out]
  *   Y        device fp16 [T, out] (output), row stride ldy (multiple of 8)
- *   ws       at least 256 bytes (status word); with awq_w4a16_workspace_size()
- *            bytes, few tokens (output tiles filling under half of the SMs)
- *            are computed with split-K: fp32 partial sums of K ranges in the
- *            workspace, added in a fixed order and rounded to fp16 once
+ *   ws       at least 256 bytes (status word), with which the weights are
+ *            dequantised tile by tile inside the GEMM.  With
+ *            awq_w4a16_workspace_size() bytes: few tokens (output tiles
+ *            filling under half of the SMs) are computed with split-K (fp32
+ *            partial sums of K ranges in the workspace, added in a fixed order
+ *            and rounded to fp16 once); 1024 tokens or more dequantise the
+ *            weights once into the workspace (the same RN16((q - z) scale)
+ *            values) and run one fp16 GEMM on the tensor cores
  * Uses cfg->group_size (32, 64 or 128); requires in % 64 == 0 and out % 32 == 0
  * (the packed words of a row are staged by TMA, whose row stride must be a
  * multiple of 16 bytes). */
@@ -329,8 +333,10 @@ awq_status awq_w4a16_gemm(const void *X, int64_t T, int64_t in, int64_t ldx, con
                           const awq_config *cfg, void *Y, int64_t ldy, void *ws, size_t ws_bytes,
                           awq_stream_t stream);
 
-/* Workspace bytes with which awq_w4a16_gemm uses split-K for this shape (256
- * when it would not split).  Returns 0 when the arguments are invalid. */
+/* Workspace bytes with which awq_w4a16_gemm runs its fastest form for this
+ * shape: 256 + in * out * 2 (the fp16 weights) from 1024 tokens on, the
+ * split-K partial sums for few tokens, else 256.  Returns 0 when the
+ * arguments are invalid. */
 size_t awq_w4a16_workspace_size(int64_t T, int64_t in, int64_t out, const awq_config *cfg);
 
 /* Synchronises `stream`, then returns and clears the device status recorded in

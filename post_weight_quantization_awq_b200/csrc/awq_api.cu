@@ -242,6 +242,17 @@ Fault fault_mode() {
   return Fault::kNone;
 }
 
+// From this many tokens on, the W4A16 product dequantises the weights once
+// into the workspace and runs one fp16 GEMM (when the workspace holds them):
+// the conversion then costs in x out work once instead of once per 256-token
+// tile, and the GEMM runs at the tensor cores' rate.
+constexpr int64_t kW4DequantMinT = 1024;
+
+// status word plus the fp16 weights [out, in]
+size_t w4a16_dequant_ws_bytes(int64_t in, int64_t out) {
+  return kHeader + align256(sizeof(__half) * (size_t)in * (size_t)out);
+}
+
 // status word plus the fp32 partial sums [splits][T][out] of a split-K W4A16 GEMM
 size_t w4a16_ws_bytes(int64_t T, int64_t out, int splits) {
   return kHeader + align256(sizeof(float) * (size_t)splits * (size_t)T * (size_t)out);
@@ -725,11 +736,26 @@ awq_status awq_w4a16_gemm(const void *X, int64_t T, int64_t in, int64_t ldx, con
   AWQ_LAUNCH_GATE();
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   DevStatus *dst = static_cast<DevStatus *>(ws);
+  AWQ_TRY_CUDA(cudaMemsetAsync(dst, 0, sizeof(DevStatus), cs), "workspace reset");
+  // many tokens, with room for the fp16 weights: dequantise once, one fp16 GEMM
+  if (T >= kW4DequantMinT && ws_bytes >= w4a16_dequant_ws_bytes(in, out)) {
+    __half *Wd = reinterpret_cast<__half *>(static_cast<uint8_t *>(ws) + kHeader);
+    {
+      ProfScope p("w4a16_dequant", cs);
+      AWQ_TRY_CUDA(launch_w4a16_dequant(qweight, qzeros, static_cast<const __half *>(scales), in, out,
+                                        cfg->group_size, Wd, cs),
+                   "w4a16_dequant launch");
+    }
+    ProfScope p("w4a16_gemm", cs);
+    AWQ_TRY_CUDA(launch_gemm_store(static_cast<const __half *>(X), T, in, ldx, Wd, out,
+                                   static_cast<__half *>(Y), ldy, dst, poll_cap(), num_sms_current(), cs),
+                 "w4a16 fp16 GEMM launch");
+    return AWQ_OK;
+  }
   // split-K for few tokens, when the workspace holds the fp32 partial sums
   int splits = w4a16_splits(T, in, out, num_sms_current());
   if (splits > 1 && ws_bytes < w4a16_ws_bytes(T, out, splits)) splits = 1;
   float *partials = splits > 1 ? reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + kHeader) : nullptr;
-  AWQ_TRY_CUDA(cudaMemsetAsync(dst, 0, sizeof(DevStatus), cs), "workspace reset");
   ProfScope p("w4a16_gemm", cs);
   AWQ_TRY_CUDA(launch_w4a16_gemm(static_cast<const __half *>(X), T, in, ldx, qweight, qzeros,
                                  static_cast<const __half *>(scales), out, cfg->group_size,
@@ -748,6 +774,7 @@ size_t awq_w4a16_workspace_size(int64_t T, int64_t in, int64_t out, const awq_co
   }
   if (check_cfg(cfg) != AWQ_OK) return 0;
   if (check_shape(T, in, out, cfg) != AWQ_OK) return 0;
+  if (T >= kW4DequantMinT) return w4a16_dequant_ws_bytes(in, out);
   const int splits = w4a16_splits(T, in, out, num_sms_current());
   return splits > 1 ? w4a16_ws_bytes(T, out, splits) : kHeader;
 }

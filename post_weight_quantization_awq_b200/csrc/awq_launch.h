@@ -70,6 +70,12 @@ cudaError_t launch_search_gemm(const __half *X, int64_t ldx, const __half *dW,
 cudaError_t launch_ref_output(const __half *X, int64_t T, int64_t in, int64_t ldx, const __half *W,
                               int64_t out, int64_t out_pad, __half *Y, DevStatus *st,
                               uint32_t max_polls, int num_sms, cudaStream_t stream);
+// Y = RN16(X W^T) into the caller's Y [T, out] (row stride ldy): the scored
+// GEMM's tiles with a bounded store epilogue; W fp16 [out, in] row-major,
+// in % 64 == 0, out % 8 == 0.
+cudaError_t launch_gemm_store(const __half *X, int64_t T, int64_t in, int64_t ldx, const __half *W,
+                              int64_t out, __half *Y, int64_t ldy, DevStatus *st, uint32_t max_polls,
+                              int num_sms, cudaStream_t stream);
 constexpr int kGemmBM = 128, kGemmBN = 256, kGemmBK = 64;
 
 // 2-D fp16 TMA descriptor over a row-major [rows, cols] matrix (row stride
@@ -131,6 +137,11 @@ cudaError_t launch_w4a16_gemm(const __half *X, int64_t T, int64_t in, int64_t ld
 // output tiles fill at least half of the SMs, else enough K splits (each of
 // at least 4 K steps of 64 channels) to occupy them.
 int w4a16_splits(int64_t T, int64_t in, int64_t out, int num_sms);
+// The dequantised weights of a packed layer, Wd [out, in] fp16 row-major,
+// Wd[o][j] = RN16((q - z) scale): the operand of the W4A16 product for many
+// tokens (dequantised once, then one fp16 GEMM).
+cudaError_t launch_w4a16_dequant(const int32_t *qweight, const int32_t *qzeros, const __half *scales,
+                                 int64_t in, int64_t out, int group, __half *Wd, cudaStream_t stream);
 
 // K8: v[j][:] = RN16(RN32(v[j][:]) / s_j).
 cudaError_t launch_fold(__half *v, int64_t rows, int64_t cols, const float *s, cudaStream_t stream);

@@ -526,14 +526,16 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
           }
           const bool store = live && c < n_clip;  // past n_clip: lane 0's ratio, not stored
           // (q - z) = clamp(rne(wt / delta), -z, qmax - z), proposed from the
-          // approximate reciprocal and proven by the remainder
+          // approximate reciprocal (one FMA rounds wt rc + 1.5 2^23 straight to
+          // an integer) and proven by the remainder
           float2 kq[4];
           float rmax = 0.0f;
 #pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            kq[h] = rne2_small(__fmul2_rn(wt[h], make_float2(rc, rc)));
+          for (int h = 0; h < 4; ++h) {  // 12582912 = 1.5 2^23
+            kq[h] = __fadd2_rn(__ffma2_rn(wt[h], make_float2(rc, rc), make_float2(12582912.0f, 12582912.0f)),
+                               make_float2(-12582912.0f, -12582912.0f));
             const float2 rem = __ffma2_rn(make_float2(-kq[h].x, -kq[h].y), make_float2(dl, dl), wt[h]);
-            rmax = fmaxf(rmax, fmaxf(fabsf(rem.x), fabsf(rem.y)));
+            rmax = fmax3(rmax, fabsf(rem.x), fabsf(rem.y));
           }
           if (!(rmax < hl)) {
 #pragma unroll

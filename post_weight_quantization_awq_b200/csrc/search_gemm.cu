@@ -95,7 +95,7 @@ __global__ void __launch_bounds__(192, 1)
     search_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                        const __grid_constant__ CUtensorMap tmB, int num_m, int num_n, int num_kb,
                        double *__restrict__ partials, __half *__restrict__ Y, int64_t ldy,
-                       int64_t y_cols, DevStatus *st, uint32_t max_polls) {
+                       int64_t y_cols, int64_t y_rows, DevStatus *st, uint32_t max_polls) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -270,9 +270,13 @@ __global__ void __launch_bounds__(192, 1)
             tmem_ld_32x32b_x32(taddr + (uint32_t)c, v);
             tmem_ld_wait();
             if constexpr (EPI == kEpiStoreY) {
-              uint4 *yp = reinterpret_cast<uint4 *>(Y + yrow + (size_t)n_blk * BN + c);
+              // rows from y_rows on and columns from y_cols on are not stored
+              const int64_t token = (int64_t)m128 * BM + q * 32 + lane;
+              const int64_t col0 = (int64_t)n_blk * BN + c;
+              uint4 *yp = reinterpret_cast<uint4 *>(Y + yrow + col0);
 #pragma unroll
               for (int u = 0; u < 4; ++u) {
+                if (token >= y_rows || col0 + 8 * u >= y_cols) break;
                 uint32_t hw[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
@@ -353,7 +357,8 @@ cudaError_t make_tmap_f16_box(CUtensorMap *m, const void *base, int64_t rows, in
 template <int EPI>
 static cudaError_t launch_gemm_epi(const CUtensorMap &tmA, const CUtensorMap &tmB,
                                    const SearchGemmShape &sh, double *partials, __half *Y,
-                                   int64_t ldy, int64_t y_cols, DevStatus *st, uint32_t max_polls,
+                                   int64_t ldy, int64_t y_cols, int64_t y_rows, DevStatus *st,
+                                   uint32_t max_polls,
                                    int num_sms, cudaStream_t stream) {
   cudaError_t e = cudaFuncSetAttribute(search_gemm_kernel<EPI>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -362,7 +367,7 @@ static cudaError_t launch_gemm_epi(const CUtensorMap &tmA, const CUtensorMap &tm
   const int tiles = ((sh.num_m + 1) / 2) * sh.num_n;  // 256-row tiles
   const int grid = tiles < num_sms ? tiles : num_sms;
   search_gemm_kernel<EPI><<<grid, 192, kGemmSmemBytes, stream>>>(
-      tmA, tmB, sh.num_m, sh.num_n, sh.num_kb, partials, Y, ldy, y_cols, st, max_polls);
+      tmA, tmB, sh.num_m, sh.num_n, sh.num_kb, partials, Y, ldy, y_cols, y_rows, st, max_polls);
   return cudaGetLastError();
 }
 
@@ -392,9 +397,9 @@ cudaError_t launch_search_gemm(const __half *X, int64_t ldx, const __half *dW,
   e = make_tmap_f16_box(&tmB, dW, sh.rows_b, sh.in, sh.in, BK, BN);
   if (e != cudaSuccess) return e;
   if (Y)
-    return launch_gemm_epi<kEpiSubY>(tmA, tmB, sh, partials, const_cast<__half *>(Y), ldy, ldy, st,
-                                     max_polls, num_sms, stream);
-  return launch_gemm_epi<kEpiSse>(tmA, tmB, sh, partials, nullptr, 0, 1, st, max_polls, num_sms,
+    return launch_gemm_epi<kEpiSubY>(tmA, tmB, sh, partials, const_cast<__half *>(Y), ldy, ldy, 0,
+                                     st, max_polls, num_sms, stream);
+  return launch_gemm_epi<kEpiSse>(tmA, tmB, sh, partials, nullptr, 0, 1, 0, st, max_polls, num_sms,
                                   stream);
 }
 
@@ -414,8 +419,28 @@ cudaError_t launch_ref_output(const __half *X, int64_t T, int64_t in, int64_t ld
   sh.num_m = (int)((T + BM - 1) / BM);
   sh.num_n = (int)(out_pad / BN);
   sh.num_kb = (int)(in / BK);
-  return launch_gemm_epi<kEpiStoreY>(tmA, tmB, sh, nullptr, Y, out_pad, out_pad, st, max_polls,
-                                     num_sms, stream);
+  return launch_gemm_epi<kEpiStoreY>(tmA, tmB, sh, nullptr, Y, out_pad, out_pad,
+                                     (int64_t)sh.num_m * BM, st, max_polls, num_sms, stream);
+}
+
+cudaError_t launch_gemm_store(const __half *X, int64_t T, int64_t in, int64_t ldx, const __half *W,
+                              int64_t out, __half *Y, int64_t ldy, DevStatus *st, uint32_t max_polls,
+                              int num_sms, cudaStream_t stream) {
+  if (in % BK != 0 || out % 8 != 0) return cudaErrorInvalidValue;
+  CUtensorMap tmA, tmB;
+  cudaError_t e = make_tmap_f16_box(&tmA, X, T, in, ldx, BK, BM2);  // rows >= T read as zeros
+  if (e != cudaSuccess) return e;
+  e = make_tmap_f16_box(&tmB, W, out, in, in, BK, BN);  // rows >= out read as zeros
+  if (e != cudaSuccess) return e;
+  SearchGemmShape sh;
+  sh.T = T;
+  sh.in = in;
+  sh.rows_b = out;
+  sh.num_m = (int)((T + BM - 1) / BM);
+  sh.num_n = (int)((out + BN - 1) / BN);
+  sh.num_kb = (int)(in / BK);
+  return launch_gemm_epi<kEpiStoreY>(tmA, tmB, sh, nullptr, Y, ldy, out, T, st, max_polls, num_sms,
+                                     stream);
 }
 
 // ---------------------------------------------------------------------------

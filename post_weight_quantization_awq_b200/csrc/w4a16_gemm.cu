@@ -480,6 +480,59 @@ __global__ void __launch_bounds__(Q_THREADS, 1) w4a16_gemm_kernel(
   }
 }
 
+// The dequantised weights Wd [out, in] fp16, Wd[o][j] = RN16((q - z) scale) --
+// the values the GEMM above builds tile by tile -- written once for a product
+// with many tokens.  A block turns a 128-input x 64-output tile of packed
+// words (input-major) into output-major rows through shared memory, so both
+// the word loads and the 16-byte row stores are contiguous.
+__global__ void __launch_bounds__(256) w4a16_dequant_kernel(
+    const int32_t *__restrict__ qweight, const int32_t *__restrict__ qzeros,
+    const __half *__restrict__ scales, int64_t in, int64_t out, int group, __half *__restrict__ Wd) {
+  constexpr int TJ = 128, TO = 64, WPR = TO / 8;  // inputs, outputs, words per input row
+  __shared__ __align__(16) __half tile[TO][TJ + 8];
+  const int64_t j0 = (int64_t)blockIdx.x * TJ, o0 = (int64_t)blockIdx.y * TO;
+  const int64_t words = out / 8;
+#pragma unroll
+  for (int i = 0; i < TJ * WPR / 256; ++i) {
+    const int w = threadIdx.x + 256 * i;
+    const int jj = w / WPR, ow = w % WPR;  // input row of the tile, word column
+    const int64_t j = j0 + jj, wc = o0 / 8 + ow;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (j < in && wc < words) {
+      const int64_t gi = j / group;
+      __half2 zp[4], sp[4];
+      nib_pairs((uint32_t)__ldg(qzeros + gi * words + wc), zp);
+      scale_pairs(__ldg(reinterpret_cast<const uint4 *>(scales + gi * out + 8 * wc)), sp);
+      v = dequant_word((uint32_t)__ldg(qweight + j * words + wc), zp, sp);
+    }
+    // v holds outputs 0,4,1,5,2,6,3,7 of the word
+    const uint32_t h[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+      const __half2 pr = *reinterpret_cast<const __half2 *>(&h[p]);
+      tile[8 * ow + p][jj] = __low2half(pr);
+      tile[8 * ow + p + 4][jj] = __high2half(pr);
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < TO * (TJ / 8) / 256; ++i) {
+    const int c = threadIdx.x + 256 * i;
+    const int oo = c / (TJ / 8), jc = c % (TJ / 8);  // output row, 8-input chunk
+    const int64_t o = o0 + oo, j = j0 + 8 * jc;
+    if (o < out && j < in)  // in % 64 == 0: a chunk is whole
+      *reinterpret_cast<uint4 *>(Wd + o * in + j) = *reinterpret_cast<const uint4 *>(&tile[oo][8 * jc]);
+  }
+}
+
+cudaError_t launch_w4a16_dequant(const int32_t *qweight, const int32_t *qzeros, const __half *scales,
+                                 int64_t in, int64_t out, int group, __half *Wd, cudaStream_t stream) {
+  if (in % 64 != 0 || out % 8 != 0 || group % 32 != 0) return cudaErrorInvalidValue;
+  dim3 grid((unsigned)((in + 127) / 128), (unsigned)((out + 63) / 64));
+  w4a16_dequant_kernel<<<grid, 256, 0, stream>>>(qweight, qzeros, scales, in, out, group, Wd);
+  return cudaGetLastError();
+}
+
 // Y[t][o] = RN16(sum over splits s of partials[s][t][o]), the splits added in
 // order (a fixed summation order: the result does not depend on scheduling).
 __global__ void w4a16_splitk_reduce_kernel(const float *__restrict__ partials, int splits, int64_t T,

@@ -169,8 +169,7 @@ def test_w4a16_split_k_for_few_tokens(T):
     unsplit GEMM and the oracle); a searched layer stays within the bound."""
     cfg = awq.AwqConfig.make()
     inn, out = 4096, 1024
-    assert awq.awq_w4a16_workspace_size(T, inn, out, cfg) > 256  # this shape splits
-    assert awq.awq_w4a16_workspace_size(65536, inn, out, cfg) == 256
+    assert 256 < awq.awq_w4a16_workspace_size(T, inn, out, cfg) < inn * out * 2  # this shape splits
     rng = np.random.default_rng(T)
     qw, qz, sc = _random_packed(inn, out, 128, rng, pow2_scales=True)
     X = rng.integers(-3, 4, size=(T, inn)).astype(np.float16)
@@ -184,4 +183,29 @@ def test_w4a16_split_k_for_few_tokens(T):
     qw, qz, sc = O.quant_pack(W.numpy(), s, None, 4, 128)
     Xs = (Xr.numpy().astype(np.float32) / s[None, :]).astype(np.float16)
     _check(_gpu_w4a16(torch.from_numpy(Xs), qw, qz, sc, cfg, split_ws=True), Xs, qw, qz, sc, 128)
+
+
+@pytest.mark.parametrize("T,group", [(1024, 128), (3000, 32), (4096, 64)])
+def test_w4a16_dequantise_once_for_many_tokens(T, group):
+    """From 1024 tokens on, with the workspace awq_w4a16_workspace_size() asks
+    for (the fp16 weights), the product dequantises the packed weights once,
+    RN16((q - z) scale) as the fused kernel does per tile, and runs one fp16
+    GEMM: exact sums stay bit-exact, and it agrees with the fused kernel."""
+    cfg = awq.AwqConfig.make(group_size=group)
+    inn, out = 1024, 800
+    assert awq.awq_w4a16_workspace_size(T, inn, out, cfg) >= inn * out * 2
+    rng = np.random.default_rng(T + group)
+    qw, qz, sc = _random_packed(inn, out, group, rng, pow2_scales=True)
+    X = rng.integers(-3, 4, size=(T, inn)).astype(np.float16)
+    a = _gpu_w4a16(torch.from_numpy(X), qw, qz, sc, cfg, split_ws=True)
+    want = O.w4a16_matmul(X, qw, qz, sc, group).astype(np.float16)
+    assert np.array_equal(a.view(np.uint16), want.view(np.uint16))
+    Xr, W = random_layer(T, inn, out, seed=T + group)
+    s = O.scale_grid(O.act_stats(Xr.numpy()), O.alpha_grid(20))[9]
+    qw, qz, sc = O.quant_pack(W.numpy(), s, None, 4, group)
+    Xs = (Xr.numpy().astype(np.float32) / s[None, :]).astype(np.float16)
+    a = _gpu_w4a16(torch.from_numpy(Xs), qw, qz, sc, cfg, split_ws=True)
+    _check(a, Xs, qw, qz, sc, group)
+    b = _gpu_w4a16(torch.from_numpy(Xs), qw, qz, sc, cfg, split_ws=False)  # the fused kernel
+    _check(b, Xs, qw, qz, sc, group)
 
