@@ -312,6 +312,78 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------- CUDA arm
+def time_workloads(awq, torch, dev, dist, timer, local, args):
+    """ms per layer of the Llama-7B-shaped MLP (gate|up jointly scaled, then
+    down_proj on its SwiGLU input) and of the Llama-13B-shaped INT3 attention
+    block (q|k|v jointly scaled, o_proj on its own input), each at 65536
+    tokens: the groups' whole paths (act stats, alpha search, clip search
+    where the workload has one, packing) run back to back as one step, with
+    their candidate-GEMM flops."""
+    from synthetic import WORKLOADS, workload_inputs
+    res = {}
+    for index in (2, 3):
+        wl = WORKLOADS[index]
+        groups = workload_inputs(index, device=str(dev))["groups"]
+        cfg = awq.AwqConfig.make(w_bit=wl.w_bit, group_size=wl.group_size, n_alpha=wl.n_alpha,
+                                 n_clip=wl.n_clip, clip_min=0.5)
+        dev_groups = [(name, X.to(dev), W.to(dev)) for name, X, W in groups]
+        need = max(awq.awq_workspace_size(X.shape[0], X.shape[1], W.shape[0], cfg)
+                   for _, X, W in dev_groups)
+        ws = torch.empty(need, dtype=torch.uint8, device=dev)
+
+        def step():
+            for _, X, W in dev_groups:
+                awq.quantize_layer(X, W, cfg, ws=ws)
+
+        for _ in range(max(1, min(args.warmup, 3))):
+            step()
+        awq.awq_device_status(ws)
+        steps = max(1, min(args.steps, 3))
+        ms = timed_steps(step, steps, dist, timer, local)
+        awq.awq_device_status(ws)
+        flops = sum(2.0 * X.shape[0] * X.shape[1] * W.shape[0] * wl.n_alpha for _, X, W in dev_groups)
+        res[wl.name] = {"ms_per_layer": round(ms, 3), "steps": steps,
+                        "groups": {name: [int(X.shape[0]), int(X.shape[1]), int(W.shape[0])]
+                                   for name, X, W in dev_groups},
+                        "candidate_gemm_flops": flops,
+                        "candidate_gemm_tflops_over_layer": round(flops / (ms * 1e-3) / 1e12, 1),
+                        "note": wl.description}
+        del dev_groups, groups, ws
+        torch.cuda.empty_cache()
+    # the 32-layer decoder: its first two layers, each timed with CUDA events
+    # around the layer's quantisation (four groups, folds, clip, packing); the
+    # fp16 forward that captures their inputs is input synthesis, untimed
+    from post_weight_quantization_awq_b200 import decoder
+    from synthetic import DecoderSpec, decoder_embeddings, decoder_layer_forward, decoder_layer_weights
+    spec = DecoderSpec()
+    cfg = awq.AwqConfig.make(w_bit=4, n_alpha=20, n_clip=20, clip_min=0.5)
+    x = decoder_embeddings(spec, device=dev)
+    ws, times = None, []
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.no_grad():
+        for layer in range(2):
+            w = decoder_layer_weights(spec, layer, device=dev)
+            caps, x_next = decoder_layer_forward(x, w, spec)
+            if ws is None:
+                ws = decoder.workspace_for_layer(caps, w, cfg)
+                decoder.quantize_layer_groups(caps, {k: v.clone() for k, v in w.items()}, cfg, ws)
+            torch.cuda.synchronize(dev)
+            e0.record()
+            decoder.quantize_layer_groups(caps, w, cfg, ws)
+            e1.record()
+            torch.cuda.synchronize(dev)
+            times.append(e0.elapsed_time(e1))
+            x = x_next
+    res["llama2_7b_decoder_layer"] = {
+        "ms_per_layer": round(statistics.mean(times), 3), "layers_timed": len(times),
+        "note": "layers 0 and 1 of the 32-layer decoder (128 x 512 calibration tokens, q|k|v, o, "
+                "gate|up, down; INT4 g128, 20 alphas + 20 clip ratios, folds, packed); "
+                "bench.py --workload decoder times all 32"}
+    del x, ws, caps, w
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_awq(args):
     import torch
     world, rank, local = dist_env()
@@ -356,10 +428,18 @@ def run_awq(args):
         kern[name] = (tot / n if n else None, n)
     awq.profile_reset()
 
-    # ---- end to end through the public API: pinned host buffers in, results out
+    # ---- end to end through the public API: pinned host buffers in, results out.
+    # Consecutive layers pipeline: a step's inputs go up on a copy stream into one
+    # of two device buffers while the previous step computes; every step still
+    # copies its whole input up and its results down inside the timed region.
     Xh, Wh = X.pin_memory(), W.pin_memory()
-    Xe = torch.empty_like(Xd)
-    We = torch.empty_like(Wd)
+    Xe = [torch.empty_like(Xd), torch.empty_like(Xd)]
+    We = [torch.empty_like(Wd), torch.empty_like(Wd)]
+    copy_stream = torch.cuda.Stream(dev)
+    ready = [torch.cuda.Event(), torch.cuda.Event()]
+    done = [torch.cuda.Event(), torch.cuda.Event()]
+    e2e_k = [0]
+    e2e_first = [True]  # the first step of a region waits for everything before it
     g = wl.group_size
     host_out = {
         "qweight": torch.empty((inn, out // 8), dtype=torch.int32).pin_memory(),
@@ -372,16 +452,28 @@ def run_awq(args):
     }
 
     def e2e_step():
-        Xe.copy_(Xh, non_blocking=True)
-        We.copy_(Wh, non_blocking=True)
-        r = awq.quantize_layer(Xe, We, cfg, ws=ws)
+        b = e2e_k[0] % 2
+        e2e_k[0] += 1
+        cur = torch.cuda.current_stream(dev)
+        if e2e_first[0]:  # not before the timed region starts
+            copy_stream.wait_stream(cur)
+            e2e_first[0] = False
+        copy_stream.wait_event(done[b])  # buffer b's last reader (two steps back) is done
+        with torch.cuda.stream(copy_stream):
+            Xe[b].copy_(Xh, non_blocking=True)
+            We[b].copy_(Wh, non_blocking=True)
+            ready[b].record(copy_stream)
+        cur.wait_event(ready[b])
+        r = awq.quantize_layer(Xe[b], We[b], cfg, ws=ws)
         for k, h in host_out.items():
             h.copy_(getattr(r, k), non_blocking=True)
+        done[b].record(cur)
 
     for _ in range(max(1, min(args.warmup, 2))):
         e2e_step()
     torch.cuda.synchronize(dev)
-    e_steps = max(1, min(args.steps, 5))
+    e_steps = max(1, min(args.steps, 10))
+    e2e_first[0] = True
     ms_e2e = timed_steps(e2e_step, e_steps, dist, timer, local)
     h2d = X.numel() * 2 + W.numel() * 2
     d2h = sum(h.numel() * h.element_size() for h in host_out.values())
@@ -487,6 +579,12 @@ def run_awq(args):
                   "note": "scores against the cached fp16 output RN16(X W^T) (one extra GEMM "
                           "with a store epilogue); candidates RN16(Qdeq/s)"}
 
+    # ---- the other workloads' layers (the MLP and the 13B INT3 attention
+    # block), each group timed as quantize_layer runs it, with its own warm-up
+    workloads = None
+    if not args.no_workloads:
+        workloads = time_workloads(awq, torch, dev, dist, timer, local, args)
+
     # ---- the Gram-form search on the same layer (same MSE, fewer flops), its
     # own timing and flop count; the headline value above is the direct form
     gram = None
@@ -549,12 +647,17 @@ def run_awq(args):
         "kernels": per_kernel,
         "clocks": clk.summary(),
         "e2e": {"value": round(ms_e2e / world, 3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "steps": e_steps},
+                "d2h_bytes_per_step": d2h, "steps": e_steps,
+                "note": "quantize_layer on inputs copied from pinned host memory every step and "
+                        "results copied back every step; consecutive layers pipeline (a step's "
+                        "upload runs on a copy stream, into one of two buffers, while the "
+                        "previous layer computes)"},
         "gpu_launches": launches,
         "cpu_baseline": cpu,
         "gram_form": gram,
         "cached_output_form": cached,
         "w4a16_gemm": w4a16,
+        "workloads": workloads,
     }
     print(json.dumps(line), flush=True)
     return 0
@@ -657,6 +760,8 @@ def main(argv=None):
                     help="skip the extra measurement of the Gram-form search")
     ap.add_argument("--no-cached-form", action="store_true",
                     help="skip the extra measurement of the cached fp16-output form")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the timing of the MLP and 13B-attention layers")
     ap.add_argument("--no-w4a16", action="store_true",
                     help="skip the measurement of the W4A16 GEMM on the packed output")
     ap.add_argument("--workload", choices=("q_proj", "decoder"), default="q_proj",

@@ -5,7 +5,8 @@
         --in 4096 --out 4096 [--alphas 20] [--clips 20] [--bits 4] [--repeat 3] [--form gram|cached_y]
 
 --op is one of: stats, search, clip, pack, layer (all four calls), w4a16 (the
-GEMM on the packed output, Y = X Wd^T with Wd dequantised on the fly).  Inputs
+GEMM on the packed output, Y = X Wd^T with Wd = RN16((q - z) scale); with
+--w4a16-form fused the weights are dequantised tile by tile inside the GEMM).  Inputs
 follow the heavy-tailed recipe of the synthetic module (1% outlier channels
 x U[20, 50], W ~ N(0, 0.02)).  Prints the CUDA-event time of the last repeat.
 """
@@ -39,6 +40,9 @@ def main(argv=None) -> int:
     ap.add_argument("--seed", type=int, default=1)
     ap.add_argument("--form", choices=("direct", "gram", "cached_y"), default="direct",
                     help="alpha-search scoring form")
+    ap.add_argument("--w4a16-form", choices=("auto", "fused"), default="auto",
+                    help="auto: the workspace awq_w4a16_workspace_size asks for (dequantise once "
+                         "for many tokens, split-K for few); fused: 256 bytes (dequantise per tile)")
     a = ap.parse_args(argv)
 
     X = heavy_tailed_activations(a.tokens, a.inn, OutlierSpec(0.01, 20.0, 50.0), a.seed).cuda()
@@ -60,7 +64,8 @@ def main(argv=None) -> int:
     if a.op == "w4a16":
         awq.awq_quant_pack(W, s_best, None, cfg, qw, qz, sc)
         Y = torch.empty((a.tokens, a.out), dtype=torch.float16, device="cuda")
-        ws16 = torch.empty(256, dtype=torch.uint8, device="cuda")
+        nws = 256 if a.w4a16_form == "fused" else awq.awq_w4a16_workspace_size(a.tokens, a.inn, a.out, cfg)
+        ws16 = torch.empty(nws, dtype=torch.uint8, device="cuda")
 
     def once():
         if a.op == "stats":

@@ -169,7 +169,7 @@ def test_w4a16_split_k_for_few_tokens(T):
     unsplit GEMM and the oracle); a searched layer stays within the bound."""
     cfg = awq.AwqConfig.make()
     inn, out = 4096, 1024
-    assert 256 < awq.awq_w4a16_workspace_size(T, inn, out, cfg) < inn * out * 2  # this shape splits
+    assert awq.awq_w4a16_workspace_size(T, inn, out, cfg) > 256  # this shape splits
     rng = np.random.default_rng(T)
     qw, qz, sc = _random_packed(inn, out, 128, rng, pow2_scales=True)
     X = rng.integers(-3, 4, size=(T, inn)).astype(np.float16)
