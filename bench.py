@@ -44,11 +44,11 @@ KERNELS_PER_STEP = {  # kernels this library launches per step (memsets excluded
 # that digest; after any change to them the line carries traffic = null until
 # the kernel is captured again.
 NCU_TRAFFIC = {
-    "bytes": None,
-    "sources_sha256": None,
+    "bytes": 12_648_916_736 + 29_601_536,  # read + write, one launch at 65536 tokens
+    "sources_sha256": "b60ddcd3b010733834ccad3d111832abf15803d4edf17ce6e2e3470aeeb90aa9",
     "command": ("ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none "
                 "-k regex:search_gemm -s 5 -c 1 python bench.py --steps 1 --warmup 5 "
-                "--no-cpu-baseline --no-gram-form --no-cached-form --no-w4a16"),
+                "--no-cpu-baseline --no-gram-form --no-cached-form --no-w4a16 --no-workloads"),
 }
 TRAFFIC_SOURCES = ("post_weight_quantization_awq_b200/csrc/search_gemm.cu",
                    "post_weight_quantization_awq_b200/csrc/awq_device.cuh")
