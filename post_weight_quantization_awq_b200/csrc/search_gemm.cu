@@ -10,7 +10,7 @@
 // K = in.  The epilogue squares and sums each accumulator tile straight out
 // of tensor memory, so no candidate output is ever written to HBM.
 //
-// sm_100a design, one CTA per SM (192 threads), 256 x 256 output tiles:
+// sm_100a design, one CTA per SM (320 threads), 256 x 256 output tiles:
 //   warp 0      TMA producer: A tile 256x64 and B tile 256x64 (fp16, 128-byte
 //               swizzle) into a 3-stage shared-memory ring;
 //   warp 1      allocates 512 TMEM columns; one thread issues two
@@ -19,9 +19,10 @@
 //               B tile, into the two halves of TMEM, and commits stage and
 //               accumulator barriers (TMEM holds one tile: the next tile's
 //               MMAs wait for the epilogue);
-//   warps 2..5  epilogue: tcgen05.ld 32 lanes x 32 columns at a time, sum of
+//   warps 2..9  epilogue, one warp per (TMEM lane quarter, row half):
+//               tcgen05.ld 32 lanes x 32 columns, two loads in flight, sum of
 //               squares in fp32 per row, fp64 warp reduction, one partial per
-//               (128-row block, N tile, warp) into HBM.
+//               (128-row block, N tile, lane quarter) into HBM.
 // Sharing each B tile between two M halves halves the B traffic from L2 to
 // shared memory per flop; under the power cap that bought 4 % more
 // throughput than 128 x 256 tiles with a double-buffered accumulator.
@@ -51,6 +52,8 @@ constexpr uint32_t IDESC = idesc_f16_f32(BM, BN);
 constexpr uint32_t DRAIN_POLLS = 1u << 22;
 constexpr int GROUP_M = 16;  // 256-row M blocks per group: 4096 rows of A in L2
 constexpr int kEpiSse = 0, kEpiStoreY = 1, kEpiSubY = 2;
+constexpr int kEpiWarps = 8;                      // two per TMEM lane quarter: one per row half
+constexpr int kGemmThreads = (2 + kEpiWarps) * 32;  // producer, MMA issuer, epilogue
 
 struct __align__(8) GemmSmemTail {
   uint64_t full[STAGES];
@@ -91,7 +94,7 @@ __device__ __forceinline__ void raise_abort(GemmSmemTail *t, DevStatus *st, uint
 //   kEpiSubY   sum of (acc - Y)^2 with the cached fp16 Y (B = candidate
 //              weights Qdeq/s: the literal "MSE against the fp16 output").
 template <int EPI>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kGemmThreads, 1)
     search_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                        const __grid_constant__ CUtensorMap tmB, int num_m, int num_n, int num_kb,
                        double *__restrict__ partials, __half *__restrict__ Y, int64_t ldy,
@@ -115,7 +118,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&tail->tfull[a], 1);
-      mbar_init(&tail->tempty[a], 4);  // one arrival per epilogue warp
+      mbar_init(&tail->tempty[a], kEpiWarps);  // one arrival per epilogue warp
     }
     mbar_init(&tail->mma_done, 1);
     tail->abort_flag = 0;
@@ -219,7 +222,8 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int q = warp & 3;           // TMEM lane quarter this warp may access
+    const int h = (warp - 2) >> 2;    // the row half (accumulator) this warp reads
     int it = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       const int acc = 0;
@@ -234,11 +238,9 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_after();
       int m_blk, n_blk;
       tile_coords(tile, num_m2, num_n, GROUP_M, m_blk, n_blk);
-      float sums[2] = {0.0f, 0.0f};
-#pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        const int m128 = 2 * m_blk + h;  // 128-row block of this half
-        if (m128 >= num_m) break;        // the last tile's second half lies past T (and past Y)
+      float sums[1] = {0.0f};
+      const int m128 = 2 * m_blk + h;  // 128-row block of this warp's half
+      if (m128 < num_m) {              // the last tile's second half may lie past T (and past Y)
         const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * BN);
         // this thread's accumulator row is token 128 m128 + 32 q + lane
         const size_t yrow = (size_t)(m128 * BM + q * 32 + lane) * (size_t)ldy;
@@ -266,6 +268,17 @@ __global__ void __launch_bounds__(192, 1)
                 sum = fmaf(d1, d1, sum);
               }
             }
+          } else if constexpr (EPI == kEpiSse) {
+            // two 32-column loads in flight per wait
+            float v2[32];
+            tmem_ld_32x32b_x32(taddr + (uint32_t)c, v);
+            tmem_ld_32x32b_x32(taddr + (uint32_t)(c + 32), v2);
+            tmem_ld_wait();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) sum = fmaf(v[i], v[i], sum);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) sum = fmaf(v2[i], v2[i], sum);
+            c += 32;
           } else {
             tmem_ld_32x32b_x32(taddr + (uint32_t)c, v);
             tmem_ld_wait();
@@ -291,20 +304,16 @@ __global__ void __launch_bounds__(192, 1)
             }
           }
         }
-        sums[h] = sum;
+        sums[0] = sum;
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tail->tempty[acc]);
       if constexpr (EPI != kEpiStoreY) {
+        double ds = (double)sums[0];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          double ds = (double)sums[h];
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) ds += __shfl_xor_sync(0xffffffffu, ds, off);
-          const int m128 = 2 * m_blk + h;
-          if (lane == 0 && m128 < num_m) partials[((size_t)n_blk * num_m + m128) * 4 + q] = ds;
-        }
+        for (int off = 16; off > 0; off >>= 1) ds += __shfl_xor_sync(0xffffffffu, ds, off);
+        if (lane == 0 && m128 < num_m) partials[((size_t)n_blk * num_m + m128) * 4 + q] = ds;
       }
     }
   }
@@ -366,7 +375,7 @@ static cudaError_t launch_gemm_epi(const CUtensorMap &tmA, const CUtensorMap &tm
   if (e != cudaSuccess) return e;
   const int tiles = ((sh.num_m + 1) / 2) * sh.num_n;  // 256-row tiles
   const int grid = tiles < num_sms ? tiles : num_sms;
-  search_gemm_kernel<EPI><<<grid, 192, kGemmSmemBytes, stream>>>(
+  search_gemm_kernel<EPI><<<grid, kGemmThreads, kGemmSmemBytes, stream>>>(
       tmA, tmB, sh.num_m, sh.num_n, sh.num_kb, partials, Y, ldy, y_cols, y_rows, st, max_polls);
   return cudaGetLastError();
 }
