@@ -432,19 +432,15 @@ __global__ void __launch_bounds__(256, 3) cand_quant_kernel(
     const float zero = (float)(zf & 255);
     const int64_t o = orow + r;
     const uint32_t wr[4] = {wv[r].x, wv[r].y, wv[r].z, wv[r].w};
-    float2 wt[4], qz[4], rem[4];
+    float2 wt[4], qz[4];
     float rmax = 0.0f;
 #pragma unroll
     for (int h = 0; h < 4; ++h) {
       wt[h] = __fmul2_rn(sk[h], __half22float2(*reinterpret_cast<const __half2 *>(&wr[h])));
       qz[h] = __fadd2_rn(__ffma2_rn(wt[h], make_float2(rc, rc), M), make_float2(-M.x, -M.y));
-      rem[h] = __ffma2_rn(make_float2(-qz[h].x, -qz[h].y), make_float2(dl, dl), wt[h]);
-      rmax = fmax3(rmax, fabsf(rem[h].x), fabsf(rem[h].y));
+      const float2 rem = __ffma2_rn(make_float2(-qz[h].x, -qz[h].y), make_float2(dl, dl), wt[h]);
+      rmax = fmax3(rmax, fabsf(rem.x), fabsf(rem.y));
     }
-    // where the proposal stands (no exact division) and no code clamps, the
-    // candidate error RN(q delta - wt) is -rem, rem = RN(wt - q delta): the
-    // same product and sum under one rounding, of opposite sign
-    const bool from_rem = (rmax < hl) && !(zf & 256);
     if (!(rmax < hl)) {
 #pragma unroll
       for (int h = 0; h < 4; ++h)
@@ -476,25 +472,15 @@ __global__ void __launch_bounds__(256, 3) cand_quant_kernel(
     }
     const float2 dl2 = make_float2(dl, dl);
     uint32_t packed[4];
-    if (from_rem && !weights_only) {
 #pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        // error form: (deq - s w) 2^k (r / s) = -rem (r / s)
-        const float2 d2 = __fmul2_rn(rem[h], make_float2(-iv[h].x, -iv[h].y));
-        const __half2 hv = __floats2half2_rn(d2.x, d2.y);
-        packed[h] = *reinterpret_cast<const uint32_t *>(&hv);
-      }
-    } else {
-#pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        // error form: (deq - s w) 2^k (r / s); weights only: deq / s
-        const float2 t = weights_only ? __fmul2_rn(qz[h], dl2)
-                                      : __ffma2_rn(qz[h], dl2, make_float2(-wt[h].x, -wt[h].y));
-        // rows past `out` and channels past `in` hold w = 0, which gives 0 here
-        const float2 d2 = __fmul2_rn(t, iv[h]);
-        const __half2 hv = __floats2half2_rn(d2.x, d2.y);
-        packed[h] = *reinterpret_cast<const uint32_t *>(&hv);
-      }
+    for (int h = 0; h < 4; ++h) {
+      // error form: (deq - s w) 2^k (r / s); weights only: deq / s
+      const float2 t = weights_only ? __fmul2_rn(qz[h], dl2)
+                                    : __ffma2_rn(qz[h], dl2, make_float2(-wt[h].x, -wt[h].y));
+      // rows past `out` and channels past `in` hold w = 0, which gives 0 here
+      const float2 d2 = __fmul2_rn(t, iv[h]);
+      const __half2 hv = __floats2half2_rn(d2.x, d2.y);
+      packed[h] = *reinterpret_cast<const uint32_t *>(&hv);
     }
     if (j_ok)
       *reinterpret_cast<uint4 *>(dW + ((int64_t)a * out_pad + o) * in + j0) =
