@@ -115,6 +115,14 @@ typedef struct {
  * the arguments are invalid (see awq_last_error()). */
 size_t awq_workspace_size(int64_t T, int64_t in, int64_t out, const awq_config *cfg);
 
+/* The smallest workspace the same calls accept.  With less than
+ * awq_workspace_size() bytes (but at least this many) the alpha search
+ * builds and scores its candidates in chunks, as many at a time as the
+ * workspace holds (down to one: the candidate operand then takes
+ * out_pad x in fp16 instead of n_alpha times that); the results are the same
+ * bit for bit, each candidate's scores coming from the same tiles. */
+size_t awq_workspace_size_min(int64_t T, int64_t in, int64_t out, const awq_config *cfg);
+
 /* Per-input-channel mean activation magnitude ("AWQ and Activation-Aware
  * Scaling", Scaling instead of protecting: abar; "05 — AWQ" §4, step 1).
  *   X    device fp16 [T, in], row stride ldx (elements)

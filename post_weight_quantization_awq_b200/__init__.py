@@ -34,6 +34,7 @@ from .abi import (  # noqa: F401
     awq_w4a16_gemm,
     awq_w4a16_workspace_size,
     awq_workspace_size,
+    awq_workspace_size_min,
     header_functions,
     last_error,
     profile_enable,

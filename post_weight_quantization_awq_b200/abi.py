@@ -66,6 +66,7 @@ _SIGNATURES = {
     "awq_version": (c_char_p, []),
     "awq_last_error": (c_char_p, []),
     "awq_workspace_size": (c_size_t, [c_int64, c_int64, c_int64, POINTER(AwqConfig)]),
+    "awq_workspace_size_min": (c_size_t, [c_int64, c_int64, c_int64, POINTER(AwqConfig)]),
     "awq_act_stats": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_void_p]),
     "awq_scale_grid": (c_int32, [c_void_p, c_int64, c_int32, c_void_p, c_void_p]),
     "awq_search_scale": (c_int32, [c_void_p, c_int64, c_int64, c_int64, c_void_p, c_int64, c_void_p,
@@ -182,6 +183,15 @@ def awq_workspace_size(T: int, inn: int, out: int, cfg: AwqConfig) -> int:
     n = LIB.awq_workspace_size(T, inn, out, ctypes.byref(cfg))
     if n == 0:
         raise AwqError("awq_workspace_size", 1, last_error())
+    return int(n)
+
+
+def awq_workspace_size_min(T: int, inn: int, out: int, cfg: AwqConfig) -> int:
+    """The smallest workspace the search and clip calls accept (the alpha
+    search then runs its candidates in chunks)."""
+    n = LIB.awq_workspace_size_min(T, inn, out, ctypes.byref(cfg))
+    if n == 0:
+        raise AwqError("awq_workspace_size_min", 1, last_error())
     return int(n)
 
 

@@ -168,7 +168,10 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 // Direct form: candidates padded to the GEMM's 256-row N tiles, partials per
 // (n tile, m tile, warp).  Gram form: candidates padded to 128-row M tiles,
 // partials per (m tile, n tile, warp), plus G, G~ hi/lo and r.
-ScaleWs scale_layout(int64_t T, int64_t in, int64_t out, const awq_config *cfg) {
+// n_chunk: candidates whose operand the workspace holds at a time (the
+// alpha search runs the grid in chunks of that many when the caller's
+// workspace is smaller than the whole grid's).
+ScaleWs scale_layout(int64_t T, int64_t in, int64_t out, const awq_config *cfg, int n_chunk) {
   ScaleWs w;
   const bool gram = cfg->search_form == AWQ_SEARCH_GRAM;
   const bool cached_y = cfg->search_form == AWQ_SEARCH_CACHED_Y;
@@ -183,7 +186,7 @@ ScaleWs scale_layout(int64_t T, int64_t in, int64_t out, const awq_config *cfg) 
   w.inv_s = off;
   off = align256(off + sizeof(float) * (size_t)cfg->n_alpha * in);
   w.dW = off;
-  off = align256(off + sizeof(__half) * (size_t)cfg->n_alpha * w.out_pad * in);
+  off = align256(off + sizeof(__half) * (size_t)n_chunk * w.out_pad * in);
   w.partials = off;
   off = align256(off + sizeof(double) * (size_t)cfg->n_alpha * w.per_alpha);
   w.G = w.ghi = w.glo = w.r = w.Y = 0;
@@ -309,7 +312,24 @@ size_t awq_workspace_size(int64_t T, int64_t in, int64_t out, const awq_config *
   }
   if (check_cfg(cfg) != AWQ_OK) return 0;
   if (check_shape(T, in, out, cfg) != AWQ_OK) return 0;
-  size_t need = scale_layout(T, in, out, cfg).end;
+  size_t need = scale_layout(T, in, out, cfg, cfg->n_alpha).end;
+  if (cfg->n_clip > 0 && in % 128 == 0) {
+    size_t c = clip_layout(T, in).end;
+    if (c > need) need = c;
+  }
+  return need;
+}
+
+size_t awq_workspace_size_min(int64_t T, int64_t in, int64_t out, const awq_config *cfg) {
+  g_err.clear();
+  NvtxCall nvtx_call_(__func__);
+  if (fault_mode() == Fault::kAlloc) {
+    fail(AWQ_ERR_WORKSPACE, "injected allocation failure (AWQ_FAULT=alloc)");
+    return 0;
+  }
+  if (check_cfg(cfg) != AWQ_OK) return 0;
+  if (check_shape(T, in, out, cfg) != AWQ_OK) return 0;
+  size_t need = scale_layout(T, in, out, cfg, 1).end;
   if (cfg->n_clip > 0 && in % 128 == 0) {
     size_t c = clip_layout(T, in).end;
     if (c > need) need = c;
@@ -368,7 +388,11 @@ awq_status search_scale_impl(const void *X, int64_t T, int64_t in, int64_t ldx, 
     return fail(AWQ_ERR_UNSUPPORTED, "in=%lld: the %s search needs in %% %d == 0", (long long)in,
                 cfg->search_form == AWQ_SEARCH_GRAM ? "Gram-form" : "direct",
                 cfg->search_form == AWQ_SEARCH_GRAM ? 128 : 64);
-  const ScaleWs L = scale_layout(T, in, out, cfg);
+  // the whole grid's candidates at once, or the largest chunk of them the
+  // caller's workspace holds (the same results, the candidates in turn)
+  ScaleWs L = scale_layout(T, in, out, cfg, cfg->n_alpha);
+  int chunk = cfg->n_alpha;
+  while (chunk > 1 && ws_bytes < L.end) L = scale_layout(T, in, out, cfg, --chunk);
   if ((st = check_ws(ws, ws_bytes, L.end)) != AWQ_OK) return st;
   const int64_t tiles = (int64_t)L.num_m * L.nb_per_alpha * cfg->n_alpha;
   if (tiles > INT32_MAX) return fail(AWQ_ERR_INVALID_ARG, "problem too large (%lld tiles)", (long long)tiles);
@@ -412,32 +436,39 @@ awq_status search_scale_impl(const void *X, int64_t T, int64_t in, int64_t ldx, 
     ProfScope p("scale_grid", s);
     AWQ_TRY_CUDA(launch_scale_grid(abar, in, cfg->n_alpha, s_grid, inv_s, s), "scale_grid launch");
   }
-  {
-    ProfScope p("cand_quant", s);
-    AWQ_TRY_CUDA(launch_cand_quant(static_cast<const __half *>(W), out, in, L.out_pad, s_grid, inv_s, r,
-                                   cfg->n_alpha, cfg->group_size, cfg->w_bit, cfg->zero_point,
-                                   cached_y ? 1 : 0, dst, dW, nsm, s),
-                 "cand_quant launch");
-  }
-  if (gram) {
-    ProfScope p("gram_score", s);
-    AWQ_TRY_CUDA(launch_gram_score(dW, (int64_t)cfg->n_alpha * L.out_pad, in,
-                                   reinterpret_cast<const __half *>(base + L.ghi),
-                                   reinterpret_cast<const __half *>(base + L.glo), partials, dst,
-                                   poll_cap(), nsm, s),
-                 "gram_score launch");
-  } else {
-    SearchGemmShape sh;
-    sh.T = T;
-    sh.in = in;
-    sh.rows_b = (int64_t)cfg->n_alpha * L.out_pad;
-    sh.num_m = L.num_m;
-    sh.num_n = (int)(sh.rows_b / kGemmBN);
-    sh.num_kb = (int)(in / kGemmBK);
-    ProfScope p("search_gemm", s);
-    AWQ_TRY_CUDA(launch_search_gemm(static_cast<const __half *>(X), ldx, dW, sh, partials, Y,
-                                    L.out_pad, dst, poll_cap(), nsm, s),
-                 "search_gemm launch");
+  // the candidates in chunks of `chunk` (all at once with a full workspace):
+  // each chunk's operand, then its scores into its slots of the partials
+  for (int a0 = 0; a0 < cfg->n_alpha; a0 += chunk) {
+    const int cnt = cfg->n_alpha - a0 < chunk ? cfg->n_alpha - a0 : chunk;
+    double *part = partials + (size_t)a0 * L.per_alpha;
+    {
+      ProfScope p("cand_quant", s);
+      AWQ_TRY_CUDA(launch_cand_quant(static_cast<const __half *>(W), out, in, L.out_pad,
+                                     s_grid + (size_t)a0 * in, inv_s + (size_t)a0 * in, r, cnt,
+                                     cfg->group_size, cfg->w_bit, cfg->zero_point, cached_y ? 1 : 0,
+                                     dst, dW, nsm, s),
+                   "cand_quant launch");
+    }
+    if (gram) {
+      ProfScope p("gram_score", s);
+      AWQ_TRY_CUDA(launch_gram_score(dW, (int64_t)cnt * L.out_pad, in,
+                                     reinterpret_cast<const __half *>(base + L.ghi),
+                                     reinterpret_cast<const __half *>(base + L.glo), part, dst,
+                                     poll_cap(), nsm, s),
+                   "gram_score launch");
+    } else {
+      SearchGemmShape sh;
+      sh.T = T;
+      sh.in = in;
+      sh.rows_b = (int64_t)cnt * L.out_pad;
+      sh.num_m = L.num_m;
+      sh.num_n = (int)(sh.rows_b / kGemmBN);
+      sh.num_kb = (int)(in / kGemmBK);
+      ProfScope p("search_gemm", s);
+      AWQ_TRY_CUDA(launch_search_gemm(static_cast<const __half *>(X), ldx, dW, sh, part, Y,
+                                      L.out_pad, dst, poll_cap(), nsm, s),
+                   "search_gemm launch");
+    }
   }
   {
     ProfScope p("mse_argmin", s);
@@ -638,7 +669,7 @@ awq_status awq_candidate_codes(const void *W, int64_t out, int64_t in, const dou
   // the s grid and 1/s as the direct-form search lays them out
   awq_config c = *cfg;
   c.search_form = AWQ_SEARCH_DIRECT;
-  const ScaleWs L = scale_layout(1, in, out, &c);
+  const ScaleWs L = scale_layout(1, in, out, &c, c.n_alpha);
   if ((st = check_ws(ws, ws_bytes, L.dW)) != AWQ_OK) return st;
   AWQ_LAUNCH_GATE();
   cudaStream_t cs = static_cast<cudaStream_t>(stream);

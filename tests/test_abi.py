@@ -27,6 +27,19 @@ def test_version_string():
     assert "sm_100a" in awq.version()
 
 
+def test_smaller_workspace_runs_the_candidates_in_chunks():
+    """The minimum workspace holds one candidate's operand at a time; the
+    full one all twenty; a call with a workspace in between is accepted on
+    the host, one below the minimum is refused before any CUDA work."""
+    cfg = awq.AwqConfig.make(n_alpha=20)
+    full = awq.awq_workspace_size(65536, 4096, 4096, cfg)
+    low = awq.awq_workspace_size_min(65536, 4096, 4096, cfg)
+    assert full - low == 19 * 4096 * 4096 * 2
+    st = abi.LIB.awq_search_scale(16, 65536, 4096, 4096, 16, 4096, 16, ctypes.byref(cfg), 256, low - 256,
+                                  16, 16, 16, None)
+    assert abi.STATUS[st] == "AWQ_ERR_WORKSPACE" and str(low) in abi.last_error()
+
+
 def test_workspace_size_grows_with_the_problem():
     cfg = awq.AwqConfig.make(n_alpha=20, n_clip=20)
     a = awq.awq_workspace_size(65536, 4096, 4096, cfg)

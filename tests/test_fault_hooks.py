@@ -72,7 +72,8 @@ def test_launch_gate_comes_after_the_argument_checks(monkeypatch):
 def test_every_launching_call_is_gated():
     """The gated calls are every call the header declares except the
     host-only ones."""
-    host_only = {"awq_version", "awq_last_error", "awq_workspace_size", "awq_w4a16_workspace_size",
+    host_only = {"awq_version", "awq_last_error", "awq_workspace_size", "awq_workspace_size_min",
+                 "awq_w4a16_workspace_size",
                  "awq_device_status",
                  "awq_profile_enable", "awq_profile_read", "awq_profile_reset"}
     assert set(abi.header_functions()) - host_only == set(_launching_calls())

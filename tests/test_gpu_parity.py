@@ -342,3 +342,38 @@ def test_quant_pack_other_group_sizes(out, inn, w_bit, group):
     for g_, w_, name in zip((qw.cpu().numpy(), qz.cpu().numpy(), sc.cpu().numpy()), want,
                             ("qweight", "qzeros", "scales")):
         assert np.array_equal(g_.view(np.uint8), w_.view(np.uint8)), name
+
+
+# ------------------------------------------------------------------ candidates in chunks
+def _search_with_ws_bytes(X, W, cfg, nbytes):
+    Xd, Wd = to_dev(X), to_dev(W)
+    T, inn = Xd.shape
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    abar = torch.empty(inn, dtype=torch.float64, device="cuda")
+    mse = torch.empty(cfg.n_alpha, dtype=torch.float64, device="cuda")
+    best = torch.empty(1, dtype=torch.int32, device="cuda")
+    s_best = torch.empty(inn, dtype=torch.float32, device="cuda")
+    awq.awq_act_stats(Xd, abar)
+    awq.awq_search_scale(Xd, Wd, abar, cfg, ws, s_best, mse, best)
+    awq.awq_device_status(ws)
+    return mse.cpu().numpy(), int(best.item()), s_best.cpu().numpy()
+
+
+@pytest.mark.parametrize("form", [0, 1, 2])
+def test_search_scale_in_chunks_is_bitwise_the_same(form):
+    """A workspace below awq_workspace_size() runs the candidates in chunks
+    (one at a time at awq_workspace_size_min()); every score comes from the
+    same tiles, so MSE, selection and s are the same bits."""
+    X, W = random_layer(2125, 1024, 520, seed=31)
+    cfg = awq.AwqConfig.make(search_form=form)
+    full = awq.awq_workspace_size(2125, 1024, 520, cfg)
+    low = awq.awq_workspace_size_min(2125, 1024, 520, cfg)
+    assert low < full
+    ref = _search_with_ws_bytes(X, W, cfg, full)
+    for nbytes in (low, low + (full - low) // 3):
+        got = _search_with_ws_bytes(X, W, cfg, nbytes)
+        assert np.array_equal(got[0], ref[0]) and got[1] == ref[1]
+        assert np.array_equal(got[2], ref[2])
+    mse_o, _, _, _ = O.search_scale(X.numpy(), W.numpy(), O.act_stats(X.numpy()), 4, 128, 20,
+                                    form="fp16_output" if form == 2 else "gram")
+    check_mse(ref[0], mse_o)
