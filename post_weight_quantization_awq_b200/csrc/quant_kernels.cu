@@ -523,10 +523,10 @@ cudaError_t launch_cand_codes(const __half *W, int64_t out, int64_t in, int64_t 
 // K7 — final codes with (s, clip ratio) and the pages' storage layout
 // ("05 — AWQ" §5): qweight [in, out/8] int32 with the code of output o in
 // nibble o%8 of word [j][o/8]; qzeros [in/g, out/8] likewise; scales
-// [in/g, out] fp16.  A block handles 128 output rows x one group of 128
-// input channels: warps quantise rows (one lane per 4 channels), codes go
-// through shared memory and are re-read transposed for packing, so every
-// global store is contiguous.
+// [in/g, out] fp16.  A block handles 64 output rows x 128 input channels:
+// warp w takes rows 8w..8w+7 -- exactly the 8 nibbles of one word column --
+// and lane l channels 4l..4l+3, so a lane builds the 4 packed words of its
+// channels in registers, with no transpose of codes.
 // ---------------------------------------------------------------------------
 constexpr int kPackRows = 64;
 
@@ -555,119 +555,167 @@ __device__ __forceinline__ float clip_ratio(int c, int n_clip, float clip_min) {
   return __double2float_rn(r);
 }
 
-// A block handles 64 output rows x a tile of 128 input channels (the last
-// tile may be narrower; g in {32, 64, 128} divides both): the W tile is
-// fetched with independent 16-byte loads into shared memory, warps quantise
-// 8 rows each (4 channels per lane, a group's g/4 lanes reduce its range by
-// shuffles), codes are re-read transposed for packing so every global store
-// is contiguous.
+// Per warp: the 8 rows' group ranges by a transposing butterfly over the
+// group's g/4 lanes (each lane ends with one row's range), the step, zero
+// point, fast-path bound and clamp need computed once per (row, group) and
+// passed through shared memory, codes proposed by the approximate reciprocal
+// and proven by one remainder test per 4 values (the correctly rounded
+// division otherwise), and the packed word of each channel summed exactly in
+// fp32 as two 16-bit halves (codes times 16^r, integers below 2^16).
 constexpr int kPackTile = 128;
 
-template <int group>  // 32, 64 or 128: divisions and the shuffle loop become constants
-__global__ void __launch_bounds__(256, 6) quant_pack_kernel(
+template <int N, int OFF>
+__device__ __forceinline__ void pack_range_reduce(float (&mx)[8], float (&mn)[8], int lane) {
+  if constexpr (OFF >= 1) {
+    if constexpr (N > 1) {
+      const bool up = (lane & OFF) != 0;
+#pragma unroll
+      for (int i = 0; i < N / 2; ++i) {
+        const float sx = up ? mx[i] : mx[i + N / 2], sn = up ? mn[i] : mn[i + N / 2];
+        const float kx = up ? mx[i + N / 2] : mx[i], kn = up ? mn[i + N / 2] : mn[i];
+        mx[i] = fmaxf(kx, __shfl_xor_sync(0xffffffffu, sx, OFF));
+        mn[i] = fminf(kn, __shfl_xor_sync(0xffffffffu, sn, OFF));
+      }
+      pack_range_reduce<N / 2, OFF / 2>(mx, mn, lane);
+    } else {
+      mx[0] = fmaxf(mx[0], __shfl_xor_sync(0xffffffffu, mx[0], OFF));
+      mn[0] = fminf(mn[0], __shfl_xor_sync(0xffffffffu, mn[0], OFF));
+      pack_range_reduce<1, OFF / 2>(mx, mn, lane);
+    }
+  }
+}
+
+template <int group>  // 32, 64 or 128: divisions and the shuffle rounds become constants
+__global__ void __launch_bounds__(256, 4) quant_pack_kernel(
     const __half *__restrict__ W, int64_t out, int64_t in, const float *__restrict__ s,
     const uint8_t *__restrict__ clip_idx, int n_clip, float clip_min, float qmax, int sym,
     int32_t *__restrict__ qweight, int32_t *__restrict__ qzeros, __half *__restrict__ scales) {
   constexpr int TC = kPackTile;
-  __shared__ __align__(16) __half wsm[kPackRows][TC + 8];
-  __shared__ uint8_t codes[kPackRows][TC + 4];
-  __shared__ uint8_t zeros[kPackRows][TC / 32];
-  __shared__ float ratios[64];  // clip ratio of each index (n_clip <= 64)
+  constexpr int gl = group / 4;      // lanes per group
+  constexpr int GPT = TC / group;    // groups per tile
+  constexpr int kShare = gl / 8;     // lanes sharing one row's range after the reduction
+  __shared__ __align__(16) float4 prm[8][GPT][8];      // per warp, group, row: delta, rcp, half_lo, flags
+  __shared__ __align__(16) uint32_t words[TC][8 + 1];  // [channel][word column]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (clip_idx && threadIdx.x < n_clip) ratios[threadIdx.x] = clip_ratio(threadIdx.x, n_clip, clip_min);
-  const int64_t j_tile = (int64_t)blockIdx.y * TC;              // first channel of the tile
-  const int cols = (int)i64min(TC, in - j_tile);                // channels in this tile
+  const int64_t j_tile = (int64_t)blockIdx.y * TC;  // first channel of the tile
+  const int cols = (int)i64min(TC, in - j_tile);    // channels here: a multiple of group
   const int64_t o0 = (int64_t)blockIdx.x * kPackRows;
+  const int rows_here = (int)i64min(kPackRows, out - o0);  // a multiple of 8 (out % 8 == 0)
   const int64_t groups = in / group;
-  const int rows_here = (int)i64min(kPackRows, out - o0);
-  constexpr int gl = group / 4;                                 // lanes per group
-  {
-    uint4 v[4];
+  const int64_t wpr = out / 8;                      // words per qweight row
+  const bool lane_ok = lane * 4 < cols;             // whole groups of lanes
+  const bool warp_ok = 8 * warp < rows_here;
+  const int gi = (lane * 4) / group;                // group within the tile
+  const int64_t kg = j_tile / group + gi;           // global group index
+  const int64_t orow = o0 + 8 * warp;
+  if (warp_ok) {  // warp-uniform: every lane of the warp takes part in the shuffles
+    float2 sv[2] = {make_float2(1.0f, 1.0f), make_float2(1.0f, 1.0f)};
+    if (s && lane_ok) {
+      const float4 f = __ldg(reinterpret_cast<const float4 *>(s + j_tile + lane * 4));
+      sv[0] = make_float2(f.x, f.y);
+      sv[1] = make_float2(f.z, f.w);
+    }
+    float2 wt[8][2];
+    float mx[8], mn[8];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int c = threadIdx.x + 256 * u;  // 16-byte chunk: row c/16, channels 8*(c%16)
-      const int r = c >> 4, cc = 8 * (c & 15);
-      v[u] = (r < rows_here && cc < cols)
-                 ? __ldg(reinterpret_cast<const uint4 *>(W + (o0 + r) * in + j_tile + cc))
-                 : make_uint4(0u, 0u, 0u, 0u);
+    for (int r = 0; r < 8; ++r) {
+      const uint2 v = lane_ok ? __ldg(reinterpret_cast<const uint2 *>(W + (orow + r) * in + j_tile + lane * 4))
+                              : make_uint2(0u, 0u);
+      wt[r][0] = __fmul2_rn(sv[0], __half22float2(*reinterpret_cast<const __half2 *>(&v.x)));
+      wt[r][1] = __fmul2_rn(sv[1], __half22float2(*reinterpret_cast<const __half2 *>(&v.y)));
+      mx[r] = fmaxf(fmax3(wt[r][0].x, wt[r][0].y, wt[r][1].x), wt[r][1].y);
+      mn[r] = fminf(fmin3(wt[r][0].x, wt[r][0].y, wt[r][1].x), wt[r][1].y);
     }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int c = threadIdx.x + 256 * u;
-      *reinterpret_cast<uint4 *>(&wsm[c >> 4][8 * (c & 15)]) = v[u];
-    }
-  }
-  const bool lane_ok = lane * 4 < cols;
-  float sv[4] = {1.0f, 1.0f, 1.0f, 1.0f};
-  if (s && lane_ok) {
-    const float4 f = __ldg(reinterpret_cast<const float4 *>(s + j_tile + lane * 4));
-    sv[0] = f.x; sv[1] = f.y; sv[2] = f.z; sv[3] = f.w;
-  }
-  const int gi = (lane * 4) / group;                            // group within the tile
-  const int64_t kg = j_tile / group + gi;                       // global group index
-  __syncthreads();
-  for (int r = warp; r < rows_here; r += 8) {
-    const int64_t o = o0 + r;
-    const uint2 wv = *reinterpret_cast<const uint2 *>(&wsm[r][lane * 4]);
-    const float2 a = __half22float2(*reinterpret_cast<const __half2 *>(&wv.x));
-    const float2 b = __half22float2(*reinterpret_cast<const __half2 *>(&wv.y));
-    const float wt[4] = {__fmul_rn(sv[0], a.x), __fmul_rn(sv[1], a.y), __fmul_rn(sv[2], b.x),
-                         __fmul_rn(sv[3], b.y)};
-    float mx = fmaxf(fmaxf(wt[0], wt[1]), fmaxf(wt[2], wt[3]));
-    float mn = fminf(fminf(wt[0], wt[1]), fminf(wt[2], wt[3]));
-#pragma unroll
-    for (int off = gl >> 1; off > 0; off >>= 1) {
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
-      mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, off));
-    }
-    if (!lane_ok) continue;  // past the last channel (its lanes form whole groups)
-    // an index past the clip grid is the caller's error: that group gets codes
-    // and zero 0 and a NaN scale, and the library status word records it
-    float r32 = 1.0f;
-    bool bad = false;
-    if (clip_idx) {
-      const int ci = clip_idx[o * groups + kg];
-      if (ci < n_clip)
-        r32 = ratios[ci];
-      else
-        bad = true;
-    }
-    // four values per lane: the scalar quantiser (the batched fast path of the
-    // candidate kernels costs more than it saves at this width)
-    const GroupQ g = group_params(mx, mn, r32, qmax, sym != 0);
-    uchar4 c4 = make_uchar4(0, 0, 0, 0);
-    if (!bad) {
-      c4.x = (uint8_t)quant_code(wt[0], g);
-      c4.y = (uint8_t)quant_code(wt[1], g);
-      c4.z = (uint8_t)quant_code(wt[2], g);
-      c4.w = (uint8_t)quant_code(wt[3], g);
-    }
-    *reinterpret_cast<uchar4 *>(&codes[r][lane * 4]) = c4;
-    if ((lane & (gl - 1)) == 0) {  // first lane of the group
-      zeros[r][gi] = bad ? (uint8_t)0 : (uint8_t)g.zero;
-      scales[kg * out + o] = bad ? __ushort_as_half((unsigned short)0x7E00u) : __float2half_rn(g.delta);
+    pack_range_reduce<8, gl / 2>(mx, mn, lane);
+    // this lane now holds the range of row (lane within the group) / kShare
+    const int rh = (lane & (gl - 1)) / kShare;
+    if (lane_ok && (lane & (kShare - 1)) == 0) {
+      // an index past the clip grid is the caller's error: that group gets
+      // codes and zero 0 and a NaN scale, and the library status word records it
+      float r32 = 1.0f;
+      bool bad = false;
+      if (clip_idx) {
+        const int ci = __ldg(clip_idx + (orow + rh) * groups + kg);
+        if (ci < n_clip)
+          r32 = clip_ratio(ci, n_clip, clip_min);
+        else
+          bad = true;
+      }
+      GroupQ g = group_params(mx[0], mn[0], r32, qmax, sym != 0);
+      fast_path_check(g, mx[0], mn[0]);
+      // every code of the group lies between those of its extremes
+      const float qhi = __fadd_rn(round_quotient(mx[0], g), g.zero);
+      const float qlo = __fadd_rn(round_quotient(mn[0], g), g.zero);
+      const int clamp = !(qlo >= 0.0f && qhi <= g.qmax);
+      const int flags = (bad ? 0 : (int)g.zero) | (clamp << 8) | ((int)bad << 9);
+      prm[warp][gi][rh] = make_float4(g.delta, g.rcp, g.half_lo, __int_as_float(flags));
+      scales[kg * out + orow + rh] = bad ? __ushort_as_half((unsigned short)0x7E00u) : __float2half_rn(g.delta);
       if (bad) dev_fail(&g_lib_status, kDevBadIndex, 0x4B0u);
     }
+    __syncwarp();
+    if (lane_ok) {  // lanes past the last channel form whole groups
+    // codes; the packed words as exact fp32 sums of code * 16^r, per 4-row half
+    float lo[4], hi[4];
+    float zlo = 0.0f, zhi = 0.0f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) lo[c] = hi[c] = 0.0f;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const float4 pv = prm[warp][gi][r];
+      const int flags = __float_as_int(pv.w);
+      const float zero = (float)(flags & 255);
+      const float dl = pv.x, rc = pv.y, hl = pv.z;
+      const float2 M = make_float2(12582912.0f, 12582912.0f);  // 1.5 2^23
+      float2 qz[2];
+      float rmax = 0.0f;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        qz[h] = __fadd2_rn(__ffma2_rn(wt[r][h], make_float2(rc, rc), M), make_float2(-M.x, -M.y));
+        const float2 rem = __ffma2_rn(make_float2(-qz[h].x, -qz[h].y), make_float2(dl, dl), wt[r][h]);
+        rmax = fmax3(rmax, fabsf(rem.x), fabsf(rem.y));
+      }
+      if (!(rmax < hl)) {
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          qz[h] = make_float2(rintf(__fdiv_rn(wt[r][h].x, dl)), rintf(__fdiv_rn(wt[r][h].y, dl)));
+      }
+      if (flags & 256) {
+        const float lo_q = -zero, hi_q = qmax - zero;  // exact (small integers)
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          qz[h] = make_float2(fminf(fmaxf(qz[h].x, lo_q), hi_q), fminf(fmaxf(qz[h].y, lo_q), hi_q));
+      }
+      if (flags & 512) qz[0] = qz[1] = make_float2(0.0f, 0.0f);  // code 0 (its zero is 0)
+      const float pw = (float)(1 << (4 * (r & 3)));  // 16^(r mod 4)
+      const float q4[4] = {qz[0].x, qz[0].y, qz[1].x, qz[1].y};
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        if (r < 4)
+          lo[c] = fmaf(q4[c], pw, lo[c]);
+        else
+          hi[c] = fmaf(q4[c], pw, hi[c]);
+      }
+      if (r < 4)
+        zlo = fmaf(zero, pw, zlo);
+      else
+        zhi = fmaf(zero, pw, zhi);
+    }
+    // (q - z) + z summed per half: the codes' half-words, exact
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const uint32_t wl = (uint32_t)__fadd_rn(lo[c], zlo), wh = (uint32_t)__fadd_rn(hi[c], zhi);
+      words[lane * 4 + c][warp] = wl | (wh << 16);
+    }
+    if ((lane & (gl - 1)) == 0)  // first lane of the group: the zero points' word
+      qzeros[kg * wpr + orow / 8] = (int32_t)((uint32_t)zlo | ((uint32_t)zhi << 16));
+    }
   }
   __syncthreads();
-  const int64_t words_per_row = out / 8;
-  const int o8_here = rows_here / 8;  // out % 8 == 0
+  // qweight rows of this tile: 8 consecutive words (32 bytes) per channel
+  const int w8 = rows_here / 8;
   for (int t = threadIdx.x; t < cols * 8; t += 256) {
-    const int o8 = t & 7, jj = t >> 3;
-    if (o8 >= o8_here) continue;
-    uint32_t word = 0;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) word |= (uint32_t)codes[o8 * 8 + e][jj] << (4 * e);
-    qweight[(j_tile + jj) * words_per_row + o0 / 8 + o8] = (int32_t)word;
-  }
-  const int g_here = cols / group;
-  for (int t = threadIdx.x; t < g_here * 8; t += 256) {
-    const int o8 = t & 7, gg = t >> 3;
-    if (o8 >= o8_here) continue;
-    uint32_t word = 0;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) word |= (uint32_t)zeros[o8 * 8 + e][gg] << (4 * e);
-    qzeros[(j_tile / group + gg) * words_per_row + o0 / 8 + o8] = (int32_t)word;
+    const int jj = t >> 3, wc = t & 7;
+    if (wc < w8) qweight[(j_tile + jj) * wpr + o0 / 8 + wc] = (int32_t)words[jj][wc];
   }
 }
 

@@ -327,18 +327,26 @@ def test_search_scale_other_group_sizes(T, inn, out, w_bit, group, form):
     assert np.array_equal(g["s_best"], S[g["best"]])
 
 
-@pytest.mark.parametrize("out,inn,w_bit,group", [(72, 96, 4, 32), (136, 320, 3, 64), (512, 4096, 4, 32),
-                                                 (64, 192, 4, 64)])
-def test_quant_pack_other_group_sizes(out, inn, w_bit, group):
-    X, W = random_layer(16, inn, out, seed=out + inn)
+@pytest.mark.parametrize("out,inn,w_bit,group,n_clip", [
+    (72, 96, 4, 32, 0), (136, 320, 3, 64, 0), (512, 4096, 4, 32, 0), (64, 192, 4, 64, 0),
+    (72, 96, 4, 32, 20), (136, 320, 3, 64, 7), (520, 1024, 4, 32, 20), (264, 640, 4, 64, 20)])
+def test_quant_pack_other_group_sizes(out, inn, w_bit, group, n_clip):
+    """Groups of 32 and 64 channels, with and without clip indices; widths
+    that leave a partial 128-channel tile (96, 320, 640) and row counts that
+    leave a partial 64-row block (72, 136, 264, 520)."""
+    X, W = random_layer(16, inn, out, seed=out + inn + n_clip)
     s = O.scale_grid(O.act_stats(X.numpy()), O.alpha_grid(20))[11]
-    cfg = awq.AwqConfig.make(w_bit=w_bit, group_size=group)
+    cfg = awq.AwqConfig.make(w_bit=w_bit, group_size=group, n_clip=n_clip)
+    clip_idx = (np.random.default_rng(out + group).integers(0, n_clip, size=(out, inn // group))
+                .astype(np.uint8) if n_clip else None)
     qw = torch.empty((inn, out // 8), dtype=torch.int32, device="cuda")
     qz = torch.empty((inn // group, out // 8), dtype=torch.int32, device="cuda")
     sc = torch.empty((inn // group, out), dtype=torch.float16, device="cuda")
-    awq.awq_quant_pack(to_dev(W), torch.from_numpy(s).cuda(), None, cfg, qw, qz, sc)
+    awq.awq_quant_pack(to_dev(W), torch.from_numpy(s).cuda(),
+                       None if clip_idx is None else torch.from_numpy(clip_idx).cuda(), cfg, qw, qz, sc)
     torch.cuda.synchronize()
-    want = O.quant_pack(W.numpy(), s, None, w_bit, group)
+    awq.awq_device_status(None)
+    want = O.quant_pack(W.numpy(), s, clip_idx, w_bit, group, max(n_clip, 1), 0.5)
     for g_, w_, name in zip((qw.cpu().numpy(), qz.cpu().numpy(), sc.cpu().numpy()), want,
                             ("qweight", "qzeros", "scales")):
         assert np.array_equal(g_.view(np.uint8), w_.view(np.uint8)), name
