@@ -320,15 +320,18 @@ awq_status awq_search_clip_grams(const void *W, int64_t out, int64_t in, const f
  * pages describe for AWQ's inference kernels):
  *   Y[t][o] = RN16( sum_j X[t][j] Wd[o][j] ),  Wd[o][j] = RN16((q - z) scale)
  * with q the 4-bit code of (o, j) (nibble o % 8 of qweight[j][o/8]), z that of
- * qzeros[j/g][o/8] and scale = scales[j/g][o]; fp32 accumulation on the tensor
- * cores.  INT3 codes use the same nibbles.
+ * qzeros[j/g][o/8] and scale = scales[j/g][o]; fp32 accumulation (on the
+ * tensor cores from 9 tokens on; up to 8 tokens, a decode step, the product
+ * is bound by reading the packed words and runs on CUDA cores, which stream
+ * each word once).  INT3 codes use the same nibbles.
  *   X        device fp16 [T, in], row stride ldx
  *   qweight  device int32 [in, out/8]; qzeros int32 [in/g, out/8]; scales fp16 [in/g, out]
  *   Y        device fp16 [T, out] (output), row stride ldy (multiple of 8)
  *   ws       at least 256 bytes (status word), with which the weights are
  *            dequantised tile by tile inside the GEMM.  With
- *            awq_w4a16_workspace_size() bytes: few tokens (output tiles
- *            filling under half of the SMs) are computed with split-K (fp32
+ *            awq_w4a16_workspace_size() bytes: few tokens (up to 8, or
+ *            output tiles filling under half of the SMs) are computed with
+ *            split-K (fp32
  *            partial sums of K ranges in the workspace, added in a fixed order
  *            and rounded to fp16 once); 1024 tokens or more dequantise the
  *            weights once into the workspace (the same RN16((q - z) scale)

@@ -250,6 +250,10 @@ Fault fault_mode() {
 // the conversion then costs in x out work once instead of once per 256-token
 // tile, and the GEMM runs at the tensor cores' rate.
 constexpr int64_t kW4DequantMinT = 1024;
+// Up to this many tokens the product is bound by reading the packed words:
+// a CUDA-core kernel streams them (the tensor-core forms would run a 128-row
+// tile for a handful of rows).
+constexpr int64_t kW4GemvMaxT = 8;
 
 // status word plus the fp16 weights [out, in]
 size_t w4a16_dequant_ws_bytes(int64_t in, int64_t out) {
@@ -783,6 +787,21 @@ awq_status awq_w4a16_gemm(const void *X, int64_t T, int64_t in, int64_t ldx, con
                  "w4a16 fp16 GEMM launch");
     return AWQ_OK;
   }
+  // a few tokens (decode): the product streams the packed words on CUDA cores,
+  // split along K when the workspace holds the fp32 partial sums
+  if (T <= kW4GemvMaxT) {
+    const int nsm = num_sms_current();
+    const int gsplits = w4a16_gemv_splits(T, in, out, nsm);
+    float *gpart = gsplits > 1 && ws_bytes >= w4a16_ws_bytes(T, out, gsplits)
+                       ? reinterpret_cast<float *>(static_cast<uint8_t *>(ws) + kHeader)
+                       : nullptr;
+    ProfScope p("w4a16_gemv", cs);
+    AWQ_TRY_CUDA(launch_w4a16_gemv(static_cast<const __half *>(X), T, in, ldx, qweight, qzeros,
+                                   static_cast<const __half *>(scales), out, cfg->group_size,
+                                   static_cast<__half *>(Y), ldy, gpart, nsm, cs),
+                 "w4a16_gemv launch");
+    return AWQ_OK;
+  }
   // split-K for few tokens, when the workspace holds the fp32 partial sums
   int splits = w4a16_splits(T, in, out, num_sms_current());
   if (splits > 1 && ws_bytes < w4a16_ws_bytes(T, out, splits)) splits = 1;
@@ -806,6 +825,10 @@ size_t awq_w4a16_workspace_size(int64_t T, int64_t in, int64_t out, const awq_co
   if (check_cfg(cfg) != AWQ_OK) return 0;
   if (check_shape(T, in, out, cfg) != AWQ_OK) return 0;
   if (T >= kW4DequantMinT) return w4a16_dequant_ws_bytes(in, out);
+  if (T <= kW4GemvMaxT) {
+    const int gsplits = w4a16_gemv_splits(T, in, out, num_sms_current());
+    return gsplits > 1 ? w4a16_ws_bytes(T, out, gsplits) : kHeader;
+  }
   const int splits = w4a16_splits(T, in, out, num_sms_current());
   return splits > 1 ? w4a16_ws_bytes(T, out, splits) : kHeader;
 }

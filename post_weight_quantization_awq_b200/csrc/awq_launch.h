@@ -136,6 +136,16 @@ cudaError_t launch_w4a16_gemm(const __half *X, int64_t T, int64_t in, int64_t ld
 // The split count the W4A16 GEMM uses when its workspace allows: 1 when the
 // output tiles fill at least half of the SMs, else enough K splits (each of
 // at least 4 K steps of 64 channels) to occupy them.
+// Decode W4A16 product (T <= 8 tokens) on CUDA cores, streaming the packed
+// words once; `partials` ([splits][T][out] fp32, splits = w4a16_gemv_splits:
+// one per 256 input rows) enables the K split, NULL runs one block column per
+// 256 outputs over all of `in`.  Requires in % 64 == 0, out % 8 == 0,
+// group % 32 == 0, ldx % 8 == 0.
+int w4a16_gemv_splits(int64_t T, int64_t in, int64_t out, int num_sms);
+cudaError_t launch_w4a16_gemv(const __half *X, int64_t T, int64_t in, int64_t ldx,
+                              const int32_t *qweight, const int32_t *qzeros, const __half *scales,
+                              int64_t out, int group, __half *Y, int64_t ldy, float *partials,
+                              int num_sms, cudaStream_t stream);
 int w4a16_splits(int64_t T, int64_t in, int64_t out, int num_sms);
 // The dequantised weights of a packed layer, Wd [out, in] fp16 row-major,
 // Wd[o][j] = RN16((q - z) scale): the operand of the W4A16 product for many

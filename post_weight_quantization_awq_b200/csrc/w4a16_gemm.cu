@@ -557,6 +557,168 @@ __global__ void w4a16_splitk_reduce_kernel(const float *__restrict__ partials, i
   }
 }
 
+// ---------------------------------------------------------------------------
+// Decode: up to kGemvMaxT tokens.  The product reads each packed word once and
+// does T x 8 multiply-adds with it, so it is bound by reading the weights, not
+// by the tensor cores: a CUDA-core kernel streams the words instead.  The
+// matrix is only a few MB, so the design goal is to have nearly all of it in
+// flight at once: a block covers 256 outputs (a warp's 32 lanes read 32
+// consecutive words of an input row: 128 contiguous bytes) and 256 input rows
+// (one K split), warp w rows 32w..32w+31 (inside one group: group | 32), and a
+// lane issues the loads of 32 / 16 / 8 of its rows together (T <= 2 / 4 / 8,
+// as registers allow).  The block's X[t][j] are staged in shared memory as
+// fp32 pairs (x, x); a lane dequantises each word to the fp16 weights
+// RN16((q - z) scale) (the values the GEMM forms use), whose halves pair
+// outputs (p, p + 4), widens them and accumulates with packed f32x2 FMAs, rows
+// in ascending order.  The warps' sums are added in a fixed order through
+// shared memory; with several K splits (blocks along y) each writes fp32 sums
+// for the split-K reduction, else the block rounds Y itself.
+// ---------------------------------------------------------------------------
+constexpr int kGemvMaxT = 8;
+constexpr int kGemvOut = 256;   // outputs per block
+constexpr int kGemvWarps = 8;
+
+// rows per warp; a K split is 8 warps x that (256 rows): about two blocks
+// per SM for a 4096 x 4096 layer, and partial sums of 1/32 of the weights'
+// bytes per token
+__host__ __device__ constexpr int gemv_warp_rows(int) { return 32; }
+
+template <int TT>
+__global__ void __launch_bounds__(kGemvWarps * 32, 2) w4a16_gemv_kernel(
+    const __half *__restrict__ X, int64_t in, int64_t ldx, const int32_t *__restrict__ qweight,
+    const int32_t *__restrict__ qzeros, const __half *__restrict__ scales, int64_t out, int group,
+    int64_t k_per_split, __half *__restrict__ Y, int64_t ldy, float *__restrict__ partials) {
+  constexpr int WR = gemv_warp_rows(TT);  // rows per warp and chunk
+  constexpr int CH = kGemvWarps * WR;     // rows per chunk
+  constexpr int RB = TT <= 2 ? 32 : TT <= 4 ? 16 : 8;  // rows whose words are loaded together
+  constexpr int kRedT = TT < 4 ? TT : 4;  // tokens reduced per pass through shared memory
+  constexpr int kXsBytes = CH * TT * 8;
+  constexpr int kRedBytes = kGemvWarps * kRedT * (kGemvOut + 4) * 4;
+  __shared__ __align__(16) unsigned char smem[kXsBytes > kRedBytes ? kXsBytes : kRedBytes];
+  float2(*xs)[TT] = reinterpret_cast<float2(*)[TT]>(smem);  // [chunk row][token]: (x, x)
+  float(*red)[kRedT][kGemvOut + 4] = reinterpret_cast<float(*)[kRedT][kGemvOut + 4]>(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t words = out / 8;
+  const int64_t wc = (int64_t)blockIdx.x * (kGemvOut / 8) + lane;  // this lane's word column
+  const bool col_ok = wc < words;
+  const int64_t j0 = (int64_t)blockIdx.y * k_per_split;
+  const int64_t j1 = j0 + k_per_split < in ? j0 + k_per_split : in;  // multiples of 64
+  float2 acc[TT][4];  // outputs (p, p + 4) of the word, p = 0..3
+#pragma unroll
+  for (int t = 0; t < TT; ++t)
+#pragma unroll
+    for (int p = 0; p < 4; ++p) acc[t][p] = make_float2(0.0f, 0.0f);
+  for (int64_t jc = j0; jc < j1; jc += CH) {
+    const int rows = (int)(j1 - jc < CH ? j1 - jc : CH);  // a multiple of 64 or CH
+    const int64_t jw = jc + WR * warp;
+    const bool live = col_ok && WR * warp < rows;
+    if (jc != j0) __syncthreads();  // the previous chunk's X is no longer read
+    for (int i = threadIdx.x; i < rows * TT; i += kGemvWarps * 32) {
+      const int t = i / rows, r = i - t * rows;
+      const float x = __half2float(__ldg(X + t * ldx + jc + r));
+      xs[r][t] = make_float2(x, x);
+    }
+    __syncthreads();
+    if (live) {
+      const int64_t gi = jw / group;
+      __half2 zp[4], sp[4];
+      nib_pairs((uint32_t)__ldg(qzeros + gi * words + wc), zp);
+      scale_pairs(__ldg(reinterpret_cast<const uint4 *>(scales + gi * out + 8 * wc)), sp);
+#pragma unroll
+      for (int rb = 0; rb < WR; rb += RB) {
+        uint32_t wv[RB];
+#pragma unroll
+        for (int r = 0; r < RB; ++r) wv[r] = (uint32_t)__ldg(qweight + (jw + rb + r) * words + wc);
+#pragma unroll
+        for (int r = 0; r < RB; ++r) {
+          const uint4 v = dequant_word(wv[r], zp, sp);
+          const uint32_t hv[4] = {v.x, v.y, v.z, v.w};
+          float2 wf[4];
+#pragma unroll
+          for (int p = 0; p < 4; ++p) wf[p] = __half22float2(*reinterpret_cast<const __half2 *>(&hv[p]));
+          const float2 *xr = xs[WR * warp + rb + r];
+#pragma unroll
+          for (int t = 0; t < TT; ++t) {
+            const float2 xx = xr[t];
+#pragma unroll
+            for (int p = 0; p < 4; ++p) acc[t][p] = __ffma2_rn(xx, wf[p], acc[t][p]);
+          }
+        }
+      }
+    }
+  }
+  __syncthreads();  // xs and red share the buffer
+  // the warps' sums, added in a fixed order, kRedT tokens at a time
+#pragma unroll
+  for (int t0 = 0; t0 < TT; t0 += kRedT) {
+#pragma unroll
+    for (int t = 0; t < kRedT; ++t)
+      if (t0 + t < TT) {
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          red[warp][t][8 * lane + p] = acc[t0 + t][p].x;
+          red[warp][t][8 * lane + p + 4] = acc[t0 + t][p].y;
+        }
+      }
+    __syncthreads();
+    const int nt = TT - t0 < kRedT ? TT - t0 : kRedT;
+    for (int i = threadIdx.x; i < nt * kGemvOut; i += blockDim.x) {
+      const int t = i / kGemvOut, oo = i % kGemvOut;
+      const int64_t o = (int64_t)blockIdx.x * kGemvOut + oo;
+      if (o >= out) continue;
+      float sum = red[0][t][oo];
+#pragma unroll
+      for (int w = 1; w < kGemvWarps; ++w) sum += red[w][t][oo];
+      if (partials)
+        partials[((int64_t)blockIdx.y * TT + t0 + t) * out + o] = sum;
+      else
+        Y[(t0 + t) * ldy + o] = __float2half_rn(sum);
+    }
+    __syncthreads();
+  }
+}
+
+// one K split per 8 x gemv_warp_rows(T) input rows
+int w4a16_gemv_splits(int64_t T, int64_t in, int64_t out, int num_sms) {
+  (void)out;
+  (void)num_sms;
+  if (T < 1 || T > kGemvMaxT) return 0;
+  const int64_t ch = kGemvWarps * gemv_warp_rows((int)T);
+  return (int)((in + ch - 1) / ch);
+}
+
+cudaError_t launch_w4a16_gemv(const __half *X, int64_t T, int64_t in, int64_t ldx,
+                              const int32_t *qweight, const int32_t *qzeros, const __half *scales,
+                              int64_t out, int group, __half *Y, int64_t ldy, float *partials,
+                              int num_sms, cudaStream_t stream) {
+  if (T < 1 || T > kGemvMaxT || in % 64 != 0 || out % 8 != 0 ||
+      group % 32 != 0 || ldx % 8 != 0)
+    return cudaErrorInvalidValue;
+  // without room for partial sums, one block column covers all of `in`
+  (void)num_sms;
+  const int64_t k = partials ? kGemvWarps * gemv_warp_rows((int)T) : in;
+  const int splits = (int)((in + k - 1) / k);
+  float *part = splits > 1 ? partials : nullptr;
+  dim3 grid((unsigned)((out + kGemvOut - 1) / kGemvOut), (unsigned)splits);
+  const unsigned nt = kGemvWarps * 32;
+  switch (T) {
+    case 1: w4a16_gemv_kernel<1><<<grid, nt, 0, stream>>>(X, in, ldx, qweight, qzeros, scales, out, group, k, Y, ldy, part); break;
+    case 2: w4a16_gemv_kernel<2><<<grid, nt, 0, stream>>>(X, in, ldx, qweight, qzeros, scales, out, group, k, Y, ldy, part); break;
+    case 3: w4a16_gemv_kernel<3><<<grid, nt, 0, stream>>>(X, in, ldx, qweight, qzeros, scales, out, group, k, Y, ldy, part); break;
+    case 4: w4a16_gemv_kernel<4><<<grid, nt, 0, stream>>>(X, in, ldx, qweight, qzeros, scales, out, group, k, Y, ldy, part); break;
+    case 5: w4a16_gemv_kernel<5><<<grid, nt, 0, stream>>>(X, in, ldx, qweight, qzeros, scales, out, group, k, Y, ldy, part); break;
+    case 6: w4a16_gemv_kernel<6><<<grid, nt, 0, stream>>>(X, in, ldx, qweight, qzeros, scales, out, group, k, Y, ldy, part); break;
+    case 7: w4a16_gemv_kernel<7><<<grid, nt, 0, stream>>>(X, in, ldx, qweight, qzeros, scales, out, group, k, Y, ldy, part); break;
+    default: w4a16_gemv_kernel<8><<<grid, nt, 0, stream>>>(X, in, ldx, qweight, qzeros, scales, out, group, k, Y, ldy, part); break;
+  }
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || splits == 1) return e;
+  const int64_t n4 = T * out / 4;
+  w4a16_splitk_reduce_kernel<<<(unsigned)((n4 + 255) / 256), 256, 0, stream>>>(partials, splits, T, out,
+                                                                              Y, ldy);
+  return cudaGetLastError();
+}
+
 int w4a16_splits(int64_t T, int64_t in, int64_t out, int num_sms) {
   const int64_t tiles = ((T + QBM - 1) / QBM) * ((out + QBN - 1) / QBN);
   const int64_t num_kb = in / QBK;

@@ -209,3 +209,76 @@ def test_w4a16_dequantise_once_for_many_tokens(T, group):
     b = _gpu_w4a16(torch.from_numpy(Xs), qw, qz, sc, cfg, split_ws=False)  # the fused kernel
     _check(b, Xs, qw, qz, sc, group)
 
+
+
+# ------------------------------------------------------------------ decode (T <= 8)
+@pytest.mark.parametrize("T", [1, 2, 3, 5, 7, 8])
+@pytest.mark.parametrize("inn,out,group", [(4096, 1024, 128), (512, 288, 32), (1024, 544, 64)])
+def test_w4a16_decode_exact_sums(T, inn, out, group):
+    """Up to 8 tokens the product streams the packed words on CUDA cores (per
+    lane one word column, 8 input rows per batch, the warps' and the K
+    splits' fp32 sums added in a fixed order).  Power-of-two scales and
+    integer X keep every sum exact: Y is the oracle's RN16 of it, bit for
+    bit, with the K split (the workspace awq_w4a16_workspace_size asks for)
+    and without it (256 bytes: one block column over all of in).  out = 288
+    and 544 leave a block with idle word columns."""
+    cfg = awq.AwqConfig.make(group_size=group)
+    rng = np.random.default_rng(T * 1000 + inn + out)
+    qw, qz, sc = _random_packed(inn, out, group, rng, pow2_scales=True)
+    X = rng.integers(-3, 4, size=(T, inn)).astype(np.float16)
+    want = O.w4a16_matmul(X, qw, qz, sc, group).astype(np.float16)
+    for split in (True, False):
+        got = _gpu_w4a16(torch.from_numpy(X), qw, qz, sc, cfg, split_ws=split)
+        assert np.array_equal(got.view(np.uint16), want.view(np.uint16)), split
+
+
+@pytest.mark.parametrize("group", [128, 32])
+def test_w4a16_decode_dequantised_weights_bitwise(group):
+    """One-hot token rows pick single input channels (first, last, a group
+    boundary, interior ones): Y[t, :] is the column RN16((q - z) scale) of
+    the dequantised weights, bit for bit, for any fp16 scale."""
+    rng = np.random.default_rng(300 + group)
+    inn, out = 1024, 800
+    qw, qz, sc = _random_packed(inn, out, group, rng, pow2_scales=False)
+    cols = [0, inn - 1, group - 1, group, 517, 640, 3, 1000]
+    X = np.zeros((len(cols), inn), dtype=np.float16)
+    X[np.arange(len(cols)), cols] = 1.0
+    Wd = O.dequant_packed(qw, qz, sc, group)
+    for split in (True, False):
+        Yg = _gpu_w4a16(torch.from_numpy(X), qw, qz, sc, awq.AwqConfig.make(group_size=group),
+                        split_ws=split)
+        assert np.array_equal(Yg.view(np.uint16), Wd[:, cols].T.view(np.uint16)), split
+
+
+@pytest.mark.parametrize("T,w_bit,zp", [(1, 4, 1), (4, 3, 1), (8, 4, 0), (6, 4, 1)])
+def test_w4a16_decode_searched_layer(T, w_bit, zp):
+    """Packed weights of a searched 4096 x 1536 layer, decode-sized X (rows
+    of the folded calibration input): within the accumulation bound."""
+    inn, out = 4096, 1536
+    Xr, W = random_layer(256, inn, out, seed=T + 17)
+    s = O.scale_grid(O.act_stats(Xr.numpy()), O.alpha_grid(20))[11]
+    qw, qz, sc = O.quant_pack(W.numpy(), s, None, w_bit, 128, zero_point=bool(zp))
+    Xs = (Xr.numpy()[:T].astype(np.float32) / s[None, :]).astype(np.float16)
+    cfg = awq.AwqConfig.make(w_bit=w_bit, zero_point=zp)
+    for split in (True, False):
+        _check(_gpu_w4a16(torch.from_numpy(Xs), qw, qz, sc, cfg, split_ws=split), Xs, qw, qz, sc, 128)
+
+
+def test_w4a16_decode_strided_x_and_y():
+    """X and Y rows with leading dimensions above in / out."""
+    cfg = awq.AwqConfig.make()
+    inn, out, T = 512, 288, 5
+    rng = np.random.default_rng(9)
+    qw, qz, sc = _random_packed(inn, out, 128, rng, pow2_scales=True)
+    X = rng.integers(-3, 4, size=(T, inn)).astype(np.float16)
+    Xbig = torch.zeros((T, inn + 64), dtype=torch.float16, device="cuda")
+    Xbig[:, :inn] = torch.from_numpy(X).cuda()
+    Ybig = torch.full((T, out + 32), 7.0, dtype=torch.float16, device="cuda")
+    ws = torch.empty(awq.awq_w4a16_workspace_size(T, inn, out, cfg), dtype=torch.uint8, device="cuda")
+    awq.awq_w4a16_gemm(Xbig[:, :inn], torch.from_numpy(qw).cuda(), torch.from_numpy(qz).cuda(),
+                       torch.from_numpy(sc).cuda(), cfg, Ybig[:, :out], ws)
+    awq.awq_device_status(ws)
+    want = O.w4a16_matmul(X, qw, qz, sc, 128).astype(np.float16)
+    Yn = Ybig.cpu().numpy()
+    assert np.array_equal(Yn[:, :out].view(np.uint16), want.view(np.uint16))
+    assert np.all(Yn[:, out:] == 7.0)  # nothing written past out
