@@ -33,6 +33,9 @@ METRIC = "AWQ search ms/layer & candidate-GEMM TFLOP/s on 1 B200; % of TC/HBM ro
 UNIT = "ms/layer"
 WORKLOAD_INDEX = 1  # Llama-7B-shaped q_proj
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# B200 datasheet figures (dense fp16/bf16 tensor rate, HGX HBM3e bandwidth), reported beside
+# the measured denominators
+NOMINAL_PEAKS = {"hbm_gbs": 7700.0, "fp16_tflops": 2250.0}
 KERNELS_PER_STEP = {  # kernels this library launches per step (memsets excluded)
     "act_stats": 2, "wmax": 1, "scale_grid": 1, "cand_quant": 1, "search_gemm": 1,
     "mse_argmin": 1, "gram_blocks": 2, "clip_eval": 1, "quant_pack": 1,
@@ -727,11 +730,14 @@ def run_awq(args):
         "roofline": {"kernel": "search_gemm", "bound": "tensor", "achieved": round(tflops, 1),
                      "peak": peak, "unit": "TFLOP/s", "frac": round(tflops / peak, 3),
                      "frac_of_burst_peak": round(tflops / float(peaks["bf16_tflops"]), 3),
+                     "frac_of_nominal_peak": round(tflops / NOMINAL_PEAKS["fp16_tflops"], 3),
                      "traffic": traffic[0], "traffic_note": traffic[1],
                      "peak_source": f"{src} bf16 dense {'sustained' if 'bf16_tflops_sustained' in peaks else 'burst'} "
                                     "(fp16 has the same nominal rate)",
                      "algorithmic_flops_per_launch": flops},
         "hbm_kernels": {"peak_gbs": hbm, "frac": hbm_frac, "bytes_per_launch": hbm_bytes,
+                        "frac_of_nominal": {k: round(v * hbm / NOMINAL_PEAKS["hbm_gbs"], 3)
+                                            for k, v in hbm_frac.items()},
                         "cand_quant_issue": cand_quant_issue(kern["cand_quant"][0], clocks.get("sm_mhz"),
                                                              num_sms)},
         "kernels": per_kernel,
