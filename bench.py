@@ -203,14 +203,17 @@ class CudaTimer:
         return self.e0.elapsed_time(self.e1)
 
 
-def timed_steps(step, steps: int, dist, timer, barrier_device=None) -> float:
+def timed_steps(step, steps: int, dist, timer, barrier_device=None, before_stop=None) -> float:
     """Times exactly `steps` calls of `step` between a barrier + device sync on
-    both sides; returns the max over ranks of ms per step."""
+    both sides; returns the max over ranks of ms per step.  `before_stop`
+    makes the timed stream wait for work the steps left on other streams."""
     barrier(dist, barrier_device)
     timer.sync()
     timer.start()
     for _ in range(steps):
         step()
+    if before_stop is not None:
+        before_stop()
     timer.stop()
     timer.sync()
     barrier(dist, barrier_device)
@@ -478,13 +481,17 @@ def run_awq(args):
 
     # ---- end to end through the public API: pinned host buffers in, results out.
     # Consecutive layers pipeline: a step's inputs go up on a copy stream into one
-    # of two device buffers while the previous step computes; every step still
-    # copies its whole input up and its results down inside the timed region.
+    # of two device buffers while the previous step computes, and its results go
+    # down on another while the next one computes; every step still copies its
+    # whole input up and its results down inside the timed region (which ends
+    # with a device synchronisation).
     Xh, Wh = X.pin_memory(), W.pin_memory()
     Xe = [torch.empty_like(Xd), torch.empty_like(Xd)]
     We = [torch.empty_like(Wd), torch.empty_like(Wd)]
     copy_stream = torch.cuda.Stream(dev)
+    d2h_stream = torch.cuda.Stream(dev)  # results go down while the next layer computes
     ready = [torch.cuda.Event(), torch.cuda.Event()]
+    computed = torch.cuda.Event()
     done = [torch.cuda.Event(), torch.cuda.Event()]
     e2e_k = [0]
     e2e_first = [True]  # the first step of a region waits for everything before it
@@ -513,16 +520,22 @@ def run_awq(args):
             ready[b].record(copy_stream)
         cur.wait_event(ready[b])
         r = awq.quantize_layer(Xe[b], We[b], cfg, ws=ws)
-        for k, h in host_out.items():
-            h.copy_(getattr(r, k), non_blocking=True)
         done[b].record(cur)
+        computed.record(cur)
+        d2h_stream.wait_event(computed)
+        with torch.cuda.stream(d2h_stream):
+            for k, h in host_out.items():
+                t = getattr(r, k)
+                t.record_stream(d2h_stream)  # not reused before its copy is done
+                h.copy_(t, non_blocking=True)
 
     for _ in range(max(1, min(args.warmup, 2))):
         e2e_step()
     torch.cuda.synchronize(dev)
-    e_steps = max(1, min(args.steps, 10))
+    e_steps = args.steps
     e2e_first[0] = True
-    ms_e2e = timed_steps(e2e_step, e_steps, dist, timer, local)
+    ms_e2e = timed_steps(e2e_step, e_steps, dist, timer, local,
+                         before_stop=lambda: torch.cuda.current_stream(dev).wait_stream(d2h_stream))
     h2d = X.numel() * 2 + W.numel() * 2
     d2h = sum(h.numel() * h.element_size() for h in host_out.values())
 
