@@ -99,9 +99,81 @@ def save_layer_checkpoint(path: str, layer: int, res: dict) -> None:
         r = res[g]
         state[g] = {k: (v.cpu() if isinstance(v, torch.Tensor) else v) for k, v in r.items()
                     if k not in ("weights_folded", "abar")}
+    _save_atomic(state, path)
+
+
+def layer_checkpoint_path(ckpt_dir: str, layer: int) -> str:
+    return os.path.join(ckpt_dir, f"layer_{layer:03d}.pt")
+
+
+def state_checkpoint_path(ckpt_dir: str, layer: int) -> str:
+    """The fp16 hidden state entering `layer`."""
+    return os.path.join(ckpt_dir, f"hidden_{layer:03d}.pt")
+
+
+def _save_atomic(obj, path: str) -> None:
     tmp = path + ".tmp"
-    torch.save(state, tmp)
+    torch.save(obj, tmp)
     os.replace(tmp, path)
+
+
+def finished_layers(ckpt_dir: str, layers) -> int:
+    """How many of `layers` (in order) have a checkpoint: the driver resumes
+    at the first one without."""
+    n = 0
+    for layer in layers:
+        if not os.path.exists(layer_checkpoint_path(ckpt_dir, layer)):
+            break
+        n += 1
+    return n
+
+
+def quantize_layers(layers, get_weights, forward, x0: torch.Tensor, cfg: AwqConfig,
+                    ckpt_dir: Optional[str] = None, resume: bool = False,
+                    ws: Optional[torch.Tensor] = None) -> list:
+    """Layer-by-layer AWQ of a decoder (the offline pass of "AWQ and
+    Activation-Aware Scaling", Why this is attractive).  For each layer l of
+    `layers` (consecutive, ascending): w = get_weights(l); caps, x_next =
+    forward(x, w) captures the inputs of the four groups from the fp16 layer
+    (the calibration states propagate through the unquantised model);
+    quantize_layer_groups(caps, w, cfg) then searches, folds (w changes in
+    place) and packs.  With ckpt_dir, after each layer the hidden state
+    entering the next layer and then the layer's results are written, each
+    atomically, so a layer's checkpoint implies the state after it.
+    resume=True skips the layers that already have a checkpoint (from the
+    first, consecutively) and restarts from the saved state after the last
+    of them.  Returns one layer_summary per layer, the skipped ones read back
+    from their checkpoints."""
+    layers = list(layers)
+    if any(b != a + 1 for a, b in zip(layers, layers[1:])):
+        raise ValueError("layers must be consecutive and ascending")
+    summaries = []
+    start = 0
+    x = x0
+    if ckpt_dir is not None:
+        os.makedirs(ckpt_dir, exist_ok=True)
+        if resume:
+            start = finished_layers(ckpt_dir, layers)
+            for layer in layers[:start]:
+                state = torch.load(layer_checkpoint_path(ckpt_dir, layer), weights_only=False)
+                summaries.append(layer_summary(layer, state))
+            if start == len(layers):
+                return summaries
+            if start > 0:
+                x = torch.load(state_checkpoint_path(ckpt_dir, layers[start]),
+                               weights_only=False).to(x0.device)
+    for layer in layers[start:]:
+        w = get_weights(layer)
+        caps, x_next = forward(x, w)
+        if ws is None:
+            ws = workspace_for_layer(caps, w, cfg)
+        res = quantize_layer_groups(caps, w, cfg, ws)
+        summaries.append(layer_summary(layer, res))
+        if ckpt_dir is not None:
+            _save_atomic(x_next.cpu(), state_checkpoint_path(ckpt_dir, layer + 1))
+            save_layer_checkpoint(layer_checkpoint_path(ckpt_dir, layer), layer, res)
+        x = x_next
+    return summaries
 
 
 # ---------------------------------------------------------------------------
