@@ -47,8 +47,8 @@ KERNELS_PER_STEP = {  # kernels this library launches per step (memsets excluded
 # that digest; after any change to them the line carries traffic = null until
 # the kernel is captured again.
 NCU_TRAFFIC = {
-    "bytes": 13476273152 + 9685248,  # dram__bytes_read.sum + dram__bytes_write.sum
-    "sources_sha256": "0e498d6f825817c43564c43b78ab2b72ec0334c8f3c7b852b9e7bd0d19e96d05",
+    "bytes": 15623107840 + 10422016,  # dram__bytes_read.sum + dram__bytes_write.sum
+    "sources_sha256": "783bdf6248aceb0daeaef22bf3c1e10e9a61b126fa91114577c6692fc2dbc398",
     "command": ("ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none "
                 "-k regex:search_gemm -s 5 -c 1 python bench.py --steps 1 --warmup 5 "
                 "--no-cpu-baseline --no-gram-form --no-cached-form --no-w4a16 --no-workloads"),
@@ -81,7 +81,7 @@ def traffic_sources_digest() -> str:
 # instructions per SM and clock).
 NCU_ISSUE = {
     "warp_instructions": 181932996,  # smsp__inst_executed.sum
-    "sources_sha256": "50d531e6081191856f35022de41bf520b27389ebc895c26cd29457a52023a7b7",
+    "sources_sha256": "d4e9882b94cf80b89bf8583d4616ebace5d5b077e023fd69fa8981bd707c7ca9",
     "command": ("ncu --metrics smsp__inst_executed.sum,gpu__time_duration.sum --clock-control none "
                 "-k regex:cand_quant -c 1 python -m post_weight_quantization_awq_b200.run_case "
                 "--op search --tokens 16384 --in 4096 --out 4096 --repeat 1"),

@@ -360,6 +360,18 @@ awq_status awq_device_status(void *ws, awq_stream_t stream);
 /* Message describing the last failure on the calling thread ("" if none). */
 const char *awq_last_error(void);
 
+/* Index checks (no counterpart on the pages; a stand-in for a memory
+ * sanitizer).  The debug library, libawq_debug.so (built with
+ * `python -m post_weight_quantization_awq_b200.build --debug-bounds`), checks
+ * the global accesses whose indices the kernels derive from their grids: a
+ * failed check skips the access and is recorded.  awq_bounds_checks_enabled
+ * returns 1 in that library, 0 in libawq.so.  awq_bounds_status synchronises
+ * the device and returns AWQ_ERR_INVALID_ARG (the message names the kernel
+ * file and the site) if any check failed since the previous call, which
+ * clears them; AWQ_OK otherwise, and always AWQ_OK in libawq.so. */
+int32_t awq_bounds_checks_enabled(void);
+awq_status awq_bounds_status(void);
+
 /* Per-kernel timing with CUDA events recorded on the launch stream.
  * awq_profile_enable(1) starts recording every kernel this library launches;
  * awq_profile_read() synchronises the recorded events and returns, for the

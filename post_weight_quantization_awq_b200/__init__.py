@@ -19,6 +19,8 @@ from .abi import (  # noqa: F401
     awq_act_stats_finish,
     awq_act_sums,
     awq_block_grams,
+    awq_bounds_checks_enabled,
+    awq_bounds_status,
     awq_candidate_codes,
     awq_clip_candidate_codes,
     awq_device_status,

@@ -16,7 +16,10 @@ from ctypes import POINTER, c_char_p, c_double, c_float, c_int32, c_int64, c_siz
 from typing import Optional
 
 PKG_DIR = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(PKG_DIR, "libawq.so")
+# AWQ_LIB=debug loads the debug library (index checks in the kernels,
+# awq_bounds_status); the default is the release library
+LIB_PATH = os.path.join(PKG_DIR, "libawq_debug.so" if os.environ.get("AWQ_LIB") == "debug"
+                        else "libawq.so")
 HEADER_PATH = os.path.join(os.path.dirname(PKG_DIR), "include", "awq.h")
 
 STATUS = {
@@ -106,6 +109,8 @@ _SIGNATURES = {
     "awq_profile_enable": (c_int32, [c_int32]),
     "awq_profile_read": (c_int32, [c_char_p, POINTER(c_double), POINTER(c_int64)]),
     "awq_profile_reset": (c_int32, []),
+    "awq_bounds_checks_enabled": (c_int32, []),
+    "awq_bounds_status": (c_int32, []),
 }
 
 
@@ -315,6 +320,17 @@ def awq_device_status(ws, stream=None) -> None:
     failure; ws=None reads the library's own status word (the calls that take
     no workspace: awq_quant_pack, awq_search_clip_noalloc)."""
     _check("awq_device_status", LIB.awq_device_status(_ptr(ws), _stream(stream)))
+
+
+def awq_bounds_checks_enabled() -> bool:
+    """True in the debug library (index checks compiled into the kernels)."""
+    return bool(LIB.awq_bounds_checks_enabled())
+
+
+def awq_bounds_status() -> None:
+    """Raises AwqError if a kernel index check failed since the last call
+    (debug library); clears the record.  A no-op in the release library."""
+    _check("awq_bounds_status", LIB.awq_bounds_status())
 
 
 def profile_enable(on: bool) -> None:

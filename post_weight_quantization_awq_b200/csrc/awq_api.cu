@@ -869,6 +869,41 @@ awq_status awq_device_status(void *ws, awq_stream_t stream) {
   return AWQ_OK;
 }
 
+int32_t awq_bounds_checks_enabled(void) {
+#ifdef AWQ_DEBUG_BOUNDS
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+awq_status awq_bounds_status(void) {
+  g_err.clear();
+  NvtxCall nvtx_call_(__func__);
+#ifdef AWQ_DEBUG_BOUNDS
+  AWQ_TRY_CUDA(cudaDeviceSynchronize(), "device synchronize");
+  struct Unit {
+    const char *name;
+    cudaError_t (*read)(DevStatus *);
+  };
+  const Unit units[] = {{"quant_kernels", bounds_status_quant}, {"search_gemm", bounds_status_gemm},
+                        {"clip_kernels", bounds_status_clip}, {"gram_search", bounds_status_gram},
+                        {"w4a16_gemm", bounds_status_w4a16}};
+  const char *bad = nullptr;
+  uint32_t site = 0;
+  for (const Unit &u : units) {
+    DevStatus h;
+    AWQ_TRY_CUDA(u.read(&h), "bounds word read");
+    if ((h.flags & kDevOutOfBounds) && !bad) {
+      bad = u.name;
+      site = h.where;
+    }
+  }
+  if (bad) return fail(AWQ_ERR_INVALID_ARG, "an index check failed in %s (site 0x%x)", bad, site);
+#endif
+  return AWQ_OK;
+}
+
 awq_status awq_profile_enable(int32_t on) {
   std::lock_guard<std::mutex> lk(g_prof_mu);
   g_prof_on = on != 0;

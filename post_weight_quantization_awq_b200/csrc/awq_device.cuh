@@ -16,6 +16,7 @@ enum : uint32_t {
   kDevTimeout = 1u << 0,    // a bounded wait ran out
   kDevNonFinite = 1u << 1,  // a score was NaN or infinite
   kDevBadIndex = 1u << 2,   // a clip index passed to the packing was >= n_clip
+  kDevOutOfBounds = 1u << 3,  // a debug index check failed (debug library only)
 };
 
 struct DevStatus {
@@ -32,6 +33,38 @@ __device__ __forceinline__ void dev_fail(DevStatus *st, uint32_t flag, uint32_t 
     atomicCAS(&st->where, 0u, where);
   }
 }
+
+// ---------------------------------------------------------------------------
+// Debug index checks.  In the debug library (compiled with -DAWQ_DEBUG_BOUNDS:
+// `python -m post_weight_quantization_awq_b200.build --debug-bounds` writes
+// libawq_debug.so) AWQ_IN_BOUNDS(cond, site) guards a global access whose
+// index the kernel derives from its grid: a failed check records
+// kDevOutOfBounds and the first site's code in this translation unit's bounds
+// word and yields false, so the access is skipped; awq_bounds_status() reads
+// and clears the words of every unit.  In the release library the macro is
+// the constant true.
+// ---------------------------------------------------------------------------
+#ifdef AWQ_DEBUG_BOUNDS
+namespace {
+__device__ DevStatus g_bounds_status;  // one per translation unit
+__device__ __forceinline__ bool in_bounds(bool ok, uint32_t site) {
+  if (!ok) dev_fail(&g_bounds_status, kDevOutOfBounds, site);
+  return ok;
+}
+}  // namespace
+#define AWQ_IN_BOUNDS(cond, site) ::awq::in_bounds((cond), (site))
+// host reader of this unit's bounds word (read, then clear)
+#define AWQ_BOUNDS_READER(fn)                                                        \
+  cudaError_t fn(DevStatus *h) {                                                     \
+    cudaError_t e = cudaMemcpyFromSymbol(h, g_bounds_status, sizeof(DevStatus));     \
+    if (e != cudaSuccess) return e;                                                  \
+    const DevStatus zero = {};                                                       \
+    return cudaMemcpyToSymbol(g_bounds_status, &zero, sizeof(DevStatus));            \
+  }
+#else
+#define AWQ_IN_BOUNDS(cond, site) true
+#define AWQ_BOUNDS_READER(fn)
+#endif
 
 // ---------------------------------------------------------------------------
 // Group quantiser ("05 — AWQ" §5/§9: groups of g input channels, asymmetric

@@ -169,4 +169,14 @@ __host__ __device__ inline int kscale_from_wmax(float wmax) {
   return k;
 }
 
+
+#ifdef AWQ_DEBUG_BOUNDS
+// bounds words of the translation units with index checks (debug library)
+cudaError_t bounds_status_quant(DevStatus *h);
+cudaError_t bounds_status_gemm(DevStatus *h);
+cudaError_t bounds_status_clip(DevStatus *h);
+cudaError_t bounds_status_gram(DevStatus *h);
+cudaError_t bounds_status_w4a16(DevStatus *h);
+#endif
+
 }  // namespace awq

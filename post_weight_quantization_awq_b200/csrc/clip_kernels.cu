@@ -173,8 +173,10 @@ __global__ void __launch_bounds__(192, 1)
       tc_fence_after();
       const int row = q * 32 + lane;
       float *dst = partials + (((int64_t)chunk * n_groups + k) * 128 + row) * 128;
+      // the block's (group, chunk) lies in the grid's n_groups x chunks
+      const bool dst_ok = AWQ_IN_BOUNDS(k < n_groups && chunk < (int)gridDim.y, 0xB040u);
 #pragma unroll 1
-      for (int c = 0; c < 128; c += 32) {
+      for (int c = 0; c < (dst_ok ? 128 : 0); c += 32) {
         float v[32];
         tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)c, v);
         tmem_ld_wait();
@@ -490,7 +492,7 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
           (void)frexpf(2.0f * bmax, &e2);
           e2 = 14 - e2;
         }
-        if (live && ch == 0 && sp == 0) S.rexp[b][rr] = e2;
+        if (live && ch == 0 && sp == 0 && AWQ_IN_BOUNDS(rr < CT_MAXR, 0xB041u)) S.rexp[b][rr] = e2;
         const float sc = ldexpf(1.0f, e2);
         float2 ae[4];  // (r_i / s_i) 2^e, exact power-of-two scaling
 #pragma unroll
@@ -693,7 +695,7 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
           const float unscale = ldexpf(1.0f, -2 * rexp_row);
           for (int c = part; c < n_clip; c += TPP) {
             const float ev = S.epart[b][kk][rr * n_clip + c] * unscale;
-            if (err) err[((o0 + rr) * n_groups + gk) * n_clip + c] = ev;
+            if (err && AWQ_IN_BOUNDS(gk < n_groups, 0xB042u)) err[((o0 + rr) * n_groups + gk) * n_clip + c] = ev;
             if (ev < best) {
               best = ev;
               bc = c;
@@ -709,7 +711,8 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
             bc = oc;
           }
         }
-        if (row_ok && part == 0) clip_idx[(o0 + rr) * n_groups + gk] = (uint8_t)bc;
+        if (row_ok && part == 0 && AWQ_IN_BOUNDS(gk < n_groups, 0xB043u))
+          clip_idx[(o0 + rr) * n_groups + gk] = (uint8_t)bc;
       }
     }
   }
@@ -744,5 +747,7 @@ cudaError_t launch_clip_eval(const __half *W, int64_t out, int64_t in, const flo
       clip_idx, err, st, max_polls, cq, cz);
   return cudaGetLastError();
 }
+
+AWQ_BOUNDS_READER(bounds_status_clip)
 
 }  // namespace awq

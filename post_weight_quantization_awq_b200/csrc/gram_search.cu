@@ -198,7 +198,7 @@ __global__ void __launch_bounds__(192, 1)
 #pragma unroll
             for (int e = 0; e < 32; e += 4)
               *reinterpret_cast<float4 *>(row + e) = make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
-            if (bi != bj) {  // mirrored block: column gi of rows gj0 + e
+            if (bi != bj && AWQ_IN_BOUNDS(gj0 + 32 <= in, 0xB051u)) {  // mirrored block: column gi of rows gj0 + e
 #pragma unroll
               for (int e = 0; e < 32; ++e) G[(gj0 + e) * in + gi] = v[e];
             }
@@ -479,7 +479,8 @@ __global__ void __launch_bounds__(192, 1)
       double ds = (double)sum;
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) ds += __shfl_xor_sync(0xffffffffu, ds, off);
-      if (lane == 0) partials[(size_t)tile * 4 + q] = ds;  // tile = m_blk * num_n + n_blk
+      if (lane == 0 && AWQ_IN_BOUNDS(tile < num_tiles, 0xB050u))
+        partials[(size_t)tile * 4 + q] = ds;  // tile = m_blk * num_n + n_blk
     }
   }
   tc_fence_before();
@@ -510,5 +511,7 @@ cudaError_t launch_gram_score(const __half *dW, int64_t rows, int64_t in, const 
                                                       st, max_polls);
   return cudaGetLastError();
 }
+
+AWQ_BOUNDS_READER(bounds_status_gram)
 
 }  // namespace awq

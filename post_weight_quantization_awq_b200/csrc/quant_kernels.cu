@@ -54,7 +54,8 @@ __global__ void __launch_bounds__(1024) act_stats_kernel(const __half *__restric
   uint4 v[kStatsDepth];
 #pragma unroll
   for (int u = 0; u < kStatsDepth; ++u)
-    v[u] = t0 + u < t1 ? __ldcs(reinterpret_cast<const uint4 *>(p + (t0 + u) * ldx))
+    v[u] = t0 + u < t1 && AWQ_IN_BOUNDS(c0 + 8 <= in && t0 + u < T, 0xB001u)
+               ? __ldcs(reinterpret_cast<const uint4 *>(p + (t0 + u) * ldx))
                        : make_uint4(0u, 0u, 0u, 0u);
   int since = 0;
   for (int64_t t = t0; t < t1; t += kStatsDepth) {
@@ -68,7 +69,8 @@ __global__ void __launch_bounds__(1024) act_stats_kernel(const __half *__restric
         sb[2 * h + 1] += mag_scaled((w[h] >> 6) & 0x01FFFC00u);
       }
       const int64_t nx = t + u + kStatsDepth;
-      v[u] = nx < t1 ? __ldcs(reinterpret_cast<const uint4 *>(p + nx * ldx))
+      v[u] = nx < t1 && AWQ_IN_BOUNDS(nx < T, 0xB002u)
+                 ? __ldcs(reinterpret_cast<const uint4 *>(p + nx * ldx))
                      : make_uint4(0u, 0u, 0u, 0u);
     }
     since += kStatsDepth;
@@ -84,7 +86,7 @@ __global__ void __launch_bounds__(1024) act_stats_kernel(const __half *__restric
 #pragma unroll
   for (int e = 0; e < 8; ++e) {
     units[e] += __double2ull_rn(__dmul_rn(__dmul_rn(sb[e], 0x1p1008), 0x1p24));
-    if (units[e]) atomicAdd(&acc[c0 + e], units[e]);
+    if (units[e] && AWQ_IN_BOUNDS(c0 + e < in, 0xB003u)) atomicAdd(&acc[c0 + e], units[e]);
   }
 }
 
@@ -339,6 +341,9 @@ __global__ void __launch_bounds__(256, 3) cand_quant_kernel(
   const bool j_ok = j0 < in;
   const int rb_per_alpha = (int)(out_pad / kCandRows);
   const int a = (int)(blockIdx.x / rb_per_alpha);
+  // the candidate of this block lies in the grid's n_alpha x (out_pad / 64) blocks
+  const bool a_ok = (int64_t)(a + 1) * rb_per_alpha <= (int64_t)gridDim.x;
+  (void)a_ok;
   const int64_t o0 = (int64_t)(blockIdx.x - (int64_t)a * rb_per_alpha) * kCandRows;
   float2 sk[4], iv[4];  // s 2^k and r / s of this lane's 8 channels
   if (j_ok) {
@@ -461,8 +466,9 @@ __global__ void __launch_bounds__(256, 3) cand_quant_kernel(
           bq[h >> 1] |= (uint32_t)__fadd_rn(qz[h].x, zero) << (16 * (h & 1));
           bq[h >> 1] |= (uint32_t)__fadd_rn(qz[h].y, zero) << (16 * (h & 1) + 8);
         }
-        *reinterpret_cast<uint2 *>(cq + ((int64_t)a * out + o) * in + j0) = make_uint2(bq[0], bq[1]);
-        if ((lane & (lanes - 1)) == 0) {
+        if (AWQ_IN_BOUNDS(a_ok && j0 + 8 <= in, 0xB011u))
+          *reinterpret_cast<uint2 *>(cq + ((int64_t)a * out + o) * in + j0) = make_uint2(bq[0], bq[1]);
+        if ((lane & (lanes - 1)) == 0 && AWQ_IN_BOUNDS(a_ok, 0xB012u)) {
           const int64_t gi = ((int64_t)a * out + o) * (in / group) + j0 / group;
           cz[gi] = (uint8_t)zero;
           cdelta[gi] = ldexpf(dl, -k);
@@ -482,7 +488,7 @@ __global__ void __launch_bounds__(256, 3) cand_quant_kernel(
       const __half2 hv = __floats2half2_rn(d2.x, d2.y);
       packed[h] = *reinterpret_cast<const uint32_t *>(&hv);
     }
-    if (j_ok)
+    if (j_ok && AWQ_IN_BOUNDS(a_ok && o < out_pad && j0 + 8 <= in, 0xB010u))
       *reinterpret_cast<uint4 *>(dW + ((int64_t)a * out_pad + o) * in + j0) =
           make_uint4(packed[0], packed[1], packed[2], packed[3]);
   }
@@ -619,7 +625,8 @@ __global__ void __launch_bounds__(256, 4) quant_pack_kernel(
     float mx[8], mn[8];
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
-      const uint2 v = lane_ok ? __ldg(reinterpret_cast<const uint2 *>(W + (orow + r) * in + j_tile + lane * 4))
+      const uint2 v = lane_ok && AWQ_IN_BOUNDS(orow + r < out && j_tile + lane * 4 + 4 <= in, 0xB023u)
+                          ? __ldg(reinterpret_cast<const uint2 *>(W + (orow + r) * in + j_tile + lane * 4))
                               : make_uint2(0u, 0u);
       wt[r][0] = __fmul2_rn(sv[0], __half22float2(*reinterpret_cast<const __half2 *>(&v.x)));
       wt[r][1] = __fmul2_rn(sv[1], __half22float2(*reinterpret_cast<const __half2 *>(&v.y)));
@@ -635,7 +642,9 @@ __global__ void __launch_bounds__(256, 4) quant_pack_kernel(
       float r32 = 1.0f;
       bool bad = false;
       if (clip_idx) {
-        const int ci = __ldg(clip_idx + (orow + rh) * groups + kg);
+        const int ci = AWQ_IN_BOUNDS(orow + rh < out && kg < groups, 0xB024u)
+                           ? __ldg(clip_idx + (orow + rh) * groups + kg)
+                           : 0;
         if (ci < n_clip)
           r32 = clip_ratio(ci, n_clip, clip_min);
         else
@@ -649,7 +658,8 @@ __global__ void __launch_bounds__(256, 4) quant_pack_kernel(
       const int clamp = !(qlo >= 0.0f && qhi <= g.qmax);
       const int flags = (bad ? 0 : (int)g.zero) | (clamp << 8) | ((int)bad << 9);
       prm[warp][gi][rh] = make_float4(g.delta, g.rcp, g.half_lo, __int_as_float(flags));
-      scales[kg * out + orow + rh] = bad ? __ushort_as_half((unsigned short)0x7E00u) : __float2half_rn(g.delta);
+      if (AWQ_IN_BOUNDS(kg < groups && orow + rh < out, 0xB020u))
+        scales[kg * out + orow + rh] = bad ? __ushort_as_half((unsigned short)0x7E00u) : __float2half_rn(g.delta);
       if (bad) dev_fail(&g_lib_status, kDevBadIndex, 0x4B0u);
     }
     __syncwarp();
@@ -707,7 +717,8 @@ __global__ void __launch_bounds__(256, 4) quant_pack_kernel(
       words[lane * 4 + c][warp] = wl | (wh << 16);
     }
     if ((lane & (gl - 1)) == 0)  // first lane of the group: the zero points' word
-      qzeros[kg * wpr + orow / 8] = (int32_t)((uint32_t)zlo | ((uint32_t)zhi << 16));
+      if (AWQ_IN_BOUNDS(kg < groups && orow / 8 < wpr, 0xB021u))
+        qzeros[kg * wpr + orow / 8] = (int32_t)((uint32_t)zlo | ((uint32_t)zhi << 16));
     }
   }
   __syncthreads();
@@ -715,7 +726,8 @@ __global__ void __launch_bounds__(256, 4) quant_pack_kernel(
   const int w8 = rows_here / 8;
   for (int t = threadIdx.x; t < cols * 8; t += 256) {
     const int jj = t >> 3, wc = t & 7;
-    if (wc < w8) qweight[(j_tile + jj) * wpr + o0 / 8 + wc] = (int32_t)words[jj][wc];
+    if (wc < w8 && AWQ_IN_BOUNDS(j_tile + jj < in && o0 / 8 + wc < wpr, 0xB022u))
+      qweight[(j_tile + jj) * wpr + o0 / 8 + wc] = (int32_t)words[jj][wc];
   }
 }
 
@@ -753,5 +765,7 @@ cudaError_t launch_fold(__half *v, int64_t rows, int64_t cols, const float *s, c
   fold_kernel<<<(unsigned)blocks, 256, 0, stream>>>(v, rows, cols, s);
   return cudaGetLastError();
 }
+
+AWQ_BOUNDS_READER(bounds_status_quant)
 
 }  // namespace awq

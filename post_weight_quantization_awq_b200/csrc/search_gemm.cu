@@ -253,8 +253,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint4 *yp = reinterpret_cast<const uint4 *>(
                 Y + yrow + (size_t)(((int64_t)n_blk * BN) % y_cols) + c);
             uint4 yv[4];
+            const bool y_ok = AWQ_IN_BOUNDS((((int64_t)n_blk * BN) % y_cols) + c + 32 <= y_cols, 0xB031u);
 #pragma unroll
-            for (int u = 0; u < 4; ++u) yv[u] = __ldg(yp + u);
+            for (int u = 0; u < 4; ++u) yv[u] = y_ok ? __ldg(yp + u) : make_uint4(0u, 0u, 0u, 0u);
             tmem_ld_32x32b_x32(taddr + (uint32_t)c, v);
             tmem_ld_wait();
 #pragma unroll
@@ -313,7 +314,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         double ds = (double)sums[0];
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) ds += __shfl_xor_sync(0xffffffffu, ds, off);
-        if (lane == 0 && m128 < num_m) partials[((size_t)n_blk * num_m + m128) * 4 + q] = ds;
+        if (lane == 0 && m128 < num_m && AWQ_IN_BOUNDS(n_blk < num_n, 0xB030u))
+          partials[((size_t)n_blk * num_m + m128) * 4 + q] = ds;
       }
     }
   }
@@ -479,7 +481,7 @@ __global__ void __launch_bounds__(1024) mse_argmin_kernel(
   }
   if (threadIdx.x == 0) {
     const double v = ldexp(red[0], -2 * k) / ((double)T * (double)out);
-    __stcg(mse + i, v);
+    if (AWQ_IN_BOUNDS(i < n_alpha, 0xB032u)) __stcg(mse + i, v);
     __threadfence();
     last_sh = atomicAdd(&st->mse_done, 1u) == (unsigned)(n_alpha - 1);
   }
@@ -515,5 +517,7 @@ cudaError_t launch_mse_argmin(const double *partials, int n_alpha, size_t per_al
                                                   st, mse, best_idx, s_best);
   return cudaGetLastError();
 }
+
+AWQ_BOUNDS_READER(bounds_status_gemm)
 
 }  // namespace awq

@@ -437,7 +437,7 @@ __global__ void __launch_bounds__(Q_THREADS, 1) w4a16_gemm_kernel(
         tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)c2, v);
         tmem_ld_wait();
         const int64_t o0 = (int64_t)n_blk * QBN + c;
-        if (partials && t_row < T) {
+        if (partials && t_row < T && AWQ_IN_BOUNDS(sp < splits, 0xB060u)) {
           // split-K: this split's fp32 sums, in output order, for the reduction
           float *prow = partials + ((int64_t)sp * T + t_row) * out + o0;
 #pragma unroll
@@ -615,7 +615,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 2) w4a16_gemv_kernel(
     if (jc != j0) __syncthreads();  // the previous chunk's X is no longer read
     for (int i = threadIdx.x; i < rows * TT; i += kGemvWarps * 32) {
       const int t = i / rows, r = i - t * rows;
-      const float x = __half2float(__ldg(X + t * ldx + jc + r));
+      const float x = AWQ_IN_BOUNDS(jc + r < in, 0xB061u) ? __half2float(__ldg(X + t * ldx + jc + r)) : 0.0f;
       xs[r][t] = make_float2(x, x);
     }
     __syncthreads();
@@ -628,7 +628,9 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 2) w4a16_gemv_kernel(
       for (int rb = 0; rb < WR; rb += RB) {
         uint32_t wv[RB];
 #pragma unroll
-        for (int r = 0; r < RB; ++r) wv[r] = (uint32_t)__ldg(qweight + (jw + rb + r) * words + wc);
+        for (int r = 0; r < RB; ++r)
+          wv[r] = AWQ_IN_BOUNDS(jw + rb + r < in, 0xB062u) ? (uint32_t)__ldg(qweight + (jw + rb + r) * words + wc)
+                                                           : 0u;
 #pragma unroll
         for (int r = 0; r < RB; ++r) {
           const uint4 v = dequant_word(wv[r], zp, sp);
@@ -670,7 +672,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 2) w4a16_gemv_kernel(
 #pragma unroll
       for (int w = 1; w < kGemvWarps; ++w) sum += red[w][t][oo];
       if (partials)
-        partials[((int64_t)blockIdx.y * TT + t0 + t) * out + o] = sum;
+        partials[((int64_t)blockIdx.y * TT + t0 + t) * out + o] = sum;  // blockIdx.y < splits (the grid)
       else
         Y[(t0 + t) * ldy + o] = __float2half_rn(sum);
     }
@@ -759,5 +761,7 @@ cudaError_t launch_w4a16_gemm(const __half *X, int64_t T, int64_t in, int64_t ld
       partials, splits, T, out, Y, ldy);
   return cudaGetLastError();
 }
+
+AWQ_BOUNDS_READER(bounds_status_w4a16)
 
 }  // namespace awq

@@ -17,6 +17,25 @@ def test_library_exports_every_header_function():
         assert abi.LIB[n] is not None
 
 
+def test_release_library_has_no_index_checks():
+    assert not awq.awq_bounds_checks_enabled()
+    awq.awq_bounds_status()  # always AWQ_OK in the release library
+
+
+def test_debug_library_exports_every_header_function():
+    """libawq_debug.so (the same kernels with index checks), when built: the
+    same exports, and it reports its checks as enabled."""
+    import os
+    path = os.path.join(abi.PKG_DIR, "libawq_debug.so")
+    if not os.path.exists(path):
+        pytest.skip("libawq_debug.so not built")
+    lib = ctypes.CDLL(path)
+    for n in abi.header_functions():
+        assert hasattr(lib, n), n
+    lib.awq_bounds_checks_enabled.restype = ctypes.c_int32
+    assert lib.awq_bounds_checks_enabled() == 1
+
+
 def test_python_binding_has_the_abi_names():
     for n in ("awq_act_stats", "awq_scale_grid", "awq_search_scale", "awq_search_clip",
               "awq_quant_pack", "awq_fold_inv_scale", "awq_device_status", "awq_workspace_size"):

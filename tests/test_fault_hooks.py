@@ -74,7 +74,7 @@ def test_every_launching_call_is_gated():
     host-only ones."""
     host_only = {"awq_version", "awq_last_error", "awq_workspace_size", "awq_workspace_size_min",
                  "awq_w4a16_workspace_size",
-                 "awq_device_status",
+                 "awq_device_status", "awq_bounds_checks_enabled", "awq_bounds_status",
                  "awq_profile_enable", "awq_profile_read", "awq_profile_reset"}
     assert set(abi.header_functions()) - host_only == set(_launching_calls())
 
