@@ -282,6 +282,18 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- oracle arm
+def oracle_threads():
+    """Threads the oracle's timed run uses: its matrix products run in the
+    BLAS thread pool (numpy's), its elementwise steps on one thread."""
+    try:
+        import threadpoolctl
+        n = max((i.get("num_threads", 0) for i in threadpoolctl.threadpool_info()
+                 if i.get("user_api") == "blas"), default=0)
+    except Exception:
+        n = 0
+    return n if n > 0 else os.cpu_count()
+
+
 def oracle_layer_ms(X, W, wl, row_fraction: float = 1.0):
     """Times the CPU oracle on one layer of the workload: abar, X^T X, the
     alpha search, the block Grams, the clip search and the packing, in that
@@ -322,7 +334,8 @@ def oracle_layer_ms(X, W, wl, row_fraction: float = 1.0):
     total = fixed + (t["search"] + t.get("clip", 0.0) + t["pack"]) * scale
     phases = json.dumps({k: round(v, 3) for k, v in t.items()})
     if rows == out:
-        sample = (f"oracle (numpy fp64, BLAS matmuls) on the whole layer, timed as it runs: "
+        sample = (f"oracle (numpy fp64; matrix products on {oracle_threads()} BLAS threads, "
+                  f"elementwise steps on one) on the whole layer, timed as it runs: "
                   f"X [{Xn.shape[0]} x {Xn.shape[1]}], all {out} output rows; phase seconds {phases}")
     else:
         sample = (f"oracle (numpy fp64, BLAS matmuls) on the full X [{Xn.shape[0]} x {Xn.shape[1]}] "
@@ -346,7 +359,7 @@ def run_reference(args):
         if i >= args.warmup:
             vals.append(ms)
     value = statistics.mean(vals)
-    cores = os.cpu_count()
+    cores = oracle_threads()
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": UNIT,
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
@@ -707,7 +720,7 @@ def run_awq(args):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         ms_cpu, sample = oracle_layer_ms(X, W, wl, args.ref_row_fraction)
-        cpu = {"value": round(ms_cpu, 1), "unit": UNIT, "cores": os.cpu_count(), "kind": "oracle",
+        cpu = {"value": round(ms_cpu, 1), "unit": UNIT, "cores": oracle_threads(), "kind": "oracle",
                "sample": sample}
 
     if dist is not None:
