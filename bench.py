@@ -773,7 +773,8 @@ def run_awq(args):
                 "note": "quantize_layer on inputs copied from pinned host memory every step and "
                         "results copied back every step; consecutive layers pipeline (a step's "
                         "upload runs on a copy stream, into one of two buffers, while the "
-                        "previous layer computes)"},
+                        "previous layer computes, and its results go down on another stream "
+                        "while the next one computes; the timed region waits for the last)"},
         "gpu_launches": launches,
         "cpu_baseline": cpu,
         "gram_form": gram,
