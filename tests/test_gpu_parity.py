@@ -313,10 +313,12 @@ def test_gram_form_matches_direct_form_full_q_proj():
 
 # ------------------------------------------------------------------ group sizes 32 / 64
 @pytest.mark.parametrize("T,inn,out,w_bit,group,form", [
-    (300, 256, 72, 4, 32, 0), (1200, 640, 264, 3, 64, 0), (500, 384, 136, 4, 32, 1), (257, 512, 512, 4, 64, 1)])
+    (300, 256, 72, 4, 32, 0), (1200, 640, 264, 3, 64, 0), (500, 384, 136, 4, 32, 1), (257, 512, 512, 4, 64, 1),
+    (300, 64, 72, 4, 32, 0), (1, 64, 8, 4, 32, 0), (90, 192, 264, 3, 64, 0)])
 def test_search_scale_other_group_sizes(T, inn, out, w_bit, group, form):
     """Groups of 32 and 64 input channels ("AWQ and Activation-Aware Scaling",
-    When it breaks: the gain narrows at g = 32), both scoring forms."""
+    When it breaks: the gain narrows at g = 32), both scoring forms; in = 64
+    and 192 give the scored GEMM one and three K blocks."""
     X, W = random_layer(T, inn, out, seed=T + inn + group)
     cfg = awq.AwqConfig.make(w_bit=w_bit, group_size=group, search_form=form)
     g = gpu_search(X, W, cfg)

@@ -213,7 +213,8 @@ def test_w4a16_dequantise_once_for_many_tokens(T, group):
 
 # ------------------------------------------------------------------ decode (T <= 8)
 @pytest.mark.parametrize("T", [1, 2, 3, 5, 7, 8])
-@pytest.mark.parametrize("inn,out,group", [(4096, 1024, 128), (512, 288, 32), (1024, 544, 64)])
+@pytest.mark.parametrize("inn,out,group", [(4096, 1024, 128), (512, 288, 32), (1024, 544, 64),
+                                            (64, 32, 32), (320, 96, 64)])
 def test_w4a16_decode_exact_sums(T, inn, out, group):
     """Up to 8 tokens the product streams the packed words on CUDA cores (per
     lane one word column, 8 input rows per batch, the warps' and the K
