@@ -80,8 +80,8 @@ def traffic_sources_digest() -> str:
 # issue, not by HBM: its roofline is the SMs' issue rate (4 warp
 # instructions per SM and clock).
 NCU_ISSUE = {
-    "warp_instructions": 181932996,  # smsp__inst_executed.sum
-    "sources_sha256": "d4e9882b94cf80b89bf8583d4616ebace5d5b077e023fd69fa8981bd707c7ca9",
+    "warp_instructions": 168989637,  # smsp__inst_executed.sum
+    "sources_sha256": "88b90d8bb72883e259c3975510d3f50c3ea6226591d351c44bacd4cb603f78e2",
     "command": ("ncu --metrics smsp__inst_executed.sum,gpu__time_duration.sum --clock-control none "
                 "-k regex:cand_quant -c 1 python -m post_weight_quantization_awq_b200.run_case "
                 "--op search --tokens 16384 --in 4096 --out 4096 --repeat 1"),

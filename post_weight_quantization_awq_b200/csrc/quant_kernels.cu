@@ -381,11 +381,15 @@ __global__ void __launch_bounds__(256, 3) cand_quant_kernel(
   uint4 wv[kCandBatch];
   float mx[kCandBatch], mn[kCandBatch];
   const int64_t orow = o0 + (int64_t)warp * kCandWarpRows + bt * kCandBatch;
+  // row pointers of the batch: one 64-bit base, rows a 32-bit offset apart
+  // (in <= 2^20 channels, kCandBatch rows)
+  const int in32 = (int)in;
+  const __half *wrow = W + orow * in + j0;
+  __half *drow = dW ? dW + ((int64_t)a * out_pad + orow) * in + j0 : nullptr;
 #pragma unroll
   for (int r = 0; r < kCandBatch; ++r) {
     const bool live = j_ok && orow + r < out;
-    wv[r] = live ? __ldg(reinterpret_cast<const uint4 *>(W + (orow + r) * in + j0))
-                 : make_uint4(0u, 0u, 0u, 0u);
+    wv[r] = live ? __ldg(reinterpret_cast<const uint4 *>(wrow + r * in32)) : make_uint4(0u, 0u, 0u, 0u);
   }
 #pragma unroll
   for (int r = 0; r < kCandBatch; ++r) {
@@ -489,8 +493,7 @@ __global__ void __launch_bounds__(256, 3) cand_quant_kernel(
       packed[h] = *reinterpret_cast<const uint32_t *>(&hv);
     }
     if (j_ok && AWQ_IN_BOUNDS(a_ok && o < out_pad && j0 + 8 <= in, 0xB010u))
-      *reinterpret_cast<uint4 *>(dW + ((int64_t)a * out_pad + o) * in + j0) =
-          make_uint4(packed[0], packed[1], packed[2], packed[3]);
+      *reinterpret_cast<uint4 *>(drow + r * in32) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
   }
   }
 }
