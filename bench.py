@@ -81,7 +81,7 @@ def traffic_sources_digest() -> str:
 # instructions per SM and clock).
 NCU_ISSUE = {
     "warp_instructions": 168989637,  # smsp__inst_executed.sum
-    "sources_sha256": "88b90d8bb72883e259c3975510d3f50c3ea6226591d351c44bacd4cb603f78e2",
+    "sources_sha256": "7c86acea45a98a4da473c89f669b5dca4cb4af6d112b8a7fe22824866b6f013d",
     "command": ("ncu --metrics smsp__inst_executed.sum,gpu__time_duration.sum --clock-control none "
                 "-k regex:cand_quant -c 1 python -m post_weight_quantization_awq_b200.run_case "
                 "--op search --tokens 16384 --in 4096 --out 4096 --repeat 1"),

@@ -58,7 +58,10 @@ __global__ void __launch_bounds__(1024) act_stats_kernel(const __half *__restric
                ? __ldcs(reinterpret_cast<const uint4 *>(p + (t0 + u) * ldx))
                        : make_uint4(0u, 0u, 0u, 0u);
   int since = 0;
-  for (int64_t t = t0; t < t1; t += kStatsDepth) {
+  // the next row to load, and the rows left from the current one (< 2^22)
+  const __half *pn = p + (t0 + kStatsDepth) * ldx;
+  int left = (int)(t1 - t0);
+  for (int64_t t = t0; t < t1; t += kStatsDepth, left -= kStatsDepth) {
 #pragma unroll
     for (int u = 0; u < kStatsDepth; ++u) {
       // rows past t1 were loaded as zeros and add nothing
@@ -68,10 +71,10 @@ __global__ void __launch_bounds__(1024) act_stats_kernel(const __half *__restric
         sb[2 * h] += mag_scaled((w[h] << 10) & 0x01FFFC00u);
         sb[2 * h + 1] += mag_scaled((w[h] >> 6) & 0x01FFFC00u);
       }
-      const int64_t nx = t + u + kStatsDepth;
-      v[u] = nx < t1 && AWQ_IN_BOUNDS(nx < T, 0xB002u)
-                 ? __ldcs(reinterpret_cast<const uint4 *>(p + nx * ldx))
-                     : make_uint4(0u, 0u, 0u, 0u);
+      v[u] = u + kStatsDepth < left && AWQ_IN_BOUNDS(t + u + kStatsDepth < T, 0xB002u)
+                 ? __ldcs(reinterpret_cast<const uint4 *>(pn))
+                 : make_uint4(0u, 0u, 0u, 0u);
+      pn += ldx;
     }
     since += kStatsDepth;
     if (since == kStatsExactRows) {
