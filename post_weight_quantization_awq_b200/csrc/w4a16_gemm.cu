@@ -489,29 +489,40 @@ __global__ void __launch_bounds__(256) w4a16_dequant_kernel(
     const int32_t *__restrict__ qweight, const int32_t *__restrict__ qzeros,
     const __half *__restrict__ scales, int64_t in, int64_t out, int group, __half *__restrict__ Wd) {
   constexpr int TJ = 128, TO = 64, WPR = TO / 8;  // inputs, outputs, words per input row
-  __shared__ __align__(16) __half tile[TO][TJ + 8];
+  // [output][input] with the 16-byte chunks of row r XOR-swizzled by r / 8, so
+  // that the 2-byte writes of one warp (8 word columns, i.e. rows 8 apart)
+  // fall in different banks and the 16-byte row reads stay aligned
+  __shared__ __align__(16) __half tile[TO][TJ];
   const int64_t j0 = (int64_t)blockIdx.x * TJ, o0 = (int64_t)blockIdx.y * TO;
   const int64_t words = out / 8;
+  // a thread converts the words of two consecutive input rows of one word
+  // column (one group: group % 32 == 0) and writes each output's two weights
+  // as one half2
 #pragma unroll
-  for (int i = 0; i < TJ * WPR / 256; ++i) {
+  for (int i = 0; i < TJ * WPR / 512; ++i) {
     const int w = threadIdx.x + 256 * i;
-    const int jj = w / WPR, ow = w % WPR;  // input row of the tile, word column
+    const int jp = w / WPR, ow = w % WPR;  // input row pair of the tile, word column
+    const int jj = 2 * jp;
     const int64_t j = j0 + jj, wc = o0 / 8 + ow;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (j < in && wc < words) {
+    uint4 v0 = make_uint4(0u, 0u, 0u, 0u), v1 = v0;
+    if (j < in && wc < words) {  // in % 64 == 0: rows j and j + 1 are both in
       const int64_t gi = j / group;
       __half2 zp[4], sp[4];
       nib_pairs((uint32_t)__ldg(qzeros + gi * words + wc), zp);
       scale_pairs(__ldg(reinterpret_cast<const uint4 *>(scales + gi * out + 8 * wc)), sp);
-      v = dequant_word((uint32_t)__ldg(qweight + j * words + wc), zp, sp);
+      const int32_t *qp = qweight + j * words + wc;
+      v0 = dequant_word((uint32_t)__ldg(qp), zp, sp);
+      v1 = dequant_word((uint32_t)__ldg(qp + words), zp, sp);
     }
-    // v holds outputs 0,4,1,5,2,6,3,7 of the word
-    const uint32_t h[4] = {v.x, v.y, v.z, v.w};
+    // v0 / v1 hold outputs 0,4,1,5,2,6,3,7 of the word in rows jj / jj + 1
+    const uint32_t h0[4] = {v0.x, v0.y, v0.z, v0.w}, h1[4] = {v1.x, v1.y, v1.z, v1.w};
+    const int col = (((jj >> 3) ^ ow) << 3) | (jj & 7);  // rows 8 ow .. 8 ow + 7 share the swizzle
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
-      const __half2 pr = *reinterpret_cast<const __half2 *>(&h[p]);
-      tile[8 * ow + p][jj] = __low2half(pr);
-      tile[8 * ow + p + 4][jj] = __high2half(pr);
+      // output p: low halves of row jj and row jj + 1; output p + 4: the high halves
+      const uint32_t lo = __byte_perm(h0[p], h1[p], 0x5410u), hi = __byte_perm(h0[p], h1[p], 0x7632u);
+      *reinterpret_cast<uint32_t *>(&tile[8 * ow + p][col]) = lo;
+      *reinterpret_cast<uint32_t *>(&tile[8 * ow + p + 4][col]) = hi;
     }
   }
   __syncthreads();
@@ -521,7 +532,8 @@ __global__ void __launch_bounds__(256) w4a16_dequant_kernel(
     const int oo = c / (TJ / 8), jc = c % (TJ / 8);  // output row, 8-input chunk
     const int64_t o = o0 + oo, j = j0 + 8 * jc;
     if (o < out && j < in)  // in % 64 == 0: a chunk is whole
-      *reinterpret_cast<uint4 *>(Wd + o * in + j) = *reinterpret_cast<const uint4 *>(&tile[oo][8 * jc]);
+      *reinterpret_cast<uint4 *>(Wd + o * in + j) =
+          *reinterpret_cast<const uint4 *>(&tile[oo][8 * (jc ^ (oo >> 3))]);
   }
 }
 
