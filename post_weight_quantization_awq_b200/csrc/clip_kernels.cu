@@ -385,24 +385,27 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
     const int cper = (n_clip + nsp - 1) / nsp;       // ratios per split, <= 16
     int64_t k_cur = -1;
     float sv[8], rv[8], av[8];                       // s_i, r_i, r_i / s_i of the chunk
+    // the unit of each pass (row rr, split sp) does not change from tile to
+    // tile: take the divisions by R once
+    const int u0 = warp * 32 + lane, u1 = u0 + CW_PROD * 32;
+    const int rr0 = (u0 >> 4) % R, sp0 = (u0 >> 4) / R, rr1 = (u1 >> 4) % R, sp1 = (u1 >> 4) / R;
     uint4 wpre[2];
-    auto load_rows = [&](int64_t it) {
-      const int64_t kk = it / n_tiles, oo = (it - kk * n_tiles) * R;
+    auto load_rows = [&](int64_t kk, int64_t oo) {
 #pragma unroll
       for (int pass = 0; pass < 2; ++pass) {
-        const int u = warp * 32 + pass * CW_PROD * 32 + lane;
-        const int rr = (u >> 4) % R;
-        const int64_t o = oo + rr;
-        wpre[pass] = (u < nunits && o < out)
+        const int64_t o = oo + (pass ? rr1 : rr0);
+        wpre[pass] = ((pass ? u1 : u0) < nunits && o < out)
                          ? __ldg(reinterpret_cast<const uint4 *>(W + o * in + kk * G + 8 * ch))
                          : make_uint4(0u, 0u, 0u, 0u);
       }
     };
-    if (item_begin < item_end) load_rows(item_begin);
+    // (group k, row tile tl) of the current item, stepped without a 64-bit
+    // division per tile
+    int64_t k = item_begin / n_tiles, tl = item_begin - k * n_tiles;
+    if (item_begin < item_end) load_rows(k, tl * R);
     for (int64_t item = item_begin; item < item_end; ++item) {
       const int t = (int)(item - item_begin);
       const int b = t & 1;
-      const int64_t k = item / n_tiles;
       const bool new_group = k != k_cur;
       // buffer b is free once tile t-2 is scored; a new G~ also needs tile t-1 done
       if (ptid == 0) {
@@ -463,7 +466,7 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
         if (ub >= nunits) break;
         const int u = ub + lane;
         const bool live = u < nunits;
-        const int rr = (u >> 4) % R, sp = (u >> 4) / R;
+        const int rr = pass ? rr1 : rr0, sp = pass ? sp1 : sp0;
         // ---- this row's range (s w) and the exponent of the d~ scaling
         const uint4 wv = pass ? wpre[1] : wpre[0];  // no dynamic register indexing
         const uint32_t wr[4] = {wv.x, wv.y, wv.z, wv.w};
@@ -557,7 +560,7 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
           }
           if (store) split_store8(ahi, alo, sw128_off(p0 + c, ch & 7), v);
           if constexpr (kCodes) {
-            const int64_t o = (item - k * n_tiles) * R + rr;
+            const int64_t o = tl * R + rr;
             if (store && o < out) {
               uint32_t cw[2] = {0u, 0u};
 #pragma unroll
@@ -573,7 +576,11 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
           }
         }
       }
-      if (item + 1 < item_end) load_rows(item + 1);
+      if (++tl == n_tiles) {
+        tl = 0;
+        ++k;
+      }
+      if (item + 1 < item_end) load_rows(k, tl * R);
       fence_async_smem();  // generic-proxy writes (A and, on a new group, B) -> tensor cores
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.a_full[b]);
@@ -619,12 +626,16 @@ __global__ void __launch_bounds__(CT_THREADS, 1) clip_tc_kernel(
     const int etid = tid - CW_EPI * 32;  // 0..127
     const int q = warp & 3;              // TMEM lane quarter of this warp
     const int p = q * 32 + lane;         // candidate (accumulator row)
-    for (int64_t item = item_begin; item < item_end; ++item) {
+    int64_t k = item_begin / n_tiles, tl = item_begin - k * n_tiles;
+    for (int64_t item = item_begin; item < item_end; ++item, ++tl) {
       const int t = (int)(item - item_begin);
       const int b = t & 1;
       const uint32_t ph = (t >> 1) & 1;
-      const int64_t k = item / n_tiles;
-      const int64_t o0 = (item - k * n_tiles) * R;
+      if (tl == n_tiles) {
+        tl = 0;
+        ++k;
+      }
+      const int64_t o0 = tl * R;
       if (etid == 0) {
         // acc_full: the products are in TMEM; a_full (already complete) makes
         // the producers' plain stores of A and the row data visible here
