@@ -66,6 +66,22 @@ def test_alpha_grid_endpoints_and_spacing():
     assert list(O.alpha_grid(1)) == [0.0]
 
 
+def test_alpha_grid_is_the_correctly_rounded_quotient():
+    """alpha_i is the double nearest the rational i / (n - 1) (the even grid
+    on [0, 1] of "05 — AWQ" §4): checked in exact arithmetic against both
+    neighbouring doubles.  A grid built as i * (1 / (n - 1)) misses this at
+    i = 13 and 17 for n = 20 (and at i = 7 for n = 10)."""
+    for n in (2, 3, 7, 10, 20, 64):
+        a = O.alpha_grid(n)
+        for i in range(n):
+            exact = Fraction(i, n - 1)
+            err = abs(Fraction(float(a[i])) - exact)
+            for nb in (math.nextafter(float(a[i]), -math.inf), math.nextafter(float(a[i]), math.inf)):
+                assert err <= abs(Fraction(nb) - exact), (n, i)
+    recip = [i * (1.0 / 19) for i in range(20)]
+    assert [i for i in range(20) if recip[i] != O.alpha_grid(20)[i]] == [13, 17]
+
+
 def test_scale_grid_closed_forms():
     rng = np.random.default_rng(2)
     abar = np.exp(rng.normal(0, 2, size=2000))
