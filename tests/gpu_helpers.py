@@ -71,3 +71,37 @@ def midpoint_report(abar: np.ndarray, alphas: np.ndarray, s_gpu: np.ndarray, s_r
         lines.append(f"alpha[{i}] ch {j}: pow={v!r} fp32 gpu={s_gpu[i, j]!r} ref={s_ref[i, j]!r} "
                      f"|pow-mid|/ulp={abs(v - mid) / (hi - lo):.3e}")
     return "\n".join(lines)
+
+
+def layer_parity(X, W, w_bit, n_alpha, n_clip, rows=None):
+    """The whole path at full T and in; with `rows`, on that sample of output
+    rows (the same launch configuration with a smaller N)."""
+    if rows is not None:
+        W = W[rows]
+    cfg = awq.AwqConfig.make(w_bit=w_bit, n_alpha=n_alpha, n_clip=n_clip)
+    Xd, Wd = to_dev(X), to_dev(W)
+    ws = awq.alloc_workspace(Xd.shape[0], Xd.shape[1], Wd.shape[0], cfg)
+    res = awq.quantize_layer(Xd, Wd, cfg, ws=ws)
+    awq.awq_device_status(ws)
+    torch.cuda.synchronize()
+    Xn, Wn = X.numpy(), W.numpy()
+    abar = O.act_stats(Xn)
+    assert np.array_equal(res.abar.cpu().numpy(), abar)
+    mse, best, s_best, S = O.search_scale(Xn, Wn, abar, w_bit, 128, n_alpha)
+    g_mse = res.mse.cpu().numpy()
+    check_mse(g_mse, mse)
+    g_best = int(res.best_idx.item())
+    check_selection(g_best, mse, "alpha")
+    s = S[g_best]
+    assert np.array_equal(res.s_best.cpu().numpy(), s)
+    clip_idx = None
+    if n_clip:
+        clip_idx = res.clip_idx.cpu().numpy()
+        idx_o, E = O.search_clip(Xn, Wn, s, w_bit, 128, n_clip, 0.5)
+        for o, k in zip(*np.nonzero(clip_idx != idx_o)):
+            check_selection(int(clip_idx[o, k]), E[o, k], f"clip row {o} group {k}")
+    qw, qz, sc = O.quant_pack(Wn, s, clip_idx, w_bit, 128, max(n_clip, 1), 0.5)
+    assert np.array_equal(res.qweight.cpu().numpy(), qw)
+    assert np.array_equal(res.qzeros.cpu().numpy(), qz)
+    assert np.array_equal(res.scales.cpu().numpy().view(np.uint16), sc.view(np.uint16))
+    return g_mse, mse

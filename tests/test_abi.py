@@ -80,6 +80,7 @@ def test_workspace_size_grows_with_the_problem():
     (dict(), (256, 500, 512), "AWQ_ERR_INVALID_ARG"),
     (dict(), (256, 512, 12), "AWQ_ERR_INVALID_ARG"),
     (dict(), (0, 512, 512), "AWQ_ERR_INVALID_ARG"),
+    (dict(), ((1 << 22) + 1, 512, 512), "AWQ_ERR_INVALID_ARG"),  # past the exact-sum bound
 ])
 def test_host_validation(kw, shape, status):
     cfg = awq.AwqConfig.make(**kw)
