@@ -3,8 +3,8 @@ activation sum sets: 2^22 tokens x 65504 x 2^24 units < 2^63), on a narrow
 layer so that the oracle still finishes in seconds: the activation statistic
 at its largest possible sums, the whole path (statistic, alpha search, clip
 search, packing) against the oracle, and the W4A16 product in both
-tensor-core forms.  Below that bound and above it, the host checks are in
-test_abi.py."""
+tensor-core forms; and a weight matrix of more than 2^31 elements.  The host
+check past the token bound is in test_abi.py."""
 
 import numpy as np
 import pytest
@@ -14,7 +14,7 @@ import post_weight_quantization_awq_b200 as awq
 from oracle import awq_oracle as O
 from synthetic import OutlierSpec, heavy_tailed_activations, random_layer
 
-from gpu_helpers import layer_parity, need_cuda, to_dev
+from gpu_helpers import check_selection, layer_parity, need_cuda, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -80,3 +80,39 @@ def test_w4a16_at_the_maximum_token_count(form):
     ulp = np.exp2(np.floor(np.log2(np.maximum(a, 2.0 ** -14))) - 10)
     err = np.abs(Yg - Yo)
     assert np.all(err <= 0.5 * ulp + acc), err.max()
+
+
+def test_weight_matrix_past_2_31_elements():
+    """W [2^20 + 64, 2048] holds 2^31 + 131072 weights, so row and element
+    offsets past 2^31 must be 64-bit in every kernel that walks W or the
+    candidate operand (candidates, scored GEMM, clip search, packing).
+    n_alpha = 1 (alpha = 0: s = 1, plain quantisation) keeps the check per
+    row: the clip indices and the packed output are compared with the oracle
+    on 8-row blocks at both ends of W and on both sides of element 2^31."""
+    T, inn, out = 64, 2048, (1 << 20) + 64
+    X = heavy_tailed_activations(T, inn, OutlierSpec(0.01, 20.0, 50.0), seed=31)
+    gen = torch.Generator(device="cuda").manual_seed(31)
+    Wd = (0.02 * torch.randn((out, inn), generator=gen, device="cuda")).half()
+    cfg = awq.AwqConfig.make(n_alpha=1, n_clip=20)
+    ws = awq.alloc_workspace(T, inn, out, cfg)
+    res = awq.quantize_layer(to_dev(X), Wd, cfg, ws=ws)
+    awq.awq_device_status(ws)
+    torch.cuda.synchronize()
+    Xn = X.numpy()
+    assert np.array_equal(res.abar.cpu().numpy(), O.act_stats(Xn))
+    assert int(res.best_idx.item()) == 0 and bool(torch.all(res.s_best == 1.0))
+    ones = np.ones(inn, dtype=np.float32)
+    Gk = O.block_grams(Xn, 128)
+    rng = np.random.default_rng(31)
+    blocks = [0, (1 << 20) - 8, 1 << 20, out - 8] + [8 * int(b) for b in rng.integers(0, out // 8, 4)]
+    for o0 in blocks:
+        Wn = Wd[o0:o0 + 8].cpu().numpy()
+        idx_o, E = O.search_clip(Xn, Wn, ones, 4, 128, 20, 0.5, Gk=Gk)
+        idx_g = res.clip_idx[o0:o0 + 8].cpu().numpy()
+        for o, k in zip(*np.nonzero(idx_g != idx_o)):
+            check_selection(int(idx_g[o, k]), E[o, k], f"clip row {o0 + o} group {k}")
+        qw, qz, sc = O.quant_pack(Wn, ones, idx_g, 4, 128, 20, 0.5)
+        w = o0 // 8
+        assert np.array_equal(res.qweight[:, w:w + 1].cpu().numpy(), qw), o0
+        assert np.array_equal(res.qzeros[:, w:w + 1].cpu().numpy(), qz), o0
+        assert np.array_equal(res.scales[:, o0:o0 + 8].cpu().numpy().view(np.uint16), sc.view(np.uint16)), o0
