@@ -493,7 +493,8 @@ __global__ void __launch_bounds__(256) w4a16_dequant_kernel(
   // that the 2-byte writes of one warp (8 word columns, i.e. rows 8 apart)
   // fall in different banks and the 16-byte row reads stay aligned
   __shared__ __align__(16) __half tile[TO][TJ];
-  const int64_t j0 = (int64_t)blockIdx.x * TJ, o0 = (int64_t)blockIdx.y * TO;
+  // outputs along x (up to 2^22 / 64 blocks), inputs along y (at most 2^20 / 128)
+  const int64_t o0 = (int64_t)blockIdx.x * TO, j0 = (int64_t)blockIdx.y * TJ;
   const int64_t words = out / 8;
   // a thread converts the words of two consecutive input rows of one word
   // column (one group: group % 32 == 0) and writes each output's two weights
@@ -540,7 +541,7 @@ __global__ void __launch_bounds__(256) w4a16_dequant_kernel(
 cudaError_t launch_w4a16_dequant(const int32_t *qweight, const int32_t *qzeros, const __half *scales,
                                  int64_t in, int64_t out, int group, __half *Wd, cudaStream_t stream) {
   if (in % 64 != 0 || out % 8 != 0 || group % 32 != 0) return cudaErrorInvalidValue;
-  dim3 grid((unsigned)((in + 127) / 128), (unsigned)((out + 63) / 64));
+  dim3 grid((unsigned)((out + 63) / 64), (unsigned)((in + 127) / 128));
   w4a16_dequant_kernel<<<grid, 256, 0, stream>>>(qweight, qzeros, scales, in, out, group, Wd);
   return cudaGetLastError();
 }
