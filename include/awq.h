@@ -88,8 +88,15 @@ typedef enum {
  *                       Y tile and sums the squares (2 T in out (n_alpha + 1)
  *                       flops; the 1/s of the activation side is folded into
  *                       the candidate weights so that every candidate shares
- *                       one staged X tile). */
-enum { AWQ_SEARCH_DIRECT = 0, AWQ_SEARCH_GRAM = 1, AWQ_SEARCH_CACHED_Y = 2 };
+ *                       one staged X tile);
+ *   AWQ_SEARCH_FUSED    the direct form with the candidates made inside the
+ *                       GEMM: each B tile is converted from the W rows in
+ *                       shared memory (from per-group steps and zero points,
+ *                       16 bytes per alpha, row and group in the workspace), so
+ *                       the n_alpha x out x in operand is never written; the
+ *                       same MSE bits as AWQ_SEARCH_DIRECT, with the conversion
+ *                       repeated for every 256-token tile. */
+enum { AWQ_SEARCH_DIRECT = 0, AWQ_SEARCH_GRAM = 1, AWQ_SEARCH_CACHED_Y = 2, AWQ_SEARCH_FUSED = 3 };
 
 /* Quantisation and search settings; the first three fields are the pages'
  * quant_config ("05 — AWQ" §9: w_bit, q_group_size, zero_point). */
@@ -106,8 +113,8 @@ typedef struct {
   int32_t n_alpha;    /* alpha grid size, 1..64; alpha_i = i/(n_alpha-1) ("05 — AWQ" §4: ~20) */
   int32_t n_clip;     /* clip grid size, 0 = no clip search, else 1..64          */
   float clip_min;     /* smallest clip ratio, in (0, 1]; ("05 — AWQ" §4: 0.5)    */
-  int32_t search_form; /* AWQ_SEARCH_DIRECT (0, default), AWQ_SEARCH_GRAM (1) or
-                          AWQ_SEARCH_CACHED_Y (2)                                */
+  int32_t search_form; /* AWQ_SEARCH_DIRECT (0, default), AWQ_SEARCH_GRAM (1),
+                          AWQ_SEARCH_CACHED_Y (2) or AWQ_SEARCH_FUSED (3)        */
 } awq_config;
 
 /* Bytes of workspace needed by awq_search_scale and awq_search_clip for a

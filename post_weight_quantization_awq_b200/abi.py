@@ -40,7 +40,7 @@ class AwqError(RuntimeError):
         super().__init__(f"{func}: {self.status_name}: {message}")
 
 
-SEARCH_DIRECT, SEARCH_GRAM, SEARCH_CACHED_Y = 0, 1, 2
+SEARCH_DIRECT, SEARCH_GRAM, SEARCH_CACHED_Y, SEARCH_FUSED = 0, 1, 2, 3
 
 
 class AwqConfig(ctypes.Structure):

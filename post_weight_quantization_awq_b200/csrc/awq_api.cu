@@ -120,9 +120,9 @@ awq_status check_cfg(const awq_config *cfg) {
   if (!(cfg->clip_min > 0.0f && cfg->clip_min <= 1.0f))
     return fail(AWQ_ERR_INVALID_ARG, "clip_min=%g (must be in (0, 1])", (double)cfg->clip_min);
   if (cfg->search_form != AWQ_SEARCH_DIRECT && cfg->search_form != AWQ_SEARCH_GRAM &&
-      cfg->search_form != AWQ_SEARCH_CACHED_Y)
-    return fail(AWQ_ERR_INVALID_ARG, "search_form=%d (0 direct, 1 Gram, 2 cached fp16 output)",
-                cfg->search_form);
+      cfg->search_form != AWQ_SEARCH_CACHED_Y && cfg->search_form != AWQ_SEARCH_FUSED)
+    return fail(AWQ_ERR_INVALID_ARG,
+                "search_form=%d (0 direct, 1 Gram, 2 cached fp16 output, 3 fused)", cfg->search_form);
   return AWQ_OK;
 }
 
@@ -185,8 +185,10 @@ ScaleWs scale_layout(int64_t T, int64_t in, int64_t out, const awq_config *cfg, 
   off = align256(off + sizeof(float) * (size_t)cfg->n_alpha * in);
   w.inv_s = off;
   off = align256(off + sizeof(float) * (size_t)cfg->n_alpha * in);
-  w.dW = off;
-  off = align256(off + sizeof(__half) * (size_t)n_chunk * w.out_pad * in);
+  w.dW = off;  // fused form: the per-group parameters instead of the operand
+  off = align256(off + (cfg->search_form == AWQ_SEARCH_FUSED
+                            ? sizeof(float4) * (size_t)cfg->n_alpha * w.out_pad * (in / cfg->group_size)
+                            : sizeof(__half) * (size_t)n_chunk * w.out_pad * in));
   w.partials = off;
   off = align256(off + sizeof(double) * (size_t)cfg->n_alpha * w.per_alpha);
   w.G = w.ghi = w.glo = w.r = w.Y = 0;
@@ -440,9 +442,27 @@ awq_status search_scale_impl(const void *X, int64_t T, int64_t in, int64_t ldx, 
     ProfScope p("scale_grid", s);
     AWQ_TRY_CUDA(launch_scale_grid(abar, in, cfg->n_alpha, s_grid, inv_s, s), "scale_grid launch");
   }
+  if (cfg->search_form == AWQ_SEARCH_FUSED) {
+    // every candidate's per-group parameters, then the GEMM that builds its
+    // B tiles from them and the W rows (the operand is never stored)
+    float4 *params = reinterpret_cast<float4 *>(base + L.dW);
+    {
+      ProfScope p("fused_params", s);
+      AWQ_TRY_CUDA(launch_fused_params(static_cast<const __half *>(W), out, in, L.out_pad, s_grid,
+                                       cfg->n_alpha, cfg->group_size, cfg->w_bit, cfg->zero_point, dst,
+                                       params, s),
+                   "fused_params launch");
+    }
+    ProfScope p("fused_gemm", s);
+    AWQ_TRY_CUDA(launch_fused_search_gemm(static_cast<const __half *>(X), T, ldx,
+                                          static_cast<const __half *>(W), out, in, L.out_pad,
+                                          cfg->n_alpha, s_grid, inv_s, params, cfg->group_size,
+                                          cfg->w_bit, partials, dst, poll_cap(), nsm, s),
+                 "fused_search_gemm launch");
+  }
   // the candidates in chunks of `chunk` (all at once with a full workspace):
   // each chunk's operand, then its scores into its slots of the partials
-  for (int a0 = 0; a0 < cfg->n_alpha; a0 += chunk) {
+  for (int a0 = 0; cfg->search_form != AWQ_SEARCH_FUSED && a0 < cfg->n_alpha; a0 += chunk) {
     const int cnt = cfg->n_alpha - a0 < chunk ? cfg->n_alpha - a0 : chunk;
     double *part = partials + (size_t)a0 * L.per_alpha;
     {
@@ -888,7 +908,7 @@ awq_status awq_bounds_status(void) {
   };
   const Unit units[] = {{"quant_kernels", bounds_status_quant}, {"search_gemm", bounds_status_gemm},
                         {"clip_kernels", bounds_status_clip}, {"gram_search", bounds_status_gram},
-                        {"w4a16_gemm", bounds_status_w4a16}};
+                        {"w4a16_gemm", bounds_status_w4a16}, {"fused_search", bounds_status_fused}};
   const char *bad = nullptr;
   uint32_t site = 0;
   for (const Unit &u : units) {

@@ -2,7 +2,7 @@
 (ncu) and quick timing.
 
     python -m post_weight_quantization_awq_b200.run_case --op search --tokens 16384 \
-        --in 4096 --out 4096 [--alphas 20] [--clips 20] [--bits 4] [--repeat 3] [--form gram|cached_y]
+        --in 4096 --out 4096 [--alphas 20] [--clips 20] [--bits 4] [--repeat 3] [--form gram|cached_y|fused]
 
 --op is one of: stats, search, clip, pack, layer (all four calls), w4a16 (the
 GEMM on the packed output, Y = X Wd^T with Wd = RN16((q - z) scale); with
@@ -38,7 +38,7 @@ def main(argv=None) -> int:
     ap.add_argument("--bits", type=int, default=4)
     ap.add_argument("--repeat", type=int, default=3)
     ap.add_argument("--seed", type=int, default=1)
-    ap.add_argument("--form", choices=("direct", "gram", "cached_y"), default="direct",
+    ap.add_argument("--form", choices=("direct", "gram", "cached_y", "fused"), default="direct",
                     help="alpha-search scoring form")
     ap.add_argument("--w4a16-form", choices=("auto", "fused"), default="auto",
                     help="auto: the workspace awq_w4a16_workspace_size asks for (dequantise once "
@@ -49,7 +49,8 @@ def main(argv=None) -> int:
     W = gaussian_weight(a.out, a.inn, a.seed).cuda()
     cfg = awq.AwqConfig.make(w_bit=a.bits, n_alpha=a.alphas, n_clip=a.clips,
                              search_form={"direct": awq.abi.SEARCH_DIRECT, "gram": awq.abi.SEARCH_GRAM,
-                                          "cached_y": awq.abi.SEARCH_CACHED_Y}[a.form])
+                                          "cached_y": awq.abi.SEARCH_CACHED_Y,
+                                          "fused": awq.abi.SEARCH_FUSED}[a.form])
     ws = awq.alloc_workspace(a.tokens, a.inn, a.out, cfg)
     abar = torch.empty(a.inn, dtype=torch.float64, device="cuda")
     mse = torch.empty(a.alphas, dtype=torch.float64, device="cuda")

@@ -28,9 +28,10 @@ def _packed(rng_seed, inn, out, group):
 def run(out_path: str) -> None:
     res = {}
     # the whole path (stats, alpha search, clip search, packing) in every scoring
-    # form, with and without a zero point, at the three group sizes
+    # form (direct, Gram, cached output, fused), with and without a zero point,
+    # at the three group sizes
     cases = [(300, 384, 136, 4, 128, 1, 0), (4173, 512, 264, 3, 128, 1, 1), (257, 256, 72, 4, 32, 1, 2),
-             (1000, 640, 520, 4, 64, 0, 0), (600, 512, 264, 4, 128, 1, 1)]
+             (1000, 640, 520, 4, 64, 0, 0), (600, 512, 264, 4, 128, 1, 1), (700, 512, 136, 4, 32, 1, 3)]
     for i, (T, inn, out, w_bit, group, zp, form) in enumerate(cases):
         X, W = (edge_layer if i == 4 else random_layer)(T, inn, out, seed=100 + i, **(
             {"group": group} if i == 4 else {}))

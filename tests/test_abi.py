@@ -182,7 +182,7 @@ def test_sharding_calls_check_their_arguments():
 
 
 def test_search_forms_and_zero_point_are_validated():
-    for kw, status in ((dict(search_form=3), "AWQ_ERR_INVALID_ARG"), (dict(zero_point=-1), "AWQ_ERR_INVALID_ARG")):
+    for kw, status in ((dict(search_form=4), "AWQ_ERR_INVALID_ARG"), (dict(zero_point=-1), "AWQ_ERR_INVALID_ARG")):
         with pytest.raises(awq.AwqError) as ei:
             awq.awq_workspace_size(256, 512, 512, awq.AwqConfig.make(**kw))
         assert ei.value.status_name == status
@@ -190,6 +190,11 @@ def test_search_forms_and_zero_point_are_validated():
     a = awq.awq_workspace_size(1000, 512, 512, awq.AwqConfig.make())
     b = awq.awq_workspace_size(1000, 512, 512, awq.AwqConfig.make(search_form=abi.SEARCH_CACHED_Y))
     assert b - a >= 1024 * 512 * 2
+    # the fused form keeps 16 bytes per (alpha, row, group) instead of the
+    # n_alpha x out_pad x in fp16 operand, whatever the workspace
+    c = awq.awq_workspace_size(1000, 512, 512, awq.AwqConfig.make(search_form=abi.SEARCH_FUSED))
+    assert a - c == 20 * 512 * 512 * 2 - 20 * 512 * 4 * 16
+    assert awq.awq_workspace_size_min(1000, 512, 512, awq.AwqConfig.make(search_form=abi.SEARCH_FUSED)) <= c
 
 
 def test_binding_constants_match_the_header():
@@ -202,3 +207,4 @@ def test_binding_constants_match_the_header():
     assert int(forms["AWQ_SEARCH_DIRECT"]) == abi.SEARCH_DIRECT
     assert int(forms["AWQ_SEARCH_GRAM"]) == abi.SEARCH_GRAM
     assert int(forms["AWQ_SEARCH_CACHED_Y"]) == abi.SEARCH_CACHED_Y
+    assert int(forms["AWQ_SEARCH_FUSED"]) == abi.SEARCH_FUSED

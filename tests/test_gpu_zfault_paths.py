@@ -57,8 +57,8 @@ def test_bounded_waits_report_timeout_and_leave_the_context_usable(monkeypatch):
 
 
 def test_timeouts_in_the_gram_cached_and_w4a16_kernels(monkeypatch):
-    """The same for the Gram-form and cached-output searches and for the W4A16
-    GEMM.  The W4A16 roles that idle for long stretches wait with a suspend
+    """The same for the Gram-form, cached-output and fused searches and for
+    the W4A16 GEMM.  The W4A16 roles that idle for long stretches wait with a suspend
     hint, so one poll may already see the phase complete: there the test
     accepts either status, and checks that nothing hangs and the next call is
     exact."""
@@ -70,7 +70,7 @@ def test_timeouts_in_the_gram_cached_and_w4a16_kernels(monkeypatch):
     Y = torch.empty((600, 256), dtype=torch.float16, device="cuda")
     ws16 = torch.empty(256, dtype=torch.uint8, device="cuda")
     cfgs = {form: awq.AwqConfig.make(search_form=form)
-            for form in (awq.abi.SEARCH_GRAM, awq.abi.SEARCH_CACHED_Y)}
+            for form in (awq.abi.SEARCH_GRAM, awq.abi.SEARCH_CACHED_Y, awq.abi.SEARCH_FUSED)}
     wss = {form: awq.alloc_workspace(600, 512, 256, cfg) for form, cfg in cfgs.items()}
     monkeypatch.setenv("AWQ_FAULT", "timeout")
     for form, cfg in cfgs.items():
@@ -89,7 +89,7 @@ def test_timeouts_in_the_gram_cached_and_w4a16_kernels(monkeypatch):
     for form, cfg in cfgs.items():
         mse, _ = _search(Xd, Wd, cfg, wss[form])
         awq.awq_device_status(wss[form])
-        check_mse(mse.cpu().numpy(), mse_o if form == awq.abi.SEARCH_GRAM else mse_y)
+        check_mse(mse.cpu().numpy(), mse_y if form == awq.abi.SEARCH_CACHED_Y else mse_o)
     awq.awq_w4a16_gemm(Xd, qw, qz, sc, cfgs[awq.abi.SEARCH_GRAM], Y, ws16)
     awq.awq_device_status(ws16)
     Y1 = Y.clone()
