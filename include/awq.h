@@ -92,7 +92,7 @@ typedef enum {
  *   AWQ_SEARCH_FUSED    the direct form with the candidates made inside the
  *                       GEMM: each B tile is converted from the W rows in
  *                       shared memory (from per-group steps and zero points,
- *                       16 bytes per alpha, row and group in the workspace), so
+ *                       8 bytes per alpha, row and group in the workspace), so
  *                       the n_alpha x out x in operand is never written; the
  *                       same MSE bits as AWQ_SEARCH_DIRECT, with the conversion
  *                       repeated for every 256-token tile. */

@@ -187,7 +187,7 @@ ScaleWs scale_layout(int64_t T, int64_t in, int64_t out, const awq_config *cfg, 
   off = align256(off + sizeof(float) * (size_t)cfg->n_alpha * in);
   w.dW = off;  // fused form: the per-group parameters instead of the operand
   off = align256(off + (cfg->search_form == AWQ_SEARCH_FUSED
-                            ? sizeof(float4) * (size_t)cfg->n_alpha * w.out_pad * (in / cfg->group_size)
+                            ? sizeof(float2) * (size_t)cfg->n_alpha * w.out_pad * (in / cfg->group_size)
                             : sizeof(__half) * (size_t)n_chunk * w.out_pad * in));
   w.partials = off;
   off = align256(off + sizeof(double) * (size_t)cfg->n_alpha * w.per_alpha);
@@ -445,7 +445,7 @@ awq_status search_scale_impl(const void *X, int64_t T, int64_t in, int64_t ldx, 
   if (cfg->search_form == AWQ_SEARCH_FUSED) {
     // every candidate's per-group parameters, then the GEMM that builds its
     // B tiles from them and the W rows (the operand is never stored)
-    float4 *params = reinterpret_cast<float4 *>(base + L.dW);
+    float2 *params = reinterpret_cast<float2 *>(base + L.dW);
     {
       ProfScope p("fused_params", s);
       AWQ_TRY_CUDA(launch_fused_params(static_cast<const __half *>(W), out, in, L.out_pad, s_grid,

@@ -87,17 +87,17 @@ cudaError_t make_tmap_i32_box(CUtensorMap *m, const void *base, int64_t rows, in
                               int64_t ld, uint32_t box_cols, uint32_t box_rows);
 
 // Fused form, K3p: per (alpha, row < out_pad, group) the candidate quantiser's
-// {delta, rcp, half_lo, bits of (zero | clamp << 8)} of s 2^k w into
+// {delta, bits of (zero | clamp << 8 | no fast path << 9)} of s 2^k w into
 // params [n_alpha * out_pad, in / group] (rows past out: w = 0).
 cudaError_t launch_fused_params(const __half *W, int64_t out, int64_t in, int64_t out_pad,
                                 const float *s, int n_alpha, int group, int w_bit, int zero_point,
-                                const DevStatus *st, float4 *params, cudaStream_t stream);
+                                const DevStatus *st, float2 *params, cudaStream_t stream);
 // Fused form, K4f: the scored GEMM with each B tile converted from the W rows
 // in shared memory (the direct form's operand values, never stored); partials
 // as launch_search_gemm's.  in % 64 == 0, out_pad % 256 == 0.
 cudaError_t launch_fused_search_gemm(const __half *X, int64_t T, int64_t ldx, const __half *W,
                                      int64_t out, int64_t in, int64_t out_pad, int n_alpha,
-                                     const float *s, const float *inv_s, const float4 *params,
+                                     const float *s, const float *inv_s, const float2 *params,
                                      int group, int w_bit, double *partials, DevStatus *st,
                                      uint32_t max_polls, int num_sms, cudaStream_t stream);
 

@@ -6,20 +6,21 @@
 // back as the GEMM's B operand.  Here the B tiles are made in shared memory
 // from W itself, so that buffer never exists:
 //   K3p  fused_params: per (alpha, row, group) the quantiser's step, its
-//        approximate reciprocal, the fast-path bound and the zero point with
-//        a clamp flag (16 bytes, 42 MB for the layer above), from the group's
+//        zero point and two flags (8 bytes, 21 MB for the layer above; the
+//        approximate reciprocal and the fast-path bound follow), from the group's
 //        range of s w -- the values the candidate kernel derives on the way;
 //   K4f  fused_search_gemm: the scored GEMM's 256 x 256 tiles (two M = 128
 //        tcgen05 MMAs share each B tile), where a TMA load brings the W rows
-//        of the B tile instead of dW, and eight converter warps turn that
-//        tile into dW in place (thread t owns row t: its 8 16-byte chunks of
-//        each 64-channel K slice) before the MMA warp may read it.
+//        of the B tile instead of dW, and sixteen converter warps turn that
+//        tile into dW in place (a thread owns one 8-channel chunk column of 4
+//        rows of each 64-channel K slice) before the MMA warp may read it.
 // Each value goes through the candidate kernel's exact steps in the same
 // order (s 2^k w, the proposed code proven by its remainder or decided by the
 // correctly rounded quotient, the clamp, (q - z) delta - s w times 1/s), so
-// the B tiles hold the same bits as the direct form's operand, and the
-// epilogue, the tile order and the partial sums are the scored GEMM's: the
-// MSE comes out bit for bit the same.  The price is the conversion, once per
+// the B tiles hold the direct form's operand values (an error of exactly
+// zero may carry the other sign, which no product or square can see), and
+// the epilogue, the tile order and the partial sums are the scored GEMM's:
+// the MSE comes out bit for bit the same.  The price is the conversion, once per
 // 256-token M tile instead of once per layer.
 #include <cuda.h>
 #include <cuda_fp16.h>
@@ -41,11 +42,12 @@ constexpr uint32_t F_TMEM_COLS = 512;
 constexpr uint32_t F_IDESC = idesc_f16_f32(FBM, FBN);
 constexpr uint32_t F_DRAIN_POLLS = 1u << 22;
 constexpr int F_GROUP_M = 16;
-constexpr int F_EPI_WARPS = 8;   // warps 2..9
-constexpr int F_CONV_WARPS = 8;  // warps 10..17: thread t converts row t of the B tile
+constexpr int F_EPI_WARPS = 4;   // warps 2..5
+constexpr int F_CONV_WARPS = 16;  // warps 6..21: 4 chunks of each B tile slice per thread
+constexpr int F_CONV_ROWS = FBN * 8 / (F_CONV_WARPS * 32);  // rows per converter thread
 constexpr int F_CONV0 = 2 + F_EPI_WARPS;
 constexpr int F_THREADS = (F_CONV0 + F_CONV_WARPS) * 32;
-static_assert(F_CONV_WARPS * 32 == FBN, "one converter thread per B row");
+static_assert(F_CONV_ROWS * F_CONV_WARPS * 32 == FBN * 8, "every 16-byte chunk of a B slice once");
 
 struct __align__(8) FusedSmemTail {
   uint64_t full[F_STAGES];  // TMA: A tile and W rows landed
@@ -90,7 +92,7 @@ __device__ __forceinline__ uint32_t sw128_chunk(int r, int c) {
 // K3p.  A warp takes one (alpha, row) of the 256-channel slab blockIdx.y; lane
 // l holds channels 8l..8l+7, reduces its group's range of RN32(s 2^k w) over
 // the group's group / 8 lanes, and the group's first lane writes
-//   {delta, rcp, half_lo, bits of (zero | clamp << 8)}
+//   {delta, bits of (zero | clamp << 8 | no fast path << 9)}
 // as the candidate kernel computes them (group_params at ratio 1 with the
 // 1e-5 2^k floor, the fast-path bound, and whether the codes of the range's
 // ends leave [0, qmax]).  Rows out..out_pad-1 read w = 0.
@@ -99,7 +101,7 @@ template <int group>
 __global__ void __launch_bounds__(256) fused_params_kernel(
     const __half *__restrict__ W, int64_t out, int64_t in, int64_t out_pad,
     const float *__restrict__ s, int n_alpha, float qmax, int sym, const DevStatus *__restrict__ st,
-    float4 *__restrict__ params) {
+    float2 *__restrict__ params) {
   constexpr int lanes = group / 8;
   const int k = kscale_from_wmax(__uint_as_float(__ldcg(&st->wmax_bits)));
   const float two_k = ldexpf(1.0f, k);
@@ -138,19 +140,21 @@ __global__ void __launch_bounds__(256) fused_params_kernel(
     const float qhi = __fadd_rn(round_quotient(m, g), g.zero);
     const float qlo = __fadd_rn(round_quotient(n, g), g.zero);
     const bool clamp = !(qlo >= 0.0f && qhi <= g.qmax);
-    const int zf = (int)g.zero | (clamp ? 256 : 0);
+    // the reciprocal and the fast-path bound follow from delta (the same
+    // instructions give the same bits), unless the bound was disabled
+    const int zf = (int)g.zero | (clamp ? 256 : 0) | (g.half_lo < 0.0f ? 512 : 0);
     const int64_t gi = j0 / group;
     if (AWQ_IN_BOUNDS(gi < in / group, 0xB070u))
-      params[row * (in / group) + gi] = make_float4(g.delta, g.rcp, g.half_lo, __int_as_float(zf));
+      params[row * (in / group) + gi] = make_float2(g.delta, __int_as_float(zf));
   }
 }
 
 // ---------------------------------------------------------------------------
 // K4f.  Warp 0 loads the A tile (X, 256 x 64) and the W rows of the B tile
-// (256 x 64) by TMA into a 3-stage ring; warps 10..17 wait for a stage, turn
+// (256 x 64) by TMA into a 3-stage ring; warps 6..21 wait for a stage, turn
 // its W rows into dW in place and arrive on the stage's conversion barrier;
 // warp 1 issues the two M = 128 MMAs per K slice once both have happened;
-// warps 2..9 square and sum the accumulators as the scored GEMM's epilogue
+// warps 2..5 square and sum the accumulators as the scored GEMM's epilogue
 // does.  Every wait is bounded; a wait that runs out records the timeout and
 // every role drains what it has in flight before the CTA frees its TMEM.
 // ---------------------------------------------------------------------------
@@ -159,7 +163,7 @@ __global__ void __launch_bounds__(F_THREADS, 1)
     fused_search_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                              const __grid_constant__ CUtensorMap tmW, int num_m, int num_n, int num_kb,
                              int64_t in, int64_t out_pad, const float *__restrict__ s,
-                             const float *__restrict__ inv_s, const float4 *__restrict__ params,
+                             const float *__restrict__ inv_s, const float2 *__restrict__ params,
                              float qmax, double *__restrict__ partials, DevStatus *st,
                              uint32_t max_polls) {
   extern __shared__ uint8_t smem_raw[];
@@ -283,8 +287,8 @@ __global__ void __launch_bounds__(F_THREADS, 1)
     }
   } else if (warp < F_CONV0) {
     // ------------------------------------------------------------ epilogue
+    // four warps, one per TMEM lane quarter, each drains both row halves
     const int q = warp & 3;
-    const int h = (warp - 2) >> 2;
     int it = 0;
     for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++it) {
       int ok = 1;
@@ -297,36 +301,44 @@ __global__ void __launch_bounds__(F_THREADS, 1)
       tc_fence_after();
       int m_blk, n_blk;
       f_tile_coords(tile, num_m2, num_n, F_GROUP_M, m_blk, n_blk);
-      const int m128 = 2 * m_blk + h;
-      float sum = 0.0f;
-      if (m128 < num_m) {
+      float sum[2] = {0.0f, 0.0f};
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        if (2 * m_blk + h >= num_m) continue;  // the last tile's second half may lie past T
         const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(h * FBN);
 #pragma unroll 1
-        for (int c = 0; c < FBN; c += 64) {  // two 32-column loads in flight per wait
-          float v[32], v2[32];
+        for (int c = 0; c < FBN; c += 32) {  // the scored GEMM's order of squares
+          float v[32];
           tmem_ld_32x32b_x32(taddr + (uint32_t)c, v);
-          tmem_ld_32x32b_x32(taddr + (uint32_t)(c + 32), v2);
           tmem_ld_wait();
 #pragma unroll
-          for (int i = 0; i < 32; ++i) sum = fmaf(v[i], v[i], sum);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) sum = fmaf(v2[i], v2[i], sum);
+          for (int i = 0; i < 32; ++i) sum[h] = fmaf(v[i], v[i], sum[h]);
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&tail->tempty);
-      double ds = (double)sum;
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) ds += __shfl_xor_sync(0xffffffffu, ds, off);
-      if (lane == 0 && m128 < num_m && AWQ_IN_BOUNDS(n_blk < num_n, 0xB071u))
-        partials[((size_t)n_blk * num_m + m128) * 4 + q] = ds;
+      for (int h = 0; h < 2; ++h) {
+        const int m128 = 2 * m_blk + h;
+        double ds = (double)sum[h];
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) ds += __shfl_xor_sync(0xffffffffu, ds, off);
+        if (lane == 0 && m128 < num_m && AWQ_IN_BOUNDS(n_blk < num_n, 0xB071u))
+          partials[((size_t)n_blk * num_m + m128) * 4 + q] = ds;
+      }
     }
   } else {
     // ------------------------------------------------------------ converters
-    // thread ct owns row ct of every B tile: candidate row n_blk * 256 + ct,
-    // i.e. alpha a and output row o = o0 + ct of W
+    // thread ct converts 16-byte chunk column cc (channels 8 cc .. 8 cc + 7 of
+    // the K slice) of rows r0 + 32 i, i = 0..7, of every B tile: its s 2^k
+    // and 1/s are loaded once per K slice, and a warp's 32 chunks are 512
+    // contiguous bytes of shared memory (four rows).  Row r of the tile is
+    // candidate row n_blk * 256 + r: alpha a and row o0 + r of W.
     const int ct = threadIdx.x - F_CONV0 * 32;
+    constexpr int kRowStep = F_CONV_WARPS * 4;  // rows between a thread's chunks
+    const int cc = ct & 7, r0 = ct >> 3;        // rows r0 + kRowStep i
+    const uint32_t off0 = sw128_chunk(r0, cc);  // kRowStep % 8 == 0: the same swizzle for every i
     const int k = kscale_from_wmax(__uint_as_float(__ldcg(&st->wmax_bits)));
     const float2 tk = make_float2(ldexpf(1.0f, k), ldexpf(1.0f, k));
     const float2 M = make_float2(12582912.0f, 12582912.0f);  // 1.5 2^23
@@ -337,11 +349,10 @@ __global__ void __launch_bounds__(F_THREADS, 1)
     for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
       int m_blk, n_blk;
       f_tile_coords(tile, num_m2, num_n, F_GROUP_M, m_blk, n_blk);
-      const int64_t crow = (int64_t)n_blk * FBN + ct;  // alpha * out_pad + o
-      const int64_t a = crow / out_pad;
-      const float *s_a = s + a * in;
-      const float *is_a = inv_s + a * in;
-      const float4 *prm = params + crow * groups;
+      const int64_t crow0 = (int64_t)n_blk * FBN;  // alpha * out_pad + o0
+      const int64_t a = crow0 / out_pad;
+      const float2 *prow = params + (crow0 + r0) * groups;
+      float2 p[F_CONV_ROWS];  // the rows' group parameters, reloaded when a group starts
       for (int kb = 0; kb < num_kb; ++kb) {
         // every lane waits (each reads what the TMA wrote); the warp gives up together
         const bool w_ok = mbar_wait_bounded(&tail->full[stage], phase, max_polls, abort_flag);
@@ -350,51 +361,69 @@ __global__ void __launch_bounds__(F_THREADS, 1)
           ok = false;
           break;
         }
-        uint8_t *b = sB + stage * F_B_BYTES;
-#pragma unroll 2
-        for (int c = 0; c < 8; ++c) {
-          const int64_t j = (int64_t)kb * FBK + 8 * c;  // first channel of the chunk
-          const float4 p = __ldg(prm + j / group);
-          const float dl = p.x, rc = p.y, hl = p.z;
-          const int zf = __float_as_int(p.w);
-          const float4 *sp = reinterpret_cast<const float4 *>(s_a + j);
-          const float4 *ip = reinterpret_cast<const float4 *>(is_a + j);
-          const float4 s0 = __ldg(sp), s1 = __ldg(sp + 1), i0 = __ldg(ip), i1 = __ldg(ip + 1);
-          const float2 sk[4] = {__fmul2_rn(make_float2(s0.x, s0.y), tk), __fmul2_rn(make_float2(s0.z, s0.w), tk),
-                                __fmul2_rn(make_float2(s1.x, s1.y), tk), __fmul2_rn(make_float2(s1.z, s1.w), tk)};
-          const float2 iv[4] = {make_float2(i0.x, i0.y), make_float2(i0.z, i0.w), make_float2(i1.x, i1.y),
-                                make_float2(i1.z, i1.w)};
-          uint4 *cp = reinterpret_cast<uint4 *>(b + sw128_chunk(ct, c));
+        const int64_t j = (int64_t)kb * FBK + 8 * cc;  // first channel of the chunk column
+        if (group < FBK || (kb * FBK) % group == 0) {
+#pragma unroll
+          for (int i = 0; i < F_CONV_ROWS; ++i) p[i] = __ldg(prow + (int64_t)(kRowStep * i) * groups + j / group);
+        }
+        const float4 *sp = reinterpret_cast<const float4 *>(s + a * in + j);
+        const float4 *ip = reinterpret_cast<const float4 *>(inv_s + a * in + j);
+        const float4 s0 = __ldg(sp), s1 = __ldg(sp + 1), i0 = __ldg(ip), i1 = __ldg(ip + 1);
+        const float2 sk[4] = {__fmul2_rn(make_float2(s0.x, s0.y), tk), __fmul2_rn(make_float2(s0.z, s0.w), tk),
+                              __fmul2_rn(make_float2(s1.x, s1.y), tk), __fmul2_rn(make_float2(s1.z, s1.w), tk)};
+        const float2 iv[4] = {make_float2(i0.x, i0.y), make_float2(i0.z, i0.w), make_float2(i1.x, i1.y),
+                              make_float2(i1.z, i1.w)};
+        uint8_t *b = sB + stage * F_B_BYTES + off0;
+#pragma unroll
+        for (int i = 0; i < F_CONV_ROWS; ++i) {
+          const float dl = p[i].x;
+          const int zf = __float_as_int(p[i].y);
+          const float rc = rcp_approx(dl);  // as group_params derives them
+          const float hl = (zf & 512) ? -1.0f : __fmul_rn(dl, 0.4999847412109375f /* 0.5 - 2^-16 */);
+          uint4 *cp = reinterpret_cast<uint4 *>(b + i * kRowStep * 128);
           const uint4 wv = *cp;
           const uint32_t wr[4] = {wv.x, wv.y, wv.z, wv.w};
-          float2 wt[4], qz[4];
+          float2 wt[4], qz[4], rem[4];
           float rmax = 0.0f;
 #pragma unroll
           for (int hh = 0; hh < 4; ++hh) {
             wt[hh] = __fmul2_rn(sk[hh], __half22float2(*reinterpret_cast<const __half2 *>(&wr[hh])));
             qz[hh] = __fadd2_rn(__ffma2_rn(wt[hh], make_float2(rc, rc), M), make_float2(-M.x, -M.y));
-            const float2 rem = __ffma2_rn(make_float2(-qz[hh].x, -qz[hh].y), make_float2(dl, dl), wt[hh]);
-            rmax = fmax3(rmax, fabsf(rem.x), fabsf(rem.y));
-          }
-          if (!(rmax < hl)) {
-#pragma unroll
-            for (int hh = 0; hh < 4; ++hh)
-              qz[hh] = make_float2(rintf(__fdiv_rn(wt[hh].x, dl)), rintf(__fdiv_rn(wt[hh].y, dl)));
-          }
-          if (zf & 256) {
-            const float zero = (float)(zf & 255);
-            const float lo = -zero, hi = qmax - zero;
-#pragma unroll
-            for (int hh = 0; hh < 4; ++hh)
-              qz[hh] = make_float2(fminf(fmaxf(qz[hh].x, lo), hi), fminf(fmaxf(qz[hh].y, lo), hi));
+            rem[hh] = __ffma2_rn(qz[hh], make_float2(-dl, -dl), wt[hh]);  // RN(wt - q delta)
+            rmax = fmax3(rmax, fabsf(rem[hh].x), fabsf(rem[hh].y));
           }
           uint32_t packed[4];
+          if (rmax < hl && !(zf & 256)) {
+            // every proposed code is proven and none is clamped: the error
+            // (q - z) delta - s w is RN(q delta - wt) = -rem (one rounding
+            // either way, up to the sign of a zero), so dW = RN(rem (-1/s))
+            // needs no further FMA
 #pragma unroll
-          for (int hh = 0; hh < 4; ++hh) {
-            const float2 t = __ffma2_rn(qz[hh], make_float2(dl, dl), make_float2(-wt[hh].x, -wt[hh].y));
-            const float2 d2 = __fmul2_rn(t, iv[hh]);
-            const __half2 hv = __floats2half2_rn(d2.x, d2.y);
-            packed[hh] = *reinterpret_cast<const uint32_t *>(&hv);
+            for (int hh = 0; hh < 4; ++hh) {
+              const float2 d2 = __fmul2_rn(rem[hh], make_float2(-iv[hh].x, -iv[hh].y));
+              const __half2 hv = __floats2half2_rn(d2.x, d2.y);
+              packed[hh] = *reinterpret_cast<const uint32_t *>(&hv);
+            }
+          } else {
+            if (!(rmax < hl)) {
+#pragma unroll
+              for (int hh = 0; hh < 4; ++hh)
+                qz[hh] = make_float2(rintf(__fdiv_rn(wt[hh].x, dl)), rintf(__fdiv_rn(wt[hh].y, dl)));
+            }
+            if (zf & 256) {
+              const float zero = (float)(zf & 255);
+              const float lo = -zero, hi = qmax - zero;
+#pragma unroll
+              for (int hh = 0; hh < 4; ++hh)
+                qz[hh] = make_float2(fminf(fmaxf(qz[hh].x, lo), hi), fminf(fmaxf(qz[hh].y, lo), hi));
+            }
+#pragma unroll
+            for (int hh = 0; hh < 4; ++hh) {
+              const float2 t = __ffma2_rn(qz[hh], make_float2(dl, dl), make_float2(-wt[hh].x, -wt[hh].y));
+              const float2 d2 = __fmul2_rn(t, iv[hh]);
+              const __half2 hv = __floats2half2_rn(d2.x, d2.y);
+              packed[hh] = *reinterpret_cast<const uint32_t *>(&hv);
+            }
           }
           *cp = make_uint4(packed[0], packed[1], packed[2], packed[3]);
         }
@@ -419,7 +448,7 @@ __global__ void __launch_bounds__(F_THREADS, 1)
 
 cudaError_t launch_fused_params(const __half *W, int64_t out, int64_t in, int64_t out_pad,
                                 const float *s, int n_alpha, int group, int w_bit, int zero_point,
-                                const DevStatus *st, float4 *params, cudaStream_t stream) {
+                                const DevStatus *st, float2 *params, cudaStream_t stream) {
   if (group != 32 && group != 64 && group != 128) return cudaErrorInvalidValue;
   dim3 grid((unsigned)(((int64_t)n_alpha * out_pad + 7) / 8), (unsigned)((in + 255) / 256));
   auto kern = group == 32 ? fused_params_kernel<32> : group == 64 ? fused_params_kernel<64>
@@ -431,7 +460,7 @@ cudaError_t launch_fused_params(const __half *W, int64_t out, int64_t in, int64_
 
 cudaError_t launch_fused_search_gemm(const __half *X, int64_t T, int64_t ldx, const __half *W,
                                      int64_t out, int64_t in, int64_t out_pad, int n_alpha,
-                                     const float *s, const float *inv_s, const float4 *params,
+                                     const float *s, const float *inv_s, const float2 *params,
                                      int group, int w_bit, double *partials, DevStatus *st,
                                      uint32_t max_polls, int num_sms, cudaStream_t stream) {
   if (group != 32 && group != 64 && group != 128) return cudaErrorInvalidValue;

@@ -190,10 +190,10 @@ def test_search_forms_and_zero_point_are_validated():
     a = awq.awq_workspace_size(1000, 512, 512, awq.AwqConfig.make())
     b = awq.awq_workspace_size(1000, 512, 512, awq.AwqConfig.make(search_form=abi.SEARCH_CACHED_Y))
     assert b - a >= 1024 * 512 * 2
-    # the fused form keeps 16 bytes per (alpha, row, group) instead of the
+    # the fused form keeps 8 bytes per (alpha, row, group) instead of the
     # n_alpha x out_pad x in fp16 operand, whatever the workspace
     c = awq.awq_workspace_size(1000, 512, 512, awq.AwqConfig.make(search_form=abi.SEARCH_FUSED))
-    assert a - c == 20 * 512 * 512 * 2 - 20 * 512 * 4 * 16
+    assert a - c == 20 * 512 * 512 * 2 - 20 * 512 * 4 * 8
     assert awq.awq_workspace_size_min(1000, 512, 512, awq.AwqConfig.make(search_form=abi.SEARCH_FUSED)) <= c
 
 
