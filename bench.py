@@ -51,7 +51,7 @@ NCU_TRAFFIC = {
     "sources_sha256": "783bdf6248aceb0daeaef22bf3c1e10e9a61b126fa91114577c6692fc2dbc398",
     "command": ("ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum --clock-control none "
                 "-k regex:search_gemm -s 5 -c 1 python bench.py --steps 1 --warmup 5 "
-                "--no-cpu-baseline --no-gram-form --no-cached-form --no-w4a16 --no-workloads"),
+                "--no-cpu-baseline --no-gram-form --no-cached-form --no-fused-form --no-w4a16 --no-workloads"),
 }
 TRAFFIC_SOURCES = ("post_weight_quantization_awq_b200/csrc/search_gemm.cu",
                    "post_weight_quantization_awq_b200/csrc/awq_device.cuh")
@@ -673,6 +673,25 @@ def run_awq(args):
                   "note": "scores against the cached fp16 output RN16(X W^T) (one extra GEMM "
                           "with a store epilogue); candidates RN16(Qdeq/s)"}
 
+    # ---- the fused form on the same layer: every candidate's B tile built
+    # inside the scored GEMM from W (no candidate operand in HBM); the same
+    # MSE bits as the direct form
+    fused = None
+    if not args.no_fused_form:
+        ms_fu, kfu = time_form(awq.abi.SEARCH_FUSED, ("fused_params", "fused_gemm"))
+        flops_fu = 2.0 * T * inn * out * wl.n_alpha
+        cfg_fu = awq.AwqConfig.make(w_bit=wl.w_bit, group_size=wl.group_size, n_alpha=wl.n_alpha,
+                                    n_clip=wl.n_clip, clip_min=0.5, search_form=awq.abi.SEARCH_FUSED)
+        fused = {"value": round(ms_fu / world, 3), "unit": UNIT, "ms_per_step": round(ms_fu, 3),
+                 "kernels_ms": {k: round(v, 4) for k, v in kfu.items() if v},
+                 "algorithmic_flops_per_step": flops_fu,
+                 "gemm_tflops": round(flops_fu / (kfu["fused_gemm"] * 1e-3) / 1e12, 1)
+                 if kfu.get("fused_gemm") else None,
+                 "workspace_bytes": awq.awq_workspace_size(T, inn, out, cfg_fu),
+                 "note": "the candidates' B tiles converted from W in shared memory inside the "
+                         "scored GEMM (per-group steps and zero points in the workspace), once "
+                         "per 256-token tile; the same MSE bits as the direct form"}
+
     # ---- the same layer in the smallest workspace: the candidates built and
     # scored one at a time (the operand takes out x in fp16 instead of 20 times that)
     low_ws = None
@@ -779,6 +798,7 @@ def run_awq(args):
         "cpu_baseline": cpu,
         "gram_form": gram,
         "cached_output_form": cached,
+        "fused_form": fused,
         "w4a16_gemm": w4a16,
         "workloads": workloads,
         "smallest_workspace": low_ws,
@@ -884,6 +904,8 @@ def main(argv=None):
                     help="skip the extra measurement of the Gram-form search")
     ap.add_argument("--no-cached-form", action="store_true",
                     help="skip the extra measurement of the cached fp16-output form")
+    ap.add_argument("--no-fused-form", action="store_true",
+                    help="skip the extra measurement of the fused-candidate form")
     ap.add_argument("--no-workloads", action="store_true",
                     help="skip the timing of the MLP and 13B-attention layers")
     ap.add_argument("--no-w4a16", action="store_true",
