@@ -331,7 +331,7 @@ __global__ void __launch_bounds__(F_THREADS, 1)
   } else {
     // ------------------------------------------------------------ converters
     // thread ct converts 16-byte chunk column cc (channels 8 cc .. 8 cc + 7 of
-    // the K slice) of rows r0 + 32 i, i = 0..7, of every B tile: its s 2^k
+    // the K slice) of rows r0 + 64 i, i = 0..3, of every B tile: its s 2^k
     // and 1/s are loaded once per K slice, and a warp's 32 chunks are 512
     // contiguous bytes of shared memory (four rows).  Row r of the tile is
     // candidate row n_blk * 256 + r: alpha a and row o0 + r of W.
