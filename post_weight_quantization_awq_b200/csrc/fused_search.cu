@@ -89,8 +89,9 @@ __device__ __forceinline__ uint32_t sw128_chunk(int r, int c) {
 }  // namespace
 
 // ---------------------------------------------------------------------------
-// K3p.  A warp takes one (alpha, row) of the 256-channel slab blockIdx.y; lane
-// l holds channels 8l..8l+7, reduces its group's range of RN32(s 2^k w) over
+// K3p.  A warp takes one row of W and the 256-channel slab blockIdx.y, and
+// walks the alphas with the row's weights in registers: lane l holds
+// channels 8l..8l+7, reduces its group's range of RN32(s 2^k w) over
 // the group's group / 8 lanes, and the group's first lane writes
 //   {delta, bits of (zero | clamp << 8 | no fast path << 9)}
 // as the candidate kernel computes them (group_params at ratio 1 with the
@@ -107,45 +108,50 @@ __global__ void __launch_bounds__(256) fused_params_kernel(
   const float two_k = ldexpf(1.0f, k);
   const float guard = __fmul_rn(1e-5f, two_k);  // exact
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t row = (int64_t)blockIdx.x * 8 + warp;  // alpha * out_pad + o
-  if (row >= (int64_t)n_alpha * out_pad) return;       // whole warps
-  const int64_t a = row / out_pad, o = row - a * out_pad;
+  const int64_t o = (int64_t)blockIdx.x * 8 + warp;  // row of W (rows past out read w = 0)
+  if (o >= out_pad) return;                          // whole warps
   const int64_t j0 = (int64_t)blockIdx.y * 256 + lane * 8;
   const bool j_ok = j0 < in;
-  float m = -INFINITY, n = INFINITY;
-  if (j_ok) {
-    const uint4 wv = o < out ? __ldg(reinterpret_cast<const uint4 *>(W + o * in + j0))
-                             : make_uint4(0u, 0u, 0u, 0u);
-    const float4 *sp = reinterpret_cast<const float4 *>(s + a * in + j0);
-    const float4 s0 = __ldg(sp), s1 = __ldg(sp + 1);
-    const float2 tk = make_float2(two_k, two_k);
-    const float2 sk[4] = {__fmul2_rn(make_float2(s0.x, s0.y), tk), __fmul2_rn(make_float2(s0.z, s0.w), tk),
-                          __fmul2_rn(make_float2(s1.x, s1.y), tk), __fmul2_rn(make_float2(s1.z, s1.w), tk)};
-    const uint32_t wr[4] = {wv.x, wv.y, wv.z, wv.w};
+  // the row's 8 weights of this lane, read once for every alpha
+  const uint4 wv = j_ok && o < out ? __ldg(reinterpret_cast<const uint4 *>(W + o * in + j0))
+                                   : make_uint4(0u, 0u, 0u, 0u);
+  const uint32_t wr[4] = {wv.x, wv.y, wv.z, wv.w};
+  float2 w2[4];
 #pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      const float2 t = __fmul2_rn(sk[h], __half22float2(*reinterpret_cast<const __half2 *>(&wr[h])));
-      m = fmax3(m, t.x, t.y);
-      n = fmin3(n, t.x, t.y);
+  for (int h = 0; h < 4; ++h) w2[h] = __half22float2(*reinterpret_cast<const __half2 *>(&wr[h]));
+  const float2 tk = make_float2(two_k, two_k);
+  for (int a = 0; a < n_alpha; ++a) {
+    float m = -INFINITY, n = INFINITY;
+    if (j_ok) {
+      const float4 *sp = reinterpret_cast<const float4 *>(s + (int64_t)a * in + j0);
+      const float4 s0 = __ldg(sp), s1 = __ldg(sp + 1);
+      const float2 sk[4] = {__fmul2_rn(make_float2(s0.x, s0.y), tk), __fmul2_rn(make_float2(s0.z, s0.w), tk),
+                            __fmul2_rn(make_float2(s1.x, s1.y), tk), __fmul2_rn(make_float2(s1.z, s1.w), tk)};
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const float2 t = __fmul2_rn(sk[h], w2[h]);
+        m = fmax3(m, t.x, t.y);
+        n = fmin3(n, t.x, t.y);
+      }
     }
-  }
 #pragma unroll
-  for (int off = lanes / 2; off >= 1; off >>= 1) {
-    m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-    n = fminf(n, __shfl_xor_sync(0xffffffffu, n, off));
-  }
-  if (j_ok && (lane & (lanes - 1)) == 0) {
-    GroupQ g = group_params(m, n, 1.0f, qmax, sym != 0, guard);
-    fast_path_check(g, m, n);
-    const float qhi = __fadd_rn(round_quotient(m, g), g.zero);
-    const float qlo = __fadd_rn(round_quotient(n, g), g.zero);
-    const bool clamp = !(qlo >= 0.0f && qhi <= g.qmax);
-    // the reciprocal and the fast-path bound follow from delta (the same
-    // instructions give the same bits), unless the bound was disabled
-    const int zf = (int)g.zero | (clamp ? 256 : 0) | (g.half_lo < 0.0f ? 512 : 0);
-    const int64_t gi = j0 / group;
-    if (AWQ_IN_BOUNDS(gi < in / group, 0xB070u))
-      params[row * (in / group) + gi] = make_float2(g.delta, __int_as_float(zf));
+    for (int off = lanes / 2; off >= 1; off >>= 1) {
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+      n = fminf(n, __shfl_xor_sync(0xffffffffu, n, off));
+    }
+    if (j_ok && (lane & (lanes - 1)) == 0) {
+      GroupQ g = group_params(m, n, 1.0f, qmax, sym != 0, guard);
+      fast_path_check(g, m, n);
+      const float qhi = __fadd_rn(round_quotient(m, g), g.zero);
+      const float qlo = __fadd_rn(round_quotient(n, g), g.zero);
+      const bool clamp = !(qlo >= 0.0f && qhi <= g.qmax);
+      // the reciprocal and the fast-path bound follow from delta (the same
+      // instructions give the same bits), unless the bound was disabled
+      const int zf = (int)g.zero | (clamp ? 256 : 0) | (g.half_lo < 0.0f ? 512 : 0);
+      const int64_t gi = j0 / group;
+      if (AWQ_IN_BOUNDS(gi < in / group, 0xB070u))
+        params[((int64_t)a * out_pad + o) * (in / group) + gi] = make_float2(g.delta, __int_as_float(zf));
+    }
   }
 }
 
@@ -450,7 +456,7 @@ cudaError_t launch_fused_params(const __half *W, int64_t out, int64_t in, int64_
                                 const float *s, int n_alpha, int group, int w_bit, int zero_point,
                                 const DevStatus *st, float2 *params, cudaStream_t stream) {
   if (group != 32 && group != 64 && group != 128) return cudaErrorInvalidValue;
-  dim3 grid((unsigned)(((int64_t)n_alpha * out_pad + 7) / 8), (unsigned)((in + 255) / 256));
+  dim3 grid((unsigned)((out_pad + 7) / 8), (unsigned)((in + 255) / 256));
   auto kern = group == 32 ? fused_params_kernel<32> : group == 64 ? fused_params_kernel<64>
                                                                   : fused_params_kernel<128>;
   kern<<<grid, 256, 0, stream>>>(W, out, in, out_pad, s, n_alpha, (float)((1 << w_bit) - 1),
