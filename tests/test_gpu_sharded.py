@@ -25,7 +25,7 @@ def _cuda():
 
 @pytest.mark.parametrize("T,inn,out,w_bit,cuts,form", [
     (2125, 1024, 264, 4, (1000,), 0), (600, 512, 136, 3, (129, 300), 0), (900, 512, 256, 4, (450,), 2),
-    (700, 384, 128, 4, (350,), 1)])
+    (700, 384, 128, 4, (350,), 1), (1100, 512, 264, 4, (400, 700), 3)])
 def test_shards_summed_on_device_match_oracle(T, inn, out, w_bit, cuts, form):
     X, W = random_layer(T, inn, out, seed=T + inn + out)
     cfg = awq.AwqConfig.make(w_bit=w_bit, n_alpha=20, n_clip=20, search_form=form)
