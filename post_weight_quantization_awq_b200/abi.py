@@ -46,7 +46,8 @@ SEARCH_DIRECT, SEARCH_GRAM, SEARCH_CACHED_Y, SEARCH_FUSED = 0, 1, 2, 3
 class AwqConfig(ctypes.Structure):
     """awq_config: w_bit, group_size, zero_point ("05 — AWQ" §9 quant_config),
     n_alpha, n_clip, clip_min ("05 — AWQ" §4), search_form (0 direct scored
-    GEMM, 1 Gram form)."""
+    GEMM, 1 Gram form, 2 cached fp16 output, 3 candidates made inside the
+    GEMM)."""
 
     _fields_ = [
         ("w_bit", c_int32),
